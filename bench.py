@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the conv1d + selective-scan hot path on B200.
+
+Default workload: the Mamba-1 layer (batch 8, 2048 tokens, d_inner 1536,
+dstate 16, conv width 4, bf16 activations, fp32 state); one step is one
+forward pass of the fused conv + scan over that batch.  Other workloads can
+be picked with ``--workload`` (Mamba-2 SSD, packed varlen Mamba-2, decode).
+
+Prints ONE JSON line (rank 0).  Device time comes from CUDA events on the
+launching stream around each step; L2 is flushed (a 256 MiB write) between
+timed steps, outside the events.  With torchrun, each rank runs its own copy
+of the workload (independent batches: weak scaling, no data-path
+collective) and the reported time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle instead, on a bounded sample
+of the same workload, on this machine's host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from state_space_model_conv1d_b200 import workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = "mamba1_layer_b8_l2048_d1536_n16"
+METRIC = "scan tokens/s"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "dram_traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+MUFU_PER_CLK_PER_SM = 16       # ex2 lanes per SM per clock (4 per SM sub-partition)
+NUM_SMS = 148
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_PATH):
+        d = json.load(open(PEAKS_PATH))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(*names):
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "state_space_model_conv1d_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except FileNotFoundError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- workloads
+class Job:
+    """One workload on the device: step(), bytes and units per step, e2e step."""
+
+    def __init__(self, w: W.Workload, rank: int, torch, ssm):
+        self.w, self.torch, self.ssm = w, torch, ssm
+        dev = torch.device("cuda", torch.cuda.current_device())
+        seed_shift = 7919 * rank
+        bf = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        self.launches_per_step = 1
+        if w.kind in ("mamba1", "mamba2", "mamba2_varlen"):
+            mode = ssm.MAMBA1 if w.kind == "mamba1" else ssm.MAMBA2
+            ww = W.Workload(**{**w.__dict__, "seed": w.seed + seed_shift})
+            d = W.workload_inputs(ww)
+            self.host = {}
+            t = {}
+            act = ("x", "z", "dt", "B", "C")
+            for k, v in d.items():
+                if v is None:
+                    t[k] = None
+                    continue
+                if k == "cu_seqlens":
+                    t[k] = torch.from_numpy(v).to(dev)
+                    continue
+                src = torch.from_numpy(np.ascontiguousarray(v)).to(bf if k in act else torch.float32)
+                self.host[k] = src.pin_memory()
+                t[k] = self.host[k].to(dev)
+            self.t = t
+            self.mode = mode
+            x = t["x"]
+            nseq = x.shape[0] if t.get("cu_seqlens") is None else t["cu_seqlens"].numel() - 1
+            self.tokens = x.shape[0] * x.shape[1]
+            self.y = torch.empty_like(x)
+            if mode == ssm.MAMBA1:
+                hshape, cdim = (nseq, x.shape[2], t["B"].shape[2]), x.shape[2]
+            else:
+                hshape = (nseq, x.shape[2], x.shape[3], t["B"].shape[3])
+                cdim = x.shape[2] * x.shape[3] + 2 * t["B"].shape[2] * t["B"].shape[3]
+            self.hf = torch.empty(hshape, dtype=torch.float32, device=dev)
+            self.cso = torch.empty((nseq, cdim, t["conv_w"].shape[1] - 1), dtype=bf, device=dev)
+            need = ssm.scan_workspace_size(mode, x, t["dt"], t["A"], t["B"], t["C"], cu_seqlens=t.get("cu_seqlens"))
+            self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev) if need else None
+            if need:
+                self.launches_per_step = 2
+            read = sum(v.numel() * v.element_size() for k, v in t.items() if v is not None)
+            wrote = sum(v.numel() * v.element_size() for v in (self.y, self.hf, self.cso))
+            self.bytes_per_step = read + wrote
+            self.units = self.tokens
+            self.kernel = "scan_m1_kernel" if mode == ssm.MAMBA1 else "scan_m2"
+            self.sources = ("scan_m1.cu",) if mode == ssm.MAMBA1 else ("scan_m2_simt.cu",)
+            if mode == ssm.MAMBA1:
+                self.mufu = x.shape[0] * x.shape[1] * x.shape[2] * t["B"].shape[2]
+            else:
+                self.mufu = None
+            self.flops = None
+        elif w.kind == "decode":
+            ww = W.Workload(**{**w.__dict__, "seed": w.seed + seed_shift})
+            d = W.workload_inputs(ww)
+            act = ("x", "z", "dt", "B", "C", "conv_state")
+            t = {}
+            self.host = {}
+            for k, v in d.items():
+                if v is None:
+                    t[k] = None
+                    continue
+                src = torch.from_numpy(np.ascontiguousarray(v)).to(bf if k in act else torch.float32)
+                self.host[k] = src.pin_memory() if k not in ("state", "conv_state") else src
+                t[k] = src.to(dev)
+            self.t = t
+            self.mode = ssm.MAMBA2
+            self.nsets = w.nsets
+            self.step_i = 0
+            self.tokens = w.batch
+            self.y = torch.empty_like(t["x"][0])
+            per_set = sum(t[k][0].numel() * t[k][0].element_size() for k in ("x", "z", "dt", "B", "C"))
+            params = sum(t[k].numel() * t[k].element_size() for k in ("A", "D", "dt_bias", "conv_w"))
+            self.bytes_per_step = (2 * t["state"].numel() * 4 + 2 * t["conv_state"].numel() * t["conv_state"].element_size()
+                                   + per_set + self.y.numel() * self.y.element_size() + params)
+            self.units = w.batch
+            self.kernel = "decode_kernel"
+            self.sources = ("decode.cu",)
+            self.mufu = None
+            self.flops = None
+        else:
+            raise ValueError(w.kind)
+
+    def step(self):
+        ssm, t = self.ssm, self.t
+        if self.w.kind == "decode":
+            i = self.step_i % self.nsets
+            self.step_i += 1
+            ssm.state_update(self.mode, t["state"], t["conv_state"], t["x"][i], t["dt"][i], t["A"], t["B"][i],
+                             t["C"][i], D=t["D"], z=t["z"][i], dt_bias=t["dt_bias"], conv_w=t["conv_w"],
+                             conv_b=t["conv_b"], y=self.y)
+            return
+        ssm.scan_fwd(self.mode, t["x"], t["dt"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"], dt_bias=t["dt_bias"],
+                     h0=t["h0"], cu_seqlens=t.get("cu_seqlens"), conv_w=t["conv_w"], conv_b=t["conv_b"],
+                     conv_state_in=t["conv_state_in"], y=self.y, h_final=self.hf, conv_state_out=self.cso,
+                     workspace=self.ws)
+
+    def e2e_step(self, out_host):
+        """Host-resident inputs: pinned H2D copies, the step, then y back to the host."""
+        torch, t = self.torch, self.t
+        h2d = 0
+        if self.w.kind == "decode":
+            i = self.step_i % self.nsets
+            for k in ("x", "z", "dt", "B", "C"):
+                t[k][i].copy_(self.host[k][i], non_blocking=True)
+                h2d += self.host[k][i].numel() * self.host[k][i].element_size()
+        else:
+            for k in ("x", "z", "dt", "B", "C", "h0"):
+                if self.host.get(k) is not None:
+                    t[k].copy_(self.host[k], non_blocking=True)
+                    h2d += self.host[k].numel() * self.host[k].element_size()
+        self.step()
+        out_host.copy_(self.y, non_blocking=True)
+        return h2d, out_host.numel() * out_host.element_size()
+
+
+def flush_l2(buf):
+    buf.add_(1)       # 256 MiB read + write, twice the 126 MB L2
+
+
+def run_cuda(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import state_space_model_conv1d_b200 as ssm
+
+    w = W.WORKLOADS[args.workload]
+    job = Job(w, rank, torch, ssm)
+    flush = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(max(args.warmup, 0)):
+        job.step()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush_l2(flush)
+        evs[i][0].record(stream)
+        job.step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if rank == 0 else None
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        tt = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / max(args.steps, 1)
+    units_total = job.units * args.steps * world
+    value = units_total / (total_ms / 1e3)
+
+    # end to end through the public API with host-resident inputs
+    e2e = None
+    if not args.no_e2e:
+        out_host = torch.empty(job.y.shape, dtype=job.y.dtype).pin_memory()
+        ne = max(1, min(args.steps, 10))
+        job.e2e_step(out_host)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        h2d = d2h = 0
+        for _ in range(ne):
+            h2d, d2h = job.e2e_step(out_host)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            tt = torch.tensor([ems], device="cuda")
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        e2e = {"value": job.units * ne * world / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": ne}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_src = load_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    gbs = job.bytes_per_step / (ms_per_step / 1e3) / 1e9
+    traffic = None
+    if os.path.exists(TRAFFIC_PATH):
+        tr = json.load(open(TRAFFIC_PATH)).get(args.workload)
+        if tr and tr.get("source_sha") == source_sha(*job.sources):
+            traffic = tr.get("dram_bytes_per_launch")
+    if job.mufu is not None:
+        clock_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+        peak_g = NUM_SMS * MUFU_PER_CLK_PER_SM * clock_mhz * 1e6 / 1e9
+        achieved = job.mufu / (ms_per_step / 1e3) / 1e9
+        roofline = {"bound": "alu", "achieved": achieved, "peak": peak_g, "unit": "Gexp/s",
+                    "frac": achieved / peak_g, "traffic": traffic, "kernel": job.kernel,
+                    "peak_source": f"derived: {NUM_SMS} SMs x {MUFU_PER_CLK_PER_SM} MUFU ex2/clk x {clock_mhz:.0f} MHz",
+                    "hbm": {"achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback"}}
+    else:
+        roofline = {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                    "traffic": traffic, "kernel": job.kernel,
+                    "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback"}
+    roofline["algorithmic_bytes_per_launch"] = int(job.bytes_per_step)
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, args)
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": (w.batch or 1) * world, "seq_len": w.seqlen or None,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "flushed between timed steps (256 MiB write, outside the events)",
+                   "tokens_per_step": job.units},
+        "hbm_gbs": gbs, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+        "gpu_launches": job.launches_per_step * args.steps, "impl": "cuda",
+        "step_ms": {"min": min(step_ms), "median": float(np.median(step_ms)), "max": max(step_ms)},
+    }
+    print(json.dumps(out), flush=True)
+
+
+# --------------------------------------------------------------- oracle side
+def oracle_sample(w: W.Workload, target_s: float):
+    """A bounded sample of the workload for the fp64 oracle: whole sequences
+    (all channels / heads), as many as fit the time budget."""
+    import oracle
+    cores = os.cpu_count() or 1
+    if w.kind == "mamba1":
+        nrows = min(w.batch, max(1, cores))
+        ww = W.Workload(**{**w.__dict__, "batch": nrows})
+        d = W.workload_inputs(ww)
+        run = lambda: oracle.scan_fwd(oracle.MAMBA1, d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                                      dt_bias=d["dt_bias"], h0=d["h0"], conv_w=d["conv_w"], nthreads=nrows)
+        return run, nrows * w.seqlen, nrows, f"{nrows} of {w.batch} batch rows x {w.seqlen} tokens, all {w.d_inner} channels"
+    if w.kind in ("mamba2", "mamba2_varlen"):
+        T = 256 if w.kind == "mamba2" else 256
+        nrows = min(4, max(1, cores))
+        ww = W.Workload(**{**w.__dict__, "kind": "mamba2", "batch": nrows, "seqlen": T})
+        d = W.workload_inputs(ww)
+        run = lambda: oracle.scan_fwd(oracle.MAMBA2, d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
+                                      dt_bias=d["dt_bias"], h0=d["h0"], conv_w=d["conv_w"], nthreads=nrows)
+        return run, nrows * T, nrows, f"{nrows} sequences x {T} tokens, all {w.nheads} heads"
+    if w.kind == "decode":
+        nb = 16
+        ww = W.Workload(**{**w.__dict__, "batch": nb, "nsets": 1})
+        d = W.workload_inputs(ww)
+        state = d["state"].astype(np.float64)
+        cs = d["conv_state"].astype(np.float64)
+        run = lambda: oracle.state_update(oracle.MAMBA2, state, cs, d["x"][0], d["dt"][0], d["A"], d["B"][0], d["C"][0],
+                                          D=d["D"], z=d["z"][0], dt_bias=d["dt_bias"], conv_w=d["conv_w"])
+        return run, nb, 1, f"one decode step of {nb} of {w.batch} rows"
+    raise ValueError(w.kind)
+
+
+def cpu_baseline(w: W.Workload, args):
+    run, units, cores, what = oracle_sample(w, 20.0)
+    t0 = time.perf_counter()
+    run()
+    dt = time.perf_counter() - t0
+    return {"value": units / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": what,
+            "seconds": dt}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = W.WORKLOADS[args.workload]
+    run, units, cores, what = oracle_sample(w, 20.0)
+    for _ in range(max(args.warmup, 0)):
+        run()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        run()
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = units * args.steps / total
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": total / max(args.steps, 1) * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.name, "global_batch": w.batch or 1, "seq_len": w.seqlen or None,
+                      "parallelism": "host cores", "sample": what},
+           "impl": "reference",
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": what},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

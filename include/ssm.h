@@ -1,0 +1,211 @@
+/*
+ * ssm.h -- C ABI of libssm.so: the Mamba short causal conv1d + SiLU and the
+ * selective state-space scan on one B200 (sm_100a).
+ *
+ * Operations (what each computes, and the passage that defines it):
+ *
+ *   ssm_conv1d_fwd   Causal depthwise conv of width K over token-major input,
+ *                    optional bias and SiLU, with a carried state of the last
+ *                    K-1 raw inputs per sequence (in and out).
+ *                    "ggml : add GPU support for Mamba models" (llama.cpp issue
+ *                    6758): GGML_OP_SSM_CONV, test-backend-ops shapes
+ *                    s [d_conv-1, d_inner, n_seqs], x [d_inner, n_tokens,
+ *                    n_seqs], c [d_conv, d_inner]; the reply on concatenating
+ *                    the state in front of the tokens.
+ *
+ *   ssm_scan_fwd     delta = softplus(dt + dt_bias);
+ *                    h_t = exp(delta_t*A) h_{t-1} + delta_t B_t x_t;
+ *                    y_t = C_t . h_t + D x_t, then y_t *= silu(z_t);
+ *                    h_0 = h0 (zeros when absent), h_T returned in h_final.
+ *                    Optionally the conv above runs in front (x for Mamba-1,
+ *                    x|B|C for Mamba-2) inside the same kernel.
+ *                    "Adding Initial Value Support to Selective Scan Forward
+ *                    Kernel" (state-spaces/mamba issue 285): the step
+ *                    h_t = A h_{t-1} + Bx, the scan element (exp(delta*A), h)
+ *                    and its seed (1, h0); llama.cpp issue 6758: the scan op
+ *                    returns the final state instead of overwriting an input;
+ *                    "Tensor-parallel SSM" (Fast-LLM PR 333): Mamba-2 heads in
+ *                    contiguous groups sharing B and C (repeat_interleave).
+ *
+ *   ssm_state_update One decode token per batch row: the conv state window is
+ *                    rolled left by one and the new input appended, the conv +
+ *                    SiLU read its last K entries, then one step of the
+ *                    recurrence above updates the fp32 state in place.
+ *                    "Clean up SSM ops directory structure" (Megatron-LM PR
+ *                    6444): causal_conv1d_update and selective_state_update,
+ *                    and slot-indexed state rows (intermediate_extraction).
+ *
+ * Conventions for every entry point:
+ *   - Pointers are device pointers unless stated otherwise; the caller owns
+ *     every buffer.  The library never allocates or frees memory, and only
+ *     ssm_workspace_error synchronizes (it reads a device word back).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream).  A return of SSM_OK means the launch was enqueued.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     rejected call launches nothing and returns a negative ssm_status.
+ *     CUDA launch failures return SSM_ERR_CUDA; ssm_last_cuda_error() gives
+ *     the underlying cudaError_t.
+ *   - Tensors are token-major with the channel dimension contiguous (stride 1).
+ *     Batch and token strides are in ELEMENTS, so x / z / B / C may be views
+ *     into a wider projection output (e.g. x and z halves of one in_proj
+ *     row).  Every pointer must be aligned to its element size, and the
+ *     decode state to 16 bytes when dstate % 4 == 0 (else SSM_ERR_ALIGNMENT).
+ *     16-byte aligned bases and strides whose byte size is a multiple of 16
+ *     let the kernels use 16-byte vector loads; other layouts take a slower
+ *     element-wise path with the same results.
+ *   - Activations (x, z, dt, B, C, y, conv states) share one dtype, SSM_F32 or
+ *     SSM_BF16.  Parameters (A, D, dt_bias, conv weight / bias) and the
+ *     recurrent state (h0, h_final, decode state) are always fp32.  All
+ *     arithmetic is fp32; y is rounded once to its dtype (nearest-even).
+ *   - Optional pointers may be NULL: dt_bias (= 0), D (= 0), z (no gate),
+ *     h0 (= 0), h_final (not written), conv_b (= 0), conv_state_in (= 0),
+ *     conv_state_out (not written).
+ *   - Outputs must not overlap inputs, except conv_state_out == conv_state_in
+ *     (same layout), which is allowed: the state is read before it is
+ *     written.
+ */
+#ifndef SSM_H_
+#define SSM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SSM_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define SSM_API __attribute__((visibility("default")))
+#else
+#define SSM_API
+#endif
+
+typedef enum {
+    SSM_OK = 0,
+    SSM_ERR_INVALID_ARG = -1,   /* bad size, NULL required pointer, bad combination */
+    SSM_ERR_UNSUPPORTED = -2,   /* valid but outside what the kernels implement (e.g. dstate too large) */
+    SSM_ERR_ALIGNMENT = -3,     /* pointer not aligned to its element size (decode state: 16 bytes) */
+    SSM_ERR_WORKSPACE = -4,     /* workspace missing or smaller than ssm_scan_workspace_size() */
+    SSM_ERR_CUDA = -5,          /* a CUDA call failed; see ssm_last_cuda_error() */
+    SSM_ERR_DEVICE = -6         /* the device rejected data it validated (e.g. cu_seqlens) */
+} ssm_status;
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
+typedef enum { SSM_MAMBA1 = 1, SSM_MAMBA2 = 2 } ssm_mode;
+
+/* Device-side error codes written into the workspace error word. */
+#define SSM_DEVERR_NONE 0
+#define SSM_DEVERR_CU_SEQLENS 1   /* cu_seqlens not 0-based, decreasing, or not ending at seqlen */
+
+/* ------------------------------------------------------------------ conv */
+typedef struct ssm_conv_args {
+    int64_t batch;            /* rows; 1 when cu_seqlens is given */
+    int64_t seqlen;           /* tokens per row (total packed tokens when varlen) */
+    int64_t channels;         /* C */
+    int64_t width;            /* K, 1..8 */
+    int32_t dtype;            /* ssm_dtype of x, out, conv states */
+    int32_t activation;       /* 0: none, 1: SiLU */
+    int32_t nseqs;            /* number of sequences in cu_seqlens (varlen only) */
+    int32_t reserved0;
+    const void *x;            /* [batch][seqlen][channels], strides below */
+    int64_t x_batch_stride, x_token_stride;
+    const float *weight;      /* [channels][width]; weight[c][width-1] multiplies the current token */
+    const float *bias;        /* [channels] or NULL */
+    const void *state_in;     /* [batch or nseqs][channels][width-1], oldest first, or NULL */
+    void *state_out;          /* same layout, or NULL */
+    const int32_t *cu_seqlens;/* [nseqs+1] device int32 offsets (0 .. seqlen), or NULL */
+    void *out;                /* [batch][seqlen][channels] */
+    int64_t out_batch_stride, out_token_stride;
+} ssm_conv_args;
+
+/* ------------------------------------------------------------------ scan */
+typedef struct ssm_scan_args {
+    int32_t mode;             /* SSM_MAMBA1 or SSM_MAMBA2 */
+    int32_t dtype;            /* ssm_dtype of x, z, dt, B, C, y, conv states */
+    int32_t delta_softplus;   /* 1: delta = softplus(dt + dt_bias); 0: delta = dt + dt_bias */
+    int32_t nseqs;            /* number of sequences when cu_seqlens != NULL */
+    int64_t batch;            /* 1 when cu_seqlens != NULL */
+    int64_t seqlen;           /* tokens per row, or total packed tokens */
+    int64_t d_inner;          /* Mamba-1: channels D; Mamba-2: nheads*headdim */
+    int64_t nheads, headdim;  /* Mamba-2 only (ignored for Mamba-1) */
+    int64_t ngroups;          /* Mamba-2: groups of B/C (nheads % ngroups == 0); Mamba-1: 1 */
+    int64_t dstate;           /* N */
+    int64_t d_conv;           /* K of the fused conv (0 = no conv; x, B, C used as given) */
+    /* activations (dtype): Mamba-1 x,z,dt,y [b][T][D]; B,C [b][T][N].
+     *                      Mamba-2 x,z,y [b][T][H*P]; dt [b][T][H]; B,C [b][T][G*N]. */
+    const void *x;  int64_t x_batch_stride, x_token_stride;
+    const void *z;  int64_t z_batch_stride, z_token_stride;
+    const void *dt; int64_t dt_batch_stride, dt_token_stride;
+    const void *B;  int64_t B_batch_stride, B_token_stride;
+    const void *C;  int64_t C_batch_stride, C_token_stride;
+    void *y;        int64_t y_batch_stride, y_token_stride;
+    /* fp32 parameters: Mamba-1 A [D][N], D, dt_bias [D]; Mamba-2 A, D, dt_bias [H] */
+    const float *A, *D, *dt_bias;
+    /* fp32 states, contiguous: Mamba-1 [nseq][D][N]; Mamba-2 [nseq][H][P][N] */
+    const float *h0;
+    float *h_final;
+    const int32_t *cu_seqlens;/* [nseqs+1] device int32, or NULL */
+    /* fused conv: weight [conv_dim][K] fp32, bias [conv_dim]; states
+     * [nseq][conv_dim][K-1] in dtype.  conv_dim = D (Mamba-1, x only) or
+     * H*P + 2*G*N (Mamba-2, channels ordered x | B | C). */
+    const float *conv_w, *conv_b;
+    const void *conv_state_in;
+    void *conv_state_out;
+    int64_t chunk;            /* Mamba-2 chunk length hint (0 = kernel default); results do not depend on it */
+} ssm_scan_args;
+
+/* ---------------------------------------------------------------- decode */
+typedef struct ssm_update_args {
+    int32_t mode, dtype, delta_softplus, reserved0;
+    int64_t batch;            /* rows, one new token each */
+    int64_t d_inner, nheads, headdim, ngroups, dstate;   /* as in ssm_scan_args */
+    int64_t d_conv;           /* K (0 = no conv) */
+    int64_t conv_state_len;   /* columns kept per channel, >= K-1 (K-1 or K typical) */
+    float *state;             /* in-out fp32, per slot: Mamba-1 [D][N]; Mamba-2 [H][P][N]; slots contiguous */
+    void *conv_state;         /* in-out dtype, per slot [conv_dim][conv_state_len], oldest first */
+    const float *conv_w, *conv_b;
+    const void *x;  int64_t x_batch_stride;   /* Mamba-1 [b][D]; Mamba-2 [b][H*P] */
+    const void *z;  int64_t z_batch_stride;
+    const void *dt; int64_t dt_batch_stride;  /* Mamba-1 [b][D]; Mamba-2 [b][H] */
+    const void *B;  int64_t B_batch_stride;   /* Mamba-1 [b][N]; Mamba-2 [b][G*N] */
+    const void *C;  int64_t C_batch_stride;
+    void *y;        int64_t y_batch_stride;
+    const float *A, *D, *dt_bias;
+    const int32_t *state_batch_indices;  /* [batch]: slot of row r (NULL = r); a negative
+                                            slot marks a padding row: nothing is read or
+                                            written for it except y, which is set to 0 */
+    int64_t nslots;           /* number of state / conv-state slots (>= batch when indices are NULL) */
+} ssm_update_args;
+
+/* Library version and status text. */
+SSM_API int32_t ssm_abi_version(void);
+SSM_API const char *ssm_status_string(ssm_status s);
+/* The cudaError_t of the last failing CUDA call made by this thread (0 if none). */
+SSM_API int32_t ssm_last_cuda_error(void);
+
+/* Standalone conv (bias, activation).  No workspace. */
+SSM_API ssm_status ssm_conv1d_fwd(const ssm_conv_args *args, void *stream);
+
+/* Bytes of device workspace ssm_scan_fwd needs for these arguments (0 when
+ * none is needed; the packed varlen path needs one).  Does not touch the GPU. */
+SSM_API size_t ssm_scan_workspace_size(const ssm_scan_args *args);
+
+/* Forward scan.  `workspace` (device, 256-byte aligned, ws_bytes long) may be
+ * NULL when ssm_scan_workspace_size() is 0.  The workspace holds the device
+ * error word (read it with ssm_workspace_error) and the varlen schedule. */
+SSM_API ssm_status ssm_scan_fwd(const ssm_scan_args *args, void *workspace, size_t ws_bytes, void *stream);
+
+/* Decode update, in place on state and conv_state.  No workspace. */
+SSM_API ssm_status ssm_state_update(const ssm_update_args *args, void *stream);
+
+/* Waits for `stream`, then reads the device error word of a workspace last
+ * used by ssm_scan_fwd: SSM_OK, or SSM_ERR_DEVICE with *code set to an
+ * SSM_DEVERR_* value.  `code` may be NULL. */
+SSM_API ssm_status ssm_workspace_error(const void *workspace, int32_t *code, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSM_H_ */

@@ -1,0 +1,121 @@
+"""ctypes mirror of ``include/ssm.h`` and the loader of ``libssm.so``.
+
+Argument marshalling only.  The library is loaded on first use; when it is
+missing (not built) the call raises immediately -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libssm.so")
+
+SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_ALIGNMENT = 0, -1, -2, -3
+SSM_ERR_WORKSPACE, SSM_ERR_CUDA, SSM_ERR_DEVICE = -4, -5, -6
+SSM_F32, SSM_BF16 = 0, 1
+SSM_MAMBA1, SSM_MAMBA2 = 1, 2
+SSM_DEVERR_NONE, SSM_DEVERR_CU_SEQLENS = 0, 1
+
+_vp = C.c_void_p
+_i64 = C.c_int64
+_i32 = C.c_int32
+
+
+class ConvArgs(C.Structure):
+    _fields_ = [
+        ("batch", _i64), ("seqlen", _i64), ("channels", _i64), ("width", _i64),
+        ("dtype", _i32), ("activation", _i32), ("nseqs", _i32), ("reserved0", _i32),
+        ("x", _vp), ("x_batch_stride", _i64), ("x_token_stride", _i64),
+        ("weight", _vp), ("bias", _vp), ("state_in", _vp), ("state_out", _vp),
+        ("cu_seqlens", _vp),
+        ("out", _vp), ("out_batch_stride", _i64), ("out_token_stride", _i64),
+    ]
+
+
+class ScanArgs(C.Structure):
+    _fields_ = [
+        ("mode", _i32), ("dtype", _i32), ("delta_softplus", _i32), ("nseqs", _i32),
+        ("batch", _i64), ("seqlen", _i64), ("d_inner", _i64), ("nheads", _i64), ("headdim", _i64),
+        ("ngroups", _i64), ("dstate", _i64), ("d_conv", _i64),
+        ("x", _vp), ("x_batch_stride", _i64), ("x_token_stride", _i64),
+        ("z", _vp), ("z_batch_stride", _i64), ("z_token_stride", _i64),
+        ("dt", _vp), ("dt_batch_stride", _i64), ("dt_token_stride", _i64),
+        ("B", _vp), ("B_batch_stride", _i64), ("B_token_stride", _i64),
+        ("C", _vp), ("C_batch_stride", _i64), ("C_token_stride", _i64),
+        ("y", _vp), ("y_batch_stride", _i64), ("y_token_stride", _i64),
+        ("A", _vp), ("D", _vp), ("dt_bias", _vp),
+        ("h0", _vp), ("h_final", _vp),
+        ("cu_seqlens", _vp),
+        ("conv_w", _vp), ("conv_b", _vp), ("conv_state_in", _vp), ("conv_state_out", _vp),
+        ("chunk", _i64),
+    ]
+
+
+class UpdateArgs(C.Structure):
+    _fields_ = [
+        ("mode", _i32), ("dtype", _i32), ("delta_softplus", _i32), ("reserved0", _i32),
+        ("batch", _i64), ("d_inner", _i64), ("nheads", _i64), ("headdim", _i64), ("ngroups", _i64),
+        ("dstate", _i64), ("d_conv", _i64), ("conv_state_len", _i64),
+        ("state", _vp), ("conv_state", _vp), ("conv_w", _vp), ("conv_b", _vp),
+        ("x", _vp), ("x_batch_stride", _i64),
+        ("z", _vp), ("z_batch_stride", _i64),
+        ("dt", _vp), ("dt_batch_stride", _i64),
+        ("B", _vp), ("B_batch_stride", _i64),
+        ("C", _vp), ("C_batch_stride", _i64),
+        ("y", _vp), ("y_batch_stride", _i64),
+        ("A", _vp), ("D", _vp), ("dt_bias", _vp),
+        ("state_batch_indices", _vp), ("nslots", _i64),
+    ]
+
+
+# Every symbol the header declares, with its ctypes signature.
+SIGNATURES = {
+    "ssm_abi_version": ([], _i32),
+    "ssm_status_string": ([_i32], C.c_char_p),
+    "ssm_last_cuda_error": ([], _i32),
+    "ssm_conv1d_fwd": ([C.POINTER(ConvArgs), _vp], _i32),
+    "ssm_scan_workspace_size": ([C.POINTER(ScanArgs)], C.c_size_t),
+    "ssm_scan_fwd": ([C.POINTER(ScanArgs), _vp, C.c_size_t, _vp], _i32),
+    "ssm_state_update": ([C.POINTER(UpdateArgs), _vp], _i32),
+    "ssm_workspace_error": ([_vp, C.POINTER(_i32), _vp], _i32),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """The loaded ``libssm.so``; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(LIB_PATH):
+                    raise RuntimeError(f"libssm.so not found at {LIB_PATH}: build it with "
+                                       "`python -m state_space_model_conv1d_b200.build` (no CPU fallback exists)")
+                handle = C.CDLL(LIB_PATH)
+                for name, (argtypes, restype) in SIGNATURES.items():
+                    fn = getattr(handle, name)
+                    fn.argtypes = argtypes
+                    fn.restype = restype
+                if handle.ssm_abi_version() != 1:
+                    raise RuntimeError("libssm.so ABI version mismatch")
+                _lib = handle
+    return _lib
+
+
+class SSMError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        l = lib()
+        msg = l.ssm_status_string(status).decode()
+        if status == SSM_ERR_CUDA:
+            msg += f" (cudaError {l.ssm_last_cuda_error()})"
+        super().__init__(f"{what}: {msg} [{status}]")
+        self.status = status
+
+
+def check(status: int, what: str) -> None:
+    if status != SSM_OK:
+        raise SSMError(status, what)

@@ -1,0 +1,255 @@
+"""Thin PyTorch-facing binding of the C ABI (same entry-point names).
+
+Argument marshalling only: shapes and strides are read from the tensors,
+outputs are allocated with PyTorch's allocator when the caller does not pass
+them, and the call is enqueued on the current CUDA stream.  Every step of the
+computation runs inside ``libssm.so``.
+
+Tensor conventions (channel dimension contiguous; batch / token strides free):
+
+Mamba-1: x, z, dt, y ``[b, T, D]``; B, C ``[b, T, N]``; A ``[D, N]``; D,
+dt_bias ``[D]``; h0 / h_final ``[nseq, D, N]``; conv_w ``[D, K]``; conv states
+``[nseq, D, K-1]``.
+
+Mamba-2: x, z, y ``[b, T, H, P]``; dt ``[b, T, H]``; B, C ``[b, T, G, N]``;
+A, D, dt_bias ``[H]``; h0 / h_final ``[nseq, H, P, N]``; conv_w
+``[H*P + 2*G*N, K]`` (x | B | C); conv states ``[nseq, H*P + 2*G*N, K-1]``.
+
+Packed varlen: b = 1 and ``cu_seqlens`` int32 ``[nseq + 1]`` on the device.
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import torch
+
+from . import _abi
+from ._abi import SSM_BF16, SSM_F32, SSM_MAMBA1, SSM_MAMBA2
+
+MAMBA1, MAMBA2 = SSM_MAMBA1, SSM_MAMBA2
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SSM_BF16
+    if t.dtype == torch.float32:
+        return SSM_F32
+    raise TypeError(f"activations must be float32 or bfloat16, got {t.dtype}")
+
+
+def _p(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype=None, device=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _rows(t, inner_dims: int, name: str):
+    """(batch stride, token stride) of a [b, T, *inner] tensor whose inner dims are contiguous."""
+    if t is None:
+        return 0, 0
+    exp = 1
+    for d in range(t.dim() - 1, t.dim() - 1 - inner_dims, -1):
+        if t.shape[d] != 1 and t.stride(d) != exp:
+            raise ValueError(f"{name}: the channel dimensions must be contiguous")
+        exp *= t.shape[d]
+    return t.stride(0), t.stride(1)
+
+
+def _c32(t, name):
+    if t is None:
+        return None
+    _need(t, name, torch.float32)
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous float32")
+    return t
+
+
+def conv1d_fwd(x, weight, bias=None, *, state_in=None, state_out=None, cu_seqlens=None, activation=True,
+               out=None, stream=None):
+    """Causal depthwise conv over ``x [b, T, C]`` with weight ``[C, K]``."""
+    _need(x, "x")
+    b, T, Cn = x.shape
+    K = weight.shape[1]
+    if out is None:
+        out = torch.empty((b, T, Cn), dtype=x.dtype, device=x.device)
+    a = _abi.ConvArgs()
+    a.batch, a.seqlen, a.channels, a.width = b, T, Cn, K
+    a.dtype, a.activation = _dtype_code(x), int(bool(activation))
+    a.nseqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    a.x = _p(x)
+    a.x_batch_stride, a.x_token_stride = _rows(x, 1, "x")
+    a.weight, a.bias = _p(_c32(weight, "weight")), _p(_c32(bias, "bias"))
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        if t is not None and (not t.is_contiguous() or t.dtype != x.dtype):
+            raise ValueError(f"{n} must be contiguous with x's dtype")
+    a.state_in, a.state_out = _p(state_in), _p(state_out)
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32)
+    a.cu_seqlens = _p(cu_seqlens)
+    a.out = _p(out)
+    a.out_batch_stride, a.out_token_stride = _rows(out, 1, "out")
+    _abi.check(_abi.lib().ssm_conv1d_fwd(C.byref(a), _stream(stream)), "ssm_conv1d_fwd")
+    return out
+
+
+def _scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, h0, h_final, cu_seqlens, conv_w, conv_b, conv_state_in,
+               conv_state_out, y, delta_softplus, chunk):
+    a = _abi.ScanArgs()
+    a.mode, a.dtype, a.delta_softplus = mode, _dtype_code(x), int(bool(delta_softplus))
+    b, T = x.shape[0], x.shape[1]
+    if mode == MAMBA1:
+        Dn, N = x.shape[2], B.shape[2]
+        H, P, G = 0, 0, 1
+        inner_x, inner_dt, inner_bc = 1, 1, 1
+    else:
+        H, P = x.shape[2], x.shape[3]
+        G, N = B.shape[2], B.shape[3]
+        Dn = H * P
+        inner_x, inner_dt, inner_bc = 2, 1, 2
+    a.batch, a.seqlen, a.d_inner, a.nheads, a.headdim, a.ngroups, a.dstate = b, T, Dn, H, P, G, N
+    a.d_conv = 0 if conv_w is None else conv_w.shape[1]
+    a.nseqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    for t, n in ((x, "x"), (dt, "dt"), (B, "B"), (C_, "C"), (z, "z"), (y, "y")):
+        _need(t, n, x.dtype)
+    a.x = _p(x); a.x_batch_stride, a.x_token_stride = _rows(x, inner_x, "x")
+    a.z = _p(z); a.z_batch_stride, a.z_token_stride = _rows(z, inner_x, "z")
+    a.dt = _p(dt); a.dt_batch_stride, a.dt_token_stride = _rows(dt, inner_dt, "dt")
+    a.B = _p(B); a.B_batch_stride, a.B_token_stride = _rows(B, inner_bc, "B")
+    a.C = _p(C_); a.C_batch_stride, a.C_token_stride = _rows(C_, inner_bc, "C")
+    a.y = _p(y); a.y_batch_stride, a.y_token_stride = _rows(y, inner_x, "y")
+    a.A, a.D, a.dt_bias = _p(_c32(A, "A")), _p(_c32(D, "D")), _p(_c32(dt_bias, "dt_bias"))
+    a.h0, a.h_final = _p(_c32(h0, "h0")), _p(_c32(h_final, "h_final"))
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32)
+    a.cu_seqlens = _p(cu_seqlens)
+    a.conv_w, a.conv_b = _p(_c32(conv_w, "conv_w")), _p(_c32(conv_b, "conv_b"))
+    for t, n in ((conv_state_in, "conv_state_in"), (conv_state_out, "conv_state_out")):
+        if t is not None and (not t.is_contiguous() or t.dtype != x.dtype):
+            raise ValueError(f"{n} must be contiguous with x's dtype")
+    a.conv_state_in, a.conv_state_out = _p(conv_state_in), _p(conv_state_out)
+    a.chunk = int(chunk)
+    return a
+
+
+def scan_workspace_size(mode, x, dt, A, B, C_, *, cu_seqlens=None, **_):
+    a = _abi.ScanArgs()
+    a.mode = mode
+    a.cu_seqlens = _p(cu_seqlens)
+    a.nseqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    return int(_abi.lib().ssm_scan_workspace_size(C.byref(a)))
+
+
+def scan_fwd(mode, x, dt, A, B, C_, *, D=None, z=None, dt_bias=None, h0=None, cu_seqlens=None, conv_w=None,
+             conv_b=None, conv_state_in=None, delta_softplus=True, y=None, h_final=None, conv_state_out=None,
+             return_final_state=True, return_conv_state=None, workspace=None, chunk=0, stream=None):
+    """Forward selective scan (conv fused in front when ``conv_w`` is given).
+
+    Returns ``(y, h_final, conv_state_out)``; the last two are None when not
+    requested.  ``workspace`` (uint8 CUDA tensor) is allocated when needed and
+    not given.
+    """
+    _need(x, "x")
+    if y is None:
+        y = torch.empty(x.shape, dtype=x.dtype, device=x.device)
+    nseq = x.shape[0] if cu_seqlens is None else cu_seqlens.numel() - 1
+    if mode == MAMBA1:
+        hshape = (nseq, x.shape[2], B.shape[2])
+        cdim = x.shape[2]
+    else:
+        hshape = (nseq, x.shape[2], x.shape[3], B.shape[3])
+        cdim = x.shape[2] * x.shape[3] + 2 * B.shape[2] * B.shape[3]
+    if h_final is None and return_final_state:
+        h_final = torch.empty(hshape, dtype=torch.float32, device=x.device)
+    if return_conv_state is None:
+        return_conv_state = conv_w is not None and conv_w.shape[1] > 1
+    if conv_state_out is None and return_conv_state and conv_w is not None and conv_w.shape[1] > 1:
+        conv_state_out = torch.empty((nseq, cdim, conv_w.shape[1] - 1), dtype=x.dtype, device=x.device)
+    a = _scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, h0, h_final, cu_seqlens, conv_w, conv_b, conv_state_in,
+                   conv_state_out, y, delta_softplus, chunk)
+    l = _abi.lib()
+    need = int(l.ssm_scan_workspace_size(C.byref(a)))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_ptr = _p(workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    _abi.check(l.ssm_scan_fwd(C.byref(a), ws_ptr, ws_bytes, _stream(stream)), "ssm_scan_fwd")
+    return y, h_final, conv_state_out
+
+
+def workspace_error(workspace, stream=None):
+    """Synchronizes and returns the device error code held in a scan workspace (0 = none)."""
+    code = _abi._i32(0)
+    st = _abi.lib().ssm_workspace_error(_p(workspace), C.byref(code), _stream(stream))
+    if st not in (_abi.SSM_OK, _abi.SSM_ERR_DEVICE):
+        _abi.check(st, "ssm_workspace_error")
+    return int(code.value)
+
+
+def state_update(mode, state, conv_state, x, dt, A, B, C_, *, D=None, z=None, dt_bias=None, conv_w=None,
+                 conv_b=None, delta_softplus=True, state_batch_indices=None, y=None, stream=None):
+    """One decode token per row, state and conv_state updated in place; returns y.
+
+    Mamba-1: x, z, dt ``[b, D]``; B, C ``[b, N]``; state ``[slots, D, N]``.
+    Mamba-2: x, z ``[b, H, P]``; dt ``[b, H]``; B, C ``[b, G, N]``; state
+    ``[slots, H, P, N]``.  conv_state ``[slots, conv_dim, L]`` with L >= K-1.
+    """
+    _need(x, "x")
+    if y is None:
+        y = torch.empty(x.shape, dtype=x.dtype, device=x.device)
+    a = _abi.UpdateArgs()
+    a.mode, a.dtype, a.delta_softplus = mode, _dtype_code(x), int(bool(delta_softplus))
+    b = x.shape[0]
+    if mode == MAMBA1:
+        Dn, N = x.shape[1], B.shape[1]
+        H, P, G = 0, 0, 1
+    else:
+        H, P = x.shape[1], x.shape[2]
+        G, N = B.shape[1], B.shape[2]
+        Dn = H * P
+    a.batch, a.d_inner, a.nheads, a.headdim, a.ngroups, a.dstate = b, Dn, H, P, G, N
+    a.d_conv = 0 if conv_w is None else conv_w.shape[1]
+    a.conv_state_len = 0 if conv_state is None else conv_state.shape[-1]
+    if not state.is_contiguous() or state.dtype != torch.float32:
+        raise ValueError("state must be contiguous float32")
+    if conv_state is not None and (not conv_state.is_contiguous() or conv_state.dtype != x.dtype):
+        raise ValueError("conv_state must be contiguous with x's dtype")
+    a.state, a.conv_state = _p(state), _p(conv_state)
+    a.conv_w, a.conv_b = _p(_c32(conv_w, "conv_w")), _p(_c32(conv_b, "conv_b"))
+
+    def bs(t, name, inner):
+        if t is None:
+            return 0
+        _need(t, name, x.dtype)
+        exp = 1
+        for d in range(t.dim() - 1, t.dim() - 1 - inner, -1):
+            if t.shape[d] != 1 and t.stride(d) != exp:
+                raise ValueError(f"{name}: the channel dimensions must be contiguous")
+            exp *= t.shape[d]
+        return t.stride(0)
+
+    inner = 1 if mode == MAMBA1 else 2
+    a.x, a.x_batch_stride = _p(x), bs(x, "x", inner)
+    a.z, a.z_batch_stride = _p(z), bs(z, "z", inner)
+    a.dt, a.dt_batch_stride = _p(dt), bs(dt, "dt", 1)
+    a.B, a.B_batch_stride = _p(B), bs(B, "B", inner)
+    a.C, a.C_batch_stride = _p(C_), bs(C_, "C", inner)
+    a.y, a.y_batch_stride = _p(y), bs(y, "y", inner)
+    a.A, a.D, a.dt_bias = _p(_c32(A, "A")), _p(_c32(D, "D")), _p(_c32(dt_bias, "dt_bias"))
+    if state_batch_indices is not None:
+        _need(state_batch_indices, "state_batch_indices", torch.int32)
+    a.state_batch_indices = _p(state_batch_indices)
+    a.nslots = state.shape[0]
+    _abi.check(_abi.lib().ssm_state_update(C.byref(a), _stream(stream)), "ssm_state_update")
+    return y

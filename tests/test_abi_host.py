@@ -1,0 +1,189 @@
+"""The C-ABI library on the host: it loads, exports every symbol the header
+declares, and rejects bad arguments before anything reaches a GPU.
+
+Every call here is one the library must refuse during host-side validation,
+so nothing is launched (no GPU is needed, and none is touched on a GPU machine).
+"""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+from state_space_model_conv1d_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+
+def declared_symbols():
+    names = set()
+    for h in HEADERS:
+        src = open(h).read()
+        names |= set(re.findall(r"SSM_API\s+[\w\s\*]+?\b(ssm_\w+)\s*\(", src))
+    return names
+
+
+def test_library_exists_and_loads():
+    assert os.path.exists(_abi.LIB_PATH), "build libssm.so first"
+    lib = _abi.lib()
+    assert lib.ssm_abi_version() == 1
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_symbols()
+    assert {"ssm_conv1d_fwd", "ssm_scan_fwd", "ssm_state_update", "ssm_scan_workspace_size"} <= names
+    out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert names <= exported, f"missing: {names - exported}"
+    assert set(_abi.SIGNATURES) == names, "ctypes signatures must mirror the header"
+    # nothing beyond the ABI leaks out of the library
+    assert {e for e in exported if e.startswith("ssm")} == names
+
+
+def test_struct_layouts_match_header(tmp_path):
+    """Compile a probe against the real header and compare every field offset
+    with the ctypes mirror."""
+    probes = []
+    for cname, py in (("ssm_conv_args", _abi.ConvArgs), ("ssm_scan_args", _abi.ScanArgs),
+                      ("ssm_update_args", _abi.UpdateArgs)):
+        probes.append(f'printf("{cname} sizeof %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            probes.append(f'printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    src = tmp_path / "probe.c"
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "ssm.h"\nint main(void){' + "".join(probes) +
+                   "return 0;}\n")
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines():
+        c, f, v = line.split()
+        got[(c, f)] = int(v)
+    for cname, py in (("ssm_conv_args", _abi.ConvArgs), ("ssm_scan_args", _abi.ScanArgs),
+                      ("ssm_update_args", _abi.UpdateArgs)):
+        assert got[(cname, "sizeof")] == C.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
+
+
+def test_status_strings():
+    lib = _abi.lib()
+    for s in range(0, -7, -1):
+        assert lib.ssm_status_string(s)
+    assert lib.ssm_status_string(-99) == b"unknown status"
+
+
+FAKE = 0x10000000  # never dereferenced: every call below is rejected on the host
+
+
+def _scan(**kw):
+    a = _abi.ScanArgs()
+    a.mode, a.dtype, a.delta_softplus = 2, _abi.SSM_BF16, 1
+    a.batch, a.seqlen, a.d_inner, a.nheads, a.headdim, a.ngroups, a.dstate = 2, 16, 8, 4, 2, 2, 16
+    for k in ("x", "dt", "B", "C", "y", "A"):
+        setattr(a, k, FAKE)
+    a.x_token_stride, a.x_batch_stride = 8, 128
+    a.y_token_stride, a.y_batch_stride = 8, 128
+    a.dt_token_stride, a.dt_batch_stride = 4, 64
+    a.B_token_stride, a.B_batch_stride = 32, 512
+    a.C_token_stride, a.C_batch_stride = 32, 512
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(mode=3), _abi.SSM_ERR_INVALID_ARG),
+    (dict(dtype=7), _abi.SSM_ERR_INVALID_ARG),
+    (dict(ngroups=3), _abi.SSM_ERR_INVALID_ARG),                 # heads not divisible into groups
+    (dict(nheads=3), _abi.SSM_ERR_INVALID_ARG),                  # nheads * headdim != d_inner
+    (dict(dstate=1024), _abi.SSM_ERR_UNSUPPORTED),
+    (dict(x=None), _abi.SSM_ERR_INVALID_ARG),
+    (dict(A=None), _abi.SSM_ERR_INVALID_ARG),
+    (dict(x=FAKE + 1), _abi.SSM_ERR_ALIGNMENT),                  # bf16 needs 2-byte alignment
+    (dict(h0=FAKE + 2), _abi.SSM_ERR_ALIGNMENT),
+    (dict(x_token_stride=4), _abi.SSM_ERR_INVALID_ARG),          # rows overlap
+    (dict(d_conv=2), _abi.SSM_ERR_INVALID_ARG),                  # conv width without weights
+    (dict(d_conv=9, conv_w=FAKE), _abi.SSM_ERR_UNSUPPORTED),
+    (dict(cu_seqlens=FAKE, nseqs=2), _abi.SSM_ERR_INVALID_ARG),  # varlen needs batch == 1
+    (dict(cu_seqlens=FAKE, nseqs=2, batch=1), _abi.SSM_ERR_WORKSPACE),
+    (dict(mode=1, ngroups=2, d_inner=8), _abi.SSM_ERR_UNSUPPORTED),
+    (dict(mode=1, ngroups=1, dstate=128), _abi.SSM_ERR_UNSUPPORTED),
+    (dict(delta_softplus=2), _abi.SSM_ERR_INVALID_ARG),
+])
+def test_scan_rejects(kw, status):
+    a = _scan(**kw)
+    assert _abi.lib().ssm_scan_fwd(C.byref(a), None, 0, None) == status
+
+
+def test_scan_rejects_null_args():
+    assert _abi.lib().ssm_scan_fwd(None, None, 0, None) == _abi.SSM_ERR_INVALID_ARG
+    assert _abi.lib().ssm_conv1d_fwd(None, None) == _abi.SSM_ERR_INVALID_ARG
+    assert _abi.lib().ssm_state_update(None, None) == _abi.SSM_ERR_INVALID_ARG
+
+
+def test_workspace_size_is_host_only():
+    a = _scan()
+    assert _abi.lib().ssm_scan_workspace_size(C.byref(a)) == 0
+    a = _scan(cu_seqlens=FAKE, nseqs=1000, batch=1)
+    n = _abi.lib().ssm_scan_workspace_size(C.byref(a))
+    assert n >= 256 + 4 * 1000 and n % 256 == 0
+
+
+def _conv(**kw):
+    a = _abi.ConvArgs()
+    a.batch, a.seqlen, a.channels, a.width, a.dtype, a.activation = 2, 8, 16, 4, _abi.SSM_F32, 1
+    a.x, a.out, a.weight = FAKE, FAKE, FAKE
+    a.x_token_stride, a.x_batch_stride, a.out_token_stride, a.out_batch_stride = 16, 128, 16, 128
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(width=0), _abi.SSM_ERR_UNSUPPORTED),
+    (dict(width=9), _abi.SSM_ERR_UNSUPPORTED),
+    (dict(weight=None), _abi.SSM_ERR_INVALID_ARG),
+    (dict(activation=2), _abi.SSM_ERR_INVALID_ARG),
+    (dict(x=FAKE + 2), _abi.SSM_ERR_ALIGNMENT),
+    (dict(out_token_stride=8), _abi.SSM_ERR_INVALID_ARG),
+    (dict(channels=0), _abi.SSM_ERR_INVALID_ARG),
+    (dict(cu_seqlens=FAKE, nseqs=3), _abi.SSM_ERR_INVALID_ARG),
+])
+def test_conv_rejects(kw, status):
+    a = _conv(**kw)
+    assert _abi.lib().ssm_conv1d_fwd(C.byref(a), None) == status
+
+
+def _upd(**kw):
+    a = _abi.UpdateArgs()
+    a.mode, a.dtype, a.delta_softplus = 2, _abi.SSM_BF16, 1
+    a.batch, a.d_inner, a.nheads, a.headdim, a.ngroups, a.dstate = 4, 8, 4, 2, 2, 16
+    a.d_conv, a.conv_state_len = 4, 4
+    for k in ("state", "conv_state", "conv_w", "x", "dt", "B", "C", "y", "A"):
+        setattr(a, k, FAKE)
+    a.x_batch_stride, a.y_batch_stride, a.dt_batch_stride = 8, 8, 4
+    a.B_batch_stride = a.C_batch_stride = 32
+    a.nslots = 4
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(conv_state_len=2), _abi.SSM_ERR_INVALID_ARG),
+    (dict(conv_state=None), _abi.SSM_ERR_INVALID_ARG),
+    (dict(state=FAKE + 4), _abi.SSM_ERR_ALIGNMENT),              # float4 state rows need 16 bytes
+    (dict(nslots=2), _abi.SSM_ERR_INVALID_ARG),                  # fewer slots than rows, no indices
+    (dict(ngroups=3), _abi.SSM_ERR_INVALID_ARG),
+    (dict(x_batch_stride=4), _abi.SSM_ERR_INVALID_ARG),
+    (dict(mode=0), _abi.SSM_ERR_INVALID_ARG),
+])
+def test_update_rejects(kw, status):
+    a = _upd(**kw)
+    assert _abi.lib().ssm_state_update(C.byref(a), None) == status
+
+
+def test_workspace_error_needs_a_workspace():
+    assert _abi.lib().ssm_workspace_error(None, None, None) == _abi.SSM_ERR_INVALID_ARG
