@@ -69,6 +69,78 @@ SSM_DEVINL float conv_roll4_bf16(__nv_bfloat16 *cs, const float *w, float b, int
     return silu(acc);
 }
 
+SSM_DEVINL int64_t hh_first(int unit, int64_t hpg) { return (int64_t)unit * hpg; }
+
+// Rows [0, nrows) of one Mamba-2 group: row = (local head, p), state row at
+// stb + (c0 + row) * N, N = 128 * NV.  Lane l owns states 4 * (l + 32 v) .. +3.
+template <int NV, typename T>
+SSM_DEVINL void stream_rows(float *stb, int64_t c0, int64_t h0, int64_t nrows, int64_t P, const float *xs,
+                            const float *Bs, const float *Cs, const float *dls, const float *das, const float *Dp,
+                            const T *zr, T *yr, int warp, int lane) {
+    constexpr int64_t N = 128 * NV;
+    constexpr int R = 4;                       // rows in flight per warp
+    float4 Bv[NV], Cv[NV];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+        Bv[v] = *reinterpret_cast<const float4 *>(Bs + 4 * (lane + 32 * v));
+        Cv[v] = *reinterpret_cast<const float4 *>(Cs + 4 * (lane + 32 * v));
+    }
+    constexpr int kWarps = kThreads / 32;
+    for (int64_t row0 = (int64_t)warp * R; row0 < nrows; row0 += (int64_t)kWarps * R) {
+        float4 sv[R][NV];
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int64_t row = row0 + i;
+            if (row < nrows) {
+                const float *srow = stb + (c0 + row) * N;
+#pragma unroll
+                for (int v = 0; v < NV; ++v) sv[i][v] = __ldcs(reinterpret_cast<const float4 *>(srow + 4 * (lane + 32 * v)));
+            }
+        }
+        float acc[R];
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int64_t row = row0 + i;
+            acc[i] = 0.f;
+            if (row < nrows) {
+                const int64_t hl = row / P;
+                const float dA = das[hl];
+                const float dxv = dls[hl] * xs[row];
+                float *srow = stb + (c0 + row) * N;
+#pragma unroll
+                for (int v = 0; v < NV; ++v) {
+                    float4 s4 = sv[i][v];
+                    s4.x = fmaf(dA, s4.x, dxv * Bv[v].x);
+                    s4.y = fmaf(dA, s4.y, dxv * Bv[v].y);
+                    s4.z = fmaf(dA, s4.z, dxv * Bv[v].z);
+                    s4.w = fmaf(dA, s4.w, dxv * Bv[v].w);
+                    __stcs(reinterpret_cast<float4 *>(srow + 4 * (lane + 32 * v)), s4);
+                    acc[i] = fmaf(Cv[v].x, s4.x, acc[i]);
+                    acc[i] = fmaf(Cv[v].y, s4.y, acc[i]);
+                    acc[i] = fmaf(Cv[v].z, s4.z, acc[i]);
+                    acc[i] = fmaf(Cv[v].w, s4.w, acc[i]);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < R; ++i)
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+        if (lane < R) {
+            const int64_t row = row0 + lane;
+            if (row < nrows) {
+                float a0 = acc[0];
+#pragma unroll
+                for (int i = 1; i < R; ++i) a0 = (lane == i) ? acc[i] : a0;
+                const int64_t hl = row / P, ch = c0 + row;
+                float yv = a0 + (Dp ? Dp[h0 + hl] : 0.f) * xs[row];
+                if (zr) yv *= silu(Elem<T>::ld(zr + ch));
+                Elem<T>::st(yr + ch, yv);
+            }
+        }
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const DecArgs a) {
     extern __shared__ __align__(16) float sm[];
@@ -89,8 +161,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecArgs a) {
         for (int64_t i = threadIdx.x; i < nx; i += kThreads) Elem<T>::st(yr + c0 + i, 0.f);
         return;
     }
-    float *xs = sm;                    // [nx] conv output of x
-    float *Bs = xs + nx;               // [N]
+    float *xs = sm;                    // [nx] conv output of x (padded to 4 for 16-byte alignment)
+    float *Bs = xs + ((nx + 3) & ~(int64_t)3);   // [N]
     float *Cs = Bs + N;                // [N]
     float *dls = Cs + N;               // [nh] delta
     float *das = dls + nh;             // [nh] exp(delta A)   (Mamba-2 only)
@@ -140,8 +212,19 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecArgs a) {
     }
     __syncthreads();
 
-    // state rows: (head, p) pairs of this CTA, N states each; LPR lanes per row
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const T *zr = a.z ? static_cast<const T *>(a.z) + r * a.z_bs : nullptr;
+    float *stb = a.state + slot * a.Dn * N;
+    if (m2 && (N == 128 || N == 256)) {
+        // Streaming fast path: one warp per 128-state row segment, each lane one
+        // float4 per 128 states; four rows in flight per warp; B / C held in
+        // registers for the whole group.
+        if (N == 128) stream_rows<1, T>(stb, c0, hh_first(unit, hpg), nh * P, P, xs, Bs, Cs, dls, das, a.D, zr, yr, warp, lane);
+        else stream_rows<2, T>(stb, c0, hh_first(unit, hpg), nh * P, P, xs, Bs, Cs, dls, das, a.D, zr, yr, warp, lane);
+        return;
+    }
+
+    // state rows: (head, p) pairs of this CTA, N states each; LPR lanes per row
     const bool vec = (N % 4 == 0);
     int lpr = 1;                                                        // lanes per row, a power of two
     if (vec)
@@ -149,8 +232,6 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecArgs a) {
     const int rpw = 32 / lpr;                                          // rows per warp pass
     const int sub = lane / lpr, sl = lane % lpr;
     const int64_t nrows = nh * P;
-    float *stb = a.state + slot * a.Dn * N;
-    const T *zr = a.z ? static_cast<const T *>(a.z) + r * a.z_bs : nullptr;
     for (int64_t row0 = (int64_t)warp * rpw; row0 < nrows; row0 += (int64_t)(kThreads / 32) * rpw) {
         const int64_t row = row0 + sub;
         const bool rv = row < nrows && vec;
@@ -219,7 +300,7 @@ cudaError_t launch_typed(const DecArgs &a, int64_t batch, cudaStream_t st) {
     const int64_t units = m2 ? a.G : (a.Dn + kM1Channels - 1) / kM1Channels;
     const int64_t nx = m2 ? (a.H / a.G) * a.P : kM1Channels;
     const int64_t nh = m2 ? a.H / a.G : kM1Channels;
-    const size_t smem = (size_t)(nx + 2 * a.N + 2 * nh) * sizeof(float);
+    const size_t smem = (size_t)(((nx + 3) & ~(int64_t)3) + 2 * a.N + 2 * nh) * sizeof(float);
     auto kern = decode_kernel<T>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -199,6 +199,7 @@ def _decode_oracle(mode, d, nsteps):
 
 @pytest.mark.parametrize("mode,H,P,G,N,Ls,dtype", [
     (M2, 8, 64, 2, 128, 4, "bf16"),
+    (M2, 4, 33, 2, 256, 4, "f32"),    # streaming path with 256 states and an odd headdim
     (M2, 6, 32, 3, 16, 3, "f32"),
     (M2, 4, 16, 1, 10, 5, "f32"),     # dstate not a multiple of 4
     (M1, 300, 1, 1, 16, 4, "bf16"),   # Mamba-1: H is d_inner
