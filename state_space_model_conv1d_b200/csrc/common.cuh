@@ -49,6 +49,26 @@ SSM_DEVINL float softplus(float u) {
 // overflows to +inf and the reciprocal gives 0, the correct limit.
 SSM_DEVINL float silu(float v) { return v * rcp(1.f + ex2(-v * kLog2e)); }
 
+// tanh on the MUFU unit (tanh.approx: relative error about 2^-11).
+SSM_DEVINL float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// silu for a given activation dtype.  bf16 data (whose own rounding is 2^-9)
+// takes sigmoid(v) = (1 + tanh(v/2)) / 2 on one MUFU op; fp32 data keeps the
+// exp + reciprocal form above.
+template <typename T>
+SSM_DEVINL float silu_fast(float v) {
+    if constexpr (sizeof(T) == 2) {
+        const float hv = 0.5f * v;
+        return fmaf(hv, tanh_approx(hv), hv);
+    } else {
+        return silu(v);
+    }
+}
+
 // ----------------------------------------------------------- element I/O
 template <typename T> struct Elem;
 template <> struct Elem<float> {

@@ -22,7 +22,7 @@
 namespace ssm {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 1024;         // 2 CTAs per SM: 296 slots, so ~7 waves of (row, group) units
 constexpr int kM1Channels = 256;
 
 struct DecArgs {
@@ -53,14 +53,17 @@ SSM_DEVINL float conv_roll(T *cs, int64_t Ls, const float *w, float b, int K, fl
 }
 
 // Fast path for bf16 with a 4-wide window: one 8-byte load and store.
-SSM_DEVINL float conv_roll4_bf16(__nv_bfloat16 *cs, const float *w, float b, int K, float u) {
+// wr holds the taps right-aligned (wr[7] multiplies the new input, wr[7 - m]
+// the input m steps back, zeros before the first tap), so no index is dynamic.
+SSM_DEVINL float conv_roll4_bf16(__nv_bfloat16 *cs, const float (&wr)[kMaxConvWidth], float b, float u) {
     uint2 r = *reinterpret_cast<const uint2 *>(cs);
     float s0 = __uint_as_float(r.x << 16), s1 = __uint_as_float(r.x & 0xffff0000u);
     float s2 = __uint_as_float(r.y << 16), s3 = __uint_as_float(r.y & 0xffff0000u);
-    const float win[4] = {s0, s1, s2, s3};
-    float acc = b;
-    for (int k = 0; k < K - 1; ++k) acc = fmaf(w[k], win[4 - (K - 1) + k], acc);
-    acc = fmaf(w[K - 1], u, acc);
+    float acc = fmaf(wr[7], u, b);
+    acc = fmaf(wr[6], s3, acc);
+    acc = fmaf(wr[5], s2, acc);
+    acc = fmaf(wr[4], s1, acc);
+    acc = fmaf(wr[3], s0, acc);
     __nv_bfloat162 lo = __floats2bfloat162_rn(s1, s2);
     __nv_bfloat162 hi = __floats2bfloat162_rn(s3, u);   // u is a bf16 value already: exact
     r.x = *reinterpret_cast<uint32_t *>(&lo);
@@ -78,7 +81,7 @@ SSM_DEVINL void stream_rows(float *stb, int64_t c0, int64_t h0, int64_t nrows, i
                             const float *Bs, const float *Cs, const float *dls, const float *das, const float *Dp,
                             const T *zr, T *yr, int warp, int lane) {
     constexpr int64_t N = 128 * NV;
-    constexpr int R = 4;                       // rows in flight per warp
+    constexpr int R = NV == 1 ? 4 : 2;         // rows in flight per warp (within 64 registers)
     float4 Bv[NV], Cv[NV];
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
@@ -181,13 +184,21 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecArgs a) {
         else { ch = a.Dn + a.G * N + unit * N + (i - nx - N); u = Elem<T>::ld(Cr + (i - nx - N)); }
         float v = u;
         if (K > 0) {
-            float w[kMaxConvWidth];
-            for (int k = 0; k < K; ++k) w[k] = a.conv_w[ch * K + k];
+            const float *w = a.conv_w + ch * K;
             const float b = a.conv_b ? a.conv_b[ch] : 0.f;
             T *cs = csb + ch * a.Ls;
             if constexpr (sizeof(T) == 2) {
-                if (a.Ls == 4 && ((uintptr_t)cs & 7) == 0) v = conv_roll4_bf16(reinterpret_cast<__nv_bfloat16 *>(cs), w, b, K, u);
-                else v = conv_roll<T>(cs, a.Ls, w, b, K, u);
+                if (a.Ls == 4 && K <= 5 && ((uintptr_t)cs & 7) == 0) {
+                    float wr[kMaxConvWidth];
+#pragma unroll
+                    for (int j = 0; j < kMaxConvWidth; ++j) {
+                        const int k = K - kMaxConvWidth + j;
+                        wr[j] = k >= 0 ? a.conv_w[ch * K + k] : 0.f;
+                    }
+                    v = conv_roll4_bf16(reinterpret_cast<__nv_bfloat16 *>(cs), wr, b, u);
+                } else {
+                    v = conv_roll<T>(cs, a.Ls, w, b, K, u);
+                }
             } else {
                 v = conv_roll<T>(cs, a.Ls, w, b, K, u);
             }

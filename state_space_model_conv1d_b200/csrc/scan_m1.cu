@@ -61,8 +61,7 @@ struct SmemM1 {
     T rC[2][kTC][NP];
     float halo[2][kHalo][kDB];
     float xc[kTC][kDB];
-    float dl[kTC][kDB];
-    float dx[kTC][kDB];
+    float2 dd[kTC][kDB];      // (delta, delta * xc)
     float g[kTC][kDB];
     float y[kTC][kDB];
     float Bf[kTC][NP];
@@ -165,7 +164,11 @@ scan_m1_kernel(const M1Args a) {
     const int sd = tid / kLanes, q = tid % kLanes;
     const int64_t sch = d0 + sd;
     const bool svalid = sch < Dn;
+    // states of this lane: n = VW * (q + 4 j) + e; kept as fp32 pairs (h2, A2p)
+    // for the packed path, or scalars when a lane holds a single state
+    constexpr int NPAIR = SPT >= 2 ? SPT / 2 : 1;
     float A2[SPT], h[SPT];
+    float2 A2p[NPAIR], h2[NPAIR];
 #pragma unroll
     for (int j = 0; j < NJ; ++j)
 #pragma unroll
@@ -175,6 +178,13 @@ scan_m1_kernel(const M1Args a) {
             A2[j * VW + e] = ok ? a.A[sch * N + n] * kLog2e : 0.f;
             h[j * VW + e] = (ok && a.h0) ? a.h0[((int64_t)s * Dn + sch) * N + n] : 0.f;
         }
+#pragma unroll
+    for (int p = 0; p < NPAIR; ++p) {
+        if constexpr (SPT >= 2) {
+            A2p[p] = make_float2(A2[2 * p], A2[2 * p + 1]);
+            h2[p] = make_float2(h[2 * p], h[2 * p + 1]);
+        }
+    }
     const float Dd = (svalid && a.D) ? a.D[sch] : 0.f;
 
     // ---- conv halo of chunk 0: the carried state (the K-1 raw inputs before the first token)
@@ -214,7 +224,7 @@ scan_m1_kernel(const M1Args a) {
                         float acc = fmaf(wr[kHalo], cur, cb);
 #pragma unroll
                         for (int j = 0; j < kHalo; ++j) acc = fmaf(wr[j], win[j], acc);
-                        xcv = silu(acc);
+                        xcv = silu_fast<T>(acc);
                     } else {
                         xcv = cur;
                     }
@@ -223,11 +233,10 @@ scan_m1_kernel(const M1Args a) {
                     win[kHalo - 1] = cur;
                     const float u = Elem<T>::ld(&sm.rdt[buf][t][pd]) + dtb;
                     dlt = a.softplus ? softplus(u) : u;
-                    if (zg) gv = silu(Elem<T>::ld(&sm.rz[buf][t][pd]));
+                    if (zg) gv = silu_fast<T>(Elem<T>::ld(&sm.rz[buf][t][pd]));
                 }
                 sm.xc[t][pd] = xcv;
-                sm.dl[t][pd] = dlt;           // delta = 0 past the end: the state stays put
-                sm.dx[t][pd] = dlt * xcv;
+                sm.dd[t][pd] = make_float2(dlt, dlt * xcv);   // delta = 0 past the end: the state stays put
                 sm.g[t][pd] = gv;
             }
             // next halo: the last K-1 raw inputs up to this chunk's end
@@ -254,32 +263,37 @@ scan_m1_kernel(const M1Args a) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int t = t4 + i;
-                const float dl = sm.dl[t][sd], dxv = sm.dx[t][sd];
-                float ac = 0.f;
+                const float2 dd = sm.dd[t][sd];                      // (delta, delta * xc)
+                if constexpr (VW >= 2) {
+                    // packed fp32x2: two states per FMUL2 / FFMA2 instruction
+                    const float2 dl2 = make_float2(dd.x, dd.x), dx2 = make_float2(dd.y, dd.y);
+                    float2 ac2 = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int j = 0; j < NJ; ++j) {
-                    float bv[VW], cv[VW];
-                    const int n0 = VW * (q + kLanes * j);
-                    if constexpr (VW == 4) {
-                        const float4 b4 = *reinterpret_cast<const float4 *>(&sm.Bf[t][n0]);
-                        const float4 c4 = *reinterpret_cast<const float4 *>(&sm.Cf[t][n0]);
-                        bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
-                        cv[0] = c4.x; cv[1] = c4.y; cv[2] = c4.z; cv[3] = c4.w;
-                    } else if constexpr (VW == 2) {
-                        const float2 b2 = *reinterpret_cast<const float2 *>(&sm.Bf[t][n0]);
-                        const float2 c2 = *reinterpret_cast<const float2 *>(&sm.Cf[t][n0]);
-                        bv[0] = b2.x; bv[1] = b2.y; cv[0] = c2.x; cv[1] = c2.y;
-                    } else {
-                        bv[0] = sm.Bf[t][n0]; cv[0] = sm.Cf[t][n0];
-                    }
+                    for (int j = 0; j < NJ; ++j) {
+                        const int n0 = VW * (q + kLanes * j);
 #pragma unroll
-                    for (int e = 0; e < VW; ++e) {
-                        const float dA = ex2(dl * A2[j * VW + e]);
-                        h[j * VW + e] = fmaf(dA, h[j * VW + e], dxv * bv[e]);
-                        ac = fmaf(cv[e], h[j * VW + e], ac);
+                        for (int e = 0; e < VW; e += 2) {
+                            const float2 b2 = *reinterpret_cast<const float2 *>(&sm.Bf[t][n0 + e]);
+                            const float2 c2 = *reinterpret_cast<const float2 *>(&sm.Cf[t][n0 + e]);
+                            const int pi = (j * VW + e) / 2;
+                            const float2 arg = __fmul2_rn(dl2, A2p[pi]);
+                            const float2 dA = make_float2(ex2(arg.x), ex2(arg.y));
+                            h2[pi] = __ffma2_rn(dA, h2[pi], __fmul2_rn(dx2, b2));
+                            ac2 = __ffma2_rn(c2, h2[pi], ac2);
+                        }
                     }
+                    acc[i] = ac2.x + ac2.y;
+                } else {
+                    float ac = 0.f;
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j) {
+                        const int n0 = q + kLanes * j;
+                        const float dA = ex2(dd.x * A2[j]);
+                        h[j] = fmaf(dA, h[j], dd.y * sm.Bf[t][n0]);
+                        ac = fmaf(sm.Cf[t][n0], h[j], ac);
+                    }
+                    acc[i] = ac;
                 }
-                acc[i] = ac;
             }
             // reduce-scatter over the 4 lanes of the channel: lane q ends with token t4 + q
             const bool hi = (q & 2) != 0;
@@ -328,6 +342,13 @@ scan_m1_kernel(const M1Args a) {
         }
     }
     asm volatile("cp.async.wait_all;\n" ::);
+    if constexpr (SPT >= 2) {
+#pragma unroll
+        for (int p = 0; p < NPAIR; ++p) {
+            h[2 * p] = h2[p].x;
+            h[2 * p + 1] = h2[p].y;
+        }
+    }
     if (a.h_final && svalid) {
 #pragma unroll
         for (int j = 0; j < NJ; ++j)
