@@ -11,16 +11,21 @@
 //
 // Design (sm_100a, CUDA cores).  One CTA owns one sequence and DB = 32
 // channels and walks the tokens in chunks of TC.  Raw x / dt / z / B / C
-// chunk tiles are staged in shared memory with 16-byte cp.async copies, two
-// chunks ahead of the compute (double buffer), so HBM latency hides behind
-// the scan.  A cooperative prologue computes conv + SiLU, delta, delta*x and
-// the gate once per (token, channel) into fp32 tiles.  Then 4 lanes per
-// channel advance N/4 states each in registers; the carry across chunks is
-// the fp32 state staying in registers, seeded from h0 (the (1, h0) seed of
-// the pair scan).  The 4 lanes' partial read-outs of 4 consecutive tokens
-// are combined by a two-level shuffle reduce-scatter, so each lane finishes
-// one token's y.  The K-1 raw rows before each chunk live in a small
-// double-buffered halo, which is also what conv_state_out receives.
+// chunk tiles are staged in shared memory with 16-byte cp.async copies into
+// a 3-deep ring.  A cooperative prologue computes conv + SiLU, delta,
+// delta*x, D*x and the gate once per (token, channel) into fp32 tiles (two
+// slots).  Then 4 lanes per channel advance N/4 states each in registers;
+// the carry across chunks is the fp32 state staying in registers, seeded
+// from h0 (the (1, h0) seed of the pair scan).  The 4 lanes' partial
+// read-outs of 4 consecutive tokens are combined by a two-level shuffle
+// reduce-scatter, so each lane finishes one token's y.
+//
+// Software pipeline, one CTA barrier per chunk: iteration c scans chunk c,
+// stores y of chunk c-1, runs the prologue of chunk c+1 and issues the copies
+// of chunk c+3.  Warps drift freely inside an iteration, so the MUFU-heavy
+// scan of one warp overlaps the load / convert work of another.  The K-1 raw
+// rows before each chunk live in a double-buffered halo, which is also what
+// conv_state_out receives.
 //
 // Per (token, channel, state) the work is one MUFU exp plus four FP32 ops:
 // with dstate 16 the kernel is bound by the MUFU exp rate, not by HBM.
@@ -51,61 +56,70 @@ struct M1Args {
     SeqView sv;
 };
 
-template <typename T, int SPT>
-struct SmemM1 {
-    static constexpr int NP = kLanes * SPT;             // padded dstate
-    T rx[2][kTC][kDB];
-    T rdt[2][kTC][kDB];
-    T rz[2][kTC][kDB];
-    T rB[2][kTC][NP];
-    T rC[2][kTC][NP];
-    float halo[2][kHalo][kDB];
-    float xc[kTC][kDB];
-    float2 dd[kTC][kDB];      // (delta, delta * xc)
-    float g[kTC][kDB];
-    float y[kTC][kDB];
-    float Bf[kTC][NP];
-    float Cf[kTC][NP];
-};
-
 SSM_DEVINL void cp_async16(void *smem, const void *gmem) {
     const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
 }
 SSM_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-SSM_DEVINL void cp_async_wait1() { asm volatile("cp.async.wait_group 1;\n" ::); }
+template <int N>
+SSM_DEVINL void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
-// Stage rows [0, nv) x cols [col0, col0 + ncols) of a token-major tensor into
-// dst[kTC][ld] (raw dtype).  16-byte cp.async when `async` (every row start
-// 16-byte aligned, ncols * sizeof(T) a multiple of 16), else plain loads.
-template <typename T>
-SSM_DEVINL void stage_tile(T *dst, int ld, const T *src, int64_t ts, int nv, int64_t col0, int ncols,
-                           int64_t col_end, bool async) {
+// Stage rows [0, nv) x cols [col0, col0 + NCOLS) of a token-major tensor into
+// dst[kTC][NCOLS] (raw dtype), columns >= col_end skipped.  16-byte cp.async
+// when `async` (row starts 16-byte aligned and col_end - col0 a multiple of
+// 16 bytes), else plain element copies.  NCOLS is a compile-time width so the
+// thread -> (row, vector) map is shifts and masks.
+template <typename T, int NCOLS>
+SSM_DEVINL void stage_tile(T *dst, const T *src, int64_t ts, int nv, int64_t col0, int64_t col_end, bool async) {
     constexpr int E = 16 / sizeof(T);
+    constexpr int PER_ROW = NCOLS / E;
+    static_assert(NCOLS % E == 0, "tile rows must be whole 16-byte vectors");
     if (async) {
-        const int per_row = ncols / E;
-        for (int i = threadIdx.x; i < nv * per_row; i += kThreads) {
-            const int r = i / per_row, v = i % per_row;
+#pragma unroll
+        for (int i0 = 0; i0 < kTC * PER_ROW; i0 += kThreads) {
+            const int i = i0 + threadIdx.x;
+            const int r = i / PER_ROW, v = i % PER_ROW;
             const int64_t c = col0 + (int64_t)v * E;
-            if (c + E <= col_end) cp_async16(dst + r * ld + v * E, src + r * ts + c);
+            if ((kTC * PER_ROW) % kThreads == 0 || i < kTC * PER_ROW)
+                if (r < nv && c + E <= col_end) cp_async16(dst + r * NCOLS + v * E, src + r * ts + c);
         }
     } else {
-        for (int i = threadIdx.x; i < nv * ncols; i += kThreads) {
-            const int r = i / ncols, v = i % ncols;
+        for (int i = threadIdx.x; i < nv * NCOLS; i += kThreads) {
+            const int r = i / NCOLS, v = i % NCOLS;
             const int64_t c = col0 + v;
-            if (c < col_end) dst[r * ld + v] = src[r * ts + c];
+            if (c < col_end) dst[r * NCOLS + v] = src[r * ts + c];
         }
     }
 }
 
 template <typename T, int SPT>
-__global__ void __launch_bounds__(kThreads)
+struct SmemM1 {
+    static constexpr int NP = kLanes * SPT;             // padded dstate
+    static constexpr int E = 16 / sizeof(T);
+    static constexpr int NPR = (NP + E - 1) / E * E;    // raw B / C row: whole 16-byte vectors
+    T rx[3][kTC][kDB];
+    T rdt[3][kTC][kDB];
+    T rz[3][kTC][kDB];
+    T rB[3][kTC][NPR];
+    T rC[3][kTC][NPR];
+    float halo[2][kHalo][kDB];
+    float2 dd[2][kTC][kDB];   // (delta, delta * xc)
+    float2 ep[2][kTC][kDB];   // (D * xc, gate)
+    float Bf[2][kTC][NP];
+    float Cf[2][kTC][NP];
+    float y[2][kTC][kDB];
+};
+
+template <typename T, int SPT, int KT>
+__global__ void __launch_bounds__(kThreads, 3)
 scan_m1_kernel(const M1Args a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     auto &sm = *reinterpret_cast<SmemM1<T, SPT> *>(smem_raw);
     constexpr int NP = SmemM1<T, SPT>::NP;
+    constexpr int NPR = SmemM1<T, SPT>::NPR;
     constexpr int VW = SPT < 4 ? SPT : 4;     // states per shared-memory vector
     constexpr int NJ = SPT / VW;
+    constexpr int KW = KT - 1;                // conv window of previous raw rows
 
     if (a.sv.err && *a.sv.err != 0) return;
     const int tid = threadIdx.x;
@@ -126,39 +140,113 @@ scan_m1_kernel(const M1Args a) {
     T *yg = static_cast<T *>(a.y) + row * a.y_bs + start * a.y_ts;
     const int K = a.K;
     const int64_t Dn = a.Dn, N = a.N;
-    const int nchunks = (int)((len + kTC - 1) / kTC);
+    const int nchunks = max(1, (int)((len + kTC - 1) / kTC));   // an empty sequence still passes its state through
+    auto chunk_len = [&](int c) { return (int)max((int64_t)0, min((int64_t)kTC, len - (int64_t)c * kTC)); };
 
+    // raw tiles of chunk c -> ring slot c % 3 (one cp.async group per chunk, empty past the end)
     auto stage = [&](int c) {
-        const int buf = c & 1;
+        const int rb = c % 3;
         const int64_t t0 = (int64_t)c * kTC;
-        const int nv = (int)min((int64_t)kTC, len - t0);
+        const int nv = chunk_len(c);
         if (nv > 0) {
-            stage_tile<T>(&sm.rx[buf][0][0], kDB, xg + t0 * a.x_ts, a.x_ts, nv, d0, kDB, Dn, a.async_act);
-            stage_tile<T>(&sm.rdt[buf][0][0], kDB, dtg + t0 * a.dt_ts, a.dt_ts, nv, d0, kDB, Dn, a.async_act);
-            if (zg) stage_tile<T>(&sm.rz[buf][0][0], kDB, zg + t0 * a.z_ts, a.z_ts, nv, d0, kDB, Dn, a.async_act);
-            stage_tile<T>(&sm.rB[buf][0][0], NP, Bg + t0 * a.B_ts, a.B_ts, nv, 0, (int)N, N, a.async_bc);
-            stage_tile<T>(&sm.rC[buf][0][0], NP, Cg + t0 * a.C_ts, a.C_ts, nv, 0, (int)N, N, a.async_bc);
+            stage_tile<T, kDB>(&sm.rx[rb][0][0], xg + t0 * a.x_ts, a.x_ts, nv, d0, Dn, a.async_act);
+            stage_tile<T, kDB>(&sm.rdt[rb][0][0], dtg + t0 * a.dt_ts, a.dt_ts, nv, d0, Dn, a.async_act);
+            if (zg) stage_tile<T, kDB>(&sm.rz[rb][0][0], zg + t0 * a.z_ts, a.z_ts, nv, d0, Dn, a.async_act);
+            stage_tile<T, NPR>(&sm.rB[rb][0][0], Bg + t0 * a.B_ts, a.B_ts, nv, 0, N, a.async_bc);
+            stage_tile<T, NPR>(&sm.rC[rb][0][0], Cg + t0 * a.C_ts, a.C_ts, nv, 0, N, a.async_bc);
         }
         cp_async_commit();
     };
-    stage(0);
-    stage(1);
 
     // ---- prologue role: channel pd = tid % 32, rows [pr0, pr0 + 8)
     const int pd = tid % kDB;
     const int pr0 = (tid / kDB) * kRowsPerThread;
     const int64_t pch = d0 + pd;
     const bool pvalid = pch < Dn;
-    // conv taps right-aligned: wr[kHalo] multiplies the current token, wr[kHalo - m]
-    // the input m tokens back; unused leading taps are 0, so every index is static
-    float wr[kMaxConvWidth], cb = 0.f, dtb = 0.f;
+    // conv taps right-aligned in KT slots: wr[KT-1] multiplies the current
+    // token, wr[KT-1-m] the input m tokens back; unused leading taps are 0, so
+    // every index is static (KT = 4 covers widths up to 4, KT = 8 the rest)
+    float wr[KT], cb = 0.f, dtb = 0.f;
 #pragma unroll
-    for (int j = 0; j < kMaxConvWidth; ++j) {
-        const int k = K - kMaxConvWidth + j;                  // tap index in [0, K)
+    for (int j = 0; j < KT; ++j) {
+        const int k = K - KT + j;                             // tap index in [0, K)
         wr[j] = (pvalid && k >= 0) ? a.conv_w[pch * K + k] : 0.f;
     }
     if (pvalid && a.conv_b) cb = a.conv_b[pch];
     if (pvalid && a.dt_bias) dtb = a.dt_bias[pch];
+    const float Dp = (pvalid && a.D) ? a.D[pch] : 0.f;
+
+    // prologue of chunk c: raw slot c % 3 + halo slot c % 2 -> work slot c % 2,
+    // and the halo of chunk c + 1
+    auto prologue = [&](int c) {
+        const int rb = c % 3, wb = c & 1;
+        const int nv = chunk_len(c);
+        float win[KW];                                              // raw rows t-KW .. t-1
+        auto raw_at = [&](int v) -> float {                         // v: row relative to the chunk
+            return v >= 0 ? Elem<T>::ld(&sm.rx[rb][v][pd]) : sm.halo[wb][kHalo + v][pd];
+        };
+#pragma unroll
+        for (int j = 0; j < KW; ++j)                                // only the last K-1 are live
+            win[j] = (j >= KW - (K - 1) && pvalid) ? raw_at(pr0 - KW + j) : 0.f;
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+            const int t = pr0 + i;
+            float xcv = 0.f, dlt = 0.f, gv = 1.f;
+            if (t < nv && pvalid) {
+                const float cur = Elem<T>::ld(&sm.rx[rb][t][pd]);
+                if (K > 0) {
+                    float acc = fmaf(wr[KW], cur, cb);
+#pragma unroll
+                    for (int j = 0; j < KW; ++j) acc = fmaf(wr[j], win[j], acc);
+                    xcv = silu_fast<T>(acc);
+                } else {
+                    xcv = cur;
+                }
+#pragma unroll
+                for (int j = 0; j + 1 < KW; ++j) win[j] = win[j + 1];
+                if (KW > 0) win[KW - 1] = cur;
+                const float u = Elem<T>::ld(&sm.rdt[rb][t][pd]) + dtb;
+                dlt = a.softplus ? softplus(u) : u;
+                if (zg) gv = silu_fast<T>(Elem<T>::ld(&sm.rz[rb][t][pd]));
+            }
+            sm.dd[wb][t][pd] = make_float2(dlt, dlt * xcv);         // delta = 0 past the end: the state stays put
+            sm.ep[wb][t][pd] = make_float2(Dp * xcv, gv);
+        }
+        // halo of the next chunk: the last K-1 raw inputs up to this chunk's end
+        if (K > 1 && tid < kDB)
+            for (int j = 0; j < K - 1; ++j) {
+                const int v = nv - (K - 1) + j;
+                sm.halo[wb ^ 1][kHalo - (K - 1) + j][pd] = pvalid ? raw_at(v) : 0.f;
+            }
+        // B and C to fp32, zero past the end of the sequence and of dstate
+        for (int i = tid; i < kTC * NP; i += kThreads) {
+            const int t = i / NP, n = i % NP;
+            const bool ok = t < nv && n < N;
+            sm.Bf[wb][t][n] = ok ? Elem<T>::ld(&sm.rB[rb][t][n]) : 0.f;
+            sm.Cf[wb][t][n] = ok ? Elem<T>::ld(&sm.rC[rb][t][n]) : 0.f;
+        }
+    };
+
+    // y of chunk c (ysm slot c % 2) -> global, 16-byte stores when aligned
+    auto store_y = [&](int c) {
+        const int yb = c & 1;
+        const int nv = chunk_len(c);
+        const int64_t t0 = (int64_t)c * kTC;
+        if (a.vec_y && d0 + kDB <= Dn) {
+            for (int i = tid; i < nv * (kDB / 8); i += kThreads) {
+                const int r = i / (kDB / 8), v = i % (kDB / 8);
+                float o[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] = sm.y[yb][r][v * 8 + e];
+                Vec8<T>::st(yg + (t0 + r) * a.y_ts + d0 + v * 8, o);
+            }
+        } else {
+            for (int i = tid; i < nv * kDB; i += kThreads) {
+                const int r = i / kDB, v = i % kDB;
+                if (d0 + v < Dn) Elem<T>::st(yg + (t0 + r) * a.y_ts + d0 + v, sm.y[yb][r][v]);
+            }
+        }
+    };
 
     // ---- scan role: channel sd = tid / 4, lane q = tid % 4
     const int sd = tid / kLanes, q = tid % kLanes;
@@ -185,85 +273,17 @@ scan_m1_kernel(const M1Args a) {
             h2[p] = make_float2(h[2 * p], h[2 * p + 1]);
         }
     }
-    const float Dd = (svalid && a.D) ? a.D[sch] : 0.f;
 
-    // ---- conv halo of chunk 0: the carried state (the K-1 raw inputs before the first token)
-    if (K > 1) {
-        const T *csi = static_cast<const T *>(a.conv_state_in);
-        for (int idx = tid; idx < (K - 1) * kDB; idx += kThreads) {
-            const int j = idx / kDB, d = idx % kDB;
-            const int64_t ch = d0 + d;
-            sm.halo[0][kHalo - (K - 1) + j][d] =
-                (csi && ch < Dn) ? Elem<T>::ld(csi + ((int64_t)s * Dn + ch) * (K - 1) + j) : 0.f;
-        }
-    }
-
-    for (int c = 0; c < nchunks || c == 0; ++c) {
-        const int buf = c & 1;
-        const int64_t t0 = (int64_t)c * kTC;
-        const int nv = (int)max((int64_t)0, min((int64_t)kTC, len - t0));
-        cp_async_wait1();
-        __syncthreads();                                               // chunk c staged, halo[buf] ready
-
-        // ---------------- prologue: once per (token, channel)
-        {
-            float win[kHalo];                                           // raw rows t-7 .. t-1
-            auto raw_at = [&](int v) -> float {                         // v: row relative to the chunk
-                return v >= 0 ? Elem<T>::ld(&sm.rx[buf][v][pd]) : sm.halo[buf][kHalo + v][pd];
-            };
+    // recurrence over chunk c (work slot c % 2), y into ysm slot c % 2
+    auto scan = [&](int c) {
+        const int wb = c & 1;
 #pragma unroll
-            for (int j = 0; j < kHalo; ++j)                             // only the last K-1 are live
-                win[j] = (j >= kHalo - (K - 1) && pvalid) ? raw_at(pr0 - kHalo + j) : 0.f;
-#pragma unroll
-            for (int i = 0; i < kRowsPerThread; ++i) {
-                const int t = pr0 + i;
-                float xcv = 0.f, dlt = 0.f, gv = 1.f;
-                if (t < nv && pvalid) {
-                    const float cur = Elem<T>::ld(&sm.rx[buf][t][pd]);
-                    if (K > 0) {
-                        float acc = fmaf(wr[kHalo], cur, cb);
-#pragma unroll
-                        for (int j = 0; j < kHalo; ++j) acc = fmaf(wr[j], win[j], acc);
-                        xcv = silu_fast<T>(acc);
-                    } else {
-                        xcv = cur;
-                    }
-#pragma unroll
-                    for (int j = 0; j + 1 < kHalo; ++j) win[j] = win[j + 1];
-                    win[kHalo - 1] = cur;
-                    const float u = Elem<T>::ld(&sm.rdt[buf][t][pd]) + dtb;
-                    dlt = a.softplus ? softplus(u) : u;
-                    if (zg) gv = silu_fast<T>(Elem<T>::ld(&sm.rz[buf][t][pd]));
-                }
-                sm.xc[t][pd] = xcv;
-                sm.dd[t][pd] = make_float2(dlt, dlt * xcv);   // delta = 0 past the end: the state stays put
-                sm.g[t][pd] = gv;
-            }
-            // next halo: the last K-1 raw inputs up to this chunk's end
-            if (K > 1 && tid < kDB)
-                for (int j = 0; j < K - 1; ++j) {
-                    const int v = nv - (K - 1) + j;
-                    sm.halo[buf ^ 1][kHalo - (K - 1) + j][pd] = pvalid ? raw_at(v) : 0.f;
-                }
-            // B and C to fp32, zero past the end of the sequence and of dstate
-            for (int i = tid; i < kTC * NP; i += kThreads) {
-                const int t = i / NP, n = i % NP;
-                const bool ok = t < nv && n < N;
-                sm.Bf[t][n] = ok ? Elem<T>::ld(&sm.rB[buf][t][n]) : 0.f;
-                sm.Cf[t][n] = ok ? Elem<T>::ld(&sm.rC[buf][t][n]) : 0.f;
-            }
-        }
-        __syncthreads();                                               // raw[buf] consumed
-        stage(c + 2);                                                  // prefetch two chunks ahead
-
-        // ---------------- recurrence, 4 tokens per step of the loop
-#pragma unroll 2
         for (int t4 = 0; t4 < kTC; t4 += 4) {
             float acc[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int t = t4 + i;
-                const float2 dd = sm.dd[t][sd];                      // (delta, delta * xc)
+                const float2 dd = sm.dd[wb][t][sd];                  // (delta, delta * xc)
                 if constexpr (VW >= 2) {
                     // packed fp32x2: two states per FMUL2 / FFMA2 instruction
                     const float2 dl2 = make_float2(dd.x, dd.x), dx2 = make_float2(dd.y, dd.y);
@@ -271,15 +291,23 @@ scan_m1_kernel(const M1Args a) {
 #pragma unroll
                     for (int j = 0; j < NJ; ++j) {
                         const int n0 = VW * (q + kLanes * j);
+                        float2 bp[VW / 2], cp[VW / 2];
+                        if constexpr (VW == 4) {
+                            const float4 b4 = *reinterpret_cast<const float4 *>(&sm.Bf[wb][t][n0]);
+                            const float4 c4 = *reinterpret_cast<const float4 *>(&sm.Cf[wb][t][n0]);
+                            bp[0] = make_float2(b4.x, b4.y); bp[1] = make_float2(b4.z, b4.w);
+                            cp[0] = make_float2(c4.x, c4.y); cp[1] = make_float2(c4.z, c4.w);
+                        } else {
+                            bp[0] = *reinterpret_cast<const float2 *>(&sm.Bf[wb][t][n0]);
+                            cp[0] = *reinterpret_cast<const float2 *>(&sm.Cf[wb][t][n0]);
+                        }
 #pragma unroll
-                        for (int e = 0; e < VW; e += 2) {
-                            const float2 b2 = *reinterpret_cast<const float2 *>(&sm.Bf[t][n0 + e]);
-                            const float2 c2 = *reinterpret_cast<const float2 *>(&sm.Cf[t][n0 + e]);
-                            const int pi = (j * VW + e) / 2;
+                        for (int e = 0; e < VW / 2; ++e) {
+                            const int pi = j * (VW / 2) + e;
                             const float2 arg = __fmul2_rn(dl2, A2p[pi]);
                             const float2 dA = make_float2(ex2(arg.x), ex2(arg.y));
-                            h2[pi] = __ffma2_rn(dA, h2[pi], __fmul2_rn(dx2, b2));
-                            ac2 = __ffma2_rn(c2, h2[pi], ac2);
+                            h2[pi] = __ffma2_rn(dA, h2[pi], __fmul2_rn(dx2, bp[e]));
+                            ac2 = __ffma2_rn(cp[e], h2[pi], ac2);
                         }
                     }
                     acc[i] = ac2.x + ac2.y;
@@ -289,8 +317,8 @@ scan_m1_kernel(const M1Args a) {
                     for (int j = 0; j < NJ; ++j) {
                         const int n0 = q + kLanes * j;
                         const float dA = ex2(dd.x * A2[j]);
-                        h[j] = fmaf(dA, h[j], dd.y * sm.Bf[t][n0]);
-                        ac = fmaf(sm.Cf[t][n0], h[j], ac);
+                        h[j] = fmaf(dA, h[j], dd.y * sm.Bf[wb][t][n0]);
+                        ac = fmaf(sm.Cf[wb][t][n0], h[j], ac);
                     }
                     acc[i] = ac;
                 }
@@ -304,44 +332,50 @@ scan_m1_kernel(const M1Args a) {
             const bool odd = (q & 1) != 0;
             const float tot = (odd ? r1 : r0) + __shfl_xor_sync(0xffffffffu, odd ? r0 : r1, 1);
             const int t = t4 + q;
-            sm.y[t][sd] = (tot + Dd * sm.xc[t][sd]) * sm.g[t][sd];
+            const float2 e2 = sm.ep[wb][t][sd];                      // (D * xc, gate)
+            sm.y[wb][t][sd] = (tot + e2.x) * e2.y;
         }
-        __syncthreads();                                               // y tile complete
+    };
 
-        if (nv > 0) {
-            // y tile -> global, 16-byte stores when aligned
-            constexpr int E = 16 / sizeof(T);
-            if (a.vec_y && d0 + kDB <= Dn) {
-                for (int i = tid; i < nv * (kDB / 8); i += kThreads) {
-                    const int r = i / (kDB / 8), v = i % (kDB / 8);
-                    float o[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) o[e] = sm.y[r][v * 8 + e];
-                    Vec8<T>::st(yg + (t0 + r) * a.y_ts + d0 + v * 8, o);
-                }
-            } else {
-                for (int i = tid; i < nv * kDB; i += kThreads) {
-                    const int r = i / kDB, v = i % kDB;
-                    if (d0 + v < Dn) Elem<T>::st(yg + (t0 + r) * a.y_ts + d0 + v, sm.y[r][v]);
-                }
-            }
-            (void)E;
-        }
-        if (c + 1 >= nchunks) {
-            // carried conv state: the halo written by this (last) chunk's prologue
-            if (K > 1 && a.conv_state_out) {
-                T *cso = static_cast<T *>(a.conv_state_out);
-                for (int idx = tid; idx < (K - 1) * kDB; idx += kThreads) {
-                    const int j = idx / kDB, d = idx % kDB;
-                    const int64_t ch = d0 + d;
-                    if (ch < Dn)
-                        Elem<T>::st(cso + ((int64_t)s * Dn + ch) * (K - 1) + j, sm.halo[buf ^ 1][kHalo - (K - 1) + j][d]);
-                }
-            }
-            break;
+    // ---- conv halo of chunk 0: the carried state (the K-1 raw inputs before the first token)
+    if (K > 1) {
+        const T *csi = static_cast<const T *>(a.conv_state_in);
+        for (int idx = tid; idx < (K - 1) * kDB; idx += kThreads) {
+            const int j = idx / kDB, d = idx % kDB;
+            const int64_t ch = d0 + d;
+            sm.halo[0][kHalo - (K - 1) + j][d] =
+                (csi && ch < Dn) ? Elem<T>::ld(csi + ((int64_t)s * Dn + ch) * (K - 1) + j) : 0.f;
         }
     }
-    asm volatile("cp.async.wait_all;\n" ::);
+    stage(0);
+    stage(1);
+    stage(2);
+    cp_async_wait<2>();                                   // chunk 0 landed (own copies)
+    __syncthreads();                                      // ... everyone's copies, halo 0
+    prologue(0);
+    cp_async_wait<1>();                                   // chunk 1 landed
+    __syncthreads();
+
+    for (int c = 0; c < nchunks; ++c) {
+        scan(c);                                          // work slot c % 2 -> ysm slot c % 2
+        if (c > 0) store_y(c - 1);                        // ysm slot (c-1) % 2
+        if (c + 1 < nchunks) prologue(c + 1);             // raw slot (c+1) % 3 -> work slot (c+1) % 2
+        stage(c + 3);                                     // raw slot c % 3, read by prologue(c) last iteration
+        cp_async_wait<1>();                               // chunk c + 2 landed
+        __syncthreads();
+    }
+    store_y(nchunks - 1);
+    // carried conv state: the halo written by the last chunk's prologue
+    if (K > 1 && a.conv_state_out) {
+        T *cso = static_cast<T *>(a.conv_state_out);
+        const int hb = nchunks & 1;
+        for (int idx = tid; idx < (K - 1) * kDB; idx += kThreads) {
+            const int j = idx / kDB, d = idx % kDB;
+            const int64_t ch = d0 + d;
+            if (ch < Dn) Elem<T>::st(cso + ((int64_t)s * Dn + ch) * (K - 1) + j, sm.halo[hb][kHalo - (K - 1) + j][d]);
+        }
+    }
+    cp_async_wait<0>();
     if constexpr (SPT >= 2) {
 #pragma unroll
         for (int p = 0; p < NPAIR; ++p) {
@@ -363,7 +397,7 @@ scan_m1_kernel(const M1Args a) {
 template <typename T, int SPT>
 cudaError_t launch_spt(const M1Args &a, int nseqs, cudaStream_t st) {
     const size_t smem = sizeof(SmemM1<T, SPT>);
-    auto kern = scan_m1_kernel<T, SPT>;
+    auto kern = a.K <= 4 ? scan_m1_kernel<T, SPT, 4> : scan_m1_kernel<T, SPT, kMaxConvWidth>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((a.Dn + kDB - 1) / kDB), (unsigned)nseqs);
