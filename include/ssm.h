@@ -98,6 +98,7 @@ typedef enum { SSM_MAMBA1 = 1, SSM_MAMBA2 = 2 } ssm_mode;
 /* Device-side error codes written into the workspace error word. */
 #define SSM_DEVERR_NONE 0
 #define SSM_DEVERR_CU_SEQLENS 1   /* cu_seqlens not 0-based, decreasing, or not ending at seqlen */
+#define SSM_DEVERR_TIMEOUT 2      /* a bounded wait for tensor-core completion ran out; outputs incomplete */
 
 /* ------------------------------------------------------------------ conv */
 typedef struct ssm_conv_args {

@@ -23,8 +23,9 @@ constexpr int kTokensPerThread = 32;
 template <typename T, int VEC, int K>
 __global__ void __launch_bounds__(kThreads)
 conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *__restrict__ w,
-              const float *__restrict__ bias, const T *__restrict__ state_in, T *__restrict__ out, int64_t o_bs,
-              int64_t o_ts, const int32_t *__restrict__ cu, int nseqs, int64_t seqlen, int64_t channels, int act) {
+              const float *__restrict__ bias, const T *__restrict__ state_in, int64_t ss, T *__restrict__ out,
+              int64_t o_bs, int64_t o_ts, const int32_t *__restrict__ cu, int nseqs, int64_t seqlen,
+              int64_t channels, int act) {
     const int64_t cv = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     const int64_t c0 = cv * VEC;
     if (c0 >= channels) return;
@@ -65,7 +66,7 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
                 const int64_t q = tau - start + (K - 1);   // index into the carried state
 #pragma unroll
                 for (int v = 0; v < VEC; ++v)
-                    hist[j][v] = (state_in && q >= 0) ? Elem<T>::ld(state_in + ((int64_t)s * channels + c0 + v) * (K - 1) + q) : 0.f;
+                    hist[j][v] = (state_in && q >= 0) ? Elem<T>::ld(state_in + (int64_t)s * ss + (c0 + v) * (K - 1) + q) : 0.f;
             }
         }
     };
@@ -115,8 +116,8 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
 // happen before the writes, so state_out may alias state_in.
 template <typename T>
 __global__ void conv_state_out_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const T *state_in,
-                                      T *state_out, const int32_t *__restrict__ cu, int nseq, int64_t seqlen,
-                                      int64_t channels, int K) {
+                                      T *state_out, int64_t ss, const int32_t *__restrict__ cu, int nseq,
+                                      int64_t seqlen, int64_t channels, int K) {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (int64_t)nseq * channels) return;
     const int s = (int)(i / channels);
@@ -131,28 +132,27 @@ __global__ void conv_state_out_kernel(const T *__restrict__ x, int64_t x_bs, int
             v[p] = Elem<T>::ld(xr + tau * x_ts + c);
         } else {
             const int64_t q = tau - start + (K - 1);
-            v[p] = (state_in && q >= 0) ? Elem<T>::ld(state_in + ((int64_t)s * channels + c) * (K - 1) + q) : 0.f;
+            v[p] = (state_in && q >= 0) ? Elem<T>::ld(state_in + (int64_t)s * ss + c * (K - 1) + q) : 0.f;
         }
     }
-    for (int p = 0; p < K - 1; ++p) Elem<T>::st(state_out + ((int64_t)s * channels + c) * (K - 1) + p, v[p]);
+    for (int p = 0; p < K - 1; ++p) Elem<T>::st(state_out + (int64_t)s * ss + c * (K - 1) + p, v[p]);
 }
 
 template <typename T, int VEC>
-cudaError_t launch_typed_vec(const ssm_conv_args &a, cudaStream_t st) {
+cudaError_t launch_typed_vec(const ConvJob &a, cudaStream_t st) {
     const int64_t nvec = (a.channels + VEC - 1) / VEC;
     dim3 grid((unsigned)((nvec + kThreads - 1) / kThreads), (unsigned)((a.seqlen + kTokensPerThread - 1) / kTokensPerThread),
               (unsigned)a.batch);
     const T *x = static_cast<const T *>(a.x);
     const T *si = static_cast<const T *>(a.state_in);
     T *o = static_cast<T *>(a.out);
-    const int ns = a.cu_seqlens ? a.nseqs : (int)a.batch;
+    const int ns = a.cu ? a.nseqs : (int)a.batch;
     if (grid.y > 0) {
 #define SSM_CONV_CASE(KK)                                                                                    \
     case KK:                                                                                                \
-        conv1d_kernel<T, VEC, KK><<<grid, kThreads, 0, st>>>(x, a.x_batch_stride, a.x_token_stride, a.weight,  \
-                                                             a.bias, si, o, a.out_batch_stride,            \
-                                                             a.out_token_stride, a.cu_seqlens, ns, a.seqlen, \
-                                                             a.channels, a.activation);                    \
+        conv1d_kernel<T, VEC, KK><<<grid, kThreads, 0, st>>>(x, a.x_bs, a.x_ts, a.w, a.b, si, a.state_stride, o, \
+                                                             a.o_bs, a.o_ts, a.cu, ns, a.seqlen, a.channels,   \
+                                                             a.act);                                           \
         break;
         switch (a.width) {
             SSM_CONV_CASE(1) SSM_CONV_CASE(2) SSM_CONV_CASE(3) SSM_CONV_CASE(4)
@@ -166,26 +166,37 @@ cudaError_t launch_typed_vec(const ssm_conv_args &a, cudaStream_t st) {
     if (a.state_out && a.width > 1 && ns > 0) {
         const int64_t n = (int64_t)ns * a.channels;
         conv_state_out_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-            x, a.x_batch_stride, a.x_token_stride, si, static_cast<T *>(a.state_out), a.cu_seqlens, ns, a.seqlen,
-            a.channels, (int)a.width);
+            x, a.x_bs, a.x_ts, si, static_cast<T *>(a.state_out), a.state_stride, a.cu, ns, a.seqlen, a.channels,
+            (int)a.width);
         return cudaGetLastError();
     }
     return cudaSuccess;
 }
 
 template <typename T>
-cudaError_t launch_typed(const ssm_conv_args &a, cudaStream_t st) {
+cudaError_t launch_typed(const ConvJob &a, cudaStream_t st) {
     const size_t es = sizeof(T);
     const bool vec_ok = a.channels % 8 == 0 && ((uintptr_t)a.x % 16 == 0) && ((uintptr_t)a.out % 16 == 0) &&
-                        (a.x_token_stride * es) % 16 == 0 && (a.x_batch_stride * es) % 16 == 0 &&
-                        (a.out_token_stride * es) % 16 == 0 && (a.out_batch_stride * es) % 16 == 0;
+                        (a.x_ts * es) % 16 == 0 && (a.x_bs * es) % 16 == 0 &&
+                        (a.o_ts * es) % 16 == 0 && (a.o_bs * es) % 16 == 0;
     return vec_ok ? launch_typed_vec<T, 8>(a, st) : launch_typed_vec<T, 1>(a, st);
 }
 
 }  // namespace
 
+cudaError_t launch_conv_job(const ConvJob &j, cudaStream_t st) {
+    return j.dtype == SSM_BF16 ? launch_typed<__nv_bfloat16>(j, st) : launch_typed<float>(j, st);
+}
+
 cudaError_t launch_conv1d(const ssm_conv_args &a, cudaStream_t st) {
-    return a.dtype == SSM_BF16 ? launch_typed<__nv_bfloat16>(a, st) : launch_typed<float>(a, st);
+    ConvJob j;
+    j.x = a.x; j.x_bs = a.x_batch_stride; j.x_ts = a.x_token_stride;
+    j.w = a.weight; j.b = a.bias;
+    j.state_in = a.state_in; j.state_out = a.state_out; j.state_stride = a.channels * (a.width - 1);
+    j.cu = a.cu_seqlens; j.nseqs = a.nseqs; j.batch = a.batch; j.seqlen = a.seqlen;
+    j.channels = a.channels; j.width = a.width; j.act = a.activation; j.dtype = a.dtype;
+    j.out = a.out; j.o_bs = a.out_batch_stride; j.o_ts = a.out_token_stride;
+    return launch_conv_job(j, st);
 }
 
 }  // namespace ssm

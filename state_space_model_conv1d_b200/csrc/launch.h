@@ -11,12 +11,11 @@ namespace ssm {
 
 // Workspace layout of ssm_scan_fwd (all offsets 256-byte aligned):
 //   [0, 256)            int32 device error word (SSM_DEVERR_*), then padding
-//   [256, 256 + 4*n)    int32 sequence schedule (longest sequence first)
+//   [256, 256 + R)      varlen only: int32 sequence schedule (longest first), R = 4*nseqs rounded to 256
+//   [256 + R, ...)      tensor-core Mamba-2 path only: conv'd bf16 B and C tiles
 constexpr size_t kWsErrorOffset = 0;
 constexpr size_t kWsOrderOffset = 256;
-inline size_t varlen_workspace_bytes(int64_t nseqs) {
-    return kWsOrderOffset + ((size_t)(nseqs > 0 ? nseqs : 1) * 4 + 255) / 256 * 256;
-}
+inline size_t order_bytes(int64_t nseqs) { return ((size_t)(nseqs > 0 ? nseqs : 1) * 4 + 255) / 256 * 256; }
 
 // Packed-sequence view shared by the scan launchers: sequence s spans tokens
 // [cu[s], cu[s+1]) of batch row 0 when cu != nullptr, else row s spans
@@ -28,11 +27,35 @@ struct SeqView {
     int nseqs;
 };
 
+// A causal depthwise conv over `channels` contiguous channels of a token-major
+// tensor.  Carried states are [seq][...] with `state_stride` elements between
+// sequences and K-1 values per channel (so a slice of a wider state works).
+struct ConvJob {
+    const void *x;
+    int64_t x_bs, x_ts;
+    const float *w, *b;                 // [channels][K], [channels] (already offset to the slice)
+    const void *state_in;               // may be null
+    void *state_out;                    // may be null
+    int64_t state_stride;
+    const int32_t *cu;
+    int nseqs;
+    int64_t batch, seqlen, channels, width;
+    int act, dtype;
+    void *out;
+    int64_t o_bs, o_ts;
+};
+
 cudaError_t launch_conv1d(const ssm_conv_args &a, cudaStream_t st);
+cudaError_t launch_conv_job(const ConvJob &j, cudaStream_t st);
 cudaError_t launch_varlen_plan(const int32_t *cu, int nseqs, int64_t total, int32_t *err, int32_t *order,
                                cudaStream_t st);
 cudaError_t launch_scan_m1(const ssm_scan_args &a, const SeqView &sv, cudaStream_t st);
 cudaError_t launch_scan_m2_simt(const ssm_scan_args &a, const SeqView &sv, cudaStream_t st);
+// Tensor-core (tcgen05) chunked Mamba-2 path: which shapes it takes, the
+// workspace it needs for the conv'd B / C, and its launcher.
+bool ssd_supported(const ssm_scan_args &a);
+size_t ssd_workspace_bytes(const ssm_scan_args &a);
+cudaError_t launch_ssd(const ssm_scan_args &a, const SeqView &sv, void *ws_bc, cudaStream_t st);
 cudaError_t launch_state_update(const ssm_update_args &a, cudaStream_t st);
 
 // Largest dstate each path supports.

@@ -1,0 +1,488 @@
+// ssd_m2.cu -- Mamba-2 scan as the chunked state-space-dual (SSD) form on the
+// sm_100a tensor cores (tcgen05 MMA, fp32 accumulators in tensor memory).
+//
+// The recurrence (scalar A per head, B / C shared by a contiguous group of
+// heads; "Tensor-parallel SSM", Fast-LLM PR 333, repeat_interleave thread):
+//   S_t = exp(delta_t A) S_{t-1} + delta_t x_t B_t^T,   y_t = S_t C_t + D x_t
+// is evaluated exactly (up to rounding) chunk by chunk.  For a chunk of Q
+// tokens with cs_i = sum_{j<=i} delta_j A (the running log-decay):
+//   G   = C B^T                                             (Q x Q)
+//   M   = G o L,  L[i, j] = exp(cs_i - cs_j) delta_j for j <= i, else 0
+//   Y   = M X + diag(exp(cs)) C S_prev^T                    (Q x P)
+//   S   = exp(cs_Q) S_prev + B'^T X,  B'[j] = exp(cs_Q - cs_j) delta_j B[j]
+// with S_prev = h0 for the first chunk ("Adding Initial Value Support to
+// Selective Scan Forward Kernel", state-spaces/mamba issue 285: the carried
+// state seeds the scan).  The kernel names in "Clean up SSM ops directory
+// structure" (Megatron-LM PR 6444: ssd_bmm, ssd_chunk_state,
+// ssd_state_passing, ssd_chunk_scan) are these four steps; here they are one
+// kernel whose carried state never leaves the SM.
+//
+// Layout of the work: one CTA per (sequence, head), 4 warps, walking the
+// sequence in chunks of Q = 64.  The B / C causal conv + SiLU is shared by the
+// heads of a group, so it runs once per group in a pre-pass that writes bf16
+// B, C into the workspace; the x conv + SiLU runs here, fused.  Per chunk:
+//   MMA1  G  = C B^T         M=64  N=64 K=128   A K-major, B K-major
+//   MMA2  Y  = M X           M=64  N=64 K=64    A K-major, B MN-major
+//   MMA3  Y += C' S_prev^T   M=64  N=64 K=128   A K-major, B MN-major
+//   MMA4  Sc = B'^T X        M=128 N=64 K=64    A MN-major (same tile as B), B MN-major
+// C' and B' are C and B rescaled in place after MMA1 has consumed them.
+// The fp32 state S (128 x 64 per head) stays in registers, one state row n
+// per thread; its bf16 copy is the MMA3 operand of the next chunk.
+//
+// Tensor memory: 128 columns (G in columns 0-63, later reused for Sc; Y in
+// 64-127), shared memory 67 KB, so three CTAs fit on one SM.
+#include "common.cuh"
+#include "launch.h"
+#include "tc05.cuh"
+
+namespace ssm {
+namespace {
+
+constexpr int kQ = 64;           // chunk length
+constexpr int kP = 64;           // headdim on this path
+constexpr int kN = 128;          // dstate on this path
+constexpr int kThreads = 128;
+constexpr int kHx = 3;           // raw x rows kept before each chunk (conv width <= 4)
+constexpr uint32_t kTmemCols = 128;
+
+// operand tiles (bf16, core-matrix layouts), byte offsets in dynamic shared memory
+constexpr uint32_t OFF_C = 0;        // C [i][n]  K-major   LBO 128  SBO 2048
+constexpr uint32_t OFF_B = 16384;    // B [j][n]  K-major   LBO 128  SBO 2048  (MN-major view: LBO 2048 SBO 128)
+constexpr uint32_t OFF_M = 32768;    // M [i][j]  K-major   LBO 128  SBO 1024
+constexpr uint32_t OFF_X = 40960;    // X (p, j)  MN-major  LBO 1024 SBO 128
+constexpr uint32_t OFF_S = 49152;    // S (p, n)  MN-major  LBO 1024 SBO 128
+constexpr uint32_t OFF_AUX = 65536;
+
+struct Aux {
+    float xh[2][kHx][kP];            // raw x rows before the chunk (double buffered)
+    float dlt[kQ];                   // delta
+    float cs2[kQ];                   // running log2-decay
+    float ecs[kQ];                   // exp(cs_i)
+    float wj[kQ];                    // exp(cs_Q - cs_j) * delta_j
+    float dAc;                       // exp(cs_Q)
+    float cw[4][kP];                 // x conv taps, right-aligned (cw[3] multiplies the current token)
+    float cb[kP];                    // x conv bias
+    uint32_t tmem;
+    uint64_t mbar[2];
+};
+constexpr size_t kSmemBytes = OFF_AUX + sizeof(Aux);
+
+constexpr uint32_t ID_G = tc::idesc_bf16(64, 64, 0, 0);
+constexpr uint32_t ID_Y = tc::idesc_bf16(64, 64, 0, 1);
+constexpr uint32_t ID_S = tc::idesc_bf16(128, 64, 1, 1);
+
+struct SsdArgs {
+    const __nv_bfloat16 *x, *z, *dt, *Bc, *Cc;
+    __nv_bfloat16 *y;
+    int64_t x_bs, x_ts, z_bs, z_ts, dt_bs, dt_ts, b_bs, b_ts, c_bs, c_ts, y_bs, y_ts;
+    const float *A, *D, *dt_bias, *h0, *conv_w, *conv_b;
+    float *h_final;
+    const __nv_bfloat16 *conv_state_in;
+    __nv_bfloat16 *conv_state_out;
+    int64_t H, G, seqlen, cdim;
+    int K, softplus;
+    SeqView sv;
+    int32_t *err;
+};
+
+SSM_DEVINL uint4 ld16(const void *p) { return *reinterpret_cast<const uint4 *>(p); }
+SSM_DEVINL void st16(void *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
+
+__global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    Aux &ax = *reinterpret_cast<Aux *>(smem + OFF_AUX);
+    if (a.sv.err && *a.sv.err != 0) return;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int hh = blockIdx.x;
+    const int s = a.sv.order ? a.sv.order[blockIdx.y] : (int)blockIdx.y;
+    int64_t start = 0, len = a.seqlen, row = s;
+    if (a.sv.cu) {
+        const int64_t c0 = min(max((int64_t)a.sv.cu[s], (int64_t)0), a.seqlen);
+        const int64_t c1 = min(max((int64_t)a.sv.cu[s + 1], c0), a.seqlen);
+        start = c0; len = c1 - c0; row = 0;
+    }
+    const int64_t H = a.H, g = hh / (H / a.G);
+    const int K = a.K;
+    const __nv_bfloat16 *xg = a.x + row * a.x_bs + start * a.x_ts + hh * kP;
+    const __nv_bfloat16 *zg = a.z ? a.z + row * a.z_bs + start * a.z_ts + hh * kP : nullptr;
+    const __nv_bfloat16 *dtg = a.dt + row * a.dt_bs + start * a.dt_ts + hh;
+    const __nv_bfloat16 *Bg = a.Bc + row * a.b_bs + start * a.b_ts + g * kN;
+    const __nv_bfloat16 *Cg = a.Cc + row * a.c_bs + start * a.c_ts + g * kN;
+    __nv_bfloat16 *yg = a.y + row * a.y_bs + start * a.y_ts + hh * kP;
+    const uint32_t sbase = tc::smem_u32(smem);
+
+    if (warp == 0) tc::tmem_alloc(&ax.tmem, kTmemCols);
+    if (tid == 0) {
+        tc::mbar_init(&ax.mbar[0], 1);
+        tc::mbar_init(&ax.mbar[1], 1);
+        tc::mbar_init_fence();
+    }
+
+    // ---- per-thread constants
+    const float A2 = a.A[hh] * kLog2e;
+    const float Dh = a.D ? a.D[hh] : 0.f;
+    const float dtb = a.dt_bias ? a.dt_bias[hh] : 0.f;
+    // x conv role: channels po*8 .. po*8+7, tokens r0 .. r0+3
+    const int po = tid & 7, r0 = (tid >> 3) * 4;
+    if (tid < kP) {
+        const int64_t ch = hh * kP + tid;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int k = K - 4 + j;
+            ax.cw[j][tid] = (K > 0 && k >= 0) ? a.conv_w[ch * K + k] : 0.f;
+        }
+        ax.cb[tid] = a.conv_b ? a.conv_b[ch] : 0.f;
+    }
+
+    // ---- carried state: thread n owns S[n][p], p = 0..63 (fp32), plus its bf16 copy
+    float S[kP];
+    {
+        const int n = tid;
+        const float *h0p = a.h0 ? a.h0 + ((int64_t)s * H + hh) * kP * kN : nullptr;
+#pragma unroll
+        for (int p = 0; p < kP; ++p) S[p] = h0p ? h0p[(int64_t)p * kN + n] : 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            st16(smem + OFF_S + tc::off_mnmajor(q * 8, n, 1024, 128), tc::pack_bf16x8(&S[q * 8]));
+    }
+    // ---- conv halo of chunk 0 (the last K-1 raw inputs before the sequence)
+    if (tid < kP) {
+        const int p = tid;
+#pragma unroll
+        for (int j = 0; j < kHx; ++j) {
+            const int q = j - (kHx - (K - 1));          // index into the carried conv state
+            float v = 0.f;
+            if (K > 1 && q >= 0 && a.conv_state_in)
+                v = __bfloat162float(a.conv_state_in[((int64_t)s * a.cdim + hh * kP + p) * (K - 1) + q]);
+            ax.xh[0][j][p] = v;
+        }
+    }
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = ax.tmem;
+    const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
+    bool ok = true;
+    int fail_bar = 0;
+    uint32_t fail_par = 0;
+
+    const int nchunks = (int)((len + kQ - 1) / kQ);
+    for (int c = 0; c < nchunks; ++c) {
+        const int64_t t0 = (int64_t)c * kQ;
+        const int nv = (int)min((int64_t)kQ, len - t0);
+        const int hb = c & 1;
+
+        // ---- (1) delta, running decay (warp 0); B, C tiles; x conv
+        if (warp == 0) {
+            float d0 = 0.f, d1 = 0.f;
+            if (lane < nv) {
+                const float u = __bfloat162float(dtg[(t0 + lane) * a.dt_ts]) + dtb;
+                d0 = a.softplus ? softplus(u) : u;
+            }
+            if (lane + 32 < nv) {
+                const float u = __bfloat162float(dtg[(t0 + lane + 32) * a.dt_ts]) + dtb;
+                d1 = a.softplus ? softplus(u) : u;
+            }
+            float s0 = d0 * A2, s1 = d1 * A2;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v0 = __shfl_up_sync(0xffffffffu, s0, o);
+                const float v1 = __shfl_up_sync(0xffffffffu, s1, o);
+                if (lane >= o) { s0 += v0; s1 += v1; }
+            }
+            s1 += __shfl_sync(0xffffffffu, s0, 31);
+            const float last = __shfl_sync(0xffffffffu, s1, 31);
+            ax.dlt[lane] = d0;
+            ax.dlt[lane + 32] = d1;
+            ax.cs2[lane] = s0;
+            ax.cs2[lane + 32] = s1;
+            ax.ecs[lane] = ex2(s0);
+            ax.ecs[lane + 32] = ex2(s1);
+            ax.wj[lane] = ex2(last - s0) * d0;
+            ax.wj[lane + 32] = ex2(last - s1) * d1;
+            if (lane == 0) ax.dAc = ex2(last);
+        }
+        for (int i = tid; i < kQ * (kN / 8); i += kThreads) {
+            const int r = i / (kN / 8), q = i % (kN / 8);
+            uint4 vb = make_uint4(0, 0, 0, 0), vc = make_uint4(0, 0, 0, 0);
+            if (r < nv) {
+                vb = ld16(Bg + (t0 + r) * a.b_ts + q * 8);
+                vc = ld16(Cg + (t0 + r) * a.c_ts + q * 8);
+            }
+            const uint32_t off = tc::off_kmajor(r, q * 8, 128, 2048);
+            st16(smem + OFF_B + off, vb);
+            st16(smem + OFF_C + off, vc);
+        }
+        {
+            // conv + SiLU of 8 channels x 4 tokens; window = raw rows r0-3 .. r0-1
+            float win[kHx][8];
+#pragma unroll
+            for (int j = 0; j < kHx; ++j) {
+                const int v = r0 - kHx + j;
+                if (v < 0) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) win[j][e] = ax.xh[hb][kHx + v][po * 8 + e];
+                } else if (v < nv) {
+                    tc::unpack_bf16x8(ld16(xg + (t0 + v) * a.x_ts + po * 8), win[j]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) win[j][e] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = r0 + i;
+                float cur[8], o[8];
+                if (r < nv) tc::unpack_bf16x8(ld16(xg + (t0 + r) * a.x_ts + po * 8), cur);
+                else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) cur[e] = 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    float acc;
+                    if (K > 0) {
+                        const int p = po * 8 + e;
+                        acc = fmaf(ax.cw[3][p], cur[e], ax.cb[p]);
+                        acc = fmaf(ax.cw[2][p], win[2][e], acc);
+                        acc = fmaf(ax.cw[1][p], win[1][e], acc);
+                        acc = fmaf(ax.cw[0][p], win[0][e], acc);
+                        acc = silu_fast<__nv_bfloat16>(acc);
+                    } else {
+                        acc = cur[e];
+                    }
+                    o[e] = r < nv ? acc : 0.f;
+                    win[0][e] = win[1][e];
+                    win[1][e] = win[2][e];
+                    win[2][e] = cur[e];
+                }
+                st16(smem + OFF_X + tc::off_mnmajor(po * 8, r, 1024, 128), tc::pack_bf16x8(o));
+            }
+        }
+        // halo of the next chunk: raw rows nv-3 .. nv-1 (from the old halo when the chunk is shorter)
+        if (tid < kP) {
+            const int p = tid;
+#pragma unroll
+            for (int j = 0; j < kHx; ++j) {
+                const int v = nv - kHx + j;
+                ax.xh[hb ^ 1][j][p] = v >= 0 ? __bfloat162float(xg[(t0 + v) * a.x_ts + p]) : ax.xh[hb][kHx + v][p];
+            }
+        }
+        tc::fence_proxy_async();
+        __syncthreads();
+
+        // ---- (2) MMA1: G = C B^T into columns 0..63
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int k = 0; k < kN / 16; ++k)
+                tc::mma_bf16(tmem, tc::desc(sbase + OFF_C + k * 256, 128, 2048), tc::desc(sbase + OFF_B + k * 256, 128, 2048),
+                             ID_G, k > 0);
+            tc::mma_commit(&ax.mbar[0]);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(&ax.mbar[0], c & 1));
+        if (!ok) { fail_bar = 0; fail_par = c & 1; break; }
+        tc::fence_after_sync();
+
+        // ---- (3) mask G -> M; rescale C -> C', B -> B'
+        {
+            float Gv[64];
+            tc::tmem_ld64(tmem + t_lane, Gv);
+            if (lane < 16) {
+                const int i = warp * 16 + lane;
+                const float ci = ax.cs2[i];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    float m[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = q * 8 + e;
+                        m[e] = j <= i ? Gv[j] * ex2(ci - ax.cs2[j]) * ax.dlt[j] : 0.f;
+                    }
+                    st16(smem + OFF_M + tc::off_kmajor(i, q * 8, 128, 1024), tc::pack_bf16x8(m));
+                }
+            }
+        }
+        for (int i = tid; i < kQ * (kN / 8); i += kThreads) {
+            const int r = i / (kN / 8), q = i % (kN / 8);
+            const uint32_t off = tc::off_kmajor(r, q * 8, 128, 2048);
+            float v[8];
+            tc::unpack_bf16x8(ld16(smem + OFF_C + off), v);
+            const float fc = ax.ecs[r];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] *= fc;
+            st16(smem + OFF_C + off, tc::pack_bf16x8(v));
+            tc::unpack_bf16x8(ld16(smem + OFF_B + off), v);
+            const float fb = ax.wj[r];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] *= fb;
+            st16(smem + OFF_B + off, tc::pack_bf16x8(v));
+        }
+        tc::fence_before_sync();
+        tc::fence_proxy_async();
+        __syncthreads();
+
+        // ---- (4) MMA2 + MMA3 into Y (columns 64..127), MMA4 into Sc (columns 0..63)
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int k = 0; k < kQ / 16; ++k)
+                tc::mma_bf16(tmem + 64, tc::desc(sbase + OFF_M + k * 256, 128, 1024),
+                             tc::desc(sbase + OFF_X + k * 2048, 1024, 128), ID_Y, k > 0);
+#pragma unroll
+            for (int k = 0; k < kN / 16; ++k)
+                tc::mma_bf16(tmem + 64, tc::desc(sbase + OFF_C + k * 256, 128, 2048),
+                             tc::desc(sbase + OFF_S + k * 2048, 1024, 128), ID_Y, 1);
+#pragma unroll
+            for (int k = 0; k < kQ / 16; ++k)
+                tc::mma_bf16(tmem, tc::desc(sbase + OFF_B + k * 4096, 2048, 128),
+                             tc::desc(sbase + OFF_X + k * 2048, 1024, 128), ID_S, k > 0);
+            tc::mma_commit(&ax.mbar[1]);
+        }
+        ok = __syncthreads_and(tc::mbar_wait(&ax.mbar[1], c & 1));
+        if (!ok) { fail_bar = 1; fail_par = c & 1; break; }
+        tc::fence_after_sync();
+
+        // ---- (5) y = (Y + D x) * silu(z); S = exp(cs_Q) S + Sc
+        {
+            float Yv[64];
+            tc::tmem_ld64(tmem + t_lane + 64, Yv);
+            if (lane < 16) {
+                const int i = warp * 16 + lane;
+                if (i < nv) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float xv[8], zv[8], o[8];
+                        tc::unpack_bf16x8(ld16(smem + OFF_X + tc::off_mnmajor(q * 8, i, 1024, 128)), xv);
+                        if (zg) tc::unpack_bf16x8(ld16(zg + (t0 + i) * a.z_ts + q * 8), zv);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            float yv = fmaf(Dh, xv[e], Yv[q * 8 + e]);
+                            o[e] = zg ? yv * silu_fast<__nv_bfloat16>(zv[e]) : yv;
+                        }
+                        st16(yg + (t0 + i) * a.y_ts + q * 8, tc::pack_bf16x8(o));
+                    }
+                }
+            }
+        }
+        {
+            float Sc[64];
+            tc::tmem_ld64(tmem + t_lane, Sc);
+            const float dAc = ax.dAc;
+            const int n = tid;
+#pragma unroll
+            for (int p = 0; p < kP; ++p) S[p] = fmaf(dAc, S[p], Sc[p]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                st16(smem + OFF_S + tc::off_mnmajor(q * 8, n, 1024, 128), tc::pack_bf16x8(&S[q * 8]));
+        }
+        tc::fence_before_sync();
+        tc::fence_proxy_async();
+        __syncthreads();
+    }
+
+    if (!ok) {
+        // a tensor-core completion never arrived: record it, give the MMAs a
+        // bounded grace period, release tensor memory and leave
+        if (tid == 0 && a.err) atomicExch(a.err, SSM_DEVERR_TIMEOUT);
+        tc::mbar_wait(&ax.mbar[fail_bar], fail_par, 1u << 20);
+    } else {
+        if (a.h_final) {
+            const int n = tid;
+            float *hf = a.h_final + ((int64_t)s * H + hh) * kP * kN;
+#pragma unroll
+            for (int p = 0; p < kP; ++p) hf[(int64_t)p * kN + n] = S[p];
+        }
+        if (K > 1 && a.conv_state_out && tid < kP) {
+            const int p = tid, hbf = nchunks & 1;
+            for (int j = 0; j < K - 1; ++j)
+                a.conv_state_out[((int64_t)s * a.cdim + hh * kP + p) * (K - 1) + j] =
+                    __float2bfloat16_rn(ax.xh[hbf][kHx - (K - 1) + j][p]);
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+bool ssd_supported(const ssm_scan_args &s) {
+    auto al16 = [](const void *p) { return p == nullptr || ((uintptr_t)p & 15) == 0; };
+    auto st16ok = [](int64_t v) { return (v * 2) % 16 == 0; };
+    return s.mode == SSM_MAMBA2 && s.dtype == SSM_BF16 && s.headdim == kP && s.dstate == kN && s.d_conv <= 4 &&
+           al16(s.x) && al16(s.z) && al16(s.y) && al16(s.B) && al16(s.C) && st16ok(s.x_token_stride) &&
+           st16ok(s.x_batch_stride) && st16ok(s.y_token_stride) && st16ok(s.y_batch_stride) &&
+           (s.z == nullptr || (st16ok(s.z_token_stride) && st16ok(s.z_batch_stride))) &&
+           st16ok(s.B_token_stride) && st16ok(s.B_batch_stride) && st16ok(s.C_token_stride) &&
+           st16ok(s.C_batch_stride);
+}
+
+size_t ssd_workspace_bytes(const ssm_scan_args &s) {
+    if (s.d_conv == 0) return 0;
+    const size_t one = (size_t)s.batch * (size_t)s.seqlen * (size_t)(s.ngroups * s.dstate) * 2;
+    return 2 * ((one + 255) / 256 * 256);
+}
+
+cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cudaStream_t st) {
+    const int nseqs = s.cu_seqlens ? s.nseqs : (int)s.batch;
+    if (nseqs == 0) return cudaSuccess;
+    const int64_t GN = s.ngroups * s.dstate;
+    const int64_t cdim = s.d_inner + 2 * GN;
+    const __nv_bfloat16 *Bc = static_cast<const __nv_bfloat16 *>(s.B), *Cc = static_cast<const __nv_bfloat16 *>(s.C);
+    int64_t b_bs = s.B_batch_stride, b_ts = s.B_token_stride, c_bs = s.C_batch_stride, c_ts = s.C_token_stride;
+    if (s.d_conv > 0) {
+        // pre-pass: conv + SiLU of the B and C channels, once per group, into the workspace
+        __nv_bfloat16 *wB = static_cast<__nv_bfloat16 *>(ws);
+        const size_t one = (size_t)s.batch * (size_t)s.seqlen * (size_t)GN * 2;
+        __nv_bfloat16 *wC = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + (one + 255) / 256 * 256);
+        for (int which = 0; which < 2; ++which) {
+            ConvJob j;
+            j.x = which == 0 ? s.B : s.C;
+            j.x_bs = which == 0 ? s.B_batch_stride : s.C_batch_stride;
+            j.x_ts = which == 0 ? s.B_token_stride : s.C_token_stride;
+            const int64_t ch0 = s.d_inner + which * GN;
+            j.w = s.conv_w + ch0 * s.d_conv;
+            j.b = s.conv_b ? s.conv_b + ch0 : nullptr;
+            const size_t es = 2;
+            j.state_in = s.conv_state_in ? static_cast<const char *>(s.conv_state_in) + ch0 * (s.d_conv - 1) * es : nullptr;
+            j.state_out = s.conv_state_out ? static_cast<char *>(s.conv_state_out) + ch0 * (s.d_conv - 1) * es : nullptr;
+            j.state_stride = cdim * (s.d_conv - 1);
+            j.cu = s.cu_seqlens; j.nseqs = s.nseqs; j.batch = s.batch; j.seqlen = s.seqlen;
+            j.channels = GN; j.width = s.d_conv; j.act = 1; j.dtype = SSM_BF16;
+            j.out = which == 0 ? (void *)wB : (void *)wC;
+            j.o_bs = s.seqlen * GN; j.o_ts = GN;
+            cudaError_t e = launch_conv_job(j, st);
+            if (e != cudaSuccess) return e;
+        }
+        Bc = wB; Cc = wC;
+        b_bs = c_bs = s.seqlen * GN;
+        b_ts = c_ts = GN;
+    }
+    SsdArgs a;
+    a.x = static_cast<const __nv_bfloat16 *>(s.x); a.z = static_cast<const __nv_bfloat16 *>(s.z);
+    a.dt = static_cast<const __nv_bfloat16 *>(s.dt); a.Bc = Bc; a.Cc = Cc;
+    a.y = static_cast<__nv_bfloat16 *>(s.y);
+    a.x_bs = s.x_batch_stride; a.x_ts = s.x_token_stride; a.z_bs = s.z_batch_stride; a.z_ts = s.z_token_stride;
+    a.dt_bs = s.dt_batch_stride; a.dt_ts = s.dt_token_stride;
+    a.b_bs = b_bs; a.b_ts = b_ts; a.c_bs = c_bs; a.c_ts = c_ts;
+    a.y_bs = s.y_batch_stride; a.y_ts = s.y_token_stride;
+    a.A = s.A; a.D = s.D; a.dt_bias = s.dt_bias; a.h0 = s.h0; a.conv_w = s.conv_w; a.conv_b = s.conv_b;
+    a.h_final = s.h_final;
+    a.conv_state_in = static_cast<const __nv_bfloat16 *>(s.conv_state_in);
+    a.conv_state_out = static_cast<__nv_bfloat16 *>(s.conv_state_out);
+    a.H = s.nheads; a.G = s.ngroups; a.seqlen = s.seqlen; a.cdim = cdim;
+    a.K = (int)s.d_conv; a.softplus = s.delta_softplus;
+    a.sv = sv;
+    a.err = sv.err;
+    cudaError_t e = cudaFuncSetAttribute(ssd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)s.nheads, (unsigned)nseqs);
+    ssd_kernel<<<grid, kThreads, kSmemBytes, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace ssm

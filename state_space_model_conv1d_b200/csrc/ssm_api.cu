@@ -166,27 +166,55 @@ ssm_status ssm_conv1d_fwd(const ssm_conv_args *args, void *stream) {
     return cuda_status(ssm::launch_conv1d(*args, (cudaStream_t)stream));
 }
 
+namespace {
+struct WsPlan {
+    size_t order_off, bc_off, total;
+    bool ssd;
+};
+WsPlan plan_workspace(const ssm_scan_args *a) {
+    WsPlan p{0, 0, 0, false};
+    p.ssd = ssm::ssd_supported(*a);
+    size_t off = 0;
+    if (a->cu_seqlens || p.ssd) off = ssm::kWsOrderOffset;      // error word
+    if (a->cu_seqlens) {
+        p.order_off = off;
+        off += ssm::order_bytes(a->nseqs);
+    }
+    if (p.ssd) {
+        p.bc_off = off;
+        off += ssm::ssd_workspace_bytes(*a);
+    }
+    p.total = off;
+    return p;
+}
+}  // namespace
+
 size_t ssm_scan_workspace_size(const ssm_scan_args *args) {
-    if (!args || !args->cu_seqlens) return 0;
-    return ssm::varlen_workspace_bytes(args->nseqs);
+    if (!args || validate_scan(args) != SSM_OK) return 0;
+    return plan_workspace(args).total;
 }
 
 ssm_status ssm_scan_fwd(const ssm_scan_args *args, void *workspace, size_t ws_bytes, void *stream) {
     SSM_TRY(validate_scan(args));
     const cudaStream_t st = (cudaStream_t)stream;
     ssm::SeqView sv{nullptr, nullptr, nullptr, (int)args->batch};
-    if (args->cu_seqlens) {
-        const size_t need = ssm::varlen_workspace_bytes(args->nseqs);
-        if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return SSM_ERR_WORKSPACE;
-        char *ws = static_cast<char *>(workspace);
-        sv.cu = args->cu_seqlens;
+    const WsPlan plan = plan_workspace(args);
+    char *ws = static_cast<char *>(workspace);
+    if (plan.total > 0) {
+        if (!workspace || ws_bytes < plan.total || !aligned(workspace, 256)) return SSM_ERR_WORKSPACE;
         sv.err = reinterpret_cast<int32_t *>(ws + ssm::kWsErrorOffset);
-        sv.order = reinterpret_cast<int32_t *>(ws + ssm::kWsOrderOffset);
+    }
+    if (args->cu_seqlens) {
+        sv.cu = args->cu_seqlens;
+        sv.order = reinterpret_cast<int32_t *>(ws + plan.order_off);
         sv.nseqs = args->nseqs;
         SSM_TRY(cuda_status(ssm::launch_varlen_plan(args->cu_seqlens, args->nseqs, args->seqlen, sv.err,
                                                     const_cast<int32_t *>(sv.order), st)));
+    } else if (sv.err) {
+        SSM_TRY(cuda_status(cudaMemsetAsync(sv.err, 0, sizeof(int32_t), st)));
     }
     if (args->mode == SSM_MAMBA1) return cuda_status(ssm::launch_scan_m1(*args, sv, st));
+    if (plan.ssd) return cuda_status(ssm::launch_ssd(*args, sv, ws + plan.bc_off, st));
     return cuda_status(ssm::launch_scan_m2_simt(*args, sv, st));
 }
 

@@ -301,3 +301,65 @@ def test_split_invariance(mode):
         assert rel_err(np.concatenate([y1, y2], 1), y) <= 1e-5
         assert rel_err(h2, hf) <= 1e-5
         assert np.array_equal(c2, cs)
+
+
+# ------------------------------------------- Mamba-2 on the tensor-core path
+# headdim 64, dstate 128, bf16 activations, conv width <= 4 take the chunked
+# tcgen05 kernel (64-token chunks); the cases cross chunk boundaries and end
+# on ragged tails.
+SSD_CASES = [
+    # (b, T, H, G, K)
+    (1, 1, 2, 1, 4),
+    (2, 64, 4, 2, 4),
+    (2, 65, 4, 2, 4),
+    (1, 200, 6, 3, 4),
+    (2, 130, 4, 4, 3),
+    (1, 97, 2, 1, 2),
+    (2, 70, 4, 2, 0),       # no conv: B, C and x used as given
+]
+
+
+@pytest.mark.parametrize("b,T,H,G,K", SSD_CASES)
+def test_ssd(b, T, H, G, K):
+    d = W.mamba2_inputs(800 + T + H + K, b, T, H, 64, G, 128, d_conv=K, dtype="bf16", conv_bias=True,
+                        conv_state=True)
+    check_scan(M2, d, "bf16", what=f"SSD b{b} T{T} H{H} G{G} K{K}")
+
+
+def test_ssd_optional_inputs_absent():
+    d = W.mamba2_inputs(820, 2, 100, 4, 64, 2, 128, dtype="bf16", with_h0=False, with_z=False)
+    d["D"] = None
+    d["dt_bias"] = None
+    check_scan(M2, d, "bf16", what="SSD minimal")
+
+
+def test_ssd_strided_views():
+    d = W.mamba2_inputs(821, 2, 90, 4, 64, 2, 128, dtype="bf16", conv_state=True)
+    check_scan(M2, d, "bf16", views=True, what="SSD views")
+
+
+def test_ssd_varlen():
+    lengths = [63, 0, 1, 64, 65, 200, 2, 130]
+    cu = W.cu_from_lengths(lengths)
+    d = W.mamba2_inputs(822, 1, int(cu[-1]), 4, 64, 2, 128, dtype="bf16", conv_state=True, nseqs=len(lengths))
+    d["cu_seqlens"] = cu
+    check_scan(M2, d, "bf16", what="SSD varlen")
+
+
+def test_ssd_split_invariance():
+    """Continuing a sequence from the returned state reproduces one long scan
+    (chunk boundaries land in different places in the two runs)."""
+    L = 180
+    d = W.mamba2_inputs(823, 2, L, 4, 64, 2, 128, dtype="bf16", conv_state=True)
+    t = to_dev(d, "bf16")
+    y, hf, cs = gpu_scan(M2, t)
+    for k in (37, 64, 100):
+        a = {kk: (v[:, :k] if kk in ("x", "z", "dt", "B", "C") else v) for kk, v in t.items()}
+        b = {kk: (v[:, k:] if kk in ("x", "z", "dt", "B", "C") else v) for kk, v in t.items()}
+        y1, h1, c1 = gpu_scan(M2, a)
+        b["h0"] = torch.from_numpy(h1).float().cuda()
+        b["conv_state_in"] = torch.from_numpy(c1).to(torch.bfloat16).cuda()
+        y2, h2, c2 = gpu_scan(M2, b)
+        assert rel_err(np.concatenate([y1, y2], 1), y) <= 2e-2
+        assert rel_err(h2, hf) <= 2e-2
+        assert np.array_equal(c2, cs)
