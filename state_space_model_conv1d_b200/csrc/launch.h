@@ -53,7 +53,8 @@ cudaError_t launch_scan_m1(const ssm_scan_args &a, const SeqView &sv, cudaStream
 cudaError_t launch_scan_m2_simt(const ssm_scan_args &a, const SeqView &sv, cudaStream_t st);
 // Tensor-core (tcgen05) chunked Mamba-2 path: which shapes it takes, the
 // workspace it needs for the conv'd B / C, and its launcher.
-bool ssd_supported(const ssm_scan_args &a);
+bool ssd_shape_ok(const ssm_scan_args &a);      // shapes only: decides the workspace size
+bool ssd_supported(const ssm_scan_args &a);     // shapes and 16-byte alignment: decides the kernel
 size_t ssd_workspace_bytes(const ssm_scan_args &a);
 cudaError_t launch_ssd(const ssm_scan_args &a, const SeqView &sv, void *ws_bc, cudaStream_t st);
 cudaError_t launch_state_update(const ssm_update_args &a, cudaStream_t st);

@@ -410,10 +410,15 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
 
 }  // namespace
 
+bool ssd_shape_ok(const ssm_scan_args &s) {
+    return s.mode == SSM_MAMBA2 && s.dtype == SSM_BF16 && s.headdim == kP && s.dstate == kN && s.d_conv >= 0 &&
+           s.d_conv <= 4;
+}
+
 bool ssd_supported(const ssm_scan_args &s) {
     auto al16 = [](const void *p) { return p == nullptr || ((uintptr_t)p & 15) == 0; };
     auto st16ok = [](int64_t v) { return (v * 2) % 16 == 0; };
-    return s.mode == SSM_MAMBA2 && s.dtype == SSM_BF16 && s.headdim == kP && s.dstate == kN && s.d_conv <= 4 &&
+    return ssd_shape_ok(s) &&
            al16(s.x) && al16(s.z) && al16(s.y) && al16(s.B) && al16(s.C) && st16ok(s.x_token_stride) &&
            st16ok(s.x_batch_stride) && st16ok(s.y_token_stride) && st16ok(s.y_batch_stride) &&
            (s.z == nullptr || (st16ok(s.z_token_stride) && st16ok(s.z_batch_stride))) &&

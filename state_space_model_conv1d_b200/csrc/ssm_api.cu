@@ -171,16 +171,19 @@ struct WsPlan {
     size_t order_off, bc_off, total;
     bool ssd;
 };
+// The workspace depends on shapes only (a call whose pointers rule out the
+// tensor-core path still finds its error word and schedule in the same place).
 WsPlan plan_workspace(const ssm_scan_args *a) {
     WsPlan p{0, 0, 0, false};
-    p.ssd = ssm::ssd_supported(*a);
+    const bool ssd_shape = ssm::ssd_shape_ok(*a);
+    p.ssd = ssd_shape && ssm::ssd_supported(*a);
     size_t off = 0;
-    if (a->cu_seqlens || p.ssd) off = ssm::kWsOrderOffset;      // error word
+    if (a->cu_seqlens || ssd_shape) off = ssm::kWsOrderOffset;      // error word
     if (a->cu_seqlens) {
         p.order_off = off;
         off += ssm::order_bytes(a->nseqs);
     }
-    if (p.ssd) {
+    if (ssd_shape) {
         p.bc_off = off;
         off += ssm::ssd_workspace_bytes(*a);
     }
@@ -190,7 +193,8 @@ WsPlan plan_workspace(const ssm_scan_args *a) {
 }  // namespace
 
 size_t ssm_scan_workspace_size(const ssm_scan_args *args) {
-    if (!args || validate_scan(args) != SSM_OK) return 0;
+    if (!args || args->batch < 0 || args->seqlen < 0 || args->nseqs < 0 || args->ngroups < 0 || args->dstate < 0)
+        return 0;
     return plan_workspace(args).total;
 }
 

@@ -143,9 +143,18 @@ def _scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, h0, h_final, cu_seqlens, co
     return a
 
 
-def scan_workspace_size(mode, x, dt, A, B, C_, *, cu_seqlens=None, **_):
+def scan_workspace_size(mode, x, dt, A, B, C_, *, cu_seqlens=None, conv_w=None, **_):
+    """Bytes of device workspace ssm_scan_fwd needs for these shapes (0 = none)."""
     a = _abi.ScanArgs()
-    a.mode = mode
+    a.mode, a.dtype = mode, _dtype_code(x)
+    a.batch, a.seqlen = x.shape[0], x.shape[1]
+    if mode == MAMBA1:
+        a.d_inner, a.ngroups, a.dstate = x.shape[2], 1, B.shape[2]
+    else:
+        a.nheads, a.headdim = x.shape[2], x.shape[3]
+        a.d_inner = a.nheads * a.headdim
+        a.ngroups, a.dstate = B.shape[2], B.shape[3]
+    a.d_conv = 0 if conv_w is None else conv_w.shape[1]
     a.cu_seqlens = _p(cu_seqlens)
     a.nseqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
     return int(_abi.lib().ssm_scan_workspace_size(C.byref(a)))

@@ -124,11 +124,17 @@ def test_scan_rejects_null_args():
 
 
 def test_workspace_size_is_host_only():
-    a = _scan()
+    a = _scan()                                         # Mamba-2 shapes off the tensor-core path
     assert _abi.lib().ssm_scan_workspace_size(C.byref(a)) == 0
     a = _scan(cu_seqlens=FAKE, nseqs=1000, batch=1)
     n = _abi.lib().ssm_scan_workspace_size(C.byref(a))
     assert n >= 256 + 4 * 1000 and n % 256 == 0
+    # headdim 64 / dstate 128 / bf16 / conv: error word + conv'd B and C (2 bytes each)
+    a = _scan(nheads=4, headdim=64, d_inner=256, ngroups=2, dstate=128, d_conv=4, conv_w=FAKE)
+    n = _abi.lib().ssm_scan_workspace_size(C.byref(a))
+    assert n == 256 + 2 * (2 * 16 * 2 * 128 * 2)
+    a = _scan(mode=1, d_inner=8, ngroups=1)             # Mamba-1 needs none
+    assert _abi.lib().ssm_scan_workspace_size(C.byref(a)) == 0
 
 
 def _conv(**kw):
