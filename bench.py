@@ -162,21 +162,37 @@ class Job:
                 cdim = x.shape[2] * x.shape[3] + 2 * t["B"].shape[2] * t["B"].shape[3]
             self.hf = torch.empty(hshape, dtype=torch.float32, device=dev)
             self.cso = torch.empty((nseq, cdim, t["conv_w"].shape[1] - 1), dtype=bf, device=dev)
-            need = ssm.scan_workspace_size(mode, x, t["dt"], t["A"], t["B"], t["C"], cu_seqlens=t.get("cu_seqlens"))
+            need = ssm.scan_workspace_size(mode, x, t["dt"], t["A"], t["B"], t["C"], cu_seqlens=t.get("cu_seqlens"),
+                                           conv_w=t["conv_w"])
             self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev) if need else None
-            if need:
-                self.launches_per_step = 2
+            self.ssd = mode == ssm.MAMBA2 and w.dtype == "bf16" and w.headdim == 64 and w.dstate == 128 and w.d_conv <= 4
+            varlen = t.get("cu_seqlens") is not None
+            if self.ssd:
+                # B and C conv pre-pass (+ their carried-state kernels), then the chunked tensor-core scan
+                self.launches_per_step = 2 + 2 + 1 + (1 if varlen else 0)
+            else:
+                self.launches_per_step = 1 + (1 if varlen else 0)
             read = sum(v.numel() * v.element_size() for k, v in t.items() if v is not None)
             wrote = sum(v.numel() * v.element_size() for v in (self.y, self.hf, self.cso))
             self.bytes_per_step = read + wrote
             self.units = self.tokens
-            self.kernel = "scan_m1_kernel" if mode == ssm.MAMBA1 else "scan_m2"
-            self.sources = ("scan_m1.cu",) if mode == ssm.MAMBA1 else ("scan_m2_simt.cu",)
             if mode == ssm.MAMBA1:
+                self.kernel, self.sources = "scan_m1_kernel", ("scan_m1.cu",)
                 self.mufu = x.shape[0] * x.shape[1] * x.shape[2] * t["B"].shape[2]
-            else:
+                self.flops = None
+            elif self.ssd:
+                self.kernel, self.sources = "ssd_kernel", ("ssd_m2.cu", "conv1d.cu")
                 self.mufu = None
-            self.flops = None
+                # tensor-core work of the 64-token chunked form: per (sequence, head, chunk)
+                # C.B^T (2 Q^2 N) + M.X (2 Q^2 P) + C'.S^T (2 Q N P) + B'^T.X (2 Q N P)
+                Q, P, N = 64, w.headdim, w.dstate
+                nchunks = int(sum((int(L) + Q - 1) // Q for L in np.diff(d["cu_seqlens"]))) if varlen else \
+                    x.shape[0] * ((x.shape[1] + Q - 1) // Q)
+                self.flops = nchunks * w.nheads * (2 * Q * Q * N + 2 * Q * Q * P + 4 * Q * N * P)
+            else:
+                self.kernel, self.sources = "scan_m2_simt_kernel", ("scan_m2_simt.cu",)
+                self.mufu = None
+                self.flops = None
         elif w.kind == "decode":
             ww = W.Workload(**{**w.__dict__, "seed": w.seed + seed_shift})
             d = W.workload_inputs(ww)
@@ -345,6 +361,11 @@ def run_cuda(args):
         roofline = {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
                     "traffic": traffic, "kernel": job.kernel,
                     "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback"}
+        if job.flops:
+            tf = job.flops / (ms_per_step / 1e3) / 1e12
+            tpk = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1400.0)))
+            roofline["tensor"] = {"achieved": tf, "peak": tpk, "unit": "TFLOP/s", "frac": tf / tpk,
+                                  "flops_per_step": int(job.flops), "peak_source": "MEASURED_PEAKS.json bf16_tflops_sustained"}
     roofline["algorithmic_bytes_per_launch"] = int(job.bytes_per_step)
 
     cpu = None
