@@ -201,6 +201,29 @@ SSM_API ssm_status ssm_scan_fwd(const ssm_scan_args *args, void *workspace, size
 /* Decode update, in place on state and conv_state.  No workspace. */
 SSM_API ssm_status ssm_state_update(const ssm_update_args *args, void *stream);
 
+/* ssm_scan_fwd without a caller-supplied workspace, for callers that cannot
+ * allocate device memory (code inside a CUDA-graph capture that must not
+ * allocate, a runtime whose memory pool belongs to another component, a
+ * plugin handed buffers but no allocator).  The paper has no counterpart:
+ * this is an interface convenience of this library, not a step of the method.
+ *
+ * The workspace comes from a file-scope device array of
+ * SSM_NOALLOC_SCRATCH_BYTES bytes (one per GPU that loads the library, held
+ * until the process exits).  Calls whose ssm_scan_workspace_size() exceeds
+ * that return SSM_ERR_WORKSPACE and launch nothing; use ssm_scan_fwd then.
+ * Nothing here allocates or frees memory.  The first call on a device looks
+ * up the array's device address (cudaGetSymbolAddress, with that device
+ * current) and caches it: make that first call before any stream capture.
+ * Every call shares the one array and the scan initialises what it reads
+ * (the error word, the varlen schedule) on each call; calls that may
+ * overlap on the GPU (different streams, or different host threads on one
+ * device) race on it, so serialise them.  The error word can be read back
+ * with ssm_workspace_error() only by code that knows the array's address,
+ * so this entry point reports device-side errors by leaving its outputs
+ * unwritten, as ssm_scan_fwd does. */
+#define SSM_NOALLOC_SCRATCH_BYTES (4u << 20)
+SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *args, void *stream);
+
 /* Waits for `stream`, then reads the device error word of a workspace last
  * used by ssm_scan_fwd: SSM_OK, or SSM_ERR_DEVICE with *code set to an
  * SSM_DEVERR_* value.  `code` may be NULL. */

@@ -80,6 +80,7 @@ SIGNATURES = {
     "ssm_scan_fwd": ([C.POINTER(ScanArgs), _vp, C.c_size_t, _vp], _i32),
     "ssm_state_update": ([C.POINTER(UpdateArgs), _vp], _i32),
     "ssm_workspace_error": ([_vp, C.POINTER(_i32), _vp], _i32),
+    "ssm_scan_fwd_noalloc": ([C.POINTER(ScanArgs), _vp], _i32),
 }
 
 _lock = threading.Lock()
