@@ -129,7 +129,7 @@ class Job:
     def __init__(self, w: W.Workload, rank: int, torch, ssm):
         self.w, self.torch, self.ssm = w, torch, ssm
         dev = torch.device("cuda", torch.cuda.current_device())
-        seed_shift = 7919 * rank
+        seed_shift = rank_seed(0, rank)
         bf = torch.bfloat16 if w.dtype == "bf16" else torch.float32
         self.launches_per_step = 1
         if w.kind in ("mamba1", "mamba2", "mamba2_varlen"):
@@ -261,6 +261,27 @@ def flush_l2(buf):
     buf.add_(1)       # 256 MiB read + write, twice the 126 MB L2
 
 
+def reduce_max_ms(ms: float, world: int, device) -> float:
+    """Max over ranks of a device-measured time (the slowest rank sets the pace)."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank processes its own batch (weak scaling)."""
+    return units_per_rank * steps * world / (max_ms / 1e3)
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own synthetic batch."""
+    return base + 7919 * rank
+
+
 def run_cuda(args):
     import torch
     import torch.distributed as dist
@@ -301,14 +322,9 @@ def run_cuda(args):
         dist.barrier()
     clk = clocks.stop() if rank == 0 else None
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        tt = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = reduce_max_ms(float(sum(step_ms)), world, "cuda")
     ms_per_step = total_ms / max(args.steps, 1)
-    units_total = job.units * args.steps * world
-    value = units_total / (total_ms / 1e3)
+    value = weak_scaling_value(job.units, args.steps, world, total_ms)
 
     # end to end through the public API with host-resident inputs
     e2e = None
@@ -326,12 +342,8 @@ def run_cuda(args):
             h2d, d2h = job.e2e_step(out_host)
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([ems], device="cuda")
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
-        e2e = {"value": job.units * ne * world / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+        ems = reduce_max_ms(e0.elapsed_time(e1), world, "cuda")
+        e2e = {"value": weak_scaling_value(job.units, ne, world, ems), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": ne}
 
     if world > 1:
