@@ -18,7 +18,7 @@ namespace ssm {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kTokensPerThread = 32;
+constexpr int kTokensPerThread = 8;
 
 template <typename T, int VEC, int K>
 __global__ void __launch_bounds__(kThreads)

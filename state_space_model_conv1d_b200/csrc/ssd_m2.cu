@@ -87,6 +87,11 @@ struct SsdArgs {
 
 SSM_DEVINL uint4 ld16(const void *p) { return *reinterpret_cast<const uint4 *>(p); }
 SSM_DEVINL void st16(void *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
+SSM_DEVINL void cp_async16(void *smem_dst, const void *gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(tc::smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+SSM_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+SSM_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -169,22 +174,61 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
     uint32_t fail_par = 0;
 
     const int nchunks = (int)((len + kQ - 1) / kQ);
+    const uint4 zero4 = make_uint4(0, 0, 0, 0);
+    // Stage chunk cn: B and C straight into their operand tiles, the raw x rows
+    // (row-major [kQ][kP] bf16) into the M tile's space, which is free from
+    // the end of MMA2 until the mask phase of the next chunk.  Asynchronous
+    // 16-byte copies; rows past the sequence end are zero-filled.
+    auto prefetch = [&](int cn) {
+        const int64_t tn = (int64_t)cn * kQ;
+        const int nvn = (int)min((int64_t)kQ, len - tn);
+        for (int i = tid; i < kQ * (kN / 8); i += kThreads) {
+            const int r = i / (kN / 8), q = i % (kN / 8);
+            const uint32_t off = tc::off_kmajor(r, q * 8, 128, 2048);
+            if (r < nvn) {
+                cp_async16(smem + OFF_B + off, Bg + (tn + r) * a.b_ts + q * 8);
+                cp_async16(smem + OFF_C + off, Cg + (tn + r) * a.c_ts + q * 8);
+            } else {
+                st16(smem + OFF_B + off, zero4);
+                st16(smem + OFF_C + off, zero4);
+            }
+        }
+        for (int i = tid; i < kQ * (kP / 8); i += kThreads) {
+            const int r = i / (kP / 8), q = i % (kP / 8);
+            unsigned char *dst = smem + OFF_M + r * (kP * 2) + q * 16;
+            if (r < nvn) cp_async16(dst, xg + (tn + r) * a.x_ts + q * 8);
+            else st16(dst, zero4);
+        }
+        cp_async_commit();
+    };
+    // raw dt of chunk cn for warp 0 (lane l holds tokens l and l + 32)
+    float dtr0 = 0.f, dtr1 = 0.f;
+    auto load_dt = [&](int cn) {
+        const int64_t tn = (int64_t)cn * kQ;
+        const int nvn = (int)min((int64_t)kQ, len - tn);
+        dtr0 = lane < nvn ? __bfloat162float(dtg[(tn + lane) * a.dt_ts]) : 0.f;
+        dtr1 = lane + 32 < nvn ? __bfloat162float(dtg[(tn + lane + 32) * a.dt_ts]) : 0.f;
+    };
+    if (nchunks > 0) {
+        prefetch(0);
+        if (warp == 0) load_dt(0);
+        cp_async_wait_all();
+        tc::fence_proxy_async();
+        __syncthreads();
+    }
+    const unsigned char *xraw = smem + OFF_M;                      // staged raw x rows of the current chunk
+    auto raw_row = [&](int r, int q, float *v) { tc::unpack_bf16x8(ld16(xraw + r * (kP * 2) + q * 16), v); };
+
     for (int c = 0; c < nchunks; ++c) {
         const int64_t t0 = (int64_t)c * kQ;
         const int nv = (int)min((int64_t)kQ, len - t0);
         const int hb = c & 1;
 
-        // ---- (1) delta, running decay (warp 0); B, C tiles; x conv
+        // ---- (1) delta and running decay (warp 0); x conv from the staged raw rows
         if (warp == 0) {
             float d0 = 0.f, d1 = 0.f;
-            if (lane < nv) {
-                const float u = __bfloat162float(dtg[(t0 + lane) * a.dt_ts]) + dtb;
-                d0 = a.softplus ? softplus(u) : u;
-            }
-            if (lane + 32 < nv) {
-                const float u = __bfloat162float(dtg[(t0 + lane + 32) * a.dt_ts]) + dtb;
-                d1 = a.softplus ? softplus(u) : u;
-            }
+            if (lane < nv) d0 = a.softplus ? softplus(dtr0 + dtb) : dtr0 + dtb;
+            if (lane + 32 < nv) d1 = a.softplus ? softplus(dtr1 + dtb) : dtr1 + dtb;
             float s0 = d0 * A2, s1 = d1 * A2;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -204,17 +248,6 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             ax.wj[lane + 32] = ex2(last - s1) * d1;
             if (lane == 0) ax.dAc = ex2(last);
         }
-        for (int i = tid; i < kQ * (kN / 8); i += kThreads) {
-            const int r = i / (kN / 8), q = i % (kN / 8);
-            uint4 vb = make_uint4(0, 0, 0, 0), vc = make_uint4(0, 0, 0, 0);
-            if (r < nv) {
-                vb = ld16(Bg + (t0 + r) * a.b_ts + q * 8);
-                vc = ld16(Cg + (t0 + r) * a.c_ts + q * 8);
-            }
-            const uint32_t off = tc::off_kmajor(r, q * 8, 128, 2048);
-            st16(smem + OFF_B + off, vb);
-            st16(smem + OFF_C + off, vc);
-        }
         {
             // conv + SiLU of 8 channels x 4 tokens; window = raw rows r0-3 .. r0-1
             float win[kHx][8];
@@ -224,22 +257,15 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
                 if (v < 0) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) win[j][e] = ax.xh[hb][kHx + v][po * 8 + e];
-                } else if (v < nv) {
-                    tc::unpack_bf16x8(ld16(xg + (t0 + v) * a.x_ts + po * 8), win[j]);
                 } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) win[j][e] = 0.f;
+                    raw_row(v, po, win[j]);                           // rows >= nv are zeros
                 }
             }
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int r = r0 + i;
                 float cur[8], o[8];
-                if (r < nv) tc::unpack_bf16x8(ld16(xg + (t0 + r) * a.x_ts + po * 8), cur);
-                else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) cur[e] = 0.f;
-                }
+                raw_row(r, po, cur);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     float acc;
@@ -267,7 +293,9 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
 #pragma unroll
             for (int j = 0; j < kHx; ++j) {
                 const int v = nv - kHx + j;
-                ax.xh[hb ^ 1][j][p] = v >= 0 ? __bfloat162float(xg[(t0 + v) * a.x_ts + p]) : ax.xh[hb][kHx + v][p];
+                ax.xh[hb ^ 1][j][p] = v >= 0 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                                                   xraw + v * (kP * 2) + p * 2))
+                                             : ax.xh[hb][kHx + v][p];
             }
         }
         tc::fence_proxy_async();
@@ -286,20 +314,22 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         if (!ok) { fail_bar = 0; fail_par = c & 1; break; }
         tc::fence_after_sync();
 
-        // ---- (3) mask G -> M; rescale C -> C', B -> B'
-        {
-            float Gv[64];
-            tc::tmem_ld64(tmem + t_lane, Gv);
+        // ---- (3) mask G -> M (over the staged raw rows, already consumed); rescale C -> C', B -> B'
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float Gv[32];
+            tc::tmem_ld32(tmem + t_lane + half * 32, Gv);
             if (lane < 16) {
                 const int i = warp * 16 + lane;
                 const float ci = ax.cs2[i];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int q = half * 4 + qq;
                     float m[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int j = q * 8 + e;
-                        m[e] = j <= i ? Gv[j] * ex2(ci - ax.cs2[j]) * ax.dlt[j] : 0.f;
+                        m[e] = j <= i ? Gv[qq * 8 + e] * ex2(ci - ax.cs2[j]) * ax.dlt[j] : 0.f;
                     }
                     st16(smem + OFF_M + tc::off_kmajor(i, q * 8, 128, 1024), tc::pack_bf16x8(m));
                 }
@@ -320,6 +350,12 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             for (int e = 0; e < 8; ++e) v[e] *= fb;
             st16(smem + OFF_B + off, tc::pack_bf16x8(v));
         }
+        // z of this chunk's rows, in flight while the tensor cores run
+        uint4 zr[8];
+        const int yi = warp * 16 + lane;
+        const bool yrow = lane < 16 && yi < nv;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) zr[q] = (zg && yrow) ? ld16(zg + (t0 + yi) * a.z_ts + q * 8) : zero4;
         tc::fence_before_sync();
         tc::fence_proxy_async();
         __syncthreads();
@@ -344,40 +380,48 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         ok = __syncthreads_and(tc::mbar_wait(&ax.mbar[1], c & 1));
         if (!ok) { fail_bar = 1; fail_par = c & 1; break; }
         tc::fence_after_sync();
+        // B, C and the M tile are free again: stage the next chunk behind the epilogue
+        if (c + 1 < nchunks) {
+            prefetch(c + 1);
+            if (warp == 0) load_dt(c + 1);
+        }
 
         // ---- (5) y = (Y + D x) * silu(z); S = exp(cs_Q) S + Sc
-        {
-            float Yv[64];
-            tc::tmem_ld64(tmem + t_lane + 64, Yv);
-            if (lane < 16) {
-                const int i = warp * 16 + lane;
-                if (i < nv) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float xv[8], zv[8], o[8];
-                        tc::unpack_bf16x8(ld16(smem + OFF_X + tc::off_mnmajor(q * 8, i, 1024, 128)), xv);
-                        if (zg) tc::unpack_bf16x8(ld16(zg + (t0 + i) * a.z_ts + q * 8), zv);
+        for (int half = 0; half < 2; ++half) {                   // 32 columns at a time keeps registers down
+            float Yv[32];
+            tc::tmem_ld32(tmem + t_lane + 64 + half * 32, Yv);
+            if (yrow) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            float yv = fmaf(Dh, xv[e], Yv[q * 8 + e]);
-                            o[e] = zg ? yv * silu_fast<__nv_bfloat16>(zv[e]) : yv;
-                        }
-                        st16(yg + (t0 + i) * a.y_ts + q * 8, tc::pack_bf16x8(o));
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int q = half * 4 + qq;
+                    float xv[8], zv[8], o[8];
+                    tc::unpack_bf16x8(ld16(smem + OFF_X + tc::off_mnmajor(q * 8, yi, 1024, 128)), xv);
+                    tc::unpack_bf16x8(zr[q], zv);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        float yv = fmaf(Dh, xv[e], Yv[qq * 8 + e]);
+                        o[e] = zg ? yv * silu_fast<__nv_bfloat16>(zv[e]) : yv;
                     }
+                    st16(yg + (t0 + yi) * a.y_ts + q * 8, tc::pack_bf16x8(o));
                 }
             }
         }
         {
-            float Sc[64];
-            tc::tmem_ld64(tmem + t_lane, Sc);
             const float dAc = ax.dAc;
             const int n = tid;
 #pragma unroll
-            for (int p = 0; p < kP; ++p) S[p] = fmaf(dAc, S[p], Sc[p]);
+            for (int half = 0; half < 2; ++half) {
+                float Sc[32];
+                tc::tmem_ld32(tmem + t_lane + half * 32, Sc);
+#pragma unroll
+                for (int p = 0; p < 32; ++p) S[half * 32 + p] = fmaf(dAc, S[half * 32 + p], Sc[p]);
+            }
 #pragma unroll
             for (int q = 0; q < 8; ++q)
                 st16(smem + OFF_S + tc::off_mnmajor(q * 8, n, 1024, 128), tc::pack_bf16x8(&S[q * 8]));
         }
+        cp_async_wait_all();
         tc::fence_before_sync();
         tc::fence_proxy_async();
         __syncthreads();
