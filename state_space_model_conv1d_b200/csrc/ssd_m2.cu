@@ -17,7 +17,7 @@
 // ssd_state_passing, ssd_chunk_scan) are these four steps; here they are one
 // kernel whose carried state never leaves the SM.
 //
-// Layout of the work: one CTA per (sequence, head), 4 warps, walking the
+// Layout of the work: one CTA per (sequence, head), 8 warps, walking the
 // sequence in chunks of Q = 64.  The B / C causal conv + SiLU is shared by the
 // heads of a group, so it runs once per group in a pre-pass that writes bf16
 // B, C into the workspace; the x conv + SiLU runs here, fused.  Per chunk:
@@ -26,8 +26,9 @@
 //   MMA3  Y += C' S_prev^T   M=64  N=64 K=128   A K-major, B MN-major
 //   MMA4  Sc = B'^T X        M=128 N=64 K=64    A MN-major (same tile as B), B MN-major
 // C' and B' are C and B rescaled in place after MMA1 has consumed them.
-// The fp32 state S (128 x 64 per head) stays in registers, one state row n
-// per thread; its bf16 copy is the MMA3 operand of the next chunk.
+// The fp32 state S (128 x 64 per head) stays in registers, half a state row
+// per thread; its bf16 copy is the MMA3 operand of the next chunk.  Warps w
+// and w+4 share a tensor-memory lane quarter and split accumulator columns.
 //
 // Tensor memory: 128 columns (G in columns 0-63, later reused for Sc; Y in
 // 64-127), shared memory 67 KB, so three CTAs fit on one SM.
@@ -41,16 +42,17 @@ namespace {
 constexpr int kQ = 64;           // chunk length
 constexpr int kP = 64;           // headdim on this path
 constexpr int kN = 128;          // dstate on this path
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int kHx = 3;           // raw x rows kept before each chunk (conv width <= 4)
 constexpr uint32_t kTmemCols = 128;
 
-// operand tiles (bf16, core-matrix layouts), byte offsets in dynamic shared memory
-constexpr uint32_t OFF_C = 0;        // C [i][n]  K-major   LBO 128  SBO 2048
-constexpr uint32_t OFF_B = 16384;    // B [j][n]  K-major   LBO 128  SBO 2048  (MN-major view: LBO 2048 SBO 128)
-constexpr uint32_t OFF_M = 32768;    // M [i][j]  K-major   LBO 128  SBO 1024
-constexpr uint32_t OFF_X = 40960;    // X (p, j)  MN-major  LBO 1024 SBO 128
-constexpr uint32_t OFF_S = 49152;    // S (p, n)  MN-major  LBO 1024 SBO 128
+// operand tiles (bf16, 128-byte swizzle, atoms of 8 rows x 64 elements), byte
+// offsets from the 1024-aligned base of dynamic shared memory
+constexpr uint32_t OFF_C = 0;        // C rows i, K = n: two 8 KB K-atoms (n 0-63 | 64-127)
+constexpr uint32_t OFF_B = 16384;    // B rows j, K = n (MMA1); read as MN-major MN = n, K = j (MMA4)
+constexpr uint32_t OFF_M = 32768;    // M rows i, K = j; raw x rows are staged here between MMA2 and the mask
+constexpr uint32_t OFF_X = 40960;    // X rows j, 64 p each: MN-major MN = p, K = j (MMA2, MMA4)
+constexpr uint32_t OFF_S = 49152;    // S rows n, 64 p each: MN-major MN = p, K = n (MMA3)
 constexpr uint32_t OFF_AUX = 65536;
 
 struct Aux {
@@ -60,12 +62,10 @@ struct Aux {
     float ecs[kQ];                   // exp(cs_i)
     float wj[kQ];                    // exp(cs_Q - cs_j) * delta_j
     float dAc;                       // exp(cs_Q)
-    float cw[4][kP];                 // x conv taps, right-aligned (cw[3] multiplies the current token)
-    float cb[kP];                    // x conv bias
     uint32_t tmem;
     uint64_t mbar[2];
 };
-constexpr size_t kSmemBytes = OFF_AUX + sizeof(Aux);
+constexpr size_t kSmemBytes = OFF_AUX + sizeof(Aux) + 1024;   // + slack to align the base to 1024
 
 constexpr uint32_t ID_G = tc::idesc_bf16(64, 64, 0, 0);
 constexpr uint32_t ID_Y = tc::idesc_bf16(64, 64, 0, 1);
@@ -94,11 +94,15 @@ SSM_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: 
 SSM_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
-    extern __shared__ __align__(1024) unsigned char smem[];
+    extern __shared__ unsigned char smem_raw[];
+    // swizzle atoms need 1024-byte alignment: round the base up (1 KB of slack is allocated)
+    unsigned char *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     Aux &ax = *reinterpret_cast<Aux *>(smem + OFF_AUX);
     if (a.sv.err && *a.sv.err != 0) return;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3;          // tensor-memory lane quarter of this warp
+    const int half = warp >> 2;       // which 32 columns of a 64-column accumulator this warp reads
     const int hh = blockIdx.x;
     const int s = a.sv.order ? a.sv.order[blockIdx.y] : (int)blockIdx.y;
     int64_t start = 0, len = a.seqlen, row = s;
@@ -128,28 +132,27 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
     const float A2 = a.A[hh] * kLog2e;
     const float Dh = a.D ? a.D[hh] : 0.f;
     const float dtb = a.dt_bias ? a.dt_bias[hh] : 0.f;
-    // x conv role: channels po*8 .. po*8+7, tokens r0 .. r0+3
-    const int po = tid & 7, r0 = (tid >> 3) * 4;
-    if (tid < kP) {
-        const int64_t ch = hh * kP + tid;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int k = K - 4 + j;
-            ax.cw[j][tid] = (K > 0 && k >= 0) ? a.conv_w[ch * K + k] : 0.f;
-        }
-        ax.cb[tid] = a.conv_b ? a.conv_b[ch] : 0.f;
+    // x conv role: channel cp = tid % 64, tokens cr0 .. cr0+15; taps right-aligned
+    // (cw3 multiplies the current token, cw0 the one 3 back)
+    const int cp = tid & (kP - 1), cr0 = (tid / kP) * (kQ / 4);
+    float cw0, cw1, cw2, cw3, cbias;
+    {
+        const int64_t ch = hh * kP + cp;
+        auto tap = [&](int j) { const int k = K - 4 + j; return (K > 0 && k >= 0) ? a.conv_w[ch * K + k] : 0.f; };
+        cw0 = tap(0); cw1 = tap(1); cw2 = tap(2); cw3 = tap(3);
+        cbias = a.conv_b ? a.conv_b[ch] : 0.f;
     }
 
-    // ---- carried state: thread n owns S[n][p], p = 0..63 (fp32), plus its bf16 copy
-    float S[kP];
+    // ---- carried state: thread owns S[n][32*half .. 32*half+31] for n = 32*q4 + lane (fp32)
+    const int sn = q4 * 32 + lane;
+    float S[32];
     {
-        const int n = tid;
         const float *h0p = a.h0 ? a.h0 + ((int64_t)s * H + hh) * kP * kN : nullptr;
 #pragma unroll
-        for (int p = 0; p < kP; ++p) S[p] = h0p ? h0p[(int64_t)p * kN + n] : 0.f;
+        for (int p = 0; p < 32; ++p) S[p] = h0p ? h0p[(int64_t)(half * 32 + p) * kN + sn] : 0.f;
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-            st16(smem + OFF_S + tc::off_mnmajor(q * 8, n, 1024, 128), tc::pack_bf16x8(&S[q * 8]));
+        for (int q = 0; q < 4; ++q)
+            st16(smem + OFF_S + tc::off_sw128(sn, half * 32 + q * 8, 8192), tc::pack_bf16x8(&S[q * 8]));
     }
     // ---- conv halo of chunk 0 (the last K-1 raw inputs before the sequence)
     if (tid < kP) {
@@ -168,23 +171,23 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = ax.tmem;
-    const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
+    const uint32_t t_lane = (uint32_t)(q4 * 32) << 16;
     bool ok = true;
     int fail_bar = 0;
     uint32_t fail_par = 0;
 
     const int nchunks = (int)((len + kQ - 1) / kQ);
     const uint4 zero4 = make_uint4(0, 0, 0, 0);
-    // Stage chunk cn: B and C straight into their operand tiles, the raw x rows
-    // (row-major [kQ][kP] bf16) into the M tile's space, which is free from
-    // the end of MMA2 until the mask phase of the next chunk.  Asynchronous
-    // 16-byte copies; rows past the sequence end are zero-filled.
+    // Stage chunk cn: B and C straight into their swizzled operand tiles, the
+    // raw x rows (row-major [kQ][kP] bf16) into the M tile's space, which is
+    // free from the end of MMA2 until the mask phase of the next chunk.
+    // Asynchronous 16-byte copies; rows past the sequence end are zero-filled.
     auto prefetch = [&](int cn) {
         const int64_t tn = (int64_t)cn * kQ;
         const int nvn = (int)min((int64_t)kQ, len - tn);
         for (int i = tid; i < kQ * (kN / 8); i += kThreads) {
             const int r = i / (kN / 8), q = i % (kN / 8);
-            const uint32_t off = tc::off_kmajor(r, q * 8, 128, 2048);
+            const uint32_t off = tc::off_sw128(r, q * 8, 8192);
             if (r < nvn) {
                 cp_async16(smem + OFF_B + off, Bg + (tn + r) * a.b_ts + q * 8);
                 cp_async16(smem + OFF_C + off, Cg + (tn + r) * a.c_ts + q * 8);
@@ -201,13 +204,16 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         }
         cp_async_commit();
     };
-    // raw dt of chunk cn for warp 0 (lane l holds tokens l and l + 32)
-    float dtr0 = 0.f, dtr1 = 0.f;
+    // raw dt of chunk cn for warp 0 (lane l holds tokens l and l + 32); kept as
+    // bf16 so the load is not waited for until the next chunk uses it
+    __nv_bfloat16 dtr0 = __float2bfloat16_rn(0.f), dtr1 = dtr0;
     auto load_dt = [&](int cn) {
         const int64_t tn = (int64_t)cn * kQ;
         const int nvn = (int)min((int64_t)kQ, len - tn);
-        dtr0 = lane < nvn ? __bfloat162float(dtg[(tn + lane) * a.dt_ts]) : 0.f;
-        dtr1 = lane + 32 < nvn ? __bfloat162float(dtg[(tn + lane + 32) * a.dt_ts]) : 0.f;
+        dtr0 = __float2bfloat16_rn(0.f);
+        dtr1 = dtr0;
+        if (lane < nvn) dtr0 = dtg[(tn + lane) * a.dt_ts];
+        if (lane + 32 < nvn) dtr1 = dtg[(tn + lane + 32) * a.dt_ts];
     };
     if (nchunks > 0) {
         prefetch(0);
@@ -217,7 +223,6 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         __syncthreads();
     }
     const unsigned char *xraw = smem + OFF_M;                      // staged raw x rows of the current chunk
-    auto raw_row = [&](int r, int q, float *v) { tc::unpack_bf16x8(ld16(xraw + r * (kP * 2) + q * 16), v); };
 
     for (int c = 0; c < nchunks; ++c) {
         const int64_t t0 = (int64_t)c * kQ;
@@ -227,8 +232,9 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         // ---- (1) delta and running decay (warp 0); x conv from the staged raw rows
         if (warp == 0) {
             float d0 = 0.f, d1 = 0.f;
-            if (lane < nv) d0 = a.softplus ? softplus(dtr0 + dtb) : dtr0 + dtb;
-            if (lane + 32 < nv) d1 = a.softplus ? softplus(dtr1 + dtb) : dtr1 + dtb;
+            const float u0 = __bfloat162float(dtr0) + dtb, u1 = __bfloat162float(dtr1) + dtb;
+            if (lane < nv) d0 = a.softplus ? softplus(u0) : u0;
+            if (lane + 32 < nv) d1 = a.softplus ? softplus(u1) : u1;
             float s0 = d0 * A2, s1 = d1 * A2;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -249,42 +255,21 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             if (lane == 0) ax.dAc = ex2(last);
         }
         {
-            // conv + SiLU of 8 channels x 4 tokens; window = raw rows r0-3 .. r0-1
-            float win[kHx][8];
+            // conv + SiLU: thread -> channel cp, tokens cr0 .. cr0+15, sliding window in registers
+            auto raw1 = [&](int v) -> float {
+                return v < 0 ? ax.xh[hb][kHx + v][cp]
+                             : __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xraw + v * (kP * 2) + cp * 2));
+            };
+            float h0v = raw1(cr0 - 3), h1v = raw1(cr0 - 2), h2v = raw1(cr0 - 1);   // raw rows t-3, t-2, t-1
 #pragma unroll
-            for (int j = 0; j < kHx; ++j) {
-                const int v = r0 - kHx + j;
-                if (v < 0) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) win[j][e] = ax.xh[hb][kHx + v][po * 8 + e];
-                } else {
-                    raw_row(v, po, win[j]);                           // rows >= nv are zeros
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = r0 + i;
-                float cur[8], o[8];
-                raw_row(r, po, cur);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float acc;
-                    if (K > 0) {
-                        const int p = po * 8 + e;
-                        acc = fmaf(ax.cw[3][p], cur[e], ax.cb[p]);
-                        acc = fmaf(ax.cw[2][p], win[2][e], acc);
-                        acc = fmaf(ax.cw[1][p], win[1][e], acc);
-                        acc = fmaf(ax.cw[0][p], win[0][e], acc);
-                        acc = silu_fast<__nv_bfloat16>(acc);
-                    } else {
-                        acc = cur[e];
-                    }
-                    o[e] = r < nv ? acc : 0.f;
-                    win[0][e] = win[1][e];
-                    win[1][e] = win[2][e];
-                    win[2][e] = cur[e];
-                }
-                st16(smem + OFF_X + tc::off_mnmajor(po * 8, r, 1024, 128), tc::pack_bf16x8(o));
+            for (int i = 0; i < kQ / 4; ++i) {
+                const int r = cr0 + i;
+                const float cur = raw1(r);                            // rows >= nv are zeros
+                float acc = cur;
+                if (K > 0) acc = silu_fast<__nv_bfloat16>(fmaf(cw0, h0v, fmaf(cw1, h1v, fmaf(cw2, h2v, fmaf(cw3, cur, cbias)))));
+                if (r >= nv) acc = 0.f;
+                h0v = h1v; h1v = h2v; h2v = cur;
+                *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_X + tc::off_sw128(r, cp, 8192)) = __float2bfloat16_rn(acc);
             }
         }
         // halo of the next chunk: raw rows nv-3 .. nv-1 (from the old halo when the chunk is shorter)
@@ -305,9 +290,11 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         if (tid == 0) {
             tc::fence_after_sync();
 #pragma unroll
-            for (int k = 0; k < kN / 16; ++k)
-                tc::mma_bf16(tmem, tc::desc(sbase + OFF_C + k * 256, 128, 2048), tc::desc(sbase + OFF_B + k * 256, 128, 2048),
+            for (int k = 0; k < kN / 16; ++k) {
+                const uint32_t ko = (k >> 2) * 8192 + (k & 3) * 32;
+                tc::mma_bf16(tmem, tc::desc_sw128(sbase + OFF_C + ko, 16, 1024), tc::desc_sw128(sbase + OFF_B + ko, 16, 1024),
                              ID_G, k > 0);
+            }
             tc::mma_commit(&ax.mbar[0]);
         }
         ok = __syncthreads_and(tc::mbar_wait(&ax.mbar[0], c & 1));
@@ -315,12 +302,11 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         tc::fence_after_sync();
 
         // ---- (3) mask G -> M (over the staged raw rows, already consumed); rescale C -> C', B -> B'
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        {
             float Gv[32];
             tc::tmem_ld32(tmem + t_lane + half * 32, Gv);
             if (lane < 16) {
-                const int i = warp * 16 + lane;
+                const int i = q4 * 16 + lane;
                 const float ci = ax.cs2[i];
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
@@ -331,13 +317,13 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
                         const int j = q * 8 + e;
                         m[e] = j <= i ? Gv[qq * 8 + e] * ex2(ci - ax.cs2[j]) * ax.dlt[j] : 0.f;
                     }
-                    st16(smem + OFF_M + tc::off_kmajor(i, q * 8, 128, 1024), tc::pack_bf16x8(m));
+                    st16(smem + OFF_M + tc::off_sw128(i, q * 8, 8192), tc::pack_bf16x8(m));
                 }
             }
         }
         for (int i = tid; i < kQ * (kN / 8); i += kThreads) {
             const int r = i / (kN / 8), q = i % (kN / 8);
-            const uint32_t off = tc::off_kmajor(r, q * 8, 128, 2048);
+            const uint32_t off = tc::off_sw128(r, q * 8, 8192);
             float v[8];
             tc::unpack_bf16x8(ld16(smem + OFF_C + off), v);
             const float fc = ax.ecs[r];
@@ -350,12 +336,12 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             for (int e = 0; e < 8; ++e) v[e] *= fb;
             st16(smem + OFF_B + off, tc::pack_bf16x8(v));
         }
-        // z of this chunk's rows, in flight while the tensor cores run
-        uint4 zr[8];
-        const int yi = warp * 16 + lane;
+        // z of this chunk's rows (this warp's 32 columns), in flight while the tensor cores run
+        uint4 zr[4];
+        const int yi = q4 * 16 + lane;
         const bool yrow = lane < 16 && yi < nv;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) zr[q] = (zg && yrow) ? ld16(zg + (t0 + yi) * a.z_ts + q * 8) : zero4;
+        for (int q = 0; q < 4; ++q) zr[q] = (zg && yrow) ? ld16(zg + (t0 + yi) * a.z_ts + half * 32 + q * 8) : zero4;
         tc::fence_before_sync();
         tc::fence_proxy_async();
         __syncthreads();
@@ -365,16 +351,16 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             tc::fence_after_sync();
 #pragma unroll
             for (int k = 0; k < kQ / 16; ++k)
-                tc::mma_bf16(tmem + 64, tc::desc(sbase + OFF_M + k * 256, 128, 1024),
-                             tc::desc(sbase + OFF_X + k * 2048, 1024, 128), ID_Y, k > 0);
+                tc::mma_bf16(tmem + 64, tc::desc_sw128(sbase + OFF_M + k * 32, 16, 1024),
+                             tc::desc_sw128(sbase + OFF_X + k * 2048, 8192, 1024), ID_Y, k > 0);
 #pragma unroll
             for (int k = 0; k < kN / 16; ++k)
-                tc::mma_bf16(tmem + 64, tc::desc(sbase + OFF_C + k * 256, 128, 2048),
-                             tc::desc(sbase + OFF_S + k * 2048, 1024, 128), ID_Y, 1);
+                tc::mma_bf16(tmem + 64, tc::desc_sw128(sbase + OFF_C + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024),
+                             tc::desc_sw128(sbase + OFF_S + k * 2048, 8192, 1024), ID_Y, 1);
 #pragma unroll
             for (int k = 0; k < kQ / 16; ++k)
-                tc::mma_bf16(tmem, tc::desc(sbase + OFF_B + k * 4096, 2048, 128),
-                             tc::desc(sbase + OFF_X + k * 2048, 1024, 128), ID_S, k > 0);
+                tc::mma_bf16(tmem, tc::desc_sw128(sbase + OFF_B + k * 2048, 8192, 1024),
+                             tc::desc_sw128(sbase + OFF_X + k * 2048, 8192, 1024), ID_S, k > 0);
             tc::mma_commit(&ax.mbar[1]);
         }
         ok = __syncthreads_and(tc::mbar_wait(&ax.mbar[1], c & 1));
@@ -386,9 +372,8 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             if (warp == 0) load_dt(c + 1);
         }
 
-        // ---- (5) y = (Y + D x) * silu(z); S = exp(cs_Q) S + Sc
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {                   // 32 columns at a time keeps registers down
+        // ---- (5) y = (Y + D x) * silu(z) for this warp's 32 columns; S = exp(cs_Q) S + Sc
+        {
             float Yv[32];
             tc::tmem_ld32(tmem + t_lane + 64 + half * 32, Yv);
             if (yrow) {
@@ -396,8 +381,8 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
                 for (int qq = 0; qq < 4; ++qq) {
                     const int q = half * 4 + qq;
                     float xv[8], zv[8], o[8];
-                    tc::unpack_bf16x8(ld16(smem + OFF_X + tc::off_mnmajor(q * 8, yi, 1024, 128)), xv);
-                    tc::unpack_bf16x8(zr[q], zv);
+                    tc::unpack_bf16x8(ld16(smem + OFF_X + tc::off_sw128(yi, q * 8, 8192)), xv);
+                    tc::unpack_bf16x8(zr[qq], zv);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         float yv = fmaf(Dh, xv[e], Yv[qq * 8 + e]);
@@ -409,17 +394,13 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         }
         {
             const float dAc = ax.dAc;
-            const int n = tid;
+            float Sc[32];
+            tc::tmem_ld32(tmem + t_lane + half * 32, Sc);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float Sc[32];
-                tc::tmem_ld32(tmem + t_lane + half * 32, Sc);
+            for (int p = 0; p < 32; ++p) S[p] = fmaf(dAc, S[p], Sc[p]);
 #pragma unroll
-                for (int p = 0; p < 32; ++p) S[half * 32 + p] = fmaf(dAc, S[half * 32 + p], Sc[p]);
-            }
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                st16(smem + OFF_S + tc::off_mnmajor(q * 8, n, 1024, 128), tc::pack_bf16x8(&S[q * 8]));
+            for (int q = 0; q < 4; ++q)
+                st16(smem + OFF_S + tc::off_sw128(sn, half * 32 + q * 8, 8192), tc::pack_bf16x8(&S[q * 8]));
         }
         cp_async_wait_all();
         tc::fence_before_sync();
@@ -434,10 +415,9 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         tc::mbar_wait(&ax.mbar[fail_bar], fail_par, 1u << 20);
     } else {
         if (a.h_final) {
-            const int n = tid;
             float *hf = a.h_final + ((int64_t)s * H + hh) * kP * kN;
 #pragma unroll
-            for (int p = 0; p < kP; ++p) hf[(int64_t)p * kN + n] = S[p];
+            for (int p = 0; p < 32; ++p) hf[(int64_t)(half * 32 + p) * kN + sn] = S[p];
         }
         if (K > 1 && a.conv_state_out && tid < kP) {
             const int p = tid, hbf = nchunks & 1;

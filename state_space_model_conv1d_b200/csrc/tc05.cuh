@@ -24,6 +24,24 @@ SSM_DEVINL uint64_t desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
+// Same with the 128-byte swizzle (layout type 2); swizzle atoms must sit on
+// 1024-byte boundaries.
+SSM_DEVINL uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return desc(saddr, lbo, sbo) | (2ull << 61);
+}
+
+// 128-byte-swizzled layouts.  An atom is 8 rows of 128 bytes (64 bf16) with
+// the 16-byte chunk index XORed by the row index within the atom.
+//   K-major  (rows r, K contiguous, K-atoms of 64 at kstride bytes, SBO = 1024):
+//     off(r, k) = (k/64)*kstride + (r/8)*1024 + (r%8)*128 + (((k%64)/8) ^ (r%8))*16 + (k%8)*2
+//   MN-major (MN contiguous in 64-element atoms at LBO bytes, K rows, SBO = 1024):
+//     off(m, k) = (m/64)*LBO + (k/8)*1024 + (k%8)*128 + (((m%64)/8) ^ (k%8))*16 + (m%8)*2
+// A K-major tile with rows j and K = n is, byte for byte, the MN-major tile
+// with MN = n and K = j (LBO = the K-atom stride), so one copy serves both views.
+SSM_DEVINL uint32_t off_sw128(int row, int col, uint32_t atom_stride) {
+    return (uint32_t)(col >> 6) * atom_stride + (uint32_t)(row >> 3) * 1024u + (uint32_t)(row & 7) * 128u +
+           ((uint32_t)(((col & 63) >> 3) ^ (row & 7)) << 4) + (uint32_t)(col & 7) * 2u;
+}
 
 // Instruction descriptor for kind::f16 with bf16 A / B and an fp32 accumulator.
 // a_mn / b_mn: operand stored MN-major (1) or K-major (0).
