@@ -61,6 +61,9 @@ struct Aux {
     float cs2[kQ];                   // running log2-decay
     float ecs[kQ];                   // exp(cs_i)
     float wj[kQ];                    // exp(cs_Q - cs_j) * delta_j
+    float rf[kQ];                    // exp(cs_i - cs_{16*(i/16)}): row factor to the start of its block
+    float cf[kQ];                    // exp(cs_{16*(j/16)+15} - cs_j) * delta_j: column factor to the end of its block
+    float bf[4][4];                  // exp(cs_{16*I} - cs_{16*J+15}) for blocks J < I
     float dAc;                       // exp(cs_Q)
     uint32_t tmem;
     uint64_t mbar[2];
@@ -92,6 +95,8 @@ SSM_DEVINL void cp_async16(void *smem_dst, const void *gmem_src) {
 }
 SSM_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 SSM_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+template <int N>
+SSM_DEVINL void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
     extern __shared__ unsigned char smem_raw[];
@@ -182,9 +187,18 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
     // raw x rows (row-major [kQ][kP] bf16) into the M tile's space, which is
     // free from the end of MMA2 until the mask phase of the next chunk.
     // Asynchronous 16-byte copies; rows past the sequence end are zero-filled.
+    // Two copy groups: the raw x rows first (needed at the top of the chunk),
+    // then B and C (needed only by MMA1, after the conv).
     auto prefetch = [&](int cn) {
         const int64_t tn = (int64_t)cn * kQ;
         const int nvn = (int)min((int64_t)kQ, len - tn);
+        for (int i = tid; i < kQ * (kP / 8); i += kThreads) {
+            const int r = i / (kP / 8), q = i % (kP / 8);
+            unsigned char *dst = smem + OFF_M + r * (kP * 2) + q * 16;
+            if (r < nvn) cp_async16(dst, xg + (tn + r) * a.x_ts + q * 8);
+            else st16(dst, zero4);
+        }
+        cp_async_commit();
         for (int i = tid; i < kQ * (kN / 8); i += kThreads) {
             const int r = i / (kN / 8), q = i % (kN / 8);
             const uint32_t off = tc::off_sw128(r, q * 8, 8192);
@@ -195,12 +209,6 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
                 st16(smem + OFF_B + off, zero4);
                 st16(smem + OFF_C + off, zero4);
             }
-        }
-        for (int i = tid; i < kQ * (kP / 8); i += kThreads) {
-            const int r = i / (kP / 8), q = i % (kP / 8);
-            unsigned char *dst = smem + OFF_M + r * (kP * 2) + q * 16;
-            if (r < nvn) cp_async16(dst, xg + (tn + r) * a.x_ts + q * 8);
-            else st16(dst, zero4);
         }
         cp_async_commit();
     };
@@ -229,31 +237,7 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         const int nv = (int)min((int64_t)kQ, len - t0);
         const int hb = c & 1;
 
-        // ---- (1) delta and running decay (warp 0); x conv from the staged raw rows
-        if (warp == 0) {
-            float d0 = 0.f, d1 = 0.f;
-            const float u0 = __bfloat162float(dtr0) + dtb, u1 = __bfloat162float(dtr1) + dtb;
-            if (lane < nv) d0 = a.softplus ? softplus(u0) : u0;
-            if (lane + 32 < nv) d1 = a.softplus ? softplus(u1) : u1;
-            float s0 = d0 * A2, s1 = d1 * A2;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v0 = __shfl_up_sync(0xffffffffu, s0, o);
-                const float v1 = __shfl_up_sync(0xffffffffu, s1, o);
-                if (lane >= o) { s0 += v0; s1 += v1; }
-            }
-            s1 += __shfl_sync(0xffffffffu, s0, 31);
-            const float last = __shfl_sync(0xffffffffu, s1, 31);
-            ax.dlt[lane] = d0;
-            ax.dlt[lane + 32] = d1;
-            ax.cs2[lane] = s0;
-            ax.cs2[lane + 32] = s1;
-            ax.ecs[lane] = ex2(s0);
-            ax.ecs[lane + 32] = ex2(s1);
-            ax.wj[lane] = ex2(last - s0) * d0;
-            ax.wj[lane + 32] = ex2(last - s1) * d1;
-            if (lane == 0) ax.dAc = ex2(last);
-        }
+        // ---- (1) x conv from the staged raw rows
         {
             // conv + SiLU: thread -> channel cp, tokens cr0 .. cr0+15, sliding window in registers
             auto raw1 = [&](int v) -> float {
@@ -283,6 +267,7 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
                                              : ax.xh[hb][kHx + v][p];
             }
         }
+        cp_async_wait_all();                                          // B and C of this chunk
         tc::fence_proxy_async();
         __syncthreads();
 
@@ -297,6 +282,44 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             }
             tc::mma_commit(&ax.mbar[0]);
         }
+        // ---- delta and running decay (warp 0, while MMA1 runs), plus the mask factor tables
+        if (warp == 0) {
+            float d0 = 0.f, d1 = 0.f;
+            const float u0 = __bfloat162float(dtr0) + dtb, u1 = __bfloat162float(dtr1) + dtb;
+            if (lane < nv) d0 = a.softplus ? softplus(u0) : u0;
+            if (lane + 32 < nv) d1 = a.softplus ? softplus(u1) : u1;
+            float s0 = d0 * A2, s1 = d1 * A2;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v0 = __shfl_up_sync(0xffffffffu, s0, o);
+                const float v1 = __shfl_up_sync(0xffffffffu, s1, o);
+                if (lane >= o) { s0 += v0; s1 += v1; }
+            }
+            s1 += __shfl_sync(0xffffffffu, s0, 31);
+            const float last = __shfl_sync(0xffffffffu, s1, 31);
+            // block boundaries: token 16*(j/16) (start) and 16*(j/16)+15 (end)
+            const float st0 = __shfl_sync(0xffffffffu, s0, lane & ~15), st1 = __shfl_sync(0xffffffffu, s1, lane & ~15);
+            const float en0 = __shfl_sync(0xffffffffu, s0, lane | 15), en1 = __shfl_sync(0xffffffffu, s1, lane | 15);
+            ax.dlt[lane] = d0;
+            ax.dlt[lane + 32] = d1;
+            ax.cs2[lane] = s0;
+            ax.cs2[lane + 32] = s1;
+            ax.ecs[lane] = ex2(s0);
+            ax.ecs[lane + 32] = ex2(s1);
+            ax.wj[lane] = ex2(last - s0) * d0;
+            ax.wj[lane + 32] = ex2(last - s1) * d1;
+            ax.rf[lane] = ex2(s0 - st0);
+            ax.rf[lane + 32] = ex2(s1 - st1);
+            ax.cf[lane] = ex2(en0 - s0) * d0;
+            ax.cf[lane + 32] = ex2(en1 - s1) * d1;
+            __syncwarp();
+            if (lane < 16) {
+                // block factor (I, J), J < I: exp(cs[16 I] - cs[16 J + 15]) (<= 1)
+                const int I = lane >> 2, J = lane & 3;
+                ax.bf[I][J] = J < I ? ex2(ax.cs2[16 * I] - ax.cs2[16 * J + 15]) : 0.f;
+            }
+            if (lane == 0) ax.dAc = ex2(last);
+        }
         ok = __syncthreads_and(tc::mbar_wait(&ax.mbar[0], c & 1));
         if (!ok) { fail_bar = 0; fail_par = c & 1; break; }
         tc::fence_after_sync();
@@ -306,18 +329,32 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             float Gv[32];
             tc::tmem_ld32(tmem + t_lane + half * 32, Gv);
             if (lane < 16) {
-                const int i = q4 * 16 + lane;
-                const float ci = ax.cs2[i];
+                // M[i, j] = G[i, j] exp(cs_i - cs_j) delta_j for j <= i, plus D on the diagonal
+                // (the skip term D x rides along in M X).  Below the diagonal 16x16 block the
+                // exponential factors as row x block x column terms, each <= 1.
+                const int i = q4 * 16 + lane, I = q4;
+                const float ci = ax.cs2[i], ri = ax.rf[i];
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const int q = half * 4 + qq;
-                    float m[8];
+                for (int jb = 0; jb < 2; ++jb) {                       // the two 16-column blocks of this half
+                    const int J = half * 2 + jb;
+                    float m[16];
+                    if (J < I) {
+                        const float f = ri * ax.bf[I][J];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = q * 8 + e;
-                        m[e] = j <= i ? Gv[qq * 8 + e] * ex2(ci - ax.cs2[j]) * ax.dlt[j] : 0.f;
+                        for (int e = 0; e < 16; ++e) m[e] = Gv[jb * 16 + e] * f * ax.cf[J * 16 + e];
+                    } else if (J == I) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const int j = J * 16 + e;
+                            m[e] = j <= i ? Gv[jb * 16 + e] * ex2(ci - ax.cs2[j]) * ax.dlt[j] : 0.f;
+                            if (j == i) m[e] += Dh;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) m[e] = 0.f;
                     }
-                    st16(smem + OFF_M + tc::off_sw128(i, q * 8, 8192), tc::pack_bf16x8(m));
+                    st16(smem + OFF_M + tc::off_sw128(i, J * 16, 8192), tc::pack_bf16x8(m));
+                    st16(smem + OFF_M + tc::off_sw128(i, J * 16 + 8, 8192), tc::pack_bf16x8(m + 8));
                 }
             }
         }
@@ -372,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             if (warp == 0) load_dt(c + 1);
         }
 
-        // ---- (5) y = (Y + D x) * silu(z) for this warp's 32 columns; S = exp(cs_Q) S + Sc
+        // ---- (5) y = Y * silu(z) for this warp's 32 columns (D x is already in Y); S = exp(cs_Q) S + Sc
         {
             float Yv[32];
             tc::tmem_ld32(tmem + t_lane + 64 + half * 32, Yv);
@@ -380,12 +417,11 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
                     const int q = half * 4 + qq;
-                    float xv[8], zv[8], o[8];
-                    tc::unpack_bf16x8(ld16(smem + OFF_X + tc::off_sw128(yi, q * 8, 8192)), xv);
+                    float zv[8], o[8];
                     tc::unpack_bf16x8(zr[qq], zv);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        float yv = fmaf(Dh, xv[e], Yv[qq * 8 + e]);
+                        const float yv = Yv[qq * 8 + e];
                         o[e] = zg ? yv * silu_fast<__nv_bfloat16>(zv[e]) : yv;
                     }
                     st16(yg + (t0 + yi) * a.y_ts + q * 8, tc::pack_bf16x8(o));
@@ -402,11 +438,12 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             for (int q = 0; q < 4; ++q)
                 st16(smem + OFF_S + tc::off_sw128(sn, half * 32 + q * 8, 8192), tc::pack_bf16x8(&S[q * 8]));
         }
-        cp_async_wait_all();
+        cp_async_wait_group<1>();                                     // next chunk's raw x rows (B, C may still fly)
         tc::fence_before_sync();
         tc::fence_proxy_async();
         __syncthreads();
     }
+    cp_async_wait_all();
 
     if (!ok) {
         // a tensor-core completion never arrived: record it, give the MMAs a
