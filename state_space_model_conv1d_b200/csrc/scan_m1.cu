@@ -278,10 +278,10 @@ scan_m1_kernel(const M1Args a) {
     auto scan = [&](int c) {
         const int wb = c & 1;
 #pragma unroll
-        for (int t4 = 0; t4 < kTC; t4 += 4) {
-            float acc[4];
+        for (int t4 = 0; t4 < kTC; t4 += kLanes) {
+            float acc[kLanes];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < kLanes; ++i) {
                 const int t = t4 + i;
                 const float2 dd = sm.dd[wb][t][sd];                  // (delta, delta * xc)
                 if constexpr (VW >= 2) {
@@ -323,14 +323,20 @@ scan_m1_kernel(const M1Args a) {
                     acc[i] = ac;
                 }
             }
-            // reduce-scatter over the 4 lanes of the channel: lane q ends with token t4 + q
-            const bool hi = (q & 2) != 0;
-            const float s0 = hi ? acc[0] : acc[2], s1 = hi ? acc[1] : acc[3];
-            const float k0 = hi ? acc[2] : acc[0], k1 = hi ? acc[3] : acc[1];
-            const float r0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 2);
-            const float r1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 2);
-            const bool odd = (q & 1) != 0;
-            const float tot = (odd ? r1 : r0) + __shfl_xor_sync(0xffffffffu, odd ? r0 : r1, 1);
+            // reduce-scatter over the lanes of the channel: at each level a lane keeps
+            // half of its partial sums (upper half when its bit is set) and adds the
+            // partner's copy of that half; lane q ends with the sum of token t4 + q
+#pragma unroll
+            for (int o = kLanes / 2; o >= 1; o >>= 1) {
+                const bool up = (q & o) != 0;
+#pragma unroll
+                for (int k = 0; k < o; ++k) {
+                    const float keep = up ? acc[o + k] : acc[k];
+                    const float send = up ? acc[k] : acc[o + k];
+                    acc[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                }
+            }
+            const float tot = acc[0];
             const int t = t4 + q;
             const float2 e2 = sm.ep[wb][t][sd];                      // (D * xc, gate)
             sm.y[wb][t][sd] = (tot + e2.x) * e2.y;
@@ -411,11 +417,11 @@ cudaError_t launch_typed(M1Args a, int nseqs, cudaStream_t st) {
     // B / C rows go through 16-byte copies only when dstate fills whole vectors
     // and the padded row (4 * SPT elements) keeps every row 16-byte aligned.
     auto bc_ok = [&](int np) { return a.async_bc && a.N % E == 0 && (np * (int)sizeof(T)) % 16 == 0; };
-    if (a.N <= 4) { a.async_bc = bc_ok(4); return launch_spt<T, 1>(a, nseqs, st); }
-    if (a.N <= 8) { a.async_bc = bc_ok(8); return launch_spt<T, 2>(a, nseqs, st); }
-    if (a.N <= 16) { a.async_bc = bc_ok(16); return launch_spt<T, 4>(a, nseqs, st); }
-    if (a.N <= 32) { a.async_bc = bc_ok(32); return launch_spt<T, 8>(a, nseqs, st); }
-    a.async_bc = bc_ok(64);
+    if (a.N <= kLanes * 1) { a.async_bc = bc_ok(kLanes * 1); return launch_spt<T, 1>(a, nseqs, st); }
+    if (a.N <= kLanes * 2) { a.async_bc = bc_ok(kLanes * 2); return launch_spt<T, 2>(a, nseqs, st); }
+    if (a.N <= kLanes * 4) { a.async_bc = bc_ok(kLanes * 4); return launch_spt<T, 4>(a, nseqs, st); }
+    if (a.N <= kLanes * 8) { a.async_bc = bc_ok(kLanes * 8); return launch_spt<T, 8>(a, nseqs, st); }
+    a.async_bc = bc_ok(kLanes * 16);
     return launch_spt<T, 16>(a, nseqs, st);
 }
 
