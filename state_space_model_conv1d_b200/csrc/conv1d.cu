@@ -71,6 +71,48 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
         }
     };
     load_hist(t0);
+    if (!cu || t1 <= end) {
+        // the whole run lies in one sequence: issue every row's load before any math
+        float cur[kTokensPerThread][VEC];
+#pragma unroll
+        for (int i = 0; i < kTokensPerThread; ++i) {
+            if (t0 + i < t1) {
+                if constexpr (VEC == 8) {
+                    Vec8<T>::ld(xr + (t0 + i) * x_ts + c0, cur[i]);
+                } else {
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) cur[i][v] = Elem<T>::ld(xr + (t0 + i) * x_ts + c0 + v);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kTokensPerThread; ++i) {
+            if (t0 + i >= t1) break;
+            float o[VEC];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                float acc = bb[v];
+#pragma unroll
+                for (int k = 0; k < K - 1; ++k) acc = fmaf(wk[k][v], hist[k][v], acc);
+                acc = fmaf(wk[K - 1][v], cur[i][v], acc);
+                o[v] = act ? silu(acc) : acc;
+            }
+            if constexpr (VEC == 8) {
+                Vec8<T>::st(orow + (t0 + i) * o_ts + c0, o);
+            } else {
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) Elem<T>::st(orow + (t0 + i) * o_ts + c0 + v, o[v]);
+            }
+#pragma unroll
+            for (int k = 0; k + 1 < K - 1; ++k)
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) hist[k][v] = hist[k + 1][v];
+            if (K > 1)
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) hist[K > 1 ? K - 2 : 0][v] = cur[i][v];
+        }
+        return;
+    }
     for (int64_t t = t0; t < t1; ++t) {
         if (cu && t >= end) {                      // next (non-empty) sequence of the packed row
             while (s + 1 < nseqs && cu[s + 1] <= t) ++s;

@@ -137,15 +137,18 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
     const float A2 = a.A[hh] * kLog2e;
     const float Dh = a.D ? a.D[hh] : 0.f;
     const float dtb = a.dt_bias ? a.dt_bias[hh] : 0.f;
-    // x conv role: channel cp = tid % 64, tokens cr0 .. cr0+15; taps right-aligned
-    // (cw3 multiplies the current token, cw0 the one 3 back)
-    const int cp = tid & (kP - 1), cr0 = (tid / kP) * (kQ / 4);
-    float cw0, cw1, cw2, cw3, cbias;
+    // x conv role: channels 2 cq, 2 cq + 1 (one packed pair), tokens cr0 .. cr0+7;
+    // taps right-aligned (cw3 multiplies the current token, cw0 the one 3 back)
+    const int cq = tid & 31, cr0 = warp * (kQ / 8);
+    float2 cw0, cw1, cw2, cw3, cbias;
     {
-        const int64_t ch = hh * kP + cp;
-        auto tap = [&](int j) { const int k = K - 4 + j; return (K > 0 && k >= 0) ? a.conv_w[ch * K + k] : 0.f; };
+        const int64_t ch = hh * kP + 2 * cq;
+        auto tap = [&](int j) {
+            const int k = K - 4 + j;
+            return (K > 0 && k >= 0) ? make_float2(a.conv_w[ch * K + k], a.conv_w[(ch + 1) * K + k]) : make_float2(0.f, 0.f);
+        };
         cw0 = tap(0); cw1 = tap(1); cw2 = tap(2); cw3 = tap(3);
-        cbias = a.conv_b ? a.conv_b[ch] : 0.f;
+        cbias = a.conv_b ? make_float2(a.conv_b[ch], a.conv_b[ch + 1]) : make_float2(0.f, 0.f);
     }
 
     // ---- carried state: thread owns S[n][32*half .. 32*half+31] for n = 32*q4 + lane (fp32)
@@ -239,21 +242,33 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
 
         // ---- (1) x conv from the staged raw rows
         {
-            // conv + SiLU: thread -> channel cp, tokens cr0 .. cr0+15, sliding window in registers
-            auto raw1 = [&](int v) -> float {
-                return v < 0 ? ax.xh[hb][kHx + v][cp]
-                             : __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(xraw + v * (kP * 2) + cp * 2));
+            // conv + SiLU of a channel pair over 8 tokens, sliding window in registers,
+            // packed fp32x2 arithmetic, one 4-byte store per token into the X tile
+            auto raw2 = [&](int v) -> float2 {
+                if (v < 0) return make_float2(ax.xh[hb][kHx + v][2 * cq], ax.xh[hb][kHx + v][2 * cq + 1]);
+                const uint32_t u = *reinterpret_cast<const uint32_t *>(xraw + v * (kP * 2) + cq * 4);
+                return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
             };
-            float h0v = raw1(cr0 - 3), h1v = raw1(cr0 - 2), h2v = raw1(cr0 - 1);   // raw rows t-3, t-2, t-1
+            float2 h0v = raw2(cr0 - 3), h1v = raw2(cr0 - 2), h2v = raw2(cr0 - 1);   // raw rows t-3, t-2, t-1
+            const float2 half2 = make_float2(0.5f, 0.5f);
 #pragma unroll
-            for (int i = 0; i < kQ / 4; ++i) {
+            for (int i = 0; i < kQ / 8; ++i) {
                 const int r = cr0 + i;
-                const float cur = raw1(r);                            // rows >= nv are zeros
-                float acc = cur;
-                if (K > 0) acc = silu_fast<__nv_bfloat16>(fmaf(cw0, h0v, fmaf(cw1, h1v, fmaf(cw2, h2v, fmaf(cw3, cur, cbias)))));
-                if (r >= nv) acc = 0.f;
+                const float2 cur = raw2(r);                           // rows >= nv are zeros
+                float2 xc = cur;
+                if (K > 0) {
+                    float2 acc = __ffma2_rn(cw3, cur, cbias);
+                    acc = __ffma2_rn(cw2, h2v, acc);
+                    acc = __ffma2_rn(cw1, h1v, acc);
+                    acc = __ffma2_rn(cw0, h0v, acc);
+                    // silu(v) = h + h tanh(h), h = v / 2
+                    const float2 hv = __fmul2_rn(acc, half2);
+                    xc = __ffma2_rn(hv, make_float2(tanh_approx(hv.x), tanh_approx(hv.y)), hv);
+                }
+                if (r >= nv) xc = make_float2(0.f, 0.f);
                 h0v = h1v; h1v = h2v; h2v = cur;
-                *reinterpret_cast<__nv_bfloat16 *>(smem + OFF_X + tc::off_sw128(r, cp, 8192)) = __float2bfloat16_rn(acc);
+                const __nv_bfloat162 b = __floats2bfloat162_rn(xc.x, xc.y);
+                *reinterpret_cast<__nv_bfloat162 *>(smem + OFF_X + tc::off_sw128(r, 2 * cq, 8192)) = b;
             }
         }
         // halo of the next chunk: raw rows nv-3 .. nv-1 (from the old halo when the chunk is shorter)
@@ -325,60 +340,71 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         tc::fence_after_sync();
 
         // ---- (3) mask G -> M (over the staged raw rows, already consumed); rescale C -> C', B -> B'
+        // Each warp reads its 16 accumulator rows (tokens i0 = 16 q4 + lane / 4 and
+        // i1 = i0 + 8) for its 32 columns, spread over all 32 threads.
+        const int i0 = q4 * 16 + (lane >> 2), i1 = i0 + 8;
+        const int jc = half * 32 + 2 * (lane & 3);                   // first column of pair k: jc + 8 k
         {
-            float Gv[32];
-            tc::tmem_ld32(tmem + t_lane + half * 32, Gv);
-            if (lane < 16) {
-                // M[i, j] = G[i, j] exp(cs_i - cs_j) delta_j for j <= i, plus D on the diagonal
-                // (the skip term D x rides along in M X).  Below the diagonal 16x16 block the
-                // exponential factors as row x block x column terms, each <= 1.
-                const int i = q4 * 16 + lane, I = q4;
-                const float ci = ax.cs2[i], ri = ax.rf[i];
+            uint32_t gr[16];
+            tc::tmem_ld16x256b_x4(tmem + t_lane + half * 32, gr);
+            const int I = q4;
+            const float ci0 = ax.cs2[i0], ci1 = ax.cs2[i1];
+            const float rf0 = ax.rf[i0], rf1 = ax.rf[i1];
+            tc::tmem_wait_ld();
+            // M[i, j] = G[i, j] exp(cs_i - cs_j) delta_j for j <= i, plus D on the diagonal
+            // (the skip term D x rides along in M X).  Below the diagonal 16x16 block the
+            // exponential factors as row x block x column terms, each <= 1.
 #pragma unroll
-                for (int jb = 0; jb < 2; ++jb) {                       // the two 16-column blocks of this half
-                    const int J = half * 2 + jb;
-                    float m[16];
-                    if (J < I) {
-                        const float f = ri * ax.bf[I][J];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) m[e] = Gv[jb * 16 + e] * f * ax.cf[J * 16 + e];
-                    } else if (J == I) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const int j = J * 16 + e;
-                            m[e] = j <= i ? Gv[jb * 16 + e] * ex2(ci - ax.cs2[j]) * ax.dlt[j] : 0.f;
-                            if (j == i) m[e] += Dh;
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) m[e] = 0.f;
-                    }
-                    st16(smem + OFF_M + tc::off_sw128(i, J * 16, 8192), tc::pack_bf16x8(m));
-                    st16(smem + OFF_M + tc::off_sw128(i, J * 16 + 8, 8192), tc::pack_bf16x8(m + 8));
+            for (int k = 0; k < 4; ++k) {
+                const int J = half * 2 + (k >> 1);                    // 16-column block (warp-uniform)
+                const int j = jc + 8 * k;
+                float m00 = 0.f, m01 = 0.f, m10 = 0.f, m11 = 0.f;     // (i0, j), (i0, j+1), (i1, j), (i1, j+1)
+                const float g00 = __uint_as_float(gr[4 * k]), g01 = __uint_as_float(gr[4 * k + 1]);
+                const float g10 = __uint_as_float(gr[4 * k + 2]), g11 = __uint_as_float(gr[4 * k + 3]);
+                if (J < I) {
+                    const float bfac = ax.bf[I][J];
+                    const float c0 = ax.cf[j] * bfac, c1 = ax.cf[j + 1] * bfac;
+                    m00 = g00 * rf0 * c0; m01 = g01 * rf0 * c1;
+                    m10 = g10 * rf1 * c0; m11 = g11 * rf1 * c1;
+                } else if (J == I) {
+                    const float cj0 = ax.cs2[j], cj1 = ax.cs2[j + 1];
+                    const float d0 = ax.dlt[j], d1 = ax.dlt[j + 1];
+                    m00 = j <= i0 ? g00 * ex2(ci0 - cj0) * d0 : 0.f;
+                    m01 = j + 1 <= i0 ? g01 * ex2(ci0 - cj1) * d1 : 0.f;
+                    m10 = j <= i1 ? g10 * ex2(ci1 - cj0) * d0 : 0.f;
+                    m11 = j + 1 <= i1 ? g11 * ex2(ci1 - cj1) * d1 : 0.f;
+                    if (j == i0) m00 += Dh;
+                    if (j + 1 == i0) m01 += Dh;
+                    if (j == i1) m10 += Dh;
+                    if (j + 1 == i1) m11 += Dh;
                 }
+                *reinterpret_cast<__nv_bfloat162 *>(smem + OFF_M + tc::off_sw128(i0, j, 8192)) = __floats2bfloat162_rn(m00, m01);
+                *reinterpret_cast<__nv_bfloat162 *>(smem + OFF_M + tc::off_sw128(i1, j, 8192)) = __floats2bfloat162_rn(m10, m11);
             }
         }
+        // C'[i] = exp(cs_i) C[i], B'[j] = exp(cs_Q - cs_j) delta_j B[j]: packed bf16 products
         for (int i = tid; i < kQ * (kN / 8); i += kThreads) {
             const int r = i / (kN / 8), q = i % (kN / 8);
             const uint32_t off = tc::off_sw128(r, q * 8, 8192);
-            float v[8];
-            tc::unpack_bf16x8(ld16(smem + OFF_C + off), v);
-            const float fc = ax.ecs[r];
+            const __nv_bfloat162 fc = __float2bfloat162_rn(ax.ecs[r]), fb = __float2bfloat162_rn(ax.wj[r]);
+            uint4 vc = ld16(smem + OFF_C + off), vb = ld16(smem + OFF_B + off);
+            __nv_bfloat162 *pc = reinterpret_cast<__nv_bfloat162 *>(&vc), *pb = reinterpret_cast<__nv_bfloat162 *>(&vb);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] *= fc;
-            st16(smem + OFF_C + off, tc::pack_bf16x8(v));
-            tc::unpack_bf16x8(ld16(smem + OFF_B + off), v);
-            const float fb = ax.wj[r];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] *= fb;
-            st16(smem + OFF_B + off, tc::pack_bf16x8(v));
+            for (int e = 0; e < 4; ++e) {
+                pc[e] = __hmul2(pc[e], fc);
+                pb[e] = __hmul2(pb[e], fb);
+            }
+            st16(smem + OFF_C + off, vc);
+            st16(smem + OFF_B + off, vb);
         }
-        // z of this chunk's rows (this warp's 32 columns), in flight while the tensor cores run
-        uint4 zr[4];
-        const int yi = q4 * 16 + lane;
-        const bool yrow = lane < 16 && yi < nv;
+        // z of this thread's accumulator positions, in flight while the tensor cores run
+        uint32_t zr[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) zr[q] = (zg && yrow) ? ld16(zg + (t0 + yi) * a.z_ts + half * 32 + q * 8) : zero4;
+        for (int k = 0; k < 4; ++k) {
+            const int p = jc + 8 * k;
+            zr[2 * k] = (zg && i0 < nv) ? *reinterpret_cast<const uint32_t *>(zg + (t0 + i0) * a.z_ts + p) : 0u;
+            zr[2 * k + 1] = (zg && i1 < nv) ? *reinterpret_cast<const uint32_t *>(zg + (t0 + i1) * a.z_ts + p) : 0u;
+        }
         tc::fence_before_sync();
         tc::fence_proxy_async();
         __syncthreads();
@@ -409,22 +435,24 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             if (warp == 0) load_dt(c + 1);
         }
 
-        // ---- (5) y = Y * silu(z) for this warp's 32 columns (D x is already in Y); S = exp(cs_Q) S + Sc
+        // ---- (5) y = Y * silu(z) for this thread's 16 positions (D x is already in Y); S = exp(cs_Q) S + Sc
         {
-            float Yv[32];
-            tc::tmem_ld32(tmem + t_lane + 64 + half * 32, Yv);
-            if (yrow) {
+            uint32_t yr[16];
+            tc::tmem_ld16x256b_x4(tmem + t_lane + 64 + half * 32, yr);
+            tc::tmem_wait_ld();
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const int q = half * 4 + qq;
-                    float zv[8], o[8];
-                    tc::unpack_bf16x8(zr[qq], zv);
+            for (int k = 0; k < 4; ++k) {
+                const int p = jc + 8 * k;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float yv = Yv[qq * 8 + e];
-                        o[e] = zg ? yv * silu_fast<__nv_bfloat16>(zv[e]) : yv;
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int i = rr ? i1 : i0;
+                    float o0 = __uint_as_float(yr[4 * k + 2 * rr]), o1 = __uint_as_float(yr[4 * k + 2 * rr + 1]);
+                    if (zg) {
+                        const uint32_t zw = zr[2 * k + rr];
+                        o0 *= silu_fast<__nv_bfloat16>(__uint_as_float(zw << 16));
+                        o1 *= silu_fast<__nv_bfloat16>(__uint_as_float(zw & 0xffff0000u));
                     }
-                    st16(yg + (t0 + yi) * a.y_ts + q * 8, tc::pack_bf16x8(o));
+                    if (i < nv) *reinterpret_cast<__nv_bfloat162 *>(yg + (t0 + i) * a.y_ts + p) = __floats2bfloat162_rn(o0, o1);
                 }
             }
         }

@@ -143,6 +143,22 @@ SSM_DEVINL void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 16 lanes x 32 columns of an M = 64 accumulator (whose rows sit in lanes
+// 0-15 of each 32-lane quarter), spread over all 32 threads of the warp: for
+// thread T and column group k (8 columns each), v[4k + e] holds
+//   e = 0, 1: lane T/4,     columns 8k + 2 (T % 4) + e
+//   e = 2, 3: lane T/4 + 8, columns 8k + 2 (T % 4) + (e - 2)
+// relative to taddr.  Issues the load only; tmem_wait_ld() completes it.
+SSM_DEVINL void tmem_ld16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+SSM_DEVINL void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+
 // Byte offsets inside the core-matrix layouts above.
 SSM_DEVINL uint32_t off_kmajor(int r, int k, uint32_t lbo, uint32_t sbo) {
     return (uint32_t)(r >> 3) * sbo + (uint32_t)(k >> 3) * lbo + (uint32_t)(r & 7) * 16u + (uint32_t)(k & 7) * 2u;
