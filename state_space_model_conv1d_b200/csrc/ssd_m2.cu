@@ -55,8 +55,8 @@ constexpr uint32_t OFF_X = 40960;    // X rows j, 64 p each: MN-major MN = p, K 
 constexpr uint32_t OFF_S = 49152;    // S rows n, 64 p each: MN-major MN = p, K = n (MMA3)
 constexpr uint32_t OFF_AUX = 65536;
 
-struct Aux {
-    float xh[2][kHx][kP];            // raw x rows before the chunk (double buffered)
+// per-chunk decay tables, written by warp 0 one chunk ahead (double buffered by chunk parity)
+struct Tables {
     float dlt[kQ];                   // delta
     float cs2[kQ];                   // running log2-decay
     float ecs[kQ];                   // exp(cs_i)
@@ -65,6 +65,10 @@ struct Aux {
     float cf[kQ];                    // exp(cs_{16*(j/16)+15} - cs_j) * delta_j: column factor to the end of its block
     float bf[4][4];                  // exp(cs_{16*I} - cs_{16*J+15}) for blocks J < I
     float dAc;                       // exp(cs_Q)
+};
+struct Aux {
+    float xh[2][kHx][kP];            // raw x rows before the chunk (double buffered)
+    Tables tab[2];
     uint32_t tmem;
     uint64_t mbar[2];
 };
@@ -226,9 +230,54 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         if (lane < nvn) dtr0 = dtg[(tn + lane) * a.dt_ts];
         if (lane + 32 < nvn) dtr1 = dtg[(tn + lane + 32) * a.dt_ts];
     };
+    // delta, running log2-decay and the mask factor tables of chunk cn (warp 0),
+    // from the raw dt loaded by load_dt(cn), into table slot cn % 2
+    auto dt_tables = [&](int cn) {
+        Tables &tw = ax.tab[cn & 1];
+        const int nvn = (int)min((int64_t)kQ, len - (int64_t)cn * kQ);
+        float d0 = 0.f, d1 = 0.f;
+        const float u0 = __bfloat162float(dtr0) + dtb, u1 = __bfloat162float(dtr1) + dtb;
+        if (lane < nvn) d0 = a.softplus ? softplus(u0) : u0;
+        if (lane + 32 < nvn) d1 = a.softplus ? softplus(u1) : u1;
+        float s0 = d0 * A2, s1 = d1 * A2;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float v0 = __shfl_up_sync(0xffffffffu, s0, o);
+            const float v1 = __shfl_up_sync(0xffffffffu, s1, o);
+            if (lane >= o) { s0 += v0; s1 += v1; }
+        }
+        s1 += __shfl_sync(0xffffffffu, s0, 31);
+        const float last = __shfl_sync(0xffffffffu, s1, 31);
+        // block boundaries: token 16*(j/16) (start) and 16*(j/16)+15 (end)
+        const float st0 = __shfl_sync(0xffffffffu, s0, lane & ~15), st1 = __shfl_sync(0xffffffffu, s1, lane & ~15);
+        const float en0 = __shfl_sync(0xffffffffu, s0, lane | 15), en1 = __shfl_sync(0xffffffffu, s1, lane | 15);
+        tw.dlt[lane] = d0;
+        tw.dlt[lane + 32] = d1;
+        tw.cs2[lane] = s0;
+        tw.cs2[lane + 32] = s1;
+        tw.ecs[lane] = ex2(s0);
+        tw.ecs[lane + 32] = ex2(s1);
+        tw.wj[lane] = ex2(last - s0) * d0;
+        tw.wj[lane + 32] = ex2(last - s1) * d1;
+        tw.rf[lane] = ex2(s0 - st0);
+        tw.rf[lane + 32] = ex2(s1 - st1);
+        tw.cf[lane] = ex2(en0 - s0) * d0;
+        tw.cf[lane + 32] = ex2(en1 - s1) * d1;
+        __syncwarp();
+        if (lane < 16) {
+            // block factor (I, J), J < I: exp(cs[16 I] - cs[16 J + 15]) (<= 1)
+            const int I = lane >> 2, J = lane & 3;
+            tw.bf[I][J] = J < I ? ex2(tw.cs2[16 * I] - tw.cs2[16 * J + 15]) : 0.f;
+        }
+        if (lane == 0) tw.dAc = ex2(last);
+    };
     if (nchunks > 0) {
         prefetch(0);
-        if (warp == 0) load_dt(0);
+        if (warp == 0) {
+            load_dt(0);
+            dt_tables(0);
+            if (nchunks > 1) load_dt(1);
+        }
         cp_async_wait_all();
         tc::fence_proxy_async();
         __syncthreads();
@@ -297,44 +346,6 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             }
             tc::mma_commit(&ax.mbar[0]);
         }
-        // ---- delta and running decay (warp 0, while MMA1 runs), plus the mask factor tables
-        if (warp == 0) {
-            float d0 = 0.f, d1 = 0.f;
-            const float u0 = __bfloat162float(dtr0) + dtb, u1 = __bfloat162float(dtr1) + dtb;
-            if (lane < nv) d0 = a.softplus ? softplus(u0) : u0;
-            if (lane + 32 < nv) d1 = a.softplus ? softplus(u1) : u1;
-            float s0 = d0 * A2, s1 = d1 * A2;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v0 = __shfl_up_sync(0xffffffffu, s0, o);
-                const float v1 = __shfl_up_sync(0xffffffffu, s1, o);
-                if (lane >= o) { s0 += v0; s1 += v1; }
-            }
-            s1 += __shfl_sync(0xffffffffu, s0, 31);
-            const float last = __shfl_sync(0xffffffffu, s1, 31);
-            // block boundaries: token 16*(j/16) (start) and 16*(j/16)+15 (end)
-            const float st0 = __shfl_sync(0xffffffffu, s0, lane & ~15), st1 = __shfl_sync(0xffffffffu, s1, lane & ~15);
-            const float en0 = __shfl_sync(0xffffffffu, s0, lane | 15), en1 = __shfl_sync(0xffffffffu, s1, lane | 15);
-            ax.dlt[lane] = d0;
-            ax.dlt[lane + 32] = d1;
-            ax.cs2[lane] = s0;
-            ax.cs2[lane + 32] = s1;
-            ax.ecs[lane] = ex2(s0);
-            ax.ecs[lane + 32] = ex2(s1);
-            ax.wj[lane] = ex2(last - s0) * d0;
-            ax.wj[lane + 32] = ex2(last - s1) * d1;
-            ax.rf[lane] = ex2(s0 - st0);
-            ax.rf[lane + 32] = ex2(s1 - st1);
-            ax.cf[lane] = ex2(en0 - s0) * d0;
-            ax.cf[lane + 32] = ex2(en1 - s1) * d1;
-            __syncwarp();
-            if (lane < 16) {
-                // block factor (I, J), J < I: exp(cs[16 I] - cs[16 J + 15]) (<= 1)
-                const int I = lane >> 2, J = lane & 3;
-                ax.bf[I][J] = J < I ? ex2(ax.cs2[16 * I] - ax.cs2[16 * J + 15]) : 0.f;
-            }
-            if (lane == 0) ax.dAc = ex2(last);
-        }
         ok = __syncthreads_and(tc::mbar_wait(&ax.mbar[0], c & 1));
         if (!ok) { fail_bar = 0; fail_par = c & 1; break; }
         tc::fence_after_sync();
@@ -342,14 +353,15 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         // ---- (3) mask G -> M (over the staged raw rows, already consumed); rescale C -> C', B -> B'
         // Each warp reads its 16 accumulator rows (tokens i0 = 16 q4 + lane / 4 and
         // i1 = i0 + 8) for its 32 columns, spread over all 32 threads.
+        const Tables &tb = ax.tab[c & 1];
         const int i0 = q4 * 16 + (lane >> 2), i1 = i0 + 8;
         const int jc = half * 32 + 2 * (lane & 3);                   // first column of pair k: jc + 8 k
         {
             uint32_t gr[16];
             tc::tmem_ld16x256b_x4(tmem + t_lane + half * 32, gr);
             const int I = q4;
-            const float ci0 = ax.cs2[i0], ci1 = ax.cs2[i1];
-            const float rf0 = ax.rf[i0], rf1 = ax.rf[i1];
+            const float ci0 = tb.cs2[i0], ci1 = tb.cs2[i1];
+            const float rf0 = tb.rf[i0], rf1 = tb.rf[i1];
             tc::tmem_wait_ld();
             // M[i, j] = G[i, j] exp(cs_i - cs_j) delta_j for j <= i, plus D on the diagonal
             // (the skip term D x rides along in M X).  Below the diagonal 16x16 block the
@@ -362,13 +374,13 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
                 const float g00 = __uint_as_float(gr[4 * k]), g01 = __uint_as_float(gr[4 * k + 1]);
                 const float g10 = __uint_as_float(gr[4 * k + 2]), g11 = __uint_as_float(gr[4 * k + 3]);
                 if (J < I) {
-                    const float bfac = ax.bf[I][J];
-                    const float c0 = ax.cf[j] * bfac, c1 = ax.cf[j + 1] * bfac;
+                    const float bfac = tb.bf[I][J];
+                    const float c0 = tb.cf[j] * bfac, c1 = tb.cf[j + 1] * bfac;
                     m00 = g00 * rf0 * c0; m01 = g01 * rf0 * c1;
                     m10 = g10 * rf1 * c0; m11 = g11 * rf1 * c1;
                 } else if (J == I) {
-                    const float cj0 = ax.cs2[j], cj1 = ax.cs2[j + 1];
-                    const float d0 = ax.dlt[j], d1 = ax.dlt[j + 1];
+                    const float cj0 = tb.cs2[j], cj1 = tb.cs2[j + 1];
+                    const float d0 = tb.dlt[j], d1 = tb.dlt[j + 1];
                     m00 = j <= i0 ? g00 * ex2(ci0 - cj0) * d0 : 0.f;
                     m01 = j + 1 <= i0 ? g01 * ex2(ci0 - cj1) * d1 : 0.f;
                     m10 = j <= i1 ? g10 * ex2(ci1 - cj0) * d0 : 0.f;
@@ -386,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         for (int i = tid; i < kQ * (kN / 8); i += kThreads) {
             const int r = i / (kN / 8), q = i % (kN / 8);
             const uint32_t off = tc::off_sw128(r, q * 8, 8192);
-            const __nv_bfloat162 fc = __float2bfloat162_rn(ax.ecs[r]), fb = __float2bfloat162_rn(ax.wj[r]);
+            const __nv_bfloat162 fc = __float2bfloat162_rn(tb.ecs[r]), fb = __float2bfloat162_rn(tb.wj[r]);
             uint4 vc = ld16(smem + OFF_C + off), vb = ld16(smem + OFF_B + off);
             __nv_bfloat162 *pc = reinterpret_cast<__nv_bfloat162 *>(&vc), *pb = reinterpret_cast<__nv_bfloat162 *>(&vb);
 #pragma unroll
@@ -426,14 +438,14 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
                              tc::desc_sw128(sbase + OFF_X + k * 2048, 8192, 1024), ID_S, k > 0);
             tc::mma_commit(&ax.mbar[1]);
         }
+        // warp 0: the next chunk's decay tables while the tensor cores run
+        if (warp == 0 && c + 1 < nchunks) dt_tables(c + 1);
         ok = __syncthreads_and(tc::mbar_wait(&ax.mbar[1], c & 1));
         if (!ok) { fail_bar = 1; fail_par = c & 1; break; }
         tc::fence_after_sync();
         // B, C and the M tile are free again: stage the next chunk behind the epilogue
-        if (c + 1 < nchunks) {
-            prefetch(c + 1);
-            if (warp == 0) load_dt(c + 1);
-        }
+        if (c + 1 < nchunks) prefetch(c + 1);
+        if (warp == 0 && c + 2 < nchunks) load_dt(c + 2);
 
         // ---- (5) y = Y * silu(z) for this thread's 16 positions (D x is already in Y); S = exp(cs_Q) S + Sc
         {
@@ -457,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             }
         }
         {
-            const float dAc = ax.dAc;
+            const float dAc = tb.dAc;
             float Sc[32];
             tc::tmem_ld32(tmem + t_lane + half * 32, Sc);
 #pragma unroll
