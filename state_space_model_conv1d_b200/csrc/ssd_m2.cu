@@ -70,7 +70,7 @@ struct Aux {
     float xh[2][kHx][kP];            // raw x rows before the chunk (double buffered)
     Tables tab[2];
     uint32_t tmem;
-    uint64_t mbar[2];
+    uint64_t mbar[4];                // MMA1 done, MMA2-4 done, raw x landed, B / C landed
 };
 constexpr size_t kSmemBytes = OFF_AUX + sizeof(Aux) + 1024;   // + slack to align the base to 1024
 
@@ -94,15 +94,15 @@ struct SsdArgs {
 
 SSM_DEVINL uint4 ld16(const void *p) { return *reinterpret_cast<const uint4 *>(p); }
 SSM_DEVINL void st16(void *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
-SSM_DEVINL void cp_async16(void *smem_dst, const void *gmem_src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(tc::smem_u32(smem_dst)), "l"(gmem_src) : "memory");
-}
-SSM_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-SSM_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
-template <int N>
-SSM_DEVINL void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
-__global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
+
+// Tensor maps (3-d: channel, token, batch row; bf16):
+//   tm_x  raw x, box 64 x 64 rows, no swizzle    -> row-major staging rows of 128 bytes
+//   tm_b, tm_c  conv'd B / C, box 64 x 64, 128-byte swizzle -> one K-atom of the operand tile
+//   tm_y  y, box 64 x 64, 128-byte swizzle       <- the y staging tile (rows past the tensor are skipped)
+__global__ void __launch_bounds__(kThreads, 3)
+ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
+           const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y) {
     extern __shared__ unsigned char smem_raw[];
     // swizzle atoms need 1024-byte alignment: round the base up (1 KB of slack is allocated)
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -122,19 +122,19 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
     }
     const int64_t H = a.H, g = hh / (H / a.G);
     const int K = a.K;
-    const __nv_bfloat16 *xg = a.x + row * a.x_bs + start * a.x_ts + hh * kP;
     const __nv_bfloat16 *zg = a.z ? a.z + row * a.z_bs + start * a.z_ts + hh * kP : nullptr;
     const __nv_bfloat16 *dtg = a.dt + row * a.dt_bs + start * a.dt_ts + hh;
-    const __nv_bfloat16 *Bg = a.Bc + row * a.b_bs + start * a.b_ts + g * kN;
-    const __nv_bfloat16 *Cg = a.Cc + row * a.c_bs + start * a.c_ts + g * kN;
     __nv_bfloat16 *yg = a.y + row * a.y_bs + start * a.y_ts + hh * kP;
     const uint32_t sbase = tc::smem_u32(smem);
 
     if (warp == 0) tc::tmem_alloc(&ax.tmem, kTmemCols);
     if (tid == 0) {
-        tc::mbar_init(&ax.mbar[0], 1);
-        tc::mbar_init(&ax.mbar[1], 1);
+        for (int i = 0; i < 4; ++i) tc::mbar_init(&ax.mbar[i], 1);
         tc::mbar_init_fence();
+        tc::prefetch_map(&tm_x);
+        tc::prefetch_map(&tm_b);
+        tc::prefetch_map(&tm_c);
+        tc::prefetch_map(&tm_y);
     }
 
     // ---- per-thread constants
@@ -189,35 +189,22 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
     uint32_t fail_par = 0;
 
     const int nchunks = (int)((len + kQ - 1) / kQ);
-    const uint4 zero4 = make_uint4(0, 0, 0, 0);
-    // Stage chunk cn: B and C straight into their swizzled operand tiles, the
-    // raw x rows (row-major [kQ][kP] bf16) into the M tile's space, which is
-    // free from the end of MMA2 until the mask phase of the next chunk.
-    // Asynchronous 16-byte copies; rows past the sequence end are zero-filled.
-    // Two copy groups: the raw x rows first (needed at the top of the chunk),
-    // then B and C (needed only by MMA1, after the conv).
+    const int crow = (int)row, g0 = (int)(g * kN);
+    // Stage chunk cn (thread 0): the raw x rows (row-major [kQ][kP] bf16) into the
+    // M tile's space, which is free from the end of MMA2 until the mask phase of
+    // the next chunk, and B / C straight into their swizzled operand tiles.  Rows
+    // past the tensor's end arrive as zeros; rows past a packed sequence's end
+    // belong to the next sequence and are zeroed after landing (B / C) or never
+    // used (x).
     auto prefetch = [&](int cn) {
-        const int64_t tn = (int64_t)cn * kQ;
-        const int nvn = (int)min((int64_t)kQ, len - tn);
-        for (int i = tid; i < kQ * (kP / 8); i += kThreads) {
-            const int r = i / (kP / 8), q = i % (kP / 8);
-            unsigned char *dst = smem + OFF_M + r * (kP * 2) + q * 16;
-            if (r < nvn) cp_async16(dst, xg + (tn + r) * a.x_ts + q * 8);
-            else st16(dst, zero4);
-        }
-        cp_async_commit();
-        for (int i = tid; i < kQ * (kN / 8); i += kThreads) {
-            const int r = i / (kN / 8), q = i % (kN / 8);
-            const uint32_t off = tc::off_sw128(r, q * 8, 8192);
-            if (r < nvn) {
-                cp_async16(smem + OFF_B + off, Bg + (tn + r) * a.b_ts + q * 8);
-                cp_async16(smem + OFF_C + off, Cg + (tn + r) * a.c_ts + q * 8);
-            } else {
-                st16(smem + OFF_B + off, zero4);
-                st16(smem + OFF_C + off, zero4);
-            }
-        }
-        cp_async_commit();
+        const int tok = (int)(start + (int64_t)cn * kQ);
+        tc::mbar_expect_tx(&ax.mbar[2], kQ * kP * 2);
+        tc::tma_load_3d(smem + OFF_M, &tm_x, (int)(hh * kP), tok, crow, &ax.mbar[2]);
+        tc::mbar_expect_tx(&ax.mbar[3], 4 * kQ * 64 * 2);
+        tc::tma_load_3d(smem + OFF_B, &tm_b, g0, tok, crow, &ax.mbar[3]);
+        tc::tma_load_3d(smem + OFF_B + 8192, &tm_b, g0 + 64, tok, crow, &ax.mbar[3]);
+        tc::tma_load_3d(smem + OFF_C, &tm_c, g0, tok, crow, &ax.mbar[3]);
+        tc::tma_load_3d(smem + OFF_C + 8192, &tm_c, g0 + 64, tok, crow, &ax.mbar[3]);
     };
     // raw dt of chunk cn for warp 0 (lane l holds tokens l and l + 32); kept as
     // bf16 so the load is not waited for until the next chunk uses it
@@ -272,14 +259,12 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         if (lane == 0) tw.dAc = ex2(last);
     };
     if (nchunks > 0) {
-        prefetch(0);
+        if (tid == 0) prefetch(0);
         if (warp == 0) {
             load_dt(0);
             dt_tables(0);
             if (nchunks > 1) load_dt(1);
         }
-        cp_async_wait_all();
-        tc::fence_proxy_async();
         __syncthreads();
     }
     const unsigned char *xraw = smem + OFF_M;                      // staged raw x rows of the current chunk
@@ -288,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         const int64_t t0 = (int64_t)c * kQ;
         const int nv = (int)min((int64_t)kQ, len - t0);
         const int hb = c & 1;
+        if (!tc::mbar_wait(&ax.mbar[2], c & 1)) { fail_bar = 2; fail_par = c & 1; ok = false; }
 
         // ---- (1) x conv from the staged raw rows
         {
@@ -331,9 +317,19 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
                                              : ax.xh[hb][kHx + v][p];
             }
         }
-        cp_async_wait_all();                                          // B and C of this chunk
+        // B and C of this chunk; rows past a packed sequence's end are zeroed
+        if (!tc::mbar_wait(&ax.mbar[3], c & 1)) { fail_bar = 3; fail_par = c & 1; ok = false; }
+        if (nv < kQ && a.sv.cu) {
+            const uint4 zero4 = make_uint4(0, 0, 0, 0);
+            for (int i = tid; i < (kQ - nv) * (kN / 8); i += kThreads) {
+                const int r = nv + i / (kN / 8), q = i % (kN / 8);
+                const uint32_t off = tc::off_sw128(r, q * 8, 8192);
+                st16(smem + OFF_B + off, zero4);
+                st16(smem + OFF_C + off, zero4);
+            }
+        }
         tc::fence_proxy_async();
-        __syncthreads();
+        if (!__syncthreads_and(ok)) { ok = false; break; }
 
         // ---- (2) MMA1: G = C B^T into columns 0..63
         if (tid == 0) {
@@ -444,10 +440,14 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
         if (!ok) { fail_bar = 1; fail_par = c & 1; break; }
         tc::fence_after_sync();
         // B, C and the M tile are free again: stage the next chunk behind the epilogue
-        if (c + 1 < nchunks) prefetch(c + 1);
+        if (tid == 0 && c + 1 < nchunks) prefetch(c + 1);
         if (warp == 0 && c + 2 < nchunks) load_dt(c + 2);
 
         // ---- (5) y = Y * silu(z) for this thread's 16 positions (D x is already in Y); S = exp(cs_Q) S + Sc
+        // Whole chunks (and the tensor's last, clipped chunk) leave through a TMA
+        // store of the staging tile in the X tile's space, free once MMA2 / MMA4
+        // completed; the partial last chunk of a packed sequence is stored directly.
+        const bool y_tma = nv == kQ || !a.sv.cu;
         {
             uint32_t yr[16];
             tc::tmem_ld16x256b_x4(tmem + t_lane + 64 + half * 32, yr);
@@ -464,9 +464,16 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
                         o0 *= silu_fast<__nv_bfloat16>(__uint_as_float(zw << 16));
                         o1 *= silu_fast<__nv_bfloat16>(__uint_as_float(zw & 0xffff0000u));
                     }
-                    if (i < nv) *reinterpret_cast<__nv_bfloat162 *>(yg + (t0 + i) * a.y_ts + p) = __floats2bfloat162_rn(o0, o1);
+                    const __nv_bfloat162 ob = __floats2bfloat162_rn(o0, o1);
+                    if (y_tma) *reinterpret_cast<__nv_bfloat162 *>(smem + OFF_X + tc::off_sw128(i, p, 8192)) = ob;
+                    else if (i < nv) *reinterpret_cast<__nv_bfloat162 *>(yg + (t0 + i) * a.y_ts + p) = ob;
                 }
             }
+        }
+        if (y_tma) {
+            tc::fence_proxy_async();
+            __syncthreads();
+            if (tid == 0) tc::tma_store_3d(&tm_y, (int)(hh * kP), (int)(start + t0), crow, smem + OFF_X);
         }
         {
             const float dAc = tb.dAc;
@@ -478,12 +485,12 @@ __global__ void __launch_bounds__(kThreads, 3) ssd_kernel(const SsdArgs a) {
             for (int q = 0; q < 4; ++q)
                 st16(smem + OFF_S + tc::off_sw128(sn, half * 32 + q * 8, 8192), tc::pack_bf16x8(&S[q * 8]));
         }
-        cp_async_wait_group<1>();                                     // next chunk's raw x rows (B, C may still fly)
+        if (tid == 0) tc::bulk_wait_read();                           // the X tile is written again by the next conv
         tc::fence_before_sync();
         tc::fence_proxy_async();
         __syncthreads();
     }
-    cp_async_wait_all();
+    if (tid == 0) tc::bulk_wait_all();
 
     if (!ok) {
         // a tensor-core completion never arrived: record it, give the MMAs a
@@ -531,6 +538,38 @@ size_t ssd_workspace_bytes(const ssm_scan_args &s) {
     if (s.d_conv == 0) return 0;
     const size_t one = (size_t)s.batch * (size_t)s.seqlen * (size_t)(s.ngroups * s.dstate) * 2;
     return 2 * ((one + 255) / 256 * 256);
+}
+
+// cuTensorMapEncodeTiled from the driver, fetched once through the runtime
+// (no link-time dependency on libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// A [batch][tokens][channels] bf16 tensor (element strides ts, bs) as a 3-d map
+// with a 64-channel x 64-token box.
+bool make_map(CUtensorMap *m, const void *base, int64_t channels, int64_t tokens, int64_t batch, int64_t ts, int64_t bs,
+              bool swizzle) {
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)channels, (cuuint64_t)tokens, (cuuint64_t)batch};
+    const cuuint64_t strides[2] = {(cuuint64_t)ts * 2, (cuuint64_t)(batch > 1 ? bs : ts * tokens) * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kQ, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cudaStream_t st) {
@@ -584,10 +623,18 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     a.K = (int)s.d_conv; a.softplus = s.delta_softplus;
     a.sv = sv;
     a.err = sv.err;
+    // tensor maps over the whole packed / batched token range
+    const int64_t rows = s.cu_seqlens ? 1 : s.batch;
+    CUtensorMap tm_x, tm_b, tm_c, tm_y;
+    if (!make_map(&tm_x, s.x, s.d_inner, s.seqlen, rows, s.x_token_stride, s.x_batch_stride, false) ||
+        !make_map(&tm_b, Bc, GN, s.seqlen, rows, b_ts, b_bs, true) ||
+        !make_map(&tm_c, Cc, GN, s.seqlen, rows, c_ts, c_bs, true) ||
+        !make_map(&tm_y, s.y, s.d_inner, s.seqlen, rows, s.y_token_stride, s.y_batch_stride, true))
+        return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(ssd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)s.nheads, (unsigned)nseqs);
-    ssd_kernel<<<grid, kThreads, kSmemBytes, st>>>(a);
+    ssd_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, tm_x, tm_b, tm_c, tm_y);
     return cudaGetLastError();
 }
 

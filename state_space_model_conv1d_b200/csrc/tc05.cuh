@@ -10,6 +10,7 @@
 // for M = 64 row r sits in lane (r % 16) + 32 * (r / 16).
 #pragma once
 
+#include <cuda.h>
 #include <stdint.h>
 
 #include "common.cuh"
@@ -67,6 +68,33 @@ SSM_DEVINL void fence_before_sync() { asm volatile("tcgen05.fence::before_thread
 SSM_DEVINL void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
 // Make this thread's generic-proxy shared-memory writes visible to the tensor core.
 SSM_DEVINL void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+// ---- tensor memory access (TMA) copies.  Every copy moves one tile between
+// this CTA's own shared memory and global memory.
+// Arm `mbar` for `bytes` of incoming copies (one arrival).
+SSM_DEVINL void mbar_expect_tx(uint64_t *mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(mbar)), "r"(bytes) : "memory");
+}
+// 3-d tile load global -> shared; completion is counted on `mbar` in bytes.
+SSM_DEVINL void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, uint64_t *mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(mbar))
+        : "memory");
+}
+// 3-d tile store shared -> global (rows outside the tensor are skipped), one bulk group per call site.
+SSM_DEVINL void tma_store_3d(const CUtensorMap *map, int c0, int c1, int c2, const void *src) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];\n"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(src))
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+}
+// Wait until the issued bulk stores have finished reading shared memory / have completed.
+SSM_DEVINL void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+SSM_DEVINL void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+SSM_DEVINL void prefetch_map(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
 
 // Warp-wide: allocate `ncols` tensor-memory columns; the base address lands in *dst.
 SSM_DEVINL void tmem_alloc(uint32_t *dst, uint32_t ncols) {
