@@ -69,6 +69,7 @@ struct Tables {
 struct Aux {
     float xh[2][kHx][kP];            // raw x rows before the chunk (double buffered)
     Tables tab[2];
+    float half_sum[2];               // per-warp sums of the two-warp delta scan
     uint32_t tmem;
     uint64_t mbar[4];                // MMA1 done, MMA2-4 done, raw x landed, B / C landed
 };
@@ -206,61 +207,56 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
         tc::tma_load_3d(smem + OFF_C, &tm_c, g0, tok, crow, &ax.mbar[3]);
         tc::tma_load_3d(smem + OFF_C + 8192, &tm_c, g0 + 64, tok, crow, &ax.mbar[3]);
     };
-    // raw dt of chunk cn for warp 0 (lane l holds tokens l and l + 32); kept as
-    // bf16 so the load is not waited for until the next chunk uses it
-    __nv_bfloat16 dtr0 = __float2bfloat16_rn(0.f), dtr1 = dtr0;
+    // raw dt of chunk cn for warps 0 and 1 (lane l of warp w holds token 32 w + l);
+    // kept as bf16 so the load is not waited for until the tables need it
+    __nv_bfloat16 dtr = __float2bfloat16_rn(0.f);
     auto load_dt = [&](int cn) {
         const int64_t tn = (int64_t)cn * kQ;
         const int nvn = (int)min((int64_t)kQ, len - tn);
-        dtr0 = __float2bfloat16_rn(0.f);
-        dtr1 = dtr0;
-        if (lane < nvn) dtr0 = dtg[(tn + lane) * a.dt_ts];
-        if (lane + 32 < nvn) dtr1 = dtg[(tn + lane + 32) * a.dt_ts];
+        const int j = warp * 32 + lane;
+        dtr = j < nvn ? dtg[(tn + j) * a.dt_ts] : __float2bfloat16_rn(0.f);
     };
-    // delta, running log2-decay and the mask factor tables of chunk cn (warp 0),
-    // from the raw dt loaded by load_dt(cn), into table slot cn % 2
+    // delta, running log2-decay and the mask factor tables of chunk cn (warps 0
+    // and 1, one token per lane), from the raw dt loaded by load_dt(cn), into
+    // table slot cn % 2.  The two half-chunk scans meet through shared memory
+    // and a 64-thread named barrier.
     auto dt_tables = [&](int cn) {
         Tables &tw = ax.tab[cn & 1];
         const int nvn = (int)min((int64_t)kQ, len - (int64_t)cn * kQ);
-        float d0 = 0.f, d1 = 0.f;
-        const float u0 = __bfloat162float(dtr0) + dtb, u1 = __bfloat162float(dtr1) + dtb;
-        if (lane < nvn) d0 = a.softplus ? softplus(u0) : u0;
-        if (lane + 32 < nvn) d1 = a.softplus ? softplus(u1) : u1;
-        float s0 = d0 * A2, s1 = d1 * A2;
+        const int j = warp * 32 + lane;
+        const float u = __bfloat162float(dtr) + dtb;
+        const float d = j < nvn ? (a.softplus ? softplus(u) : u) : 0.f;
+        float sc = d * A2;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const float v0 = __shfl_up_sync(0xffffffffu, s0, o);
-            const float v1 = __shfl_up_sync(0xffffffffu, s1, o);
-            if (lane >= o) { s0 += v0; s1 += v1; }
+            const float v = __shfl_up_sync(0xffffffffu, sc, o);
+            if (lane >= o) sc += v;
         }
-        s1 += __shfl_sync(0xffffffffu, s0, 31);
-        const float last = __shfl_sync(0xffffffffu, s1, 31);
+        if (lane == 31) ax.half_sum[warp] = sc;
+        asm volatile("bar.sync 1, 64;\n" ::: "memory");
+        const float h0s = ax.half_sum[0];
+        if (warp == 1) sc += h0s;
+        const float last = h0s + ax.half_sum[1];
         // block boundaries: token 16*(j/16) (start) and 16*(j/16)+15 (end)
-        const float st0 = __shfl_sync(0xffffffffu, s0, lane & ~15), st1 = __shfl_sync(0xffffffffu, s1, lane & ~15);
-        const float en0 = __shfl_sync(0xffffffffu, s0, lane | 15), en1 = __shfl_sync(0xffffffffu, s1, lane | 15);
-        tw.dlt[lane] = d0;
-        tw.dlt[lane + 32] = d1;
-        tw.cs2[lane] = s0;
-        tw.cs2[lane + 32] = s1;
-        tw.ecs[lane] = ex2(s0);
-        tw.ecs[lane + 32] = ex2(s1);
-        tw.wj[lane] = ex2(last - s0) * d0;
-        tw.wj[lane + 32] = ex2(last - s1) * d1;
-        tw.rf[lane] = ex2(s0 - st0);
-        tw.rf[lane + 32] = ex2(s1 - st1);
-        tw.cf[lane] = ex2(en0 - s0) * d0;
-        tw.cf[lane + 32] = ex2(en1 - s1) * d1;
-        __syncwarp();
-        if (lane < 16) {
+        const float st = __shfl_sync(0xffffffffu, sc, lane & ~15);
+        const float en = __shfl_sync(0xffffffffu, sc, lane | 15);
+        tw.dlt[j] = d;
+        tw.cs2[j] = sc;
+        tw.ecs[j] = ex2(sc);
+        tw.wj[j] = ex2(last - sc) * d;
+        tw.rf[j] = ex2(sc - st);
+        tw.cf[j] = ex2(en - sc) * d;
+        asm volatile("bar.sync 1, 64;\n" ::: "memory");
+        if (warp == 0 && lane < 16) {
             // block factor (I, J), J < I: exp(cs[16 I] - cs[16 J + 15]) (<= 1)
             const int I = lane >> 2, J = lane & 3;
             tw.bf[I][J] = J < I ? ex2(tw.cs2[16 * I] - tw.cs2[16 * J + 15]) : 0.f;
         }
-        if (lane == 0) tw.dAc = ex2(last);
+        if (warp == 0 && lane == 16) tw.dAc = ex2(last);
     };
     if (nchunks > 0) {
         if (tid == 0) prefetch(0);
-        if (warp == 0) {
+        if (warp < 2) {
             load_dt(0);
             dt_tables(0);
             if (nchunks > 1) load_dt(1);
@@ -273,6 +269,32 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
         const int64_t t0 = (int64_t)c * kQ;
         const int nv = (int)min((int64_t)kQ, len - t0);
         const int hb = c & 1;
+        // rows past a packed sequence's end belong to the next sequence: zero them in B / C
+        const bool zfill = nv < kQ && a.sv.cu != nullptr;
+        if (zfill) {
+            if (!tc::mbar_wait(&ax.mbar[3], c & 1)) { fail_bar = 3; fail_par = c & 1; ok = false; }
+            const uint4 zero4 = make_uint4(0, 0, 0, 0);
+            for (int i = tid; i < (kQ - nv) * (kN / 8); i += kThreads) {
+                const int r = nv + i / (kN / 8), q = i % (kN / 8);
+                const uint32_t off = tc::off_sw128(r, q * 8, 8192);
+                st16(smem + OFF_B + off, zero4);
+                st16(smem + OFF_C + off, zero4);
+            }
+            tc::fence_proxy_async();
+            __syncthreads();
+        }
+        // ---- MMA1: G = C B^T into columns 0..63, issued as soon as B / C have landed; runs under the conv
+        if (tid == 0) {
+            if (!zfill && !tc::mbar_wait(&ax.mbar[3], c & 1)) { fail_bar = 3; fail_par = c & 1; ok = false; }
+            tc::fence_after_sync();
+#pragma unroll
+            for (int k = 0; k < kN / 16; ++k) {
+                const uint32_t ko = (k >> 2) * 8192 + (k & 3) * 32;
+                tc::mma_bf16(tmem, tc::desc_sw128(sbase + OFF_C + ko, 16, 1024), tc::desc_sw128(sbase + OFF_B + ko, 16, 1024),
+                             ID_G, k > 0);
+            }
+            tc::mma_commit(&ax.mbar[0]);
+        }
         if (!tc::mbar_wait(&ax.mbar[2], c & 1)) { fail_bar = 2; fail_par = c & 1; ok = false; }
 
         // ---- (1) x conv from the staged raw rows
@@ -317,33 +339,15 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                                              : ax.xh[hb][kHx + v][p];
             }
         }
-        // B and C of this chunk; rows past a packed sequence's end are zeroed
-        if (!tc::mbar_wait(&ax.mbar[3], c & 1)) { fail_bar = 3; fail_par = c & 1; ok = false; }
-        if (nv < kQ && a.sv.cu) {
-            const uint4 zero4 = make_uint4(0, 0, 0, 0);
-            for (int i = tid; i < (kQ - nv) * (kN / 8); i += kThreads) {
-                const int r = nv + i / (kN / 8), q = i % (kN / 8);
-                const uint32_t off = tc::off_sw128(r, q * 8, 8192);
-                st16(smem + OFF_B + off, zero4);
-                st16(smem + OFF_C + off, zero4);
-            }
-        }
+        // B / C visible to every thread (the rescale reads them); X visible to the tensor core
+        if (!zfill && !tc::mbar_wait(&ax.mbar[3], c & 1)) { fail_bar = 3; fail_par = c & 1; ok = false; }
         tc::fence_proxy_async();
-        if (!__syncthreads_and(ok)) { ok = false; break; }
-
-        // ---- (2) MMA1: G = C B^T into columns 0..63
-        if (tid == 0) {
-            tc::fence_after_sync();
-#pragma unroll
-            for (int k = 0; k < kN / 16; ++k) {
-                const uint32_t ko = (k >> 2) * 8192 + (k & 3) * 32;
-                tc::mma_bf16(tmem, tc::desc_sw128(sbase + OFF_C + ko, 16, 1024), tc::desc_sw128(sbase + OFF_B + ko, 16, 1024),
-                             ID_G, k > 0);
-            }
-            tc::mma_commit(&ax.mbar[0]);
+        {
+            const bool got = tc::mbar_wait(&ax.mbar[0], c & 1);
+            if (!got) { fail_bar = 0; fail_par = c & 1; }
+            ok = __syncthreads_and(ok && got);
         }
-        ok = __syncthreads_and(tc::mbar_wait(&ax.mbar[0], c & 1));
-        if (!ok) { fail_bar = 0; fail_par = c & 1; break; }
+        if (!ok) break;
         tc::fence_after_sync();
 
         // ---- (3) mask G -> M (over the staged raw rows, already consumed); rescale C -> C', B -> B'
@@ -435,13 +439,13 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
             tc::mma_commit(&ax.mbar[1]);
         }
         // warp 0: the next chunk's decay tables while the tensor cores run
-        if (warp == 0 && c + 1 < nchunks) dt_tables(c + 1);
+        if (warp < 2 && c + 1 < nchunks) dt_tables(c + 1);
         ok = __syncthreads_and(tc::mbar_wait(&ax.mbar[1], c & 1));
         if (!ok) { fail_bar = 1; fail_par = c & 1; break; }
         tc::fence_after_sync();
         // B, C and the M tile are free again: stage the next chunk behind the epilogue
         if (tid == 0 && c + 1 < nchunks) prefetch(c + 1);
-        if (warp == 0 && c + 2 < nchunks) load_dt(c + 2);
+        if (warp < 2 && c + 2 < nchunks) load_dt(c + 2);
 
         // ---- (5) y = Y * silu(z) for this thread's 16 positions (D x is already in Y); S = exp(cs_Q) S + Sc
         // Whole chunks (and the tensor's last, clipped chunk) leave through a TMA
