@@ -22,7 +22,7 @@
 namespace ssm {
 namespace {
 
-constexpr int kThreads = 1024;         // 2 CTAs per SM: 296 slots, so ~7 waves of (row, group) units
+constexpr int kThreads = 1024;         // one CTA of 32 warps per SM (64 registers a thread)
 constexpr int kM1Channels = 256;
 
 struct DecArgs {
@@ -76,17 +76,23 @@ SSM_DEVINL int64_t hh_first(int unit, int64_t hpg) { return (int64_t)unit * hpg;
 
 // Rows [0, nrows) of one Mamba-2 group: row = (local head, p), state row at
 // stb + (c0 + row) * N, N = 128 * NV.  Lane l owns states 4 * (l + 32 v) .. +3.
+// dxr[row] = delta * x and dar[row] = exp(delta A) of the row's head.  The R
+// rows a warp has in flight are summed with a reduce-scatter: lanes exchange
+// halves of their partial sums until each lane holds one row's, then finish
+// that row with a butterfly, and lane 32 / R * i writes row i.
 template <int NV, typename T>
 SSM_DEVINL void stream_rows(float *stb, int64_t c0, int64_t h0, int64_t nrows, int64_t P, const float *xs,
-                            const float *Bs, const float *Cs, const float *dls, const float *das, const float *Dp,
+                            const float *Bs, const float *Cs, const float *dxr, const float *dar, const float *Dp,
                             const T *zr, T *yr, int warp, int lane) {
     constexpr int64_t N = 128 * NV;
     constexpr int R = NV == 1 ? 4 : 2;         // rows in flight per warp (within 64 registers)
-    float4 Bv[NV], Cv[NV];
+    float2 Bv[NV][2], Cv[NV][2];
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
-        Bv[v] = *reinterpret_cast<const float4 *>(Bs + 4 * (lane + 32 * v));
-        Cv[v] = *reinterpret_cast<const float4 *>(Cs + 4 * (lane + 32 * v));
+        const float4 b4 = *reinterpret_cast<const float4 *>(Bs + 4 * (lane + 32 * v));
+        const float4 c4 = *reinterpret_cast<const float4 *>(Cs + 4 * (lane + 32 * v));
+        Bv[v][0] = make_float2(b4.x, b4.y); Bv[v][1] = make_float2(b4.z, b4.w);
+        Cv[v][0] = make_float2(c4.x, c4.y); Cv[v][1] = make_float2(c4.z, c4.w);
     }
     constexpr int kWarps = kThreads / 32;
     for (int64_t row0 = (int64_t)warp * R; row0 < nrows; row0 += (int64_t)kWarps * R) {
@@ -106,37 +112,44 @@ SSM_DEVINL void stream_rows(float *stb, int64_t c0, int64_t h0, int64_t nrows, i
             const int64_t row = row0 + i;
             acc[i] = 0.f;
             if (row < nrows) {
-                const int64_t hl = row / P;
-                const float dA = das[hl];
-                const float dxv = dls[hl] * xs[row];
+                const float2 dA = make_float2(dar[row], dar[row]);
+                const float2 dx = make_float2(dxr[row], dxr[row]);
                 float *srow = stb + (c0 + row) * N;
+                float2 ac = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int v = 0; v < NV; ++v) {
-                    float4 s4 = sv[i][v];
-                    s4.x = fmaf(dA, s4.x, dxv * Bv[v].x);
-                    s4.y = fmaf(dA, s4.y, dxv * Bv[v].y);
-                    s4.z = fmaf(dA, s4.z, dxv * Bv[v].z);
-                    s4.w = fmaf(dA, s4.w, dxv * Bv[v].w);
-                    __stcs(reinterpret_cast<float4 *>(srow + 4 * (lane + 32 * v)), s4);
-                    acc[i] = fmaf(Cv[v].x, s4.x, acc[i]);
-                    acc[i] = fmaf(Cv[v].y, s4.y, acc[i]);
-                    acc[i] = fmaf(Cv[v].z, s4.z, acc[i]);
-                    acc[i] = fmaf(Cv[v].w, s4.w, acc[i]);
+                    float2 lo = make_float2(sv[i][v].x, sv[i][v].y), hi = make_float2(sv[i][v].z, sv[i][v].w);
+                    lo = __ffma2_rn(dA, lo, __fmul2_rn(dx, Bv[v][0]));
+                    hi = __ffma2_rn(dA, hi, __fmul2_rn(dx, Bv[v][1]));
+                    __stcs(reinterpret_cast<float4 *>(srow + 4 * (lane + 32 * v)), make_float4(lo.x, lo.y, hi.x, hi.y));
+                    ac = __ffma2_rn(Cv[v][0], lo, ac);
+                    ac = __ffma2_rn(Cv[v][1], hi, ac);
                 }
+                acc[i] = ac.x + ac.y;
+            }
+        }
+        // reduce-scatter over the R rows, then a butterfly over the remaining lanes
+#pragma unroll
+        for (int o = 16, w = R / 2; w >= 1; o >>= 1, w >>= 1) {
+            const bool up = (lane & o) != 0;
+#pragma unroll
+            for (int k = 0; k < w; ++k) {
+                const float keep = up ? acc[w + k] : acc[k];
+                const float send = up ? acc[k] : acc[w + k];
+                acc[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
             }
         }
 #pragma unroll
-        for (int i = 0; i < R; ++i)
+        for (int o = 32 / R / 2; o >= 1; o >>= 1) acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], o);
+        // lane bits 4, 3 (R = 4) or bit 4 (R = 2) name the row this lane now holds
+        int q = 0;
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
-        if (lane < R) {
-            const int64_t row = row0 + lane;
+        for (int o = 16, w = R / 2; w >= 1; o >>= 1, w >>= 1) q += (lane & o) ? w : 0;
+        if ((lane & (32 / R - 1)) == 0) {
+            const int64_t row = row0 + q;
             if (row < nrows) {
-                float a0 = acc[0];
-#pragma unroll
-                for (int i = 1; i < R; ++i) a0 = (lane == i) ? acc[i] : a0;
                 const int64_t hl = row / P, ch = c0 + row;
-                float yv = a0 + (Dp ? Dp[h0 + hl] : 0.f) * xs[row];
+                float yv = acc[0] + (Dp ? Dp[h0 + hl] : 0.f) * xs[row];
                 if (zr) yv *= silu(Elem<T>::ld(zr + ch));
                 Elem<T>::st(yr + ch, yv);
             }
@@ -169,6 +182,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecArgs a) {
     float *Cs = Bs + N;                // [N]
     float *dls = Cs + N;               // [nh] delta
     float *das = dls + nh;             // [nh] exp(delta A)   (Mamba-2 only)
+    float *dxr = das + nh;             // [nx] delta * x per state row (Mamba-2 streaming path)
+    float *dar = dxr + nx;             // [nx] exp(delta A) per state row
     const int64_t cdim = m2 ? a.Dn + 2 * a.G * N : a.Dn;
     T *csb = static_cast<T *>(a.conv_state) + slot * cdim * a.Ls;
     const T *Br = static_cast<const T *>(a.B) + r * a.B_bs + (m2 ? unit * N : 0);
@@ -227,11 +242,17 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecArgs a) {
     const T *zr = a.z ? static_cast<const T *>(a.z) + r * a.z_bs : nullptr;
     float *stb = a.state + slot * a.Dn * N;
     if (m2 && (N == 128 || N == 256)) {
+        for (int64_t i = threadIdx.x; i < nx; i += kThreads) {
+            const int64_t hl = i / P;
+            dxr[i] = dls[hl] * xs[i];
+            dar[i] = das[hl];
+        }
+        __syncthreads();
         // Streaming fast path: one warp per 128-state row segment, each lane one
         // float4 per 128 states; four rows in flight per warp; B / C held in
         // registers for the whole group.
-        if (N == 128) stream_rows<1, T>(stb, c0, hh_first(unit, hpg), nh * P, P, xs, Bs, Cs, dls, das, a.D, zr, yr, warp, lane);
-        else stream_rows<2, T>(stb, c0, hh_first(unit, hpg), nh * P, P, xs, Bs, Cs, dls, das, a.D, zr, yr, warp, lane);
+        if (N == 128) stream_rows<1, T>(stb, c0, hh_first(unit, hpg), nh * P, P, xs, Bs, Cs, dxr, dar, a.D, zr, yr, warp, lane);
+        else stream_rows<2, T>(stb, c0, hh_first(unit, hpg), nh * P, P, xs, Bs, Cs, dxr, dar, a.D, zr, yr, warp, lane);
         return;
     }
 
@@ -311,7 +332,7 @@ cudaError_t launch_typed(const DecArgs &a, int64_t batch, cudaStream_t st) {
     const int64_t units = m2 ? a.G : (a.Dn + kM1Channels - 1) / kM1Channels;
     const int64_t nx = m2 ? (a.H / a.G) * a.P : kM1Channels;
     const int64_t nh = m2 ? a.H / a.G : kM1Channels;
-    const size_t smem = (size_t)(((nx + 3) & ~(int64_t)3) + 2 * a.N + 2 * nh) * sizeof(float);
+    const size_t smem = (size_t)(((nx + 3) & ~(int64_t)3) + 2 * a.N + 2 * nh + 2 * nx) * sizeof(float);
     auto kern = decode_kernel<T>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
