@@ -22,7 +22,7 @@
 namespace ssm {
 namespace {
 
-constexpr int kThreads = 1024;         // one CTA of 32 warps per SM (64 registers a thread)
+constexpr int kThreads = 512;          // two CTAs of 16 warps per SM: one's prologue overlaps the other's streaming
 constexpr int kM1Channels = 256;
 
 struct DecArgs {
@@ -158,7 +158,7 @@ SSM_DEVINL void stream_rows(float *stb, int64_t c0, int64_t h0, int64_t nrows, i
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const DecArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
     extern __shared__ __align__(16) float sm[];
     const int r = blockIdx.y;
     const int unit = blockIdx.x;
