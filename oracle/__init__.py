@@ -49,6 +49,9 @@ class _ScanArgs(C.Structure):
         ("h0", _dp),
         ("conv_w", _dp), ("conv_b", _dp), ("conv_state_in", _dp),
         ("y", _dp), ("h_final", _dp), ("conv_state_out", _dp),
+        ("state_interval", C.c_int64), ("inter_slots", C.POINTER(C.c_int32)),
+        ("inter_stride", C.c_int64), ("inter_nslots", C.c_int64),
+        ("inter_states", _dp), ("inter_conv", _dp),
     ]
 
 
@@ -114,11 +117,19 @@ def _seq_start(batch, seqlen, cu_seqlens):
 
 
 def scan_fwd(mode, x, dt, A, B, C_, *, D=None, z=None, dt_bias=None, h0=None, cu_seqlens=None,
-             conv_w=None, conv_b=None, conv_state_in=None, delta_softplus=True, nthreads=1, mutant=0):
+             conv_w=None, conv_b=None, conv_state_in=None, delta_softplus=True, nthreads=1, mutant=0,
+             state_interval=0, inter_slots=None, inter_states=None, inter_conv=None):
     """Forward scan (optionally with the causal conv + SiLU in front).
 
     Returns ``(y, h_final, conv_state_out)`` as float64 arrays
     (``conv_state_out`` is None without a conv).
+
+    Intermediate states: with ``state_interval > 0`` and ``inter_slots``
+    (int ``[nseq, stride]``), the state and conv history after every
+    ``state_interval`` tokens of each sequence are written into the float64
+    pools ``inter_states [nslots, ...state]`` / ``inter_conv [nslots, conv_dim,
+    K-1]`` (modified in place) at the rows the slot table names; negative or
+    out-of-range slots write nothing.
     """
     x = _f64(x)
     b, T = x.shape[0], x.shape[1]
@@ -148,6 +159,17 @@ def scan_fwd(mode, x, dt, A, B, C_, *, D=None, z=None, dt_bias=None, h0=None, cu
     for k, v in arrs.items():
         setattr(a, k, _ptr(v))
     a.y, a.h_final, a.conv_state_out = _ptr(y), _ptr(hf), _ptr(cso)
+    slots_keep = None
+    if state_interval and inter_slots is not None:
+        slots_keep = np.ascontiguousarray(inter_slots, dtype=np.int32)
+        for pool in (inter_states, inter_conv):
+            if pool is not None and (pool.dtype != np.float64 or not pool.flags.c_contiguous):
+                raise ValueError("intermediate pools must be C-contiguous float64 arrays")
+        a.state_interval = int(state_interval)
+        a.inter_slots = slots_keep.ctypes.data_as(C.POINTER(C.c_int32))
+        a.inter_stride = slots_keep.shape[1] if slots_keep.ndim == 2 else slots_keep.size
+        a.inter_nslots = inter_states.shape[0] if inter_states is not None else inter_conv.shape[0]
+        a.inter_states, a.inter_conv = _ptr(inter_states), _ptr(inter_conv)
     rc = _lib(mutant).oracle_scan_fwd(C.byref(a))
     if rc != 0:
         raise ValueError(f"oracle_scan_fwd rejected its arguments ({rc})")

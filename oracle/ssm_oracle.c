@@ -83,6 +83,19 @@ typedef struct {
     const double *h0;      /* may be NULL (zeros) */
     const double *conv_w, *conv_b, *conv_state_in; /* conv_b / state_in may be NULL */
     double *y, *h_final, *conv_state_out;          /* conv_state_out may be NULL */
+    /* Intermediate states for prefix caching ("Clean up SSM ops directory
+     * structure", Megatron-LM PR 6444: intermediate_extraction, a conditional
+     * scatter of flat state rows into slots).  When state_interval > 0, after
+     * every state_interval tokens of a sequence (boundary k at token
+     * (k+1)*state_interval from the sequence start, k < inter_stride) the
+     * state and the conv history are copied to pool row
+     * inter_slots[s*inter_stride + k] when that index lies in [0, inter_nslots);
+     * other indices write nothing. */
+    int64_t state_interval;
+    const int32_t *inter_slots;    /* [nseqs][inter_stride] */
+    int64_t inter_stride, inter_nslots;
+    double *inter_states;          /* [inter_nslots][state size] */
+    double *inter_conv;            /* [inter_nslots][conv_dim][K-1] or NULL */
 } oracle_scan_args;
 
 typedef struct {
@@ -254,6 +267,24 @@ static void scan_one_sequence(const oracle_scan_args *a, int64_t s) {
                 if (a->z) yv *= o_silu(a->z[t * Dn + ch]);
 #endif
                 a->y[t * Dn + ch] = yv;
+            }
+        }
+        /* intermediate state after this token, when it closes an interval */
+#if SSM_ORACLE_MUTANT == 13
+        const int64_t done = t - t0 + 2;             /* mutant: boundary one token early */
+#else
+        const int64_t done = t - t0 + 1;             /* tokens of this sequence processed so far */
+#endif
+        if (a->state_interval > 0 && a->inter_slots && done % a->state_interval == 0) {
+            const int64_t k = done / a->state_interval - 1;
+            if (k < a->inter_stride) {
+                const int64_t slot = a->inter_slots[s * a->inter_stride + k];
+                if (slot >= 0 && slot < a->inter_nslots) {
+                    if (a->inter_states)
+                        for (int64_t i = 0; i < hsz; ++i) a->inter_states[slot * hsz + i] = h[i];
+                    if (a->inter_conv && K > 1)
+                        for (int64_t i = 0; i < cdim * (K - 1); ++i) a->inter_conv[slot * cdim * (K - 1) + i] = hist[i];
+                }
             }
         }
     }

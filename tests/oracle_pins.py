@@ -361,6 +361,58 @@ def check_varlen_equals_per_sequence(mutant=0):
         raise AssertionError("perturbing sequence 2 changed another sequence's state")
 
 
+def check_intermediate_states_are_prefix_states(mutant=0):
+    """Intermediate-state extraction (the conditional slot scatter that prefix
+    caching uses): the state and conv history stored for boundary k equal the
+    final state and conv state of a separate run over the sequence's first
+    (k + 1) * interval tokens; negative and out-of-range slots write nothing,
+    and pool rows nobody names keep their contents."""
+    interval = 3
+    lengths = [7, 0, 9, 3]
+    cu = W.cu_from_lengths(lengths)
+    tot = int(cu[-1])
+    for mode in (M1, M2):
+        if mode == M1:
+            d = W.mamba1_inputs(75, 1, tot, 4, 3, dtype="f32", conv_bias=True, conv_state=True, nseqs=len(lengths))
+            run = _m1_scan
+        else:
+            d = W.mamba2_inputs(76, 1, tot, 4, 2, 2, 3, dtype="f32", conv_bias=True, conv_state=True, nseqs=len(lengths))
+            run = _m2_scan
+        stride = 3
+        # sequence 0: boundaries at 3, 6 -> slots 4, 0 (third entry unused: 9 > 7)
+        # sequence 2: boundaries at 3, 6, 9 -> slots -1 (skip), 9 (out of range: skip), 2
+        # sequence 3: boundary at 3 -> slot 5
+        slots = np.array([[4, 0, 1], [6, 6, 6], [-1, 9, 2], [5, 3, 3]], dtype=np.int32)
+        nslots = 7
+        hs_shape = (nslots,) + (d["h0"].shape[1:])
+        cdim = d["conv_w"].shape[0]
+        rng = np.random.default_rng(77)
+        pool_h = rng.standard_normal(hs_shape)
+        pool_c = rng.standard_normal((nslots, cdim, d["conv_w"].shape[1] - 1))
+        before_h, before_c = pool_h.copy(), pool_c.copy()
+        run(d, mutant, cu_seqlens=cu, state_interval=interval, inter_slots=slots, inter_states=pool_h, inter_conv=pool_c)
+        written = {}
+        for s, L in enumerate(lengths):
+            for k in range(stride):
+                if (k + 1) * interval <= L and 0 <= slots[s, k] < nslots:
+                    written[int(slots[s, k])] = (s, (k + 1) * interval)
+        for slot in range(nslots):
+            if slot not in written:
+                _close(pool_h[slot], before_h[slot], rtol=0, atol=0, what=f"slot {slot} untouched (state)")
+                _close(pool_c[slot], before_c[slot], rtol=0, atol=0, what=f"slot {slot} untouched (conv)")
+                continue
+            s, n = written[slot]
+            a = cu[s]
+            sub = {k: (v[:, a:a + n] if k in ("x", "z", "dt", "B", "C") else v) for k, v in d.items()}
+            sub["h0"] = d["h0"][s:s + 1]
+            sub["conv_state_in"] = d["conv_state_in"][s:s + 1]
+            _, hp, cp = run(sub, mutant)
+            _close(pool_h[slot], hp[0], rtol=0, atol=0, what=f"mode {mode} slot {slot} state = prefix state")
+            _close(pool_c[slot], cp[0], rtol=0, atol=0, what=f"mode {mode} slot {slot} conv = prefix conv state")
+        if sorted(written) != [0, 2, 4, 5]:
+            raise AssertionError(f"unexpected written slots {sorted(written)}")
+
+
 # ------------------------------------------------------------ conv pins
 def check_conv_impulse(mutant=0):
     """A unit impulse at t = 0 through a conv without activation returns each
@@ -425,5 +477,5 @@ ALL_CHECKS = [
     check_A_zero_is_cumsum, check_zero_delta_keeps_h0, check_geometric_fixed_point, check_bruteforce_m1,
     check_bruteforce_m2, check_split_invariance, check_m2_reduces_to_m1, check_prefill_equals_decode,
     check_decode_wide_conv_state, check_varlen_equals_per_sequence, check_conv_impulse, check_conv_width_one,
-    check_conv_reformulations, check_fused_conv_matches_standalone,
+    check_conv_reformulations, check_fused_conv_matches_standalone, check_intermediate_states_are_prefix_states,
 ]

@@ -56,6 +56,7 @@ MUTANTS = {
     10: "conv state ignored",
     11: "softplus switch inverted",
     12: "skip term on the pre-conv x",
+    13: "intermediate state recorded one token early",
 }
 
 
