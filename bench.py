@@ -174,6 +174,23 @@ class Job:
                 self.launches_per_step = 1 + (1 if varlen else 0)
             read = sum(v.numel() * v.element_size() for k, v in t.items() if v is not None)
             wrote = sum(v.numel() * v.element_size() for v in (self.y, self.hf, self.cso))
+            self.inter = {}
+            if w.state_interval:
+                # every boundary of every sequence gets its own pool row, in order
+                lens = np.diff(d["cu_seqlens"]) if d.get("cu_seqlens") is not None else np.full(nseq, x.shape[1])
+                stride = max(1, int(lens.max()) // w.state_interval)
+                tab = np.full((nseq, stride), -1, dtype=np.int32)
+                nslots = 0
+                for si, L in enumerate(lens):
+                    for k in range(int(L) // w.state_interval):
+                        tab[si, k] = nslots
+                        nslots += 1
+                self.inter = dict(state_interval=w.state_interval, inter_slots=torch.from_numpy(tab).to(dev),
+                                  inter_states=torch.zeros((nslots,) + tuple(self.hf.shape[1:]), dtype=torch.float32,
+                                                           device=dev),
+                                  inter_conv=torch.zeros((nslots,) + tuple(self.cso.shape[1:]), dtype=bf, device=dev))
+                read += tab.nbytes
+                wrote += sum(self.inter[k].numel() * self.inter[k].element_size() for k in ("inter_states", "inter_conv"))
             self.bytes_per_step = read + wrote
             self.units = self.tokens
             if mode == ssm.MAMBA1:
@@ -236,7 +253,7 @@ class Job:
         ssm.scan_fwd(self.mode, t["x"], t["dt"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"], dt_bias=t["dt_bias"],
                      h0=t["h0"], cu_seqlens=t.get("cu_seqlens"), conv_w=t["conv_w"], conv_b=t["conv_b"],
                      conv_state_in=t["conv_state_in"], y=self.y, h_final=self.hf, conv_state_out=self.cso,
-                     workspace=self.ws)
+                     workspace=self.ws, **self.inter)
 
     def e2e_step(self, out_host):
         """Host-resident inputs: pinned H2D copies, the step, then y back to the host."""

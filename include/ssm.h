@@ -155,6 +155,23 @@ typedef struct ssm_scan_args {
     const void *conv_state_in;
     void *conv_state_out;
     int64_t chunk;            /* Mamba-2 chunk length hint (0 = kernel default); results do not depend on it */
+    /* Intermediate states for prefix caching (optional): the conditional
+     * scatter of flat state rows into slots that "Clean up SSM ops directory
+     * structure" (Megatron-LM PR 6444) names intermediate_extraction
+     * (scatter_intermediate_ssm / scatter_intermediate_conv).  With
+     * state_interval > 0, after every state_interval tokens of a sequence
+     * (boundary k at token (k+1)*state_interval from the sequence's start,
+     * k < inter_stride) the fp32 state and the conv history (the last K-1 raw
+     * conv inputs) are written to row inter_slots[s*inter_stride + k] of the
+     * pools when that index lies in [0, inter_nslots); any other index writes
+     * nothing, and pool rows nobody names keep their contents.
+     * state_interval must be a positive multiple of 64 (0 disables). */
+    int64_t state_interval;
+    const int32_t *inter_slots;   /* device int32 [nseqs][inter_stride] */
+    int64_t inter_stride;         /* slot entries per sequence (>= 0) */
+    int64_t inter_nslots;         /* pool rows (>= 0) */
+    float *inter_states;          /* [inter_nslots][state size] fp32, rows laid out as h_final's; may be NULL */
+    void *inter_conv;             /* [inter_nslots][conv_dim][K-1] in dtype; may be NULL */
 } ssm_scan_args;
 
 /* ---------------------------------------------------------------- decode */

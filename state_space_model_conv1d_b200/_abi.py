@@ -50,6 +50,8 @@ class ScanArgs(C.Structure):
         ("cu_seqlens", _vp),
         ("conv_w", _vp), ("conv_b", _vp), ("conv_state_in", _vp), ("conv_state_out", _vp),
         ("chunk", _i64),
+        ("state_interval", _i64), ("inter_slots", _vp), ("inter_stride", _i64), ("inter_nslots", _i64),
+        ("inter_states", _vp), ("inter_conv", _vp),
     ]
 
 

@@ -27,6 +27,29 @@ struct SeqView {
     int nseqs;
 };
 
+// Intermediate-state extraction (prefix caching): after every `interval`
+// tokens of a sequence, the state and conv history go to pool row
+// slots[s * stride + k] (boundary k) when it lies in [0, nslots).  interval 0
+// disables it.  `conv` is in the activation dtype, [nslots][conv_dim][K-1].
+struct InterView {
+    int64_t interval;
+    const int32_t *slots;
+    int64_t stride, nslots;
+    float *states;
+    void *conv;
+    // pool row for the boundary that ends `done` tokens into sequence s, or -1
+    __device__ __forceinline__ int64_t slot_after(int s, int64_t done) const {
+        if (interval <= 0 || done <= 0 || done % interval != 0) return -1;
+        const int64_t k = done / interval - 1;
+        if (k >= stride) return -1;
+        const int64_t r = slots[(int64_t)s * stride + k];
+        return (r >= 0 && r < nslots) ? r : -1;
+    }
+};
+inline InterView inter_view(const ssm_scan_args &a) {
+    return InterView{a.state_interval, a.inter_slots, a.inter_stride, a.inter_nslots, a.inter_states, a.inter_conv};
+}
+
 // A causal depthwise conv over `channels` contiguous channels of a token-major
 // tensor.  Carried states are [seq][...] with `state_stride` elements between
 // sequences and K-1 values per channel (so a slice of a wider state works).

@@ -54,6 +54,7 @@ struct M1Args {
     int K, softplus;
     bool async_act, async_bc, vec_y;
     SeqView sv;
+    InterView iv;
 };
 
 SSM_DEVINL void cp_async16(void *smem, const void *gmem) {
@@ -110,7 +111,9 @@ struct SmemM1 {
     float y[2][kTC][kDB];
 };
 
-template <typename T, int SPT, int KT>
+// INTER: the intermediate-state stores are compiled in (a separate instance,
+// so the plain scan's register allocation is not perturbed by them).
+template <typename T, int SPT, int KT, bool INTER>
 __global__ void __launch_bounds__(kThreads, 3)
 scan_m1_kernel(const M1Args a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -343,6 +346,40 @@ scan_m1_kernel(const M1Args a) {
         }
     };
 
+    // ---- intermediate state after chunk c when it closes a state interval: the
+    // lanes' register states, and the conv history, which is the halo of chunk
+    // c + 1 (written by the prologue of chunk c)
+    auto inter_store = [&](int c) {
+        const int64_t slot = a.iv.slot_after(s, (int64_t)(c + 1) * kTC);
+        if (slot < 0) return;
+        if (a.iv.states && svalid) {
+            float *dst = a.iv.states + (slot * Dn + sch) * N;
+#pragma unroll
+            for (int j = 0; j < NJ; ++j)
+#pragma unroll
+                for (int e = 0; e < VW; ++e) {
+                    const int64_t n = (int64_t)VW * (q + kLanes * j) + e;
+                    float v;
+                    if constexpr (SPT >= 2) {
+                        const int i = j * VW + e;
+                        v = (i & 1) ? h2[i / 2].y : h2[i / 2].x;
+                    } else {
+                        v = h[j * VW + e];
+                    }
+                    if (n < N) dst[n] = v;
+                }
+        }
+        if (a.iv.conv && K > 1) {
+            T *cdst = static_cast<T *>(a.iv.conv) + slot * Dn * (K - 1);
+            const int hb = (c + 1) & 1;
+            for (int idx = tid; idx < (K - 1) * kDB; idx += kThreads) {
+                const int j = idx / kDB, d = idx % kDB;
+                const int64_t ch = d0 + d;
+                if (ch < Dn) Elem<T>::st(cdst + ch * (K - 1) + j, sm.halo[hb][kHalo - (K - 1) + j][d]);
+            }
+        }
+    };
+
     // ---- conv halo of chunk 0: the carried state (the K-1 raw inputs before the first token)
     if (K > 1) {
         const T *csi = static_cast<const T *>(a.conv_state_in);
@@ -364,6 +401,9 @@ scan_m1_kernel(const M1Args a) {
 
     for (int c = 0; c < nchunks; ++c) {
         scan(c);                                          // work slot c % 2 -> ysm slot c % 2
+        if constexpr (INTER) {
+            if (chunk_len(c) == kTC) inter_store(c);
+        }
         if (c > 0) store_y(c - 1);                        // ysm slot (c-1) % 2
         if (c + 1 < nchunks) prologue(c + 1);             // raw slot (c+1) % 3 -> work slot (c+1) % 2
         stage(c + 3);                                     // raw slot c % 3, read by prologue(c) last iteration
@@ -403,7 +443,9 @@ scan_m1_kernel(const M1Args a) {
 template <typename T, int SPT>
 cudaError_t launch_spt(const M1Args &a, int nseqs, cudaStream_t st) {
     const size_t smem = sizeof(SmemM1<T, SPT>);
-    auto kern = a.K <= 4 ? scan_m1_kernel<T, SPT, 4> : scan_m1_kernel<T, SPT, kMaxConvWidth>;
+    auto kern = a.iv.interval > 0 ? scan_m1_kernel<T, SPT, kMaxConvWidth, true>
+                : a.K <= 4          ? scan_m1_kernel<T, SPT, 4, false>
+                                    : scan_m1_kernel<T, SPT, kMaxConvWidth, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((a.Dn + kDB - 1) / kDB), (unsigned)nseqs);
@@ -453,6 +495,7 @@ cudaError_t launch_scan_m1(const ssm_scan_args &s, const SeqView &sv, cudaStream
                  vec_ok(s.C, s.C_batch_stride, s.C_token_stride, es);
     a.vec_y = vec_ok(s.y, s.y_batch_stride, s.y_token_stride, es);
     a.sv = sv;
+    a.iv = inter_view(s);
     const int nseqs = s.cu_seqlens ? s.nseqs : (int)s.batch;
     if (nseqs == 0) return cudaSuccess;
     return s.dtype == SSM_BF16 ? launch_typed<__nv_bfloat16>(a, nseqs, st) : launch_typed<float>(a, nseqs, st);

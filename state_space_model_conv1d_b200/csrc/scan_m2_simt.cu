@@ -43,6 +43,7 @@ struct M2Args {
     int K, softplus, npb;
     bool vec_x, vec_z, vec_B, vec_C, vec_y;
     SeqView sv;
+    InterView iv;
 };
 
 template <int SPT>
@@ -229,6 +230,40 @@ scan_m2_simt_kernel(const M2Args a) {
             }
         }
         __syncthreads();
+        // intermediate state after this chunk when it closes a state interval: the
+        // lanes' register states, and the last K-1 raw rows of the tiles (before the slide)
+        if (a.iv.interval > 0 && nv == kTC) {
+            const int64_t slot = a.iv.slot_after(s, t0 + kTC);
+            if (slot >= 0) {
+                if (a.iv.states && svalid) {
+                    float *dst = a.iv.states + ((slot * H + hh) * P + pch) * N;
+#pragma unroll
+                    for (int j = 0; j < NJ; ++j)
+#pragma unroll
+                        for (int e = 0; e < VW; ++e) {
+                            const int64_t n = (int64_t)VW * (q + kLanes * j) + e;
+                            if (n < N) dst[n] = h[j * VW + e];
+                        }
+                }
+                if (a.iv.conv && K > 1) {
+                    T *cdst = static_cast<T *>(a.iv.conv) + slot * cdim * (K - 1);
+                    const bool bc_owner = (hh % (H / G) == 0) && pb == 0;   // one writer per group
+                    for (int idx = tid; idx < (K - 1) * (kPB + 2 * NP); idx += kThreads) {
+                        const int j = idx % (K - 1), c = idx / (K - 1);
+                        const int r = kHalo + kTC - (K - 1) + j;
+                        if (c < kPB) {
+                            if (p0 + c < P) Elem<T>::st(cdst + (xch0 + c) * (K - 1) + j, sm.xraw[r][c]);
+                        } else if (bc_owner && c < kPB + NP) {
+                            const int n = c - kPB;
+                            if (n < N) Elem<T>::st(cdst + (bch0 + n) * (K - 1) + j, sm.braw[r][n]);
+                        } else if (bc_owner) {
+                            const int n = c - kPB - NP;
+                            if (n < N) Elem<T>::st(cdst + (cch0 + n) * (K - 1) + j, sm.craw[r][n]);
+                        }
+                    }
+                }
+            }
+        }
         if (nv > 0) {
             store_tile_f32<T, kThreads>(yg + t0 * a.y_ts, a.y_ts, &sm.xc[0][0], kPB, nv, p0, ncols, P, a.vec_y);
             if (K > 1 && nv == kTC) {
@@ -338,6 +373,7 @@ cudaError_t launch_scan_m2_simt(const ssm_scan_args &s, const SeqView &sv, cudaS
     a.vec_B = vec_ok(s.B, s.B_batch_stride, s.B_token_stride, es, s.dstate);
     a.vec_C = vec_ok(s.C, s.C_batch_stride, s.C_token_stride, es, s.dstate);
     a.sv = sv;
+    a.iv = inter_view(s);
     const int nseqs = s.cu_seqlens ? s.nseqs : (int)s.batch;
     if (nseqs == 0) return cudaSuccess;
     return s.dtype == SSM_BF16 ? launch_typed<__nv_bfloat16>(a, nseqs, st) : launch_typed<float>(a, nseqs, st);

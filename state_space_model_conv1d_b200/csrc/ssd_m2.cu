@@ -91,6 +91,9 @@ struct SsdArgs {
     int K, softplus;
     SeqView sv;
     int32_t *err;
+    InterView iv;
+    const __nv_bfloat16 *Braw, *Craw;   // the unconvolved B / C (intermediate conv history)
+    int64_t braw_bs, braw_ts, craw_bs, craw_ts;
 };
 
 SSM_DEVINL uint4 ld16(const void *p) { return *reinterpret_cast<const uint4 *>(p); }
@@ -489,6 +492,35 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
             for (int q = 0; q < 4; ++q)
                 st16(smem + OFF_S + tc::off_sw128(sn, half * 32 + q * 8, 8192), tc::pack_bf16x8(&S[q * 8]));
         }
+        // intermediate state after this chunk when it closes a state interval
+        if (a.iv.interval > 0 && nv == kQ) {
+            const int64_t slot = a.iv.slot_after(s, t0 + kQ);
+            if (slot >= 0) {
+                if (a.iv.states) {
+                    float *dst = a.iv.states + (slot * H + hh) * kP * kN;
+#pragma unroll
+                    for (int p = 0; p < 32; ++p) dst[(int64_t)(half * 32 + p) * kN + sn] = S[p];
+                }
+                if (a.iv.conv && K > 1) {
+                    // x channels of this head: the halo of the next chunk; B / C of the
+                    // group (written by its first head): the raw inputs before the boundary
+                    __nv_bfloat16 *cdst = static_cast<__nv_bfloat16 *>(a.iv.conv) + slot * a.cdim * (K - 1);
+                    if (tid < kP)
+                        for (int j = 0; j < K - 1; ++j)
+                            cdst[(hh * kP + tid) * (K - 1) + j] = __float2bfloat16_rn(ax.xh[hb ^ 1][kHx - (K - 1) + j][tid]);
+                    if (hh % (H / a.G) == 0) {
+                        const int64_t GN = a.G * kN;
+                        for (int i = tid; i < 2 * kN * (K - 1); i += kThreads) {
+                            const int which = i / (kN * (K - 1)), n = (i / (K - 1)) % kN, j = i % (K - 1);
+                            const int64_t tok = start + t0 + kQ - (K - 1) + j;
+                            const __nv_bfloat16 v = which ? a.Craw[row * a.craw_bs + tok * a.craw_ts + g * kN + n]
+                                                          : a.Braw[row * a.braw_bs + tok * a.braw_ts + g * kN + n];
+                            cdst[(a.H * kP + which * GN + g * kN + n) * (K - 1) + j] = v;
+                        }
+                    }
+                }
+            }
+        }
         if (tid == 0) tc::bulk_wait_read();                           // the X tile is written again by the next conv
         tc::fence_before_sync();
         tc::fence_proxy_async();
@@ -627,6 +659,10 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     a.K = (int)s.d_conv; a.softplus = s.delta_softplus;
     a.sv = sv;
     a.err = sv.err;
+    a.iv = inter_view(s);
+    a.Braw = static_cast<const __nv_bfloat16 *>(s.B); a.Craw = static_cast<const __nv_bfloat16 *>(s.C);
+    a.braw_bs = s.B_batch_stride; a.braw_ts = s.B_token_stride;
+    a.craw_bs = s.C_batch_stride; a.craw_ts = s.C_token_stride;
     // tensor maps over the whole packed / batched token range
     const int64_t rows = s.cu_seqlens ? 1 : s.batch;
     CUtensorMap tm_x, tm_b, tm_c, tm_y;

@@ -99,6 +99,13 @@ ssm_status validate_scan(const ssm_scan_args *a) {
         return SSM_ERR_ALIGNMENT;
     if (!aligned(a->conv_state_in, es) || !aligned(a->conv_state_out, es)) return SSM_ERR_ALIGNMENT;
     if (a->chunk < 0) return SSM_ERR_INVALID_ARG;
+    if (a->state_interval != 0) {
+        if (a->state_interval < 0 || a->state_interval % 64 != 0 || !a->inter_slots || a->inter_stride < 0 ||
+            a->inter_nslots < 0 || (!a->inter_states && !a->inter_conv))
+            return SSM_ERR_INVALID_ARG;
+        if (!aligned(a->inter_slots, 4) || !aligned(a->inter_states, 4) || !aligned(a->inter_conv, es))
+            return SSM_ERR_ALIGNMENT;
+    }
     return SSM_OK;
 }
 

@@ -162,12 +162,20 @@ def scan_workspace_size(mode, x, dt, A, B, C_, *, cu_seqlens=None, conv_w=None, 
 
 def scan_fwd(mode, x, dt, A, B, C_, *, D=None, z=None, dt_bias=None, h0=None, cu_seqlens=None, conv_w=None,
              conv_b=None, conv_state_in=None, delta_softplus=True, y=None, h_final=None, conv_state_out=None,
-             return_final_state=True, return_conv_state=None, workspace=None, chunk=0, stream=None):
+             return_final_state=True, return_conv_state=None, workspace=None, chunk=0, stream=None,
+             state_interval=0, inter_slots=None, inter_states=None, inter_conv=None):
     """Forward selective scan (conv fused in front when ``conv_w`` is given).
 
     Returns ``(y, h_final, conv_state_out)``; the last two are None when not
     requested.  ``workspace`` (uint8 CUDA tensor) is allocated when needed and
     not given.
+
+    Intermediate states (prefix caching): with ``state_interval`` (a positive
+    multiple of 64) and ``inter_slots`` (int32 ``[nseq, stride]``), the state
+    after every ``state_interval`` tokens of each sequence is written to row
+    ``inter_slots[s, k]`` of ``inter_states`` (fp32 ``[nslots, ...state]``) and
+    its conv history to ``inter_conv`` (``[nslots, conv_dim, K-1]``, x's
+    dtype); negative or out-of-range slots write nothing.
     """
     _need(x, "x")
     if y is None:
@@ -187,6 +195,22 @@ def scan_fwd(mode, x, dt, A, B, C_, *, D=None, z=None, dt_bias=None, h0=None, cu
         conv_state_out = torch.empty((nseq, cdim, conv_w.shape[1] - 1), dtype=x.dtype, device=x.device)
     a = _scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, h0, h_final, cu_seqlens, conv_w, conv_b, conv_state_in,
                    conv_state_out, y, delta_softplus, chunk)
+    if state_interval:
+        if inter_slots is None or (inter_states is None and inter_conv is None):
+            raise ValueError("state_interval needs inter_slots and a pool")
+        _need(inter_slots, "inter_slots", torch.int32)
+        if not inter_slots.is_contiguous():
+            raise ValueError("inter_slots must be contiguous")
+        if inter_states is not None and (inter_states.dtype != torch.float32 or not inter_states.is_contiguous()):
+            raise ValueError("inter_states must be contiguous fp32")
+        if inter_conv is not None and (inter_conv.dtype != x.dtype or not inter_conv.is_contiguous()):
+            raise ValueError("inter_conv must be contiguous with x's dtype")
+        a.state_interval = int(state_interval)
+        a.inter_slots = _p(inter_slots)
+        a.inter_stride = inter_slots.shape[1] if inter_slots.dim() == 2 else inter_slots.numel()
+        pool = inter_states if inter_states is not None else inter_conv
+        a.inter_nslots = pool.shape[0]
+        a.inter_states, a.inter_conv = _p(inter_states), _p(inter_conv)
     l = _abi.lib()
     need = int(l.ssm_scan_workspace_size(C.byref(a)))
     if need and workspace is None:

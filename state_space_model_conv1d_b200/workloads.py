@@ -183,10 +183,12 @@ class Workload:
     conv_state_len: int = 4
     steps: int = 0
     nsets: int = 1
+    state_interval: int = 0   # > 0: intermediate states every this many tokens (prefix caching)
     seed: int = BASE_SEED
 
 
-# The five workloads of the hot path.  Seeds are BASE_SEED + position.
+# The five workloads of the hot path (seeds BASE_SEED + position), then the
+# varlen workload again with intermediate-state extraction (same inputs).
 WORKLOADS = {
     "mamba1_tiny_f32": Workload("mamba1_tiny_f32", "mamba1", "f32", batch=1, seqlen=64, d_inner=16, dstate=4,
                                 seed=BASE_SEED + 0),
@@ -201,6 +203,11 @@ WORKLOADS = {
     "mamba2_decode_b256_h128_p64_g8_n128": Workload("mamba2_decode_b256_h128_p64_g8_n128", "decode", "bf16",
                                                     batch=256, nheads=128, headdim=64, ngroups=8, dstate=128,
                                                     conv_state_len=4, steps=1000, nsets=8, seed=BASE_SEED + 4),
+    # the packed varlen workload again, also storing every sequence's state and
+    # conv history after each 512 tokens (prefix-caching extraction)
+    "mamba2_varlen_16seq_h64_p64_g1_n128_states512": Workload(
+        "mamba2_varlen_16seq_h64_p64_g1_n128_states512", "mamba2_varlen", "bf16", nheads=64, headdim=64, ngroups=1,
+        dstate=128, nseqs=16, len_lo=128, len_hi=8192, chunk=256, state_interval=512, seed=BASE_SEED + 3),
 }
 
 

@@ -111,6 +111,14 @@ def _scan(**kw):
     (dict(mode=1, ngroups=2, d_inner=8), _abi.SSM_ERR_UNSUPPORTED),
     (dict(mode=1, ngroups=1, dstate=128), _abi.SSM_ERR_UNSUPPORTED),
     (dict(delta_softplus=2), _abi.SSM_ERR_INVALID_ARG),
+    # intermediate-state extraction
+    (dict(state_interval=32, inter_slots=FAKE, inter_states=FAKE), _abi.SSM_ERR_INVALID_ARG),   # not a multiple of 64
+    (dict(state_interval=-64, inter_slots=FAKE, inter_states=FAKE), _abi.SSM_ERR_INVALID_ARG),
+    (dict(state_interval=64, inter_states=FAKE), _abi.SSM_ERR_INVALID_ARG),                     # no slot table
+    (dict(state_interval=64, inter_slots=FAKE), _abi.SSM_ERR_INVALID_ARG),                      # no pool
+    (dict(state_interval=64, inter_slots=FAKE, inter_states=FAKE, inter_nslots=-1), _abi.SSM_ERR_INVALID_ARG),
+    (dict(state_interval=64, inter_slots=FAKE + 2, inter_states=FAKE), _abi.SSM_ERR_ALIGNMENT),
+    (dict(state_interval=64, inter_slots=FAKE, inter_conv=FAKE + 1), _abi.SSM_ERR_ALIGNMENT),
 ])
 def test_scan_rejects(kw, status):
     a = _scan(**kw)
