@@ -218,6 +218,17 @@ SSM_API ssm_status ssm_scan_fwd(const ssm_scan_args *args, void *workspace, size
 /* Decode update, in place on state and conv_state.  No workspace. */
 SSM_API ssm_status ssm_state_update(const ssm_update_args *args, void *stream);
 
+/* Per-kernel device timing of the dominant kernel of each call (the scan
+ * kernel of ssm_scan_fwd, the update kernel of ssm_state_update), for
+ * roofline measurements.  The papers have no counterpart.  While enabled
+ * (process-wide, off by default), every such launch is bracketed by a CUDA
+ * event pair recorded on the call's own stream (events are created on first
+ * use and reused).  ssm_kernel_time_ms synchronizes on the recorded events,
+ * returns the summed elapsed time and the number of launches since the last
+ * read, and starts a new tally.  Not for use inside stream capture. */
+SSM_API ssm_status ssm_kernel_timing(int32_t enable);
+SSM_API ssm_status ssm_kernel_time_ms(float *total_ms, int32_t *launches);
+
 /* ssm_scan_fwd without a caller-supplied workspace, for callers that cannot
  * allocate device memory (code inside a CUDA-graph capture that must not
  * allocate, a runtime whose memory pool belongs to another component, a

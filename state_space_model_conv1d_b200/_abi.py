@@ -83,6 +83,8 @@ SIGNATURES = {
     "ssm_state_update": ([C.POINTER(UpdateArgs), _vp], _i32),
     "ssm_workspace_error": ([_vp, C.POINTER(_i32), _vp], _i32),
     "ssm_scan_fwd_noalloc": ([C.POINTER(ScanArgs), _vp], _i32),
+    "ssm_kernel_timing": ([_i32], _i32),
+    "ssm_kernel_time_ms": ([C.POINTER(C.c_float), C.POINTER(_i32)], _i32),
 }
 
 _lock = threading.Lock()

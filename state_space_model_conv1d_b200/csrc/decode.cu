@@ -337,7 +337,9 @@ cudaError_t launch_typed(const DecArgs &a, int64_t batch, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)units, (unsigned)batch);
+    timing_begin(st);
     kern<<<grid, kThreads, smem, st>>>(a);
+    timing_end(st);
     return cudaGetLastError();
 }
 

@@ -82,6 +82,11 @@ size_t ssd_workspace_bytes(const ssm_scan_args &a);
 cudaError_t launch_ssd(const ssm_scan_args &a, const SeqView &sv, void *ws_bc, cudaStream_t st);
 cudaError_t launch_state_update(const ssm_update_args &a, cudaStream_t st);
 
+// Device timing of the dominant kernel of a call (ssm_kernel_timing): a no-op
+// unless enabled; otherwise records one event before and one after on `st`.
+void timing_begin(cudaStream_t st);
+void timing_end(cudaStream_t st);
+
 // Largest dstate each path supports.
 constexpr int64_t kMaxDstateM1 = 64;
 constexpr int64_t kMaxDstateM2 = 256;

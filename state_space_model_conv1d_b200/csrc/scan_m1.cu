@@ -449,7 +449,9 @@ cudaError_t launch_spt(const M1Args &a, int nseqs, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)((a.Dn + kDB - 1) / kDB), (unsigned)nseqs);
+    timing_begin(st);
     kern<<<grid, kThreads, smem, st>>>(a);
+    timing_end(st);
     return cudaGetLastError();
 }
 

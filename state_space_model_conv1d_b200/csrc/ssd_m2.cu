@@ -674,7 +674,9 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     cudaError_t e = cudaFuncSetAttribute(ssd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)s.nheads, (unsigned)nseqs);
+    timing_begin(st);
     ssd_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, tm_x, tm_b, tm_c, tm_y);
+    timing_end(st);
     return cudaGetLastError();
 }
 

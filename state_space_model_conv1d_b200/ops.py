@@ -286,3 +286,16 @@ def state_update(mode, state, conv_state, x, dt, A, B, C_, *, D=None, z=None, dt
     a.nslots = state.shape[0]
     _abi.check(_abi.lib().ssm_state_update(C.byref(a), _stream(stream)), "ssm_state_update")
     return y
+
+
+def kernel_timing(enable: bool) -> None:
+    """Turn on / off device timing of each call's dominant kernel (process-wide)."""
+    _abi.check(_abi.lib().ssm_kernel_timing(int(bool(enable))), "ssm_kernel_timing")
+
+
+def kernel_time_ms():
+    """(summed milliseconds, launches) of the timed kernels since the last read; synchronizes."""
+    ms, n = C.c_float(0.0), _abi._i32(0)
+    _abi.check(_abi.lib().ssm_kernel_time_ms(C.byref(ms), C.byref(n)), "ssm_kernel_time_ms")
+    return float(ms.value), int(n.value)
+
