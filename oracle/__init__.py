@@ -55,6 +55,18 @@ class _ScanArgs(C.Structure):
     ]
 
 
+class _ScanBwdArgs(C.Structure):
+    _fields_ = [
+        ("fwd", _ScanArgs),
+        ("dy", _dp), ("dh_final", _dp), ("dconv_state_out", _dp),
+        ("dx", _dp), ("dz", _dp), ("ddt", _dp), ("dB", _dp), ("dC", _dp),
+        ("dA", _dp), ("dD", _dp), ("ddt_bias", _dp),
+        ("dh0", _dp),
+        ("dconv_w", _dp), ("dconv_b", _dp),
+        ("dconv_state_in", _dp),
+    ]
+
+
 class _ConvArgs(C.Structure):
     _fields_ = [
         ("activation", C.c_int32), ("pad_", C.c_int32),
@@ -92,6 +104,8 @@ def _lib(mutant: int = 0) -> C.CDLL:
         lib.oracle_conv1d_fwd.restype = C.c_int
         lib.oracle_state_update.argtypes = [C.POINTER(_UpdateArgs)]
         lib.oracle_state_update.restype = C.c_int
+        lib.oracle_scan_bwd.argtypes = [C.POINTER(_ScanBwdArgs)]
+        lib.oracle_scan_bwd.restype = C.c_int
         lib.oracle_mutant_id.restype = C.c_int
         _LIBS[mutant] = lib
     return _LIBS[mutant]
@@ -174,6 +188,56 @@ def scan_fwd(mode, x, dt, A, B, C_, *, D=None, z=None, dt_bias=None, h0=None, cu
     if rc != 0:
         raise ValueError(f"oracle_scan_fwd rejected its arguments ({rc})")
     return y, hf, cso
+
+
+def scan_bwd(mode, x, dt, A, B, C_, dy, *, D=None, z=None, dt_bias=None, h0=None, cu_seqlens=None,
+             conv_w=None, conv_b=None, conv_state_in=None, delta_softplus=True, dh_final=None,
+             dconv_state_out=None, mutant=0):
+    """Gradients of ``sum(dy*y) + sum(dh_final*h_final) + sum(dconv_state_out*conv_state_out)``
+    with respect to every input of :func:`scan_fwd` (same arguments).
+
+    Returns a dict of float64 arrays shaped like the inputs: ``dx, dz, ddt, dB,
+    dC`` (raw inputs, before the conv), ``dA, dD, ddt_bias, dh0, dconv_w,
+    dconv_b, dconv_state_in`` (None where the input is None).
+    """
+    x = _f64(x)
+    b, T = x.shape[0], x.shape[1]
+    if mode == MAMBA1:
+        Dn = x.shape[2]
+        N = np.asarray(B).shape[2]
+        H, P, G = Dn, 1, 1
+    else:
+        H, P = x.shape[2], x.shape[3]
+        G, N = np.asarray(B).shape[2], np.asarray(B).shape[3]
+        Dn = H * P
+    seq = _seq_start(b, T, cu_seqlens)
+    nseq = len(seq) - 1
+    K = 0 if conv_w is None else np.asarray(conv_w).shape[1]
+    cdim = Dn if mode == MAMBA1 else Dn + 2 * G * N
+    ins = dict(x=x, dt=_f64(dt), A=_f64(A), B=_f64(B), C=_f64(C_), D=_f64(D), z=_f64(z),
+               dt_bias=_f64(dt_bias), h0=_f64(h0), conv_w=_f64(conv_w), conv_b=_f64(conv_b),
+               conv_state_in=_f64(conv_state_in))
+    hshape = (nseq, Dn, N) if mode == MAMBA1 else (nseq, H, P, N)
+    z0 = lambda k: None if ins[k] is None else np.zeros(ins[k].shape, dtype=np.float64)
+    out = dict(dx=z0("x"), dz=z0("z"), ddt=z0("dt"), dB=z0("B"), dC=z0("C"), dA=z0("A"), dD=z0("D"),
+               ddt_bias=z0("dt_bias"), dh0=np.zeros(hshape, dtype=np.float64), dconv_w=z0("conv_w"),
+               dconv_b=z0("conv_b"),
+               dconv_state_in=np.zeros((nseq, cdim, K - 1), dtype=np.float64) if K > 1 else None)
+    a = _ScanBwdArgs()
+    f = a.fwd
+    f.mode, f.delta_softplus, f.nthreads = mode, int(bool(delta_softplus)), 1
+    f.nseqs, f.seq_start = nseq, seq.ctypes.data_as(_lp)
+    f.d_inner, f.nheads, f.headdim, f.ngroups, f.dstate, f.d_conv = Dn, H, P, G, N, K
+    for k, v in ins.items():
+        setattr(f, k, _ptr(v))
+    dyv, dhf, dcs = _f64(dy), _f64(dh_final), _f64(dconv_state_out)
+    a.dy, a.dh_final, a.dconv_state_out = _ptr(dyv), _ptr(dhf), _ptr(dcs)
+    for k, v in out.items():
+        setattr(a, k, _ptr(v))
+    rc = _lib(mutant).oracle_scan_bwd(C.byref(a))
+    if rc != 0:
+        raise ValueError(f"oracle_scan_bwd rejected its arguments ({rc})")
+    return out
 
 
 def conv1d_fwd(x, w, *, b=None, state_in=None, cu_seqlens=None, activation=True, mutant=0):

@@ -311,6 +311,207 @@ int oracle_scan_fwd(const oracle_scan_args *a) {
     return 0;
 }
 
+/* ---- backward of the forward scan (reverse mode, plain loops) ----
+ *
+ * Gradients of L = sum(dy * y) + sum(dh_final * h_final) + sum(dconv_state_out
+ * * conv_state_out) with respect to every input of oracle_scan_fwd, for the
+ * same arguments.  The step h_t = a_t h_{t-1} + delta_t B_t x_t with
+ * a_t = exp(delta_t A) is differentiated as it stands ("Adding Initial Value
+ * Support to Selective Scan Forward Kernel", state-spaces/mamba issue 285: the
+ * backward carries dh back through exp(delta A) down to the initial state,
+ * whose gradient is the carried dh after the first token).  The forward
+ * trajectory (every h_t, every conv output and pre-activation) is stored and
+ * walked backwards; nothing is chunked.
+ */
+typedef struct {
+    oracle_scan_args fwd;          /* the forward call (its y / h_final / conv_state_out are scratch) */
+    const double *dy;              /* [tok][D_] */
+    const double *dh_final;        /* [seq][state] or NULL */
+    const double *dconv_state_out; /* [seq][conv_dim][K-1] or NULL */
+    double *dx, *dz, *ddt, *dB, *dC;  /* like x, z, dt, B, C (raw, before the conv) */
+    double *dA, *dD, *ddt_bias;       /* like A, D, dt_bias (dD / ddt_bias may be NULL) */
+    double *dh0;                      /* [seq][state] */
+    double *dconv_w, *dconv_b;        /* [conv_dim][K], [conv_dim] (may be NULL) */
+    double *dconv_state_in;           /* [seq][conv_dim][K-1] (may be NULL) */
+} oracle_scan_bwd_args;
+
+static double o_sigmoid(double v) { return 1.0 / (1.0 + exp(-v)); }
+static double o_dsilu(double v) { const double sg = o_sigmoid(v); return sg * (1.0 + v * (1.0 - sg)); }
+
+static void bwd_one_sequence(const oracle_scan_bwd_args *b, int64_t s) {
+    const oracle_scan_args *a = &b->fwd;
+    const int64_t t0 = a->seq_start[s], t1 = a->seq_start[s + 1], T = t1 - t0;
+    const int64_t N = a->dstate, K = a->d_conv, Dn = a->d_inner;
+    const int64_t cdim = o_conv_dim(a);
+    const int m1 = a->mode == ORACLE_M1;
+    const int64_t H = m1 ? Dn : a->nheads, P = m1 ? 1 : a->headdim, G = m1 ? 1 : a->ngroups;
+    const int64_t hsz = Dn * N, KW = K > 1 ? K - 1 : 0;
+
+    /* forward trajectory: raw inputs r, pre-activations pre, conv outputs u, deltas, states */
+    double *raw = (double *)calloc((size_t)((T + KW) * cdim + 1), sizeof(double)); /* KW history rows first */
+    double *pre = (double *)calloc((size_t)(T * cdim + 1), sizeof(double));
+    double *u = (double *)calloc((size_t)(T * cdim + 1), sizeof(double));
+    double *dl = (double *)calloc((size_t)(T * H + 1), sizeof(double));
+    double *hs = (double *)calloc((size_t)((T + 1) * hsz), sizeof(double));
+    double *du = (double *)calloc((size_t)(T * cdim + 1), sizeof(double));
+    double *g = (double *)calloc((size_t)hsz, sizeof(double));
+    for (int64_t j = 0; j < KW; ++j)
+        for (int64_t c = 0; c < cdim; ++c)
+            raw[j * cdim + c] = a->conv_state_in ? a->conv_state_in[(s * cdim + c) * KW + j] : 0.0;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t c = 0; c < cdim; ++c) {
+            const int64_t tt = t0 + t;
+            double r;
+            if (c < Dn) r = a->x[tt * Dn + c];
+            else if (c < Dn + G * N) r = a->B[tt * G * N + (c - Dn)];
+            else r = a->C[tt * G * N + (c - Dn - G * N)];
+            raw[(KW + t) * cdim + c] = r;
+        }
+    const int64_t ccov = m1 ? Dn : cdim;    /* channels that pass through the conv */
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t c = 0; c < cdim; ++c) {
+            const double r = raw[(KW + t) * cdim + c];
+            if (K > 0 && c < ccov) {
+                double acc = a->conv_b ? a->conv_b[c] : 0.0;
+                for (int64_t k = 0; k < K; ++k) acc += a->conv_w[c * K + k] * raw[(KW + t - (K - 1) + k) * cdim + c];
+                pre[t * cdim + c] = acc;
+                u[t * cdim + c] = o_silu(acc);
+            } else {
+                u[t * cdim + c] = r;
+            }
+        }
+    if (a->h0)
+        for (int64_t i = 0; i < hsz; ++i) hs[i] = a->h0[s * hsz + i];
+    for (int64_t t = 0; t < T; ++t) {
+        const int64_t tt = t0 + t;
+        for (int64_t hh = 0; hh < H; ++hh) {
+            const double dtv = m1 ? a->dt[tt * Dn + hh] : a->dt[tt * H + hh];
+            dl[t * H + hh] = o_delta(dtv, a->dt_bias ? a->dt_bias[hh] : 0.0, a->delta_softplus);
+        }
+        const double *Bt = m1 ? a->B + tt * N : u + t * cdim + Dn;
+        for (int64_t hh = 0; hh < H; ++hh) {
+            const int64_t gg = m1 ? 0 : hh / (H / G);
+            const double delta = dl[t * H + hh];
+            for (int64_t p = 0; p < P; ++p) {
+                const int64_t ch = hh * P + p;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double An = m1 ? a->A[hh * N + n] : a->A[hh];
+                    hs[(t + 1) * hsz + ch * N + n] = exp(delta * An) * hs[t * hsz + ch * N + n] +
+                                                     delta * Bt[gg * N + n] * u[t * cdim + ch];
+                }
+            }
+        }
+    }
+
+    /* reverse sweep over the recurrence */
+    for (int64_t i = 0; i < hsz; ++i) g[i] = b->dh_final ? b->dh_final[s * hsz + i] : 0.0;
+    for (int64_t t = T - 1; t >= 0; --t) {
+        const int64_t tt = t0 + t;
+        const double *Bt = m1 ? a->B + tt * N : u + t * cdim + Dn;
+        const double *Ct = m1 ? a->C + tt * N : u + t * cdim + Dn + G * N;
+        for (int64_t hh = 0; hh < H; ++hh) {
+            const int64_t gg = m1 ? 0 : hh / (H / G);
+            const double delta = dl[t * H + hh];
+            double ddelta = 0.0;
+            for (int64_t p = 0; p < P; ++p) {
+                const int64_t ch = hh * P + p;
+                const double xv = u[t * cdim + ch];
+                const double *ht = hs + (t + 1) * hsz + ch * N, *hp = hs + t * hsz + ch * N;
+                double ybase = 0.0;
+                for (int64_t n = 0; n < N; ++n) ybase += Ct[gg * N + n] * ht[n];
+                const double Dv = a->D ? a->D[m1 ? ch : hh] : 0.0;
+                ybase += Dv * xv;
+                const double dyv = b->dy[tt * Dn + ch];
+                double dyb = dyv;
+                if (a->z) {
+                    const double zv = a->z[tt * Dn + ch];
+                    b->dz[tt * Dn + ch] = dyv * ybase * o_dsilu(zv);
+                    dyb = dyv * o_silu(zv);
+                }
+                if (b->dD && a->D) b->dD[m1 ? ch : hh] += dyb * xv;
+                du[t * cdim + ch] += dyb * Dv;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double dCv = dyb * ht[n];
+                    if (m1) b->dC[tt * N + n] += dCv;
+                    else du[t * cdim + Dn + G * N + gg * N + n] += dCv;
+                    g[ch * N + n] += dyb * Ct[gg * N + n];
+                }
+                for (int64_t n = 0; n < N; ++n) {
+                    const double An = m1 ? a->A[hh * N + n] : a->A[hh];
+                    const double av = exp(delta * An);
+                    const double gn = g[ch * N + n];
+                    const double dBv = gn * delta * xv;
+                    if (m1) b->dB[tt * N + n] += dBv;
+                    else du[t * cdim + Dn + gg * N + n] += dBv;
+                    du[t * cdim + ch] += gn * delta * Bt[gg * N + n];
+                    ddelta += gn * (hp[n] * av * An + Bt[gg * N + n] * xv);
+                    if (m1) b->dA[hh * N + n] += gn * hp[n] * av * delta;
+                    else b->dA[hh] += gn * hp[n] * av * delta;
+#if SSM_ORACLE_MUTANT == 14
+                    g[ch * N + n] = gn;                      /* mutant: dh not carried through exp(delta A) */
+#else
+                    g[ch * N + n] = gn * av;
+#endif
+                }
+            }
+            const double dtv = m1 ? a->dt[tt * Dn + hh] : a->dt[tt * H + hh];
+            const double uarg = dtv + (a->dt_bias ? a->dt_bias[hh] : 0.0);
+            const double dd = a->delta_softplus ? ddelta * o_sigmoid(uarg) : ddelta;
+            b->ddt[m1 ? tt * Dn + hh : tt * H + hh] = dd;
+            if (b->ddt_bias && a->dt_bias) b->ddt_bias[hh] += dd;
+        }
+    }
+    for (int64_t i = 0; i < hsz; ++i) b->dh0[s * hsz + i] = g[i];
+
+    /* reverse sweep over the conv: d(raw) over the sequence and its history */
+    double *draw = (double *)calloc((size_t)((T + KW) * cdim + 1), sizeof(double));
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t c = 0; c < cdim; ++c) {
+            const double dv = du[t * cdim + c];
+            if (K > 0 && c < ccov) {
+                const double dp = dv * o_dsilu(pre[t * cdim + c]);
+                if (b->dconv_b) b->dconv_b[c] += dp;
+                for (int64_t k = 0; k < K; ++k) {
+                    const int64_t r = KW + t - (K - 1) + k;
+                    if (b->dconv_w) b->dconv_w[c * K + k] += dp * raw[r * cdim + c];
+                    draw[r * cdim + c] += dp * a->conv_w[c * K + k];
+                }
+            } else {
+                draw[(KW + t) * cdim + c] += dv;
+            }
+        }
+    /* the carried conv state out is the last K-1 raw rows of history + sequence */
+    if (b->dconv_state_out && KW > 0)
+        for (int64_t j = 0; j < KW; ++j)
+            for (int64_t c = 0; c < cdim; ++c) draw[(T + j) * cdim + c] += b->dconv_state_out[(s * cdim + c) * KW + j];
+    for (int64_t j = 0; j < KW; ++j)
+        for (int64_t c = 0; c < cdim; ++c)
+            if (b->dconv_state_in) b->dconv_state_in[(s * cdim + c) * KW + j] = draw[j * cdim + c];
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t c = 0; c < cdim; ++c) {
+            const int64_t tt = t0 + t;
+            const double v = draw[(KW + t) * cdim + c];
+            if (c < Dn) b->dx[tt * Dn + c] = v;
+            else if (c < Dn + G * N) b->dB[tt * G * N + (c - Dn)] += m1 ? 0.0 : v;
+            else b->dC[tt * G * N + (c - Dn - G * N)] += m1 ? 0.0 : v;
+        }
+    free(draw); free(raw); free(pre); free(u); free(dl); free(hs); free(du); free(g);
+}
+
+int oracle_scan_bwd(const oracle_scan_bwd_args *b) {
+    if (!b || !b->dy || !b->dx || !b->ddt || !b->dA || !b->dB || !b->dC || !b->dh0) return -1;
+    const oracle_scan_args *a = &b->fwd;
+    if (!a->seq_start || !a->x || !a->dt || !a->A || !a->B || !a->C) return -1;
+    if (a->mode != ORACLE_M1 && a->mode != ORACLE_M2) return -1;
+    if (a->mode == ORACLE_M2 && (a->nheads * a->headdim != a->d_inner || a->ngroups <= 0 ||
+                                 a->nheads % a->ngroups != 0)) return -1;
+    if (a->d_conv > 0 && !a->conv_w) return -1;
+    if (a->z && !b->dz) return -1;
+    /* accumulated outputs start at zero; sequences run one after another (shared dA, dB, ...) */
+    for (int64_t s = 0; s < a->nseqs; ++s) bwd_one_sequence(b, s);
+    return 0;
+}
+
 /* ---- standalone causal depthwise conv ---- */
 int oracle_conv1d_fwd(const oracle_conv_args *a) {
     if (!a || !a->seq_start || !a->x || !a->w || !a->out || a->width < 1) return -1;

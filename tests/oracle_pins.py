@@ -413,6 +413,54 @@ def check_intermediate_states_are_prefix_states(mutant=0):
             raise AssertionError(f"unexpected written slots {sorted(written)}")
 
 
+def check_backward_matches_finite_differences(mutant=0):
+    """The backward (reverse mode over the stored trajectory) against central
+    finite differences of the forward oracle, for every input: the loss is
+    sum(dy*y) + sum(dh_final*h_final) + sum(dconv_state_out*conv_state_out) on
+    packed sequences with an empty one, a conv with bias and carried state,
+    grouped heads, and softplus on and off."""
+    lengths = [5, 0, 4]
+    cu = W.cu_from_lengths(lengths)
+    tot = int(cu[-1])
+    names = {"x": "dx", "z": "dz", "dt": "ddt", "B": "dB", "C": "dC", "A": "dA", "D": "dD", "dt_bias": "ddt_bias",
+             "h0": "dh0", "conv_w": "dconv_w", "conv_b": "dconv_b", "conv_state_in": "dconv_state_in"}
+    for mode, sp in ((M1, True), (M2, True), (M2, False)):
+        if mode == M1:
+            d = W.mamba1_inputs(90, 1, tot, 3, 2, d_conv=3, dtype="f32", conv_bias=True, conv_state=True, nseqs=3)
+        else:
+            d = W.mamba2_inputs(91, 1, tot, 4, 2, 2, 2, d_conv=3, dtype="f32", conv_bias=True, conv_state=True, nseqs=3)
+        d = {k: (np.asarray(v, np.float64) if isinstance(v, np.ndarray) else v) for k, v in d.items()}
+        if not sp:                         # delta = dt + dt_bias directly: keep it small and positive
+            d["dt"] = np.abs(d["dt"]) * 0.1
+            d["dt_bias"] = np.full_like(d["dt_bias"], 0.01)
+        run = _m1_scan if mode == M1 else _m2_scan
+        y, hf, cs = run(d, mutant, cu_seqlens=cu, delta_softplus=sp)
+        rng = np.random.default_rng(92)
+        dy, dhf, dcs = rng.standard_normal(y.shape), rng.standard_normal(hf.shape), rng.standard_normal(cs.shape)
+
+        def loss():
+            y2, h2, c2 = run(d, 0, cu_seqlens=cu, delta_softplus=sp)
+            return float(np.sum(dy * y2) + np.sum(dhf * h2) + np.sum(dcs * c2))
+
+        g = oracle.scan_bwd(mode, d["x"], d["dt"], d["A"], d["B"], d["C"], dy, D=d["D"], z=d["z"], dt_bias=d["dt_bias"],
+                            h0=d["h0"], cu_seqlens=cu, conv_w=d["conv_w"], conv_b=d["conv_b"],
+                            conv_state_in=d["conv_state_in"], delta_softplus=sp, dh_final=dhf, dconv_state_out=dcs,
+                            mutant=mutant)
+        eps = 1e-6
+        for k, gk in names.items():
+            arr = d[k]
+            fd = np.zeros_like(arr)
+            for i in range(arr.size):
+                old = arr.flat[i]
+                arr.flat[i] = old + eps
+                lp = loss()
+                arr.flat[i] = old - eps
+                lm = loss()
+                arr.flat[i] = old
+                fd.flat[i] = (lp - lm) / (2 * eps)
+            _close(g[gk], fd, rtol=1e-6, atol=1e-9, what=f"mode {mode} softplus {sp}: {gk} vs finite differences")
+
+
 # ------------------------------------------------------------ conv pins
 def check_conv_impulse(mutant=0):
     """A unit impulse at t = 0 through a conv without activation returns each
@@ -478,4 +526,5 @@ ALL_CHECKS = [
     check_bruteforce_m2, check_split_invariance, check_m2_reduces_to_m1, check_prefill_equals_decode,
     check_decode_wide_conv_state, check_varlen_equals_per_sequence, check_conv_impulse, check_conv_width_one,
     check_conv_reformulations, check_fused_conv_matches_standalone, check_intermediate_states_are_prefix_states,
+    check_backward_matches_finite_differences,
 ]

@@ -363,3 +363,18 @@ def test_ssd_split_invariance():
         assert rel_err(np.concatenate([y1, y2], 1), y) <= 2e-2
         assert rel_err(h2, hf) <= 2e-2
         assert np.array_equal(c2, cs)
+
+
+def test_kernel_timing_counts_launches():
+    """ssm_kernel_timing brackets each call's dominant kernel with events on the call's stream."""
+    d = W.mamba1_inputs(901, 1, 96, 32, 16, dtype="bf16")
+    t = to_dev(d, "bf16")
+    ssm.kernel_time_ms()
+    ssm.kernel_timing(True)
+    gpu_scan(M1, t)
+    gpu_scan(M1, t)
+    ssm.kernel_timing(False)
+    ms, n = ssm.kernel_time_ms()
+    assert n == 2 and ms > 0.0
+    gpu_scan(M1, t)
+    assert ssm.kernel_time_ms() == (0.0, 0)

@@ -57,6 +57,7 @@ MUTANTS = {
     11: "softplus switch inverted",
     12: "skip term on the pre-conv x",
     13: "intermediate state recorded one token early",
+    14: "backward: dh not carried back through exp(delta A)",
 }
 
 
