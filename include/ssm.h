@@ -197,6 +197,34 @@ typedef struct ssm_update_args {
     int64_t nslots;           /* number of state / conv-state slots (>= batch when indices are NULL) */
 } ssm_update_args;
 
+/* Backward of ssm_scan_fwd: gradients of
+ *   L = sum(dy * y) + sum(dh_final * h_final) + sum(dconv_state_out * conv_state_out)
+ * with respect to every input of the forward call described by `fwd` (its
+ * y, h_final, conv_state_out and intermediate-state fields are ignored).
+ * The step h_t = exp(delta_t A) h_{t-1} + delta_t B_t x_t is differentiated
+ * as it stands, carrying dh back through exp(delta A) to the initial state
+ * ("Adding Initial Value Support to Selective Scan Forward Kernel",
+ * state-spaces/mamba issue 285, on the backward pass and dh0).
+ *
+ * Every gradient is fp32 and contiguous:
+ *   dx, dz [b][T][d_inner]; ddt [b][T][D or H]; dB, dC [b][T][G*N] (the raw,
+ *   pre-conv B / C); dA, dD, ddt_bias like A, D, dt_bias; dh0 [nseq][state];
+ *   dconv_w [conv_dim][K], dconv_b [conv_dim]; dconv_state_in [nseq][conv_dim][K-1].
+ * dx, dB, dC, ddt, dA, dh0 are required; dz is required when z is given; the
+ * others may be NULL when not wanted (dD needs D, ddt_bias needs dt_bias,
+ * dconv_* need the conv).  Every requested output is overwritten. */
+typedef struct ssm_scan_bwd_args {
+    ssm_scan_args fwd;
+    const void *dy; int64_t dy_batch_stride, dy_token_stride;   /* like y (dtype) */
+    const float *dh_final;          /* [nseq][state] or NULL */
+    const void *dconv_state_out;    /* [nseq][conv_dim][K-1] dtype, or NULL */
+    float *dx, *dz, *ddt, *dB, *dC;
+    float *dA, *dD, *ddt_bias;
+    float *dh0;
+    float *dconv_w, *dconv_b;
+    float *dconv_state_in;
+} ssm_scan_bwd_args;
+
 /* Library version and status text. */
 SSM_API int32_t ssm_abi_version(void);
 SSM_API const char *ssm_status_string(ssm_status s);
@@ -214,6 +242,13 @@ SSM_API size_t ssm_scan_workspace_size(const ssm_scan_args *args);
  * NULL when ssm_scan_workspace_size() is 0.  The workspace holds the device
  * error word (read it with ssm_workspace_error) and the varlen schedule. */
 SSM_API ssm_status ssm_scan_fwd(const ssm_scan_args *args, void *workspace, size_t ws_bytes, void *stream);
+
+/* Backward scan (see ssm_scan_bwd_args).  Needs a workspace of
+ * ssm_scan_bwd_workspace_size() bytes (device, 256-byte aligned): chunk-start
+ * state checkpoints of a recomputed forward pass and the fp32 accumulators of
+ * the grouped B / C gradients.  Supports dstate <= 256. */
+SSM_API size_t ssm_scan_bwd_workspace_size(const ssm_scan_bwd_args *args);
+SSM_API ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *args, void *workspace, size_t ws_bytes, void *stream);
 
 /* Decode update, in place on state and conv_state.  No workspace. */
 SSM_API ssm_status ssm_state_update(const ssm_update_args *args, void *stream);

@@ -72,6 +72,19 @@ class UpdateArgs(C.Structure):
     ]
 
 
+class ScanBwdArgs(C.Structure):
+    _fields_ = [
+        ("fwd", ScanArgs),
+        ("dy", _vp), ("dy_batch_stride", _i64), ("dy_token_stride", _i64),
+        ("dh_final", _vp), ("dconv_state_out", _vp),
+        ("dx", _vp), ("dz", _vp), ("ddt", _vp), ("dB", _vp), ("dC", _vp),
+        ("dA", _vp), ("dD", _vp), ("ddt_bias", _vp),
+        ("dh0", _vp),
+        ("dconv_w", _vp), ("dconv_b", _vp),
+        ("dconv_state_in", _vp),
+    ]
+
+
 # Every symbol the header declares, with its ctypes signature.
 SIGNATURES = {
     "ssm_abi_version": ([], _i32),
@@ -83,6 +96,8 @@ SIGNATURES = {
     "ssm_state_update": ([C.POINTER(UpdateArgs), _vp], _i32),
     "ssm_workspace_error": ([_vp, C.POINTER(_i32), _vp], _i32),
     "ssm_scan_fwd_noalloc": ([C.POINTER(ScanArgs), _vp], _i32),
+    "ssm_scan_bwd_workspace_size": ([C.POINTER(ScanBwdArgs)], C.c_size_t),
+    "ssm_scan_bwd": ([C.POINTER(ScanBwdArgs), _vp, C.c_size_t, _vp], _i32),
     "ssm_kernel_timing": ([_i32], _i32),
     "ssm_kernel_time_ms": ([C.POINTER(C.c_float), C.POINTER(_i32)], _i32),
 }

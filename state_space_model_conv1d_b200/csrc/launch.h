@@ -81,6 +81,10 @@ bool ssd_supported(const ssm_scan_args &a);     // shapes and 16-byte alignment:
 size_t ssd_workspace_bytes(const ssm_scan_args &a);
 cudaError_t launch_ssd(const ssm_scan_args &a, const SeqView &sv, void *ws_bc, cudaStream_t st);
 cudaError_t launch_state_update(const ssm_update_args &a, cudaStream_t st);
+// Backward scan: workspace bytes for the checkpoints and B / C accumulators
+// (after the error word and the varlen order), and its launcher.
+size_t scan_bwd_workspace_bytes(const ssm_scan_bwd_args &a);
+cudaError_t launch_scan_bwd(const ssm_scan_bwd_args &a, const SeqView &sv, void *ws, cudaStream_t st);
 
 // Device timing of the dominant kernel of a call (ssm_kernel_timing): a no-op
 // unless enabled; otherwise records one event before and one after on `st`.

@@ -1,0 +1,576 @@
+// scan_bwd.cu -- backward of the fused causal conv + selective scan.
+//
+// Gradients of L = sum(dy y) + sum(dh_final h_final) + sum(dconv_state_out
+// conv_state_out) for both forms.  The step
+//   h_t = a_t h_{t-1} + delta_t B_t xc_t,   a_t = exp(delta_t A),
+//   y_t = (C_t . h_t + D xc_t) silu(z_t)
+// is differentiated as it stands: with g = dL/dh_t,
+//   g += dy_t silu(z_t) C_t;  dB_t += g delta_t xc_t;  dxc_t += g . B_t delta_t;
+//   ddelta_t += g . (h_{t-1} a_t A + B_t xc_t);  dA += g h_{t-1} a_t delta_t;
+//   g *= a_t  (then the next token back), and dh0 is the g left after the
+// first token ("Adding Initial Value Support to Selective Scan Forward
+// Kernel", state-spaces/mamba issue 285: the backward carries dh back through
+// exp(delta A) to the initial state).  The conv gradients follow from
+// xc = silu(b + sum_k w_k u_{t-K+1+k}) with u before the sequence taken from
+// the carried conv state.
+//
+// Work layout (SIMT, correctness first): one CTA per (sequence, block of
+// channels) -- for Mamba-2 the block lies inside one head.  L lanes per
+// channel hold NS states each.  Pass A walks the sequence forward in chunks of
+// TC tokens and stores each chunk's start state in the workspace; pass B
+// walks the chunks backwards, recomputes the chunk's states from its
+// checkpoint into shared memory and runs the reverse recurrence.  Gradients
+// summed over channels (B, C and, for Mamba-2, delta and A) go through
+// shared-memory then global float atomics.  The Mamba-2 B / C conv backward
+// runs afterwards, once per (sequence, B / C channel), on the summed
+// gradients of the conv outputs.
+#include "common.cuh"
+#include "launch.h"
+
+namespace ssm {
+namespace {
+
+constexpr int kBT = 128;     // threads per CTA
+constexpr int kTCb = 16;     // tokens per chunk
+
+struct BwdArgs {
+    const void *x, *z, *dt, *B, *C;
+    int64_t x_bs, x_ts, z_bs, z_ts, dt_bs, dt_ts, B_bs, B_ts, C_bs, C_ts;
+    const float *A, *D, *dt_bias, *h0, *conv_w, *conv_b;
+    const void *conv_state_in;
+    const void *dy;
+    int64_t dy_bs, dy_ts;
+    const float *dh_final;
+    const void *dcs_out;
+    float *dx, *dz, *ddt, *dB, *dC, *dA, *dD, *ddt_bias, *dh0, *dconv_w, *dconv_b, *dcs_in;
+    float *ckpt;            // [slots][Dn][NP] chunk-start states
+    float *dBc, *dCc;       // Mamba-2: [b*T][G*N] gradients of the conv'd B / C
+    int64_t Dn, H, P, G, N, T, rows, slots_per_row;
+    int K, softplus, mode, L, CPB, NP, units_per_head;
+    SeqView sv;
+};
+
+SSM_DEVINL float sigmoidf_(float v) { return rcp(1.f + ex2(-v * kLog2e)); }
+SSM_DEVINL float dsilu(float v) {
+    const float s = sigmoidf_(v);
+    return s * (1.f + v * (1.f - s));
+}
+
+// sequence bounds of CTA row `si` (packed or batched)
+struct Seq {
+    int s;
+    int64_t start, len, row, slot0;
+};
+SSM_DEVINL Seq seq_bounds(const BwdArgs &a, int si) {
+    Seq q;
+    q.s = si;
+    q.start = 0; q.len = a.T; q.row = si;
+    if (a.sv.cu) {
+        const int64_t c0 = min(max((int64_t)a.sv.cu[si], (int64_t)0), a.T);
+        const int64_t c1 = min(max((int64_t)a.sv.cu[si + 1], c0), a.T);
+        q.start = c0; q.len = c1 - c0; q.row = 0;
+        q.slot0 = si + c0 / kTCb;              // disjoint per sequence (see the workspace sizing)
+    } else {
+        q.slot0 = (int64_t)si * a.slots_per_row;
+    }
+    return q;
+}
+
+template <typename T, int NS>
+__global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
+    extern __shared__ __align__(16) float smb[];
+    const int tid = threadIdx.x;
+    const int L = a.L, CPB = a.CPB, NP = a.NP, K = a.K;
+    const bool m1 = a.mode == SSM_MAMBA1;
+    const int j = tid / L, l = tid % L;
+    const Seq q = seq_bounds(a, blockIdx.y);
+    // channels of this CTA
+    int64_t hh, p0;
+    if (m1) { hh = 0; p0 = (int64_t)blockIdx.x * CPB; }
+    else { hh = blockIdx.x / a.units_per_head; p0 = (int64_t)(blockIdx.x % a.units_per_head) * CPB; }
+    const int64_t P = m1 ? a.Dn : a.P;
+    const int64_t pj = p0 + j;
+    const bool cvalid = j < CPB && pj < P;
+    const int64_t ch = m1 ? pj : hh * a.P + pj;            // x channel
+    const int64_t g = m1 ? 0 : hh / (a.H / a.G);
+    const int64_t N = a.N, Dn = a.Dn, GN = a.G * a.N;
+    const int64_t cdim = m1 ? Dn : Dn + 2 * GN;
+
+    // shared memory
+    float *hs = smb;                                         // [TC+1][kBT][NS]
+    float *xc = hs + (kTCb + 1) * kBT * NS;                  // [TC][CPB] each below
+    float *pre = xc + kTCb * CPB;
+    float *dl = pre + kTCb * CPB;
+    float *spd = dl + kTCb * CPB;
+    float *gate = spd + kTCb * CPB;
+    float *dgate = gate + kTCb * CPB;
+    float *dyv = dgate + kTCb * CPB;
+    float *dxc = dyv + kTCb * CPB;
+    float *Bt = dxc + kTCb * CPB;                            // [TC][NP]
+    float *Ct = Bt + kTCb * NP;
+    float *sdB = Ct + kTCb * NP;
+    float *sdC = sdB + kTCb * NP;
+    float *sddt = sdC + kTCb * NP;                           // [TC]
+    float *carry = sddt + kTCb;                              // [CPB][kMaxConvWidth]
+    float *dcw = carry + CPB * kMaxConvWidth;                // [CPB][kMaxConvWidth]
+
+    const T *xg = static_cast<const T *>(a.x);
+    const T *csi = static_cast<const T *>(a.conv_state_in);
+    // raw conv input of conv channel cc at position pos of the sequence (pos < 0: carried state)
+    auto raw_at = [&](const T *src, int64_t bs, int64_t ts, int64_t col, int64_t cc, int64_t pos) -> float {
+        if (pos >= 0) return Elem<T>::ld(src + q.row * bs + (q.start + pos) * ts + col);
+        const int64_t qq = pos + (K - 1);
+        return (csi && qq >= 0) ? Elem<T>::ld(csi + ((int64_t)q.s * cdim + cc) * (K - 1) + qq) : 0.f;
+    };
+    auto conv_pre = [&](const T *src, int64_t bs, int64_t ts, int64_t col, int64_t cc, int64_t pos) -> float {
+        float acc = a.conv_b ? a.conv_b[cc] : 0.f;
+        for (int k = 0; k < K; ++k) acc = fmaf(a.conv_w[cc * K + k], raw_at(src, bs, ts, col, cc, pos - (K - 1) + k), acc);
+        return acc;
+    };
+
+    const int nch = (int)((q.len + kTCb - 1) / kTCb);
+    auto stage = [&](int c) {
+        const int64_t t0 = (int64_t)c * kTCb;
+        const int nv = (int)min((int64_t)kTCb, q.len - t0);
+        for (int idx = tid; idx < kTCb * CPB; idx += kBT) {
+            const int t = idx / CPB, jj = idx % CPB;
+            const int64_t pp = p0 + jj;
+            float vxc = 0.f, vpre = 0.f, vdl = 0.f, vsp = 0.f, vg = 1.f, vdg = 0.f, vdy = 0.f;
+            if (t < nv && pp < P) {
+                const int64_t cc = m1 ? pp : hh * a.P + pp;
+                const int64_t tok = q.start + t0 + t;
+                if (K > 0) {
+                    vpre = conv_pre(xg, a.x_bs, a.x_ts, cc, cc, t0 + t);
+                    vxc = silu(vpre);
+                } else {
+                    vxc = Elem<T>::ld(xg + q.row * a.x_bs + tok * a.x_ts + cc);
+                }
+                const int64_t dcol = m1 ? cc : hh;
+                const float u = Elem<T>::ld(static_cast<const T *>(a.dt) + q.row * a.dt_bs + tok * a.dt_ts + dcol) +
+                                (a.dt_bias ? a.dt_bias[dcol] : 0.f);
+                vdl = a.softplus ? softplus(u) : u;
+                vsp = a.softplus ? sigmoidf_(u) : 1.f;
+                if (a.z) {
+                    const float zv = Elem<T>::ld(static_cast<const T *>(a.z) + q.row * a.z_bs + tok * a.z_ts + cc);
+                    vg = silu(zv);
+                    vdg = dsilu(zv);
+                }
+                vdy = Elem<T>::ld(static_cast<const T *>(a.dy) + q.row * a.dy_bs + tok * a.dy_ts + cc);
+            }
+            xc[t * CPB + jj] = vxc; pre[t * CPB + jj] = vpre; dl[t * CPB + jj] = vdl; spd[t * CPB + jj] = vsp;
+            gate[t * CPB + jj] = vg; dgate[t * CPB + jj] = vdg; dyv[t * CPB + jj] = vdy;
+        }
+        for (int idx = tid; idx < kTCb * NP; idx += kBT) {
+            const int t = idx / NP, n = idx % NP;
+            float vb = 0.f, vc = 0.f;
+            if (t < nv && n < N) {
+                const int64_t tok = q.start + t0 + t;
+                const T *Bs = static_cast<const T *>(a.B), *Cs = static_cast<const T *>(a.C);
+                if (m1 || K == 0) {
+                    vb = Elem<T>::ld(Bs + q.row * a.B_bs + tok * a.B_ts + g * N + n);
+                    vc = Elem<T>::ld(Cs + q.row * a.C_bs + tok * a.C_ts + g * N + n);
+                } else {
+                    vb = silu(conv_pre(Bs, a.B_bs, a.B_ts, g * N + n, Dn + g * N + n, t0 + t));
+                    vc = silu(conv_pre(Cs, a.C_bs, a.C_ts, g * N + n, Dn + GN + g * N + n, t0 + t));
+                }
+            }
+            Bt[t * NP + n] = vb;
+            Ct[t * NP + n] = vc;
+        }
+    };
+    auto A_of = [&](int e) -> float {
+        const int64_t n = (int64_t)l * NS + e;
+        if (n >= N || !cvalid) return 0.f;
+        return m1 ? a.A[ch * N + n] : a.A[hh];
+    };
+    float An[NS];
+#pragma unroll
+    for (int e = 0; e < NS; ++e) An[e] = A_of(e);
+
+    // ---- pass A: forward, storing chunk-start states
+    float h[NS];
+    const int64_t hbase = ((int64_t)q.s * Dn + ch) * N;
+#pragma unroll
+    for (int e = 0; e < NS; ++e) {
+        const int64_t n = (int64_t)l * NS + e;
+        h[e] = (cvalid && n < N && a.h0) ? a.h0[hbase + n] : 0.f;
+    }
+    for (int c = 0; c < nch; ++c) {
+        if (cvalid) {
+            float *dst = a.ckpt + ((q.slot0 + c) * Dn + ch) * NP + (int64_t)l * NS;
+#pragma unroll
+            for (int e = 0; e < NS; ++e) dst[e] = h[e];
+        }
+        __syncthreads();
+        stage(c);
+        __syncthreads();
+        const int nv = (int)min((int64_t)kTCb, q.len - (int64_t)c * kTCb);
+        if (cvalid)
+            for (int t = 0; t < nv; ++t) {
+                const float d = dl[t * CPB + j], xv = xc[t * CPB + j];
+#pragma unroll
+                for (int e = 0; e < NS; ++e) h[e] = fmaf(__expf(d * An[e]), h[e], d * Bt[t * NP + l * NS + e] * xv);
+            }
+    }
+
+    // ---- pass B: reverse
+    float gr[NS], dAa[NS];
+#pragma unroll
+    for (int e = 0; e < NS; ++e) {
+        const int64_t n = (int64_t)l * NS + e;
+        gr[e] = (cvalid && n < N && a.dh_final) ? a.dh_final[hbase + n] : 0.f;
+        dAa[e] = 0.f;
+    }
+    float dDa = 0.f, dbias_a = 0.f, dcb_a = 0.f;
+    if (tid < CPB)
+        for (int k = 0; k < kMaxConvWidth; ++k) { carry[tid * kMaxConvWidth + k] = 0.f; dcw[tid * kMaxConvWidth + k] = 0.f; }
+    const float Dv = (cvalid && a.D) ? a.D[m1 ? ch : hh] : 0.f;
+    const unsigned gmask = L >= 32 ? 0xffffffffu : (((1u << L) - 1u) << ((threadIdx.x & 31) / L * L));
+    auto lane_sum = [&](float v) {
+        for (int o = L / 2; o >= 1; o >>= 1) v += __shfl_xor_sync(gmask, v, o);
+        return v;
+    };
+    const T *dcso = static_cast<const T *>(a.dcs_out);
+
+    for (int c = nch - 1; c >= 0; --c) {
+        const int64_t t0 = (int64_t)c * kTCb;
+        const int nv = (int)min((int64_t)kTCb, q.len - t0);
+        __syncthreads();
+        stage(c);
+        for (int idx = tid; idx < kTCb * NP; idx += kBT) { sdB[idx] = 0.f; sdC[idx] = 0.f; }
+        if (tid < kTCb) sddt[tid] = 0.f;
+        __syncthreads();
+        // states of the chunk from its checkpoint
+        {
+            const float *src = a.ckpt + ((q.slot0 + c) * Dn + (cvalid ? ch : 0)) * NP + (int64_t)l * NS;
+#pragma unroll
+            for (int e = 0; e < NS; ++e) h[e] = cvalid ? src[e] : 0.f;
+#pragma unroll
+            for (int e = 0; e < NS; ++e) hs[tid * NS + e] = h[e];
+            for (int t = 0; t < nv; ++t) {
+                const float d = dl[t * CPB + (cvalid ? j : 0)], xv = cvalid ? xc[t * CPB + j] : 0.f;
+#pragma unroll
+                for (int e = 0; e < NS; ++e) {
+                    h[e] = fmaf(__expf(d * An[e]), h[e], d * Bt[t * NP + l * NS + e] * xv);
+                    hs[((t + 1) * kBT + tid) * NS + e] = h[e];
+                }
+            }
+        }
+        // reverse recurrence over the chunk
+        for (int t = nv - 1; t >= 0; --t) {
+            const int jj = cvalid ? j : 0;
+            const float d = dl[t * CPB + jj], xv = xc[t * CPB + jj];
+            float yb = 0.f;
+#pragma unroll
+            for (int e = 0; e < NS; ++e) yb = fmaf(Ct[t * NP + l * NS + e], hs[((t + 1) * kBT + tid) * NS + e], yb);
+            yb = lane_sum(yb) + Dv * xv;
+            const float dyt = dyv[t * CPB + jj];
+            const float dyb = dyt * gate[t * CPB + jj];
+            float dxp = 0.f, ddp = 0.f;
+#pragma unroll
+            for (int e = 0; e < NS; ++e) {
+                const int n = l * NS + e;
+                const float hc = hs[((t + 1) * kBT + tid) * NS + e], hp = hs[(t * kBT + tid) * NS + e];
+                if (cvalid) atomicAdd(&sdC[t * NP + n], dyb * hc);
+                gr[e] = fmaf(dyb, Ct[t * NP + n], gr[e]);
+                const float av = __expf(d * An[e]);
+                if (cvalid) atomicAdd(&sdB[t * NP + n], gr[e] * d * xv);
+                dxp = fmaf(gr[e] * d, Bt[t * NP + n], dxp);
+                ddp = fmaf(gr[e], hp * av * An[e] + Bt[t * NP + n] * xv, ddp);
+                dAa[e] = fmaf(gr[e], hp * av * d, dAa[e]);
+                gr[e] *= av;
+            }
+            dxp = lane_sum(dxp);
+            ddp = lane_sum(ddp);
+            if (cvalid && l == 0) {
+                const int64_t tok = q.start + t0 + t;
+                const int64_t rt = q.row * a.T + tok;
+                if (a.z) a.dz[rt * Dn + ch] = dyt * yb * dgate[t * CPB + j];
+                dDa = fmaf(dyb, xv, dDa);
+                dxc[t * CPB + j] = dxp + dyb * Dv;
+                const float dd = ddp * spd[t * CPB + j];
+                if (m1) {
+                    a.ddt[rt * Dn + ch] = dd;
+                    dbias_a += dd;
+                } else {
+                    atomicAdd(&sddt[t], dd);
+                }
+            }
+        }
+        __syncthreads();
+        // chunk sums over this CTA's channels -> global
+        for (int idx = tid; idx < kTCb * NP; idx += kBT) {
+            const int t = idx / NP, n = idx % NP;
+            if (t < nv && n < N) {
+                const int64_t rt = q.row * a.T + q.start + t0 + t;
+                if (m1) {
+                    atomicAdd(&a.dB[rt * N + n], sdB[idx]);
+                    atomicAdd(&a.dC[rt * N + n], sdC[idx]);
+                } else {
+                    atomicAdd(&a.dBc[rt * GN + g * N + n], sdB[idx]);
+                    atomicAdd(&a.dCc[rt * GN + g * N + n], sdC[idx]);
+                }
+            }
+        }
+        if (!m1 && tid < nv) {
+            const int64_t rt = q.row * a.T + q.start + t0 + tid;
+            atomicAdd(&a.ddt[rt * a.H + hh], sddt[tid]);
+            dbias_a += sddt[tid];                 // summed below by threads < kTCb
+        }
+        // conv backward of this chunk's x channels (one thread per channel)
+        if (tid < CPB && p0 + tid < P) {
+            const int jj = tid;
+            const int64_t cc = m1 ? p0 + jj : hh * a.P + p0 + jj;
+            float *cr = carry + jj * kMaxConvWidth;
+            float *dw = dcw + jj * kMaxConvWidth;
+            // dpre of the chunk, in place over dxc
+            for (int t = 0; t < nv; ++t) {
+                const float dv = dxc[t * CPB + jj];
+                dxc[t * CPB + jj] = K > 0 ? dv * dsilu(pre[t * CPB + jj]) : dv;
+            }
+            auto dp_at = [&](int64_t x) -> float {           // dpre at sequence position x >= t0
+                if (x < t0 + nv) return dxc[(x - t0) * CPB + jj];
+                const int64_t i = x - (t0 + nv);
+                return (x < q.len && i < kMaxConvWidth) ? cr[i] : 0.f;
+            };
+            if (K > 0) {
+                for (int t = 0; t < nv; ++t) {
+                    const float dp = dxc[t * CPB + jj];
+                    dcb_a += dp;
+                    for (int k = 0; k < K; ++k) dw[k] += dp * raw_at(xg, a.x_bs, a.x_ts, cc, cc, t0 + t - (K - 1) + k);
+                }
+            }
+            for (int t = nv - 1; t >= 0; --t) {
+                const int64_t pos = t0 + t;
+                float v;
+                if (K > 0) {
+                    v = 0.f;
+                    for (int k = 0; k < K; ++k) v = fmaf(dp_at(pos + (K - 1) - k), a.conv_w[cc * K + k], v);
+                } else {
+                    v = dxc[t * CPB + jj];
+                }
+                if (dcso && K > 1 && pos >= q.len - (K - 1))
+                    v += Elem<T>::ld(dcso + ((int64_t)q.s * cdim + cc) * (K - 1) + (pos - (q.len - (K - 1))));
+                a.dx[(q.row * a.T + q.start + pos) * Dn + cc] = v;
+            }
+            // new carry: dpre at positions t0 .. t0+K-2
+            float nc[kMaxConvWidth];
+            for (int i = 0; i < kMaxConvWidth; ++i) nc[i] = (i < K - 1) ? dp_at(t0 + i) : 0.f;
+            for (int i = 0; i < kMaxConvWidth; ++i) cr[i] = nc[i];
+        }
+    }
+    __syncthreads();
+    // carried-state gradients, dh0, and the sums over the whole sequence
+    if (tid < CPB && p0 + tid < P && K > 1 && a.dcs_in) {
+        const int jj = tid;
+        const int64_t cc = m1 ? p0 + jj : hh * a.P + p0 + jj;
+        const float *cr = carry + jj * kMaxConvWidth;
+        for (int qq = 0; qq < K - 1; ++qq) {
+            const int64_t pos = qq - (K - 1);                  // history position
+            float v = 0.f;
+            for (int k = 0; k < K; ++k) {
+                const int64_t x = pos + (K - 1) - k;
+                if (x >= 0 && x < q.len && x < K - 1) v = fmaf(cr[x], a.conv_w[cc * K + k], v);
+            }
+            if (dcso && pos >= q.len - (K - 1))
+                v += Elem<T>::ld(dcso + ((int64_t)q.s * cdim + cc) * (K - 1) + (pos - (q.len - (K - 1))));
+            a.dcs_in[((int64_t)q.s * cdim + cc) * (K - 1) + qq] = v;
+        }
+    }
+    if (tid < CPB && p0 + tid < P && K > 0) {
+        const int64_t cc = m1 ? p0 + tid : hh * a.P + p0 + tid;
+        if (a.dconv_w)
+            for (int k = 0; k < K; ++k) atomicAdd(&a.dconv_w[cc * K + k], dcw[tid * kMaxConvWidth + k]);
+        if (a.dconv_b) atomicAdd(&a.dconv_b[cc], dcb_a);
+    }
+    if (cvalid) {
+#pragma unroll
+        for (int e = 0; e < NS; ++e) {
+            const int64_t n = (int64_t)l * NS + e;
+            if (n < N) {
+                a.dh0[hbase + n] = gr[e];
+                if (m1) atomicAdd(&a.dA[ch * N + n], dAa[e]);
+            }
+        }
+        if (!m1) {
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < NS; ++e) s += dAa[e];
+            atomicAdd(&a.dA[hh], s);
+        }
+        if (l == 0) {
+            if (a.dD && a.D) atomicAdd(&a.dD[m1 ? ch : hh], dDa);
+            if (m1 && a.ddt_bias && a.dt_bias) atomicAdd(&a.ddt_bias[ch], dbias_a);
+        }
+    }
+    if (!m1 && tid < kTCb && a.ddt_bias && a.dt_bias) atomicAdd(&a.ddt_bias[hh], dbias_a);
+}
+
+// Mamba-2 B / C conv backward: one thread per (sequence, B / C channel), walking
+// the sequence backwards over the summed gradients of the conv outputs.
+template <typename T>
+__global__ void bc_conv_bwd_kernel(const BwdArgs a) {
+    const int64_t GN = a.G * a.N, Dn = a.Dn, cdim = Dn + 2 * GN;
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int nseq = a.sv.cu ? a.sv.nseqs : (int)a.rows;
+    if (i >= (int64_t)nseq * 2 * GN) return;
+    const int si = (int)(i / (2 * GN));
+    const int64_t cc2 = i % (2 * GN);
+    const int which = (int)(cc2 / GN);
+    const int64_t col = cc2 % GN;
+    const int64_t cc = Dn + which * GN + col;                 // conv channel
+    const Seq q = seq_bounds(a, si);
+    const int K = a.K;
+    const T *src = static_cast<const T *>(which ? a.C : a.B);
+    const int64_t bs = which ? a.C_bs : a.B_bs, ts = which ? a.C_ts : a.B_ts;
+    const float *gin = which ? a.dCc : a.dBc;
+    float *gout = which ? a.dC : a.dB;
+    const T *csi = static_cast<const T *>(a.conv_state_in);
+    const T *dcso = static_cast<const T *>(a.dcs_out);
+    auto raw_at = [&](int64_t pos) -> float {
+        if (pos >= 0) return Elem<T>::ld(src + q.row * bs + (q.start + pos) * ts + col);
+        const int64_t qq = pos + (K - 1);
+        return (csi && qq >= 0) ? Elem<T>::ld(csi + ((int64_t)q.s * cdim + cc) * (K - 1) + qq) : 0.f;
+    };
+    auto dout_at = [&](int64_t pos) -> float { return gin[(q.row * a.T + q.start + pos) * GN + col]; };
+    auto dcso_at = [&](int64_t pos) -> float {
+        return (dcso && K > 1 && pos >= q.len - (K - 1))
+                   ? Elem<T>::ld(dcso + ((int64_t)q.s * cdim + cc) * (K - 1) + (pos - (q.len - (K - 1))))
+                   : 0.f;
+    };
+    if (K == 0) {
+        for (int64_t pos = 0; pos < q.len; ++pos) gout[(q.row * a.T + q.start + pos) * GN + col] = dout_at(pos);
+        return;
+    }
+    float w[kMaxConvWidth], dw[kMaxConvWidth], ring[kMaxConvWidth];   // ring: dpre at pos+1 .. pos+K-1
+    for (int k = 0; k < kMaxConvWidth; ++k) { w[k] = k < K ? a.conv_w[cc * K + k] : 0.f; dw[k] = 0.f; ring[k] = 0.f; }
+    const float bias = a.conv_b ? a.conv_b[cc] : 0.f;
+    float db = 0.f;
+    for (int64_t pos = q.len - 1; pos >= -(int64_t)(K - 1); --pos) {
+        float dp = 0.f;
+        if (pos >= 0) {
+            float pre = bias;
+            for (int k = 0; k < K; ++k) pre = fmaf(w[k], raw_at(pos - (K - 1) + k), pre);
+            dp = dout_at(pos) * dsilu(pre);
+            db += dp;
+            for (int k = 0; k < K; ++k) dw[k] += dp * raw_at(pos - (K - 1) + k);
+        }
+        // d raw(pos) = sum_k dpre(pos + K-1-k) w[k]; dpre(pos) is dp, dpre(pos + m) is ring[m-1]
+        float v = dp * w[K - 1];
+        for (int k = 0; k + 1 < K; ++k) v = fmaf(ring[K - 2 - k], w[k], v);
+        v += dcso_at(pos);
+        if (pos >= 0) gout[(q.row * a.T + q.start + pos) * GN + col] = v;
+        else if (a.dcs_in) a.dcs_in[((int64_t)q.s * cdim + cc) * (K - 1) + (pos + (K - 1))] = v;
+        for (int m = kMaxConvWidth - 1; m >= 1; --m) ring[m] = ring[m - 1];
+        ring[0] = dp;
+    }
+    if (a.dconv_w)
+        for (int k = 0; k < K; ++k) atomicAdd(&a.dconv_w[cc * K + k], dw[k]);
+    if (a.dconv_b) atomicAdd(&a.dconv_b[cc], db);
+}
+
+}  // namespace
+
+// Lanes per channel and states per lane for dstate N.
+static void bwd_layout(int64_t N, int *L, int *NS) {
+    *NS = N > 128 ? 8 : 4;
+    int l = 1;
+    while (l * *NS < N) l *= 2;
+    *L = l;
+}
+
+size_t scan_bwd_workspace_bytes(const ssm_scan_bwd_args &b) {
+    const ssm_scan_args &s = b.fwd;
+    int L, NS;
+    bwd_layout(s.dstate, &L, &NS);
+    const int64_t NP = (int64_t)L * NS;
+    const int64_t nseq = s.cu_seqlens ? s.nseqs : s.batch;
+    const int64_t slots = s.cu_seqlens ? (int64_t)nseq + (s.seqlen + kTCb - 1) / kTCb + 1
+                                       : s.batch * ((s.seqlen + kTCb - 1) / kTCb);
+    size_t bytes = ((size_t)slots * (size_t)s.d_inner * (size_t)NP * 4 + 255) / 256 * 256;
+    if (s.mode == SSM_MAMBA2)
+        bytes += 2 * (((size_t)s.batch * (size_t)s.seqlen * (size_t)(s.ngroups * s.dstate) * 4 + 255) / 256 * 256);
+    return bytes;
+}
+
+cudaError_t launch_scan_bwd(const ssm_scan_bwd_args &b, const SeqView &sv, void *ws, cudaStream_t st) {
+    const ssm_scan_args &s = b.fwd;
+    const bool m1 = s.mode == SSM_MAMBA1;
+    int L, NS;
+    bwd_layout(s.dstate, &L, &NS);
+    BwdArgs a;
+    a.x = s.x; a.z = s.z; a.dt = s.dt; a.B = s.B; a.C = s.C;
+    a.x_bs = s.x_batch_stride; a.x_ts = s.x_token_stride; a.z_bs = s.z_batch_stride; a.z_ts = s.z_token_stride;
+    a.dt_bs = s.dt_batch_stride; a.dt_ts = s.dt_token_stride; a.B_bs = s.B_batch_stride; a.B_ts = s.B_token_stride;
+    a.C_bs = s.C_batch_stride; a.C_ts = s.C_token_stride;
+    a.A = s.A; a.D = s.D; a.dt_bias = s.dt_bias; a.h0 = s.h0; a.conv_w = s.conv_w; a.conv_b = s.conv_b;
+    a.conv_state_in = s.conv_state_in;
+    a.dy = b.dy; a.dy_bs = b.dy_batch_stride; a.dy_ts = b.dy_token_stride;
+    a.dh_final = b.dh_final; a.dcs_out = b.dconv_state_out;
+    a.dx = b.dx; a.dz = b.dz; a.ddt = b.ddt; a.dB = b.dB; a.dC = b.dC; a.dA = b.dA; a.dD = b.dD;
+    a.ddt_bias = b.ddt_bias; a.dh0 = b.dh0; a.dconv_w = b.dconv_w; a.dconv_b = b.dconv_b; a.dcs_in = b.dconv_state_in;
+    a.Dn = s.d_inner; a.N = s.dstate; a.T = s.seqlen; a.rows = s.batch;
+    a.H = m1 ? s.d_inner : s.nheads; a.P = m1 ? 1 : s.headdim; a.G = m1 ? 1 : s.ngroups;
+    a.slots_per_row = (s.seqlen + kTCb - 1) / kTCb;
+    a.K = (int)s.d_conv; a.softplus = s.delta_softplus; a.mode = s.mode;
+    a.L = L; a.NP = L * NS; a.CPB = kBT / L;
+    a.units_per_head = m1 ? 0 : (int)((s.headdim + a.CPB - 1) / a.CPB);
+    a.sv = sv;
+    const int64_t nseq = s.cu_seqlens ? s.nseqs : s.batch;
+    const int64_t slots = s.cu_seqlens ? nseq + (s.seqlen + kTCb - 1) / kTCb + 1 : s.batch * a.slots_per_row;
+    char *w = static_cast<char *>(ws);
+    a.ckpt = reinterpret_cast<float *>(w);
+    w += ((size_t)slots * (size_t)s.d_inner * (size_t)a.NP * 4 + 255) / 256 * 256;
+    const size_t bc_bytes = (size_t)s.batch * (size_t)s.seqlen * (size_t)(a.G * s.dstate) * 4;
+    a.dBc = a.dCc = nullptr;
+    if (!m1) {
+        a.dBc = reinterpret_cast<float *>(w);
+        a.dCc = reinterpret_cast<float *>(w + (bc_bytes + 255) / 256 * 256);
+    }
+    // accumulated outputs start at zero
+    auto zero = [&](void *p, size_t bytes) { return p ? cudaMemsetAsync(p, 0, bytes, st) : cudaSuccess; };
+    const int64_t K = s.d_conv, cdim = m1 ? s.d_inner : s.d_inner + 2 * a.G * s.dstate;
+    cudaError_t e;
+    if ((e = zero(b.dA, (size_t)(m1 ? s.d_inner * s.dstate : s.nheads) * 4)) != cudaSuccess) return e;
+    if ((e = zero(b.dD, (size_t)a.H * 4)) != cudaSuccess) return e;
+    if ((e = zero(b.ddt_bias, (size_t)a.H * 4)) != cudaSuccess) return e;
+    if (K > 0) {
+        if ((e = zero(b.dconv_w, (size_t)(cdim * K) * 4)) != cudaSuccess) return e;
+        if ((e = zero(b.dconv_b, (size_t)cdim * 4)) != cudaSuccess) return e;
+    }
+    if (m1) {
+        if ((e = zero(b.dB, bc_bytes)) != cudaSuccess) return e;
+        if ((e = zero(b.dC, bc_bytes)) != cudaSuccess) return e;
+    } else {
+        if ((e = zero(b.ddt, (size_t)s.batch * (size_t)s.seqlen * (size_t)s.nheads * 4)) != cudaSuccess) return e;
+        if ((e = zero(a.dBc, bc_bytes)) != cudaSuccess) return e;
+        if ((e = zero(a.dCc, bc_bytes)) != cudaSuccess) return e;
+    }
+    const size_t smem = (size_t)((kTCb + 1) * kBT * NS + 8 * kTCb * a.CPB + 4 * kTCb * a.NP + kTCb +
+                                 2 * a.CPB * kMaxConvWidth) * 4;
+    const unsigned gx = m1 ? (unsigned)((s.d_inner + a.CPB - 1) / a.CPB) : (unsigned)(s.nheads * a.units_per_head);
+    dim3 grid(gx, (unsigned)nseq);
+    if (nseq > 0) {
+        auto run = [&](auto kern) -> cudaError_t {
+            cudaError_t ee = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (ee != cudaSuccess) return ee;
+            timing_begin(st);
+            kern<<<grid, kBT, smem, st>>>(a);
+            timing_end(st);
+            return cudaGetLastError();
+        };
+        if (s.dtype == SSM_BF16) e = NS == 4 ? run(scan_bwd_kernel<__nv_bfloat16, 4>) : run(scan_bwd_kernel<__nv_bfloat16, 8>);
+        else e = NS == 4 ? run(scan_bwd_kernel<float, 4>) : run(scan_bwd_kernel<float, 8>);
+        if (e != cudaSuccess) return e;
+        if (!m1) {
+            const int64_t n = nseq * 2 * a.G * s.dstate;
+            const unsigned blocks = (unsigned)((n + 127) / 128);
+            if (s.dtype == SSM_BF16) bc_conv_bwd_kernel<__nv_bfloat16><<<blocks, 128, 0, st>>>(a);
+            else bc_conv_bwd_kernel<float><<<blocks, 128, 0, st>>>(a);
+            e = cudaGetLastError();
+        }
+    }
+    return e;
+}
+
+}  // namespace ssm

@@ -199,6 +199,58 @@ WsPlan plan_workspace(const ssm_scan_args *a) {
 }
 }  // namespace
 
+namespace {
+// The backward validates its forward description with y standing in as dy
+// (same shape, strides and dtype), then its own outputs.
+ssm_status validate_bwd(const ssm_scan_bwd_args *b) {
+    if (!b) return SSM_ERR_INVALID_ARG;
+    ssm_scan_args f = b->fwd;
+    f.y = const_cast<void *>(b->dy);
+    f.y_batch_stride = b->dy_batch_stride;
+    f.y_token_stride = b->dy_token_stride;
+    f.state_interval = 0;
+    SSM_TRY(validate_scan(&f));
+    if (!b->dx || !b->ddt || !b->dB || !b->dC || !b->dA || !b->dh0) return SSM_ERR_INVALID_ARG;
+    if (f.z && !b->dz) return SSM_ERR_INVALID_ARG;
+    const float *outs[] = {b->dx, b->dz, b->ddt, b->dB, b->dC, b->dA, b->dD, b->ddt_bias, b->dh0,
+                           b->dconv_w, b->dconv_b, b->dconv_state_in, b->dh_final};
+    for (const float *o : outs)
+        if (!aligned(o, 4)) return SSM_ERR_ALIGNMENT;
+    if (!aligned(b->dconv_state_out, esize(f.dtype))) return SSM_ERR_ALIGNMENT;
+    return SSM_OK;
+}
+size_t bwd_ws_prefix(const ssm_scan_args &f) {
+    return ssm::kWsOrderOffset + (f.cu_seqlens ? ssm::order_bytes(f.nseqs) : 0);
+}
+}  // namespace
+
+size_t ssm_scan_bwd_workspace_size(const ssm_scan_bwd_args *args) {
+    if (!args) return 0;
+    const ssm_scan_args &f = args->fwd;
+    if (f.batch < 0 || f.seqlen < 0 || f.nseqs < 0 || f.ngroups < 0 || f.dstate < 1 || f.d_inner < 1) return 0;
+    return bwd_ws_prefix(f) + ssm::scan_bwd_workspace_bytes(*args);
+}
+
+ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *args, void *workspace, size_t ws_bytes, void *stream) {
+    SSM_TRY(validate_bwd(args));
+    const ssm_scan_args &f = args->fwd;
+    const cudaStream_t st = (cudaStream_t)stream;
+    const size_t need = bwd_ws_prefix(f) + ssm::scan_bwd_workspace_bytes(*args);
+    char *ws = static_cast<char *>(workspace);
+    if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return SSM_ERR_WORKSPACE;
+    ssm::SeqView sv{nullptr, nullptr, reinterpret_cast<int32_t *>(ws + ssm::kWsErrorOffset), (int)f.batch};
+    if (f.cu_seqlens) {
+        sv.cu = f.cu_seqlens;
+        sv.nseqs = f.nseqs;
+        // validates cu_seqlens into the error word (the schedule it also writes is not used here)
+        SSM_TRY(cuda_status(ssm::launch_varlen_plan(f.cu_seqlens, f.nseqs, f.seqlen, sv.err,
+                                                    reinterpret_cast<int32_t *>(ws + ssm::kWsOrderOffset), st)));
+    } else {
+        SSM_TRY(cuda_status(cudaMemsetAsync(sv.err, 0, sizeof(int32_t), st)));
+    }
+    return cuda_status(ssm::launch_scan_bwd(*args, sv, ws + bwd_ws_prefix(f), st));
+}
+
 size_t ssm_scan_workspace_size(const ssm_scan_args *args) {
     if (!args || args->batch < 0 || args->seqlen < 0 || args->nseqs < 0 || args->ngroups < 0 || args->dstate < 0)
         return 0;

@@ -47,7 +47,7 @@ def test_struct_layouts_match_header(tmp_path):
     with the ctypes mirror."""
     probes = []
     for cname, py in (("ssm_conv_args", _abi.ConvArgs), ("ssm_scan_args", _abi.ScanArgs),
-                      ("ssm_update_args", _abi.UpdateArgs)):
+                      ("ssm_update_args", _abi.UpdateArgs), ("ssm_scan_bwd_args", _abi.ScanBwdArgs)):
         probes.append(f'printf("{cname} sizeof %zu\\n", sizeof({cname}));')
         for fname, _ in py._fields_:
             probes.append(f'printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
@@ -61,7 +61,7 @@ def test_struct_layouts_match_header(tmp_path):
         c, f, v = line.split()
         got[(c, f)] = int(v)
     for cname, py in (("ssm_conv_args", _abi.ConvArgs), ("ssm_scan_args", _abi.ScanArgs),
-                      ("ssm_update_args", _abi.UpdateArgs)):
+                      ("ssm_update_args", _abi.UpdateArgs), ("ssm_scan_bwd_args", _abi.ScanBwdArgs)):
         assert got[(cname, "sizeof")] == C.sizeof(py), cname
         for fname, _ in py._fields_:
             assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
