@@ -193,7 +193,33 @@ class Job:
                 wrote += sum(self.inter[k].numel() * self.inter[k].element_size() for k in ("inter_states", "inter_conv"))
             self.bytes_per_step = read + wrote
             self.units = self.tokens
-            if mode == ssm.MAMBA1:
+            self.bwd = None
+            if w.backward:
+                # upstream gradients of y and h_final; the step is ssm_scan_bwd, whose fp32
+                # gradients of every input are what it writes
+                rng = np.random.default_rng(w.seed + 7)
+                dy = torch.from_numpy(rng.standard_normal(tuple(x.shape)).astype(np.float32)).to(bf)
+                self.host["dy"] = dy.pin_memory()
+                self.t["dy"] = self.host["dy"].to(dev)
+                self.t["dh_final"] = torch.from_numpy(rng.standard_normal(tuple(self.hf.shape)).astype(np.float32)).to(dev)
+                self.bwd = ssm.scan_bwd(mode, x, t["dt"], t["A"], t["B"], t["C"], self.t["dy"], D=t["D"], z=t["z"],
+                                        dt_bias=t["dt_bias"], h0=t["h0"], cu_seqlens=t.get("cu_seqlens"),
+                                        conv_w=t["conv_w"], conv_b=t["conv_b"], conv_state_in=t["conv_state_in"],
+                                        dh_final=self.t["dh_final"])
+                self.bwd_ws = torch.empty(max(1, ssm.ops.scan_bwd_workspace_size(
+                    mode, x, t["dt"], t["A"], t["B"], t["C"], self.t["dy"], cu_seqlens=t.get("cu_seqlens"),
+                    conv_w=t["conv_w"])), dtype=torch.uint8, device=dev)
+                read = sum(v.numel() * v.element_size() for k, v in self.t.items() if v is not None and k != "cu_seqlens")
+                wrote = sum(v.numel() * v.element_size() for v in self.bwd.values() if v is not None)
+                self.bytes_per_step = read + wrote
+                self.y = self.bwd["dx"]                       # what the end-to-end leg copies back
+            if w.backward:
+                # executed exps: the checkpoint pass, the per-chunk recompute and the reverse step
+                self.kernel, self.sources = "scan_bwd_kernel", ("scan_bwd.cu",)
+                self.mufu = 3 * x.shape[0] * x.shape[1] * x.shape[2] * t["B"].shape[2]
+                self.flops = None
+                self.launches_per_step = 1 + (1 if mode == ssm.MAMBA2 else 0)
+            elif mode == ssm.MAMBA1:
                 self.kernel, self.sources = "scan_m1_kernel", ("scan_m1.cu",)
                 self.mufu = x.shape[0] * x.shape[1] * x.shape[2] * t["B"].shape[2]
                 self.flops = None
@@ -250,6 +276,12 @@ class Job:
                              t["C"][i], D=t["D"], z=t["z"][i], dt_bias=t["dt_bias"], conv_w=t["conv_w"],
                              conv_b=t["conv_b"], y=self.y)
             return
+        if self.bwd is not None:
+            ssm.scan_bwd(self.mode, t["x"], t["dt"], t["A"], t["B"], t["C"], t["dy"], D=t["D"], z=t["z"],
+                         dt_bias=t["dt_bias"], h0=t["h0"], cu_seqlens=t.get("cu_seqlens"), conv_w=t["conv_w"],
+                         conv_b=t["conv_b"], conv_state_in=t["conv_state_in"], dh_final=t["dh_final"],
+                         workspace=self.bwd_ws, out=self.bwd)
+            return
         ssm.scan_fwd(self.mode, t["x"], t["dt"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"], dt_bias=t["dt_bias"],
                      h0=t["h0"], cu_seqlens=t.get("cu_seqlens"), conv_w=t["conv_w"], conv_b=t["conv_b"],
                      conv_state_in=t["conv_state_in"], y=self.y, h_final=self.hf, conv_state_out=self.cso,
@@ -265,7 +297,7 @@ class Job:
                 t[k][i].copy_(self.host[k][i], non_blocking=True)
                 h2d += self.host[k][i].numel() * self.host[k][i].element_size()
         else:
-            for k in ("x", "z", "dt", "B", "C", "h0"):
+            for k in ("x", "z", "dt", "B", "C", "h0", "dy"):
                 if self.host.get(k) is not None:
                     t[k].copy_(self.host[k], non_blocking=True)
                     h2d += self.host[k].numel() * self.host[k].element_size()
@@ -432,6 +464,16 @@ def oracle_sample(w: W.Workload, target_s: float):
     (all channels / heads), as many as fit the time budget."""
     import oracle
     cores = os.cpu_count() or 1
+    if w.kind == "mamba1" and w.backward:
+        # the backward keeps every step's state: one batch row (all channels)
+        nch = w.d_inner
+        ww = W.Workload(**{**w.__dict__, "batch": 1, "d_inner": nch})
+        d = W.workload_inputs(ww)
+        dy = np.random.default_rng(w.seed + 7).standard_normal(d["x"].shape)
+        run = lambda: oracle.scan_bwd(oracle.MAMBA1, d["x"], d["dt"], d["A"], d["B"], d["C"], dy, D=d["D"], z=d["z"],
+                                      dt_bias=d["dt_bias"], h0=d["h0"], conv_w=d["conv_w"])
+        return (run, w.seqlen * nch / w.d_inner, 1,
+                f"1 of {w.batch} batch rows x {w.seqlen} tokens, all {w.d_inner} channels")
     if w.kind == "mamba1":
         nrows = min(w.batch, max(1, cores))
         ww = W.Workload(**{**w.__dict__, "batch": nrows})

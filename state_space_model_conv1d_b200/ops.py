@@ -303,13 +303,14 @@ def kernel_time_ms():
 
 def scan_bwd(mode, x, dt, A, B, C_, dy, *, D=None, z=None, dt_bias=None, h0=None, cu_seqlens=None, conv_w=None,
              conv_b=None, conv_state_in=None, delta_softplus=True, dh_final=None, dconv_state_out=None,
-             workspace=None, stream=None):
+             workspace=None, out=None, stream=None):
     """Backward of :func:`scan_fwd`: gradients of sum(dy*y) + sum(dh_final*h_final)
     + sum(dconv_state_out*conv_state_out) with respect to every input.
 
     Returns a dict of fp32 CUDA tensors shaped like the inputs: ``dx, dz, ddt,
     dB, dC`` (raw, before the conv), ``dA, dD, ddt_bias, dh0, dconv_w, dconv_b,
-    dconv_state_in`` (None where the input is None).
+    dconv_state_in`` (None where the input is None).  ``out`` (such a dict from
+    an earlier call with the same shapes) is filled instead of allocating.
     """
     _need(dy, "dy", x.dtype)
     nseq = x.shape[0] if cu_seqlens is None else cu_seqlens.numel() - 1
@@ -322,12 +323,13 @@ def scan_bwd(mode, x, dt, A, B, C_, dy, *, D=None, z=None, dt_bias=None, h0=None
     dev = x.device
     f32 = lambda shape: torch.empty(shape, dtype=torch.float32, device=dev)
     K = 0 if conv_w is None else conv_w.shape[1]
-    out = dict(dx=f32(x.shape), dz=None if z is None else f32(z.shape), ddt=f32(dt.shape), dB=f32(B.shape),
-               dC=f32(C_.shape), dA=f32(A.shape), dD=None if D is None else f32(D.shape),
-               ddt_bias=None if dt_bias is None else f32(dt_bias.shape), dh0=f32(hshape),
-               dconv_w=None if conv_w is None else f32(conv_w.shape),
-               dconv_b=None if conv_b is None or conv_w is None else f32(conv_b.shape),
-               dconv_state_in=f32((nseq, cdim, K - 1)) if K > 1 else None)
+    if out is None:
+        out = dict(dx=f32(x.shape), dz=None if z is None else f32(z.shape), ddt=f32(dt.shape), dB=f32(B.shape),
+                   dC=f32(C_.shape), dA=f32(A.shape), dD=None if D is None else f32(D.shape),
+                   ddt_bias=None if dt_bias is None else f32(dt_bias.shape), dh0=f32(hshape),
+                   dconv_w=None if conv_w is None else f32(conv_w.shape),
+                   dconv_b=None if conv_b is None or conv_w is None else f32(conv_b.shape),
+                   dconv_state_in=f32((nseq, cdim, K - 1)) if K > 1 else None)
     b = _abi.ScanBwdArgs()
     b.fwd = _scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, h0, None, cu_seqlens, conv_w, conv_b, conv_state_in,
                        None, dy, delta_softplus, 0)
@@ -345,3 +347,12 @@ def scan_bwd(mode, x, dt, A, B, C_, dy, *, D=None, z=None, dt_bias=None, h0=None
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     _abi.check(l.ssm_scan_bwd(C.byref(b), _p(workspace), workspace.numel(), _stream(stream)), "ssm_scan_bwd")
     return out
+
+
+def scan_bwd_workspace_size(mode, x, dt, A, B, C_, dy, *, cu_seqlens=None, conv_w=None, **_):
+    """Bytes of device workspace ssm_scan_bwd needs for these shapes."""
+    b = _abi.ScanBwdArgs()
+    b.fwd = _scan_args(mode, x, dt, A, B, C_, None, None, None, None, None, cu_seqlens, conv_w, None, None, None, dy,
+                       True, 0)
+    b.dy = _p(dy)
+    return int(_abi.lib().ssm_scan_bwd_workspace_size(C.byref(b)))

@@ -184,11 +184,13 @@ class Workload:
     steps: int = 0
     nsets: int = 1
     state_interval: int = 0   # > 0: intermediate states every this many tokens (prefix caching)
+    backward: bool = False    # the step is the backward of the scan (gradients of every input)
     seed: int = BASE_SEED
 
 
 # The five workloads of the hot path (seeds BASE_SEED + position), then the
-# varlen workload again with intermediate-state extraction (same inputs).
+# varlen workload again with intermediate-state extraction and the Mamba-1
+# layer's backward (same inputs as their forward workloads).
 WORKLOADS = {
     "mamba1_tiny_f32": Workload("mamba1_tiny_f32", "mamba1", "f32", batch=1, seqlen=64, d_inner=16, dstate=4,
                                 seed=BASE_SEED + 0),
@@ -208,6 +210,10 @@ WORKLOADS = {
     "mamba2_varlen_16seq_h64_p64_g1_n128_states512": Workload(
         "mamba2_varlen_16seq_h64_p64_g1_n128_states512", "mamba2_varlen", "bf16", nheads=64, headdim=64, ngroups=1,
         dstate=128, nseqs=16, len_lo=128, len_hi=8192, chunk=256, state_interval=512, seed=BASE_SEED + 3),
+    # the Mamba-1 layer's backward (same inputs; upstream gradients drawn alongside)
+    "mamba1_layer_b8_l2048_d1536_n16_bwd": Workload("mamba1_layer_b8_l2048_d1536_n16_bwd", "mamba1", "bf16", batch=8,
+                                                    seqlen=2048, d_inner=1536, dstate=16, backward=True,
+                                                    seed=BASE_SEED + 1),
 }
 
 
