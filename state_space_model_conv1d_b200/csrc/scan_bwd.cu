@@ -76,11 +76,12 @@ SSM_DEVINL Seq seq_bounds(const BwdArgs &a, int si) {
     return q;
 }
 
-template <typename T, int NS>
+template <typename T, int NS, int LT>
 __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
     extern __shared__ __align__(16) float smb[];
     const int tid = threadIdx.x;
-    const int L = a.L, CPB = a.CPB, NP = a.NP, K = a.K;
+    constexpr int L = LT, CPB = kBT / LT, NP = LT * NS;
+    const int K = a.K;
     const bool m1 = a.mode == SSM_MAMBA1;
     const int j = tid / L, l = tid % L;
     const Seq q = seq_bounds(a, blockIdx.y);
@@ -113,6 +114,8 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
     float *sddt = sdC + kTCb * NP;                           // [TC]
     float *carry = sddt + kTCb;                              // [CPB][kMaxConvWidth]
     float *dcw = carry + CPB * kMaxConvWidth;                // [CPB][kMaxConvWidth]
+    float *rawx = dcw + CPB * kMaxConvWidth;                 // [TC + K-1][CPB] raw x rows t0-(K-1) ..
+    float *wts = rawx + (kTCb + kMaxConvWidth - 1) * CPB;    // [CPB][kMaxConvWidth] conv taps of the x channels
 
     const T *xg = static_cast<const T *>(a.x);
     const T *csi = static_cast<const T *>(a.conv_state_in);
@@ -132,6 +135,18 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
     auto stage = [&](int c) {
         const int64_t t0 = (int64_t)c * kTCb;
         const int nv = (int)min((int64_t)kTCb, q.len - t0);
+        const int KW = K > 0 ? K - 1 : 0;
+        for (int idx = tid; idx < (kTCb + KW) * CPB; idx += kBT) {
+            const int r = idx / CPB, jj = idx % CPB;
+            const int64_t pp = p0 + jj, pos = t0 - KW + r;
+            float v = 0.f;
+            if (pp < P && pos < q.len) {
+                const int64_t cc = m1 ? pp : hh * a.P + pp;
+                v = raw_at(xg, a.x_bs, a.x_ts, cc, cc, pos);
+            }
+            rawx[idx] = v;
+        }
+        __syncthreads();
         for (int idx = tid; idx < kTCb * CPB; idx += kBT) {
             const int t = idx / CPB, jj = idx % CPB;
             const int64_t pp = p0 + jj;
@@ -140,10 +155,12 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
                 const int64_t cc = m1 ? pp : hh * a.P + pp;
                 const int64_t tok = q.start + t0 + t;
                 if (K > 0) {
-                    vpre = conv_pre(xg, a.x_bs, a.x_ts, cc, cc, t0 + t);
+                    float acc = a.conv_b ? a.conv_b[cc] : 0.f;
+                    for (int k = 0; k < K; ++k) acc = fmaf(wts[jj * kMaxConvWidth + k], rawx[(t + k) * CPB + jj], acc);
+                    vpre = acc;
                     vxc = silu(vpre);
                 } else {
-                    vxc = Elem<T>::ld(xg + q.row * a.x_bs + tok * a.x_ts + cc);
+                    vxc = rawx[t * CPB + jj];
                 }
                 const int64_t dcol = m1 ? cc : hh;
                 const float u = Elem<T>::ld(static_cast<const T *>(a.dt) + q.row * a.dt_bs + tok * a.dt_ts + dcol) +
@@ -187,6 +204,12 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
 #pragma unroll
     for (int e = 0; e < NS; ++e) An[e] = A_of(e);
 
+    for (int idx = tid; idx < CPB * kMaxConvWidth; idx += kBT) {
+        const int jj = idx / kMaxConvWidth, k = idx % kMaxConvWidth;
+        const int64_t pp = p0 + jj;
+        const int64_t cc = m1 ? pp : hh * a.P + pp;
+        wts[idx] = (pp < P && k < K) ? a.conv_w[cc * K + k] : 0.f;
+    }
     // ---- pass A: forward, storing chunk-start states
     float h[NS];
     const int64_t hbase = ((int64_t)q.s * Dn + ch) * N;
@@ -267,18 +290,56 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
             const float dyt = dyv[t * CPB + jj];
             const float dyb = dyt * gate[t * CPB + jj];
             float dxp = 0.f, ddp = 0.f;
+            float vals[2 * NS];                                 // this lane's dB (e) and dC (NS + e) terms
 #pragma unroll
             for (int e = 0; e < NS; ++e) {
                 const int n = l * NS + e;
                 const float hc = hs[((t + 1) * kBT + tid) * NS + e], hp = hs[(t * kBT + tid) * NS + e];
-                if (cvalid) atomicAdd(&sdC[t * NP + n], dyb * hc);
+                vals[NS + e] = cvalid ? dyb * hc : 0.f;
                 gr[e] = fmaf(dyb, Ct[t * NP + n], gr[e]);
                 const float av = __expf(d * An[e]);
-                if (cvalid) atomicAdd(&sdB[t * NP + n], gr[e] * d * xv);
+                vals[e] = cvalid ? gr[e] * d * xv : 0.f;
                 dxp = fmaf(gr[e] * d, Bt[t * NP + n], dxp);
                 ddp = fmaf(gr[e], hp * av * An[e] + Bt[t * NP + n] * xv, ddp);
                 dAa[e] = fmaf(gr[e], hp * av * d, dAa[e]);
                 gr[e] *= av;
+            }
+            // sum over the warp's channels (lane bits above the L state lanes): halve the
+            // values at each level until one is left, then plain butterflies; each
+            // (dB / dC, state) sum lands on one lane, which adds it to the chunk tile
+            {
+                int base = 0, cnt = 2 * NS;
+                bool writer = true;
+#pragma unroll
+                for (int o = 16; o >= LT; o >>= 1) {
+                    const bool up = (threadIdx.x & o) != 0;
+                    if (cnt >= 2) {
+                        const int hlf = cnt / 2;
+#pragma unroll
+                        for (int k = 0; k < 2 * NS / 2; ++k) {
+                            if (k < hlf) {
+                                const float keep = up ? vals[hlf + k] : vals[k];
+                                const float send = up ? vals[k] : vals[hlf + k];
+                                vals[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                            }
+                        }
+                        base += up ? hlf : 0;
+                        cnt = hlf;
+                    } else {
+                        vals[0] += __shfl_xor_sync(0xffffffffu, vals[0], o);
+                        writer = writer && !up;
+                    }
+                }
+                if (writer) {
+#pragma unroll
+                    for (int k = 0; k < 2 * NS; ++k) {
+                        if (k < cnt) {
+                            const int idx = base + k;
+                            float *dst = idx < NS ? sdB : sdC;
+                            atomicAdd(&dst[t * NP + l * NS + (idx % NS)], vals[k]);
+                        }
+                    }
+                }
             }
             dxp = lane_sum(dxp);
             ddp = lane_sum(ddp);
@@ -337,7 +398,7 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
                 for (int t = 0; t < nv; ++t) {
                     const float dp = dxc[t * CPB + jj];
                     dcb_a += dp;
-                    for (int k = 0; k < K; ++k) dw[k] += dp * raw_at(xg, a.x_bs, a.x_ts, cc, cc, t0 + t - (K - 1) + k);
+                    for (int k = 0; k < K; ++k) dw[k] += dp * rawx[(t + k) * CPB + jj];
                 }
             }
             for (int t = nv - 1; t >= 0; --t) {
@@ -345,7 +406,7 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
                 float v;
                 if (K > 0) {
                     v = 0.f;
-                    for (int k = 0; k < K; ++k) v = fmaf(dp_at(pos + (K - 1) - k), a.conv_w[cc * K + k], v);
+                    for (int k = 0; k < K; ++k) v = fmaf(dp_at(pos + (K - 1) - k), wts[jj * kMaxConvWidth + k], v);
                 } else {
                     v = dxc[t * CPB + jj];
                 }
@@ -471,6 +532,20 @@ __global__ void bc_conv_bwd_kernel(const BwdArgs a) {
 
 }  // namespace
 
+// The kernel instance for (states per lane, lanes per channel).
+template <typename T, typename Run>
+cudaError_t dispatch(Run &&run, int NS, int L) {
+    if (NS == 8) return run(scan_bwd_kernel<T, 8, 32>);
+    switch (L) {
+        case 1: return run(scan_bwd_kernel<T, 4, 1>);
+        case 2: return run(scan_bwd_kernel<T, 4, 2>);
+        case 4: return run(scan_bwd_kernel<T, 4, 4>);
+        case 8: return run(scan_bwd_kernel<T, 4, 8>);
+        case 16: return run(scan_bwd_kernel<T, 4, 16>);
+        default: return run(scan_bwd_kernel<T, 4, 32>);
+    }
+}
+
 // Lanes per channel and states per lane for dstate N.
 static void bwd_layout(int64_t N, int *L, int *NS) {
     *NS = N > 128 ? 8 : 4;
@@ -547,7 +622,7 @@ cudaError_t launch_scan_bwd(const ssm_scan_bwd_args &b, const SeqView &sv, void 
         if ((e = zero(a.dCc, bc_bytes)) != cudaSuccess) return e;
     }
     const size_t smem = (size_t)((kTCb + 1) * kBT * NS + 8 * kTCb * a.CPB + 4 * kTCb * a.NP + kTCb +
-                                 2 * a.CPB * kMaxConvWidth) * 4;
+                                 3 * a.CPB * kMaxConvWidth + (kTCb + kMaxConvWidth - 1) * a.CPB) * 4;
     const unsigned gx = m1 ? (unsigned)((s.d_inner + a.CPB - 1) / a.CPB) : (unsigned)(s.nheads * a.units_per_head);
     dim3 grid(gx, (unsigned)nseq);
     if (nseq > 0) {
@@ -559,8 +634,8 @@ cudaError_t launch_scan_bwd(const ssm_scan_bwd_args &b, const SeqView &sv, void 
             timing_end(st);
             return cudaGetLastError();
         };
-        if (s.dtype == SSM_BF16) e = NS == 4 ? run(scan_bwd_kernel<__nv_bfloat16, 4>) : run(scan_bwd_kernel<__nv_bfloat16, 8>);
-        else e = NS == 4 ? run(scan_bwd_kernel<float, 4>) : run(scan_bwd_kernel<float, 8>);
+        if (s.dtype == SSM_BF16) e = dispatch<__nv_bfloat16>(run, NS, L);
+        else e = dispatch<float>(run, NS, L);
         if (e != cudaSuccess) return e;
         if (!m1) {
             const int64_t n = nseq * 2 * a.G * s.dstate;

@@ -80,3 +80,37 @@ def test_decode_fullsize_sampled_rows():
         assert_close(y[r:r + 1].float().cpu().numpy(), ry, "bf16", f"decode row {r} y")
         assert_close(state[r:r + 1].cpu().numpy(), st, "bf16", f"decode row {r} state")
         assert_close(cstate[r:r + 1].float().cpu().numpy(), cst, "bf16", f"decode row {r} conv state")
+
+
+def test_mamba1_layer_backward_fullsize():
+    """The backward at the Mamba-1 layer's full size: per-channel gradients on
+    sampled channels of every row, and the channel-summed dB / dC of row 0
+    from a full-width oracle run of that row."""
+    w = W.WORKLOADS["mamba1_layer_b8_l2048_d1536_n16_bwd"]
+    d = W.workload_inputs(w)
+    rng = np.random.default_rng(w.seed + 7)
+    dy = W.round_bf16(rng.standard_normal(d["x"].shape))
+    dhf = rng.standard_normal(d["h0"].shape).astype(np.float32).astype(np.float64)
+    t = to_dev(d, "bf16")
+    import state_space_model_conv1d_b200 as ssm
+    g = ssm.scan_bwd(M1, t["x"], t["dt"], t["A"], t["B"], t["C"], torch.from_numpy(dy).to("cuda", torch.bfloat16),
+                     D=t["D"], z=t["z"], dt_bias=t["dt_bias"], h0=t["h0"], conv_w=t["conv_w"],
+                     dh_final=torch.from_numpy(dhf).float().cuda())
+    torch.cuda.synchronize()
+    g = {k: (None if v is None else v.cpu().numpy()) for k, v in g.items()}
+    sel = np.array([0, 1, 31, 32, 777, 1535])
+    r = oracle.scan_bwd(M1, d["x"][:, :, sel], d["dt"][:, :, sel], d["A"][sel], d["B"], d["C"], dy[:, :, sel],
+                        D=d["D"][sel], z=d["z"][:, :, sel], dt_bias=d["dt_bias"][sel], h0=d["h0"][:, sel],
+                        conv_w=d["conv_w"][sel], dh_final=dhf[:, sel])
+    assert_close(g["dx"][:, :, sel], r["dx"], "bf16", "bwd dx")
+    assert_close(g["dz"][:, :, sel], r["dz"], "bf16", "bwd dz")
+    assert_close(g["ddt"][:, :, sel], r["ddt"], "bf16", "bwd ddt")
+    assert_close(g["dA"][sel], r["dA"], "bf16", "bwd dA")
+    assert_close(g["dD"][sel], r["dD"], "bf16", "bwd dD")
+    assert_close(g["ddt_bias"][sel], r["ddt_bias"], "bf16", "bwd ddt_bias")
+    assert_close(g["dh0"][:, sel], r["dh0"], "bf16", "bwd dh0")
+    assert_close(g["dconv_w"][sel], r["dconv_w"], "bf16", "bwd dconv_w")
+    row = oracle.scan_bwd(M1, d["x"][:1], d["dt"][:1], d["A"], d["B"][:1], d["C"][:1], dy[:1], D=d["D"], z=d["z"][:1],
+                          dt_bias=d["dt_bias"], h0=d["h0"][:1], conv_w=d["conv_w"], dh_final=dhf[:1])
+    assert_close(g["dB"][:1], row["dB"], "bf16", "bwd dB row 0")
+    assert_close(g["dC"][:1], row["dC"], "bf16", "bwd dC row 0")
