@@ -19,6 +19,7 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr int kTokensPerThread = 8;
+constexpr int kRunsPerThread = 4;      // consecutive 8-token runs per thread: taps loaded once, history carried
 
 template <typename T, int VEC, int K>
 __global__ void __launch_bounds__(kThreads)
@@ -30,19 +31,30 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
     const int64_t c0 = cv * VEC;
     if (c0 >= channels) return;
     const int row = blockIdx.z;
-    const int64_t t0 = (int64_t)blockIdx.y * kTokensPerThread;
-    if (t0 >= seqlen) return;
-    const int64_t t1 = min(t0 + (int64_t)kTokensPerThread, seqlen);
+    const int64_t tr0 = (int64_t)blockIdx.y * kTokensPerThread * kRunsPerThread;
+    if (tr0 >= seqlen) return;
 
     float wk[K][VEC], bb[VEC];
+    const bool w4 = K == 4 && ((uintptr_t)w & 15) == 0;       // each channel's 4 taps as one 16-byte load
 #pragma unroll
     for (int v = 0; v < VEC; ++v) {
+        if (w4) {
+            const float4 q = *reinterpret_cast<const float4 *>(w + (c0 + v) * 4);
+            wk[0][v] = q.x; wk[1 % K][v] = q.y; wk[2 % K][v] = q.z; wk[3 % K][v] = q.w;
+        } else {
 #pragma unroll
-        for (int k = 0; k < K; ++k) wk[k][v] = w[(c0 + v) * K + k];
+            for (int k = 0; k < K; ++k) wk[k][v] = w[(c0 + v) * K + k];
+        }
         bb[v] = bias ? bias[c0 + v] : 0.f;
     }
     const T *xr = x + row * x_bs;
     T *orow = out + row * o_bs;
+    float hist[K > 1 ? K - 1 : 1][VEC];
+    bool have_hist = false;                    // hist already holds the rows before t0 (same sequence)
+  for (int run = 0; run < kRunsPerThread; ++run) {
+    const int64_t t0 = tr0 + (int64_t)run * kTokensPerThread;
+    if (t0 >= seqlen) break;
+    const int64_t t1 = min(t0 + (int64_t)kTokensPerThread, seqlen);
 
     // Offsets are clamped into [0, seqlen] so a malformed cu_seqlens can give
     // wrong values but never an out-of-bounds access.
@@ -50,7 +62,6 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
     int64_t start = cu ? min(max((int64_t)cu[s], (int64_t)0), seqlen) : 0;
     int64_t end = cu ? min(max((int64_t)cu[s + 1], start), seqlen) : seqlen;
 
-    float hist[K > 1 ? K - 1 : 1][VEC];
     auto load_hist = [&](int64_t t) {
 #pragma unroll
         for (int j = 0; j < K - 1; ++j) {          // hist[j] holds time t-(K-1)+j
@@ -70,7 +81,8 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
             }
         }
     };
-    load_hist(t0);
+    if (!(have_hist && !cu)) load_hist(t0);
+    have_hist = true;
     if (!cu || t1 <= end) {
         // the whole run lies in one sequence: issue every row's load before any math
         float cur[kTokensPerThread][VEC];
@@ -111,7 +123,7 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
 #pragma unroll
                 for (int v = 0; v < VEC; ++v) hist[K > 1 ? K - 2 : 0][v] = cur[i][v];
         }
-        return;
+        continue;
     }
     for (int64_t t = t0; t < t1; ++t) {
         if (cu && t >= end) {                      // next (non-empty) sequence of the packed row
@@ -151,6 +163,7 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
 #pragma unroll
             for (int v = 0; v < VEC; ++v) hist[K > 1 ? K - 2 : 0][v] = cur[v];
     }
+  }
 }
 
 // Carried state after the sequence: the last K-1 raw inputs of
@@ -183,7 +196,8 @@ __global__ void conv_state_out_kernel(const T *__restrict__ x, int64_t x_bs, int
 template <typename T, int VEC>
 cudaError_t launch_typed_vec(const ConvJob &a, cudaStream_t st) {
     const int64_t nvec = (a.channels + VEC - 1) / VEC;
-    dim3 grid((unsigned)((nvec + kThreads - 1) / kThreads), (unsigned)((a.seqlen + kTokensPerThread - 1) / kTokensPerThread),
+    const int64_t per_cta = (int64_t)kTokensPerThread * kRunsPerThread;
+    dim3 grid((unsigned)((nvec + kThreads - 1) / kThreads), (unsigned)((a.seqlen + per_cta - 1) / per_cta),
               (unsigned)a.batch);
     const T *x = static_cast<const T *>(a.x);
     const T *si = static_cast<const T *>(a.state_in);

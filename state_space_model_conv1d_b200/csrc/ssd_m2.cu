@@ -615,11 +615,30 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     const int64_t cdim = s.d_inner + 2 * GN;
     const __nv_bfloat16 *Bc = static_cast<const __nv_bfloat16 *>(s.B), *Cc = static_cast<const __nv_bfloat16 *>(s.C);
     int64_t b_bs = s.B_batch_stride, b_ts = s.B_token_stride, c_bs = s.C_batch_stride, c_ts = s.C_token_stride;
+    __nv_bfloat16 *wB = nullptr, *wC = nullptr;
+    if (s.d_conv > 0) {
+        // the conv'd B and C live in the workspace
+        wB = static_cast<__nv_bfloat16 *>(ws);
+        const size_t one = (size_t)s.batch * (size_t)s.seqlen * (size_t)GN * 2;
+        wC = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + (one + 255) / 256 * 256);
+        Bc = wB; Cc = wC;
+        b_bs = c_bs = s.seqlen * GN;
+        b_ts = c_ts = GN;
+    }
+    // Host work first (tensor maps over the whole packed / batched token range,
+    // the kernel attribute), so nothing on the host separates the pre-pass
+    // launches from the scan launch.
+    const int64_t rows = s.cu_seqlens ? 1 : s.batch;
+    CUtensorMap tm_x, tm_b, tm_c, tm_y;
+    if (!make_map(&tm_x, s.x, s.d_inner, s.seqlen, rows, s.x_token_stride, s.x_batch_stride, false) ||
+        !make_map(&tm_b, Bc, GN, s.seqlen, rows, b_ts, b_bs, true) ||
+        !make_map(&tm_c, Cc, GN, s.seqlen, rows, c_ts, c_bs, true) ||
+        !make_map(&tm_y, s.y, s.d_inner, s.seqlen, rows, s.y_token_stride, s.y_batch_stride, true))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(ssd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
     if (s.d_conv > 0) {
         // pre-pass: conv + SiLU of the B and C channels, once per group, into the workspace
-        __nv_bfloat16 *wB = static_cast<__nv_bfloat16 *>(ws);
-        const size_t one = (size_t)s.batch * (size_t)s.seqlen * (size_t)GN * 2;
-        __nv_bfloat16 *wC = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + (one + 255) / 256 * 256);
         for (int which = 0; which < 2; ++which) {
             ConvJob j;
             j.x = which == 0 ? s.B : s.C;
@@ -636,12 +655,9 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
             j.channels = GN; j.width = s.d_conv; j.act = 1; j.dtype = SSM_BF16;
             j.out = which == 0 ? (void *)wB : (void *)wC;
             j.o_bs = s.seqlen * GN; j.o_ts = GN;
-            cudaError_t e = launch_conv_job(j, st);
+            e = launch_conv_job(j, st);
             if (e != cudaSuccess) return e;
         }
-        Bc = wB; Cc = wC;
-        b_bs = c_bs = s.seqlen * GN;
-        b_ts = c_ts = GN;
     }
     SsdArgs a;
     a.x = static_cast<const __nv_bfloat16 *>(s.x); a.z = static_cast<const __nv_bfloat16 *>(s.z);
@@ -663,16 +679,6 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     a.Braw = static_cast<const __nv_bfloat16 *>(s.B); a.Craw = static_cast<const __nv_bfloat16 *>(s.C);
     a.braw_bs = s.B_batch_stride; a.braw_ts = s.B_token_stride;
     a.craw_bs = s.C_batch_stride; a.craw_ts = s.C_token_stride;
-    // tensor maps over the whole packed / batched token range
-    const int64_t rows = s.cu_seqlens ? 1 : s.batch;
-    CUtensorMap tm_x, tm_b, tm_c, tm_y;
-    if (!make_map(&tm_x, s.x, s.d_inner, s.seqlen, rows, s.x_token_stride, s.x_batch_stride, false) ||
-        !make_map(&tm_b, Bc, GN, s.seqlen, rows, b_ts, b_bs, true) ||
-        !make_map(&tm_c, Cc, GN, s.seqlen, rows, c_ts, c_bs, true) ||
-        !make_map(&tm_y, s.y, s.d_inner, s.seqlen, rows, s.y_token_stride, s.y_batch_stride, true))
-        return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(ssd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
     dim3 grid((unsigned)s.nheads, (unsigned)nseqs);
     timing_begin(st);
     ssd_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, tm_x, tm_b, tm_c, tm_y);
