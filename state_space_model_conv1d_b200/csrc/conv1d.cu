@@ -26,12 +26,14 @@ __global__ void __launch_bounds__(kThreads)
 conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *__restrict__ w,
               const float *__restrict__ bias, const T *__restrict__ state_in, int64_t ss, T *__restrict__ out,
               int64_t o_bs, int64_t o_ts, const int32_t *__restrict__ cu, int nseqs, int64_t seqlen,
-              int64_t channels, int act) {
-    const int64_t cv = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+              int64_t channels, int act, int vpc) {
+    // a CTA covers vpc channel vectors x (kThreads / vpc) groups of token runs
+    const int64_t cv = (int64_t)blockIdx.x * vpc + threadIdx.x % vpc;
     const int64_t c0 = cv * VEC;
     if (c0 >= channels) return;
     const int row = blockIdx.z;
-    const int64_t tr0 = (int64_t)blockIdx.y * kTokensPerThread * kRunsPerThread;
+    const int64_t grp = (int64_t)blockIdx.y * (kThreads / vpc) + threadIdx.x / vpc;
+    const int64_t tr0 = grp * kTokensPerThread * kRunsPerThread;
     if (tr0 >= seqlen) return;
 
     float wk[K][VEC], bb[VEC];
@@ -50,18 +52,11 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
     const T *xr = x + row * x_bs;
     T *orow = out + row * o_bs;
     float hist[K > 1 ? K - 1 : 1][VEC];
-    bool have_hist = false;                    // hist already holds the rows before t0 (same sequence)
-  for (int run = 0; run < kRunsPerThread; ++run) {
-    const int64_t t0 = tr0 + (int64_t)run * kTokensPerThread;
-    if (t0 >= seqlen) break;
-    const int64_t t1 = min(t0 + (int64_t)kTokensPerThread, seqlen);
-
     // Offsets are clamped into [0, seqlen] so a malformed cu_seqlens can give
     // wrong values but never an out-of-bounds access.
-    int s = cu ? seq_of_token(cu, nseqs, t0) : row;
+    int s = cu ? seq_of_token(cu, nseqs, tr0) : row;
     int64_t start = cu ? min(max((int64_t)cu[s], (int64_t)0), seqlen) : 0;
     int64_t end = cu ? min(max((int64_t)cu[s + 1], start), seqlen) : seqlen;
-
     auto load_hist = [&](int64_t t) {
 #pragma unroll
         for (int j = 0; j < K - 1; ++j) {          // hist[j] holds time t-(K-1)+j
@@ -81,7 +76,18 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
             }
         }
     };
-    if (!(have_hist && !cu)) load_hist(t0);
+    bool have_hist = false;                    // hist holds the K-1 rows before t0 of sequence s
+  for (int run = 0; run < kRunsPerThread; ++run) {
+    const int64_t t0 = tr0 + (int64_t)run * kTokensPerThread;
+    if (t0 >= seqlen) break;
+    const int64_t t1 = min(t0 + (int64_t)kTokensPerThread, seqlen);
+    if (cu && t0 >= end) {                     // the run starts in a later sequence
+        while (s + 1 < nseqs && cu[s + 1] <= t0) ++s;
+        start = min(max((int64_t)cu[s], (int64_t)0), seqlen);
+        end = min(max((int64_t)cu[s + 1], start), seqlen);
+        have_hist = false;
+    }
+    if (!have_hist) load_hist(t0);
     have_hist = true;
     if (!cu || t1 <= end) {
         // the whole run lies in one sequence: issue every row's load before any math
@@ -196,9 +202,11 @@ __global__ void conv_state_out_kernel(const T *__restrict__ x, int64_t x_bs, int
 template <typename T, int VEC>
 cudaError_t launch_typed_vec(const ConvJob &a, cudaStream_t st) {
     const int64_t nvec = (a.channels + VEC - 1) / VEC;
-    const int64_t per_cta = (int64_t)kTokensPerThread * kRunsPerThread;
-    dim3 grid((unsigned)((nvec + kThreads - 1) / kThreads), (unsigned)((a.seqlen + per_cta - 1) / per_cta),
-              (unsigned)a.batch);
+    // narrow tensors (few channel vectors) put several token-run groups in one CTA
+    int vpc = kThreads;
+    while (vpc / 2 >= nvec && vpc > 1) vpc /= 2;
+    const int64_t per_cta = (int64_t)kTokensPerThread * kRunsPerThread * (kThreads / vpc);
+    dim3 grid((unsigned)((nvec + vpc - 1) / vpc), (unsigned)((a.seqlen + per_cta - 1) / per_cta), (unsigned)a.batch);
     const T *x = static_cast<const T *>(a.x);
     const T *si = static_cast<const T *>(a.state_in);
     T *o = static_cast<T *>(a.out);
@@ -208,7 +216,7 @@ cudaError_t launch_typed_vec(const ConvJob &a, cudaStream_t st) {
     case KK:                                                                                                \
         conv1d_kernel<T, VEC, KK><<<grid, kThreads, 0, st>>>(x, a.x_bs, a.x_ts, a.w, a.b, si, a.state_stride, o, \
                                                              a.o_bs, a.o_ts, a.cu, ns, a.seqlen, a.channels,   \
-                                                             a.act);                                           \
+                                                             a.act, vpc);                                      \
         break;
         switch (a.width) {
             SSM_CONV_CASE(1) SSM_CONV_CASE(2) SSM_CONV_CASE(3) SSM_CONV_CASE(4)
