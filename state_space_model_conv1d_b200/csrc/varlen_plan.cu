@@ -1,7 +1,7 @@
 // varlen_plan.cu -- device pre-pass for packed variable-length batches.
 //
 // Checks cu_seqlens on the device (0-based, non-decreasing, ending at the
-// packed token count) and writes the verdict into the workspace error word,
+// packed token count) and writes the outcome into the workspace error word,
 // then writes a schedule that lists sequences longest first, so the scan
 // kernels start the long chains first and short ones fill in behind them.
 // No host synchronisation: the scan kernels read the error word and return

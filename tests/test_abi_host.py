@@ -2,7 +2,7 @@
 declares, and rejects bad arguments before anything reaches a GPU.
 
 Every call here is one the library must refuse during host-side validation,
-so nothing is launched (no GPU is needed, and none is touched on a GPU machine).
+so nothing is launched (no GPU is needed, and none is touched when one is present).
 """
 import ctypes as C
 import os
