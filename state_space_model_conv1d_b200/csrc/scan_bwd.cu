@@ -24,6 +24,8 @@
 // shared-memory then global float atomics.  The Mamba-2 B / C conv backward
 // runs afterwards, once per (sequence, B / C channel), on the summed
 // gradients of the conv outputs.
+#include <type_traits>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -132,28 +134,84 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
     };
 
     const int nch = (int)((q.len + kTCb - 1) / kTCb);
-    auto stage = [&](int c) {
+    // Stage chunk c into shared memory.  Every thread first issues all of its
+    // global loads (compile-time trip counts), then does the math, so the load
+    // latencies overlap.  FULL = false (the checkpoint pass) skips what only
+    // the reverse pass reads: z, dy, C and the softplus derivative.
+    constexpr int kRawIt = ((kTCb + kMaxConvWidth - 1) * CPB + kBT - 1) / kBT;
+    constexpr int kTokIt = (kTCb * CPB + kBT - 1) / kBT;
+    constexpr int kStIt = (kTCb * NP + kBT - 1) / kBT;
+    const T *dtp = static_cast<const T *>(a.dt), *zp = static_cast<const T *>(a.z), *dyp = static_cast<const T *>(a.dy);
+    const T *Bs = static_cast<const T *>(a.B), *Cs = static_cast<const T *>(a.C);
+    // Staging is split in two: issue(c) loads chunk c's inputs into registers,
+    // finish(c) writes / computes them into shared memory.  issue runs one
+    // chunk ahead, so the load latency hides behind the current chunk's work.
+    float rv[kRawIt], rdt[kTokIt], rz[kTokIt], rdy[kTokIt], rb[kStIt], rc[kStIt];
+    const bool bc_raw = m1 || K == 0;
+    auto issue = [&](int c, auto full_tag) {
+        constexpr bool FULL = decltype(full_tag)::value;
         const int64_t t0 = (int64_t)c * kTCb;
         const int nv = (int)min((int64_t)kTCb, q.len - t0);
         const int KW = K > 0 ? K - 1 : 0;
-        for (int idx = tid; idx < (kTCb + KW) * CPB; idx += kBT) {
+#pragma unroll
+        for (int i = 0; i < kRawIt; ++i) {
+            const int idx = tid + i * kBT;
             const int r = idx / CPB, jj = idx % CPB;
             const int64_t pp = p0 + jj, pos = t0 - KW + r;
-            float v = 0.f;
-            if (pp < P && pos < q.len) {
+            rv[i] = 0.f;
+            if (r < kTCb + KW && pp < P && pos < q.len) {
                 const int64_t cc = m1 ? pp : hh * a.P + pp;
-                v = raw_at(xg, a.x_bs, a.x_ts, cc, cc, pos);
+                rv[i] = raw_at(xg, a.x_bs, a.x_ts, cc, cc, pos);
             }
-            rawx[idx] = v;
         }
-        __syncthreads();
-        for (int idx = tid; idx < kTCb * CPB; idx += kBT) {
+#pragma unroll
+        for (int i = 0; i < kTokIt; ++i) {
+            const int idx = tid + i * kBT;
             const int t = idx / CPB, jj = idx % CPB;
             const int64_t pp = p0 + jj;
-            float vxc = 0.f, vpre = 0.f, vdl = 0.f, vsp = 0.f, vg = 1.f, vdg = 0.f, vdy = 0.f;
+            rdt[i] = 0.f; rz[i] = 0.f; rdy[i] = 0.f;
             if (t < nv && pp < P) {
                 const int64_t cc = m1 ? pp : hh * a.P + pp;
                 const int64_t tok = q.start + t0 + t;
+                rdt[i] = Elem<T>::ld(dtp + q.row * a.dt_bs + tok * a.dt_ts + (m1 ? cc : hh));
+                if (FULL) {
+                    if (zp) rz[i] = Elem<T>::ld(zp + q.row * a.z_bs + tok * a.z_ts + cc);
+                    rdy[i] = Elem<T>::ld(dyp + q.row * a.dy_bs + tok * a.dy_ts + cc);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kStIt; ++i) {
+            const int idx = tid + i * kBT;
+            const int t = idx / NP, n = idx % NP;
+            rb[i] = 0.f; rc[i] = 0.f;
+            if (bc_raw && t < nv && n < N) {
+                const int64_t tok = q.start + t0 + t;
+                rb[i] = Elem<T>::ld(Bs + q.row * a.B_bs + tok * a.B_ts + g * N + n);
+                if (FULL) rc[i] = Elem<T>::ld(Cs + q.row * a.C_bs + tok * a.C_ts + g * N + n);
+            }
+        }
+    };
+    auto stage = [&](int c, auto full_tag) {
+        constexpr bool FULL = decltype(full_tag)::value;
+        const int64_t t0 = (int64_t)c * kTCb;
+        const int nv = (int)min((int64_t)kTCb, q.len - t0);
+        const int KW = K > 0 ? K - 1 : 0;
+#pragma unroll
+        for (int i = 0; i < kRawIt; ++i) {
+            const int idx = tid + i * kBT;
+            if (idx < (kTCb + KW) * CPB) rawx[idx] = rv[i];
+        }
+        __syncthreads();                                    // rawx complete
+#pragma unroll
+        for (int i = 0; i < kTokIt; ++i) {
+            const int idx = tid + i * kBT;
+            if (idx >= kTCb * CPB) break;
+            const int t = idx / CPB, jj = idx % CPB;
+            const int64_t pp = p0 + jj;
+            float vxc = 0.f, vpre = 0.f, vdl = 0.f, vsp = 0.f, vg = 1.f, vdg = 0.f;
+            if (t < nv && pp < P) {
+                const int64_t cc = m1 ? pp : hh * a.P + pp;
                 if (K > 0) {
                     float acc = a.conv_b ? a.conv_b[cc] : 0.f;
                     for (int k = 0; k < K; ++k) acc = fmaf(wts[jj * kMaxConvWidth + k], rawx[(t + k) * CPB + jj], acc);
@@ -163,38 +221,38 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
                     vxc = rawx[t * CPB + jj];
                 }
                 const int64_t dcol = m1 ? cc : hh;
-                const float u = Elem<T>::ld(static_cast<const T *>(a.dt) + q.row * a.dt_bs + tok * a.dt_ts + dcol) +
-                                (a.dt_bias ? a.dt_bias[dcol] : 0.f);
+                const float u = rdt[i] + (a.dt_bias ? a.dt_bias[dcol] : 0.f);
                 vdl = a.softplus ? softplus(u) : u;
-                vsp = a.softplus ? sigmoidf_(u) : 1.f;
-                if (a.z) {
-                    const float zv = Elem<T>::ld(static_cast<const T *>(a.z) + q.row * a.z_bs + tok * a.z_ts + cc);
-                    vg = silu(zv);
-                    vdg = dsilu(zv);
+                if (FULL) {
+                    vsp = a.softplus ? sigmoidf_(u) : 1.f;
+                    if (zp) {
+                        vg = silu(rz[i]);
+                        vdg = dsilu(rz[i]);
+                    }
                 }
-                vdy = Elem<T>::ld(static_cast<const T *>(a.dy) + q.row * a.dy_bs + tok * a.dy_ts + cc);
             }
-            xc[t * CPB + jj] = vxc; pre[t * CPB + jj] = vpre; dl[t * CPB + jj] = vdl; spd[t * CPB + jj] = vsp;
-            gate[t * CPB + jj] = vg; dgate[t * CPB + jj] = vdg; dyv[t * CPB + jj] = vdy;
+            xc[t * CPB + jj] = vxc; dl[t * CPB + jj] = vdl;
+            if (FULL) {
+                pre[t * CPB + jj] = vpre; spd[t * CPB + jj] = vsp;
+                gate[t * CPB + jj] = vg; dgate[t * CPB + jj] = vdg; dyv[t * CPB + jj] = rdy[i];
+            }
         }
-        for (int idx = tid; idx < kTCb * NP; idx += kBT) {
+#pragma unroll
+        for (int i = 0; i < kStIt; ++i) {
+            const int idx = tid + i * kBT;
+            if (idx >= kTCb * NP) break;
             const int t = idx / NP, n = idx % NP;
-            float vb = 0.f, vc = 0.f;
-            if (t < nv && n < N) {
-                const int64_t tok = q.start + t0 + t;
-                const T *Bs = static_cast<const T *>(a.B), *Cs = static_cast<const T *>(a.C);
-                if (m1 || K == 0) {
-                    vb = Elem<T>::ld(Bs + q.row * a.B_bs + tok * a.B_ts + g * N + n);
-                    vc = Elem<T>::ld(Cs + q.row * a.C_bs + tok * a.C_ts + g * N + n);
-                } else {
-                    vb = silu(conv_pre(Bs, a.B_bs, a.B_ts, g * N + n, Dn + g * N + n, t0 + t));
-                    vc = silu(conv_pre(Cs, a.C_bs, a.C_ts, g * N + n, Dn + GN + g * N + n, t0 + t));
-                }
+            float vb = rb[i], vc = rc[i];
+            if (!bc_raw && t < nv && n < N) {
+                vb = silu(conv_pre(Bs, a.B_bs, a.B_ts, g * N + n, Dn + g * N + n, t0 + t));
+                if (FULL) vc = silu(conv_pre(Cs, a.C_bs, a.C_ts, g * N + n, Dn + GN + g * N + n, t0 + t));
             }
             Bt[t * NP + n] = vb;
-            Ct[t * NP + n] = vc;
+            if (FULL) Ct[t * NP + n] = vc;
         }
     };
+    using FullT = std::integral_constant<bool, true>;
+    using LightT = std::integral_constant<bool, false>;
     auto A_of = [&](int e) -> float {
         const int64_t n = (int64_t)l * NS + e;
         if (n >= N || !cvalid) return 0.f;
@@ -218,6 +276,7 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
         const int64_t n = (int64_t)l * NS + e;
         h[e] = (cvalid && n < N && a.h0) ? a.h0[hbase + n] : 0.f;
     }
+    if (nch > 0) issue(0, LightT{});
     for (int c = 0; c < nch; ++c) {
         if (cvalid) {
             float *dst = a.ckpt + ((q.slot0 + c) * Dn + ch) * NP + (int64_t)l * NS;
@@ -225,8 +284,9 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
             for (int e = 0; e < NS; ++e) dst[e] = h[e];
         }
         __syncthreads();
-        stage(c);
+        stage(c, LightT{});
         __syncthreads();
+        if (c + 1 < nch) issue(c + 1, LightT{});
         const int nv = (int)min((int64_t)kTCb, q.len - (int64_t)c * kTCb);
         if (cvalid)
             for (int t = 0; t < nv; ++t) {
@@ -255,11 +315,13 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
     };
     const T *dcso = static_cast<const T *>(a.dcs_out);
 
+    if (nch > 0) issue(nch - 1, FullT{});
     for (int c = nch - 1; c >= 0; --c) {
         const int64_t t0 = (int64_t)c * kTCb;
         const int nv = (int)min((int64_t)kTCb, q.len - t0);
         __syncthreads();
-        stage(c);
+        stage(c, FullT{});
+        if (c > 0) issue(c - 1, FullT{});
         for (int idx = tid; idx < kTCb * NP; idx += kBT) { sdB[idx] = 0.f; sdC[idx] = 0.f; }
         if (tid < kTCb) sddt[tid] = 0.f;
         __syncthreads();
