@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
     float *dcw = carry + CPB * kMaxConvWidth;                // [CPB][kMaxConvWidth]
     float *rawx = dcw + CPB * kMaxConvWidth;                 // [TC + K-1][CPB] raw x rows t0-(K-1) ..
     float *wts = rawx + (kTCb + kMaxConvWidth - 1) * CPB;    // [CPB][kMaxConvWidth] conv taps of the x channels
+    float *dcb = wts + CPB * kMaxConvWidth;                  // [CPB] conv bias gradient of the x channels
 
     const T *xg = static_cast<const T *>(a.x);
     const T *csi = static_cast<const T *>(a.conv_state_in);
@@ -304,9 +305,11 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
         gr[e] = (cvalid && n < N && a.dh_final) ? a.dh_final[hbase + n] : 0.f;
         dAa[e] = 0.f;
     }
-    float dDa = 0.f, dbias_a = 0.f, dcb_a = 0.f;
-    if (tid < CPB)
+    float dDa = 0.f, dbias_a = 0.f;
+    if (tid < CPB) {
         for (int k = 0; k < kMaxConvWidth; ++k) { carry[tid * kMaxConvWidth + k] = 0.f; dcw[tid * kMaxConvWidth + k] = 0.f; }
+        dcb[tid] = 0.f;
+    }
     const float Dv = (cvalid && a.D) ? a.D[m1 ? ch : hh] : 0.f;
     const unsigned gmask = L >= 32 ? 0xffffffffu : (((1u << L) - 1u) << ((threadIdx.x & 31) / L * L));
     auto lane_sum = [&](float v) {
@@ -440,46 +443,54 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
             atomicAdd(&a.ddt[rt * a.H + hh], sddt[tid]);
             dbias_a += sddt[tid];                 // summed below by threads < kTCb
         }
-        // conv backward of this chunk's x channels (one thread per channel)
-        if (tid < CPB && p0 + tid < P) {
-            const int jj = tid;
+        // conv backward of this chunk's x channels, spread over the CTA:
+        // dpre per (token, channel), then d raw per (token, channel), the tap
+        // gradients per (channel, tap), and the carried dpre of this chunk's
+        // first K-1 tokens for the chunk before it
+        __syncthreads();                                  // dxc of every channel written
+        for (int idx = tid; idx < kTCb * CPB; idx += kBT) {
+            const int t = idx / CPB, jj = idx % CPB;
+            if (t < nv && K > 0) dxc[idx] = dxc[idx] * dsilu(pre[idx]);
+        }
+        __syncthreads();
+        auto dp_at = [&](int jj, int64_t x) -> float {    // dpre at sequence position x >= t0
+            if (x < t0 + nv) return dxc[(x - t0) * CPB + jj];
+            const int64_t i = x - (t0 + nv);
+            return (x < q.len && i < kMaxConvWidth) ? carry[jj * kMaxConvWidth + i] : 0.f;
+        };
+        for (int idx = tid; idx < kTCb * CPB; idx += kBT) {
+            const int t = idx / CPB, jj = idx % CPB;
+            if (t >= nv || p0 + jj >= P) continue;
             const int64_t cc = m1 ? p0 + jj : hh * a.P + p0 + jj;
-            float *cr = carry + jj * kMaxConvWidth;
-            float *dw = dcw + jj * kMaxConvWidth;
-            // dpre of the chunk, in place over dxc
-            for (int t = 0; t < nv; ++t) {
-                const float dv = dxc[t * CPB + jj];
-                dxc[t * CPB + jj] = K > 0 ? dv * dsilu(pre[t * CPB + jj]) : dv;
-            }
-            auto dp_at = [&](int64_t x) -> float {           // dpre at sequence position x >= t0
-                if (x < t0 + nv) return dxc[(x - t0) * CPB + jj];
-                const int64_t i = x - (t0 + nv);
-                return (x < q.len && i < kMaxConvWidth) ? cr[i] : 0.f;
-            };
+            const int64_t pos = t0 + t;
+            float v;
             if (K > 0) {
+                v = 0.f;
+                for (int k = 0; k < K; ++k) v = fmaf(dp_at(jj, pos + (K - 1) - k), wts[jj * kMaxConvWidth + k], v);
+            } else {
+                v = dxc[idx];
+            }
+            if (dcso && K > 1 && pos >= q.len - (K - 1))
+                v += Elem<T>::ld(dcso + ((int64_t)q.s * cdim + cc) * (K - 1) + (pos - (q.len - (K - 1))));
+            a.dx[(q.row * a.T + q.start + pos) * Dn + cc] = v;
+        }
+        if (K > 0)
+            for (int idx = tid; idx < CPB * K; idx += kBT) {
+                const int jj = idx / K, k = idx % K;
+                if (p0 + jj >= P) continue;
+                float sw = 0.f, sb = 0.f;
                 for (int t = 0; t < nv; ++t) {
                     const float dp = dxc[t * CPB + jj];
-                    dcb_a += dp;
-                    for (int k = 0; k < K; ++k) dw[k] += dp * rawx[(t + k) * CPB + jj];
+                    sw = fmaf(dp, rawx[(t + k) * CPB + jj], sw);
+                    sb += dp;
                 }
+                dcw[jj * kMaxConvWidth + k] += sw;
+                if (k == 0) dcb[jj] += sb;
             }
-            for (int t = nv - 1; t >= 0; --t) {
-                const int64_t pos = t0 + t;
-                float v;
-                if (K > 0) {
-                    v = 0.f;
-                    for (int k = 0; k < K; ++k) v = fmaf(dp_at(pos + (K - 1) - k), wts[jj * kMaxConvWidth + k], v);
-                } else {
-                    v = dxc[t * CPB + jj];
-                }
-                if (dcso && K > 1 && pos >= q.len - (K - 1))
-                    v += Elem<T>::ld(dcso + ((int64_t)q.s * cdim + cc) * (K - 1) + (pos - (q.len - (K - 1))));
-                a.dx[(q.row * a.T + q.start + pos) * Dn + cc] = v;
-            }
-            // new carry: dpre at positions t0 .. t0+K-2
-            float nc[kMaxConvWidth];
-            for (int i = 0; i < kMaxConvWidth; ++i) nc[i] = (i < K - 1) ? dp_at(t0 + i) : 0.f;
-            for (int i = 0; i < kMaxConvWidth; ++i) cr[i] = nc[i];
+        __syncthreads();                                  // the old carry has been read
+        for (int idx = tid; idx < CPB * (kMaxConvWidth - 1); idx += kBT) {
+            const int jj = idx / (kMaxConvWidth - 1), i = idx % (kMaxConvWidth - 1);
+            if (i < K - 1) carry[jj * kMaxConvWidth + i] = dp_at(jj, t0 + i);
         }
     }
     __syncthreads();
@@ -504,7 +515,7 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
         const int64_t cc = m1 ? p0 + tid : hh * a.P + p0 + tid;
         if (a.dconv_w)
             for (int k = 0; k < K; ++k) atomicAdd(&a.dconv_w[cc * K + k], dcw[tid * kMaxConvWidth + k]);
-        if (a.dconv_b) atomicAdd(&a.dconv_b[cc], dcb_a);
+        if (a.dconv_b) atomicAdd(&a.dconv_b[cc], dcb[tid]);
     }
     if (cvalid) {
 #pragma unroll
@@ -684,7 +695,7 @@ cudaError_t launch_scan_bwd(const ssm_scan_bwd_args &b, const SeqView &sv, void 
         if ((e = zero(a.dCc, bc_bytes)) != cudaSuccess) return e;
     }
     const size_t smem = (size_t)((kTCb + 1) * kBT * NS + 8 * kTCb * a.CPB + 4 * kTCb * a.NP + kTCb +
-                                 3 * a.CPB * kMaxConvWidth + (kTCb + kMaxConvWidth - 1) * a.CPB) * 4;
+                                 3 * a.CPB * kMaxConvWidth + (kTCb + kMaxConvWidth - 1) * a.CPB + a.CPB) * 4;
     const unsigned gx = m1 ? (unsigned)((s.d_inner + a.CPB - 1) / a.CPB) : (unsigned)(s.nheads * a.units_per_head);
     dim3 grid(gx, (unsigned)nseq);
     if (nseq > 0) {
