@@ -54,3 +54,23 @@ def test_two_gloo_ranks_max_time_and_weak_scaling():
     assert out[0][1] != out[1][1], "ranks draw different batches"
     # 1000 tokens x 10 steps x 2 ranks in 15 ms
     assert out[0][2] == pytest.approx(1000 * 10 * 2 / 0.015)
+
+
+def test_reference_arm_prints_the_contract_line():
+    """bench.py --impl reference (the fp64 oracle on the host) prints one JSON
+    line with the contract's keys, on the tiny Mamba-1 workload."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload",
+                          "mamba1_tiny_f32", "--steps", "1", "--warmup", "0"], capture_output=True, text=True,
+                         timeout=300, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = [l for l in out.stdout.splitlines() if l.startswith("{")][-1]
+    d = json.loads(line)
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
