@@ -11,6 +11,8 @@
 // keeping the K-1 previous rows in registers, so every input element is read
 // once from DRAM (plus a (K-1)/TT halo re-read) and every output written once.
 // A warp covers 256 contiguous channels of one token: 512-byte coalesced rows.
+#include <type_traits>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -18,11 +20,13 @@ namespace ssm {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kTokensPerThread = 8;
-constexpr int kRunsPerThread = 4;      // consecutive 8-token runs per thread: taps loaded once, history carried
+constexpr int kTokensPerThread = 4;
+constexpr int kRunsPerThread = 8;      // consecutive 4-token runs per thread: taps loaded once, history carried
 
+// four CTAs per SM: short runs keep the rows in flight per thread small, and
+// the extra resident warps keep more rows in flight per SM
 template <typename T, int VEC, int K>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
 conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *__restrict__ w,
               const float *__restrict__ bias, const T *__restrict__ state_in, int64_t ss, T *__restrict__ out,
               int64_t o_bs, int64_t o_ts, const int32_t *__restrict__ cu, int nseqs, int64_t seqlen,
@@ -90,29 +94,53 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
     if (!have_hist) load_hist(t0);
     have_hist = true;
     if (!cu || t1 <= end) {
-        // the whole run lies in one sequence: issue every row's load before any math
-        float cur[kTokensPerThread][VEC];
+        // the whole run lies in one sequence: issue every row's load before any
+        // math; rows are held in their raw 16-byte form (bf16 rows take half the
+        // registers of fp32 ones) and widened when used
+        using Row = typename std::conditional<VEC == 8, uint4[sizeof(T) == 2 ? 1 : 2], float[VEC]>::type;
+        Row cur[kTokensPerThread];
 #pragma unroll
         for (int i = 0; i < kTokensPerThread; ++i) {
             if (t0 + i < t1) {
+                const T *src = xr + (t0 + i) * x_ts + c0;
                 if constexpr (VEC == 8) {
-                    Vec8<T>::ld(xr + (t0 + i) * x_ts + c0, cur[i]);
+                    cur[i][0] = *reinterpret_cast<const uint4 *>(src);
+                    if constexpr (sizeof(T) == 4) cur[i][1] = *reinterpret_cast<const uint4 *>(src + 4);
                 } else {
 #pragma unroll
-                    for (int v = 0; v < VEC; ++v) cur[i][v] = Elem<T>::ld(xr + (t0 + i) * x_ts + c0 + v);
+                    for (int v = 0; v < VEC; ++v) cur[i][v] = Elem<T>::ld(src + v);
                 }
             }
         }
+        auto widen = [&](const Row &r, float (&f)[VEC]) {
+            if constexpr (VEC == 8 && sizeof(T) == 2) {
+                const uint32_t w[4] = {r[0].x, r[0].y, r[0].z, r[0].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    f[2 * q] = __uint_as_float(w[q] << 16);
+                    f[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
+                }
+            } else if constexpr (VEC == 8) {
+                const uint4 a0 = r[0], a1 = r[1];
+                f[0] = __uint_as_float(a0.x); f[1] = __uint_as_float(a0.y); f[2] = __uint_as_float(a0.z); f[3] = __uint_as_float(a0.w);
+                f[4] = __uint_as_float(a1.x); f[5] = __uint_as_float(a1.y); f[6] = __uint_as_float(a1.z); f[7] = __uint_as_float(a1.w);
+            } else {
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) f[v] = r[v];
+            }
+        };
 #pragma unroll
         for (int i = 0; i < kTokensPerThread; ++i) {
             if (t0 + i >= t1) break;
+            float cf[VEC];
+            widen(cur[i], cf);
             float o[VEC];
 #pragma unroll
             for (int v = 0; v < VEC; ++v) {
                 float acc = bb[v];
 #pragma unroll
                 for (int k = 0; k < K - 1; ++k) acc = fmaf(wk[k][v], hist[k][v], acc);
-                acc = fmaf(wk[K - 1][v], cur[i][v], acc);
+                acc = fmaf(wk[K - 1][v], cf[v], acc);
                 o[v] = act ? silu(acc) : acc;
             }
             if constexpr (VEC == 8) {
@@ -127,7 +155,7 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
                 for (int v = 0; v < VEC; ++v) hist[k][v] = hist[k + 1][v];
             if (K > 1)
 #pragma unroll
-                for (int v = 0; v < VEC; ++v) hist[K > 1 ? K - 2 : 0][v] = cur[i][v];
+                for (int v = 0; v < VEC; ++v) hist[K > 1 ? K - 2 : 0][v] = cf[v];
         }
         continue;
     }

@@ -449,8 +449,7 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
         // first K-1 tokens for the chunk before it
         __syncthreads();                                  // dxc of every channel written
         for (int idx = tid; idx < kTCb * CPB; idx += kBT) {
-            const int t = idx / CPB, jj = idx % CPB;
-            if (t < nv && K > 0) dxc[idx] = dxc[idx] * dsilu(pre[idx]);
+            if (idx / CPB < nv && K > 0) dxc[idx] = dxc[idx] * dsilu(pre[idx]);
         }
         __syncthreads();
         auto dp_at = [&](int jj, int64_t x) -> float {    // dpre at sequence position x >= t0

@@ -78,13 +78,9 @@ ssm_status validate_scan(const ssm_scan_args *a) {
         G = a->ngroups;
         dtw = a->nheads;
     }
-    int64_t nseq = a->batch;
-    if (a->cu_seqlens) {
-        if (a->batch != 1 || a->nseqs < 0 || a->nseqs > 65535 || (a->nseqs == 0 && a->seqlen > 0))
-            return SSM_ERR_INVALID_ARG;
-        nseq = a->nseqs;
-    }
-    (void)nseq;
+    if (a->cu_seqlens &&
+        (a->batch != 1 || a->nseqs < 0 || a->nseqs > 65535 || (a->nseqs == 0 && a->seqlen > 0)))
+        return SSM_ERR_INVALID_ARG;
     const size_t es = esize(a->dtype);
     const bool work = a->batch > 0 && a->seqlen > 0;
     SSM_TRY(check_act(a->x, a->x_batch_stride, a->x_token_stride, a->d_inner, a->batch, a->seqlen, es, work));
