@@ -194,6 +194,9 @@ class Job:
             self.bytes_per_step = read + wrote
             self.units = self.tokens
             self.bwd = None
+            self.split = None
+            if w.split_ranks:
+                self._split_setup(w, mode, t, dev, bf)
             if w.backward:
                 # upstream gradients of y and h_final; the step is ssm_scan_bwd, whose fp32
                 # gradients of every input are what it writes
@@ -213,6 +216,8 @@ class Job:
                 wrote = sum(v.numel() * v.element_size() for v in self.bwd.values() if v is not None)
                 self.bytes_per_step = read + wrote
                 self.y = self.bwd["dx"]                       # what the end-to-end leg copies back
+            if self.split is not None:
+                x = self.t["x"]
             if w.backward:
                 # executed exps: the checkpoint pass, the per-chunk recompute and the reverse step
                 self.kernel, self.sources = "scan_bwd_kernel", ("scan_bwd.cu",)
@@ -267,8 +272,63 @@ class Job:
         else:
             raise ValueError(w.kind)
 
+    def _split_setup(self, w, mode, t, dev, bf):
+        """One rank's part of an equal token split: the other ranks' conv tails and
+        (sum of delta, end state) pairs are computed once here and staged in HBM, so
+        the step runs exactly this rank's kernels and reads what the exchanges
+        would have delivered."""
+        from state_space_model_conv1d_b200 import seq_split
+        torch, R, r = self.torch, w.split_ranks, w.split_rank
+        seq = ("x", "z", "dt", "B", "C")
+        bounds = [w.seqlen * k // R for k in range(R + 1)]
+        kw = dict(D=t["D"], dt_bias=t["dt_bias"], h0=t["h0"], conv_w=t["conv_w"], conv_b=t["conv_b"],
+                  conv_state_in=t["conv_state_in"])
+        segs = []
+        for k in range(R):
+            s = {n: t[n][:, bounds[k]:bounds[k + 1]] for n in seq}
+            segs.append(seq_split.SegmentScan(mode, k, R, s["x"], s["dt"], t["A"], s["B"], s["C"], z=s["z"], **kw))
+        tails = torch.stack([s_.tail() for s_ in segs])
+        pairs = torch.stack([s_.scan(tails) for s_ in segs])
+        torch.cuda.synchronize()
+        del segs
+        # this rank's segment becomes the job's input (contiguous, pinned on the host for e2e)
+        for n in seq:
+            seg = self.host[n][:, bounds[r]:bounds[r + 1]].contiguous()
+            self.host[n] = seg.pin_memory()
+            t[n] = self.host[n].to(dev)
+        self.host["h0"] = None
+        self.split = dict(R=R, r=r, tails=tails, pairs=pairs, kw=dict(kw, h0=t["h0"] if r == 0 else None,
+                                                                      conv_state_in=t["conv_state_in"] if r == 0 else None),
+                          mod=seq_split)
+        self.tokens = self.units = t["x"].shape[0] * t["x"].shape[1]
+        self.y = torch.empty_like(t["x"])
+        # algorithmic bytes: the segment's inputs and parameters, what the exchanges
+        # deliver (the previous rank's tail, every rank's pair) and what the rank
+        # writes (y, its outgoing state, its tail and its pair)
+        read = sum(t[n].numel() * t[n].element_size() for n in seq if t[n] is not None)
+        read += sum(t[n].numel() * t[n].element_size() for n in ("A", "D", "dt_bias", "conv_w", "conv_b")
+                    if t[n] is not None)
+        read += tails[0].numel() * tails.element_size() + pairs.numel() * pairs.element_size()
+        wrote = self.y.numel() * self.y.element_size() + self.hf.numel() * 4 + tails[0].numel() * tails.element_size() \
+            + pairs[0].numel() * pairs.element_size()
+        self.bytes_per_step = read + wrote
+        # tail, the scan's launches, cum_delta, combine, fix-up (the pair packing and the
+        # staging copy are torch's)
+        self.launches_per_step = 1 + self.launches_per_step + 3
+
+    def _split_step(self):
+        sp, t = self.split, self.t
+        seg = sp["mod"].SegmentScan(self.mode, sp["r"], sp["R"], t["x"], t["dt"], t["A"], t["B"], t["C"], z=t["z"],
+                                    **sp["kw"])
+        seg.tail()
+        sp["pairs"][sp["r"]].copy_(seg.scan(sp["tails"]))
+        self.y, self.hf, _ = seg.join(sp["pairs"])
+
     def step(self):
         ssm, t = self.ssm, self.t
+        if self.split is not None:
+            self._split_step()
+            return
         if self.w.kind == "decode":
             i = self.step_i % self.nsets
             self.step_i += 1
@@ -448,7 +508,8 @@ def run_cuda(args):
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "global_batch": (w.batch or 1) * world, "seq_len": w.seqlen or None,
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "parallelism": (f"seqsplit{w.split_ranks}: rank {w.split_rank}'s step, exchanges staged in HBM"
+                                   if w.split_ranks else (f"replicas{world}" if world > 1 else "single")),
                    "l2": "flushed between timed steps (256 MiB write, outside the events)",
                    "tokens_per_step": job.units},
         "hbm_gbs": gbs, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,

@@ -292,6 +292,64 @@ SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *args, void *stream)
  * SSM_DEVERR_* value.  `code` may be NULL. */
 SSM_API ssm_status ssm_workspace_error(const void *workspace, int32_t *code, void *stream);
 
+/* ------------------------------------------------------- sequence split */
+/* One batch of sequences split along its tokens across R ranks: rank r holds
+ * the contiguous segment r of every batch row (batch mode; no cu_seqlens).
+ * The scan's element (exp(delta*A), h) composes associatively, with seed
+ * (1, h0) ("Adding Initial Value Support to Selective Scan Forward Kernel",
+ * state-spaces/mamba issue 285), so each rank scans its own segment from a
+ * zero state and one exchange of per-segment pairs joins the segments.  Per
+ * rank, in this order:
+ *
+ *   1. ssm_split_conv_tail: the segment's last K-1 raw conv inputs.  Rank r
+ *      passes rank r-1's tail as conv_state_in of its scan (exchange 1).
+ *   2. ssm_scan_fwd on the segment, with the caller's h0 on rank 0 and
+ *      h0 = NULL elsewhere: y_loc and h_loc (its h_final).
+ *   3. ssm_split_cum_delta: cs_t = sum of delta over the segment's tokens up
+ *      to and including t, per batch row and delta unit (channel for
+ *      Mamba-1, head for Mamba-2), and the segment total sum_delta; the
+ *      segment multiplies an incoming state by exp(A * sum_delta).
+ *   4. all ranks exchange (sum_delta, h_loc) (exchange 2, an all-gather).
+ *   5. ssm_split_combine: H_0 = h_loc_0, H_k = exp(A sum_delta_k) H_{k-1}
+ *      + h_loc_k; h_in = H_{r-1} (zero on rank 0) is the state entering the
+ *      segment and h_out = H_r the state leaving it.
+ *   6. ssm_split_fixup (ranks r > 0): y_t += silu(z_t) * C_t . (exp(A cs_t) h_in)
+ *      for every token of the segment (C_t after the conv for Mamba-2).
+ *
+ * y and h_out then equal an unsplit scan of the whole sequence up to
+ * rounding (y is rounded to its dtype twice on ranks r > 0), and the last
+ * rank's h_out and conv_state_out are the sequence's final states.
+ * Every segment must hold at least K-1 tokens so that a tail does not depend
+ * on the segments before it. */
+typedef struct ssm_split_args {
+    int32_t mode;             /* SSM_MAMBA1 or SSM_MAMBA2 */
+    int32_t rank, nranks;     /* 0 <= rank < nranks */
+    int32_t reserved0;
+    int64_t batch, d_inner, nheads, headdim, dstate;   /* as in ssm_scan_args */
+    const float *A;           /* as in ssm_scan_args */
+    const float *sum_delta;   /* [nranks][batch][U] fp32, every rank's step-3 output (U = D or H) */
+    const float *h_local;     /* [nranks][batch][state] fp32, every rank's h_loc */
+    float *h_in;              /* [batch][state] out, or NULL */
+    float *h_out;             /* [batch][state] out, or NULL */
+} ssm_split_args;
+
+/* Step 1.  `tail` is [batch][conv_dim][K-1] in the activation dtype, oldest
+ * first, in the layout of conv_state_out; positions before the segment's
+ * first token come from conv_state_in (zeros when NULL).  Needs d_conv > 1. */
+SSM_API ssm_status ssm_split_conv_tail(const ssm_scan_args *args, void *tail, void *stream);
+/* Step 3.  cum_delta [batch][seqlen][U] fp32 (may be NULL), sum_delta
+ * [batch][U] fp32.  delta as in ssm_scan_fwd (dt + dt_bias, then softplus
+ * when delta_softplus). */
+SSM_API ssm_status ssm_split_cum_delta(const ssm_scan_args *args, float *cum_delta, float *sum_delta,
+                                       void *stream);
+/* Step 5.  No workspace. */
+SSM_API ssm_status ssm_split_combine(const ssm_split_args *args, void *stream);
+/* Step 6.  `args` describes the segment's ssm_scan_fwd call; its y is
+ * updated in place, its h0 / h_final / conv_state_out fields are ignored.
+ * cum_delta is step 3's output, h_in step 5's. */
+SSM_API ssm_status ssm_split_fixup(const ssm_scan_args *args, const float *cum_delta, const float *h_in,
+                                   void *stream);
+
 #ifdef __cplusplus
 }
 #endif

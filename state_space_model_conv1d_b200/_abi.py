@@ -85,6 +85,14 @@ class ScanBwdArgs(C.Structure):
     ]
 
 
+class SplitArgs(C.Structure):
+    _fields_ = [
+        ("mode", _i32), ("rank", _i32), ("nranks", _i32), ("reserved0", _i32),
+        ("batch", _i64), ("d_inner", _i64), ("nheads", _i64), ("headdim", _i64), ("dstate", _i64),
+        ("A", _vp), ("sum_delta", _vp), ("h_local", _vp), ("h_in", _vp), ("h_out", _vp),
+    ]
+
+
 # Every symbol the header declares, with its ctypes signature.
 SIGNATURES = {
     "ssm_abi_version": ([], _i32),
@@ -100,6 +108,10 @@ SIGNATURES = {
     "ssm_scan_bwd": ([C.POINTER(ScanBwdArgs), _vp, C.c_size_t, _vp], _i32),
     "ssm_kernel_timing": ([_i32], _i32),
     "ssm_kernel_time_ms": ([C.POINTER(C.c_float), C.POINTER(_i32)], _i32),
+    "ssm_split_conv_tail": ([C.POINTER(ScanArgs), _vp, _vp], _i32),
+    "ssm_split_cum_delta": ([C.POINTER(ScanArgs), _vp, _vp, _vp], _i32),
+    "ssm_split_combine": ([C.POINTER(SplitArgs), _vp], _i32),
+    "ssm_split_fixup": ([C.POINTER(ScanArgs), _vp, _vp, _vp], _i32),
 }
 
 _lock = threading.Lock()

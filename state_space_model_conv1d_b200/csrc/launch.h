@@ -86,6 +86,16 @@ cudaError_t launch_state_update(const ssm_update_args &a, cudaStream_t st);
 size_t scan_bwd_workspace_bytes(const ssm_scan_bwd_args &a);
 cudaError_t launch_scan_bwd(const ssm_scan_bwd_args &a, const SeqView &sv, void *ws, cudaStream_t st);
 
+// Sequence split across ranks (batch mode): the conv tail a segment hands on,
+// the in-segment prefix sums of delta, the combine of the exchanged pairs,
+// and the fix-up of y by the entering state.
+cudaError_t launch_split_tail(const ssm_scan_args &a, void *tail, cudaStream_t st);
+cudaError_t launch_split_cum_delta(const ssm_scan_args &a, float *cum, float *sum, cudaStream_t st);
+cudaError_t launch_split_combine(const ssm_split_args &a, cudaStream_t st);
+cudaError_t launch_split_fixup(const ssm_scan_args &a, const float *cum, const float *h_in, cudaStream_t st);
+// The fix-up grids tile the tokens along grid.y (16 tokens per CTA row).
+constexpr int64_t kMaxSplitSeqlen = 65535LL * 16;
+
 // Device timing of the dominant kernel of a call (ssm_kernel_timing): a no-op
 // unless enabled; otherwise records one event before and one after on `st`.
 void timing_begin(cudaStream_t st);

@@ -282,6 +282,53 @@ ssm_status ssm_state_update(const ssm_update_args *args, void *stream) {
     return cuda_status(ssm::launch_state_update(*args, (cudaStream_t)stream));
 }
 
+namespace {
+// The split entry points take the segment's ssm_scan_fwd description: batch
+// mode only, and token counts the fix-up grids can tile.
+ssm_status validate_split_scan(const ssm_scan_args *a) {
+    SSM_TRY(validate_scan(a));
+    if (a->cu_seqlens) return SSM_ERR_UNSUPPORTED;
+    if (a->seqlen > ssm::kMaxSplitSeqlen) return SSM_ERR_UNSUPPORTED;
+    return SSM_OK;
+}
+}  // namespace
+
+ssm_status ssm_split_conv_tail(const ssm_scan_args *args, void *tail, void *stream) {
+    SSM_TRY(validate_split_scan(args));
+    if (args->d_conv < 2 || !tail) return SSM_ERR_INVALID_ARG;
+    if (!aligned(tail, esize(args->dtype))) return SSM_ERR_ALIGNMENT;
+    return cuda_status(ssm::launch_split_tail(*args, tail, (cudaStream_t)stream));
+}
+
+ssm_status ssm_split_cum_delta(const ssm_scan_args *args, float *cum_delta, float *sum_delta, void *stream) {
+    SSM_TRY(validate_split_scan(args));
+    if (!sum_delta) return SSM_ERR_INVALID_ARG;
+    if (!aligned(cum_delta, 4) || !aligned(sum_delta, 4)) return SSM_ERR_ALIGNMENT;
+    return cuda_status(ssm::launch_split_cum_delta(*args, cum_delta, sum_delta, (cudaStream_t)stream));
+}
+
+ssm_status ssm_split_combine(const ssm_split_args *a, void *stream) {
+    if (!a) return SSM_ERR_INVALID_ARG;
+    if (a->mode != SSM_MAMBA1 && a->mode != SSM_MAMBA2) return SSM_ERR_INVALID_ARG;
+    if (a->nranks < 1 || a->rank < 0 || a->rank >= a->nranks) return SSM_ERR_INVALID_ARG;
+    if (a->batch < 0 || a->d_inner < 1 || a->dstate < 1) return SSM_ERR_INVALID_ARG;
+    if (a->mode == SSM_MAMBA2 &&
+        (a->nheads < 1 || a->headdim < 1 || a->nheads * a->headdim != a->d_inner))
+        return SSM_ERR_INVALID_ARG;
+    if (!a->A || !a->sum_delta || !a->h_local) return SSM_ERR_INVALID_ARG;
+    if (!aligned(a->A, 4) || !aligned(a->sum_delta, 4) || !aligned(a->h_local, 4) || !aligned(a->h_in, 4) ||
+        !aligned(a->h_out, 4))
+        return SSM_ERR_ALIGNMENT;
+    return cuda_status(ssm::launch_split_combine(*a, (cudaStream_t)stream));
+}
+
+ssm_status ssm_split_fixup(const ssm_scan_args *args, const float *cum_delta, const float *h_in, void *stream) {
+    SSM_TRY(validate_split_scan(args));
+    if (!cum_delta || !h_in) return SSM_ERR_INVALID_ARG;
+    if (!aligned(cum_delta, 4) || !aligned(h_in, 4)) return SSM_ERR_ALIGNMENT;
+    return cuda_status(ssm::launch_split_fixup(*args, cum_delta, h_in, (cudaStream_t)stream));
+}
+
 ssm_status ssm_workspace_error(const void *workspace, int32_t *code, void *stream) {
     if (!workspace) return SSM_ERR_INVALID_ARG;
     SSM_TRY(cuda_status(cudaStreamSynchronize((cudaStream_t)stream)));

@@ -356,3 +356,77 @@ def scan_bwd_workspace_size(mode, x, dt, A, B, C_, dy, *, cu_seqlens=None, conv_
                        True, 0)
     b.dy = _p(dy)
     return int(_abi.lib().ssm_scan_bwd_workspace_size(C.byref(b)))
+
+
+# ---------------------------------------------------------------- sequence split
+# One batch of sequences split along its tokens across ranks (see
+# seq_split.py for the whole protocol).  Each call below takes the segment's
+# tensors as scan_fwd does; y stands in for the output layout and is only
+# written by split_fixup.
+
+def _split_scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, conv_w, conv_b, conv_state_in, y, delta_softplus):
+    return _scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, None, None, None, conv_w, conv_b, conv_state_in, None,
+                      x if y is None else y, delta_softplus, 0)
+
+
+def _conv_dim(mode, x, B):
+    return x.shape[2] if mode == MAMBA1 else x.shape[2] * x.shape[3] + 2 * B.shape[2] * B.shape[3]
+
+
+def split_conv_tail(mode, x, dt, A, B, C_, *, conv_w, D=None, z=None, dt_bias=None, conv_b=None,
+                    conv_state_in=None, delta_softplus=True, tail=None, stream=None):
+    """The segment's last K-1 raw conv inputs, ``[b, conv_dim, K-1]`` in x's dtype (conv_state_out layout)."""
+    K = conv_w.shape[1]
+    if tail is None:
+        tail = torch.empty((x.shape[0], _conv_dim(mode, x, B), K - 1), dtype=x.dtype, device=x.device)
+    a = _split_scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, conv_w, conv_b, conv_state_in, None, delta_softplus)
+    _abi.check(_abi.lib().ssm_split_conv_tail(C.byref(a), _p(tail), _stream(stream)), "ssm_split_conv_tail")
+    return tail
+
+
+def split_cum_delta(mode, x, dt, A, B, C_, *, dt_bias=None, delta_softplus=True, cum=True, D=None, z=None,
+                    conv_w=None, conv_b=None, conv_state_in=None, stream=None):
+    """``(cum_delta [b, T, U] or None, sum_delta [b, U])`` of the segment, fp32 (U = channels or heads)."""
+    U = x.shape[2]
+    b, T = x.shape[0], x.shape[1]
+    cd = torch.empty((b, T, U), dtype=torch.float32, device=x.device) if cum else None
+    sd = torch.empty((b, U), dtype=torch.float32, device=x.device)
+    a = _split_scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, conv_w, conv_b, conv_state_in, None, delta_softplus)
+    _abi.check(_abi.lib().ssm_split_cum_delta(C.byref(a), _p(cd), _p(sd), _stream(stream)), "ssm_split_cum_delta")
+    return cd, sd
+
+
+def split_combine(mode, A, sum_delta_all, h_local_all, rank, *, h_in=None, h_out=None, stream=None):
+    """Fold the gathered ``(sum_delta, h_loc)`` of ranks 0..rank: ``(h_in, h_out)`` of this rank's segment.
+
+    ``sum_delta_all`` is ``[R, b, U]`` and ``h_local_all`` ``[R, b, *state]``, both fp32 contiguous.
+    """
+    R, b = h_local_all.shape[0], h_local_all.shape[1]
+    state = tuple(h_local_all.shape[2:])
+    _c32(sum_delta_all, "sum_delta_all")
+    _c32(h_local_all, "h_local_all")
+    if h_in is None:
+        h_in = torch.empty((b,) + state, dtype=torch.float32, device=h_local_all.device)
+    if h_out is None:
+        h_out = torch.empty((b,) + state, dtype=torch.float32, device=h_local_all.device)
+    a = _abi.SplitArgs()
+    a.mode, a.rank, a.nranks = mode, int(rank), R
+    a.batch = b
+    if mode == MAMBA1:
+        a.d_inner, a.dstate = state[0], state[1]
+    else:
+        a.nheads, a.headdim, a.dstate = state
+        a.d_inner = state[0] * state[1]
+    a.A, a.sum_delta, a.h_local = _p(_c32(A, "A")), _p(sum_delta_all), _p(h_local_all)
+    a.h_in, a.h_out = _p(_c32(h_in, "h_in")), _p(_c32(h_out, "h_out"))
+    _abi.check(_abi.lib().ssm_split_combine(C.byref(a), _stream(stream)), "ssm_split_combine")
+    return h_in, h_out
+
+
+def split_fixup(mode, x, dt, A, B, C_, y, cum_delta, h_in, *, D=None, z=None, dt_bias=None, conv_w=None,
+                conv_b=None, conv_state_in=None, delta_softplus=True, stream=None):
+    """Add the entering state's contribution to the segment's y, in place."""
+    a = _split_scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, conv_w, conv_b, conv_state_in, y, delta_softplus)
+    _abi.check(_abi.lib().ssm_split_fixup(C.byref(a), _p(_c32(cum_delta, "cum_delta")), _p(_c32(h_in, "h_in")),
+                                          _stream(stream)), "ssm_split_fixup")
+    return y

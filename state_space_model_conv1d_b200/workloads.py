@@ -185,6 +185,8 @@ class Workload:
     nsets: int = 1
     state_interval: int = 0   # > 0: intermediate states every this many tokens (prefix caching)
     backward: bool = False    # the step is the backward of the scan (gradients of every input)
+    split_ranks: int = 0      # > 0: the tokens of every row are split into this many equal segments, one per rank
+    split_rank: int = 0       # the rank whose step is measured (its segment, fix-up included)
     seed: int = BASE_SEED
 
 
@@ -210,6 +212,15 @@ WORKLOADS = {
     "mamba2_varlen_16seq_h64_p64_g1_n128_states512": Workload(
         "mamba2_varlen_16seq_h64_p64_g1_n128_states512", "mamba2_varlen", "bf16", nheads=64, headdim=64, ngroups=1,
         dstate=128, nseqs=16, len_lo=128, len_hi=8192, chunk=256, state_interval=512, seed=BASE_SEED + 3),
+    # one rank's step of a two-way token split of the Mamba-2 and Mamba-1
+    # workloads (the second rank: scan of its half from zero, then the fold of
+    # both ranks' pairs and the fix-up of y)
+    "mamba2_ssd_b4_l4096_h80_p64_g8_n128_split2": Workload(
+        "mamba2_ssd_b4_l4096_h80_p64_g8_n128_split2", "mamba2", "bf16", batch=4, seqlen=4096, nheads=80, headdim=64,
+        ngroups=8, dstate=128, chunk=256, split_ranks=2, split_rank=1, seed=BASE_SEED + 2),
+    "mamba1_layer_b8_l2048_d1536_n16_split2": Workload(
+        "mamba1_layer_b8_l2048_d1536_n16_split2", "mamba1", "bf16", batch=8, seqlen=2048, d_inner=1536, dstate=16,
+        split_ranks=2, split_rank=1, seed=BASE_SEED + 1),
     # the Mamba-1 layer's backward (same inputs; upstream gradients drawn alongside)
     "mamba1_layer_b8_l2048_d1536_n16_bwd": Workload("mamba1_layer_b8_l2048_d1536_n16_bwd", "mamba1", "bf16", batch=8,
                                                     seqlen=2048, d_inner=1536, dstate=16, backward=True,

@@ -42,12 +42,15 @@ def test_every_declared_symbol_is_exported():
     assert {e for e in exported if e.startswith("ssm")} == names
 
 
+STRUCTS = (("ssm_conv_args", _abi.ConvArgs), ("ssm_scan_args", _abi.ScanArgs), ("ssm_update_args", _abi.UpdateArgs),
+           ("ssm_scan_bwd_args", _abi.ScanBwdArgs), ("ssm_split_args", _abi.SplitArgs))
+
+
 def test_struct_layouts_match_header(tmp_path):
     """Compile a probe against the real header and compare every field offset
     with the ctypes mirror."""
     probes = []
-    for cname, py in (("ssm_conv_args", _abi.ConvArgs), ("ssm_scan_args", _abi.ScanArgs),
-                      ("ssm_update_args", _abi.UpdateArgs), ("ssm_scan_bwd_args", _abi.ScanBwdArgs)):
+    for cname, py in STRUCTS:
         probes.append(f'printf("{cname} sizeof %zu\\n", sizeof({cname}));')
         for fname, _ in py._fields_:
             probes.append(f'printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
@@ -60,8 +63,7 @@ def test_struct_layouts_match_header(tmp_path):
     for line in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines():
         c, f, v = line.split()
         got[(c, f)] = int(v)
-    for cname, py in (("ssm_conv_args", _abi.ConvArgs), ("ssm_scan_args", _abi.ScanArgs),
-                      ("ssm_update_args", _abi.UpdateArgs), ("ssm_scan_bwd_args", _abi.ScanBwdArgs)):
+    for cname, py in STRUCTS:
         assert got[(cname, "sizeof")] == C.sizeof(py), cname
         for fname, _ in py._fields_:
             assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
@@ -201,3 +203,58 @@ def test_update_rejects(kw, status):
 
 def test_workspace_error_needs_a_workspace():
     assert _abi.lib().ssm_workspace_error(None, None, None) == _abi.SSM_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- sequence split
+@pytest.mark.parametrize("kw,status", [
+    (dict(cu_seqlens=FAKE, nseqs=2, batch=1), _abi.SSM_ERR_UNSUPPORTED),   # batch mode only
+    (dict(seqlen=65535 * 16 + 1, batch=1), _abi.SSM_ERR_UNSUPPORTED),     # longer than the fix-up grid tiles
+    (dict(dstate=1024), _abi.SSM_ERR_UNSUPPORTED),                         # the scan's own checks apply
+    (dict(x=None), _abi.SSM_ERR_INVALID_ARG),
+])
+def test_split_scan_calls_reject(kw, status):
+    lib = _abi.lib()
+    a = _scan(d_conv=4, conv_w=FAKE, **kw)
+    assert lib.ssm_split_conv_tail(C.byref(a), FAKE, None) == status
+    assert lib.ssm_split_cum_delta(C.byref(a), FAKE, FAKE, None) == status
+    assert lib.ssm_split_fixup(C.byref(a), FAKE, FAKE, None) == status
+
+
+def test_split_own_arguments_rejected():
+    lib = _abi.lib()
+    a = _scan(d_conv=4, conv_w=FAKE)
+    assert lib.ssm_split_conv_tail(C.byref(a), None, None) == _abi.SSM_ERR_INVALID_ARG        # no tail buffer
+    assert lib.ssm_split_conv_tail(C.byref(a), FAKE + 1, None) == _abi.SSM_ERR_ALIGNMENT
+    a1 = _scan(d_conv=1, conv_w=FAKE)
+    assert lib.ssm_split_conv_tail(C.byref(a1), FAKE, None) == _abi.SSM_ERR_INVALID_ARG       # no history to hand on
+    assert lib.ssm_split_cum_delta(C.byref(a), FAKE, None, None) == _abi.SSM_ERR_INVALID_ARG  # sum_delta required
+    assert lib.ssm_split_cum_delta(C.byref(a), FAKE + 2, FAKE, None) == _abi.SSM_ERR_ALIGNMENT
+    assert lib.ssm_split_fixup(C.byref(a), None, FAKE, None) == _abi.SSM_ERR_INVALID_ARG
+    assert lib.ssm_split_fixup(C.byref(a), FAKE, None, None) == _abi.SSM_ERR_INVALID_ARG
+
+
+def _split(**kw):
+    a = _abi.SplitArgs()
+    a.mode, a.rank, a.nranks = 2, 1, 2
+    a.batch, a.d_inner, a.nheads, a.headdim, a.dstate = 2, 8, 4, 2, 16
+    a.A, a.sum_delta, a.h_local, a.h_in, a.h_out = FAKE, FAKE, FAKE, FAKE, FAKE
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(rank=2), _abi.SSM_ERR_INVALID_ARG),
+    (dict(rank=-1), _abi.SSM_ERR_INVALID_ARG),
+    (dict(nranks=0, rank=0), _abi.SSM_ERR_INVALID_ARG),
+    (dict(mode=0), _abi.SSM_ERR_INVALID_ARG),
+    (dict(nheads=3), _abi.SSM_ERR_INVALID_ARG),
+    (dict(h_local=None), _abi.SSM_ERR_INVALID_ARG),
+    (dict(sum_delta=None), _abi.SSM_ERR_INVALID_ARG),
+    (dict(A=FAKE + 2), _abi.SSM_ERR_ALIGNMENT),
+    (dict(h_out=FAKE + 1), _abi.SSM_ERR_ALIGNMENT),
+])
+def test_split_combine_rejects(kw, status):
+    a = _split(**kw)
+    assert _abi.lib().ssm_split_combine(C.byref(a), None) == status
+    assert _abi.lib().ssm_split_combine(None, None) == _abi.SSM_ERR_INVALID_ARG

@@ -1,0 +1,90 @@
+"""The sequence split on the GPU against the oracle's unsplit scan.
+
+R ranks are emulated in one process on one GPU: each rank's SegmentScan runs
+its kernels (ssm_split_conv_tail, ssm_scan_fwd, ssm_split_cum_delta,
+ssm_split_combine, ssm_split_fixup) on its own token segment, and the two
+exchanges are stacks of the ranks' tensors.  No kernel waits on another.
+The joined y, every rank's outgoing state and the last rank's conv state are
+compared with the oracle's scan of the whole sequence (and of its prefixes).
+Segment boundaries are ragged and unequal; the cases cover the Mamba-1
+kernel, the tensor-core Mamba-2 kernel (bf16, headdim 64, dstate 128) and the
+SIMT Mamba-2 kernel.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from state_space_model_conv1d_b200 import seq_split
+from state_space_model_conv1d_b200 import workloads as W
+
+from gpu_util import assert_close, oracle_scan, to_dev
+
+pytestmark = pytest.mark.gpu
+M1, M2 = oracle.MAMBA1, oracle.MAMBA2
+SEQ = ("x", "z", "dt", "B", "C")
+
+
+def run_split_gpu(mode, t, bounds):
+    R = len(bounds) - 1
+    segs = []
+    for r in range(R):
+        lo, hi = bounds[r], bounds[r + 1]
+        s = {k: (None if t.get(k) is None else t[k][:, lo:hi]) for k in SEQ}
+        segs.append(seq_split.SegmentScan(mode, r, R, s["x"], s["dt"], t["A"], s["B"], s["C"], D=t["D"], z=s["z"],
+                                          dt_bias=t["dt_bias"], h0=t["h0"], conv_w=t.get("conv_w"),
+                                          conv_b=t.get("conv_b"), conv_state_in=t.get("conv_state_in")))
+    tails = [s.tail() for s in segs]
+    tails = None if tails[0] is None else torch.stack(tails)
+    pairs = torch.stack([s.scan(tails) for s in segs])
+    outs = [s.join(pairs) for s in segs]
+    torch.cuda.synchronize()
+    f = lambda a: None if a is None else a.float().cpu().numpy().astype(np.float64)
+    y = np.concatenate([f(o[0]) for o in outs], axis=1)
+    return y, [f(o[1]) for o in outs], f(outs[-1][2])
+
+
+def _prefix(d, T):
+    return {k: (None if v is None else (v[:, :T] if k in SEQ else v)) for k, v in d.items()}
+
+
+def _check(mode, d, dtype, bounds):
+    y, houts, conv_out = run_split_gpu(mode, to_dev(d, dtype), bounds)
+    ry, rh, rc = oracle_scan(mode, d)
+    assert_close(y, ry, dtype, "y")
+    assert_close(houts[-1], rh, dtype, "h_out of the last rank")
+    for r in range(len(bounds) - 2):
+        _, rhr, _ = oracle_scan(mode, _prefix(d, bounds[r + 1]))
+        assert_close(houts[r], rhr, dtype, f"h_out of rank {r}")
+    if rc is not None:
+        np.testing.assert_array_equal(conv_out, rc)
+
+
+@pytest.mark.parametrize("dtype,bounds", [("bf16", [0, 100, 229, 300]), ("f32", [0, 64, 131]),
+                                          ("bf16", [0, 3, 40, 41 + 64, 170])])
+def test_mamba1(dtype, bounds):
+    d = W.mamba1_inputs(901, 2, bounds[-1], 96, 16, dtype=dtype, conv_bias=True, conv_state=True)
+    _check(M1, d, dtype, bounds)
+
+
+def test_mamba1_no_gate_no_conv():
+    d = W.mamba1_inputs(902, 3, 150, 40, 8, d_conv=0, dtype="f32", with_z=False)
+    _check(M1, d, "f32", [0, 50, 51, 150])
+
+
+@pytest.mark.parametrize("bounds", [[0, 128, 320], [0, 77, 200, 320]])
+def test_mamba2_tensor_core_shape(bounds):
+    d = W.mamba2_inputs(903, 2, bounds[-1], 4, 64, 2, 128, dtype="bf16", conv_bias=True, conv_state=True)
+    _check(M2, d, "bf16", bounds)
+
+
+@pytest.mark.parametrize("dtype,P,N,bounds", [("f32", 8, 16, [0, 30, 61, 95, 130]), ("bf16", 48, 64, [0, 90, 200]),
+                                              ("f32", 64, 256, [0, 40, 97])])
+def test_mamba2_simt_shapes(dtype, P, N, bounds):
+    d = W.mamba2_inputs(904, 2, bounds[-1], 4, P, 2, N, dtype=dtype, conv_bias=True, conv_state=True)
+    _check(M2, d, dtype, bounds)
+
+
+def test_single_rank_is_the_plain_scan():
+    d = W.mamba2_inputs(905, 2, 96, 4, 8, 2, 16, dtype="f32", conv_bias=True, conv_state=True)
+    _check(M2, d, "f32", [0, 96])
