@@ -55,9 +55,10 @@ __global__ void split_tail_kernel(ConvSrc s, const T *__restrict__ state_in, T *
 
 // ----------------------------------------------------------- cum delta
 // A CTA owns 32 delta units of one row and walks the tokens in tiles of
-// 8 warps x 32 tokens: each lane sums its unit over its warp's 32 tokens in
-// registers, the warps' totals go through shared memory, and a running carry
-// joins the tiles.  Loads and stores are 32 consecutive units wide.
+// 8 warps x 32 tokens: each lane issues its 32 loads, then sums its unit over
+// its warp's 32 tokens in registers; the warps' totals go through shared
+// memory, and a running carry joins the tiles.  Loads and stores are 32
+// consecutive units wide.
 constexpr int kCdWarps = 8;
 
 template <typename T>
@@ -75,15 +76,17 @@ split_cum_delta_kernel(const T *__restrict__ dt, int64_t dbs, int64_t dts, const
     float carry = 0.f;
     for (int64_t t0 = 0; t0 < seqlen; t0 += 32 * kCdWarps) {
         const int64_t tw = t0 + 32 * w;
+        const int nv = ok ? (int)max((int64_t)0, min((int64_t)32, seqlen - tw)) : 0;
+        const T *p = src + tw * dts;
         float v[32];
 #pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = i < nv ? Elem<T>::ld(p + i * dts) : 0.f;
+#pragma unroll
         for (int i = 0; i < 32; ++i) {
-            float d = 0.f;
-            if (ok && tw + i < seqlen) {
-                const float r = Elem<T>::ld(src + (tw + i) * dts) + bias;
-                d = softplus_on ? softplus(r) : r;
+            if (i < nv) {
+                const float r = v[i] + bias;
+                v[i] = softplus_on ? softplus(r) : r;
             }
-            v[i] = d;
         }
 #pragma unroll
         for (int i = 1; i < 32; ++i) v[i] += v[i - 1];
@@ -171,6 +174,7 @@ __global__ void __launch_bounds__(kF1Threads) split_fixup_m1_kernel(FixArgs f) {
     }
     const float *Ad = f.A + d * N;
     const float *hd = f.h_in + (b * f.D + d) * N;
+#pragma unroll 4
     for (int n = 0; n < N; ++n) {
         const float a = Ad[n], hv = hd[n];
 #pragma unroll
@@ -188,98 +192,118 @@ __global__ void __launch_bounds__(kF1Threads) split_fixup_m1_kernel(FixArgs f) {
 }
 
 // ------------------------------------------------------- fix-up, Mamba-2
-// A CTA covers 32 tokens of one (row, head) and 64 head channels at a time:
-// the 32 C rows of the head's group after the conv + SiLU (recomputed from
-// the raw inputs and the carried conv state), and the entering state
-// transposed to [n][p] (row stride 65 keeps both the coalesced fill and the
-// read conflict-free).  Each thread owns 8 tokens x 2 channels.
-constexpr int kF2Tok = 32;
+// A CTA covers 64 tokens of one (row, group) and walks the group's heads.
+// The group's 64 C rows after the conv + SiLU (recomputed from the raw inputs
+// and the carried conv state) are built once per CTA; per head and per 64
+// head channels, the entering state is staged transposed ([n][p], row stride
+// 65: the coalesced fill and the reads are both conflict-free).  Warp w owns
+// tokens 16w..16w+15, lane l channels l and l+32: 32 accumulators per thread,
+// C read as broadcast float4 along n when N % 4 == 0.
+constexpr int kF2Tok = 64;
 constexpr int kF2P = 64;
 constexpr int kF2Stride = kF2P + 1;
 constexpr int kF2Threads = 128;
+constexpr int kF2TokPerWarp = kF2Tok / (kF2Threads / 32);
 
 inline size_t fixup_m2_smem(int64_t N) { return (size_t)(kF2Tok * N + N * kF2Stride) * sizeof(float); }
 
-template <typename T>
+template <typename T, bool V4>
 __global__ void __launch_bounds__(kF2Threads) split_fixup_m2_kernel(FixArgs f) {
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     const int N = (int)f.N;
     float *Cs = sm;                      // [kF2Tok][N]
     float *Hs = sm + kF2Tok * N;         // [N][kF2Stride]
-    const int64_t h = blockIdx.x;
+    const int64_t g = blockIdx.x;
     const int64_t t0 = (int64_t)blockIdx.y * kF2Tok;
     const int64_t b = blockIdx.z;
-    const int64_t g = h / (f.H / f.G);
+    const int64_t hpg = f.H / f.G;
     const int nt = (int)min((int64_t)kF2Tok, f.seqlen - t0);
-    const int tid = threadIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const T *Cb = static_cast<const T *>(f.C) + b * f.cbs;
     const T *si = static_cast<const T *>(f.conv_state_in);
     const int K = (int)f.K;
-    for (int idx = tid; idx < kF2Tok * N; idx += kF2Threads) {
-        const int t = idx / N, n = idx % N;
-        float v = 0.f;
-        if (t < nt) {
-            const int64_t tt = t0 + t, col = g * N + n;
-            if (K > 0) {
-                const int64_t ch = f.H * f.P + f.G * N + col;   // conv channel of this C column
-                float acc = f.conv_b ? f.conv_b[ch] : 0.f;
-                for (int k = 0; k < K; ++k) {
-                    const int64_t tau = tt - (K - 1) + k;
-                    float u = 0.f;
-                    if (tau >= 0)
-                        u = Elem<T>::ld(Cb + tau * f.cts + col);
-                    else if (si)
-                        u = Elem<T>::ld(si + (b * f.cdim + ch) * (K - 1) + (tau + K - 1));
-                    acc = fmaf(f.conv_w[ch * K + k], u, acc);
+    for (int t = warp; t < kF2Tok; t += kF2Threads / 32) {
+        for (int n = lane; n < N; n += 32) {
+            float v = 0.f;
+            if (t < nt) {
+                const int64_t tt = t0 + t, col = g * N + n;
+                if (K > 0) {
+                    const int64_t ch = f.H * f.P + f.G * N + col;   // conv channel of this C column
+                    float acc = f.conv_b ? f.conv_b[ch] : 0.f;
+                    for (int k = 0; k < K; ++k) {
+                        const int64_t tau = tt - (K - 1) + k;
+                        float u = 0.f;
+                        if (tau >= 0)
+                            u = Elem<T>::ld(Cb + tau * f.cts + col);
+                        else if (si)
+                            u = Elem<T>::ld(si + (b * f.cdim + ch) * (K - 1) + (tau + K - 1));
+                        acc = fmaf(f.conv_w[ch * K + k], u, acc);
+                    }
+                    v = silu(acc);
+                } else {
+                    v = Elem<T>::ld(Cb + tt * f.cts + col);
                 }
-                v = silu(acc);
+            }
+            Cs[t * N + n] = v;
+        }
+    }
+    const int tb = warp * kF2TokPerWarp;
+    for (int64_t hi = 0; hi < hpg; ++hi) {
+        const int64_t h = g * hpg + hi;
+        const float ah = f.A[h] * kLog2e;
+        const float *hb = f.h_in + (b * f.H + h) * f.P * N;
+        T *yb = static_cast<T *>(const_cast<void *>(f.y)) + b * f.ybs + h * f.P;
+        const T *zb = f.z ? static_cast<const T *>(f.z) + b * f.zbs + h * f.P : nullptr;
+        for (int64_t p0 = 0; p0 < f.P; p0 += kF2P) {
+            __syncthreads();                              // Cs built / the previous Hs consumed
+            for (int p = warp; p < kF2P; p += kF2Threads / 32)
+                for (int n = lane; n < N; n += 32)
+                    Hs[n * kF2Stride + p] = (p0 + p < f.P) ? hb[(p0 + p) * N + n] : 0.f;
+            __syncthreads();
+            float a0[kF2TokPerWarp], a1[kF2TokPerWarp];
+#pragma unroll
+            for (int i = 0; i < kF2TokPerWarp; ++i) a0[i] = a1[i] = 0.f;
+            if constexpr (V4) {
+                for (int n = 0; n < N; n += 4) {
+                    float h0v[4], h1v[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        h0v[j] = Hs[(n + j) * kF2Stride + lane];
+                        h1v[j] = Hs[(n + j) * kF2Stride + lane + 32];
+                    }
+#pragma unroll
+                    for (int i = 0; i < kF2TokPerWarp; ++i) {
+                        const float4 c = *reinterpret_cast<const float4 *>(&Cs[(tb + i) * N + n]);
+                        a0[i] = fmaf(c.x, h0v[0], a0[i]); a1[i] = fmaf(c.x, h1v[0], a1[i]);
+                        a0[i] = fmaf(c.y, h0v[1], a0[i]); a1[i] = fmaf(c.y, h1v[1], a1[i]);
+                        a0[i] = fmaf(c.z, h0v[2], a0[i]); a1[i] = fmaf(c.z, h1v[2], a1[i]);
+                        a0[i] = fmaf(c.w, h0v[3], a0[i]); a1[i] = fmaf(c.w, h1v[3], a1[i]);
+                    }
+                }
             } else {
-                v = Elem<T>::ld(Cb + tt * f.cts + col);
+                for (int n = 0; n < N; ++n) {
+                    const float h0v = Hs[n * kF2Stride + lane], h1v = Hs[n * kF2Stride + lane + 32];
+#pragma unroll
+                    for (int i = 0; i < kF2TokPerWarp; ++i) {
+                        const float c = Cs[(tb + i) * N + n];
+                        a0[i] = fmaf(c, h0v, a0[i]);
+                        a1[i] = fmaf(c, h1v, a1[i]);
+                    }
+                }
             }
-        }
-        Cs[idx] = v;
-    }
-    const int lane = tid & 31, tq = tid >> 5;
-    const float ah = f.A[h] * kLog2e;
-    float e[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int t = tq * 8 + i;
-        e[i] = t < nt ? ex2(ah * f.cum[(b * f.seqlen + t0 + t) * f.H + h]) : 0.f;
-    }
-    const float *hb = f.h_in + (b * f.H + h) * f.P * N;
-    T *yb = static_cast<T *>(const_cast<void *>(f.y)) + b * f.ybs + h * f.P;
-    const T *zb = f.z ? static_cast<const T *>(f.z) + b * f.zbs + h * f.P : nullptr;
-    for (int64_t p0 = 0; p0 < f.P; p0 += kF2P) {
-        __syncthreads();                                  // Cs written / the previous Hs consumed
-        for (int idx = tid; idx < kF2P * N; idx += kF2Threads) {
-            const int p = idx / N, n = idx % N;
-            Hs[n * kF2Stride + p] = (p0 + p < f.P) ? hb[(p0 + p) * N + n] : 0.f;
-        }
-        __syncthreads();
-        float a0[8], a1[8];
+            for (int i = 0; i < kF2TokPerWarp; ++i) {
+                const int t = tb + i;
+                if (t >= nt) break;
+                const float e = ex2(ah * f.cum[(b * f.seqlen + t0 + t) * f.H + h]);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) a0[i] = a1[i] = 0.f;
-        for (int n = 0; n < N; ++n) {
-            const float h0v = Hs[n * kF2Stride + lane], h1v = Hs[n * kF2Stride + lane + 32];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float c = Cs[(tq * 8 + i) * N + n];
-                a0[i] = fmaf(c, h0v, a0[i]);
-                a1[i] = fmaf(c, h1v, a1[i]);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int t = tq * 8 + i;
-            if (t >= nt) break;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int64_t p = p0 + lane + 32 * half;
-                if (p >= f.P) continue;
-                const float gz = zb ? silu(Elem<T>::ld(zb + (t0 + t) * f.zts + p)) : 1.f;
-                T *yp = yb + (t0 + t) * f.yts + p;
-                Elem<T>::st(yp, fmaf(gz * e[i], half ? a1[i] : a0[i], Elem<T>::ld(yp)));
+                for (int half = 0; half < 2; ++half) {
+                    const int64_t p = p0 + lane + 32 * half;
+                    if (p >= f.P) continue;
+                    const float gz = zb ? silu(Elem<T>::ld(zb + (t0 + t) * f.zts + p)) : 1.f;
+                    T *yp = yb + (t0 + t) * f.yts + p;
+                    Elem<T>::st(yp, fmaf(gz * e, half ? a1[i] : a0[i], Elem<T>::ld(yp)));
+                }
             }
         }
     }
@@ -332,11 +356,13 @@ cudaError_t fixup_typed(const ssm_scan_args &a, const float *cum, const float *h
         return cudaGetLastError();
     }
     const size_t smem = fixup_m2_smem(a.dstate);
-    cudaError_t e = cudaFuncSetAttribute(split_fixup_m2_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    dim3 grid((unsigned)a.ngroups, (unsigned)((a.seqlen + kF2Tok - 1) / kF2Tok), (unsigned)a.batch);
+    const bool v4 = a.dstate % 4 == 0;
+    auto kern = v4 ? split_fixup_m2_kernel<T, true> : split_fixup_m2_kernel<T, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)fixup_m2_smem(kMaxDstateM2));
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)a.nheads, (unsigned)((a.seqlen + kF2Tok - 1) / kF2Tok), (unsigned)a.batch);
-    split_fixup_m2_kernel<T><<<grid, kF2Threads, smem, st>>>(f);
+    kern<<<grid, kF2Threads, smem, st>>>(f);
     return cudaGetLastError();
 }
 
