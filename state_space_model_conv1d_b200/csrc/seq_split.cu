@@ -193,19 +193,26 @@ __global__ void __launch_bounds__(kF1Threads) split_fixup_m1_kernel(FixArgs f) {
 
 // ------------------------------------------------------- fix-up, Mamba-2
 // A CTA covers 64 tokens of one (row, group) and walks the group's heads.
-// The group's 64 C rows after the conv + SiLU (recomputed from the raw inputs
-// and the carried conv state) are built once per CTA; per head and per 64
-// head channels, the entering state is staged transposed ([n][p], row stride
-// 65: the coalesced fill and the reads are both conflict-free).  Warp w owns
-// tokens 16w..16w+15, lane l channels l and l+32: 32 accumulators per thread,
-// C read as broadcast float4 along n when N % 4 == 0.
+// The group's raw C rows (from K-1 tokens before the tile, the carried conv
+// state where those precede the segment) are staged once, then convolved
+// (+ SiLU) into the 64 C rows; per head and per 64 head channels, the
+// entering state is staged transposed ([n][p], row stride 65: the coalesced
+// fill and the reads are both conflict-free).  Every staging loop keeps 8 or
+// 16 loads in flight per thread.  Warp w owns tokens 16w..16w+15, lane l
+// channels l and l+32: 32 accumulators per thread, C read as broadcast float4
+// along n when N % 4 == 0.
 constexpr int kF2Tok = 64;
 constexpr int kF2P = 64;
 constexpr int kF2Stride = kF2P + 1;
 constexpr int kF2Threads = 128;
 constexpr int kF2TokPerWarp = kF2Tok / (kF2Threads / 32);
 
-inline size_t fixup_m2_smem(int64_t N) { return (size_t)(kF2Tok * N + N * kF2Stride) * sizeof(float); }
+// C rows, then one region that first holds the staged raw C rows (at most
+// kF2Tok + 7 of them) and later the transposed state
+inline size_t fixup_m2_smem(int64_t N) {
+    return (size_t)(kF2Tok * N + N * (kF2Tok + kMaxConvWidth - 1 > kF2Stride ? kF2Tok + kMaxConvWidth - 1 : kF2Stride)) *
+           sizeof(float);
+}
 
 template <typename T, bool V4>
 __global__ void __launch_bounds__(kF2Threads) split_fixup_m2_kernel(FixArgs f) {
@@ -213,6 +220,7 @@ __global__ void __launch_bounds__(kF2Threads) split_fixup_m2_kernel(FixArgs f) {
     const int N = (int)f.N;
     float *Cs = sm;                      // [kF2Tok][N]
     float *Hs = sm + kF2Tok * N;         // [N][kF2Stride]
+    float *Rs = Hs;                      // [kF2Tok + K - 1][N] raw rows, before the first head
     const int64_t g = blockIdx.x;
     const int64_t t0 = (int64_t)blockIdx.y * kF2Tok;
     const int64_t b = blockIdx.z;
@@ -222,26 +230,51 @@ __global__ void __launch_bounds__(kF2Threads) split_fixup_m2_kernel(FixArgs f) {
     const T *Cb = static_cast<const T *>(f.C) + b * f.cbs;
     const T *si = static_cast<const T *>(f.conv_state_in);
     const int K = (int)f.K;
-    for (int t = warp; t < kF2Tok; t += kF2Threads / 32) {
-        for (int n = lane; n < N; n += 32) {
+    const int Ke = K > 0 ? K : 1;                    // rows of history per output (no conv: the row itself)
+    const int R = kF2Tok + Ke - 1;                   // staged raw rows: tokens t0-Ke+1 .. t0+kF2Tok-1
+    for (int n = lane; n < N; n += 32) {
+        const int64_t col = g * N + n;
+        const int64_t ch = f.H * f.P + f.G * N + col;   // conv channel of this C column
+        for (int r0 = warp; r0 < R; r0 += 8 * (kF2Threads / 32)) {
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = r0 + j * (kF2Threads / 32);
+                const int64_t tau = t0 - (Ke - 1) + r;
+                float u = 0.f;
+                if (r < R && tau < f.seqlen) {
+                    if (tau >= 0)
+                        u = Elem<T>::ld(Cb + tau * f.cts + col);
+                    else if (si)
+                        u = Elem<T>::ld(si + (b * f.cdim + ch) * (K - 1) + (tau + K - 1));
+                }
+                v[j] = u;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = r0 + j * (kF2Threads / 32);
+                if (r < R) Rs[r * N + n] = v[j];
+            }
+        }
+    }
+    __syncthreads();
+    for (int n = lane; n < N; n += 32) {
+        const int64_t ch = f.H * f.P + f.G * N + g * N + n;
+        float w[kMaxConvWidth];
+#pragma unroll
+        for (int k = 0; k < kMaxConvWidth; ++k) w[k] = (k < K) ? f.conv_w[ch * K + k] : 0.f;
+        const float bias = (K > 0 && f.conv_b) ? f.conv_b[ch] : 0.f;
+        for (int t = warp; t < kF2Tok; t += kF2Threads / 32) {
             float v = 0.f;
             if (t < nt) {
-                const int64_t tt = t0 + t, col = g * N + n;
                 if (K > 0) {
-                    const int64_t ch = f.H * f.P + f.G * N + col;   // conv channel of this C column
-                    float acc = f.conv_b ? f.conv_b[ch] : 0.f;
-                    for (int k = 0; k < K; ++k) {
-                        const int64_t tau = tt - (K - 1) + k;
-                        float u = 0.f;
-                        if (tau >= 0)
-                            u = Elem<T>::ld(Cb + tau * f.cts + col);
-                        else if (si)
-                            u = Elem<T>::ld(si + (b * f.cdim + ch) * (K - 1) + (tau + K - 1));
-                        acc = fmaf(f.conv_w[ch * K + k], u, acc);
-                    }
+                    float acc = bias;
+#pragma unroll
+                    for (int k = 0; k < kMaxConvWidth; ++k)
+                        if (k < K) acc = fmaf(w[k], Rs[(t + k) * N + n], acc);
                     v = silu(acc);
                 } else {
-                    v = Elem<T>::ld(Cb + tt * f.cts + col);
+                    v = Rs[t * N + n];
                 }
             }
             Cs[t * N + n] = v;
@@ -255,10 +288,18 @@ __global__ void __launch_bounds__(kF2Threads) split_fixup_m2_kernel(FixArgs f) {
         T *yb = static_cast<T *>(const_cast<void *>(f.y)) + b * f.ybs + h * f.P;
         const T *zb = f.z ? static_cast<const T *>(f.z) + b * f.zbs + h * f.P : nullptr;
         for (int64_t p0 = 0; p0 < f.P; p0 += kF2P) {
-            __syncthreads();                              // Cs built / the previous Hs consumed
-            for (int p = warp; p < kF2P; p += kF2Threads / 32)
-                for (int n = lane; n < N; n += 32)
-                    Hs[n * kF2Stride + p] = (p0 + p < f.P) ? hb[(p0 + p) * N + n] : 0.f;
+            __syncthreads();                              // Cs built (Rs consumed) / the previous Hs consumed
+            for (int n = lane; n < N; n += 32) {
+                constexpr int kRows = kF2P / (kF2Threads / 32);
+                float v[kRows];
+#pragma unroll
+                for (int j = 0; j < kRows; ++j) {
+                    const int p = warp + j * (kF2Threads / 32);
+                    v[j] = (p0 + p < f.P) ? hb[(p0 + p) * N + n] : 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < kRows; ++j) Hs[n * kF2Stride + warp + j * (kF2Threads / 32)] = v[j];
+            }
             __syncthreads();
             float a0[kF2TokPerWarp], a1[kF2TokPerWarp];
 #pragma unroll
