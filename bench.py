@@ -56,7 +56,8 @@ def parse():
 
 def load_peaks():
     if os.path.exists(PEAKS_PATH):
-        d = json.load(open(PEAKS_PATH))
+        with open(PEAKS_PATH) as f:
+            d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
 
@@ -64,7 +65,8 @@ def load_peaks():
 def source_sha(*names):
     h = hashlib.sha256()
     for n in names:
-        h.update(open(os.path.join(ROOT, "state_space_model_conv1d_b200", "csrc", n), "rb").read())
+        with open(os.path.join(ROOT, "state_space_model_conv1d_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -473,7 +475,8 @@ def run_cuda(args):
     kgbs = job.bytes_per_step / (kern_ms / 1e3) / 1e9 if kern_ms > 0 else gbs
     traffic = None
     if os.path.exists(TRAFFIC_PATH):
-        tr = json.load(open(TRAFFIC_PATH)).get(args.workload)
+        with open(TRAFFIC_PATH) as f:
+            tr = json.load(f).get(args.workload)
         if tr and tr.get("source_sha") == source_sha(*job.sources):
             traffic = tr.get("dram_bytes_per_launch")
     if job.mufu is not None:

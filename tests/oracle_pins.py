@@ -78,7 +78,8 @@ def _close(a, b, rtol=1e-11, atol=1e-12, what=""):
     b = np.asarray(b, np.float64)
     if a.shape != b.shape:
         raise AssertionError(f"{what}: shape {a.shape} vs {b.shape}")
-    err = np.max(np.abs(a - b)) if a.size else 0.0
+    with np.errstate(invalid="ignore", over="ignore"):     # a planted mistake may produce inf / nan: it fails below
+        err = np.max(np.abs(a - b)) if a.size else 0.0
     ref = np.max(np.abs(b)) if b.size else 0.0
     if not err <= atol + rtol * ref:
         raise AssertionError(f"{what}: max|err| {err:.3e} (max|ref| {ref:.3e})")

@@ -20,7 +20,8 @@ HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROO
 def declared_symbols():
     names = set()
     for h in HEADERS:
-        src = open(h).read()
+        with open(h) as fh:
+            src = fh.read()
         names |= set(re.findall(r"SSM_API\s+[\w\s\*]+?\b(ssm_\w+)\s*\(", src))
     return names
 

@@ -17,13 +17,18 @@ import oracle_pins as P
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")
 
 
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
 @pytest.mark.parametrize("check", P.ALL_CHECKS, ids=lambda f: f.__name__)
 def test_pin(check):
     check(0)
 
 
 def test_hand_example_scan():
-    g = json.load(open(GOLDEN))["scan_mamba1_two_steps"]
+    g = _golden()["scan_mamba1_two_steps"]
     i = g["inputs"]
     y, hf, _ = oracle.scan_fwd(oracle.MAMBA1, np.array(i["x"]).reshape(1, 2, 1), np.array(i["dt"]).reshape(1, 2, 1),
                                np.array([[i["A"]]]), np.array(i["B"]).reshape(1, 2, 1), np.array(i["C"]).reshape(1, 2, 1),
@@ -34,7 +39,7 @@ def test_hand_example_scan():
 
 
 def test_hand_example_conv():
-    g = json.load(open(GOLDEN))["conv_with_state"]
+    g = _golden()["conv_with_state"]
     i = g["inputs"]
     out, so = oracle.conv1d_fwd(np.array(i["x"]).reshape(1, 2, 1), np.array(i["w"]).reshape(1, 4),
                                 b=np.array([i["bias"]]), state_in=np.array(i["state_in"]).reshape(1, 1, 3),
