@@ -27,7 +27,6 @@ from __future__ import annotations
 import torch
 
 from . import ops
-from .ops import MAMBA1
 
 
 def dist_all_gather(group=None):
@@ -113,4 +112,4 @@ def scan_fwd_seq_split(mode, x, dt, A, B, C_, *, rank, nranks, all_gather=None, 
     return seg.join(pairs)
 
 
-__all__ = ["SegmentScan", "scan_fwd_seq_split", "dist_all_gather", "MAMBA1"]
+__all__ = ["SegmentScan", "scan_fwd_seq_split", "dist_all_gather"]
