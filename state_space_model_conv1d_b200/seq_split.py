@@ -104,6 +104,10 @@ class SegmentScan:
 
 def scan_fwd_seq_split(mode, x, dt, A, B, C_, *, rank, nranks, all_gather=None, group=None, **kw):
     """This rank's segment of a split scan: ``(y, h_out, conv_state_out)`` (see :class:`SegmentScan`)."""
+    if all_gather is None:
+        import torch.distributed as dist
+        if dist.get_world_size(group) != nranks or dist.get_rank(group) != rank:
+            raise ValueError("rank / nranks do not match the process group")
     gather = all_gather if all_gather is not None else dist_all_gather(group)
     seg = SegmentScan(mode, rank, nranks, x, dt, A, B, C_, **kw)
     tail = seg.tail()
