@@ -259,3 +259,14 @@ def test_split_combine_rejects(kw, status):
     a = _split(**kw)
     assert _abi.lib().ssm_split_combine(C.byref(a), None) == status
     assert _abi.lib().ssm_split_combine(None, None) == _abi.SSM_ERR_INVALID_ARG
+
+
+def test_plain_c_consumer(tmp_path):
+    """A C program built against include/ssm.h and linked to libssm.so (no Python in the call path)."""
+    exe = tmp_path / "consumer"
+    libdir = os.path.dirname(_abi.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_consumer.c"), "-o", str(exe), "-L", libdir, "-lssm",
+                    f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout + out.stderr
