@@ -9,8 +9,9 @@ equal the oracle's scan of the whole sequence to rounding.
 
 Mutants of the stand-in show that the comparison sees the mistakes a split
 can make: a dropped segment decay, an exclusive instead of an inclusive
-prefix of delta in the fix-up, and the conv tail handed to the wrong rank.
-The last test runs the protocol on two gloo ranks through torch.distributed.
+prefix of delta in the fix-up, and a lost conv tail.  The protocol also runs
+on two gloo ranks through torch.distributed, and with a rank that holds no
+tokens.
 """
 import os
 import socket
@@ -48,7 +49,7 @@ def _segment(d, lo, hi):
     return out
 
 
-def _kw(s, rank):
+def _kw(s):
     return dict(D=s["D"], z=s["z"], dt_bias=s["dt_bias"], h0=s["h0"], conv_w=s["conv_w"], conv_b=s["conv_b"],
                 conv_state_in=s["conv_state_in"])
 
@@ -56,9 +57,11 @@ def _kw(s, rank):
 def run_split(mode, d, bounds, backend):
     """Every rank's SegmentScan with the exchanges done by stacking: (y, h_outs, conv_out of the last)."""
     R = len(bounds) - 1
-    segs = [seq_split.SegmentScan(mode, r, R, *(lambda s: (s["x"], s["dt"], s["A"], s["B"], s["C"]))(
-        _segment(d, bounds[r], bounds[r + 1])), backend=backend, **_kw(_segment(d, bounds[r], bounds[r + 1]), r))
-        for r in range(R)]
+    segs = []
+    for r in range(R):
+        s = _segment(d, bounds[r], bounds[r + 1])
+        segs.append(seq_split.SegmentScan(mode, r, R, s["x"], s["dt"], s["A"], s["B"], s["C"], backend=backend,
+                                          **_kw(s)))
     tails = [s.tail() for s in segs]
     tails = torch.stack(tails) if tails[0] is not None else None
     pairs = torch.stack([s.scan(tails) for s in segs])
@@ -162,7 +165,7 @@ def _gloo_rank(rank, world, port, mode, bounds, out):
         d = _inputs(mode, 750, bounds[-1])
         s = _segment(d, bounds[rank], bounds[rank + 1])
         y, h_out, conv_out = ss.scan_fwd_seq_split(mode, s["x"], s["dt"], s["A"], s["B"], s["C"], rank=rank,
-                                                   nranks=world, backend=sd_backend, **_kw(s, rank))
+                                                   nranks=world, backend=sd_backend, **_kw(s))
         out[rank] = (y.numpy(), h_out.numpy(), conv_out.numpy())
     finally:
         dist.destroy_process_group()
@@ -187,3 +190,18 @@ def test_two_gloo_ranks_join_to_the_unsplit_scan(mode):
     assert _rel(y, ry) < 1e-11
     assert _rel(out[1][1], rh) < 1e-11
     np.testing.assert_array_equal(out[1][2], rc)
+
+
+@pytest.mark.parametrize("mode", [M1, M2])
+def test_empty_segment_without_conv(mode):
+    """A rank holding no tokens passes the state through unchanged (decay exp(0) = 1, no input)."""
+    bounds = [0, 13, 13, 30]
+    if mode == M1:
+        d = W.mamba1_inputs(760, 2, bounds[-1], 12, 6, d_conv=0, dtype="f32")
+    else:
+        d = W.mamba2_inputs(761, 2, bounds[-1], 4, 3, 2, 5, d_conv=0, dtype="f32")
+    y, houts, _ = run_split(mode, d, bounds, split_double)
+    ry, rh, _ = _ref(mode, d)
+    assert _rel(y, ry) < 1e-11
+    assert _rel(houts[-1], rh) < 1e-11
+    np.testing.assert_array_equal(houts[1], houts[0])
