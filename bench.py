@@ -1,10 +1,13 @@
 #!/usr/bin/env python
 """Throughput benchmark of the conv1d + selective-scan hot path on B200.
 
-Default workload: the Mamba-1 layer (batch 8, 2048 tokens, d_inner 1536,
-dstate 16, conv width 4, bf16 activations, fp32 state); one step is one
-forward pass of the fused conv + scan over that batch.  Other workloads can
-be picked with ``--workload`` (Mamba-2 SSD, packed varlen Mamba-2, decode).
+Default workload: the packed variable-length Mamba-2 batch (16 sequences of
+128..8192 tokens given by cu_seqlens, 56 501 tokens in all, 64 heads of
+headdim 64, one group, dstate 128, conv width 4 over x|B|C, bf16
+activations, fp32 state); one step is one forward pass of the fused conv +
+chunked scan over that batch.  Other workloads can be picked with
+``--workload`` (the Mamba-1 layer, fixed-length Mamba-2, decode, the
+backward, the sequence split).
 
 Prints ONE JSON line (rank 0).  Device time comes from CUDA events on the
 launching stream around each step; L2 is flushed (a 256 MiB write) between
@@ -33,7 +36,7 @@ sys.path.insert(0, ROOT)
 
 from state_space_model_conv1d_b200 import workloads as W  # noqa: E402
 
-DEFAULT_WORKLOAD = "mamba1_layer_b8_l2048_d1536_n16"
+DEFAULT_WORKLOAD = "mamba2_varlen_16seq_h64_p64_g1_n128"
 METRIC = "scan tokens/s"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "dram_traffic.json")
@@ -170,8 +173,8 @@ class Job:
             self.ssd = mode == ssm.MAMBA2 and w.dtype == "bf16" and w.headdim == 64 and w.dstate == 128 and w.d_conv <= 4
             varlen = t.get("cu_seqlens") is not None
             if self.ssd:
-                # B and C conv pre-pass (+ their carried-state kernels), then the chunked tensor-core scan
-                self.launches_per_step = 2 + 2 + 1 + (1 if varlen else 0)
+                # the B / C conv pre-pass, then the chunked tensor-core scan (+ the varlen plan)
+                self.launches_per_step = 2 + (1 if varlen else 0)
             else:
                 self.launches_per_step = 1 + (1 if varlen else 0)
             read = sum(v.numel() * v.element_size() for k, v in t.items() if v is not None)
@@ -231,7 +234,7 @@ class Job:
                 self.mufu = x.shape[0] * x.shape[1] * x.shape[2] * t["B"].shape[2]
                 self.flops = None
             elif self.ssd:
-                self.kernel, self.sources = "ssd_kernel", ("ssd_m2.cu", "conv1d.cu")
+                self.kernel, self.sources = "ssd_kernel", ("ssd_m2.cu",)
                 self.mufu = None
                 # tensor-core work of the 64-token chunked form: per (sequence, head, chunk)
                 # C.B^T (2 Q^2 N) + M.X (2 Q^2 P) + C'.S^T (2 Q N P) + B'^T.X (2 Q N P)

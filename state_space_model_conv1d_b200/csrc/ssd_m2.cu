@@ -6,10 +6,10 @@
 //   S_t = exp(delta_t A) S_{t-1} + delta_t x_t B_t^T,   y_t = S_t C_t + D x_t
 // is evaluated exactly (up to rounding) chunk by chunk.  For a chunk of Q
 // tokens with cs_i = sum_{j<=i} delta_j A (the running log-decay):
-//   G   = C B^T                                             (Q x Q)
-//   M   = G o L,  L[i, j] = exp(cs_i - cs_j) delta_j for j <= i, else 0
-//   Y   = M X + diag(exp(cs)) C S_prev^T                    (Q x P)
-//   S   = exp(cs_Q) S_prev + B'^T X,  B'[j] = exp(cs_Q - cs_j) delta_j B[j]
+//   G     = C B^T                                             (Q x Q)
+//   M     = G o L,  L[i, j] = exp(cs_i - cs_j) delta_j for j <= i, else 0
+//   Y     = M X + diag(exp(cs)) (C S_prev^T)                  (Q x P)
+//   S     = exp(cs_Q) S_prev + B^T X',  X'[j] = exp(cs_Q - cs_j) delta_j X[j]
 // with S_prev = h0 for the first chunk ("Adding Initial Value Support to
 // Selective Scan Forward Kernel", state-spaces/mamba issue 285: the carried
 // state seeds the scan).  The kernel names in "Clean up SSM ops directory
@@ -17,21 +17,42 @@
 // ssd_state_passing, ssd_chunk_scan) are these four steps; here they are one
 // kernel whose carried state never leaves the SM.
 //
-// Layout of the work: one CTA per (sequence, head), 8 warps, walking the
-// sequence in chunks of Q = 64.  The B / C causal conv + SiLU is shared by the
-// heads of a group, so it runs once per group in a pre-pass that writes bf16
-// B, C into the workspace; the x conv + SiLU runs here, fused.  Per chunk:
-//   MMA1  G  = C B^T         M=64  N=64 K=128   A K-major, B K-major
-//   MMA2  Y  = M X           M=64  N=64 K=64    A K-major, B MN-major
-//   MMA3  Y += C' S_prev^T   M=64  N=64 K=128   A K-major, B MN-major
-//   MMA4  Sc = B'^T X        M=128 N=64 K=64    A MN-major (same tile as B), B MN-major
-// C' and B' are C and B rescaled in place after MMA1 has consumed them.
-// The fp32 state S (128 x 64 per head) stays in registers, half a state row
-// per thread; its bf16 copy is the MMA3 operand of the next chunk.  Warps w
-// and w+4 share a tensor-memory lane quarter and split accumulator columns.
+// Work: one CTA per (sequence, head), two CTAs per SM.  The B / C causal
+// conv + SiLU is shared by the heads of a group, so it runs once per group in
+// a pre-pass that writes bf16 B, C into the workspace; the x conv + SiLU runs
+// here.  Per chunk of Q = 64 tokens, four tensor-core products:
+//   G   = C B^T     M=64  N=64 K=128  A K-major,  B K-major      -> TMEM 0..63
+//   Yo  = C S^T     M=64  N=64 K=128  A K-major,  B MN-major     -> TMEM 128..191
+//   Sc  = B^T X'    M=128 N=64 K=64   A MN-major, B MN-major     -> TMEM 192..255
+//   Y   = M X       M=64  N=64 K=64   A K-major,  B MN-major     -> TMEM 64..127
+// B and C are used as loaded (shared by every head of the group): the decay
+// of the chunk-state product rides on X' (written by the x conv next to X),
+// and the exp(cs_i) factor of the state read-out is applied to Yo in the
+// epilogue, so no operand tile is rescaled in place.
 //
-// Tensor memory: 128 columns (G in columns 0-63, later reused for Sc; Y in
-// 64-127), shared memory 67 KB, so three CTAs fit on one SM.
+// Warp roles.  Warps 0-7 compute; warp 8 is the control warp.  Its lane 0
+// issues every TMA load and every MMA as soon as the inputs are ready
+// (mbarriers), and the whole warp computes the per-chunk decay tables three
+// chunks ahead, so no compute warp issues, waits to issue, or scans delta.
+// Compute iteration k:
+//   conv(k+1)   raw x -> X (double-buffered), X'             overlaps MMA Y(k)
+//   epilogue(k) y = (Y + exp(cs) Yo) silu(z) -> TMA store
+//   S(k)        S = exp(cs_Q) S + Sc (fp32 registers) -> bf16 copy for Yo(k+1)
+//   mask(k+1)   G -> M
+// and the control warp, for chunk k+1: G as soon as B / C have landed; the
+// raw x of chunk k+3 once conv(k+1) has read its staging buffer (raw x is
+// double-buffered, so a load has two chunks to land); z of chunk k+1 once the
+// epilogue has read z(k); Sc and Yo once S(k) is written; Y once the mask is
+// written; B / C of chunk k+2 once G, Sc and Yo have read them.  The serial
+// chain across chunks is only the fp32 state update.
+//
+// Tensor memory: 256 columns.  Shared memory ~111 KB.  All mbarrier waits
+// are bounded; a wait that runs out records SSM_DEVERR_TIMEOUT, raises a CTA
+// abort flag that ends every other wait, and the CTA drains its in-flight
+// copies and MMAs before it frees tensor memory and returns.
+#include <stddef.h>
+#include <string.h>
+
 #include "common.cuh"
 #include "launch.h"
 #include "tc05.cuh"
@@ -39,24 +60,32 @@
 namespace ssm {
 namespace {
 
-constexpr int kQ = 64;           // chunk length
-constexpr int kP = 64;           // headdim on this path
-constexpr int kN = 128;          // dstate on this path
-constexpr int kThreads = 256;
-constexpr int kHx = 3;           // raw x rows kept before each chunk (conv width <= 4)
-constexpr uint32_t kTmemCols = 128;
+constexpr int kQ = 64;                     // chunk length
+constexpr int kP = 64;                     // headdim on this path
+constexpr int kN = 128;                    // dstate on this path
+constexpr int kComputeWarps = 8;
+constexpr int kComputeThreads = kComputeWarps * 32;
+constexpr int kThreads = kComputeThreads + 32;   // + the control warp
+constexpr int kHx = 3;                     // raw x rows kept before each chunk (conv width <= 4)
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t TM_G = 0, TM_Y = 64, TM_YO = 128, TM_SC = 192;
 
-// operand tiles (bf16, 128-byte swizzle, atoms of 8 rows x 64 elements), byte
-// offsets from the 1024-aligned base of dynamic shared memory
-constexpr uint32_t OFF_C = 0;        // C rows i, K = n: two 8 KB K-atoms (n 0-63 | 64-127)
-constexpr uint32_t OFF_B = 16384;    // B rows j, K = n (MMA1); read as MN-major MN = n, K = j (MMA4)
-constexpr uint32_t OFF_M = 32768;    // M rows i, K = j; raw x rows are staged here between MMA2 and the mask
-constexpr uint32_t OFF_X = 40960;    // X rows j, 64 p each: MN-major MN = p, K = j (MMA2, MMA4)
-constexpr uint32_t OFF_S = 49152;    // S rows n, 64 p each: MN-major MN = p, K = n (MMA3)
-constexpr uint32_t OFF_AUX = 65536;
+// Operand tiles (bf16, 128-byte swizzle, atoms of 8 rows x 64 elements), byte
+// offsets from the 1024-aligned base of dynamic shared memory.
+constexpr uint32_t OFF_C = 0;          // C rows i, K = n: two 8 KB K-atoms (n 0-63 | 64-127)
+constexpr uint32_t OFF_B = 16384;      // B rows j, K = n (G); read as MN-major MN = n, K = j (Sc)
+constexpr uint32_t OFF_S = 32768;      // bf16 S rows n, 64 p each: MN-major MN = p, K = n (Yo)
+constexpr uint32_t OFF_M = 49152;      // M rows i, K = j (blocks above the diagonal stay zero)
+constexpr uint32_t OFF_X = 57344;      // X rows j, 64 p: two buffers (chunk parity); y staging
+constexpr uint32_t OFF_XP = 73728;     // X' rows j, 64 p
+constexpr uint32_t OFF_XR = 81920;     // raw x rows (row-major, 128 bytes each): two buffers
+constexpr uint32_t OFF_Z = 98304;      // z rows i, 64 p (128-byte swizzle)
+constexpr uint32_t OFF_AUX = 106496;
 
-// per-chunk decay tables, written by warp 0 one chunk ahead (double buffered by chunk parity)
-struct Tables {
+// per-chunk decay tables (three slots: chunk c lives in slot c % 3 and is read
+// in compute iterations c-1 and c; the control warp fills slot c % 3 with
+// chunk c + 3 once S(c) is done)
+struct alignas(16) Tables {            // 16-byte aligned: the x conv reads wj as float4
     float dlt[kQ];                   // delta
     float cs2[kQ];                   // running log2-decay
     float ecs[kQ];                   // exp(cs_i)
@@ -66,13 +95,20 @@ struct Tables {
     float bf[4][4];                  // exp(cs_{16*I} - cs_{16*J+15}) for blocks J < I
     float dAc;                       // exp(cs_Q)
 };
+// mbarriers.  Raw x has one barrier per buffer (a buffer completes every
+// other chunk); the tables one per slot.
+enum {
+    MB_X0, MB_X1, MB_BC, MB_Z, MB_G, MB_MMA, MB_BCFREE, MB_CONV, MB_ZFREE, MB_SREADY, MB_MREADY,
+    MB_T0, MB_T1, MB_T2, MB_DRAIN, kNumMbar
+};
 struct Aux {
     float xh[2][kHx][kP];            // raw x rows before the chunk (double buffered)
-    Tables tab[2];
-    float half_sum[2];               // per-warp sums of the two-warp delta scan
+    Tables tab[3];                   // at a 16-byte offset (xh is 1536 bytes)
     uint32_t tmem;
-    uint64_t mbar[4];                // MMA1 done, MMA2-4 done, raw x landed, B / C landed
+    int abort;
+    uint64_t mb[kNumMbar];
 };
+static_assert(sizeof(Tables) % 16 == 0 && offsetof(Aux, tab) % 16 == 0, "table slots must be 16-byte aligned");
 constexpr size_t kSmemBytes = OFF_AUX + sizeof(Aux) + 1024;   // + slack to align the base to 1024
 
 constexpr uint32_t ID_G = tc::idesc_bf16(64, 64, 0, 0);
@@ -96,26 +132,48 @@ struct SsdArgs {
     int64_t braw_bs, braw_ts, craw_bs, craw_ts;
 };
 
-SSM_DEVINL uint4 ld16(const void *p) { return *reinterpret_cast<const uint4 *>(p); }
 SSM_DEVINL void st16(void *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
+SSM_DEVINL void bar_compute() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+SSM_DEVINL void mb_arrive(uint64_t *mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(tc::smem_u32(mbar)) : "memory");
+}
 
+// Bounded wait on one mbarrier phase that also gives up as soon as another
+// thread of the CTA has raised the abort flag.  The waiting thread sleeps in
+// try_wait (100 us hint) rather than spinning; a wait that lasts longer than
+// two seconds raises the flag itself and records the timeout in the device
+// error word.
+constexpr uint32_t kSleepHintNs = 100000;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+SSM_DEVINL bool wait_mb(Aux &ax, int i, uint32_t parity, int32_t *err) {
+    if (tc::mbar_try_wait_sleep(&ax.mb[i], parity, kSleepHintNs)) return true;
+    const uint64_t t0 = tc::globaltimer_ns();
+    for (;;) {
+        if (*reinterpret_cast<volatile int *>(&ax.abort)) return false;
+        if (tc::mbar_try_wait_sleep(&ax.mb[i], parity, kSleepHintNs)) return true;
+        if (tc::globaltimer_ns() - t0 > kWaitLimitNs) break;
+    }
+    *reinterpret_cast<volatile int *>(&ax.abort) = 1;
+    if (err) atomicExch(err, SSM_DEVERR_TIMEOUT);
+    return false;
+}
+SSM_DEVINL bool aborted(Aux &ax) { return *reinterpret_cast<volatile int *>(&ax.abort) != 0; }
 
 // Tensor maps (3-d: channel, token, batch row; bf16):
 //   tm_x  raw x, box 64 x 64 rows, no swizzle    -> row-major staging rows of 128 bytes
 //   tm_b, tm_c  conv'd B / C, box 64 x 64, 128-byte swizzle -> one K-atom of the operand tile
+//   tm_z  z, box 64 x 64, 128-byte swizzle       -> the z tile the epilogue reads
 //   tm_y  y, box 64 x 64, 128-byte swizzle       <- the y staging tile (rows past the tensor are skipped)
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 2)
 ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-           const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y) {
+           const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_z,
+           const __grid_constant__ CUtensorMap tm_y) {
     extern __shared__ unsigned char smem_raw[];
     // swizzle atoms need 1024-byte alignment: round the base up (1 KB of slack is allocated)
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     Aux &ax = *reinterpret_cast<Aux *>(smem + OFF_AUX);
-    if (a.sv.err && *a.sv.err != 0) return;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q4 = warp & 3;          // tensor-memory lane quarter of this warp
-    const int half = warp >> 2;       // which 32 columns of a 64-column accumulator this warp reads
     const int hh = blockIdx.x;
     const int s = a.sv.order ? a.sv.order[blockIdx.y] : (int)blockIdx.y;
     int64_t start = 0, len = a.seqlen, row = s;
@@ -126,430 +184,667 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
     }
     const int64_t H = a.H, g = hh / (H / a.G);
     const int K = a.K;
-    const __nv_bfloat16 *zg = a.z ? a.z + row * a.z_bs + start * a.z_ts + hh * kP : nullptr;
-    const __nv_bfloat16 *dtg = a.dt + row * a.dt_bs + start * a.dt_ts + hh;
-    __nv_bfloat16 *yg = a.y + row * a.y_bs + start * a.y_ts + hh * kP;
+    const int n = (int)((len + kQ - 1) / kQ);
+    const int crow = (int)row, g0 = (int)(g * kN);
     const uint32_t sbase = tc::smem_u32(smem);
+    const float A2 = a.A[hh] * kLog2e;
 
-    if (warp == 0) tc::tmem_alloc(&ax.tmem, kTmemCols);
     if (tid == 0) {
-        for (int i = 0; i < 4; ++i) tc::mbar_init(&ax.mbar[i], 1);
+        // one thread reads the error word, so every thread of the CTA takes the same branch below
+        ax.abort = (a.sv.err && *a.sv.err != 0) ? 1 : 0;
+        for (int i = 0; i < kNumMbar; ++i)
+            tc::mbar_init(&ax.mb[i], (i == MB_CONV || i == MB_ZFREE || i == MB_SREADY || i == MB_MREADY) ? kComputeWarps : 1);
         tc::mbar_init_fence();
         tc::prefetch_map(&tm_x);
         tc::prefetch_map(&tm_b);
         tc::prefetch_map(&tm_c);
+        if (a.z) tc::prefetch_map(&tm_z);
         tc::prefetch_map(&tm_y);
     }
-
-    // ---- per-thread constants
-    const float A2 = a.A[hh] * kLog2e;
-    const float Dh = a.D ? a.D[hh] : 0.f;
-    const float dtb = a.dt_bias ? a.dt_bias[hh] : 0.f;
-    // x conv role: channels 2 cq, 2 cq + 1 (one packed pair), tokens cr0 .. cr0+7;
-    // taps right-aligned (cw3 multiplies the current token, cw0 the one 3 back)
-    const int cq = tid & 31, cr0 = warp * (kQ / 8);
-    float2 cw0, cw1, cw2, cw3, cbias;
-    {
-        const int64_t ch = hh * kP + 2 * cq;
-        auto tap = [&](int j) {
-            const int k = K - 4 + j;
-            return (K > 0 && k >= 0) ? make_float2(a.conv_w[ch * K + k], a.conv_w[(ch + 1) * K + k]) : make_float2(0.f, 0.f);
-        };
-        cw0 = tap(0); cw1 = tap(1); cw2 = tap(2); cw3 = tap(3);
-        cbias = a.conv_b ? make_float2(a.conv_b[ch], a.conv_b[ch + 1]) : make_float2(0.f, 0.f);
-    }
-
-    // ---- carried state: thread owns S[n][32*half .. 32*half+31] for n = 32*q4 + lane (fp32)
-    const int sn = q4 * 32 + lane;
-    float S[32];
-    {
-        const float *h0p = a.h0 ? a.h0 + ((int64_t)s * H + hh) * kP * kN : nullptr;
-#pragma unroll
-        for (int p = 0; p < 32; ++p) S[p] = h0p ? h0p[(int64_t)(half * 32 + p) * kN + sn] : 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            st16(smem + OFF_S + tc::off_sw128(sn, half * 32 + q * 8, 8192), tc::pack_bf16x8(&S[q * 8]));
-    }
-    // ---- conv halo of chunk 0 (the last K-1 raw inputs before the sequence)
-    if (tid < kP) {
-        const int p = tid;
-#pragma unroll
-        for (int j = 0; j < kHx; ++j) {
-            const int q = j - (kHx - (K - 1));          // index into the carried conv state
-            float v = 0.f;
-            if (K > 1 && q >= 0 && a.conv_state_in)
-                v = __bfloat162float(a.conv_state_in[((int64_t)s * a.cdim + hh * kP + p) * (K - 1) + q]);
-            ax.xh[0][j][p] = v;
-        }
-    }
+    if (warp == kComputeWarps) tc::tmem_alloc(&ax.tmem, kTmemCols);
+    // the mask tile's blocks above the diagonal are zero for good
+    for (int i = tid; i < 8192 / 16; i += kThreads) st16(smem + OFF_M + i * 16, make_uint4(0, 0, 0, 0));
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = ax.tmem;
-    const uint32_t t_lane = (uint32_t)(q4 * 32) << 16;
-    bool ok = true;
-    int fail_bar = 0;
-    uint32_t fail_par = 0;
-
-    const int nchunks = (int)((len + kQ - 1) / kQ);
-    const int crow = (int)row, g0 = (int)(g * kN);
-    // Stage chunk cn (thread 0): the raw x rows (row-major [kQ][kP] bf16) into the
-    // M tile's space, which is free from the end of MMA2 until the mask phase of
-    // the next chunk, and B / C straight into their swizzled operand tiles.  Rows
-    // past the tensor's end arrive as zeros; rows past a packed sequence's end
-    // belong to the next sequence and are zeroed after landing (B / C) or never
-    // used (x).
-    auto prefetch = [&](int cn) {
-        const int tok = (int)(start + (int64_t)cn * kQ);
-        tc::mbar_expect_tx(&ax.mbar[2], kQ * kP * 2);
-        tc::tma_load_3d(smem + OFF_M, &tm_x, (int)(hh * kP), tok, crow, &ax.mbar[2]);
-        tc::mbar_expect_tx(&ax.mbar[3], 4 * kQ * 64 * 2);
-        tc::tma_load_3d(smem + OFF_B, &tm_b, g0, tok, crow, &ax.mbar[3]);
-        tc::tma_load_3d(smem + OFF_B + 8192, &tm_b, g0 + 64, tok, crow, &ax.mbar[3]);
-        tc::tma_load_3d(smem + OFF_C, &tm_c, g0, tok, crow, &ax.mbar[3]);
-        tc::tma_load_3d(smem + OFF_C + 8192, &tm_c, g0 + 64, tok, crow, &ax.mbar[3]);
-    };
-    // raw dt of chunk cn for warps 0 and 1 (lane l of warp w holds token 32 w + l);
-    // kept as bf16 so the load is not waited for until the tables need it
-    __nv_bfloat16 dtr = __float2bfloat16_rn(0.f);
-    auto load_dt = [&](int cn) {
-        const int64_t tn = (int64_t)cn * kQ;
-        const int nvn = (int)min((int64_t)kQ, len - tn);
-        const int j = warp * 32 + lane;
-        dtr = j < nvn ? dtg[(tn + j) * a.dt_ts] : __float2bfloat16_rn(0.f);
-    };
-    // delta, running log2-decay and the mask factor tables of chunk cn (warps 0
-    // and 1, one token per lane), from the raw dt loaded by load_dt(cn), into
-    // table slot cn % 2.  The two half-chunk scans meet through shared memory
-    // and a 64-thread named barrier.
-    auto dt_tables = [&](int cn) {
-        Tables &tw = ax.tab[cn & 1];
-        const int nvn = (int)min((int64_t)kQ, len - (int64_t)cn * kQ);
-        const int j = warp * 32 + lane;
-        const float u = __bfloat162float(dtr) + dtb;
-        const float d = j < nvn ? (a.softplus ? softplus(u) : u) : 0.f;
-        float sc = d * A2;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float v = __shfl_up_sync(0xffffffffu, sc, o);
-            if (lane >= o) sc += v;
-        }
-        if (lane == 31) ax.half_sum[warp] = sc;
-        asm volatile("bar.sync 1, 64;\n" ::: "memory");
-        const float h0s = ax.half_sum[0];
-        if (warp == 1) sc += h0s;
-        const float last = h0s + ax.half_sum[1];
-        // block boundaries: token 16*(j/16) (start) and 16*(j/16)+15 (end)
-        const float st = __shfl_sync(0xffffffffu, sc, lane & ~15);
-        const float en = __shfl_sync(0xffffffffu, sc, lane | 15);
-        tw.dlt[j] = d;
-        tw.cs2[j] = sc;
-        tw.ecs[j] = ex2(sc);
-        tw.wj[j] = ex2(last - sc) * d;
-        tw.rf[j] = ex2(sc - st);
-        tw.cf[j] = ex2(en - sc) * d;
-        asm volatile("bar.sync 1, 64;\n" ::: "memory");
-        if (warp == 0 && lane < 16) {
-            // block factor (I, J), J < I: exp(cs[16 I] - cs[16 J + 15]) (<= 1)
-            const int I = lane >> 2, J = lane & 3;
-            tw.bf[I][J] = J < I ? ex2(tw.cs2[16 * I] - tw.cs2[16 * J + 15]) : 0.f;
-        }
-        if (warp == 0 && lane == 16) tw.dAc = ex2(last);
-    };
-    if (nchunks > 0) {
-        if (tid == 0) prefetch(0);
-        if (warp < 2) {
-            load_dt(0);
-            dt_tables(0);
-            if (nchunks > 1) load_dt(1);
-        }
+    if (ax.abort) {
         __syncthreads();
+        if (warp == kComputeWarps) tc::tmem_dealloc(tmem, kTmemCols);
+        return;
     }
-    const unsigned char *xraw = smem + OFF_M;                      // staged raw x rows of the current chunk
 
-    for (int c = 0; c < nchunks; ++c) {
-        const int64_t t0 = (int64_t)c * kQ;
-        const int nv = (int)min((int64_t)kQ, len - t0);
-        const int hb = c & 1;
-        // rows past a packed sequence's end belong to the next sequence: zero them in B / C
-        const bool zfill = nv < kQ && a.sv.cu != nullptr;
-        if (zfill) {
-            if (!tc::mbar_wait(&ax.mbar[3], c & 1)) { fail_bar = 3; fail_par = c & 1; ok = false; }
-            const uint4 zero4 = make_uint4(0, 0, 0, 0);
-            for (int i = tid; i < (kQ - nv) * (kN / 8); i += kThreads) {
-                const int r = nv + i / (kN / 8), q = i % (kN / 8);
-                const uint32_t off = tc::off_sw128(r, q * 8, 8192);
-                st16(smem + OFF_B + off, zero4);
-                st16(smem + OFF_C + off, zero4);
-            }
-            tc::fence_proxy_async();
-            __syncthreads();
-        }
-        // ---- MMA1: G = C B^T into columns 0..63, issued as soon as B / C have landed; runs under the conv
-        if (tid == 0) {
-            if (!zfill && !tc::mbar_wait(&ax.mbar[3], c & 1)) { fail_bar = 3; fail_par = c & 1; ok = false; }
-            tc::fence_after_sync();
+    if (warp == kComputeWarps) {
+        // ------------------------------------------------------------ control warp
+        const bool lead = lane == 0;
+        const float dtb = a.dt_bias ? a.dt_bias[hh] : 0.f;
+        const __nv_bfloat16 *dtg = a.dt + row * a.dt_bs + start * a.dt_ts + hh;
+        int last_x[2] = {-1, -1};
+        int last_bc = -1, last_z = -1;
+        auto load_x = [&](int cn) {
+            const int b = cn & 1;
+            tc::mbar_expect_tx(&ax.mb[MB_X0 + b], kQ * kP * 2);
+            tc::tma_load_3d(smem + OFF_XR + b * 8192, &tm_x, (int)(hh * kP), (int)(start + (int64_t)cn * kQ), crow,
+                            &ax.mb[MB_X0 + b]);
+            last_x[b] = cn;
+        };
+        auto load_bc = [&](int cn) {
+            const int tok = (int)(start + (int64_t)cn * kQ);
+            tc::mbar_expect_tx(&ax.mb[MB_BC], 4 * kQ * 64 * 2);
+            tc::tma_load_3d(smem + OFF_B, &tm_b, g0, tok, crow, &ax.mb[MB_BC]);
+            tc::tma_load_3d(smem + OFF_B + 8192, &tm_b, g0 + 64, tok, crow, &ax.mb[MB_BC]);
+            tc::tma_load_3d(smem + OFF_C, &tm_c, g0, tok, crow, &ax.mb[MB_BC]);
+            tc::tma_load_3d(smem + OFF_C + 8192, &tm_c, g0 + 64, tok, crow, &ax.mb[MB_BC]);
+            last_bc = cn;
+        };
+        auto load_z = [&](int cn) {
+            tc::mbar_expect_tx(&ax.mb[MB_Z], kQ * kP * 2);
+            tc::tma_load_3d(smem + OFF_Z, &tm_z, (int)(hh * kP), (int)(start + (int64_t)cn * kQ), crow, &ax.mb[MB_Z]);
+            last_z = cn;
+        };
+        // raw dt of chunk cn: lane l holds tokens l and l + 32 (kept as bf16 until the tables need them)
+        auto load_dt = [&](int cn, __nv_bfloat16 (&d)[2]) {
+            const int64_t tn = (int64_t)cn * kQ;
+            const int nvn = (int)min((int64_t)kQ, len - tn);
 #pragma unroll
-            for (int k = 0; k < kN / 16; ++k) {
-                const uint32_t ko = (k >> 2) * 8192 + (k & 3) * 32;
-                tc::mma_bf16(tmem, tc::desc_sw128(sbase + OFF_C + ko, 16, 1024), tc::desc_sw128(sbase + OFF_B + ko, 16, 1024),
-                             ID_G, k > 0);
+            for (int h = 0; h < 2; ++h) {
+                const int j = lane + 32 * h;
+                d[h] = j < nvn ? dtg[(tn + j) * a.dt_ts] : __float2bfloat16_rn(0.f);
             }
-            tc::mma_commit(&ax.mbar[0]);
-        }
-        if (!tc::mbar_wait(&ax.mbar[2], c & 1)) { fail_bar = 2; fail_par = c & 1; ok = false; }
-
-        // ---- (1) x conv from the staged raw rows
-        {
-            // conv + SiLU of a channel pair over 8 tokens, sliding window in registers,
-            // packed fp32x2 arithmetic, one 4-byte store per token into the X tile
-            auto raw2 = [&](int v) -> float2 {
-                if (v < 0) return make_float2(ax.xh[hb][kHx + v][2 * cq], ax.xh[hb][kHx + v][2 * cq + 1]);
-                const uint32_t u = *reinterpret_cast<const uint32_t *>(xraw + v * (kP * 2) + cq * 4);
-                return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
-            };
-            float2 h0v = raw2(cr0 - 3), h1v = raw2(cr0 - 2), h2v = raw2(cr0 - 1);   // raw rows t-3, t-2, t-1
-            const float2 half2 = make_float2(0.5f, 0.5f);
+        };
+        // delta, running log2-decay and the decay factor tables of chunk cn into
+        // slot cn % 3 (lane l: tokens l and l + 32), then the slot's barrier
+        auto tables = [&](int cn, const __nv_bfloat16 (&draw)[2]) {
+            Tables &tw = ax.tab[cn % 3];
+            const int nvn = (int)min((int64_t)kQ, len - (int64_t)cn * kQ);
+            float d[2], sc[2];
 #pragma unroll
-            for (int i = 0; i < kQ / 8; ++i) {
-                const int r = cr0 + i;
-                const float2 cur = raw2(r);                           // rows >= nv are zeros
-                float2 xc = cur;
-                if (K > 0) {
-                    float2 acc = __ffma2_rn(cw3, cur, cbias);
-                    acc = __ffma2_rn(cw2, h2v, acc);
-                    acc = __ffma2_rn(cw1, h1v, acc);
-                    acc = __ffma2_rn(cw0, h0v, acc);
-                    // silu(v) = h + h tanh(h), h = v / 2
-                    const float2 hv = __fmul2_rn(acc, half2);
-                    xc = __ffma2_rn(hv, make_float2(tanh_approx(hv.x), tanh_approx(hv.y)), hv);
+            for (int h = 0; h < 2; ++h) {
+                const int j = lane + 32 * h;
+                const float u = __bfloat162float(draw[h]) + dtb;
+                d[h] = j < nvn ? (a.softplus ? softplus(u) : u) : 0.f;
+                sc[h] = d[h] * A2;
+            }
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v0 = __shfl_up_sync(0xffffffffu, sc[0], o);
+                const float v1 = __shfl_up_sync(0xffffffffu, sc[1], o);
+                if (lane >= o) { sc[0] += v0; sc[1] += v1; }
+            }
+            const float tot0 = __shfl_sync(0xffffffffu, sc[0], 31);
+            sc[1] += tot0;
+            const float last = __shfl_sync(0xffffffffu, sc[1], 31);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int j = lane + 32 * h;
+                // block boundaries: token 16*(j/16) (start) and 16*(j/16)+15 (end)
+                const float st = __shfl_sync(0xffffffffu, sc[h], lane & ~15);
+                const float en = __shfl_sync(0xffffffffu, sc[h], lane | 15);
+                tw.dlt[j] = d[h];
+                tw.cs2[j] = sc[h];
+                tw.ecs[j] = ex2(sc[h]);
+                tw.wj[j] = ex2(last - sc[h]) * d[h];
+                tw.rf[j] = ex2(sc[h] - st);
+                tw.cf[j] = ex2(en - sc[h]) * d[h];
+            }
+            // block factor (I, J), J < I: exp(cs[16 I] - cs[16 J + 15]) (<= 1); lanes 0-15
+            {
+                const int I = (lane >> 2) & 3, J = lane & 3;
+                const float s0 = __shfl_sync(0xffffffffu, sc[0], (I & 1) * 16);
+                const float s1 = __shfl_sync(0xffffffffu, sc[1], (I & 1) * 16);
+                const float e0 = __shfl_sync(0xffffffffu, sc[0], (J & 1) * 16 + 15);
+                const float e1 = __shfl_sync(0xffffffffu, sc[1], (J & 1) * 16 + 15);
+                const float bv = J < I ? ex2((I < 2 ? s0 : s1) - (J < 2 ? e0 : e1)) : 0.f;
+                if (lane < 16) tw.bf[I][J] = bv;
+            }
+            if (lane == 0) tw.dAc = ex2(last);
+            __syncwarp();
+            if (lead) mb_arrive(&ax.mb[MB_T0 + cn % 3]);
+        };
+        if (n > 0) {
+            if (lead) {
+                load_x(0);
+                if (n > 1) load_x(1);
+                load_bc(0);
+                if (a.z) load_z(0);
+            }
+            for (int cn = 0; cn < 3 && cn < n; ++cn) {
+                __nv_bfloat16 dr[2];
+                load_dt(cn, dr);
+                tables(cn, dr);
+            }
+        }
+        bool ok = true;
+        for (int k = -1; k < n; ++k) {
+            const int c1 = k + 1;
+            __nv_bfloat16 dnext[2];
+            if (k >= 0 && k + 3 < n) load_dt(k + 3, dnext);       // consumed after S(k)
+            if (c1 < n) {
+                // G(c1) = C B^T as soon as B / C have landed (mask(k) has read G(k))
+                ok = wait_mb(ax, MB_BC, c1 & 1, a.err) && ok;
+                tc::fence_after_sync();
+                if (lead && ok) {
+#pragma unroll
+                    for (int kk = 0; kk < kN / 16; ++kk) {
+                        const uint32_t ko = (kk >> 2) * 8192 + (kk & 3) * 32;
+                        tc::mma_bf16(tmem + TM_G, tc::desc_sw128(sbase + OFF_C + ko, 16, 1024),
+                                     tc::desc_sw128(sbase + OFF_B + ko, 16, 1024), ID_G, kk > 0);
+                    }
+                    tc::mma_commit(&ax.mb[MB_G]);
                 }
-                if (r >= nv) xc = make_float2(0.f, 0.f);
-                h0v = h1v; h1v = h2v; h2v = cur;
-                const __nv_bfloat162 b = __floats2bfloat162_rn(xc.x, xc.y);
-                *reinterpret_cast<__nv_bfloat162 *>(smem + OFF_X + tc::off_sw128(r, 2 * cq, 8192)) = b;
+                __syncwarp();
+                // raw x of chunk c1 + 2 once conv(c1) has read its staging buffer
+                ok = wait_mb(ax, MB_CONV, c1 & 1, a.err) && ok;
+                if (lead && ok && c1 + 2 < n) load_x(c1 + 2);
+                __syncwarp();
+            }
+            if (k >= 0) {
+                // z of chunk c1 once the epilogue has read z(k)
+                ok = wait_mb(ax, MB_ZFREE, k & 1, a.err) && ok;
+                if (lead && ok && a.z && c1 < n) load_z(c1);
+                __syncwarp();
+            }
+            // S(k) written (h0 for k = -1): Sc(c1) and Yo(c1)
+            ok = wait_mb(ax, MB_SREADY, c1 & 1, a.err) && ok;
+            tc::fence_after_sync();
+            if (c1 < n) {
+                if (lead && ok) {
+#pragma unroll
+                    for (int kk = 0; kk < kQ / 16; ++kk)
+                        tc::mma_bf16(tmem + TM_SC, tc::desc_sw128(sbase + OFF_B + kk * 2048, 8192, 1024),
+                                     tc::desc_sw128(sbase + OFF_XP + kk * 2048, 8192, 1024), ID_S, kk > 0);
+#pragma unroll
+                    for (int kk = 0; kk < kN / 16; ++kk)
+                        tc::mma_bf16(tmem + TM_YO, tc::desc_sw128(sbase + OFF_C + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                                     tc::desc_sw128(sbase + OFF_S + kk * 2048, 8192, 1024), ID_Y, kk > 0);
+                    tc::mma_commit(&ax.mb[MB_BCFREE]);
+                }
+                __syncwarp();
+            }
+            // the tables of chunk k + 3 into the slot S(k) has finished with
+            if (k >= 0 && k + 3 < n) tables(k + 3, dnext);
+            if (c1 < n) {
+                // Y(c1) = M X once the mask is written
+                ok = wait_mb(ax, MB_MREADY, c1 & 1, a.err) && ok;
+                tc::fence_after_sync();
+                const uint32_t xo = OFF_X + (c1 & 1) * 8192;
+                if (lead && ok) {
+#pragma unroll
+                    for (int kk = 0; kk < kQ / 16; ++kk)
+                        tc::mma_bf16(tmem + TM_Y, tc::desc_sw128(sbase + OFF_M + kk * 32, 16, 1024),
+                                     tc::desc_sw128(sbase + xo + kk * 2048, 8192, 1024), ID_Y, kk > 0);
+                    tc::mma_commit(&ax.mb[MB_MMA]);
+                }
+                __syncwarp();
+                // B / C of chunk c1 + 1 once G, Sc and Yo have read them
+                if (c1 + 1 < n) {
+                    ok = wait_mb(ax, MB_BCFREE, c1 & 1, a.err) && ok;
+                    if (lead && ok) load_bc(c1 + 1);
+                    __syncwarp();
+                }
             }
         }
-        // halo of the next chunk: raw rows nv-3 .. nv-1 (from the old halo when the chunk is shorter)
+        if (lead && aborted(ax)) {
+            // drain: every MMA this thread issued, and the last copies into each buffer
+            tc::mma_commit(&ax.mb[MB_DRAIN]);
+            tc::mbar_wait(&ax.mb[MB_DRAIN], 0, 1u << 22);
+            for (int b = 0; b < 2; ++b)
+                if (last_x[b] >= 0) tc::mbar_wait(&ax.mb[MB_X0 + b], (last_x[b] >> 1) & 1, 1u << 22);
+            if (last_bc >= 0) tc::mbar_wait(&ax.mb[MB_BC], last_bc & 1, 1u << 22);
+            if (last_z >= 0) tc::mbar_wait(&ax.mb[MB_Z], last_z & 1, 1u << 22);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ compute warps
+        const int q4 = warp & 3;          // tensor-memory lane quarter of this warp
+        const int half = warp >> 2;       // which 32 columns of a 64-column accumulator this warp reads
+        const bool zg = a.z != nullptr;
+        __nv_bfloat16 *yg = a.y + row * a.y_bs + start * a.y_ts + hh * kP;
+        const float Dh = a.D ? a.D[hh] : 0.f;
+        const uint32_t t_lane = (uint32_t)(q4 * 32) << 16;
+        bool ok = true;
+
+        // x conv role: channels 2 cq, 2 cq + 1 (one packed pair), tokens cr0 .. cr0+7;
+        // taps right-aligned (cw3 multiplies the current token, cw0 the one 3 back)
+        const int cq = lane, cr0 = warp * (kQ / 8);
+        float2 cw0, cw1, cw2, cw3, cbias;
+        {
+            const int64_t ch = hh * kP + 2 * cq;
+            auto tap = [&](int j) {
+                const int k = K - 4 + j;
+                return (K > 0 && k >= 0) ? make_float2(a.conv_w[ch * K + k], a.conv_w[(ch + 1) * K + k]) : make_float2(0.f, 0.f);
+            };
+            cw0 = tap(0); cw1 = tap(1); cw2 = tap(2); cw3 = tap(3);
+            cbias = a.conv_b ? make_float2(a.conv_b[ch], a.conv_b[ch + 1]) : make_float2(0.f, 0.f);
+        }
+        // swizzled byte offset of (row cr0 + i, channel 2 cq) in an X tile:
+        // row block = warp, row in block = i, 16-byte chunk (cq / 4) ^ i
+        const uint32_t obase = (uint32_t)warp * 1024u + (uint32_t)(cq & 3) * 4u;
+
+        // carried state: thread owns S[n][32*half .. 32*half+31] for n = 32*q4 + lane (fp32 pairs)
+        const int sn = q4 * 32 + lane;
+        float2 S[16];
+        {
+            const float *h0p = a.h0 ? a.h0 + ((int64_t)s * H + hh) * kP * kN : nullptr;
+#pragma unroll
+            for (int p = 0; p < 16; ++p)
+                S[p] = h0p ? make_float2(h0p[(int64_t)(half * 32 + 2 * p) * kN + sn], h0p[(int64_t)(half * 32 + 2 * p + 1) * kN + sn])
+                           : make_float2(0.f, 0.f);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                st16(smem + OFF_S + tc::off_sw128(sn, half * 32 + q * 8, 8192), tc::pack_bf16x8(reinterpret_cast<const float *>(&S[q * 4])));
+        }
+        // conv halo of chunk 0 (the last K-1 raw inputs before the sequence)
         if (tid < kP) {
             const int p = tid;
 #pragma unroll
             for (int j = 0; j < kHx; ++j) {
-                const int v = nv - kHx + j;
-                ax.xh[hb ^ 1][j][p] = v >= 0 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-                                                   xraw + v * (kP * 2) + p * 2))
-                                             : ax.xh[hb][kHx + v][p];
+                const int q = j - (kHx - (K - 1));          // index into the carried conv state
+                float v = 0.f;
+                if (K > 1 && q >= 0 && a.conv_state_in)
+                    v = __bfloat162float(a.conv_state_in[((int64_t)s * a.cdim + hh * kP + p) * (K - 1) + q]);
+                ax.xh[0][j][p] = v;
             }
         }
-        // B / C visible to every thread (the rescale reads them); X visible to the tensor core
-        if (!zfill && !tc::mbar_wait(&ax.mbar[3], c & 1)) { fail_bar = 3; fail_par = c & 1; ok = false; }
-        tc::fence_proxy_async();
-        {
-            const bool got = tc::mbar_wait(&ax.mbar[0], c & 1);
-            if (!got) { fail_bar = 0; fail_par = c & 1; }
-            ok = __syncthreads_and(ok && got);
-        }
-        if (!ok) break;
-        tc::fence_after_sync();
 
-        // ---- (3) mask G -> M (over the staged raw rows, already consumed); rescale C -> C', B -> B'
-        // Each warp reads its 16 accumulator rows (tokens i0 = 16 q4 + lane / 4 and
-        // i1 = i0 + 8) for its 32 columns, spread over all 32 threads.
-        const Tables &tb = ax.tab[c & 1];
+        // accumulator fragment of this thread (16-lane TMEM loads of an M = 64
+        // accumulator): rows i0 = 16 q4 + lane / 4 and i1 = i0 + 8, columns
+        // jc + 8 k and jc + 8 k + 1 for k = 0..3
         const int i0 = q4 * 16 + (lane >> 2), i1 = i0 + 8;
-        const int jc = half * 32 + 2 * (lane & 3);                   // first column of pair k: jc + 8 k
-        {
-            uint32_t gr[16];
-            tc::tmem_ld16x256b_x4(tmem + t_lane + half * 32, gr);
-            const int I = q4;
-            const float ci0 = tb.cs2[i0], ci1 = tb.cs2[i1];
-            const float rf0 = tb.rf[i0], rf1 = tb.rf[i1];
-            tc::tmem_wait_ld();
-            // M[i, j] = G[i, j] exp(cs_i - cs_j) delta_j for j <= i, plus D on the diagonal
-            // (the skip term D x rides along in M X).  Below the diagonal 16x16 block the
-            // exponential factors as row x block x column terms, each <= 1.
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int J = half * 2 + (k >> 1);                    // 16-column block (warp-uniform)
-                const int j = jc + 8 * k;
-                float m00 = 0.f, m01 = 0.f, m10 = 0.f, m11 = 0.f;     // (i0, j), (i0, j+1), (i1, j), (i1, j+1)
-                const float g00 = __uint_as_float(gr[4 * k]), g01 = __uint_as_float(gr[4 * k + 1]);
-                const float g10 = __uint_as_float(gr[4 * k + 2]), g11 = __uint_as_float(gr[4 * k + 3]);
-                if (J < I) {
-                    const float bfac = tb.bf[I][J];
-                    const float c0 = tb.cf[j] * bfac, c1 = tb.cf[j + 1] * bfac;
-                    m00 = g00 * rf0 * c0; m01 = g01 * rf0 * c1;
-                    m10 = g10 * rf1 * c0; m11 = g11 * rf1 * c1;
-                } else if (J == I) {
-                    const float cj0 = tb.cs2[j], cj1 = tb.cs2[j + 1];
-                    const float d0 = tb.dlt[j], d1 = tb.dlt[j + 1];
-                    m00 = j <= i0 ? g00 * ex2(ci0 - cj0) * d0 : 0.f;
-                    m01 = j + 1 <= i0 ? g01 * ex2(ci0 - cj1) * d1 : 0.f;
-                    m10 = j <= i1 ? g10 * ex2(ci1 - cj0) * d0 : 0.f;
-                    m11 = j + 1 <= i1 ? g11 * ex2(ci1 - cj1) * d1 : 0.f;
-                    if (j == i0) m00 += Dh;
-                    if (j + 1 == i0) m01 += Dh;
-                    if (j == i1) m10 += Dh;
-                    if (j + 1 == i1) m11 += Dh;
+        const int jc = half * 32 + 2 * (lane & 3);
+        // swizzled byte offset of (i0, jc + 8 k) in a 64 x 64 bf16 tile is
+        // frag_off + (((4 half + k) ^ (lane / 4)) << 4); row i1 is 1024 bytes further
+        const uint32_t frag_off = (uint32_t)q4 * 2048u + (uint32_t)(lane >> 2) * 128u + (uint32_t)(lane & 3) * 4u;
+
+        for (int k = -1; k < n; ++k) {
+            const int c1 = k + 1;
+            // the y staging of chunk k - 1 sat in the X buffer conv(c1) writes now
+            if (tid == 0) tc::bulk_wait_read();
+            bar_compute();
+
+            // ---- conv(c1): raw x rows -> X and X' (bf16, swizzled), halo of chunk c1 + 1
+            if (c1 < n) {
+                ok = wait_mb(ax, MB_T0 + c1 % 3, (c1 / 3) & 1, a.err) && ok;
+                ok = wait_mb(ax, MB_X0 + (c1 & 1), (c1 >> 1) & 1, a.err) && ok;
+                if (c1 > 0) ok = wait_mb(ax, MB_BCFREE, (c1 - 1) & 1, a.err) && ok;   // Sc(c1-1) has read X'
+                const int nv = (int)min((int64_t)kQ, len - (int64_t)c1 * kQ);
+                const int hb = c1 & 1;
+                const Tables &tb = ax.tab[c1 % 3];
+                const unsigned char *xraw = smem + OFF_XR + hb * 8192;
+                unsigned char *xo = smem + OFF_X + hb * 8192;
+                unsigned char *xpo = smem + OFF_XP;
+                auto rawrow = [&](int v) -> float2 {
+                    const uint32_t u = *reinterpret_cast<const uint32_t *>(xraw + v * (kP * 2) + cq * 4);
+                    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+                };
+                float2 h0v, h1v, h2v;                                   // raw rows t-3, t-2, t-1
+                if (warp == 0) {
+                    h0v = *reinterpret_cast<const float2 *>(&ax.xh[hb][0][2 * cq]);
+                    h1v = *reinterpret_cast<const float2 *>(&ax.xh[hb][1][2 * cq]);
+                    h2v = *reinterpret_cast<const float2 *>(&ax.xh[hb][2][2 * cq]);
+                } else {
+                    h0v = rawrow(cr0 - 3); h1v = rawrow(cr0 - 2); h2v = rawrow(cr0 - 1);
                 }
-                *reinterpret_cast<__nv_bfloat162 *>(smem + OFF_M + tc::off_sw128(i0, j, 8192)) = __floats2bfloat162_rn(m00, m01);
-                *reinterpret_cast<__nv_bfloat162 *>(smem + OFF_M + tc::off_sw128(i1, j, 8192)) = __floats2bfloat162_rn(m10, m11);
-            }
-        }
-        // C'[i] = exp(cs_i) C[i], B'[j] = exp(cs_Q - cs_j) delta_j B[j]: packed bf16 products
-        for (int i = tid; i < kQ * (kN / 8); i += kThreads) {
-            const int r = i / (kN / 8), q = i % (kN / 8);
-            const uint32_t off = tc::off_sw128(r, q * 8, 8192);
-            const __nv_bfloat162 fc = __float2bfloat162_rn(tb.ecs[r]), fb = __float2bfloat162_rn(tb.wj[r]);
-            uint4 vc = ld16(smem + OFF_C + off), vb = ld16(smem + OFF_B + off);
-            __nv_bfloat162 *pc = reinterpret_cast<__nv_bfloat162 *>(&vc), *pb = reinterpret_cast<__nv_bfloat162 *>(&vb);
+                const float2 half2 = make_float2(0.5f, 0.5f);
+                float wv[8];                                            // X' weights of the 8 tokens
+                {
+                    const float4 w0 = *reinterpret_cast<const float4 *>(&tb.wj[cr0]);
+                    const float4 w1 = *reinterpret_cast<const float4 *>(&tb.wj[cr0 + 4]);
+                    wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
+                    wv[4] = w1.x; wv[5] = w1.y; wv[6] = w1.z; wv[7] = w1.w;
+                }
+                const bool full = nv == kQ;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                pc[e] = __hmul2(pc[e], fc);
-                pb[e] = __hmul2(pb[e], fb);
-            }
-            st16(smem + OFF_C + off, vc);
-            st16(smem + OFF_B + off, vb);
-        }
-        // z of this thread's accumulator positions, in flight while the tensor cores run
-        uint32_t zr[8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int p = jc + 8 * k;
-            zr[2 * k] = (zg && i0 < nv) ? *reinterpret_cast<const uint32_t *>(zg + (t0 + i0) * a.z_ts + p) : 0u;
-            zr[2 * k + 1] = (zg && i1 < nv) ? *reinterpret_cast<const uint32_t *>(zg + (t0 + i1) * a.z_ts + p) : 0u;
-        }
-        tc::fence_before_sync();
-        tc::fence_proxy_async();
-        __syncthreads();
-
-        // ---- (4) MMA2 + MMA3 into Y (columns 64..127), MMA4 into Sc (columns 0..63)
-        if (tid == 0) {
-            tc::fence_after_sync();
-#pragma unroll
-            for (int k = 0; k < kQ / 16; ++k)
-                tc::mma_bf16(tmem + 64, tc::desc_sw128(sbase + OFF_M + k * 32, 16, 1024),
-                             tc::desc_sw128(sbase + OFF_X + k * 2048, 8192, 1024), ID_Y, k > 0);
-#pragma unroll
-            for (int k = 0; k < kN / 16; ++k)
-                tc::mma_bf16(tmem + 64, tc::desc_sw128(sbase + OFF_C + (k >> 2) * 8192 + (k & 3) * 32, 16, 1024),
-                             tc::desc_sw128(sbase + OFF_S + k * 2048, 8192, 1024), ID_Y, 1);
-#pragma unroll
-            for (int k = 0; k < kQ / 16; ++k)
-                tc::mma_bf16(tmem, tc::desc_sw128(sbase + OFF_B + k * 2048, 8192, 1024),
-                             tc::desc_sw128(sbase + OFF_X + k * 2048, 8192, 1024), ID_S, k > 0);
-            tc::mma_commit(&ax.mbar[1]);
-        }
-        // warp 0: the next chunk's decay tables while the tensor cores run
-        if (warp < 2 && c + 1 < nchunks) dt_tables(c + 1);
-        ok = __syncthreads_and(tc::mbar_wait(&ax.mbar[1], c & 1));
-        if (!ok) { fail_bar = 1; fail_par = c & 1; break; }
-        tc::fence_after_sync();
-        // B, C and the M tile are free again: stage the next chunk behind the epilogue
-        if (tid == 0 && c + 1 < nchunks) prefetch(c + 1);
-        if (warp < 2 && c + 2 < nchunks) load_dt(c + 2);
-
-        // ---- (5) y = Y * silu(z) for this thread's 16 positions (D x is already in Y); S = exp(cs_Q) S + Sc
-        // Whole chunks (and the tensor's last, clipped chunk) leave through a TMA
-        // store of the staging tile in the X tile's space, free once MMA2 / MMA4
-        // completed; the partial last chunk of a packed sequence is stored directly.
-        const bool y_tma = nv == kQ || !a.sv.cu;
-        {
-            uint32_t yr[16];
-            tc::tmem_ld16x256b_x4(tmem + t_lane + 64 + half * 32, yr);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int p = jc + 8 * k;
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    const int i = rr ? i1 : i0;
-                    float o0 = __uint_as_float(yr[4 * k + 2 * rr]), o1 = __uint_as_float(yr[4 * k + 2 * rr + 1]);
-                    if (zg) {
-                        const uint32_t zw = zr[2 * k + rr];
-                        o0 *= silu_fast<__nv_bfloat16>(__uint_as_float(zw << 16));
-                        o1 *= silu_fast<__nv_bfloat16>(__uint_as_float(zw & 0xffff0000u));
+                for (int i = 0; i < kQ / 8; ++i) {
+                    const float2 cur = rawrow(cr0 + i);                 // rows >= nv are zeroed below
+                    float2 xc = cur;
+                    if (K > 0) {
+                        float2 acc = __ffma2_rn(cw3, cur, cbias);
+                        acc = __ffma2_rn(cw2, h2v, acc);
+                        acc = __ffma2_rn(cw1, h1v, acc);
+                        acc = __ffma2_rn(cw0, h0v, acc);
+                        // silu(v) = h + h tanh(h), h = v / 2
+                        const float2 hv = __fmul2_rn(acc, half2);
+                        xc = __ffma2_rn(hv, make_float2(tanh_approx(hv.x), tanh_approx(hv.y)), hv);
                     }
-                    const __nv_bfloat162 ob = __floats2bfloat162_rn(o0, o1);
-                    if (y_tma) *reinterpret_cast<__nv_bfloat162 *>(smem + OFF_X + tc::off_sw128(i, p, 8192)) = ob;
-                    else if (i < nv) *reinterpret_cast<__nv_bfloat162 *>(yg + (t0 + i) * a.y_ts + p) = ob;
+                    if (!full && cr0 + i >= nv) xc = make_float2(0.f, 0.f);
+                    h0v = h1v; h1v = h2v; h2v = cur;
+                    const float2 xw = __fmul2_rn(xc, make_float2(wv[i], wv[i]));
+                    const uint32_t off = obase + (uint32_t)i * 128u + ((uint32_t)((cq >> 2) ^ i) << 4);
+                    *reinterpret_cast<__nv_bfloat162 *>(xo + off) = __floats2bfloat162_rn(xc.x, xc.y);
+                    *reinterpret_cast<__nv_bfloat162 *>(xpo + off) = __floats2bfloat162_rn(xw.x, xw.y);
                 }
+                // halo of the next chunk: raw rows nv-3 .. nv-1 (from the old halo when the chunk is shorter)
+                if (tid < kP) {
+                    const int p = tid;
+#pragma unroll
+                    for (int j = 0; j < kHx; ++j) {
+                        const int v = nv - kHx + j;
+                        ax.xh[hb ^ 1][j][p] = v >= 0 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                                                           xraw + v * (kP * 2) + p * 2))
+                                                     : ax.xh[hb][kHx + v][p];
+                    }
+                }
+                tc::fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mb_arrive(&ax.mb[MB_CONV]);
             }
-        }
-        if (y_tma) {
-            tc::fence_proxy_async();
-            __syncthreads();
-            if (tid == 0) tc::tma_store_3d(&tm_y, (int)(hh * kP), (int)(start + t0), crow, smem + OFF_X);
-        }
-        {
-            const float dAc = tb.dAc;
-            float Sc[32];
-            tc::tmem_ld32(tmem + t_lane + half * 32, Sc);
+
+            // ---- epilogue(k): y = (Y + exp(cs_i) Yo) * silu(z); S(k) = exp(cs_Q) S + Sc
+            if (k >= 0) {
+                const int64_t t0 = (int64_t)k * kQ;
+                const int nv = (int)min((int64_t)kQ, len - t0);
+                const Tables &tb = ax.tab[k % 3];
+                unsigned char *stg = smem + OFF_X + (k & 1) * 8192;
+                // Whole chunks (and the tensor's last, clipped chunk) leave through a TMA
+                // store of the staging tile; the partial last chunk of a packed sequence
+                // is stored directly.
+                const bool y_tma = nv == kQ || !a.sv.cu;
+                ok = wait_mb(ax, MB_MMA, k & 1, a.err) && ok;
+                if (zg) ok = wait_mb(ax, MB_Z, k & 1, a.err) && ok;
+                tc::fence_after_sync();
+                {
+                    const float e0 = tb.ecs[i0], e1 = tb.ecs[i1];
+                    const bool st_ok = !aborted(ax);
+                    const float2 half2 = make_float2(0.5f, 0.5f);
+                    // two passes of 16 columns keep the accumulator fragments at 16 registers
 #pragma unroll
-            for (int p = 0; p < 32; ++p) S[p] = fmaf(dAc, S[p], Sc[p]);
+                    for (int hp = 0; hp < 2; ++hp) {
+                        uint32_t yr[8], yo[8];
+                        tc::tmem_ld16x256b_x2(tmem + t_lane + TM_Y + half * 32 + hp * 16, yr);
+                        tc::tmem_ld16x256b_x2(tmem + t_lane + TM_YO + half * 32 + hp * 16, yo);
+                        tc::tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                st16(smem + OFF_S + tc::off_sw128(sn, half * 32 + q * 8, 8192), tc::pack_bf16x8(&S[q * 8]));
-        }
-        // intermediate state after this chunk when it closes a state interval
-        if (a.iv.interval > 0 && nv == kQ) {
-            const int64_t slot = a.iv.slot_after(s, t0 + kQ);
-            if (slot >= 0) {
-                if (a.iv.states) {
-                    float *dst = a.iv.states + (slot * H + hh) * kP * kN;
+                        for (int kq = 0; kq < 2; ++kq) {
+                            const int kk = hp * 2 + kq;
+                            const int p = jc + 8 * kk;
+                            const uint32_t off0 = frag_off + ((uint32_t)((half * 4 + kk) ^ (lane >> 2)) << 4);
 #pragma unroll
-                    for (int p = 0; p < 32; ++p) dst[(int64_t)(half * 32 + p) * kN + sn] = S[p];
-                }
-                if (a.iv.conv && K > 1) {
-                    // x channels of this head: the halo of the next chunk; B / C of the
-                    // group (written by its first head): the raw inputs before the boundary
-                    __nv_bfloat16 *cdst = static_cast<__nv_bfloat16 *>(a.iv.conv) + slot * a.cdim * (K - 1);
-                    if (tid < kP)
-                        for (int j = 0; j < K - 1; ++j)
-                            cdst[(hh * kP + tid) * (K - 1) + j] = __float2bfloat16_rn(ax.xh[hb ^ 1][kHx - (K - 1) + j][tid]);
-                    if (hh % (H / a.G) == 0) {
-                        const int64_t GN = a.G * kN;
-                        for (int i = tid; i < 2 * kN * (K - 1); i += kThreads) {
-                            const int which = i / (kN * (K - 1)), n = (i / (K - 1)) % kN, j = i % (K - 1);
-                            const int64_t tok = start + t0 + kQ - (K - 1) + j;
-                            const __nv_bfloat16 v = which ? a.Craw[row * a.craw_bs + tok * a.craw_ts + g * kN + n]
-                                                          : a.Braw[row * a.braw_bs + tok * a.braw_ts + g * kN + n];
-                            cdst[(a.H * kP + which * GN + g * kN + n) * (K - 1) + j] = v;
+                            for (int rr = 0; rr < 2; ++rr) {
+                                const int i = rr ? i1 : i0;
+                                const uint32_t off = off0 + rr * 1024u;
+                                const float e = rr ? e1 : e0;
+                                float2 o = __ffma2_rn(make_float2(e, e),
+                                                      make_float2(__uint_as_float(yo[4 * kq + 2 * rr]), __uint_as_float(yo[4 * kq + 2 * rr + 1])),
+                                                      make_float2(__uint_as_float(yr[4 * kq + 2 * rr]), __uint_as_float(yr[4 * kq + 2 * rr + 1])));
+                                if (zg) {
+                                    // silu(z) = h + h tanh(h), h = z / 2
+                                    const uint32_t zw = *reinterpret_cast<const uint32_t *>(smem + OFF_Z + off);
+                                    const float2 hz = __fmul2_rn(make_float2(__uint_as_float(zw << 16), __uint_as_float(zw & 0xffff0000u)), half2);
+                                    o = __fmul2_rn(o, __ffma2_rn(hz, make_float2(tanh_approx(hz.x), tanh_approx(hz.y)), hz));
+                                }
+                                const __nv_bfloat162 ob = __floats2bfloat162_rn(o.x, o.y);
+                                if (y_tma) *reinterpret_cast<__nv_bfloat162 *>(stg + off) = ob;
+                                else if (i < nv && st_ok) *reinterpret_cast<__nv_bfloat162 *>(yg + (t0 + i) * a.y_ts + p) = ob;
+                            }
                         }
                     }
                 }
+                // z(k) has been read: the control warp may load z(k + 1)
+                __syncwarp();
+                if (lane == 0) mb_arrive(&ax.mb[MB_ZFREE]);
+                if (y_tma) {
+                    tc::fence_proxy_async();
+                    bar_compute();
+                    if (tid == 0 && !aborted(ax)) tc::tma_store_3d(&tm_y, (int)(hh * kP), (int)(start + t0), crow, stg);
+                }
+                {
+                    const float2 dA2 = make_float2(tb.dAc, tb.dAc);
+                    float Sc[32];
+                    tc::tmem_ld32(tmem + t_lane + TM_SC + half * 32, Sc);
+#pragma unroll
+                    for (int p = 0; p < 16; ++p) S[p] = __ffma2_rn(dA2, S[p], make_float2(Sc[2 * p], Sc[2 * p + 1]));
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        st16(smem + OFF_S + tc::off_sw128(sn, half * 32 + q * 8, 8192),
+                             tc::pack_bf16x8(reinterpret_cast<const float *>(&S[q * 4])));
+                }
+                tc::fence_proxy_async();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mb_arrive(&ax.mb[MB_SREADY]);
+                // intermediate state after this chunk when it closes a state interval
+                if (a.iv.interval > 0 && nv == kQ && !aborted(ax)) {
+                    const int64_t slot = a.iv.slot_after(s, t0 + kQ);
+                    if (slot >= 0) {
+                        if (a.iv.states) {
+                            float *dst = a.iv.states + (slot * H + hh) * kP * kN;
+#pragma unroll
+                            for (int p = 0; p < 16; ++p) {
+                                dst[(int64_t)(half * 32 + 2 * p) * kN + sn] = S[p].x;
+                                dst[(int64_t)(half * 32 + 2 * p + 1) * kN + sn] = S[p].y;
+                            }
+                        }
+                        if (a.iv.conv && K > 1) {
+                            // x channels of this head: the halo conv(k) left for chunk k + 1;
+                            // B / C of the group (written by its first head): the raw inputs
+                            // before the boundary
+                            __nv_bfloat16 *cdst = static_cast<__nv_bfloat16 *>(a.iv.conv) + slot * a.cdim * (K - 1);
+                            if (tid < kP)
+                                for (int j = 0; j < K - 1; ++j)
+                                    cdst[(hh * kP + tid) * (K - 1) + j] =
+                                        __float2bfloat16_rn(ax.xh[(k + 1) & 1][kHx - (K - 1) + j][tid]);
+                            if (hh % (H / a.G) == 0) {
+                                const int64_t GN = a.G * kN;
+                                for (int i = tid; i < 2 * kN * (K - 1); i += kComputeThreads) {
+                                    const int which = i / (kN * (K - 1)), nn = (i / (K - 1)) % kN, j = i % (K - 1);
+                                    const int64_t tok = start + t0 + kQ - (K - 1) + j;
+                                    const __nv_bfloat16 v = which ? a.Craw[row * a.craw_bs + tok * a.craw_ts + g * kN + nn]
+                                                                  : a.Braw[row * a.braw_bs + tok * a.braw_ts + g * kN + nn];
+                                    cdst[(a.H * kP + which * GN + g * kN + nn) * (K - 1) + j] = v;
+                                }
+                            }
+                        }
+                    }
+                }
+            } else {
+                // S(-1) = h0: its bf16 copy was written before the loop
+                tc::fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mb_arrive(&ax.mb[MB_SREADY]);
+            }
+
+            // ---- mask(c1): G -> M (blocks on or below the diagonal)
+            // Each warp reads its 16 accumulator rows (tokens i0, i1) for its 32 columns.
+            // M[i, j] = G[i, j] exp(cs_i - cs_j) delta_j for j <= i, plus D on the diagonal
+            // (the skip term D x rides along in M X).  Below the diagonal 16x16 block the
+            // exponential factors as row x block x column terms, each <= 1.
+            if (c1 < n) {
+                ok = wait_mb(ax, MB_G, c1 & 1, a.err) && ok;
+                tc::fence_after_sync();
+                const Tables &tb = ax.tab[c1 % 3];
+                const int I = q4;
+                if (half * 2 <= I) {                                   // some block of this warp is on or below the diagonal
+                    uint32_t gr[16];
+                    tc::tmem_ld16x256b_x4(tmem + t_lane + TM_G + half * 32, gr);
+                    const float ci0 = tb.cs2[i0], ci1 = tb.cs2[i1];
+                    const float rf0 = tb.rf[i0], rf1 = tb.rf[i1];
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const int J = half * 2 + (kk >> 1);                    // 16-column block (warp-uniform)
+                        if (J > I) continue;
+                        const int j = jc + 8 * kk;
+                        float m00, m01, m10, m11;                              // (i0, j), (i0, j+1), (i1, j), (i1, j+1)
+                        const float g00 = __uint_as_float(gr[4 * kk]), g01 = __uint_as_float(gr[4 * kk + 1]);
+                        const float g10 = __uint_as_float(gr[4 * kk + 2]), g11 = __uint_as_float(gr[4 * kk + 3]);
+                        const float2 cf = *reinterpret_cast<const float2 *>(&tb.cf[j]);
+                        if (J < I) {
+                            const float bfac = tb.bf[I][J];
+                            const float r0 = rf0 * bfac, r1 = rf1 * bfac;
+                            m00 = g00 * (r0 * cf.x); m01 = g01 * (r0 * cf.y);
+                            m10 = g10 * (r1 * cf.x); m11 = g11 * (r1 * cf.y);
+                        } else {
+                            // diagonal block: direct exponentials, selected (not branched) below the diagonal
+                            const float2 cj = *reinterpret_cast<const float2 *>(&tb.cs2[j]);
+                            const float2 dj = *reinterpret_cast<const float2 *>(&tb.dlt[j]);
+                            const float v00 = g00 * ex2(ci0 - cj.x) * dj.x, v01 = g01 * ex2(ci0 - cj.y) * dj.y;
+                            const float v10 = g10 * ex2(ci1 - cj.x) * dj.x, v11 = g11 * ex2(ci1 - cj.y) * dj.y;
+                            m00 = j < i0 ? v00 : (j == i0 ? v00 + Dh : 0.f);
+                            m01 = j + 1 < i0 ? v01 : (j + 1 == i0 ? v01 + Dh : 0.f);
+                            m10 = j < i1 ? v10 : (j == i1 ? v10 + Dh : 0.f);
+                            m11 = j + 1 < i1 ? v11 : (j + 1 == i1 ? v11 + Dh : 0.f);
+                        }
+                        const uint32_t off = frag_off + ((uint32_t)((half * 4 + kk) ^ (lane >> 2)) << 4);
+                        *reinterpret_cast<__nv_bfloat162 *>(smem + OFF_M + off) = __floats2bfloat162_rn(m00, m01);
+                        *reinterpret_cast<__nv_bfloat162 *>(smem + OFF_M + off + 1024) = __floats2bfloat162_rn(m10, m11);
+                    }
+                }
+                tc::fence_proxy_async();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mb_arrive(&ax.mb[MB_MREADY]);
             }
         }
-        if (tid == 0) tc::bulk_wait_read();                           // the X tile is written again by the next conv
-        tc::fence_before_sync();
-        tc::fence_proxy_async();
-        __syncthreads();
-    }
-    if (tid == 0) tc::bulk_wait_all();
-
-    if (!ok) {
-        // a tensor-core completion never arrived: record it, give the MMAs a
-        // bounded grace period, release tensor memory and leave
-        if (tid == 0 && a.err) atomicExch(a.err, SSM_DEVERR_TIMEOUT);
-        tc::mbar_wait(&ax.mbar[fail_bar], fail_par, 1u << 20);
-    } else {
-        if (a.h_final) {
-            float *hf = a.h_final + ((int64_t)s * H + hh) * kP * kN;
+        if (tid == 0) tc::bulk_wait_all();
+        if (!aborted(ax)) {
+            if (a.h_final) {
+                float *hf = a.h_final + ((int64_t)s * H + hh) * kP * kN;
 #pragma unroll
-            for (int p = 0; p < 32; ++p) hf[(int64_t)(half * 32 + p) * kN + sn] = S[p];
+                for (int p = 0; p < 16; ++p) {
+                    hf[(int64_t)(half * 32 + 2 * p) * kN + sn] = S[p].x;
+                    hf[(int64_t)(half * 32 + 2 * p + 1) * kN + sn] = S[p].y;
+                }
+            }
+            if (K > 1 && a.conv_state_out && tid < kP) {
+                const int p = tid, hbf = n & 1;
+                for (int j = 0; j < K - 1; ++j)
+                    a.conv_state_out[((int64_t)s * a.cdim + hh * kP + p) * (K - 1) + j] =
+                        __float2bfloat16_rn(ax.xh[hbf][kHx - (K - 1) + j][p]);
+            }
+            if (K > 1 && a.conv_state_out && hh % (H / a.G) == 0) {
+                // the group's B / C channels (first head of the group): the last K-1 raw
+                // inputs of the sequence, from the carried state when it is shorter.  One
+                // thread per channel reads all K-1 values before it writes, so the state
+                // may be updated in place.
+                const int which = tid / kN, nn = tid % kN;            // 256 threads: B then C
+                const int64_t ch = a.H * kP + which * a.G * kN + g * kN + nn;
+                const __nv_bfloat16 *raw = which ? a.Craw + row * a.craw_bs + g * kN + nn
+                                                 : a.Braw + row * a.braw_bs + g * kN + nn;
+                const int64_t rts = which ? a.craw_ts : a.braw_ts;
+                __nv_bfloat16 v[kHx];
+#pragma unroll
+                for (int j = 0; j < kHx; ++j) {
+                    const int64_t tau = len - (K - 1) + j;           // within the sequence
+                    v[j] = __float2bfloat16_rn(0.f);
+                    if (j < K - 1) {
+                        if (tau >= 0) v[j] = raw[(start + tau) * rts];
+                        else if (a.conv_state_in) v[j] = a.conv_state_in[((int64_t)s * a.cdim + ch) * (K - 1) + tau + (K - 1)];
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < kHx; ++j)
+                    if (j < K - 1) a.conv_state_out[((int64_t)s * a.cdim + ch) * (K - 1) + j] = v[j];
+            }
         }
-        if (K > 1 && a.conv_state_out && tid < kP) {
-            const int p = tid, hbf = nchunks & 1;
-            for (int j = 0; j < K - 1; ++j)
-                a.conv_state_out[((int64_t)s * a.cdim + hh * kP + p) * (K - 1) + j] =
-                    __float2bfloat16_rn(ax.xh[hbf][kHx - (K - 1) + j][p]);
-        }
+        (void)ok;
     }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if (warp == 0) tc::tmem_dealloc(tmem, kTmemCols);
+    if (warp == kComputeWarps) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ B / C pre-pass
+// Causal conv + SiLU of the B and C channels of x|B|C, once per group (every
+// head of the group reads the result), into bf16 [tokens][G*N] workspace
+// tiles.  One thread per (8 channels of B or C, 8 consecutive tokens): the
+// K-1 rows before the run are loaded first (from the sequence's carried conv
+// state before its first token), every row is one 16-byte load, and a warp
+// covers 32 consecutive channel vectors of one token row.  Packed sequences
+// restart the history at every sequence start.
+struct BcArgs {
+    const __nv_bfloat16 *B, *C;
+    int64_t b_bs, b_ts, c_bs, c_ts;
+    const float *w, *bias;            // full conv weight [conv_dim][K] and bias (or null)
+    const __nv_bfloat16 *state_in;    // [nseq][conv_dim][K-1] or null
+    __nv_bfloat16 *oB, *oC;           // [rows * seqlen][GN]
+    const int32_t *cu;
+    int nseqs;
+    int64_t seqlen, GN, HP, cdim;
+};
+
+template <int K>
+__global__ void __launch_bounds__(128, 3) bc_conv_kernel(const BcArgs a) {
+    const int64_t nvec = a.GN / 4;                        // B and C vectors of one token row
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t vec = idx % nvec, run = idx / nvec;
+    const int64_t t0 = run * 8;
+    if (t0 >= a.seqlen) return;
+    const int64_t row = blockIdx.y;
+    const int which = vec >= nvec / 2;                    // 0: B, 1: C
+    const int64_t c0 = (vec - which * (nvec / 2)) * 8;    // channel within B (or C)
+    const __nv_bfloat16 *src = which ? a.C + row * a.c_bs : a.B + row * a.b_bs;
+    const int64_t ts = which ? a.c_ts : a.b_ts;
+    __nv_bfloat16 *dst = (which ? a.oC : a.oB) + row * a.seqlen * a.GN + c0;
+    const int64_t cch = a.HP + which * a.GN + c0;         // conv channel of the first of the 8
+    float wk[K][8], bb[8];
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+#pragma unroll
+        for (int k = 0; k < K; ++k) wk[k][v] = a.w[(cch + v) * K + k];
+        bb[v] = a.bias ? a.bias[cch + v] : 0.f;
+    }
+    // sequence of the run's first token and its bounds (clamped: a malformed
+    // cu_seqlens gives wrong values but no out-of-bounds access)
+    int s = a.cu ? seq_of_token(a.cu, a.nseqs, t0) : (int)row;
+    int64_t start = a.cu ? min(max((int64_t)a.cu[s], (int64_t)0), a.seqlen) : 0;
+    int64_t end = a.cu ? min(max((int64_t)a.cu[s + 1], start), a.seqlen) : a.seqlen;
+    float hist[K > 1 ? K - 1 : 1][8];
+    auto load_hist = [&](int64_t t) {
+#pragma unroll
+        for (int j = 0; j < K - 1; ++j) {                 // hist[j] holds token t-(K-1)+j
+            const int64_t tau = t - (K - 1) + j;
+            if (tau >= start) {
+                Vec8<__nv_bfloat16>::ld(src + tau * ts + c0, hist[j]);
+            } else {
+                const int64_t q = tau - start + (K - 1);
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                    hist[j][v] = (a.state_in && q >= 0)
+                                     ? __bfloat162float(a.state_in[((int64_t)s * a.cdim + cch + v) * (K - 1) + q])
+                                     : 0.f;
+            }
+        }
+    };
+    load_hist(t0);
+    const int64_t t1 = min(t0 + 8, a.seqlen);
+    // every row's load is issued before any math
+    uint4 rows[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        if (t0 + i < t1) rows[i] = *reinterpret_cast<const uint4 *>(src + (t0 + i) * ts + c0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int64_t t = t0 + i;
+        if (t >= t1) break;
+        if (a.cu && t >= end) {                           // the next non-empty sequence starts here
+            while (s + 1 < a.nseqs && a.cu[s + 1] <= t) ++s;
+            start = min(max((int64_t)a.cu[s], (int64_t)0), a.seqlen);
+            end = min(max((int64_t)a.cu[s + 1], start), a.seqlen);
+            if (t < start || t >= end) return;
+            load_hist(t);
+        }
+        float cur[8], o[8];
+        tc::unpack_bf16x8(rows[i], cur);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            float acc = bb[v];
+#pragma unroll
+            for (int k = 0; k < K - 1; ++k) acc = fmaf(wk[k][v], hist[k][v], acc);
+            acc = fmaf(wk[K - 1][v], cur[v], acc);
+            o[v] = silu_fast<__nv_bfloat16>(acc);
+        }
+        *reinterpret_cast<uint4 *>(dst + t * a.GN) = tc::pack_bf16x8(o);
+#pragma unroll
+        for (int k = 0; k + 1 < K - 1; ++k)
+#pragma unroll
+            for (int v = 0; v < 8; ++v) hist[k][v] = hist[k + 1][v];
+        if (K > 1)
+#pragma unroll
+            for (int v = 0; v < 8; ++v) hist[K > 1 ? K - 2 : 0][v] = cur[v];
+    }
 }
 
 }  // namespace
@@ -629,7 +924,10 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     // the kernel attribute), so nothing on the host separates the pre-pass
     // launches from the scan launch.
     const int64_t rows = s.cu_seqlens ? 1 : s.batch;
-    CUtensorMap tm_x, tm_b, tm_c, tm_y;
+    CUtensorMap tm_x, tm_b, tm_c, tm_z, tm_y;
+    memset(&tm_z, 0, sizeof(tm_z));
+    if (s.z && !make_map(&tm_z, s.z, s.d_inner, s.seqlen, rows, s.z_token_stride, s.z_batch_stride, true))
+        return cudaErrorInvalidValue;
     if (!make_map(&tm_x, s.x, s.d_inner, s.seqlen, rows, s.x_token_stride, s.x_batch_stride, false) ||
         !make_map(&tm_b, Bc, GN, s.seqlen, rows, b_ts, b_bs, true) ||
         !make_map(&tm_c, Cc, GN, s.seqlen, rows, c_ts, c_bs, true) ||
@@ -639,23 +937,24 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     if (e != cudaSuccess) return e;
     if (s.d_conv > 0) {
         // pre-pass: conv + SiLU of the B and C channels, once per group, into the workspace
-        for (int which = 0; which < 2; ++which) {
-            ConvJob j;
-            j.x = which == 0 ? s.B : s.C;
-            j.x_bs = which == 0 ? s.B_batch_stride : s.C_batch_stride;
-            j.x_ts = which == 0 ? s.B_token_stride : s.C_token_stride;
-            const int64_t ch0 = s.d_inner + which * GN;
-            j.w = s.conv_w + ch0 * s.d_conv;
-            j.b = s.conv_b ? s.conv_b + ch0 : nullptr;
-            const size_t es = 2;
-            j.state_in = s.conv_state_in ? static_cast<const char *>(s.conv_state_in) + ch0 * (s.d_conv - 1) * es : nullptr;
-            j.state_out = s.conv_state_out ? static_cast<char *>(s.conv_state_out) + ch0 * (s.d_conv - 1) * es : nullptr;
-            j.state_stride = cdim * (s.d_conv - 1);
-            j.cu = s.cu_seqlens; j.nseqs = s.nseqs; j.batch = s.batch; j.seqlen = s.seqlen;
-            j.channels = GN; j.width = s.d_conv; j.act = 1; j.dtype = SSM_BF16;
-            j.out = which == 0 ? (void *)wB : (void *)wC;
-            j.o_bs = s.seqlen * GN; j.o_ts = GN;
-            e = launch_conv_job(j, st);
+        BcArgs b;
+        b.B = static_cast<const __nv_bfloat16 *>(s.B); b.C = static_cast<const __nv_bfloat16 *>(s.C);
+        b.b_bs = s.B_batch_stride; b.b_ts = s.B_token_stride; b.c_bs = s.C_batch_stride; b.c_ts = s.C_token_stride;
+        b.w = s.conv_w; b.bias = s.conv_b;
+        b.state_in = static_cast<const __nv_bfloat16 *>(s.conv_state_in);
+        b.oB = wB; b.oC = wC;
+        b.cu = s.cu_seqlens; b.nseqs = s.nseqs;
+        b.seqlen = s.seqlen; b.GN = GN; b.HP = s.d_inner; b.cdim = cdim;
+        const int64_t threads = (s.seqlen + 7) / 8 * (GN / 4);
+        const dim3 bgrid((unsigned)((threads + 127) / 128), (unsigned)rows);
+        if (threads > 0) {
+            switch (s.d_conv) {
+                case 1: bc_conv_kernel<1><<<bgrid, 128, 0, st>>>(b); break;
+                case 2: bc_conv_kernel<2><<<bgrid, 128, 0, st>>>(b); break;
+                case 3: bc_conv_kernel<3><<<bgrid, 128, 0, st>>>(b); break;
+                default: bc_conv_kernel<4><<<bgrid, 128, 0, st>>>(b); break;
+            }
+            e = cudaGetLastError();
             if (e != cudaSuccess) return e;
         }
     }
@@ -681,7 +980,7 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     a.craw_bs = s.C_batch_stride; a.craw_ts = s.C_token_stride;
     dim3 grid((unsigned)s.nheads, (unsigned)nseqs);
     timing_begin(st);
-    ssd_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, tm_x, tm_b, tm_c, tm_y);
+    ssd_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, tm_x, tm_b, tm_c, tm_z, tm_y);
     timing_end(st);
     return cudaGetLastError();
 }

@@ -121,6 +121,25 @@ SSM_DEVINL bool mbar_try_wait(uint64_t *mbar, uint32_t parity) {
     return ok != 0;
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete yet
+// sleeps until it completes or about `hint_ns` nanoseconds pass, instead of
+// spinning on the barrier (spinning threads take issue slots from the warps
+// that do the work).
+SSM_DEVINL bool mbar_try_wait_sleep(uint64_t *mbar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\nselp.b32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(mbar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+SSM_DEVINL uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
 // Bounded wait for the phase with `parity` to complete.  Returns false when
 // the limit runs out (the caller records an error and leaves cleanly).
 SSM_DEVINL bool mbar_wait(uint64_t *mbar, uint32_t parity, uint32_t limit = (1u << 24)) {
@@ -184,6 +203,12 @@ SSM_DEVINL void tmem_ld16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
+}
+// Same for 16 columns (column groups k = 0, 1 of the layout above).
+SSM_DEVINL void tmem_ld16x256b_x2(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
 }
 SSM_DEVINL void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 
