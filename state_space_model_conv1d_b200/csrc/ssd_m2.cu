@@ -53,6 +53,8 @@
 #include <stddef.h>
 #include <string.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "launch.h"
 #include "tc05.cuh"
@@ -218,6 +220,15 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
     if (warp == kComputeWarps) {
         // ------------------------------------------------------------ control warp
         const bool lead = lane == 0;
+        // shared-memory descriptors of the operand tiles; a K step adds its byte
+        // offset / 16 to the start-address field (addresses stay below 256 KB)
+        const uint64_t dCk = tc::desc_sw128(sbase + OFF_C, 16, 1024);     // K-major C (G, Yo)
+        const uint64_t dBk = tc::desc_sw128(sbase + OFF_B, 16, 1024);     // K-major B (G)
+        const uint64_t dBm = tc::desc_sw128(sbase + OFF_B, 8192, 1024);   // MN-major B^T (Sc)
+        const uint64_t dXPm = tc::desc_sw128(sbase + OFF_XP, 8192, 1024); // MN-major X' (Sc)
+        const uint64_t dSm = tc::desc_sw128(sbase + OFF_S, 8192, 1024);   // MN-major S^T (Yo)
+        const uint64_t dMk = tc::desc_sw128(sbase + OFF_M, 16, 1024);     // K-major M (Y)
+        const uint64_t dX0m = tc::desc_sw128(sbase + OFF_X, 8192, 1024);  // MN-major X, buffer 0 (Y)
         const float dtb = a.dt_bias ? a.dt_bias[hh] : 0.f;
         const __nv_bfloat16 *dtg = a.dt + row * a.dt_bs + start * a.dt_ts + hh;
         int last_x[2] = {-1, -1};
@@ -327,9 +338,8 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                 if (lead && ok) {
 #pragma unroll
                     for (int kk = 0; kk < kN / 16; ++kk) {
-                        const uint32_t ko = (kk >> 2) * 8192 + (kk & 3) * 32;
-                        tc::mma_bf16(tmem + TM_G, tc::desc_sw128(sbase + OFF_C + ko, 16, 1024),
-                                     tc::desc_sw128(sbase + OFF_B + ko, 16, 1024), ID_G, kk > 0);
+                        const uint32_t ko = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+                        tc::mma_bf16(tmem + TM_G, dCk + ko, dBk + ko, ID_G, kk > 0);
                     }
                     tc::mma_commit(&ax.mb[MB_G]);
                 }
@@ -352,12 +362,11 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                 if (lead && ok) {
 #pragma unroll
                     for (int kk = 0; kk < kQ / 16; ++kk)
-                        tc::mma_bf16(tmem + TM_SC, tc::desc_sw128(sbase + OFF_B + kk * 2048, 8192, 1024),
-                                     tc::desc_sw128(sbase + OFF_XP + kk * 2048, 8192, 1024), ID_S, kk > 0);
+                        tc::mma_bf16(tmem + TM_SC, dBm + kk * 128, dXPm + kk * 128, ID_S, kk > 0);
 #pragma unroll
                     for (int kk = 0; kk < kN / 16; ++kk)
-                        tc::mma_bf16(tmem + TM_YO, tc::desc_sw128(sbase + OFF_C + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                                     tc::desc_sw128(sbase + OFF_S + kk * 2048, 8192, 1024), ID_Y, kk > 0);
+                        tc::mma_bf16(tmem + TM_YO, dCk + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), dSm + kk * 128, ID_Y,
+                                     kk > 0);
                     tc::mma_commit(&ax.mb[MB_BCFREE]);
                 }
                 __syncwarp();
@@ -368,12 +377,11 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                 // Y(c1) = M X once the mask is written
                 ok = wait_mb(ax, MB_MREADY, c1 & 1, a.err) && ok;
                 tc::fence_after_sync();
-                const uint32_t xo = OFF_X + (c1 & 1) * 8192;
+                const uint64_t dXm = dX0m + (uint64_t)((c1 & 1) * (8192 >> 4));
                 if (lead && ok) {
 #pragma unroll
                     for (int kk = 0; kk < kQ / 16; ++kk)
-                        tc::mma_bf16(tmem + TM_Y, tc::desc_sw128(sbase + OFF_M + kk * 32, 16, 1024),
-                                     tc::desc_sw128(sbase + xo + kk * 2048, 8192, 1024), ID_Y, kk > 0);
+                        tc::mma_bf16(tmem + TM_Y, dMk + kk * 2, dXm + kk * 128, ID_Y, kk > 0);
                     tc::mma_commit(&ax.mb[MB_MMA]);
                 }
                 __syncwarp();
@@ -494,27 +502,32 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                     wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
                     wv[4] = w1.x; wv[5] = w1.y; wv[6] = w1.z; wv[7] = w1.w;
                 }
-                const bool full = nv == kQ;
+                // full chunks take a copy of the loop without the end-of-sequence test
+                auto conv_rows = [&](auto full_tag) {
+                    constexpr bool kFull = decltype(full_tag)::value;
 #pragma unroll
-                for (int i = 0; i < kQ / 8; ++i) {
-                    const float2 cur = rawrow(cr0 + i);                 // rows >= nv are zeroed below
-                    float2 xc = cur;
-                    if (K > 0) {
-                        float2 acc = __ffma2_rn(cw3, cur, cbias);
-                        acc = __ffma2_rn(cw2, h2v, acc);
-                        acc = __ffma2_rn(cw1, h1v, acc);
-                        acc = __ffma2_rn(cw0, h0v, acc);
-                        // silu(v) = h + h tanh(h), h = v / 2
-                        const float2 hv = __fmul2_rn(acc, half2);
-                        xc = __ffma2_rn(hv, make_float2(tanh_approx(hv.x), tanh_approx(hv.y)), hv);
+                    for (int i = 0; i < kQ / 8; ++i) {
+                        const float2 cur = rawrow(cr0 + i);             // rows >= nv are zeroed below
+                        float2 xc = cur;
+                        if (K > 0) {
+                            float2 acc = __ffma2_rn(cw3, cur, cbias);
+                            acc = __ffma2_rn(cw2, h2v, acc);
+                            acc = __ffma2_rn(cw1, h1v, acc);
+                            acc = __ffma2_rn(cw0, h0v, acc);
+                            // silu(v) = h + h tanh(h), h = v / 2
+                            const float2 hv = __fmul2_rn(acc, half2);
+                            xc = __ffma2_rn(hv, make_float2(tanh_approx(hv.x), tanh_approx(hv.y)), hv);
+                        }
+                        if (!kFull && cr0 + i >= nv) xc = make_float2(0.f, 0.f);
+                        h0v = h1v; h1v = h2v; h2v = cur;
+                        const float2 xw = __fmul2_rn(xc, make_float2(wv[i], wv[i]));
+                        const uint32_t off = obase + (uint32_t)i * 128u + ((uint32_t)((cq >> 2) ^ i) << 4);
+                        *reinterpret_cast<__nv_bfloat162 *>(xo + off) = __floats2bfloat162_rn(xc.x, xc.y);
+                        *reinterpret_cast<__nv_bfloat162 *>(xpo + off) = __floats2bfloat162_rn(xw.x, xw.y);
                     }
-                    if (!full && cr0 + i >= nv) xc = make_float2(0.f, 0.f);
-                    h0v = h1v; h1v = h2v; h2v = cur;
-                    const float2 xw = __fmul2_rn(xc, make_float2(wv[i], wv[i]));
-                    const uint32_t off = obase + (uint32_t)i * 128u + ((uint32_t)((cq >> 2) ^ i) << 4);
-                    *reinterpret_cast<__nv_bfloat162 *>(xo + off) = __floats2bfloat162_rn(xc.x, xc.y);
-                    *reinterpret_cast<__nv_bfloat162 *>(xpo + off) = __floats2bfloat162_rn(xw.x, xw.y);
-                }
+                };
+                if (nv == kQ) conv_rows(std::true_type{});
+                else conv_rows(std::false_type{});
                 // halo of the next chunk: raw rows nv-3 .. nv-1 (from the old halo when the chunk is shorter)
                 if (tid < kP) {
                     const int p = tid;
@@ -546,40 +559,48 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                 tc::fence_after_sync();
                 {
                     const float e0 = tb.ecs[i0], e1 = tb.ecs[i1];
-                    const bool st_ok = !aborted(ax);
+                    const float2 e02 = make_float2(e0, e0), e12 = make_float2(e1, e1);
                     const float2 half2 = make_float2(0.5f, 0.5f);
-                    // two passes of 16 columns keep the accumulator fragments at 16 registers
+                    // two passes of 16 columns keep the accumulator fragments at 16 registers;
+                    // the staged (TMA) and the direct-store forms are separate copies
+                    auto epi = [&](auto tma_tag) {
+                        constexpr bool kTma = decltype(tma_tag)::value;
+                        const bool st_ok = kTma || !aborted(ax);
 #pragma unroll
-                    for (int hp = 0; hp < 2; ++hp) {
-                        uint32_t yr[8], yo[8];
-                        tc::tmem_ld16x256b_x2(tmem + t_lane + TM_Y + half * 32 + hp * 16, yr);
-                        tc::tmem_ld16x256b_x2(tmem + t_lane + TM_YO + half * 32 + hp * 16, yo);
-                        tc::tmem_wait_ld();
+                        for (int hp = 0; hp < 2; ++hp) {
+                            uint32_t yr[8], yo[8];
+                            tc::tmem_ld16x256b_x2(tmem + t_lane + TM_Y + half * 32 + hp * 16, yr);
+                            tc::tmem_ld16x256b_x2(tmem + t_lane + TM_YO + half * 32 + hp * 16, yo);
+                            tc::tmem_wait_ld();
 #pragma unroll
-                        for (int kq = 0; kq < 2; ++kq) {
-                            const int kk = hp * 2 + kq;
-                            const int p = jc + 8 * kk;
-                            const uint32_t off0 = frag_off + ((uint32_t)((half * 4 + kk) ^ (lane >> 2)) << 4);
+                            for (int kq = 0; kq < 2; ++kq) {
+                                const int kk = hp * 2 + kq;
+                                const uint32_t off0 = frag_off + ((uint32_t)((half * 4 + kk) ^ (lane >> 2)) << 4);
 #pragma unroll
-                            for (int rr = 0; rr < 2; ++rr) {
-                                const int i = rr ? i1 : i0;
-                                const uint32_t off = off0 + rr * 1024u;
-                                const float e = rr ? e1 : e0;
-                                float2 o = __ffma2_rn(make_float2(e, e),
-                                                      make_float2(__uint_as_float(yo[4 * kq + 2 * rr]), __uint_as_float(yo[4 * kq + 2 * rr + 1])),
-                                                      make_float2(__uint_as_float(yr[4 * kq + 2 * rr]), __uint_as_float(yr[4 * kq + 2 * rr + 1])));
-                                if (zg) {
-                                    // silu(z) = h + h tanh(h), h = z / 2
-                                    const uint32_t zw = *reinterpret_cast<const uint32_t *>(smem + OFF_Z + off);
-                                    const float2 hz = __fmul2_rn(make_float2(__uint_as_float(zw << 16), __uint_as_float(zw & 0xffff0000u)), half2);
-                                    o = __fmul2_rn(o, __ffma2_rn(hz, make_float2(tanh_approx(hz.x), tanh_approx(hz.y)), hz));
+                                for (int rr = 0; rr < 2; ++rr) {
+                                    const uint32_t off = off0 + rr * 1024u;
+                                    float2 o = __ffma2_rn(rr ? e12 : e02,
+                                                          make_float2(__uint_as_float(yo[4 * kq + 2 * rr]), __uint_as_float(yo[4 * kq + 2 * rr + 1])),
+                                                          make_float2(__uint_as_float(yr[4 * kq + 2 * rr]), __uint_as_float(yr[4 * kq + 2 * rr + 1])));
+                                    if (zg) {
+                                        // silu(z) = h + h tanh(h), h = z / 2
+                                        const uint32_t zw = *reinterpret_cast<const uint32_t *>(smem + OFF_Z + off);
+                                        const float2 hz = __fmul2_rn(make_float2(__uint_as_float(zw << 16), __uint_as_float(zw & 0xffff0000u)), half2);
+                                        o = __fmul2_rn(o, __ffma2_rn(hz, make_float2(tanh_approx(hz.x), tanh_approx(hz.y)), hz));
+                                    }
+                                    const __nv_bfloat162 ob = __floats2bfloat162_rn(o.x, o.y);
+                                    if (kTma) {
+                                        *reinterpret_cast<__nv_bfloat162 *>(stg + off) = ob;
+                                    } else {
+                                        const int i = rr ? i1 : i0;
+                                        if (i < nv && st_ok) *reinterpret_cast<__nv_bfloat162 *>(yg + (t0 + i) * a.y_ts + jc + 8 * kk) = ob;
+                                    }
                                 }
-                                const __nv_bfloat162 ob = __floats2bfloat162_rn(o.x, o.y);
-                                if (y_tma) *reinterpret_cast<__nv_bfloat162 *>(stg + off) = ob;
-                                else if (i < nv && st_ok) *reinterpret_cast<__nv_bfloat162 *>(yg + (t0 + i) * a.y_ts + p) = ob;
                             }
                         }
-                    }
+                    };
+                    if (y_tma) epi(std::true_type{});
+                    else epi(std::false_type{});
                 }
                 // z(k) has been read: the control warp may load z(k + 1)
                 __syncwarp();
@@ -655,40 +676,49 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                 tc::fence_after_sync();
                 const Tables &tb = ax.tab[c1 % 3];
                 const int I = q4;
-                if (half * 2 <= I) {                                   // some block of this warp is on or below the diagonal
+                // The warp's two 16-column blocks J0 = 2 half (column groups k = 0, 1)
+                // and J1 = 2 half + 1 (k = 2, 3) against its row block I = q4: J0 on the
+                // diagonal and J1 above (I = 2 half), J0 below and J1 on the diagonal
+                // (I = 2 half + 1), both below (I > 2 half + 1), or both above.
+                if (I >= 2 * half) {
                     uint32_t gr[16];
                     tc::tmem_ld16x256b_x4(tmem + t_lane + TM_G + half * 32, gr);
                     const float ci0 = tb.cs2[i0], ci1 = tb.cs2[i1];
                     const float rf0 = tb.rf[i0], rf1 = tb.rf[i1];
                     tc::tmem_wait_ld();
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const int J = half * 2 + (kk >> 1);                    // 16-column block (warp-uniform)
-                        if (J > I) continue;
-                        const int j = jc + 8 * kk;
-                        float m00, m01, m10, m11;                              // (i0, j), (i0, j+1), (i1, j), (i1, j+1)
-                        const float g00 = __uint_as_float(gr[4 * kk]), g01 = __uint_as_float(gr[4 * kk + 1]);
-                        const float g10 = __uint_as_float(gr[4 * kk + 2]), g11 = __uint_as_float(gr[4 * kk + 3]);
-                        const float2 cf = *reinterpret_cast<const float2 *>(&tb.cf[j]);
-                        if (J < I) {
-                            const float bfac = tb.bf[I][J];
-                            const float r0 = rf0 * bfac, r1 = rf1 * bfac;
-                            m00 = g00 * (r0 * cf.x); m01 = g01 * (r0 * cf.y);
-                            m10 = g10 * (r1 * cf.x); m11 = g11 * (r1 * cf.y);
-                        } else {
-                            // diagonal block: direct exponentials, selected (not branched) below the diagonal
-                            const float2 cj = *reinterpret_cast<const float2 *>(&tb.cs2[j]);
-                            const float2 dj = *reinterpret_cast<const float2 *>(&tb.dlt[j]);
-                            const float v00 = g00 * ex2(ci0 - cj.x) * dj.x, v01 = g01 * ex2(ci0 - cj.y) * dj.y;
-                            const float v10 = g10 * ex2(ci1 - cj.x) * dj.x, v11 = g11 * ex2(ci1 - cj.y) * dj.y;
-                            m00 = j < i0 ? v00 : (j == i0 ? v00 + Dh : 0.f);
-                            m01 = j + 1 < i0 ? v01 : (j + 1 == i0 ? v01 + Dh : 0.f);
-                            m10 = j < i1 ? v10 : (j == i1 ? v10 + Dh : 0.f);
-                            m11 = j + 1 < i1 ? v11 : (j + 1 == i1 ? v11 + Dh : 0.f);
-                        }
+                    auto put = [&](int kk, float m00, float m01, float m10, float m11) {
                         const uint32_t off = frag_off + ((uint32_t)((half * 4 + kk) ^ (lane >> 2)) << 4);
                         *reinterpret_cast<__nv_bfloat162 *>(smem + OFF_M + off) = __floats2bfloat162_rn(m00, m01);
                         *reinterpret_cast<__nv_bfloat162 *>(smem + OFF_M + off + 1024) = __floats2bfloat162_rn(m10, m11);
+                    };
+                    // below the diagonal: G exp(cs_i - cs_j) delta_j = G * row * block * column factors
+                    auto below = [&](int kk) {
+                        const int j = jc + 8 * kk;
+                        const float bfac = tb.bf[I][half * 2 + (kk >> 1)];
+                        const float2 cf = *reinterpret_cast<const float2 *>(&tb.cf[j]);
+                        const float r0 = rf0 * bfac, r1 = rf1 * bfac;
+                        put(kk, __uint_as_float(gr[4 * kk]) * (r0 * cf.x), __uint_as_float(gr[4 * kk + 1]) * (r0 * cf.y),
+                            __uint_as_float(gr[4 * kk + 2]) * (r1 * cf.x), __uint_as_float(gr[4 * kk + 3]) * (r1 * cf.y));
+                    };
+                    // on the diagonal: direct exponentials, selected (not branched) at and below
+                    // the diagonal, plus D on it (the skip term D x rides along in M X)
+                    auto diag = [&](int kk) {
+                        const int j = jc + 8 * kk;
+                        const float2 cj = *reinterpret_cast<const float2 *>(&tb.cs2[j]);
+                        const float2 dj = *reinterpret_cast<const float2 *>(&tb.dlt[j]);
+                        const float v00 = __uint_as_float(gr[4 * kk]) * ex2(ci0 - cj.x) * dj.x;
+                        const float v01 = __uint_as_float(gr[4 * kk + 1]) * ex2(ci0 - cj.y) * dj.y;
+                        const float v10 = __uint_as_float(gr[4 * kk + 2]) * ex2(ci1 - cj.x) * dj.x;
+                        const float v11 = __uint_as_float(gr[4 * kk + 3]) * ex2(ci1 - cj.y) * dj.y;
+                        put(kk, j < i0 ? v00 : (j == i0 ? v00 + Dh : 0.f), j + 1 < i0 ? v01 : (j + 1 == i0 ? v01 + Dh : 0.f),
+                            j < i1 ? v10 : (j == i1 ? v10 + Dh : 0.f), j + 1 < i1 ? v11 : (j + 1 == i1 ? v11 + Dh : 0.f));
+                    };
+                    if (I == 2 * half) {
+                        diag(0); diag(1);
+                    } else if (I == 2 * half + 1) {
+                        below(0); below(1); diag(2); diag(3);
+                    } else {
+                        below(0); below(1); below(2); below(3);
                     }
                 }
                 tc::fence_proxy_async();
