@@ -562,10 +562,22 @@ int oracle_state_update(const oracle_update_args *a) {
             if (K > 0) {
                 double *cs = a->conv_state + (r * cdim + c) * Ls;
                 /* window = last K-1 stored inputs + the new input */
+#if SSM_ORACLE_MUTANT == 16
+                /* mutant: with a width-K state the window is read one position too old */
+                double pre = o_conv_tap(a->conv_w + c * K, a->conv_b ? a->conv_b[c] : 0.0,
+                                        cs + (Ls >= K ? Ls - K : Ls - (K - 1)), raw, K);
+#else
                 double pre = o_conv_tap(a->conv_w + c * K, a->conv_b ? a->conv_b[c] : 0.0,
                                         cs + (Ls - (K - 1)), raw, K);
+#endif
+#if SSM_ORACLE_MUTANT == 15
+                /* mutant: the state rolled the wrong way (new input stored at the oldest end) */
+                for (int64_t k = Ls - 1; k > 0; --k) cs[k] = cs[k - 1];
+                if (Ls > 0) cs[0] = raw;
+#else
                 for (int64_t k = 0; k + 1 < Ls; ++k) cs[k] = cs[k + 1];
                 if (Ls > 0) cs[Ls - 1] = raw;
+#endif
                 u[c] = o_silu(pre);
             } else {
                 u[c] = raw;

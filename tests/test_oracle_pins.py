@@ -63,6 +63,8 @@ MUTANTS = {
     12: "skip term on the pre-conv x",
     13: "intermediate state recorded one token early",
     14: "backward: dh not carried back through exp(delta A)",
+    15: "decode: conv state rolled the wrong way",
+    16: "decode: conv window read one position too old (width-K state)",
 }
 
 
