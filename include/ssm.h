@@ -277,13 +277,17 @@ SSM_API ssm_status ssm_kernel_time_ms(float *total_ms, int32_t *launches);
  * Nothing here allocates or frees memory.  The first call on a device looks
  * up the array's device address (cudaGetSymbolAddress, with that device
  * current) and caches it: make that first call before any stream capture.
- * Every call shares the one array and the scan initialises what it reads
- * (the error word, the varlen schedule) on each call; calls that may
- * overlap on the GPU (different streams, or different host threads on one
- * device) race on it, so serialise them.  The error word can be read back
- * with ssm_workspace_error() only by code that knows the array's address,
- * so this entry point reports device-side errors by leaving its outputs
- * unwritten, as ssm_scan_fwd does. */
+ * The cached address belongs to the device's primary context: it does not
+ * survive cudaDeviceReset() (the module may come back at another address),
+ * so a process that resets a device must not call this entry point on that
+ * device again.  Every call shares the one array and the scan initialises
+ * what it reads (the error word, the varlen schedule) on each call; calls
+ * that may overlap on the GPU (different streams, or different host threads
+ * on one device) race on it, so serialise them.  The error word can be read
+ * back with ssm_workspace_error() only by code that knows the array's
+ * address.  A malformed cu_seqlens leaves every output (y, h_final,
+ * conv_state_out) unwritten, as in ssm_scan_fwd; a bounded wait that runs
+ * out (SSM_DEVERR_TIMEOUT) can leave them partly written. */
 #define SSM_NOALLOC_SCRATCH_BYTES (4u << 20)
 SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *args, void *stream);
 
@@ -335,7 +339,11 @@ typedef struct ssm_split_args {
 
 /* Step 1.  `tail` is [batch][conv_dim][K-1] in the activation dtype, oldest
  * first, in the layout of conv_state_out; positions before the segment's
- * first token come from conv_state_in (zeros when NULL).  Needs d_conv > 1. */
+ * first token come from conv_state_in (zeros when NULL).  Needs d_conv > 1.
+ * On ranks r > 0 the tail is built before the previous rank's tail arrives,
+ * so it is only right when the segment holds at least K-1 tokens: a caller
+ * must not split a sequence into shorter segments (this call cannot see the
+ * rank and does not check it). */
 SSM_API ssm_status ssm_split_conv_tail(const ssm_scan_args *args, void *tail, void *stream);
 /* Step 3.  cum_delta [batch][seqlen][U] fp32 (may be NULL), sum_delta
  * [batch][U] fp32.  delta as in ssm_scan_fwd (dt + dt_bias, then softplus

@@ -42,7 +42,8 @@ def _m2_head_problem(d, h, H, P, G, N):
     rows = np.concatenate([xch, bch, cch])
     sub = dict(x=d["x"][:, :, h:h + 1], z=d["z"][:, :, h:h + 1], dt=d["dt"][:, :, h:h + 1],
                B=d["B"][:, :, g:g + 1], C=d["C"][:, :, g:g + 1], A=d["A"][h:h + 1], D=d["D"][h:h + 1],
-               dt_bias=d["dt_bias"][h:h + 1], h0=d["h0"][:, h:h + 1], conv_w=d["conv_w"][rows])
+               dt_bias=d["dt_bias"][h:h + 1], h0=d["h0"][:, h:h + 1], conv_w=d["conv_w"][rows],
+               conv_state_in=None if d.get("conv_state_in") is None else d["conv_state_in"][:, rows], rows=rows)
     return sub
 
 
@@ -54,11 +55,13 @@ def test_mamba2_fullsize_sampled_heads(name):
     H, P, G, N = w.nheads, w.headdim, w.ngroups, w.dstate
     for h in (0, H // 2 - 1, H // 2, H - 1):
         sub = _m2_head_problem(d, h, H, P, G, N)
-        ry, rh, _ = oracle.scan_fwd(M2, sub["x"], sub["dt"], sub["A"], sub["B"], sub["C"], D=sub["D"], z=sub["z"],
-                                    dt_bias=sub["dt_bias"], h0=sub["h0"], conv_w=sub["conv_w"],
-                                    cu_seqlens=d.get("cu_seqlens"), nthreads=8)
+        ry, rh, rc = oracle.scan_fwd(M2, sub["x"], sub["dt"], sub["A"], sub["B"], sub["C"], D=sub["D"], z=sub["z"],
+                                     dt_bias=sub["dt_bias"], h0=sub["h0"], conv_w=sub["conv_w"],
+                                     conv_state_in=sub["conv_state_in"], cu_seqlens=d.get("cu_seqlens"), nthreads=8)
         assert_close(y[:, :, h:h + 1], ry, "bf16", f"{name} head {h} y")
         assert_close(hf[:, h:h + 1], rh, "bf16", f"{name} head {h} h_final")
+        # the head's x channels and its group's B / C channels of the carried conv state
+        assert_close(cs[:, sub["rows"]], rc, "bf16", f"{name} head {h} conv_state_out")
 
 
 def test_decode_fullsize_sampled_rows():

@@ -73,6 +73,7 @@ M1_CASES = [
     (1, 150, 32, 64, 2, "f32"),       # the widest dstate of the path
     (2, 70, 24, 13, 4, "f32"),        # dstate not a multiple of 4
     (2, 65, 64, 16, 0, "bf16"),       # no conv in front
+    (1, 2113, 48, 16, 4, "f32"),      # fp32 over many chunks (66 of 32 tokens) and a ragged tail
 ]
 
 
@@ -106,6 +107,7 @@ M2_CASES = [
     (2, 65, 4, 32, 1, 16, 3, "f32"),
     (1, 40, 2, 64, 2, 200, 4, "bf16"),    # dstate beyond 128, not a power of two
     (2, 33, 4, 64, 4, 64, 0, "bf16"),     # no conv
+    (1, 2081, 2, 64, 1, 128, 4, "f32"),   # fp32 over many chunks and a ragged tail
 ]
 
 
