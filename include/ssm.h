@@ -99,6 +99,7 @@ typedef enum { SSM_MAMBA1 = 1, SSM_MAMBA2 = 2 } ssm_mode;
 #define SSM_DEVERR_NONE 0
 #define SSM_DEVERR_CU_SEQLENS 1   /* cu_seqlens not 0-based, decreasing, or not ending at seqlen */
 #define SSM_DEVERR_TIMEOUT 2      /* a bounded wait for tensor-core completion ran out; outputs incomplete */
+#define SSM_DEVERR_BOUNDS 3       /* bounds-checked build only: an index fell outside its tensor (see ssm_bounds_record) */
 
 /* ------------------------------------------------------------------ conv */
 typedef struct ssm_conv_args {
@@ -290,6 +291,23 @@ SSM_API ssm_status ssm_kernel_time_ms(float *total_ms, int32_t *launches);
  * out (SSM_DEVERR_TIMEOUT) can leave them partly written. */
 #define SSM_NOALLOC_SCRATCH_BYTES (4u << 20)
 SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *args, void *stream);
+
+/* Bounds-checked build (libssm_checked.so, compiled with SSM_CHECK_BOUNDS).
+ * The paper has no counterpart: this is a debugging aid of the library.  In
+ * that build every kernel tests the element indices it derives (sequence
+ * ranges from cu_seqlens, head / channel / group ranges, state and conv-state
+ * rows, pool slots, store positions) against the extent the call's shapes
+ * give the tensor.  A failing test does not trap: it records the first
+ * failure of the process on that device (code SSM_DEVERR_BOUNDS, the check
+ * site, the index and the extent) and the access is skipped (a CTA whose
+ * ranges fail returns before touching memory), so the context stays usable.
+ *
+ * ssm_check_bounds_enabled: 1 in the checked build, 0 in libssm.so.
+ * ssm_bounds_record: waits for the device, then reads the record into the
+ * non-NULL pointers (code 0 when no check failed) and clears it when `clear`
+ * is nonzero.  Returns SSM_ERR_UNSUPPORTED in the normal build. */
+SSM_API int32_t ssm_check_bounds_enabled(void);
+SSM_API ssm_status ssm_bounds_record(int32_t *code, int32_t *site, int64_t *index, int64_t *extent, int32_t clear);
 
 /* Waits for `stream`, then reads the device error word of a workspace last
  * used by ssm_scan_fwd: SSM_OK, or SSM_ERR_DEVICE with *code set to an

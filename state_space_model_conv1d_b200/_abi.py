@@ -16,7 +16,7 @@ SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_ALIGNMENT = 0, -1, -2,
 SSM_ERR_WORKSPACE, SSM_ERR_CUDA, SSM_ERR_DEVICE = -4, -5, -6
 SSM_F32, SSM_BF16 = 0, 1
 SSM_MAMBA1, SSM_MAMBA2 = 1, 2
-SSM_DEVERR_NONE, SSM_DEVERR_CU_SEQLENS = 0, 1
+SSM_DEVERR_NONE, SSM_DEVERR_CU_SEQLENS, SSM_DEVERR_TIMEOUT, SSM_DEVERR_BOUNDS = 0, 1, 2, 3
 
 _vp = C.c_void_p
 _i64 = C.c_int64
@@ -112,6 +112,8 @@ SIGNATURES = {
     "ssm_split_cum_delta": ([C.POINTER(ScanArgs), _vp, _vp, _vp], _i32),
     "ssm_split_combine": ([C.POINTER(SplitArgs), _vp], _i32),
     "ssm_split_fixup": ([C.POINTER(ScanArgs), _vp, _vp, _vp], _i32),
+    "ssm_check_bounds_enabled": ([], _i32),
+    "ssm_bounds_record": ([C.POINTER(_i32), C.POINTER(_i32), C.POINTER(_i64), C.POINTER(_i64), _i32], _i32),
 }
 
 _lock = threading.Lock()
@@ -136,6 +138,29 @@ def lib() -> C.CDLL:
                     raise RuntimeError("libssm.so ABI version mismatch")
                 _lib = handle
     return _lib
+
+
+_checked = None
+
+
+def checked_lib() -> C.CDLL:
+    """The bounds-checked build ``libssm_checked.so`` (same symbols and
+    signatures); raises if it has not been built (``build --check-bounds``)."""
+    global _checked
+    if _checked is None:
+        with _lock:
+            if _checked is None:
+                path = os.path.join(_HERE, "libssm_checked.so")
+                if not os.path.exists(path):
+                    raise RuntimeError(f"libssm_checked.so not found at {path}: build it with "
+                                       "`python -m state_space_model_conv1d_b200.build --check-bounds`")
+                handle = C.CDLL(path)
+                for name, (argtypes, restype) in SIGNATURES.items():
+                    fn = getattr(handle, name)
+                    fn.argtypes = argtypes
+                    fn.restype = restype
+                _checked = handle
+    return _checked
 
 
 class SSMError(RuntimeError):

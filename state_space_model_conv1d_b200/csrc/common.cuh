@@ -69,6 +69,42 @@ SSM_DEVINL float silu_fast(float v) {
     }
 }
 
+// ----------------------------------------------------------- bounds checks
+// In the bounds-checked build (SSM_CHECK_BOUNDS) SSM_BOUNDS(index, extent,
+// site) tests 0 <= index < extent; a failing test records the first failure
+// (SSM_DEVERR_BOUNDS, the site, the index, the extent) in one device-wide
+// record and yields false, so the caller skips the access.  Nothing traps.
+// In the normal build it is the constant true and costs nothing.
+enum BoundsSite {
+    BS_SSD_SEQ = 1, BS_SSD_HEAD, BS_SSD_GROUP, BS_SSD_STATE, BS_SSD_CONV_STATE, BS_SSD_Y, BS_SSD_POOL, BS_SSD_RAW_BC,
+    BS_BC_ROW, BS_BC_CHANNEL, BS_BC_STATE,
+    BS_M1_SEQ, BS_M1_CHANNEL, BS_M1_STATE, BS_M1_CONV_STATE, BS_M1_Y, BS_M1_POOL,
+    BS_M2S_SEQ, BS_M2S_HEAD, BS_M2S_STATE,
+    BS_DEC_ROW, BS_DEC_SLOT, BS_DEC_CHANNEL,
+    BS_CONV_TOKEN, BS_CONV_CHANNEL, BS_CONV_STATE,
+    BS_BWD_SEQ, BS_BWD_CHANNEL, BS_SPLIT_ROW, BS_SPLIT_CHANNEL,
+};
+#ifdef SSM_CHECK_BOUNDS
+struct BoundsRecord {
+    int32_t code, site;
+    long long index, extent;
+};
+extern __device__ BoundsRecord g_ssm_bounds;
+SSM_DEVINL bool bounds_ok(int64_t index, int64_t extent, int site) {
+    if (index >= 0 && index < extent) return true;
+    if (atomicCAS(&g_ssm_bounds.code, 0, SSM_DEVERR_BOUNDS) == 0) {
+        g_ssm_bounds.site = site;
+        g_ssm_bounds.index = (long long)index;
+        g_ssm_bounds.extent = (long long)extent;
+        __threadfence();
+    }
+    return false;
+}
+#define SSM_BOUNDS(index, extent, site) ::ssm::bounds_ok((int64_t)(index), (int64_t)(extent), (int)(site))
+#else
+#define SSM_BOUNDS(index, extent, site) true
+#endif
+
 // ----------------------------------------------------------- element I/O
 template <typename T> struct Elem;
 template <> struct Elem<float> {

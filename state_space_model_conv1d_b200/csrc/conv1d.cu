@@ -59,6 +59,10 @@ conv1d_kernel(const T *__restrict__ x, int64_t x_bs, int64_t x_ts, const float *
     // Offsets are clamped into [0, seqlen] so a malformed cu_seqlens can give
     // wrong values but never an out-of-bounds access.
     int s = cu ? seq_of_token(cu, nseqs, tr0) : row;
+    // bounds-checked build: this thread's channels and sequence
+    if (!SSM_BOUNDS(c0 + VEC - 1 < channels ? c0 + VEC - 1 : c0, channels, BS_CONV_CHANNEL) ||
+        !SSM_BOUNDS(s, cu ? nseqs : (int)gridDim.z, BS_CONV_STATE))
+        return;
     int64_t start = cu ? min(max((int64_t)cu[s], (int64_t)0), seqlen) : 0;
     int64_t end = cu ? min(max((int64_t)cu[s + 1], start), seqlen) : seqlen;
     auto load_hist = [&](int64_t t) {

@@ -173,6 +173,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
     int64_t slot = a.idx ? (int64_t)a.idx[r] : r;
     const T *xr = static_cast<const T *>(a.x) + r * a.x_bs;
     T *yr = static_cast<T *>(a.y) + r * a.y_bs;
+    // bounds-checked build: the CTA's channel range (uniform, so the whole CTA returns together)
+    if (!SSM_BOUNDS(c0 + nx - 1, a.Dn, BS_DEC_CHANNEL) || !SSM_BOUNDS(r, (int64_t)gridDim.y, BS_DEC_ROW)) return;
     if (slot < 0 || slot >= a.nslots) {                 // padding row: y = 0, nothing else touched
         for (int64_t i = threadIdx.x; i < nx; i += kThreads) Elem<T>::st(yr + c0 + i, 0.f);
         return;

@@ -98,6 +98,10 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdArgs a) {
     const int64_t g = m1 ? 0 : hh / (a.H / a.G);
     const int64_t N = a.N, Dn = a.Dn, GN = a.G * a.N;
     const int64_t cdim = m1 ? Dn : Dn + 2 * GN;
+    // bounds-checked build: the CTA's ranges (uniform, so the whole CTA returns together)
+    if (!SSM_BOUNDS(q.len > 0 ? q.start + q.len - 1 : 0, a.T > 0 ? a.T : 1, BS_BWD_SEQ) ||
+        !SSM_BOUNDS(m1 ? p0 : hh * a.P + p0, Dn, BS_BWD_CHANNEL))
+        return;
 
     // shared memory
     float *hs = smb;                                         // [TC+1][kBT][NS]

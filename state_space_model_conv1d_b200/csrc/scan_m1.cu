@@ -148,6 +148,10 @@ scan_m1_kernel(const M1Args a) {
     const T *Bg = static_cast<const T *>(a.B) + row * a.B_bs + start * a.B_ts;
     const T *Cg = static_cast<const T *>(a.C) + row * a.C_bs + start * a.C_ts;
     T *yg = static_cast<T *>(a.y) + row * a.y_bs + start * a.y_ts;
+    // bounds-checked build: the CTA's ranges (uniform, so the whole CTA returns together)
+    if (!SSM_BOUNDS(len > 0 ? start + len - 1 : 0, a.seqlen > 0 ? a.seqlen : 1, BS_M1_SEQ) ||
+        !SSM_BOUNDS(d0, a.Dn, BS_M1_CHANNEL) || !SSM_BOUNDS(s, a.sv.nseqs, BS_M1_STATE))
+        return;
     const int K = a.K;
     const int64_t Dn = a.Dn, N = a.N;
     const int nchunks = max(1, (int)((len + kTC - 1) / kTC));   // an empty sequence still passes its state through
@@ -248,12 +252,13 @@ scan_m1_kernel(const M1Args a) {
                 float o[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[e] = sm.y[yb][r][v * 8 + e];
-                Vec8<T>::st(yg + (t0 + r) * a.y_ts + d0 + v * 8, o);
+                if (SSM_BOUNDS(start + t0 + r, a.seqlen, BS_M1_Y)) Vec8<T>::st(yg + (t0 + r) * a.y_ts + d0 + v * 8, o);
             }
         } else {
             for (int i = tid; i < nv * kDB; i += kThreads) {
                 const int r = i / kDB, v = i % kDB;
-                if (d0 + v < Dn) Elem<T>::st(yg + (t0 + r) * a.y_ts + d0 + v, sm.y[yb][r][v]);
+                if (d0 + v < Dn && SSM_BOUNDS(start + t0 + r, a.seqlen, BS_M1_Y))
+                    Elem<T>::st(yg + (t0 + r) * a.y_ts + d0 + v, sm.y[yb][r][v]);
             }
         }
     };
@@ -358,7 +363,7 @@ scan_m1_kernel(const M1Args a) {
     // c + 1 (written by the prologue of chunk c)
     auto inter_store = [&](int c) {
         const int64_t slot = a.iv.slot_after(s, (int64_t)(c + 1) * kTC);
-        if (slot < 0) return;
+        if (slot < 0 || !SSM_BOUNDS(slot, a.iv.nslots, BS_M1_POOL)) return;
         if (a.iv.states && svalid) {
             float *dst = a.iv.states + (slot * Dn + sch) * N;
 #pragma unroll
@@ -581,6 +586,10 @@ scan_m1_tp_kernel(const M1Args a) {
     const T *Bg = static_cast<const T *>(a.B) + row * a.B_bs + start * a.B_ts;
     const T *Cg = static_cast<const T *>(a.C) + row * a.C_bs + start * a.C_ts;
     T *yg = static_cast<T *>(a.y) + row * a.y_bs + start * a.y_ts;
+    // bounds-checked build: the CTA's ranges (uniform, so the whole CTA returns together)
+    if (!SSM_BOUNDS(len > 0 ? start + len - 1 : 0, a.seqlen > 0 ? a.seqlen : 1, BS_M1_SEQ) ||
+        !SSM_BOUNDS(d0, a.Dn, BS_M1_CHANNEL) || !SSM_BOUNDS(s, a.sv.nseqs, BS_M1_STATE))
+        return;
     const int K = a.K;
     const int64_t Dn = a.Dn;
     const int nchunks = max(1, (int)((len + TP_TC - 1) / TP_TC));   // an empty sequence still passes its state through
@@ -677,12 +686,13 @@ scan_m1_tp_kernel(const M1Args a) {
                 float o[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[e] = sm.y[yb][r][v * 8 + e];
-                Vec8<T>::st(yg + (t0 + r) * a.y_ts + d0 + v * 8, o);
+                if (SSM_BOUNDS(start + t0 + r, a.seqlen, BS_M1_Y)) Vec8<T>::st(yg + (t0 + r) * a.y_ts + d0 + v * 8, o);
             }
         } else {
             for (int i = tid; i < nv * TP_DB; i += TP_THREADS) {
                 const int r = i / TP_DB, v = i % TP_DB;
-                if (d0 + v < Dn) Elem<T>::st(yg + (t0 + r) * a.y_ts + d0 + v, sm.y[yb][r][v]);
+                if (d0 + v < Dn && SSM_BOUNDS(start + t0 + r, a.seqlen, BS_M1_Y))
+                    Elem<T>::st(yg + (t0 + r) * a.y_ts + d0 + v, sm.y[yb][r][v]);
             }
         }
     };
@@ -795,7 +805,7 @@ scan_m1_tp_kernel(const M1Args a) {
     // is the halo the prologue of chunk c left for chunk c + 1
     auto inter_store = [&](int c) {
         const int64_t slot = a.iv.slot_after(s, (int64_t)(c + 1) * TP_TC);
-        if (slot < 0) return;
+        if (slot < 0 || !SSM_BOUNDS(slot, a.iv.nslots, BS_M1_POOL)) return;
         if (a.iv.states)
             for (int i = tid; i < TP_DB * N; i += TP_THREADS) {
                 const int cidx = i / N, n = i % N;

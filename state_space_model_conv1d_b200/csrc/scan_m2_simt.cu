@@ -100,6 +100,10 @@ scan_m2_simt_kernel(const M2Args a) {
     const T *Bg = static_cast<const T *>(a.B) + row * a.B_bs + start * a.B_ts + g * N;
     const T *Cg = static_cast<const T *>(a.C) + row * a.C_bs + start * a.C_ts + g * N;
     T *yg = static_cast<T *>(a.y) + row * a.y_bs + start * a.y_ts + hh * P;
+    // bounds-checked build: the CTA's ranges (uniform, so the whole CTA returns together)
+    if (!SSM_BOUNDS(len > 0 ? start + len - 1 : 0, a.seqlen > 0 ? a.seqlen : 1, BS_M2S_SEQ) ||
+        !SSM_BOUNDS((int64_t)hh * P + p0, Dn, BS_M2S_HEAD) || !SSM_BOUNDS(s, a.sv.nseqs, BS_M2S_STATE))
+        return;
     const int ncols = (int)min((int64_t)kPB, P - p0);
     // conv channel indices of this block's x columns and of the group's B / C
     const int64_t xch0 = hh * P + p0, bch0 = Dn + g * N, cch0 = Dn + G * N + g * N;

@@ -189,6 +189,13 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
     const int n = (int)((len + kQ - 1) / kQ);
     const int crow = (int)row, g0 = (int)(g * kN);
     const uint32_t sbase = tc::smem_u32(smem);
+    // bounds-checked build: the CTA's ranges (uniform, so the whole CTA returns together)
+    if (!SSM_BOUNDS(len > 0 ? start + len - 1 : 0, a.seqlen > 0 ? a.seqlen : 1, BS_SSD_SEQ) ||
+        !SSM_BOUNDS((int64_t)hh * kP + kP - 1, a.H * kP, BS_SSD_HEAD) ||
+        !SSM_BOUNDS((int64_t)g0 + kN - 1, a.G * kN, BS_SSD_GROUP) ||
+        !SSM_BOUNDS((int64_t)s * H + hh, (int64_t)a.sv.nseqs * H, BS_SSD_STATE) ||
+        !SSM_BOUNDS(((int64_t)s + 1) * a.cdim - 1, (int64_t)a.sv.nseqs * a.cdim, BS_SSD_CONV_STATE))
+        return;
     const float A2 = a.A[hh] * kLog2e;
 
     if (tid == 0) {
@@ -593,7 +600,8 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                                         *reinterpret_cast<__nv_bfloat162 *>(stg + off) = ob;
                                     } else {
                                         const int i = rr ? i1 : i0;
-                                        if (i < nv && st_ok) *reinterpret_cast<__nv_bfloat162 *>(yg + (t0 + i) * a.y_ts + jc + 8 * kk) = ob;
+                                        if (i < nv && st_ok && SSM_BOUNDS(start + t0 + i, a.seqlen, BS_SSD_Y))
+                                            *reinterpret_cast<__nv_bfloat162 *>(yg + (t0 + i) * a.y_ts + jc + 8 * kk) = ob;
                                     }
                                 }
                             }
@@ -628,7 +636,7 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                 // intermediate state after this chunk when it closes a state interval
                 if (a.iv.interval > 0 && nv == kQ && !aborted(ax)) {
                     const int64_t slot = a.iv.slot_after(s, t0 + kQ);
-                    if (slot >= 0) {
+                    if (slot >= 0 && SSM_BOUNDS(slot, a.iv.nslots, BS_SSD_POOL)) {
                         if (a.iv.states) {
                             float *dst = a.iv.states + (slot * H + hh) * kP * kN;
 #pragma unroll
@@ -651,6 +659,7 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                                 for (int i = tid; i < 2 * kN * (K - 1); i += kComputeThreads) {
                                     const int which = i / (kN * (K - 1)), nn = (i / (K - 1)) % kN, j = i % (K - 1);
                                     const int64_t tok = start + t0 + kQ - (K - 1) + j;
+                                    if (!SSM_BOUNDS(tok, a.seqlen, BS_SSD_RAW_BC)) continue;
                                     const __nv_bfloat16 v = which ? a.Craw[row * a.craw_bs + tok * a.craw_ts + g * kN + nn]
                                                                   : a.Braw[row * a.braw_bs + tok * a.braw_ts + g * kN + nn];
                                     cdst[(a.H * kP + which * GN + g * kN + nn) * (K - 1) + j] = v;
@@ -759,7 +768,9 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                     const int64_t tau = len - (K - 1) + j;           // within the sequence
                     v[j] = __float2bfloat16_rn(0.f);
                     if (j < K - 1) {
-                        if (tau >= 0) v[j] = raw[(start + tau) * rts];
+                        if (tau >= 0) {
+                            if (SSM_BOUNDS(start + tau, a.seqlen, BS_SSD_RAW_BC)) v[j] = raw[(start + tau) * rts];
+                        }
                         else if (a.conv_state_in) v[j] = a.conv_state_in[((int64_t)s * a.cdim + ch) * (K - 1) + tau + (K - 1)];
                     }
                 }
@@ -801,14 +812,26 @@ __global__ void __launch_bounds__(128, 3) bc_conv_kernel(const BcArgs a) {
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t vec = idx % nvec, run = idx / nvec;
     const int64_t t0 = run * 8;
-    if (t0 >= a.seqlen) return;
     const int64_t row = blockIdx.y;
+    // packed sequences: one thread finds the sequence of the CTA's first token,
+    // every thread walks on from there (its run starts at most a few tokens later)
+    __shared__ int s_first;
+    if (a.cu) {
+        if (threadIdx.x == 0) {
+            const int64_t tf = ((int64_t)blockIdx.x * blockDim.x / nvec) * 8;
+            s_first = seq_of_token(a.cu, a.nseqs, min(tf, a.seqlen > 0 ? a.seqlen - 1 : (int64_t)0));
+        }
+        __syncthreads();
+    }
+    if (t0 >= a.seqlen) return;
     const int which = vec >= nvec / 2;                    // 0: B, 1: C
     const int64_t c0 = (vec - which * (nvec / 2)) * 8;    // channel within B (or C)
     const __nv_bfloat16 *src = which ? a.C + row * a.c_bs : a.B + row * a.b_bs;
     const int64_t ts = which ? a.c_ts : a.b_ts;
     __nv_bfloat16 *dst = (which ? a.oC : a.oB) + row * a.seqlen * a.GN + c0;
     const int64_t cch = a.HP + which * a.GN + c0;         // conv channel of the first of the 8
+    if (!SSM_BOUNDS(c0 + 7, a.GN, BS_BC_CHANNEL) || !SSM_BOUNDS(row * a.seqlen + t0, (int64_t)gridDim.y * a.seqlen, BS_BC_ROW))
+        return;
     float wk[K][8], bb[8];
 #pragma unroll
     for (int v = 0; v < 8; ++v) {
@@ -818,7 +841,11 @@ __global__ void __launch_bounds__(128, 3) bc_conv_kernel(const BcArgs a) {
     }
     // sequence of the run's first token and its bounds (clamped: a malformed
     // cu_seqlens gives wrong values but no out-of-bounds access)
-    int s = a.cu ? seq_of_token(a.cu, a.nseqs, t0) : (int)row;
+    int s = (int)row;
+    if (a.cu) {
+        s = s_first;
+        while (s + 1 < a.nseqs && a.cu[s + 1] <= t0) ++s;
+    }
     int64_t start = a.cu ? min(max((int64_t)a.cu[s], (int64_t)0), a.seqlen) : 0;
     int64_t end = a.cu ? min(max((int64_t)a.cu[s + 1], start), a.seqlen) : a.seqlen;
     float hist[K > 1 ? K - 1 : 1][8];
@@ -830,11 +857,12 @@ __global__ void __launch_bounds__(128, 3) bc_conv_kernel(const BcArgs a) {
                 Vec8<__nv_bfloat16>::ld(src + tau * ts + c0, hist[j]);
             } else {
                 const int64_t q = tau - start + (K - 1);
+                const bool in = a.state_in && q >= 0 &&
+                                SSM_BOUNDS(((int64_t)s * a.cdim + cch + 7) * (K - 1) + q,
+                                           (int64_t)(a.cu ? a.nseqs : gridDim.y) * a.cdim * (K - 1), BS_BC_STATE);
 #pragma unroll
                 for (int v = 0; v < 8; ++v)
-                    hist[j][v] = (a.state_in && q >= 0)
-                                     ? __bfloat162float(a.state_in[((int64_t)s * a.cdim + cch + v) * (K - 1) + q])
-                                     : 0.f;
+                    hist[j][v] = in ? __bfloat162float(a.state_in[((int64_t)s * a.cdim + cch + v) * (K - 1) + q]) : 0.f;
             }
         }
     };

@@ -5,7 +5,14 @@
 #include <cuda_runtime.h>
 
 #include "../../include/ssm.h"
+#include "common.cuh"
 #include "launch.h"
+
+#ifdef SSM_CHECK_BOUNDS
+namespace ssm {
+__device__ BoundsRecord g_ssm_bounds;
+}
+#endif
 
 namespace {
 
@@ -327,6 +334,34 @@ ssm_status ssm_split_fixup(const ssm_scan_args *args, const float *cum_delta, co
     if (!cum_delta || !h_in) return SSM_ERR_INVALID_ARG;
     if (!aligned(cum_delta, 4) || !aligned(h_in, 4)) return SSM_ERR_ALIGNMENT;
     return cuda_status(ssm::launch_split_fixup(*args, cum_delta, h_in, (cudaStream_t)stream));
+}
+
+int32_t ssm_check_bounds_enabled(void) {
+#ifdef SSM_CHECK_BOUNDS
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+ssm_status ssm_bounds_record(int32_t *code, int32_t *site, int64_t *index, int64_t *extent, int32_t clear) {
+#ifdef SSM_CHECK_BOUNDS
+    SSM_TRY(cuda_status(cudaDeviceSynchronize()));
+    ssm::BoundsRecord r{};
+    SSM_TRY(cuda_status(cudaMemcpyFromSymbol(&r, ssm::g_ssm_bounds, sizeof(r))));
+    if (code) *code = r.code;
+    if (site) *site = r.site;
+    if (index) *index = r.index;
+    if (extent) *extent = r.extent;
+    if (clear) {
+        const ssm::BoundsRecord z{};
+        SSM_TRY(cuda_status(cudaMemcpyToSymbol(ssm::g_ssm_bounds, &z, sizeof(z))));
+    }
+    return SSM_OK;
+#else
+    (void)code; (void)site; (void)index; (void)extent; (void)clear;
+    return SSM_ERR_UNSUPPORTED;
+#endif
 }
 
 ssm_status ssm_workspace_error(const void *workspace, int32_t *code, void *stream) {

@@ -270,3 +270,21 @@ def test_plain_c_consumer(tmp_path):
                     f"-Wl,-rpath,{libdir}"], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout + out.stderr
+
+
+def test_bounds_checked_build_plumbing():
+    """The bounds-checked build exports the same ABI and reports itself as
+    checked; the normal build reports that it is not and has no record to read."""
+    lib = _abi.lib()
+    assert lib.ssm_check_bounds_enabled() == 0
+    assert lib.ssm_bounds_record(None, None, None, None, 0) == _abi.SSM_ERR_UNSUPPORTED
+    path = os.path.join(os.path.dirname(_abi.LIB_PATH), "libssm_checked.so")
+    assert os.path.exists(path), "build the checked library: python -m state_space_model_conv1d_b200.build --check-bounds"
+    chk = _abi.checked_lib()
+    assert chk.ssm_check_bounds_enabled() == 1
+    assert chk.ssm_abi_version() == 1
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    assert declared_symbols() <= exported
+    # host-side validation is the same code in both builds
+    assert chk.ssm_scan_fwd(None, None, 0, None) == _abi.SSM_ERR_INVALID_ARG
