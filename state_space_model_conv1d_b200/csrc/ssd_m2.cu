@@ -804,6 +804,7 @@ struct BcArgs {
     const int32_t *cu;
     int nseqs;
     int64_t seqlen, GN, HP, cdim;
+    bool w16, b16;                    // taps / bias of every 8-channel vector start 16-byte aligned
 };
 
 template <int K>
@@ -832,12 +833,29 @@ __global__ void __launch_bounds__(128, 3) bc_conv_kernel(const BcArgs a) {
     const int64_t cch = a.HP + which * a.GN + c0;         // conv channel of the first of the 8
     if (!SSM_BOUNDS(c0 + 7, a.GN, BS_BC_CHANNEL) || !SSM_BOUNDS(row * a.seqlen + t0, (int64_t)gridDim.y * a.seqlen, BS_BC_ROW))
         return;
+    // taps and bias of the 8 channels: 16-byte loads when they are aligned (the
+    // weight rows are contiguous: 8 channels x K taps), scalar loads otherwise
     float wk[K][8], bb[8];
+    if (K == 4 && a.w16) {
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
+        for (int v = 0; v < 8; ++v) {
+            const float4 q = *reinterpret_cast<const float4 *>(a.w + (cch + v) * 4);
+            wk[0][v] = q.x; wk[1 % K][v] = q.y; wk[2 % K][v] = q.z; wk[3 % K][v] = q.w;
+        }
+    } else {
 #pragma unroll
-        for (int k = 0; k < K; ++k) wk[k][v] = a.w[(cch + v) * K + k];
-        bb[v] = a.bias ? a.bias[cch + v] : 0.f;
+        for (int v = 0; v < 8; ++v)
+#pragma unroll
+            for (int k = 0; k < K; ++k) wk[k][v] = a.w[(cch + v) * K + k];
+    }
+    if (a.bias && a.b16) {
+        const float4 b0 = *reinterpret_cast<const float4 *>(a.bias + cch);
+        const float4 b1 = *reinterpret_cast<const float4 *>(a.bias + cch + 4);
+        bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w;
+        bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
+    } else {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) bb[v] = a.bias ? a.bias[cch + v] : 0.f;
     }
     // sequence of the run's first token and its bounds (clamped: a malformed
     // cu_seqlens gives wrong values but no out-of-bounds access)
@@ -1003,6 +1021,10 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
         b.oB = wB; b.oC = wC;
         b.cu = s.cu_seqlens; b.nseqs = s.nseqs;
         b.seqlen = s.seqlen; b.GN = GN; b.HP = s.d_inner; b.cdim = cdim;
+        // channel offsets are multiples of 8 (d_inner = H * 64, G * N = G * 128), so the
+        // rows start 16-byte aligned whenever the arrays do
+        b.w16 = ((uintptr_t)s.conv_w % 16) == 0;
+        b.b16 = s.conv_b != nullptr && ((uintptr_t)s.conv_b % 16) == 0;
         const int64_t threads = (s.seqlen + 7) / 8 * (GN / 4);
         const dim3 bgrid((unsigned)((threads + 127) / 128), (unsigned)rows);
         if (threads > 0) {
