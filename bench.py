@@ -230,7 +230,12 @@ class Job:
                 self.flops = None
                 self.launches_per_step = 1 + (1 if mode == ssm.MAMBA2 else 0)
             elif mode == ssm.MAMBA1:
-                self.kernel, self.sources = "scan_m1_kernel", ("scan_m1.cu",)
+                # the library runs the time-parallel form when the sequential one would
+                # leave the SMs short of warps (fewer than 7 per SM, dstate 16 / 32)
+                nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+                tp = w.dstate in (16, 32) and w.d_conv <= 4 and nseq * ((w.d_inner + 31) // 32) * 4 < 7 * nsm
+                self.kernel = "scan_m1_tp_kernel" if tp else "scan_m1_kernel"
+                self.sources = ("scan_m1.cu",)
                 self.mufu = x.shape[0] * x.shape[1] * x.shape[2] * t["B"].shape[2]
                 self.flops = None
             elif self.ssd:

@@ -221,6 +221,11 @@ WORKLOADS = {
     "mamba1_layer_b8_l2048_d1536_n16_split2": Workload(
         "mamba1_layer_b8_l2048_d1536_n16_split2", "mamba1", "bf16", batch=8, seqlen=2048, d_inner=1536, dstate=16,
         split_ranks=2, split_rank=1, seed=BASE_SEED + 1),
+    # one long Mamba-1 sequence (a single-prompt prefill): too few channels x
+    # batch rows to fill the GPU with the sequential scan, so the time-parallel
+    # (warp-shuffle pair scan) form runs
+    "mamba1_seq_b1_l8192_d1536_n16": Workload("mamba1_seq_b1_l8192_d1536_n16", "mamba1", "bf16", batch=1,
+                                              seqlen=8192, d_inner=1536, dstate=16, seed=BASE_SEED + 5),
     # the Mamba-1 layer's backward (same inputs; upstream gradients drawn alongside)
     "mamba1_layer_b8_l2048_d1536_n16_bwd": Workload("mamba1_layer_b8_l2048_d1536_n16_bwd", "mamba1", "bf16", batch=8,
                                                     seqlen=2048, d_inner=1536, dstate=16, backward=True,
