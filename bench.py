@@ -137,6 +137,8 @@ class Job:
         seed_shift = rank_seed(0, rank)
         bf = torch.bfloat16 if w.dtype == "bf16" else torch.float32
         self.launches_per_step = 1
+        self.split = None          # set by the sequence-split workloads
+        self.bwd = None            # set by the backward workloads
         if w.kind in ("mamba1", "mamba2", "mamba2_varlen"):
             mode = ssm.MAMBA1 if w.kind == "mamba1" else ssm.MAMBA2
             ww = W.Workload(**{**w.__dict__, "seed": w.seed + seed_shift})
