@@ -139,6 +139,7 @@ class Job:
         self.launches_per_step = 1
         self.split = None          # set by the sequence-split workloads
         self.bwd = None            # set by the backward workloads
+        self.timing_on = False     # kernel timing enabled (the timed region)
         if w.kind in ("mamba1", "mamba2", "mamba2_varlen"):
             mode = ssm.MAMBA1 if w.kind == "mamba1" else ssm.MAMBA2
             ww = W.Workload(**{**w.__dict__, "seed": w.seed + seed_shift})
@@ -253,6 +254,10 @@ class Job:
                 self.kernel, self.sources = "scan_m2_simt_kernel", ("scan_m2_simt.cu",)
                 self.mufu = None
                 self.flops = None
+            if self.split is not None:
+                # a rank's step of the split: its largest kernel is the fix-up
+                self.kernel = "split_fixup_m1_kernel" if mode == ssm.MAMBA1 else "split_fixup_m2_kernel"
+                self.sources = ("seq_split.cu",)
         elif w.kind == "decode":
             ww = W.Workload(**{**w.__dict__, "seed": w.seed + seed_shift})
             d = W.workload_inputs(ww)
@@ -327,13 +332,33 @@ class Job:
         # tail, the scan's launches, cum_delta, combine, fix-up (the pair packing and the
         # staging copy are torch's)
         self.launches_per_step = 1 + self.launches_per_step + 3
+        # The fix-up is the step's largest kernel: the roofline names it, with its own
+        # algorithmic bytes (y read and written, z, the raw C rows and their conv taps,
+        # the prefix sums of delta and the entering state) and, for Mamba-2, the
+        # fp32 FMAs of C_t . h_in (2 N P per token and head).  Its launches alone
+        # are bracketed by the kernel-timing events (see _split_step).
+        cum_units = w.d_inner if mode == self.ssm.MAMBA1 else w.nheads
+        b_, T_ = t["x"].shape[0], t["x"].shape[1]
+        self.fix_bytes = (3 * self.y.numel() * self.y.element_size() + t["C"].numel() * t["C"].element_size()
+                          + b_ * T_ * cum_units * 4 + self.hf.numel() * 4)
+        if mode == self.ssm.MAMBA1:
+            self.fix_mufu = b_ * T_ * w.d_inner * w.dstate          # exp(A cs_t) per (token, channel, state)
+            self.fix_flops = None
+        else:
+            self.fix_mufu = None
+            self.fix_flops = 2 * b_ * T_ * w.nheads * w.headdim * w.dstate
 
     def _split_step(self):
         sp, t = self.split, self.t
         seg = sp["mod"].SegmentScan(self.mode, sp["r"], sp["R"], t["x"], t["dt"], t["A"], t["B"], t["C"], z=t["z"],
                                     **sp["kw"])
+        timed = self.timing_on
+        if timed:
+            self.ssm.kernel_timing(False)         # only the fix-up is bracketed
         seg.tail()
         sp["pairs"][sp["r"]].copy_(seg.scan(sp["tails"]))
+        if timed:
+            self.ssm.kernel_timing(True)
         self.y, self.hf, _ = seg.join(sp["pairs"])
 
     def step(self):
@@ -435,6 +460,7 @@ def run_cuda(args):
     torch.cuda.synchronize()
     ssm.kernel_time_ms()                       # drop any earlier tally
     ssm.kernel_timing(True)                    # events around the dominant kernel of each call, on its stream
+    job.timing_on = True
     for i in range(args.steps):
         flush_l2(flush)
         evs[i][0].record(stream)
@@ -442,6 +468,7 @@ def run_cuda(args):
         evs[i][1].record(stream)
     torch.cuda.synchronize()
     ssm.kernel_timing(False)
+    job.timing_on = False
     kern_ms_total, kern_launches = ssm.kernel_time_ms()
     if world > 1:
         dist.barrier()
@@ -482,7 +509,10 @@ def run_cuda(args):
     peaks, peak_src = load_peaks()
     hbm_peak = float(peaks["hbm_gbs"])
     gbs = job.bytes_per_step / (ms_per_step / 1e3) / 1e9
-    kgbs = job.bytes_per_step / (kern_ms / 1e3) / 1e9 if kern_ms > 0 else gbs
+    kbytes = job.fix_bytes if job.split is not None else job.bytes_per_step   # the timed kernel's own bytes
+    kgbs = kbytes / (kern_ms / 1e3) / 1e9 if kern_ms > 0 else gbs
+    if job.split is not None:
+        job.mufu, job.flops = job.fix_mufu, None
     traffic = None
     if os.path.exists(TRAFFIC_PATH):
         with open(TRAFFIC_PATH) as f:
@@ -507,7 +537,13 @@ def run_cuda(args):
             tpk = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1400.0)))
             roofline["tensor"] = {"achieved": tf, "peak": tpk, "unit": "TFLOP/s", "frac": tf / tpk,
                                   "flops_per_step": int(job.flops), "peak_source": "MEASURED_PEAKS.json bf16_tflops_sustained"}
-    roofline["algorithmic_bytes_per_launch"] = int(job.bytes_per_step)
+    if job.split is not None and job.fix_flops:
+        fma_peak = NUM_SMS * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+        ftf = job.fix_flops / (kern_ms / 1e3) / 1e12
+        roofline["fma"] = {"achieved": ftf, "peak": fma_peak, "unit": "TFLOP/s", "frac": ftf / fma_peak,
+                           "flops_per_launch": int(job.fix_flops),
+                           "peak_source": f"derived: {NUM_SMS} SMs x 128 fp32 FMA/clk x 2 x clock"}
+    roofline["algorithmic_bytes_per_launch"] = int(kbytes)
     roofline["kernel_ms"] = kern_ms
     roofline["kernel_launches_timed"] = kern_launches
     roofline["timing"] = ("CUDA events around every launch of the kernel, on its stream, inside the timed region "

@@ -255,7 +255,8 @@ SSM_API ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *args, void *workspace, 
 SSM_API ssm_status ssm_state_update(const ssm_update_args *args, void *stream);
 
 /* Per-kernel device timing of the dominant kernel of each call (the scan
- * kernel of ssm_scan_fwd, the update kernel of ssm_state_update), for
+ * kernel of ssm_scan_fwd, the update kernel of ssm_state_update, the backward
+ * kernel of ssm_scan_bwd, the fix-up kernel of ssm_split_fixup), for
  * roofline measurements.  The papers have no counterpart.  While enabled
  * (process-wide, off by default), every such launch is bracketed by a CUDA
  * event pair recorded on the call's own stream (events are created on first
@@ -372,7 +373,8 @@ SSM_API ssm_status ssm_split_cum_delta(const ssm_scan_args *args, float *cum_del
 SSM_API ssm_status ssm_split_combine(const ssm_split_args *args, void *stream);
 /* Step 6.  `args` describes the segment's ssm_scan_fwd call; its y is
  * updated in place, its h0 / h_final / conv_state_out fields are ignored.
- * cum_delta is step 3's output, h_in step 5's. */
+ * cum_delta is step 3's output, h_in step 5's.  A segment with no tokens
+ * returns SSM_OK without touching anything (the pointers may be NULL). */
 SSM_API ssm_status ssm_split_fixup(const ssm_scan_args *args, const float *cum_delta, const float *h_in,
                                    void *stream);
 

@@ -393,7 +393,9 @@ cudaError_t fixup_typed(const ssm_scan_args &a, const float *cum, const float *h
     if (!m2) {
         dim3 grid((unsigned)((a.d_inner + kF1Threads - 1) / kF1Threads), (unsigned)((a.seqlen + kF1Tok - 1) / kF1Tok),
                   (unsigned)a.batch);
+        timing_begin(st);
         split_fixup_m1_kernel<T><<<grid, kF1Threads, 0, st>>>(f);
+        timing_end(st);
         return cudaGetLastError();
     }
     const size_t smem = fixup_m2_smem(a.dstate);
@@ -403,7 +405,9 @@ cudaError_t fixup_typed(const ssm_scan_args &a, const float *cum, const float *h
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)fixup_m2_smem(kMaxDstateM2));
     if (e != cudaSuccess) return e;
+    timing_begin(st);
     kern<<<grid, kF2Threads, smem, st>>>(f);
+    timing_end(st);
     return cudaGetLastError();
 }
 

@@ -204,11 +204,13 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
         for (int i = 0; i < kNumMbar; ++i)
             tc::mbar_init(&ax.mb[i], (i == MB_CONV || i == MB_ZFREE || i == MB_SREADY || i == MB_MREADY) ? kComputeWarps : 1);
         tc::mbar_init_fence();
-        tc::prefetch_map(&tm_x);
-        tc::prefetch_map(&tm_b);
-        tc::prefetch_map(&tm_c);
-        if (a.z) tc::prefetch_map(&tm_z);
-        tc::prefetch_map(&tm_y);
+        if (n > 0) {                       // a CTA with no chunk touches no tensor map
+            tc::prefetch_map(&tm_x);
+            tc::prefetch_map(&tm_b);
+            tc::prefetch_map(&tm_c);
+            if (a.z) tc::prefetch_map(&tm_z);
+            tc::prefetch_map(&tm_y);
+        }
     }
     if (warp == kComputeWarps) tc::tmem_alloc(&ax.tmem, kTmemCols);
     // the mask tile's blocks above the diagonal are zero for good
@@ -1001,14 +1003,19 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     // launches from the scan launch.
     const int64_t rows = s.cu_seqlens ? 1 : s.batch;
     CUtensorMap tm_x, tm_b, tm_c, tm_z, tm_y;
-    memset(&tm_z, 0, sizeof(tm_z));
-    if (s.z && !make_map(&tm_z, s.z, s.d_inner, s.seqlen, rows, s.z_token_stride, s.z_batch_stride, true))
-        return cudaErrorInvalidValue;
-    if (!make_map(&tm_x, s.x, s.d_inner, s.seqlen, rows, s.x_token_stride, s.x_batch_stride, false) ||
-        !make_map(&tm_b, Bc, GN, s.seqlen, rows, b_ts, b_bs, true) ||
-        !make_map(&tm_c, Cc, GN, s.seqlen, rows, c_ts, c_bs, true) ||
-        !make_map(&tm_y, s.y, s.d_inner, s.seqlen, rows, s.y_token_stride, s.y_batch_stride, true))
-        return cudaErrorInvalidValue;
+    memset(&tm_x, 0, sizeof(tm_x)); memset(&tm_b, 0, sizeof(tm_b)); memset(&tm_c, 0, sizeof(tm_c));
+    memset(&tm_z, 0, sizeof(tm_z)); memset(&tm_y, 0, sizeof(tm_y));
+    // With no tokens at all no CTA has a chunk, so no copy is issued and the
+    // maps (which cannot describe an empty tensor) are left unset.
+    if (s.seqlen > 0) {
+        if (s.z && !make_map(&tm_z, s.z, s.d_inner, s.seqlen, rows, s.z_token_stride, s.z_batch_stride, true))
+            return cudaErrorInvalidValue;
+        if (!make_map(&tm_x, s.x, s.d_inner, s.seqlen, rows, s.x_token_stride, s.x_batch_stride, false) ||
+            !make_map(&tm_b, Bc, GN, s.seqlen, rows, b_ts, b_bs, true) ||
+            !make_map(&tm_c, Cc, GN, s.seqlen, rows, c_ts, c_bs, true) ||
+            !make_map(&tm_y, s.y, s.d_inner, s.seqlen, rows, s.y_token_stride, s.y_batch_stride, true))
+            return cudaErrorInvalidValue;
+    }
     cudaError_t e = cudaFuncSetAttribute(ssd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     if (s.d_conv > 0) {

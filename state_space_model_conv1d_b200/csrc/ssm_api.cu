@@ -331,6 +331,7 @@ ssm_status ssm_split_combine(const ssm_split_args *a, void *stream) {
 
 ssm_status ssm_split_fixup(const ssm_scan_args *args, const float *cum_delta, const float *h_in, void *stream) {
     SSM_TRY(validate_split_scan(args));
+    if (args->batch == 0 || args->seqlen == 0) return SSM_OK;   // a segment with no tokens has no y to fix
     if (!cum_delta || !h_in) return SSM_ERR_INVALID_ARG;
     if (!aligned(cum_delta, 4) || !aligned(h_in, 4)) return SSM_ERR_ALIGNMENT;
     return cuda_status(ssm::launch_split_fixup(*args, cum_delta, h_in, (cudaStream_t)stream));

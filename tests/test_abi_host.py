@@ -234,6 +234,14 @@ def test_split_own_arguments_rejected():
     assert lib.ssm_split_fixup(C.byref(a), FAKE, None, None) == _abi.SSM_ERR_INVALID_ARG
 
 
+def test_split_fixup_of_an_empty_segment_is_a_no_op():
+    # A rank whose segment holds no tokens has no y to fix; its cum_delta and
+    # h_in are empty, so their pointers may be NULL.
+    lib = _abi.lib()
+    a = _scan(seqlen=0)
+    assert lib.ssm_split_fixup(C.byref(a), None, None, None) == _abi.SSM_OK
+
+
 def _split(**kw):
     a = _abi.SplitArgs()
     a.mode, a.rank, a.nranks = 2, 1, 2

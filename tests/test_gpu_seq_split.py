@@ -88,3 +88,32 @@ def test_mamba2_simt_shapes(dtype, P, N, bounds):
 def test_single_rank_is_the_plain_scan():
     d = W.mamba2_inputs(905, 2, 96, 4, 8, 2, 16, dtype="f32", conv_bias=True, conv_state=True)
     _check(M2, d, "f32", [0, 96])
+
+
+def test_mamba2_scalar_fixup_dstate_not_multiple_of_4():
+    """dstate 5: the Mamba-2 fix-up's scalar path (no float4 state rows)."""
+    d = W.mamba2_inputs(906, 2, 30, 4, 8, 2, 5, dtype="f32", conv_bias=True, conv_state=True)
+    _check(M2, d, "f32", [0, 13, 30])
+
+
+@pytest.mark.parametrize("K", [0, 1])
+@pytest.mark.parametrize("shape", ["tensor_core", "simt"])
+def test_mamba2_conv_width_0_and_1(K, shape):
+    """A Mamba-2 split with no conv history to hand on (width 0 or 1): the
+    fix-up stages the raw C (width 0) or its pointwise conv (width 1)."""
+    P, N, dtype = (64, 128, "bf16") if shape == "tensor_core" else (16, 24, "f32")
+    d = W.mamba2_inputs(907 + K, 2, 130, 4, P, 2, N, d_conv=K, dtype=dtype, conv_bias=K > 0, conv_state=False)
+    _check(M2, d, dtype, [0, 13, 70, 130])
+
+
+@pytest.mark.parametrize("mode,shape", [(M1, None), (M2, "tensor_core"), (M2, "simt")])
+def test_rank_with_no_tokens(mode, shape):
+    """Without a conv a rank may hold no tokens: it passes the state through
+    (its pair is (sum of delta 0, zero state)) and writes no y."""
+    if mode == M1:
+        d = W.mamba1_inputs(909, 2, 30, 40, 8, d_conv=0, dtype="f32", with_z=True)
+        dtype = "f32"
+    else:
+        P, N, dtype = (64, 128, "bf16") if shape == "tensor_core" else (16, 24, "f32")
+        d = W.mamba2_inputs(910, 2, 30, 4, P, 2, N, d_conv=0, dtype=dtype, conv_state=False)
+    _check(mode, d, dtype, [0, 13, 13, 30])
