@@ -140,6 +140,7 @@ class Job:
         self.split = None          # set by the sequence-split workloads
         self.bwd = None            # set by the backward workloads
         self.timing_on = False     # kernel timing enabled (the timed region)
+        self.segments = 1          # token segments per row (tensor-core Mamba-2 path)
         if w.kind in ("mamba1", "mamba2", "mamba2_varlen"):
             mode = ssm.MAMBA1 if w.kind == "mamba1" else ssm.MAMBA2
             ww = W.Workload(**{**w.__dict__, "seed": w.seed + seed_shift})
@@ -243,6 +244,13 @@ class Job:
                 self.flops = None
             elif self.ssd:
                 self.kernel, self.sources = "ssd_kernel", ("ssd_m2.cu",)
+                # rows the library cuts into token segments add the state-only pass, which
+                # the kernel timing brackets together with the scan
+                self.segments = ssm.scan_segments(mode, x, t["dt"], t["A"], t["B"], t["C"], z=t["z"],
+                                                  cu_seqlens=t.get("cu_seqlens"), conv_w=t["conv_w"])
+                if self.segments > 1:
+                    self.kernel = "ssd_state_kernel+ssd_kernel"
+                    self.launches_per_step += 1
                 self.mufu = None
                 # tensor-core work of the 64-token chunked form: per (sequence, head, chunk)
                 # C.B^T (2 Q^2 N) + M.X (2 Q^2 P) + C'.S^T (2 Q N P) + B'^T.X (2 Q N P)
@@ -560,7 +568,7 @@ def run_cuda(args):
                    "parallelism": (f"seqsplit{w.split_ranks}: rank {w.split_rank}'s step, exchanges staged in HBM"
                                    if w.split_ranks else (f"replicas{world}" if world > 1 else "single")),
                    "l2": "flushed between timed steps (256 MiB write, outside the events)",
-                   "tokens_per_step": job.units},
+                   "tokens_per_step": job.units, "token_segments_per_row": job.segments},
         "hbm_gbs": gbs, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         "gpu_launches": job.launches_per_step * args.steps, "impl": "cuda",
         "step_ms": {"min": min(step_ms), "median": float(np.median(step_ms)), "max": max(step_ms)},

@@ -74,7 +74,7 @@
 extern "C" {
 #endif
 
-#define SSM_ABI_VERSION 1
+#define SSM_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define SSM_API __attribute__((visibility("default")))
@@ -173,6 +173,16 @@ typedef struct ssm_scan_args {
     int64_t inter_nslots;         /* pool rows (>= 0) */
     float *inter_states;          /* [inter_nslots][state size] fp32, rows laid out as h_final's; may be NULL */
     void *inter_conv;             /* [inter_nslots][conv_dim][K-1] in dtype; may be NULL */
+    /* Token segments of the Mamba-2 tensor-core path (rows without
+     * cu_seqlens; ignored elsewhere): 0 lets the library choose, 1 keeps one
+     * CTA per (row, head), n >= 2 cuts every row into about n runs of whole
+     * 64-token chunks that separate CTAs scan at the same time.  Each run's
+     * entering state comes from a state-only pass over the runs before it (the
+     * pair (exp(delta A), h) composes associatively, seed (1, h0): "Adding
+     * Initial Value Support to Selective Scan Forward Kernel"), so results
+     * agree with the unsegmented scan up to fp32 rounding.  The workspace size
+     * depends on it. */
+    int64_t segments;
 } ssm_scan_args;
 
 /* ---------------------------------------------------------------- decode */
@@ -236,8 +246,14 @@ SSM_API int32_t ssm_last_cuda_error(void);
 SSM_API ssm_status ssm_conv1d_fwd(const ssm_conv_args *args, void *stream);
 
 /* Bytes of device workspace ssm_scan_fwd needs for these arguments (0 when
- * none is needed; the packed varlen path needs one).  Does not touch the GPU. */
+ * none is needed; the packed varlen path needs one).  Launches nothing; it
+ * reads the current device's SM count (148 when no device answers), which
+ * the choice of token segments depends on. */
 SSM_API size_t ssm_scan_workspace_size(const ssm_scan_args *args);
+/* Token segments ssm_scan_fwd cuts every row into for these arguments: 1 when
+ * rows stay whole (packed sequences, Mamba-1, the SIMT Mamba-2 path, rows of
+ * one chunk), 0 for arguments ssm_scan_fwd would reject.  Launches nothing. */
+SSM_API int64_t ssm_scan_segments(const ssm_scan_args *args);
 
 /* Forward scan.  `workspace` (device, 256-byte aligned, ws_bytes long) may be
  * NULL when ssm_scan_workspace_size() is 0.  The workspace holds the device

@@ -6,6 +6,6 @@ library is loaded on first use and a missing library raises immediately:
 there is no CPU fallback.
 """
 from .ops import (MAMBA1, MAMBA2, conv1d_fwd, kernel_time_ms, kernel_timing, scan_bwd, scan_fwd,  # noqa: F401
-                  scan_workspace_size, state_update, workspace_error)
+                  scan_segments, scan_workspace_size, state_update, workspace_error)
 from ._abi import LIB_PATH, SSMError  # noqa: F401
 from .seq_split import SegmentScan, scan_fwd_seq_split  # noqa: F401

@@ -15,6 +15,7 @@ LIB_PATH = os.path.join(_HERE, "libssm.so")
 SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_ALIGNMENT = 0, -1, -2, -3
 SSM_ERR_WORKSPACE, SSM_ERR_CUDA, SSM_ERR_DEVICE = -4, -5, -6
 SSM_F32, SSM_BF16 = 0, 1
+ABI_VERSION = 2                # SSM_ABI_VERSION of the header this mirror follows
 SSM_MAMBA1, SSM_MAMBA2 = 1, 2
 SSM_DEVERR_NONE, SSM_DEVERR_CU_SEQLENS, SSM_DEVERR_TIMEOUT, SSM_DEVERR_BOUNDS = 0, 1, 2, 3
 
@@ -52,6 +53,7 @@ class ScanArgs(C.Structure):
         ("chunk", _i64),
         ("state_interval", _i64), ("inter_slots", _vp), ("inter_stride", _i64), ("inter_nslots", _i64),
         ("inter_states", _vp), ("inter_conv", _vp),
+        ("segments", _i64),
     ]
 
 
@@ -100,6 +102,7 @@ SIGNATURES = {
     "ssm_last_cuda_error": ([], _i32),
     "ssm_conv1d_fwd": ([C.POINTER(ConvArgs), _vp], _i32),
     "ssm_scan_workspace_size": ([C.POINTER(ScanArgs)], C.c_size_t),
+    "ssm_scan_segments": ([C.POINTER(ScanArgs)], _i64),
     "ssm_scan_fwd": ([C.POINTER(ScanArgs), _vp, C.c_size_t, _vp], _i32),
     "ssm_state_update": ([C.POINTER(UpdateArgs), _vp], _i32),
     "ssm_workspace_error": ([_vp, C.POINTER(_i32), _vp], _i32),
@@ -134,7 +137,7 @@ def lib() -> C.CDLL:
                     fn = getattr(handle, name)
                     fn.argtypes = argtypes
                     fn.restype = restype
-                if handle.ssm_abi_version() != 1:
+                if handle.ssm_abi_version() != ABI_VERSION:
                     raise RuntimeError("libssm.so ABI version mismatch")
                 _lib = handle
     return _lib

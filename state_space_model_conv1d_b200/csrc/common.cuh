@@ -82,7 +82,7 @@ enum BoundsSite {
     BS_M2S_SEQ, BS_M2S_HEAD, BS_M2S_STATE,
     BS_DEC_ROW, BS_DEC_SLOT, BS_DEC_CHANNEL,
     BS_CONV_TOKEN, BS_CONV_CHANNEL, BS_CONV_STATE,
-    BS_BWD_SEQ, BS_BWD_CHANNEL, BS_SPLIT_ROW, BS_SPLIT_CHANNEL,
+    BS_BWD_SEQ, BS_BWD_CHANNEL, BS_SPLIT_ROW, BS_SPLIT_CHANNEL, BS_SSD_SEGMENT,
 };
 #ifdef SSM_CHECK_BOUNDS
 struct BoundsRecord {

@@ -79,6 +79,7 @@ cudaError_t launch_scan_m2_simt(const ssm_scan_args &a, const SeqView &sv, cudaS
 bool ssd_shape_ok(const ssm_scan_args &a);      // shapes only: decides the workspace size
 bool ssd_supported(const ssm_scan_args &a);     // shapes and 16-byte alignment: decides the kernel
 size_t ssd_workspace_bytes(const ssm_scan_args &a);
+int ssd_segments(const ssm_scan_args &a);       // token segments per row (1 = rows stay whole)
 cudaError_t launch_ssd(const ssm_scan_args &a, const SeqView &sv, void *ws_bc, cudaStream_t st);
 cudaError_t launch_state_update(const ssm_update_args &a, cudaStream_t st);
 // Backward scan: workspace bytes for the checkpoints and B / C accumulators
@@ -100,6 +101,9 @@ constexpr int64_t kMaxSplitSeqlen = 65535LL * 16;
 // unless enabled; otherwise records one event before and one after on `st`.
 void timing_begin(cudaStream_t st);
 void timing_end(cudaStream_t st);
+
+// SM count of the current device (148 when none answers).
+int sm_count();
 
 // Largest dstate each path supports.
 constexpr int64_t kMaxDstateM1 = 64;

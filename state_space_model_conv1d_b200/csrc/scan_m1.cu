@@ -901,17 +901,6 @@ cudaError_t launch_tp(M1Args a, int nseqs, cudaStream_t st) {
 }
 
 
-// SM count of the current device (queried once per device).
-int sm_count() {
-    static int counts[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (counts[dev] == 0) {
-        int n = 0;
-        counts[dev] = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0 ? n : 148;
-    }
-    return counts[dev];
-}
 
 inline bool vec_ok(const void *p, int64_t bs, int64_t ts, size_t es) {
     return p == nullptr || ((uintptr_t)p % 16 == 0 && (bs * (int64_t)es) % 16 == 0 && (ts * (int64_t)es) % 16 == 0);
@@ -954,6 +943,19 @@ cudaError_t launch_scan_m1(const ssm_scan_args &s, const SeqView &sv, cudaStream
     if (tp_supported(a) && seq_warps < 7 * (int64_t)sm_count())
         return s.dtype == SSM_BF16 ? launch_tp<__nv_bfloat16>(a, nseqs, st) : launch_tp<float>(a, nseqs, st);
     return s.dtype == SSM_BF16 ? launch_typed<__nv_bfloat16>(a, nseqs, st) : launch_typed<float>(a, nseqs, st);
+}
+
+// SM count of the current device (queried once per device; 148 when there is
+// no device to ask, so host-only callers still get a deterministic answer).
+int sm_count() {
+    static int counts[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (counts[dev] == 0) {
+        int n = 0;
+        counts[dev] = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0 ? n : 148;
+    }
+    return counts[dev];
 }
 
 }  // namespace ssm

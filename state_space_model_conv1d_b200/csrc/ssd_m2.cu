@@ -51,6 +51,7 @@
 // abort flag that ends every other wait, and the CTA drains its in-flight
 // copies and MMAs before it frees tensor memory and returns.
 #include <stddef.h>
+#include <cmath>
 #include <string.h>
 
 #include <type_traits>
@@ -132,6 +133,13 @@ struct SsdArgs {
     InterView iv;
     const __nv_bfloat16 *Braw, *Craw;   // the unconvolved B / C (intermediate conv history)
     int64_t braw_bs, braw_ts, craw_bs, craw_ts;
+    // Segments (fixed-length batches only; nseg = 1 otherwise): row s is cut into
+    // nseg runs of seg_len tokens (whole chunks; the last one takes the rest).
+    // sloc / slog hold, for every segment but the last, the state it leaves when
+    // scanned from zero and its total log2-decay ([s][sg][H] rows of P x N, [s][sg][H]).
+    int nseg;
+    int64_t seg_len;
+    float *sloc, *slog;
 };
 
 SSM_DEVINL void st16(void *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
@@ -147,19 +155,33 @@ SSM_DEVINL void mb_arrive(uint64_t *mbar) {
 // error word.
 constexpr uint32_t kSleepHintNs = 100000;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-SSM_DEVINL bool wait_mb(Aux &ax, int i, uint32_t parity, int32_t *err) {
-    if (tc::mbar_try_wait_sleep(&ax.mb[i], parity, kSleepHintNs)) return true;
+SSM_DEVINL bool wait_bar(uint64_t *mb, int *abort, uint32_t parity, int32_t *err) {
+    if (tc::mbar_try_wait_sleep(mb, parity, kSleepHintNs)) return true;
     const uint64_t t0 = tc::globaltimer_ns();
     for (;;) {
-        if (*reinterpret_cast<volatile int *>(&ax.abort)) return false;
-        if (tc::mbar_try_wait_sleep(&ax.mb[i], parity, kSleepHintNs)) return true;
+        if (*reinterpret_cast<volatile int *>(abort)) return false;
+        if (tc::mbar_try_wait_sleep(mb, parity, kSleepHintNs)) return true;
         if (tc::globaltimer_ns() - t0 > kWaitLimitNs) break;
     }
-    *reinterpret_cast<volatile int *>(&ax.abort) = 1;
+    *reinterpret_cast<volatile int *>(abort) = 1;
     if (err) atomicExch(err, SSM_DEVERR_TIMEOUT);
     return false;
 }
+SSM_DEVINL bool wait_mb(Aux &ax, int i, uint32_t parity, int32_t *err) { return wait_bar(&ax.mb[i], &ax.abort, parity, err); }
 SSM_DEVINL bool aborted(Aux &ax) { return *reinterpret_cast<volatile int *>(&ax.abort) != 0; }
+
+// Causal width-<=4 conv of one channel pair at one token plus SiLU: taps
+// right-aligned (w3 multiplies the current token, w0 the one three back);
+// silu(v) = h + h tanh(h), h = v / 2.
+SSM_DEVINL float2 conv_silu2(float2 cur, float2 h2, float2 h1, float2 h0, float2 w3, float2 w2, float2 w1, float2 w0,
+                             float2 bias) {
+    float2 acc = __ffma2_rn(w3, cur, bias);
+    acc = __ffma2_rn(w2, h2, acc);
+    acc = __ffma2_rn(w1, h1, acc);
+    acc = __ffma2_rn(w0, h0, acc);
+    const float2 hv = __fmul2_rn(acc, make_float2(0.5f, 0.5f));
+    return __ffma2_rn(hv, make_float2(tanh_approx(hv.x), tanh_approx(hv.y)), hv);
+}
 
 // Tensor maps (3-d: channel, token, batch row; bf16):
 //   tm_x  raw x, box 64 x 64 rows, no swizzle    -> row-major staging rows of 128 bytes
@@ -177,13 +199,21 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int hh = blockIdx.x;
-    const int s = a.sv.order ? a.sv.order[blockIdx.y] : (int)blockIdx.y;
-    int64_t start = 0, len = a.seqlen, row = s;
+    // sequence s, segment sg of it (packed sequences and plain rows without
+    // segments: sg = 0 and the segment is the whole sequence)
+    const int s = a.sv.order ? a.sv.order[blockIdx.y] : (int)blockIdx.y / a.nseg;
+    const int sg = a.sv.order ? 0 : (int)blockIdx.y % a.nseg;
+    int64_t seq_start = 0, seq_len = a.seqlen, row = s;
     if (a.sv.cu) {
         const int64_t c0 = min(max((int64_t)a.sv.cu[s], (int64_t)0), a.seqlen);
         const int64_t c1 = min(max((int64_t)a.sv.cu[s + 1], c0), a.seqlen);
-        start = c0; len = c1 - c0; row = 0;
+        seq_start = c0; seq_len = c1 - c0; row = 0;
     }
+    const int64_t start = seq_start + (int64_t)sg * a.seg_len;
+    const int64_t len = max(min(a.seg_len, seq_len - (int64_t)sg * a.seg_len), (int64_t)0);
+    // tokens of the sequence before the segment, recomputed where needed (keeps
+    // it out of the registers the chunk loop holds)
+    auto seg_off = [&]() -> int64_t { return a.sv.order ? 0 : (int64_t)((int)blockIdx.y % a.nseg) * a.seg_len; };
     const int64_t H = a.H, g = hh / (H / a.G);
     const int K = a.K;
     const int n = (int)((len + kQ - 1) / kQ);
@@ -194,7 +224,8 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
         !SSM_BOUNDS((int64_t)hh * kP + kP - 1, a.H * kP, BS_SSD_HEAD) ||
         !SSM_BOUNDS((int64_t)g0 + kN - 1, a.G * kN, BS_SSD_GROUP) ||
         !SSM_BOUNDS((int64_t)s * H + hh, (int64_t)a.sv.nseqs * H, BS_SSD_STATE) ||
-        !SSM_BOUNDS(((int64_t)s + 1) * a.cdim - 1, (int64_t)a.sv.nseqs * a.cdim, BS_SSD_CONV_STATE))
+        !SSM_BOUNDS(((int64_t)s + 1) * a.cdim - 1, (int64_t)a.sv.nseqs * a.cdim, BS_SSD_CONV_STATE) ||
+        !SSM_BOUNDS(sg, a.nseg, BS_SSD_SEGMENT))
         return;
     const float A2 = a.A[hh] * kLog2e;
 
@@ -448,18 +479,33 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
             for (int p = 0; p < 16; ++p)
                 S[p] = h0p ? make_float2(h0p[(int64_t)(half * 32 + 2 * p) * kN + sn], h0p[(int64_t)(half * 32 + 2 * p + 1) * kN + sn])
                            : make_float2(0.f, 0.f);
+            // the state entering segment sg: fold (exp(cs_end), S_loc) of every
+            // segment before it onto h0, in order
+            for (int t = 0; t < sg; ++t) {
+                const int64_t q = ((int64_t)s * (a.nseg - 1) + t) * H + hh;
+                const float e = ex2(a.slog[q]);
+                const float2 e2 = make_float2(e, e);
+                const float *lp = a.sloc + q * kP * kN;
+#pragma unroll
+                for (int p = 0; p < 16; ++p)
+                    S[p] = __ffma2_rn(e2, S[p], make_float2(lp[(int64_t)(half * 32 + 2 * p) * kN + sn],
+                                                            lp[(int64_t)(half * 32 + 2 * p + 1) * kN + sn]));
+            }
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 st16(smem + OFF_S + tc::off_sw128(sn, half * 32 + q * 8, 8192), tc::pack_bf16x8(reinterpret_cast<const float *>(&S[q * 4])));
         }
-        // conv halo of chunk 0 (the last K-1 raw inputs before the sequence)
+        // conv halo of chunk 0: the last K-1 raw inputs before the sequence (its
+        // carried conv state), or the raw x rows before a later segment
         if (tid < kP) {
             const int p = tid;
 #pragma unroll
             for (int j = 0; j < kHx; ++j) {
                 const int q = j - (kHx - (K - 1));          // index into the carried conv state
                 float v = 0.f;
-                if (K > 1 && q >= 0 && a.conv_state_in)
+                if (sg > 0)
+                    v = __bfloat162float(a.x[row * a.x_bs + (start - kHx + j) * a.x_ts + hh * kP + p]);
+                else if (K > 1 && q >= 0 && a.conv_state_in)
                     v = __bfloat162float(a.conv_state_in[((int64_t)s * a.cdim + hh * kP + p) * (K - 1) + q]);
                 ax.xh[0][j][p] = v;
             }
@@ -503,7 +549,6 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                 } else {
                     h0v = rawrow(cr0 - 3); h1v = rawrow(cr0 - 2); h2v = rawrow(cr0 - 1);
                 }
-                const float2 half2 = make_float2(0.5f, 0.5f);
                 float wv[8];                                            // X' weights of the 8 tokens
                 {
                     const float4 w0 = *reinterpret_cast<const float4 *>(&tb.wj[cr0]);
@@ -518,15 +563,7 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                     for (int i = 0; i < kQ / 8; ++i) {
                         const float2 cur = rawrow(cr0 + i);             // rows >= nv are zeroed below
                         float2 xc = cur;
-                        if (K > 0) {
-                            float2 acc = __ffma2_rn(cw3, cur, cbias);
-                            acc = __ffma2_rn(cw2, h2v, acc);
-                            acc = __ffma2_rn(cw1, h1v, acc);
-                            acc = __ffma2_rn(cw0, h0v, acc);
-                            // silu(v) = h + h tanh(h), h = v / 2
-                            const float2 hv = __fmul2_rn(acc, half2);
-                            xc = __ffma2_rn(hv, make_float2(tanh_approx(hv.x), tanh_approx(hv.y)), hv);
-                        }
+                        if (K > 0) xc = conv_silu2(cur, h2v, h1v, h0v, cw3, cw2, cw1, cw0, cbias);
                         if (!kFull && cr0 + i >= nv) xc = make_float2(0.f, 0.f);
                         h0v = h1v; h1v = h2v; h2v = cur;
                         const float2 xw = __fmul2_rn(xc, make_float2(wv[i], wv[i]));
@@ -637,7 +674,7 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                 if (lane == 0) mb_arrive(&ax.mb[MB_SREADY]);
                 // intermediate state after this chunk when it closes a state interval
                 if (a.iv.interval > 0 && nv == kQ && !aborted(ax)) {
-                    const int64_t slot = a.iv.slot_after(s, t0 + kQ);
+                    const int64_t slot = a.iv.slot_after(s, seg_off() + t0 + kQ);
                     if (slot >= 0 && SSM_BOUNDS(slot, a.iv.nslots, BS_SSD_POOL)) {
                         if (a.iv.states) {
                             float *dst = a.iv.states + (slot * H + hh) * kP * kN;
@@ -739,7 +776,7 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
             }
         }
         if (tid == 0) tc::bulk_wait_all();
-        if (!aborted(ax)) {
+        if (!aborted(ax) && (a.sv.order || (int)blockIdx.y % a.nseg == a.nseg - 1)) {   // the last segment
             if (a.h_final) {
                 float *hf = a.h_final + ((int64_t)s * H + hh) * kP * kN;
 #pragma unroll
@@ -767,11 +804,12 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                 __nv_bfloat16 v[kHx];
 #pragma unroll
                 for (int j = 0; j < kHx; ++j) {
-                    const int64_t tau = len - (K - 1) + j;           // within the sequence
+                    const int64_t tau = seg_off() + len - (K - 1) + j;  // within the sequence
                     v[j] = __float2bfloat16_rn(0.f);
                     if (j < K - 1) {
                         if (tau >= 0) {
-                            if (SSM_BOUNDS(start + tau, a.seqlen, BS_SSD_RAW_BC)) v[j] = raw[(start + tau) * rts];
+                            const int64_t tok = start - seg_off() + tau;
+                            if (SSM_BOUNDS(tok, a.seqlen, BS_SSD_RAW_BC)) v[j] = raw[tok * rts];
                         }
                         else if (a.conv_state_in) v[j] = a.conv_state_in[((int64_t)s * a.cdim + ch) * (K - 1) + tau + (K - 1)];
                     }
@@ -787,6 +825,278 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
     __syncthreads();
     tc::fence_after_sync();
     if (warp == kComputeWarps) tc::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ segment states
+// A fixed-length batch with fewer (row, head) chains than the GPU holds CTAs
+// is cut along its tokens: every row into nseg segments of whole chunks, one
+// scan CTA per (segment, head).  The scan CTA of segment sg needs the state
+// that enters it; the pair (exp(cs), S) of a segment composes associatively
+// with seed (1, h0) ("Adding Initial Value Support to Selective Scan Forward
+// Kernel", state-spaces/mamba issue 285), so this pass scans every segment but
+// the last from a zero state and leaves
+//   S_loc[p, n] = sum_j exp(cs_end - cs_j) delta_j X_j[p] B_j[n]
+//   slog        = cs_end            (log2 units, cs over the segment's tokens)
+// and the scan CTA folds h_in = exp(slog) h_in + S_loc over the segments before
+// its own, starting from h0 (the ssd_chunk_state -> ssd_state_passing order of
+// "Clean up SSM ops directory structure").  S_loc is one tensor-core
+// accumulation over the segment: A = B^T (MN-major, M = 128 states), B = X'
+// (MN-major, N = 64), K = the segment's tokens, X' = exp(cs_end - cs_j)
+// delta_j X_j written by the fused x conv.
+//
+// Warp roles as in the scan kernel.  Before the chunk loop the compute warps
+// sum delta A over every half chunk, then (after suffix sums over the chunks)
+// write every token's X' weight into a shared table, so the loop itself reads
+// no dt.  In the loop the control warp's lane 0 keeps three chunks of B and
+// raw x in flight (TMA) and issues chunk c's four MMAs once the eight compute
+// warps have written its X' (one of two buffers); the compute warps run the
+// conv + SiLU + weight of chunk c as soon as its tiles have landed and the
+// MMAs of chunk c - 2 have released the buffer.  The last conv warp hands the
+// chunk's final raw rows (its rolling registers) to warp 0 as the next chunk's
+// conv halo.  All waits are bounded as in the scan kernel.
+constexpr int kStStages = 3;
+constexpr int kMaxSegChunks = 64;
+constexpr uint32_t ST_STAGE = 24576;                   // per stage: B tile (two 8 KB K-atoms), raw x rows (8 KB)
+constexpr uint32_t ST_OFF_XP = kStStages * ST_STAGE;   // two X' buffers of 8 KB
+constexpr uint32_t ST_OFF_W = ST_OFF_XP + 16384;       // fp32 X' weight of every token of the segment
+constexpr uint32_t ST_OFF_AUX = ST_OFF_W + kMaxSegChunks * kQ * 4;
+enum { SB_LD0 = 0, SB_MMA0 = kStStages, SB_CONV0 = kStStages + 2, SB_DRAIN = kStStages + 4, kNumStBar };
+struct StAux {
+    float xh[3][kHx][kP];                // conv halo of chunk c in slot c % 3
+    float half[2 * kMaxSegChunks];       // sum of delta A (log2) over each half chunk
+    float suf[kMaxSegChunks + 1];        // suf[c]: sum over chunks c .. n-1
+    uint32_t tmem;
+    int abort;
+    uint64_t mb[kNumStBar];
+};
+constexpr size_t kStSmemBytes = ST_OFF_AUX + sizeof(StAux) + 1024;
+
+__global__ void __launch_bounds__(kThreads, 2)
+ssd_state_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+    StAux &ax = *reinterpret_cast<StAux *>(smem + ST_OFF_AUX);
+    float *wt = reinterpret_cast<float *>(smem + ST_OFF_W);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int hh = blockIdx.x;
+    const int nsp = a.nseg - 1;                           // segments that have a successor
+    const int s = (int)blockIdx.y / nsp, sg = (int)blockIdx.y % nsp;
+    const int64_t start = (int64_t)sg * a.seg_len, row = s;
+    const int n = (int)(a.seg_len / kQ);                  // only whole segments come here
+    const int64_t H = a.H, g = hh / (H / a.G);
+    const int crow = (int)row, g0 = (int)(g * kN), K = a.K;
+    const int64_t q = ((int64_t)s * nsp + sg) * H + hh;   // row of sloc / slog
+    if (!SSM_BOUNDS(start + a.seg_len - 1, a.seqlen, BS_SSD_SEQ) || !SSM_BOUNDS(n - 1, kMaxSegChunks, BS_SSD_SEGMENT) ||
+        !SSM_BOUNDS((int64_t)hh * kP + kP - 1, a.H * kP, BS_SSD_HEAD) ||
+        !SSM_BOUNDS((int64_t)g0 + kN - 1, a.G * kN, BS_SSD_GROUP) ||
+        !SSM_BOUNDS(q, (int64_t)a.sv.nseqs * nsp * H, BS_SSD_STATE))
+        return;
+    const float A2 = a.A[hh] * kLog2e;
+    const float dtb = a.dt_bias ? a.dt_bias[hh] : 0.f;
+    const __nv_bfloat16 *dtg = a.dt + row * a.dt_bs + start * a.dt_ts + hh;
+    // delta of token t (lane l of half chunk hc: t = 32 hc + l) and its inclusive
+    // prefix of delta A over the half chunk
+    auto half_scan = [&](int hc, float &d, float &sc) {
+        const float u = __bfloat162float(dtg[((int64_t)hc * 32 + lane) * a.dt_ts]) + dtb;
+        d = a.softplus ? softplus(u) : u;
+        sc = d * A2;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float v = __shfl_up_sync(0xffffffffu, sc, o);
+            if (lane >= o) sc += v;
+        }
+    };
+
+    if (tid == 0) {
+        ax.abort = (a.err && *a.err != 0) ? 1 : 0;
+        for (int i = 0; i < kNumStBar; ++i)
+            tc::mbar_init(&ax.mb[i], (i == SB_CONV0 || i == SB_CONV0 + 1) ? kComputeWarps : 1);
+        tc::mbar_init_fence();
+        tc::prefetch_map(&tm_x);
+        tc::prefetch_map(&tm_b);
+    }
+    if (warp == kComputeWarps) {
+        tc::tmem_alloc(&ax.tmem, 64);
+    } else {
+        for (int hc = warp; hc < 2 * n; hc += kComputeWarps) {
+            float d, sc;
+            half_scan(hc, d, sc);
+            if (lane == 31) ax.half[hc] = sc;
+        }
+        // conv halo of chunk 0: the row's carried conv state before its first
+        // segment, else the raw x rows before the segment
+        if (tid < kP) {
+            const int p = tid;
+#pragma unroll
+            for (int j = 0; j < kHx; ++j) {
+                const int qq = j - (kHx - (K - 1));
+                float v = 0.f;
+                if (sg > 0)
+                    v = __bfloat162float(a.x[row * a.x_bs + (start - kHx + j) * a.x_ts + hh * kP + p]);
+                else if (K > 1 && qq >= 0 && a.conv_state_in)
+                    v = __bfloat162float(a.conv_state_in[((int64_t)s * a.cdim + hh * kP + p) * (K - 1) + qq]);
+                ax.xh[0][j][p] = v;
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = ax.tmem;
+    if (ax.abort) {
+        __syncthreads();
+        if (warp == kComputeWarps) tc::tmem_dealloc(tmem, 64);
+        return;
+    }
+    if (tid == 0) {
+        ax.suf[n] = 0.f;
+        for (int c = n - 1; c >= 0; --c) ax.suf[c] = (ax.half[2 * c] + ax.half[2 * c + 1]) + ax.suf[c + 1];
+    }
+    __syncthreads();
+    if (warp < kComputeWarps) {
+        // X' weight of every token: the decay left in its chunk after it, then
+        // that of the later chunks, times its delta
+        for (int hc = warp; hc < 2 * n; hc += kComputeWarps) {
+            const int c = hc >> 1;
+            float d, sc;
+            half_scan(hc, d, sc);
+            const float pre = (hc & 1) ? ax.half[hc - 1] : 0.f;
+            const float tot = ax.half[2 * c] + ax.half[2 * c + 1];
+            wt[hc * 32 + lane] = ex2((tot - (pre + sc)) + ax.suf[c + 1]) * d;
+        }
+    }
+    __syncthreads();
+
+    const uint32_t sbase = tc::smem_u32(smem);
+    if (warp == kComputeWarps) {
+        // ------------------------------------------------------------ control warp
+        if (lane == 0) {
+            int last_ld[kStStages] = {-1, -1, -1};
+            auto load = [&](int c) {
+                const int st = c % kStStages;
+                unsigned char *base = smem + st * ST_STAGE;
+                const int tok = (int)(start + (int64_t)c * kQ);
+                tc::mbar_expect_tx(&ax.mb[SB_LD0 + st], 2 * kQ * 64 * 2 + kQ * kP * 2);
+                tc::tma_load_3d(base, &tm_b, g0, tok, crow, &ax.mb[SB_LD0 + st]);
+                tc::tma_load_3d(base + 8192, &tm_b, g0 + 64, tok, crow, &ax.mb[SB_LD0 + st]);
+                tc::tma_load_3d(base + 16384, &tm_x, (int)(hh * kP), tok, crow, &ax.mb[SB_LD0 + st]);
+                last_ld[st] = c;
+            };
+            for (int c = 0; c < kStStages && c < n; ++c) load(c);
+            for (int c = 0; c < n; ++c) {
+                const int st = c % kStStages, xb = c & 1;
+                if (!wait_bar(&ax.mb[SB_CONV0 + xb], &ax.abort, (c >> 1) & 1, a.err)) break;
+                tc::fence_after_sync();
+                const uint64_t dBm = tc::desc_sw128(sbase + st * ST_STAGE, 8192, 1024);          // MN-major B^T
+                const uint64_t dXm = tc::desc_sw128(sbase + ST_OFF_XP + xb * 8192, 8192, 1024);  // MN-major X'
+#pragma unroll
+                for (int kk = 0; kk < kQ / 16; ++kk)
+                    tc::mma_bf16(tmem, dBm + kk * 128, dXm + kk * 128, ID_S, (c > 0 || kk > 0) ? 1u : 0u);
+                tc::mma_commit(&ax.mb[SB_MMA0 + xb]);
+                // the stage of chunk c takes chunk c + 3 once MMA(c) has read its B
+                // (every conv warp has read its raw x: conv(c) is complete)
+                if (c + kStStages < n) {
+                    if (!wait_bar(&ax.mb[SB_MMA0 + xb], &ax.abort, (c >> 1) & 1, a.err)) break;
+                    load(c + kStStages);
+                }
+            }
+            if (*reinterpret_cast<volatile int *>(&ax.abort)) {
+                // drain: every MMA issued, and the last copy into each stage
+                tc::mma_commit(&ax.mb[SB_DRAIN]);
+                tc::mbar_wait(&ax.mb[SB_DRAIN], 0, 1u << 22);
+                for (int b = 0; b < kStStages; ++b)
+                    if (last_ld[b] >= 0) tc::mbar_wait(&ax.mb[SB_LD0 + b], (last_ld[b] / kStStages) & 1, 1u << 22);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ compute warps
+        // x conv as in the scan kernel: channels 2 lane, 2 lane + 1; tokens 8 warp .. 8 warp + 7
+        const int cq = lane, cr0 = warp * (kQ / 8);
+        float2 cw0, cw1, cw2, cw3, cbias;
+        {
+            const int64_t ch = hh * kP + 2 * cq;
+            auto tap = [&](int j) {
+                const int k = K - 4 + j;
+                return (K > 0 && k >= 0) ? make_float2(a.conv_w[ch * K + k], a.conv_w[(ch + 1) * K + k])
+                                         : make_float2(0.f, 0.f);
+            };
+            cw0 = tap(0); cw1 = tap(1); cw2 = tap(2); cw3 = tap(3);
+            cbias = a.conv_b ? make_float2(a.conv_b[ch], a.conv_b[ch + 1]) : make_float2(0.f, 0.f);
+        }
+        const uint32_t obase = (uint32_t)warp * 1024u + (uint32_t)(cq & 3) * 4u;
+        bool ok = true;
+        for (int c = 0; c < n; ++c) {
+            const int st = c % kStStages, xb = c & 1;
+            ok = wait_bar(&ax.mb[SB_LD0 + st], &ax.abort, (c / kStStages) & 1, a.err) && ok;
+            if (c >= 2) ok = wait_bar(&ax.mb[SB_MMA0 + xb], &ax.abort, ((c - 2) >> 1) & 1, a.err) && ok;   // X' free
+            // warp 0 reads the halo the last conv warp left with conv(c - 1)
+            if (warp == 0 && c > 0) ok = wait_bar(&ax.mb[SB_CONV0 + ((c - 1) & 1)], &ax.abort, ((c - 1) >> 1) & 1, a.err) && ok;
+            float wv[8];
+            {
+                const float4 w0 = *reinterpret_cast<const float4 *>(&wt[c * kQ + cr0]);
+                const float4 w1 = *reinterpret_cast<const float4 *>(&wt[c * kQ + cr0 + 4]);
+                wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
+                wv[4] = w1.x; wv[5] = w1.y; wv[6] = w1.z; wv[7] = w1.w;
+            }
+            const unsigned char *xraw = smem + st * ST_STAGE + 16384;
+            unsigned char *xpo = smem + ST_OFF_XP + xb * 8192;
+            auto rawrow = [&](int v) -> float2 {
+                const uint32_t u = *reinterpret_cast<const uint32_t *>(xraw + v * (kP * 2) + cq * 4);
+                return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+            };
+            float2 h0v, h1v, h2v;
+            if (warp == 0) {
+                const int hs = c % 3;
+                h0v = *reinterpret_cast<const float2 *>(&ax.xh[hs][0][2 * cq]);
+                h1v = *reinterpret_cast<const float2 *>(&ax.xh[hs][1][2 * cq]);
+                h2v = *reinterpret_cast<const float2 *>(&ax.xh[hs][2][2 * cq]);
+            } else {
+                h0v = rawrow(cr0 - 3); h1v = rawrow(cr0 - 2); h2v = rawrow(cr0 - 1);
+            }
+#pragma unroll
+            for (int i = 0; i < kQ / 8; ++i) {
+                const float2 cur = rawrow(cr0 + i);
+                const float2 xc = K > 0 ? conv_silu2(cur, h2v, h1v, h0v, cw3, cw2, cw1, cw0, cbias) : cur;
+                h0v = h1v; h1v = h2v; h2v = cur;
+                const float2 xw = __fmul2_rn(xc, make_float2(wv[i], wv[i]));
+                const uint32_t off = obase + (uint32_t)i * 128u + ((uint32_t)((cq >> 2) ^ i) << 4);
+                *reinterpret_cast<__nv_bfloat162 *>(xpo + off) = __floats2bfloat162_rn(xw.x, xw.y);
+            }
+            if (warp == kComputeWarps - 1) {
+                // the chunk's last three raw rows: the halo of chunk c + 1
+                const int hs = (c + 1) % 3;
+                *reinterpret_cast<float2 *>(&ax.xh[hs][0][2 * cq]) = h0v;
+                *reinterpret_cast<float2 *>(&ax.xh[hs][1][2 * cq]) = h1v;
+                *reinterpret_cast<float2 *>(&ax.xh[hs][2][2 * cq]) = h2v;
+            }
+            tc::fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mb_arrive(&ax.mb[SB_CONV0 + xb]);
+        }
+        // the last accumulation
+        ok = wait_bar(&ax.mb[SB_MMA0 + ((n - 1) & 1)], &ax.abort, ((n - 1) >> 1) & 1, a.err) && ok;
+        (void)ok;
+    }
+    // No wait follows this barrier, so the abort flag (raised by any failed
+    // wait) reads the same in every thread and the warp-wide loads stay converged.
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp < kComputeWarps && !*reinterpret_cast<volatile int *>(&ax.abort)) {
+        const int q4 = warp & 3, hf = warp >> 2;
+        float v[32];
+        tc::tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + hf * 32, v);
+        float *dst = a.sloc + q * kP * kN;
+        const int nn = q4 * 32 + lane;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dst[(int64_t)(hf * 32 + i) * kN + nn] = v[i];
+        if (tid == 0) a.slog[q] = ax.suf[0];
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == kComputeWarps) tc::tmem_dealloc(tmem, 64);
 }
 
 // ------------------------------------------------------------------ B / C pre-pass
@@ -943,10 +1253,65 @@ bool ssd_supported(const ssm_scan_args &s) {
            st16ok(s.C_batch_stride);
 }
 
+namespace {
+inline size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+// Segments of a fixed-length batch.  Requested (segments >= 2): about that
+// many runs of whole chunks, at most kMaxSegChunks chunks per run.  Chosen
+// (segments = 0): the count that minimises a model of the two launches in
+// units of one chunk of one scan CTA, two CTAs per SM for both kernels, fitted
+// to B200 timings of 4 x 4096 tokens x 80 heads at 1 to 8 segments:
+//   scan   waves x (chunks per run + 1 + 0.15 (nseg - 1))  (pipeline fill, fold)
+//   state  waves x (0.45 chunks per run + 2.5)               (prologue)
+// A candidate must beat the whole-row plan by 3%.
+struct SegPlan {
+    int nseg;
+    int64_t seg_len;
+};
+SegPlan plan_segments(const ssm_scan_args &s) {
+    SegPlan one{1, s.seqlen};
+    if (s.cu_seqlens || s.batch <= 0 || s.seqlen <= kQ || s.segments == 1) return one;
+    const int64_t nch = (s.seqlen + kQ - 1) / kQ;
+    auto make = [&](int64_t k) {
+        int64_t per = (nch + k - 1) / k;
+        if (per > kMaxSegChunks) per = kMaxSegChunks;
+        return SegPlan{(int)((nch + per - 1) / per), per * kQ};
+    };
+    auto fits = [&](const SegPlan &p) { return p.nseg >= 2 && s.batch * p.nseg <= 65535; };
+    if (s.segments >= 2) {
+        const SegPlan p = make(s.segments < nch ? s.segments : nch);
+        return fits(p) ? p : one;
+    }
+    const double chains = (double)s.batch * (double)s.nheads, slots = 2.0 * sm_count();
+    auto cost = [&](const SegPlan &p) {
+        const double per = (double)(p.seg_len / kQ);
+        double c = std::ceil(chains * p.nseg / slots) * (per + 1.0 + 0.15 * (p.nseg - 1));
+        if (p.nseg > 1) c += std::ceil(chains * (p.nseg - 1) / slots) * (0.45 * per + 2.5);
+        return c;
+    };
+    SegPlan best = one;
+    double best_cost = std::ceil(chains / slots) * ((double)nch + 1.0);
+    for (int64_t k = 2; k <= 8 && k <= nch; ++k) {
+        const SegPlan p = make(k);
+        if (!fits(p)) continue;
+        const double c = cost(p);
+        if (c < 0.97 * best_cost) { best = p; best_cost = c; }
+    }
+    return best;
+}
+}  // namespace
+
+int ssd_segments(const ssm_scan_args &s) { return plan_segments(s).nseg; }
+
 size_t ssd_workspace_bytes(const ssm_scan_args &s) {
-    if (s.d_conv == 0) return 0;
-    const size_t one = (size_t)s.batch * (size_t)s.seqlen * (size_t)(s.ngroups * s.dstate) * 2;
-    return 2 * ((one + 255) / 256 * 256);
+    size_t total = 0;
+    if (s.d_conv > 0) total += 2 * round256((size_t)s.batch * (size_t)s.seqlen * (size_t)(s.ngroups * s.dstate) * 2);
+    const SegPlan sp = plan_segments(s);
+    if (sp.nseg > 1) {
+        const size_t rows = (size_t)s.batch * (size_t)(sp.nseg - 1) * (size_t)s.nheads;
+        total += round256(rows * (size_t)(kP * kN) * 4) + round256(rows * 4);
+    }
+    return total;
 }
 
 // cuTensorMapEncodeTiled from the driver, fetched once through the runtime
@@ -989,14 +1354,24 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     const __nv_bfloat16 *Bc = static_cast<const __nv_bfloat16 *>(s.B), *Cc = static_cast<const __nv_bfloat16 *>(s.C);
     int64_t b_bs = s.B_batch_stride, b_ts = s.B_token_stride, c_bs = s.C_batch_stride, c_ts = s.C_token_stride;
     __nv_bfloat16 *wB = nullptr, *wC = nullptr;
+    char *wp = static_cast<char *>(ws);
     if (s.d_conv > 0) {
         // the conv'd B and C live in the workspace
-        wB = static_cast<__nv_bfloat16 *>(ws);
-        const size_t one = (size_t)s.batch * (size_t)s.seqlen * (size_t)GN * 2;
-        wC = reinterpret_cast<__nv_bfloat16 *>(static_cast<char *>(ws) + (one + 255) / 256 * 256);
+        const size_t one = round256((size_t)s.batch * (size_t)s.seqlen * (size_t)GN * 2);
+        wB = reinterpret_cast<__nv_bfloat16 *>(wp);
+        wC = reinterpret_cast<__nv_bfloat16 *>(wp + one);
+        wp += 2 * one;
         Bc = wB; Cc = wC;
         b_bs = c_bs = s.seqlen * GN;
         b_ts = c_ts = GN;
+    }
+    // then the segment states (fixed-length rows cut into segments)
+    const SegPlan sp = plan_segments(s);
+    float *sloc = nullptr, *slog = nullptr;
+    if (sp.nseg > 1) {
+        const size_t rows = (size_t)s.batch * (size_t)(sp.nseg - 1) * (size_t)s.nheads;
+        sloc = reinterpret_cast<float *>(wp);
+        slog = reinterpret_cast<float *>(wp + round256(rows * (size_t)(kP * kN) * 4));
     }
     // Host work first (tensor maps over the whole packed / batched token range,
     // the kernel attribute), so nothing on the host separates the pre-pass
@@ -1018,6 +1393,10 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     }
     cudaError_t e = cudaFuncSetAttribute(ssd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
+    if (sp.nseg > 1) {
+        e = cudaFuncSetAttribute(ssd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStSmemBytes);
+        if (e != cudaSuccess) return e;
+    }
     if (s.d_conv > 0) {
         // pre-pass: conv + SiLU of the B and C channels, once per group, into the workspace
         BcArgs b;
@@ -1065,8 +1444,21 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     a.Braw = static_cast<const __nv_bfloat16 *>(s.B); a.Craw = static_cast<const __nv_bfloat16 *>(s.C);
     a.braw_bs = s.B_batch_stride; a.braw_ts = s.B_token_stride;
     a.craw_bs = s.C_batch_stride; a.craw_ts = s.C_token_stride;
-    dim3 grid((unsigned)s.nheads, (unsigned)nseqs);
+    a.nseg = sp.nseg; a.seg_len = sp.nseg > 1 ? sp.seg_len : (s.seqlen > 0 ? s.seqlen : 1);
+    a.sloc = sloc; a.slog = slog;
+    // the timed region holds the state pass and the scan
     timing_begin(st);
+    if (sp.nseg > 1) {
+        // the state each segment but the last leaves, from zero
+        const dim3 sgrid((unsigned)s.nheads, (unsigned)(nseqs * (sp.nseg - 1)));
+        ssd_state_kernel<<<sgrid, kThreads, kStSmemBytes, st>>>(a, tm_x, tm_b);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) {
+            timing_end(st);
+            return e;
+        }
+    }
+    dim3 grid((unsigned)s.nheads, (unsigned)(nseqs * sp.nseg));
     ssd_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, tm_x, tm_b, tm_c, tm_z, tm_y);
     timing_end(st);
     return cudaGetLastError();

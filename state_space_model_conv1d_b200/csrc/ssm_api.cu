@@ -101,7 +101,7 @@ ssm_status validate_scan(const ssm_scan_args *a) {
         !aligned(a->h_final, 4) || !aligned(a->conv_w, 4) || !aligned(a->conv_b, 4) || !aligned(a->cu_seqlens, 4))
         return SSM_ERR_ALIGNMENT;
     if (!aligned(a->conv_state_in, es) || !aligned(a->conv_state_out, es)) return SSM_ERR_ALIGNMENT;
-    if (a->chunk < 0) return SSM_ERR_INVALID_ARG;
+    if (a->chunk < 0 || a->segments < 0) return SSM_ERR_INVALID_ARG;
     if (a->state_interval != 0) {
         if (a->state_interval < 0 || a->state_interval % 64 != 0 || !a->inter_slots || a->inter_stride < 0 ||
             a->inter_nslots < 0 || (!a->inter_states && !a->inter_conv))
@@ -255,9 +255,16 @@ ssm_status ssm_scan_bwd(const ssm_scan_bwd_args *args, void *workspace, size_t w
 }
 
 size_t ssm_scan_workspace_size(const ssm_scan_args *args) {
-    if (!args || args->batch < 0 || args->seqlen < 0 || args->nseqs < 0 || args->ngroups < 0 || args->dstate < 0)
+    if (!args || args->batch < 0 || args->seqlen < 0 || args->nseqs < 0 || args->ngroups < 0 || args->dstate < 0 ||
+        args->segments < 0)
         return 0;
     return plan_workspace(args).total;
+}
+
+int64_t ssm_scan_segments(const ssm_scan_args *args) {
+    if (validate_scan(args) != SSM_OK) return 0;
+    if (args->mode != SSM_MAMBA2 || !plan_workspace(args).ssd) return 1;
+    return ssm::ssd_segments(*args);
 }
 
 ssm_status ssm_scan_fwd(const ssm_scan_args *args, void *workspace, size_t ws_bytes, void *stream) {

@@ -143,7 +143,7 @@ def _scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, h0, h_final, cu_seqlens, co
     return a
 
 
-def scan_workspace_size(mode, x, dt, A, B, C_, *, cu_seqlens=None, conv_w=None, **_):
+def scan_workspace_size(mode, x, dt, A, B, C_, *, cu_seqlens=None, conv_w=None, segments=0, **_):
     """Bytes of device workspace ssm_scan_fwd needs for these shapes (0 = none)."""
     a = _abi.ScanArgs()
     a.mode, a.dtype = mode, _dtype_code(x)
@@ -157,13 +157,21 @@ def scan_workspace_size(mode, x, dt, A, B, C_, *, cu_seqlens=None, conv_w=None, 
     a.d_conv = 0 if conv_w is None else conv_w.shape[1]
     a.cu_seqlens = _p(cu_seqlens)
     a.nseqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    a.segments = int(segments)
     return int(_abi.lib().ssm_scan_workspace_size(C.byref(a)))
+
+
+def scan_segments(mode, x, dt, A, B, C_, *, z=None, cu_seqlens=None, conv_w=None, segments=0, **_):
+    """Token segments ``scan_fwd`` cuts each row into for these tensors (1 = rows stay whole)."""
+    a = _scan_args(mode, x, dt, A, B, C_, None, z, None, None, None, cu_seqlens, conv_w, None, None, None, x, True, 0)
+    a.segments = int(segments)
+    return int(_abi.lib().ssm_scan_segments(C.byref(a)))
 
 
 def scan_fwd(mode, x, dt, A, B, C_, *, D=None, z=None, dt_bias=None, h0=None, cu_seqlens=None, conv_w=None,
              conv_b=None, conv_state_in=None, delta_softplus=True, y=None, h_final=None, conv_state_out=None,
              return_final_state=True, return_conv_state=None, workspace=None, chunk=0, stream=None,
-             state_interval=0, inter_slots=None, inter_states=None, inter_conv=None):
+             state_interval=0, inter_slots=None, inter_states=None, inter_conv=None, segments=0):
     """Forward selective scan (conv fused in front when ``conv_w`` is given).
 
     Returns ``(y, h_final, conv_state_out)``; the last two are None when not
@@ -176,6 +184,10 @@ def scan_fwd(mode, x, dt, A, B, C_, *, D=None, z=None, dt_bias=None, h0=None, cu
     ``inter_slots[s, k]`` of ``inter_states`` (fp32 ``[nslots, ...state]``) and
     its conv history to ``inter_conv`` (``[nslots, conv_dim, K-1]``, x's
     dtype); negative or out-of-range slots write nothing.
+
+    ``segments`` (Mamba-2 tensor-core path, rows without ``cu_seqlens``): 0 lets
+    the library choose, 1 keeps one CTA per (row, head), n >= 2 scans about n
+    runs of every row at the same time (see ``ssm_scan_args.segments``).
     """
     _need(x, "x")
     if y is None:
@@ -195,6 +207,7 @@ def scan_fwd(mode, x, dt, A, B, C_, *, D=None, z=None, dt_bias=None, h0=None, cu
         conv_state_out = torch.empty((nseq, cdim, conv_w.shape[1] - 1), dtype=x.dtype, device=x.device)
     a = _scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, h0, h_final, cu_seqlens, conv_w, conv_b, conv_state_in,
                    conv_state_out, y, delta_softplus, chunk)
+    a.segments = int(segments)
     if state_interval:
         if inter_slots is None or (inter_states is None and inter_conv is None):
             raise ValueError("state_interval needs inter_slots and a pool")

@@ -226,6 +226,11 @@ WORKLOADS = {
     # (warp-shuffle pair scan) form runs
     "mamba1_seq_b1_l8192_d1536_n16": Workload("mamba1_seq_b1_l8192_d1536_n16", "mamba1", "bf16", batch=1,
                                               seqlen=8192, d_inner=1536, dstate=16, seed=BASE_SEED + 5),
+    # one long Mamba-2 sequence (a single-prompt prefill): 80 (row, head) chains
+    # for 296 CTA slots, so the rows are cut into token segments scanned at once
+    "mamba2_seq_b1_l16384_h80_p64_g8_n128": Workload("mamba2_seq_b1_l16384_h80_p64_g8_n128", "mamba2", "bf16",
+                                                     batch=1, seqlen=16384, nheads=80, headdim=64, ngroups=8,
+                                                     dstate=128, chunk=256, seed=BASE_SEED + 6),
     # the Mamba-1 layer's backward (same inputs; upstream gradients drawn alongside)
     "mamba1_layer_b8_l2048_d1536_n16_bwd": Workload("mamba1_layer_b8_l2048_d1536_n16_bwd", "mamba1", "bf16", batch=8,
                                                     seqlen=2048, d_inner=1536, dstate=16, backward=True,

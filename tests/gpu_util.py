@@ -88,11 +88,11 @@ def as_views(t: dict, mode: int) -> dict:
     return t
 
 
-def gpu_scan(mode, t: dict, chunk=0, delta_softplus=True):
+def gpu_scan(mode, t: dict, chunk=0, delta_softplus=True, segments=0):
     y, hf, cs = ssm.scan_fwd(mode, t["x"], t["dt"], t["A"], t["B"], t["C"], D=t.get("D"), z=t.get("z"),
                              dt_bias=t.get("dt_bias"), h0=t.get("h0"), cu_seqlens=t.get("cu_seqlens"),
                              conv_w=t.get("conv_w"), conv_b=t.get("conv_b"), conv_state_in=t.get("conv_state_in"),
-                             delta_softplus=delta_softplus, chunk=chunk)
+                             delta_softplus=delta_softplus, chunk=chunk, segments=segments)
     torch.cuda.synchronize()
     f = lambda a: None if a is None else a.float().cpu().numpy().astype(np.float64)
     return f(y), f(hf), f(cs)
@@ -105,11 +105,11 @@ def oracle_scan(mode, d: dict, delta_softplus=True):
                            delta_softplus=delta_softplus, nthreads=8)
 
 
-def check_scan(mode, d: dict, dtype: str, views=False, chunk=0, what=""):
+def check_scan(mode, d: dict, dtype: str, views=False, chunk=0, what="", segments=0):
     t = to_dev(d, dtype)
     if views:
         t = as_views(t, mode)
-    y, hf, cs = gpu_scan(mode, t, chunk=chunk)
+    y, hf, cs = gpu_scan(mode, t, chunk=chunk, segments=segments)
     ry, rh, rc = oracle_scan(mode, d)
     assert_close(y, ry, dtype, f"{what} y")
     assert_close(hf, rh, dtype, f"{what} h_final")

@@ -29,7 +29,7 @@ def declared_symbols():
 def test_library_exists_and_loads():
     assert os.path.exists(_abi.LIB_PATH), "build libssm.so first"
     lib = _abi.lib()
-    assert lib.ssm_abi_version() == 1
+    assert lib.ssm_abi_version() == _abi.ABI_VERSION == 2
 
 
 def test_every_declared_symbol_is_exported():
@@ -146,6 +146,45 @@ def test_workspace_size_is_host_only():
     assert n == 256 + 2 * (2 * 16 * 2 * 128 * 2)
     a = _scan(mode=1, d_inner=8, ngroups=1)             # Mamba-1 needs none
     assert _abi.lib().ssm_scan_workspace_size(C.byref(a)) == 0
+
+
+def test_segment_plan_is_host_only():
+    lib = _abi.lib()
+    big = dict(batch=4, seqlen=4096, nheads=80, headdim=64, d_inner=5120, ngroups=8, dstate=128, d_conv=4,
+               conv_w=FAKE, x_token_stride=5120, x_batch_stride=5120 * 4096, y_token_stride=5120,
+               y_batch_stride=5120 * 4096, dt_token_stride=80, dt_batch_stride=80 * 4096, B_token_stride=1024,
+               B_batch_stride=1024 * 4096, C_token_stride=1024, C_batch_stride=1024 * 4096)
+    # 320 (row, head) chains of 64 chunks: cut when the library chooses
+    assert lib.ssm_scan_segments(C.byref(_scan(**big))) >= 2
+    assert lib.ssm_scan_segments(C.byref(_scan(segments=1, **big))) == 1
+    assert lib.ssm_scan_segments(C.byref(_scan(segments=4, **big))) == 4
+    assert lib.ssm_scan_segments(C.byref(_scan(segments=3, **big))) == 3          # runs of 22, 22, 20 chunks
+    # many chains already fill the GPU: rows stay whole
+    assert lib.ssm_scan_segments(C.byref(_scan(**dict(big, batch=64, x_batch_stride=5120 * 4096)))) == 1
+    # packed sequences and Mamba-1 are never cut; bad arguments give 0
+    assert lib.ssm_scan_segments(C.byref(_scan(segments=4, **dict(big, batch=1, cu_seqlens=FAKE, nseqs=3)))) == 1
+    assert lib.ssm_scan_segments(C.byref(_scan(mode=1, d_inner=8, ngroups=1, dt_token_stride=8, dt_batch_stride=128))) == 1
+    assert lib.ssm_scan_segments(C.byref(_scan(segments=-1, **big))) == 0
+    assert lib.ssm_scan_fwd(C.byref(_scan(segments=-1, **big)), None, 0, None) == _abi.SSM_ERR_INVALID_ARG
+
+
+def test_workspace_holds_segment_states():
+    # 640 tokens = 10 chunks asked in 4 segments: runs of 3 chunks, 4 segments;
+    # the three with a successor keep an fp32 P x N state and a log-decay per
+    # (row, head) after the conv'd B and C
+    kw = dict(nheads=4, headdim=64, d_inner=256, ngroups=2, dstate=128, d_conv=4, conv_w=FAKE, seqlen=640,
+              x_token_stride=256, x_batch_stride=256 * 640, y_token_stride=256, y_batch_stride=256 * 640,
+              dt_token_stride=4, dt_batch_stride=4 * 640, B_token_stride=256, B_batch_stride=256 * 640,
+              C_token_stride=256, C_batch_stride=256 * 640)
+    lib = _abi.lib()
+    one = lib.ssm_scan_workspace_size(C.byref(_scan(segments=1, **kw)))
+    four = lib.ssm_scan_workspace_size(C.byref(_scan(segments=4, **kw)))
+    rows = 2 * 3 * 4
+    assert four - one == rows * 64 * 128 * 4 + 256
+    # packed sequences are never cut
+    packed = dict(kw, batch=1, cu_seqlens=FAKE, nseqs=2)
+    assert lib.ssm_scan_workspace_size(C.byref(_scan(segments=4, **packed))) == \
+        lib.ssm_scan_workspace_size(C.byref(_scan(segments=1, **packed)))
 
 
 def _conv(**kw):
@@ -290,7 +329,7 @@ def test_bounds_checked_build_plumbing():
     assert os.path.exists(path), "build the checked library: python -m state_space_model_conv1d_b200.build --check-bounds"
     chk = _abi.checked_lib()
     assert chk.ssm_check_bounds_enabled() == 1
-    assert chk.ssm_abi_version() == 1
+    assert chk.ssm_abi_version() == _abi.ABI_VERSION
     out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
     exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
     assert declared_symbols() <= exported

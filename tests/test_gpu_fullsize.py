@@ -9,6 +9,7 @@ import pytest
 import torch
 
 import oracle
+import state_space_model_conv1d_b200 as ssm
 from state_space_model_conv1d_b200 import workloads as W
 
 from gpu_util import TOL, assert_close, gpu_scan, to_dev
@@ -47,11 +48,18 @@ def _m2_head_problem(d, h, H, P, G, N):
     return sub
 
 
-@pytest.mark.parametrize("name", ["mamba2_ssd_b4_l4096_h80_p64_g8_n128", "mamba2_varlen_16seq_h64_p64_g1_n128"])
+# The fixed-length workloads run cut into token segments (the library's choice
+# for these shapes), the packed one whole.
+@pytest.mark.parametrize("name", ["mamba2_ssd_b4_l4096_h80_p64_g8_n128", "mamba2_varlen_16seq_h64_p64_g1_n128",
+                                  "mamba2_seq_b1_l16384_h80_p64_g8_n128"])
 def test_mamba2_fullsize_sampled_heads(name):
     w = W.WORKLOADS[name]
     d = W.workload_inputs(w)
-    y, hf, cs = gpu_scan(M2, to_dev(d, "bf16"))
+    t = to_dev(d, "bf16")
+    nseg = ssm.scan_segments(M2, t["x"], t["dt"], t["A"], t["B"], t["C"], z=t["z"], cu_seqlens=t.get("cu_seqlens"),
+                             conv_w=t["conv_w"])
+    assert (nseg == 1) == (d.get("cu_seqlens") is not None), nseg
+    y, hf, cs = gpu_scan(M2, t)
     H, P, G, N = w.nheads, w.headdim, w.ngroups, w.dstate
     for h in (0, H // 2 - 1, H // 2, H - 1):
         sub = _m2_head_problem(d, h, H, P, G, N)

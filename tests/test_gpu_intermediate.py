@@ -35,7 +35,7 @@ def _slots(nseq, stride, nslots, seed):
     return tab
 
 
-def _run(mode, d, dtype, interval, stride, nslots, seed):
+def _run(mode, d, dtype, interval, stride, nslots, seed, segments=0):
     cu = d.get("cu_seqlens")
     nseq = d["h0"].shape[0]
     tab = _slots(nseq, stride, nslots, seed)
@@ -52,7 +52,7 @@ def _run(mode, d, dtype, interval, stride, nslots, seed):
     ssm.scan_fwd(mode, t["x"], t["dt"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"], dt_bias=t["dt_bias"], h0=t["h0"],
                  cu_seqlens=t.get("cu_seqlens"), conv_w=t["conv_w"], conv_b=t.get("conv_b"),
                  conv_state_in=t.get("conv_state_in"), state_interval=interval,
-                 inter_slots=torch.from_numpy(tab).cuda(), inter_states=gh, inter_conv=gc)
+                 inter_slots=torch.from_numpy(tab).cuda(), inter_states=gh, inter_conv=gc, segments=segments)
     torch.cuda.synchronize()
     # oracle on the same values
     rh = pool_h.astype(np.float64)
@@ -96,10 +96,11 @@ def test_mamba1_varlen():
     _run(M1, d, "bf16", 64, stride=4, nslots=8, seed=12)
 
 
+@pytest.mark.parametrize("segments", [1, 3])
 @pytest.mark.parametrize("interval", [64, 128])
-def test_mamba2_tensor_core_batch(interval):
+def test_mamba2_tensor_core_batch(interval, segments):
     d = W.mamba2_inputs(803, 2, 320, 4, 64, 2, 128, dtype="bf16", conv_bias=True, conv_state=True)
-    _run(M2, d, "bf16", interval, stride=5, nslots=7, seed=13)
+    _run(M2, d, "bf16", interval, stride=5, nslots=7, seed=13, segments=segments)
 
 
 def test_mamba2_tensor_core_varlen():

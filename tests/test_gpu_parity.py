@@ -118,6 +118,41 @@ def test_mamba2(b, T, H, P, G, N, K, dtype):
     check_scan(M2, d, dtype, what=f"M2 b{b} T{T} H{H} P{P} G{G} N{N}")
 
 
+# Rows cut into token segments on the tensor-core path: a state-only pass over
+# every segment but the last, then one scan CTA per (segment, head) from the
+# folded entering state.  Requested counts become runs of whole chunks.
+SEG_CASES = [
+    # (b, T, H, G, K, segments)
+    (2, 300, 4, 2, 4, 2),      # 5 chunks: runs of 3 and 2, the last chunk ragged
+    (1, 520, 2, 1, 4, 4),      # 9 chunks: three runs of 3
+    (2, 256, 4, 4, 3, 3),      # 4 chunks asked in 3 runs: two runs of 2
+    (1, 640, 2, 2, 0, 5),      # no conv in front
+    (1, 200, 2, 1, 2, 2),      # conv width 2
+    (1, 65, 2, 1, 4, 2),       # the last run is a single token
+    (1, 4160, 2, 1, 4, 0),     # 65 chunks, count chosen by the library
+]
+
+
+@pytest.mark.parametrize("b,T,H,G,K,segments", SEG_CASES)
+def test_mamba2_segments(b, T, H, G, K, segments):
+    d = W.mamba2_inputs(450 + T + H + K, b, T, H, 64, G, 128, d_conv=K, dtype="bf16", conv_bias=True,
+                        conv_state=True)
+    check_scan(M2, d, "bf16", segments=segments, what=f"M2 segments={segments} b{b} T{T} H{H} G{G} K{K}")
+
+
+def test_mamba2_segments_match_unsegmented():
+    """Segmenting changes only the fp32 rounding of the carried state."""
+    d = W.mamba2_inputs(460, 2, 1000, 4, 64, 2, 128, dtype="bf16", conv_bias=True, conv_state=True)
+    t = to_dev(d, "bf16")
+    y1, h1, c1 = gpu_scan(M2, t, segments=1)
+    for nseg in (2, 4, 8):
+        y2, h2, c2 = gpu_scan(M2, t, segments=nseg)
+        # both sides round X' (the decay-weighted x) to bf16, with different weights
+        assert rel_err(y2, y1) <= TOL["bf16"], nseg
+        assert rel_err(h2, h1) <= TOL["bf16"], nseg
+        assert np.array_equal(c2, c1), nseg
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_mamba2_strided_views(dtype):
     d = W.mamba2_inputs(410, 2, 50, 4, 32, 2, 32, dtype=dtype, conv_state=True)
