@@ -264,7 +264,12 @@ class Job:
                 self.flops = None
             if self.split is not None:
                 # a rank's step of the split: its largest kernel is the fix-up
-                self.kernel = "split_fixup_m1_kernel" if mode == ssm.MAMBA1 else "split_fixup_m2_kernel"
+                if mode == ssm.MAMBA1:
+                    self.kernel = "split_fixup_m1_kernel"
+                elif w.dtype == "bf16" and w.headdim == 64 and w.dstate == 128:
+                    self.kernel = "split_fixup_tc_kernel"      # C'.h_in^T on the tensor cores
+                else:
+                    self.kernel = "split_fixup_m2_kernel"
                 self.sources = ("seq_split.cu",)
         elif w.kind == "decode":
             ww = W.Workload(**{**w.__dict__, "seed": w.seed + seed_shift})
@@ -545,7 +550,12 @@ def run_cuda(args):
             tpk = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1400.0)))
             roofline["tensor"] = {"achieved": tf, "peak": tpk, "unit": "TFLOP/s", "frac": tf / tpk,
                                   "flops_per_step": int(job.flops), "peak_source": "MEASURED_PEAKS.json bf16_tflops_sustained"}
-    if job.split is not None and job.fix_flops:
+    if job.split is not None and job.fix_flops and job.kernel == "split_fixup_tc_kernel":
+        tpk = float(peaks.get("bf16_tflops", 1590.0))
+        ftf = job.fix_flops / (kern_ms / 1e3) / 1e12
+        roofline["tensor"] = {"achieved": ftf, "peak": tpk, "unit": "TFLOP/s", "frac": ftf / tpk,
+                              "flops_per_launch": int(job.fix_flops), "peak_source": "MEASURED_PEAKS.json bf16_tflops"}
+    elif job.split is not None and job.fix_flops:
         fma_peak = NUM_SMS * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
         ftf = job.fix_flops / (kern_ms / 1e3) / 1e12
         roofline["fma"] = {"achieved": ftf, "peak": fma_peak, "unit": "TFLOP/s", "frac": ftf / fma_peak,

@@ -2,6 +2,7 @@
 // Arguments reaching these functions have already been validated by ssm_api.cu.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -81,6 +82,10 @@ bool ssd_supported(const ssm_scan_args &a);     // shapes and 16-byte alignment:
 size_t ssd_workspace_bytes(const ssm_scan_args &a);
 int ssd_segments(const ssm_scan_args &a);       // token segments per row (1 = rows stay whole)
 cudaError_t launch_ssd(const ssm_scan_args &a, const SeqView &sv, void *ws_bc, cudaStream_t st);
+// A [batch][tokens][channels] bf16 tensor (element strides ts, bs) as a 3-d
+// TMA map with a 64-channel x box_rows-token box (128-byte swizzle or none).
+bool make_map_box(CUtensorMap *m, const void *base, int64_t channels, int64_t tokens, int64_t batch, int64_t ts,
+                  int64_t bs, bool swizzle, int box_rows);
 cudaError_t launch_state_update(const ssm_update_args &a, cudaStream_t st);
 // Backward scan: workspace bytes for the checkpoints and B / C accumulators
 // (after the error word and the varlen order), and its launcher.

@@ -11,8 +11,11 @@
 // its state at token t differs from the zero-start one by exp(A cs_t) h_in,
 // cs_t the in-segment prefix sum of delta.  The read-out is linear in the
 // state, so y_t differs by silu(z_t) * C_t . (exp(A cs_t) h_in).
+#include <string.h>
+
 #include "common.cuh"
 #include "launch.h"
+#include "tc05.cuh"
 
 namespace ssm {
 namespace {
@@ -350,6 +353,276 @@ __global__ void __launch_bounds__(kF2Threads) split_fixup_m2_kernel(FixArgs f) {
     }
 }
 
+// ------------------------------------------- fix-up, Mamba-2 on the tensor cores
+// The same fix-up as a matrix product per head: for a tile of 128 tokens of
+// one (row, group), Yh = C' h_in^T with C' the group's conv'd C rows (128 x N,
+// bf16, K-major) and h_in^T (N x P, bf16, MN-major), one tcgen05 chain of
+// eight K = 16 MMAs into a 128 x 64 fp32 tensor-memory accumulator; then
+// y_t += exp(A cs_t) silu(z_t) Yh_t.  Shapes of the tensor-core scan (bf16,
+// P = 64, N = 128).  The CTA builds C' once (raw rows staged in shared memory,
+// conv + SiLU into the 128-byte-swizzled operand tile) and walks the group's
+// heads.  Per head the y and z tiles (128 tokens x 64 channels) come in and y
+// goes out by TMA (rows past the segment are zero-filled on the way in and
+// clipped on the way out; y double-buffered), so each thread updates its
+// token's row in shared memory.  While head h's epilogue runs, head h+1's
+// state is already on its way into registers and its z and y tiles into
+// shared memory; its state tile is written, and its MMAs issued, right after.
+// A wait that runs out (two seconds; not expected) stores the tile's y as NaN
+// instead of fixing it.
+constexpr int kFtTok = 128;                       // tokens per CTA (the MMA's M)
+constexpr int kFtP = 64, kFtN = 128;
+constexpr int kFtThreads = 256;
+constexpr uint32_t FT_OFF_A = 0;                  // C' tile: two K-atoms of 128 rows x 64 n (16 KB each)
+constexpr uint32_t FT_OFF_B = 32768;              // h_in^T tile: 128 n rows x 64 p (16 KB)
+constexpr uint32_t FT_OFF_R = 32768;              // raw C rows, bf16 [kFtTok + K - 1][N], before the tiles below
+constexpr uint32_t FT_OFF_Z = 49152;              // z tile, 128 rows x 64 p (128-byte swizzle)
+constexpr uint32_t FT_OFF_Y = 65536;              // two y tiles, same layout
+constexpr uint32_t FT_OFF_AUX = 98304;
+static_assert(FT_OFF_R + (kFtTok + kMaxConvWidth - 1) * kFtN * 2 <= FT_OFF_AUX, "raw rows overflow");
+enum { FB_MMA0, FB_MMA1, FB_Z, FB_Y0, FB_Y1, FB_DRAIN, kNumFtBar };
+struct FtAux {
+    uint32_t tmem;
+    int abort;
+    uint64_t mb[kNumFtBar];
+};
+constexpr size_t kFtSmemBytes = FT_OFF_AUX + sizeof(FtAux) + 1024;
+constexpr uint32_t ID_FT = tc::idesc_bf16(128, 64, 0, 1);
+
+SSM_DEVINL bool ft_wait(FtAux &ax, int i, uint32_t parity) {
+    if (tc::mbar_try_wait_sleep(&ax.mb[i], parity, 20000)) return true;
+    const uint64_t t0 = tc::globaltimer_ns();
+    for (;;) {
+        if (*reinterpret_cast<volatile int *>(&ax.abort)) return false;
+        if (tc::mbar_try_wait_sleep(&ax.mb[i], parity, 20000)) return true;
+        if (tc::globaltimer_ns() - t0 > 2000000000ull) break;
+    }
+    *reinterpret_cast<volatile int *>(&ax.abort) = 1;
+    return false;
+}
+
+__global__ void __launch_bounds__(kFtThreads, 2)
+split_fixup_tc_kernel(const FixArgs f, const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_z) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
+    FtAux &ax = *reinterpret_cast<FtAux *>(smem + FT_OFF_AUX);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t g = blockIdx.x, b = blockIdx.z;
+    const int64_t t0 = (int64_t)blockIdx.y * kFtTok;
+    const int nt = (int)min((int64_t)kFtTok, f.seqlen - t0);
+    const int64_t hpg = f.H / f.G;
+    const int K = (int)f.K, Ke = K > 0 ? K : 1;
+    const bool zg = f.z != nullptr;
+    if (!SSM_BOUNDS(t0 + nt - 1, f.seqlen, BS_SPLIT_ROW) || !SSM_BOUNDS((g + 1) * kFtN - 1, f.G * kFtN, BS_SPLIT_CHANNEL))
+        return;
+    const __nv_bfloat16 *Cb = static_cast<const __nv_bfloat16 *>(f.C) + b * f.cbs + g * kFtN;
+    const __nv_bfloat16 *si = static_cast<const __nv_bfloat16 *>(f.conv_state_in);
+    if (tid == 0) {
+        ax.abort = 0;
+        for (int i = 0; i < kNumFtBar; ++i) tc::mbar_init(&ax.mb[i], 1);
+        tc::mbar_init_fence();
+        tc::prefetch_map(&tm_y);
+        if (zg) tc::prefetch_map(&tm_z);
+    }
+    if (warp == 0) tc::tmem_alloc(&ax.tmem, 128);
+    // raw C rows of the tile: tokens t0 - (Ke - 1) .. t0 + kFtTok - 1, 16 bytes (8 channels) per load,
+    // every load of a thread issued before its stores
+    const int R = kFtTok + Ke - 1;
+    unsigned char *raw = smem + FT_OFF_R;
+    {
+        constexpr int kMaxIt = ((kFtTok + kMaxConvWidth - 1) * (kFtN / 8) + kFtThreads - 1) / kFtThreads;
+        uint4 v[kMaxIt];
+#pragma unroll
+        for (int it = 0; it < kMaxIt; ++it) {
+            const int i = tid + it * kFtThreads;
+            const int r = i / (kFtN / 8), c8 = i % (kFtN / 8);
+            const int64_t tau = t0 - (Ke - 1) + r;
+            v[it] = make_uint4(0, 0, 0, 0);
+            if (r < R) {
+                if (tau >= 0 && tau < f.seqlen) {
+                    v[it] = *reinterpret_cast<const uint4 *>(Cb + tau * f.cts + c8 * 8);
+                } else if (tau < 0 && si) {
+                    // before the segment: the carried conv state [row][channel][K-1]
+                    alignas(16) __nv_bfloat16 e[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int64_t ch = f.H * f.P + f.G * kFtN + g * kFtN + c8 * 8 + j;
+                        e[j] = si[(b * f.cdim + ch) * (K - 1) + (tau + K - 1)];
+                    }
+                    v[it] = *reinterpret_cast<const uint4 *>(e);
+                }
+            }
+        }
+#pragma unroll
+        for (int it = 0; it < kMaxIt; ++it) {
+            const int i = tid + it * kFtThreads;
+            const int r = i / (kFtN / 8), c8 = i % (kFtN / 8);
+            if (r < R) *reinterpret_cast<uint4 *>(raw + r * (kFtN * 2) + c8 * 16) = v[it];
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = ax.tmem;
+    // C' = SiLU(conv(C)) (or C itself without a conv): thread -> 8 channels c8 of rows tid / 16 + 16 i;
+    // rows past the segment are zero
+    {
+        const int c8 = tid % (kFtN / 8);
+        float w[kMaxConvWidth][8], bias[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int64_t ch = f.H * f.P + f.G * kFtN + g * kFtN + c8 * 8 + j;
+#pragma unroll
+            for (int k = 0; k < kMaxConvWidth; ++k) w[k][j] = k < K ? f.conv_w[ch * K + k] : 0.f;
+            bias[j] = (K > 0 && f.conv_b) ? f.conv_b[ch] : 0.f;
+        }
+        for (int t = tid / (kFtN / 8); t < kFtTok; t += kFtThreads / (kFtN / 8)) {
+            float o[8];
+            if (K > 0) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o[j] = bias[j];
+#pragma unroll
+                for (int k = 0; k < kMaxConvWidth; ++k) {
+                    if (k < K) {
+                        float v[8];
+                        tc::unpack_bf16x8(*reinterpret_cast<const uint4 *>(raw + (t + k) * (kFtN * 2) + c8 * 16), v);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) o[j] = fmaf(w[k][j], v[j], o[j]);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o[j] = silu_fast<__nv_bfloat16>(o[j]);
+            } else {
+                tc::unpack_bf16x8(*reinterpret_cast<const uint4 *>(raw + t * (kFtN * 2) + c8 * 16), o);
+            }
+            if (t >= nt) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o[j] = 0.f;
+            }
+            *reinterpret_cast<uint4 *>(smem + FT_OFF_A + tc::off_sw128(t, c8 * 8, 16384)) = tc::pack_bf16x8(o);
+        }
+    }
+    // the raw rows are consumed: the state, z and y tiles may take their space
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    auto load_z = [&](int64_t h) {
+        if (!zg) return;
+        tc::mbar_expect_tx(&ax.mb[FB_Z], kFtTok * kFtP * 2);
+        tc::tma_load_3d(smem + FT_OFF_Z, &tm_z, (int)(h * kFtP), (int)t0, (int)b, &ax.mb[FB_Z]);
+    };
+    auto load_y = [&](int64_t h, int yb) {
+        tc::mbar_expect_tx(&ax.mb[FB_Y0 + yb], kFtTok * kFtP * 2);
+        tc::tma_load_3d(smem + FT_OFF_Y + yb * 16384, &tm_y, (int)(h * kFtP), (int)t0, (int)b, &ax.mb[FB_Y0 + yb]);
+    };
+    if (tid == 0) {
+        load_z(g * hpg);
+        load_y(g * hpg, 0);
+    }
+    // h_in^T of one head: rows n, 64 p (MN-major).  Lanes over n keep the loads
+    // coalesced; a thread's 32 loads are issued together (fetch), converted and
+    // stored once the tile is free (put).
+    constexpr int kIt = kFtN * (kFtP / 8) / kFtThreads;
+    float hv[kIt][8];
+    auto fetch_state = [&](int64_t h) {
+        const float *hb = f.h_in + (b * f.H + h) * kFtP * kFtN;
+#pragma unroll
+        for (int it = 0; it < kIt; ++it) {
+            const int i = tid + it * kFtThreads, n = i % kFtN, p8 = i / kFtN;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) hv[it][j] = hb[(int64_t)(p8 * 8 + j) * kFtN + n];
+        }
+    };
+    auto put_state = [&]() {
+#pragma unroll
+        for (int it = 0; it < kIt; ++it) {
+            const int i = tid + it * kFtThreads, n = i % kFtN, p8 = i / kFtN;
+            *reinterpret_cast<uint4 *>(smem + FT_OFF_B + tc::off_sw128(n, p8 * 8, 8192)) = tc::pack_bf16x8(hv[it]);
+        }
+    };
+    const uint32_t sbase = tc::smem_u32(smem);
+    const uint64_t dA = tc::desc_sw128(sbase + FT_OFF_A, 16, 1024);
+    const uint64_t dB = tc::desc_sw128(sbase + FT_OFF_B, 8192, 1024);
+    auto issue = [&](int bb) {
+#pragma unroll
+        for (int kk = 0; kk < kFtN / 16; ++kk)
+            tc::mma_bf16(tmem + bb * 64, dA + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), dB + kk * 128, ID_FT, kk > 0);
+        tc::mma_commit(&ax.mb[FB_MMA0 + bb]);
+    };
+    fetch_state(g * hpg);
+    put_state();
+    tc::fence_proxy_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (tid == 0) issue(0);
+
+    // epilogue mapping: warp quarter q4 -> tokens 32 q4 .. 32 q4 + 31 (lane = token), half -> p 32 half ..
+    const int q4 = warp & 3, half = warp >> 2;
+    const int t = q4 * 32 + lane;
+    const float *cum_t = f.cum + (b * f.seqlen + t0 + t) * f.H;
+    float cum_next = t < nt ? cum_t[g * hpg] : 0.f;
+    for (int64_t hi = 0; hi < hpg; ++hi) {
+        const int64_t h = g * hpg + hi;
+        const int bb = (int)(hi & 1), yb = (int)(hi & 1);
+        const bool more = hi + 1 < hpg;
+        const float cum_h = cum_next;
+        if (more) {
+            if (t < nt) cum_next = cum_t[h + 1];
+            fetch_state(h + 1);                  // in flight during this head's epilogue
+        }
+        bool ok = ft_wait(ax, FB_MMA0 + bb, (uint32_t)(hi >> 1) & 1u);
+        ok = ft_wait(ax, FB_Y0 + yb, (uint32_t)(hi >> 1) & 1u) && ok;
+        if (zg) ok = ft_wait(ax, FB_Z, (uint32_t)hi & 1u) && ok;
+        ok = __all_sync(0xffffffffu, ok);
+        tc::fence_after_sync();
+        const float e = ex2(f.A[h] * kLog2e * cum_h);
+        float acc[32];
+        if (ok) tc::tmem_ld32(tmem + ((uint32_t)(q4 * 32) << 16) + bb * 64 + half * 32, acc);
+        unsigned char *ytile = smem + FT_OFF_Y + yb * 16384;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t off = (uint32_t)(t >> 3) * 1024u + (uint32_t)(t & 7) * 128u +
+                                 ((uint32_t)((half * 4 + q) ^ (t & 7)) << 4);
+            float yv[8], zv[8], o[8];
+            tc::unpack_bf16x8(*reinterpret_cast<const uint4 *>(ytile + off), yv);
+            if (zg) tc::unpack_bf16x8(*reinterpret_cast<const uint4 *>(smem + FT_OFF_Z + off), zv);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                o[j] = ok ? fmaf(e * (zg ? silu_fast<__nv_bfloat16>(zv[j]) : 1.f), acc[q * 8 + j], yv[j])
+                          : __int_as_float(0x7fc00000);
+            *reinterpret_cast<uint4 *>(ytile + off) = tc::pack_bf16x8(o);
+        }
+        // head hi+1's state tile (MMA(hi) has read the previous one)
+        if (more) put_state();
+        tc::fence_proxy_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        if (tid == 0) {
+            tc::tma_store_3d(&tm_y, (int)(h * kFtP), (int)t0, (int)b, ytile);
+            if (more) {
+                load_z(h + 1);                    // the epilogue has read z
+                if (!*reinterpret_cast<volatile int *>(&ax.abort)) issue(bb ^ 1);
+                tc::bulk_wait_read_1();           // y tile yb ^ 1 (stored one head ago) has been read
+                load_y(h + 1, yb ^ 1);
+            }
+        }
+    }
+    if (tid == 0) {
+        tc::bulk_wait_all();
+        if (*reinterpret_cast<volatile int *>(&ax.abort)) {
+            tc::mma_commit(&ax.mb[FB_DRAIN]);
+            tc::mbar_wait(&ax.mb[FB_DRAIN], 0, 1u << 22);
+            tc::mbar_wait(&ax.mb[FB_Z], (uint32_t)(hpg - 1) & 1u, 1u << 22);
+            tc::mbar_wait(&ax.mb[FB_Y0 + (int)((hpg - 1) & 1)], (uint32_t)((hpg - 1) >> 1) & 1u, 1u << 22);
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 0) tc::tmem_dealloc(tmem, 128);
+}
+
 template <typename T>
 cudaError_t tail_typed(const ssm_scan_args &a, void *tail, cudaStream_t st) {
     const bool m2 = a.mode == SSM_MAMBA2;
@@ -377,6 +650,17 @@ cudaError_t cum_delta_typed(const ssm_scan_args &a, float *cum, float *sum, cuda
     return cudaGetLastError();
 }
 
+// The tensor-core fix-up takes the tensor-core scan's shapes with 16-byte
+// aligned C, y and z rows (its loads and stores move 8 channels at a time).
+bool fixup_tc_ok(const ssm_scan_args &a) {
+    auto al16 = [](const void *p) { return p == nullptr || ((uintptr_t)p & 15) == 0; };
+    auto st8 = [](int64_t v) { return v % 8 == 0; };
+    return a.mode == SSM_MAMBA2 && a.dtype == SSM_BF16 && a.headdim == kFtP && a.dstate == kFtN &&
+           a.d_conv <= kMaxConvWidth && al16(a.C) && al16(a.y) && al16(a.z) && st8(a.C_token_stride) &&
+           st8(a.C_batch_stride) && st8(a.y_token_stride) && st8(a.y_batch_stride) &&
+           (a.z == nullptr || (st8(a.z_token_stride) && st8(a.z_batch_stride)));
+}
+
 template <typename T>
 cudaError_t fixup_typed(const ssm_scan_args &a, const float *cum, const float *h_in, cudaStream_t st) {
     if (a.batch == 0 || a.seqlen == 0) return cudaSuccess;
@@ -395,6 +679,23 @@ cudaError_t fixup_typed(const ssm_scan_args &a, const float *cum, const float *h
                   (unsigned)a.batch);
         timing_begin(st);
         split_fixup_m1_kernel<T><<<grid, kF1Threads, 0, st>>>(f);
+        timing_end(st);
+        return cudaGetLastError();
+    }
+    if (fixup_tc_ok(a)) {
+        CUtensorMap tm_y, tm_z;
+        memset(&tm_y, 0, sizeof(tm_y));
+        memset(&tm_z, 0, sizeof(tm_z));
+        if (!make_map_box(&tm_y, a.y, a.d_inner, a.seqlen, a.batch, a.y_token_stride, a.y_batch_stride, true, kFtTok) ||
+            (a.z && !make_map_box(&tm_z, a.z, a.d_inner, a.seqlen, a.batch, a.z_token_stride, a.z_batch_stride, true,
+                                  kFtTok)))
+            return cudaErrorInvalidValue;
+        cudaError_t e = cudaFuncSetAttribute(split_fixup_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kFtSmemBytes);
+        if (e != cudaSuccess) return e;
+        dim3 grid((unsigned)a.ngroups, (unsigned)((a.seqlen + kFtTok - 1) / kFtTok), (unsigned)a.batch);
+        timing_begin(st);
+        split_fixup_tc_kernel<<<grid, kFtThreads, kFtSmemBytes, st>>>(f, tm_y, tm_z);
         timing_end(st);
         return cudaGetLastError();
     }

@@ -1333,17 +1333,21 @@ EncodeTiledFn encode_tiled() {
 
 // A [batch][tokens][channels] bf16 tensor (element strides ts, bs) as a 3-d map
 // with a 64-channel x 64-token box.
-bool make_map(CUtensorMap *m, const void *base, int64_t channels, int64_t tokens, int64_t batch, int64_t ts, int64_t bs,
-              bool swizzle) {
+bool make_map_box(CUtensorMap *m, const void *base, int64_t channels, int64_t tokens, int64_t batch, int64_t ts,
+                  int64_t bs, bool swizzle, int box_rows) {
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)channels, (cuuint64_t)tokens, (cuuint64_t)batch};
     const cuuint64_t strides[2] = {(cuuint64_t)ts * 2, (cuuint64_t)(batch > 1 ? bs : ts * tokens) * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)kQ, 1};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+bool make_map(CUtensorMap *m, const void *base, int64_t channels, int64_t tokens, int64_t batch, int64_t ts, int64_t bs,
+              bool swizzle) {
+    return make_map_box(m, base, channels, tokens, batch, ts, bs, swizzle, kQ);
 }
 
 cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cudaStream_t st) {

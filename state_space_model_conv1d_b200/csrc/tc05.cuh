@@ -91,6 +91,8 @@ SSM_DEVINL void tma_store_3d(const CUtensorMap *map, int c0, int c1, int c2, con
 }
 // Wait until the issued bulk stores have finished reading shared memory / have completed.
 SSM_DEVINL void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+// ... all but the most recent bulk group have finished reading shared memory
+SSM_DEVINL void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;\n" ::: "memory"); }
 SSM_DEVINL void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
 SSM_DEVINL void prefetch_map(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -78,6 +78,17 @@ def test_mamba2_tensor_core_shape(bounds):
     _check(M2, d, "bf16", bounds)
 
 
+@pytest.mark.parametrize("H,G,gate", [(4, 2, True), (6, 1, False), (2, 2, True)])
+def test_mamba2_tensor_core_fixup_tiles(H, G, gate):
+    """The tensor-core fix-up over several 128-token tiles with a ragged last
+    one, one to six heads per group (both accumulator buffers), with and
+    without the gate."""
+    d = W.mamba2_inputs(915 + H, 2, 701, H, 64, G, 128, dtype="bf16", conv_bias=True, conv_state=True)
+    if not gate:
+        d["z"] = None
+    _check(M2, d, "bf16", [0, 300, 701])
+
+
 @pytest.mark.parametrize("dtype,P,N,bounds", [("f32", 8, 16, [0, 30, 61, 95, 130]), ("bf16", 48, 64, [0, 90, 200]),
                                               ("f32", 64, 256, [0, 40, 97])])
 def test_mamba2_simt_shapes(dtype, P, N, bounds):
