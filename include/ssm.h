@@ -390,7 +390,12 @@ SSM_API ssm_status ssm_split_combine(const ssm_split_args *args, void *stream);
 /* Step 6.  `args` describes the segment's ssm_scan_fwd call; its y is
  * updated in place, its h0 / h_final / conv_state_out fields are ignored.
  * cum_delta is step 3's output, h_in step 5's.  A segment with no tokens
- * returns SSM_OK without touching anything (the pointers may be NULL). */
+ * returns SSM_OK without touching anything (the pointers may be NULL).
+ * Mamba-2 in bf16 with headdim 64, dstate 128 and 16-byte aligned C, y, z
+ * rows runs the correction as a tensor-core product per head (h_in rounded
+ * to bf16 as the operand, fp32 accumulation); its device waits are bounded,
+ * and one that runs out (not expected) leaves that tile's y as NaN, since
+ * this call has no workspace for an error word. */
 SSM_API ssm_status ssm_split_fixup(const ssm_scan_args *args, const float *cum_delta, const float *h_in,
                                    void *stream);
 

@@ -17,10 +17,13 @@
 // ssd_state_passing, ssd_chunk_scan) are these four steps; here they are one
 // kernel whose carried state never leaves the SM.
 //
-// Work: one CTA per (sequence, head), two CTAs per SM.  The B / C causal
-// conv + SiLU is shared by the heads of a group, so it runs once per group in
-// a pre-pass that writes bf16 B, C into the workspace; the x conv + SiLU runs
-// here.  Per chunk of Q = 64 tokens, four tensor-core products:
+// Work: one CTA per (sequence, head), two CTAs per SM; fixed-length rows that
+// leave the GPU short of CTAs are cut into token segments, one CTA per
+// (segment, head), seeded by a state-only pass (the segment-states section
+// below).  The B / C causal conv + SiLU is shared by the heads of a group, so
+// it runs once per group in a pre-pass that writes bf16 B, C into the
+// workspace; the x conv + SiLU runs here.  Per chunk of Q = 64 tokens, four
+// tensor-core products:
 //   G   = C B^T     M=64  N=64 K=128  A K-major,  B K-major      -> TMEM 0..63
 //   Yo  = C S^T     M=64  N=64 K=128  A K-major,  B MN-major     -> TMEM 128..191
 //   Sc  = B^T X'    M=128 N=64 K=64   A MN-major, B MN-major     -> TMEM 192..255
