@@ -113,6 +113,98 @@ split_cum_delta_kernel(const T *__restrict__ dt, int64_t dbs, int64_t dts, const
     if (ok && w == 0) sum[b * U + u] = carry;
 }
 
+// In parallel over token blocks of 32 * kCdWarps tokens, when cs is wanted:
+// (1) each CTA the in-block prefix of one block (the loop body above, no
+// carry); (2) one thread per (row, unit) turns the blocks' last entries into
+// the prefix up to there, in order, and writes the total; (3) each CTA of a
+// later block adds the prefix that ends the block before it to its other
+// entries.  Every entry is written by one thread of one launch, so the
+// result does not depend on scheduling.
+constexpr int kCdBlock = 32 * kCdWarps;
+
+template <typename T>
+__global__ void __launch_bounds__(kCdWarps * 32)
+split_cum_local_kernel(const T *__restrict__ dt, int64_t dbs, int64_t dts, const float *__restrict__ dt_bias,
+                       int softplus_on, int64_t U, int64_t seqlen, float *__restrict__ cum) {
+    __shared__ float tot[kCdWarps][32];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t u = (int64_t)blockIdx.x * 32 + lane;
+    const int64_t b = blockIdx.y;
+    const bool ok = u < U;
+    const float bias = (ok && dt_bias) ? dt_bias[u] : 0.f;
+    const int64_t tw = (int64_t)blockIdx.z * kCdBlock + 32 * w;
+    const int nv = ok ? (int)max((int64_t)0, min((int64_t)32, seqlen - tw)) : 0;
+    const T *p = dt + b * dbs + u + tw * dts;
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = i < nv ? Elem<T>::ld(p + i * dts) : 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        if (i < nv) {
+            const float r = v[i] + bias;
+            v[i] = softplus_on ? softplus(r) : r;
+        }
+    }
+#pragma unroll
+    for (int i = 1; i < 32; ++i) v[i] += v[i - 1];
+    tot[w][lane] = v[31];
+    __syncthreads();
+    float off = 0.f;
+#pragma unroll
+    for (int k = 0; k < kCdWarps; ++k)
+        if (k < w) off += tot[k][lane];
+    if (ok) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (i < nv) cum[(b * seqlen + tw + i) * U + u] = v[i] + off;
+    }
+}
+
+__global__ void split_cum_ends_kernel(int64_t batch, int64_t U, int64_t seqlen, float *__restrict__ cum,
+                                      float *__restrict__ sum) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= batch * U) return;
+    const int64_t b = i / U, u = i % U;
+    const int64_t nblk = (seqlen + kCdBlock - 1) / kCdBlock;
+    float run = 0.f;
+    for (int64_t k0 = 0; k0 < nblk; k0 += 16) {
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int64_t k = k0 + j;
+            const int64_t e = min((k + 1) * kCdBlock, seqlen) - 1;
+            v[j] = k < nblk ? cum[(b * seqlen + e) * U + u] : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int64_t k = k0 + j;
+            if (k < nblk) {
+                run += v[j];
+                cum[(b * seqlen + min((k + 1) * kCdBlock, seqlen) - 1) * U + u] = run;
+            }
+        }
+    }
+    sum[b * U + u] = run;
+}
+
+__global__ void __launch_bounds__(kCdWarps * 32)
+split_cum_offset_kernel(int64_t U, int64_t seqlen, float *__restrict__ cum) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t u = (int64_t)blockIdx.x * 32 + lane;
+    const int64_t b = blockIdx.y;
+    const int64_t blk = (int64_t)blockIdx.z + 1;            // blocks after the first
+    if (u >= U) return;
+    const int64_t t0 = blk * kCdBlock, tend = min(t0 + kCdBlock, seqlen) - 1;   // tend already holds its prefix
+    const float off = cum[(b * seqlen + t0 - 1) * U + u];
+    const int64_t tw = t0 + 32 * w;
+    float v[32];                                          // every load before any store
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = tw + i < tend ? cum[(b * seqlen + tw + i) * U + u] : 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        if (tw + i < tend) cum[(b * seqlen + tw + i) * U + u] = v[i] + off;
+}
+
 // ------------------------------------------------------------- combine
 // One thread per (row, state element): the pairs of segments 0..rank folded
 // in order.  `per_unit` state elements share one delta unit (N for Mamba-1,
@@ -643,6 +735,18 @@ template <typename T>
 cudaError_t cum_delta_typed(const ssm_scan_args &a, float *cum, float *sum, cudaStream_t st) {
     const int64_t U = a.mode == SSM_MAMBA2 ? a.nheads : a.d_inner;
     if (a.batch == 0) return cudaSuccess;
+    const int64_t nblk = (a.seqlen + kCdBlock - 1) / kCdBlock;
+    if (cum && nblk > 1 && nblk <= 65535) {
+        const dim3 g1((unsigned)((U + 31) / 32), (unsigned)a.batch, (unsigned)nblk);
+        split_cum_local_kernel<T><<<g1, kCdWarps * 32, 0, st>>>(static_cast<const T *>(a.dt), a.dt_batch_stride,
+                                                               a.dt_token_stride, a.dt_bias, a.delta_softplus, U,
+                                                               a.seqlen, cum);
+        const int64_t n = a.batch * U;
+        split_cum_ends_kernel<<<(unsigned)((n + 127) / 128), 128, 0, st>>>(a.batch, U, a.seqlen, cum, sum);
+        const dim3 g3((unsigned)((U + 31) / 32), (unsigned)a.batch, (unsigned)(nblk - 1));
+        split_cum_offset_kernel<<<g3, kCdWarps * 32, 0, st>>>(U, a.seqlen, cum);
+        return cudaGetLastError();
+    }
     dim3 grid((unsigned)((U + 31) / 32), (unsigned)a.batch);
     split_cum_delta_kernel<T><<<grid, kCdWarps * 32, 0, st>>>(static_cast<const T *>(a.dt), a.dt_batch_stride,
                                                               a.dt_token_stride, a.dt_bias, a.delta_softplus, U,

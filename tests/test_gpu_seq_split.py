@@ -128,3 +128,36 @@ def test_rank_with_no_tokens(mode, shape):
         P, N, dtype = (64, 128, "bf16") if shape == "tensor_core" else (16, 24, "f32")
         d = W.mamba2_inputs(910, 2, 30, 4, P, 2, N, d_conv=0, dtype=dtype, conv_state=False)
     _check(mode, d, dtype, [0, 13, 13, 30])
+
+
+@pytest.mark.parametrize("mode,T,U", [(M2, 5000, 40), (M1, 700, 70), (M2, 256, 8), (M2, 257, 3)])
+def test_cum_delta_prefix_sums(mode, T, U):
+    """ssm_split_cum_delta against the running sum of softplus(dt + dt_bias)
+    in fp64: several token blocks of 256 (more than 16, one, and one plus a
+    single token), a unit count that is not a multiple of 32; the total alone
+    (no cs requested) agrees with the total of the blocked path."""
+    from state_space_model_conv1d_b200 import ops
+    rng = np.random.default_rng(930 + T + U)
+    b = 2
+    dt = W.round_bf16(rng.standard_normal((b, T, U)).astype(np.float32))
+    bias = rng.uniform(-4.0, -1.0, U).astype(np.float32)
+    ref = np.cumsum(np.log1p(np.exp(dt.astype(np.float64) + bias.astype(np.float64))), axis=1)
+    dev = torch.from_numpy(dt).to("cuda", torch.bfloat16)
+    tb = torch.from_numpy(bias).cuda()
+    if mode == M1:
+        x = torch.zeros((b, T, U), dtype=torch.bfloat16, device="cuda")
+        Bm = torch.zeros((b, T, 4), dtype=torch.bfloat16, device="cuda")
+        A = torch.zeros((U, 4), dtype=torch.float32, device="cuda")
+    else:
+        x = torch.zeros((b, T, U, 8), dtype=torch.bfloat16, device="cuda")
+        Bm = torch.zeros((b, T, 1, 16), dtype=torch.bfloat16, device="cuda")
+        A = torch.zeros((U,), dtype=torch.float32, device="cuda")
+    cs, sd = ops.split_cum_delta(mode, x, dev, A, Bm, Bm, dt_bias=tb)
+    _, sd_only = ops.split_cum_delta(mode, x, dev, A, Bm, Bm, dt_bias=tb, cum=False)
+    torch.cuda.synchronize()
+    got = cs.cpu().numpy().astype(np.float64)
+    # softplus on the GPU is within 2e-5 relative of log1p(exp(u)) in each of its regimes
+    assert np.max(np.abs(got - ref) / np.maximum(np.abs(ref), 1.0)) < 5e-5
+    np.testing.assert_allclose(sd.cpu().numpy(), ref[:, -1], rtol=5e-5)
+    np.testing.assert_allclose(sd_only.cpu().numpy(), sd.cpu().numpy(), rtol=1e-6)
+    np.testing.assert_array_equal(sd.cpu().numpy(), got[:, -1].astype(np.float32))
