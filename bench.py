@@ -382,9 +382,7 @@ class Job:
         if self.w.kind == "decode":
             i = self.step_i % self.nsets
             self.step_i += 1
-            ssm.state_update(self.mode, t["state"], t["conv_state"], t["x"][i], t["dt"][i], t["A"], t["B"][i],
-                             t["C"][i], D=t["D"], z=t["z"][i], dt_bias=t["dt_bias"], conv_w=t["conv_w"],
-                             conv_b=t["conv_b"], y=self.y)
+            self._decode(i, self.y)
             return
         if self.bwd is not None:
             ssm.scan_bwd(self.mode, t["x"], t["dt"], t["A"], t["B"], t["C"], t["dy"], D=t["D"], z=t["z"],
@@ -392,10 +390,111 @@ class Job:
                          conv_b=t["conv_b"], conv_state_in=t["conv_state_in"], dh_final=t["dh_final"],
                          workspace=self.bwd_ws, out=self.bwd)
             return
-        ssm.scan_fwd(self.mode, t["x"], t["dt"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"], dt_bias=t["dt_bias"],
-                     h0=t["h0"], cu_seqlens=t.get("cu_seqlens"), conv_w=t["conv_w"], conv_b=t["conv_b"],
-                     conv_state_in=t["conv_state_in"], y=self.y, h_final=self.hf, conv_state_out=self.cso,
-                     workspace=self.ws, **self.inter)
+        self._scan(t, self.y)
+
+    def _decode(self, i, y):
+        t = self.t
+        self.ssm.state_update(self.mode, t["state"], t["conv_state"], t["x"][i], t["dt"][i], t["A"], t["B"][i],
+                              t["C"][i], D=t["D"], z=t["z"][i], dt_bias=t["dt_bias"], conv_w=t["conv_w"],
+                              conv_b=t["conv_b"], y=y)
+
+    def _scan(self, t, y):
+        self.ssm.scan_fwd(self.mode, t["x"], t["dt"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"], dt_bias=t["dt_bias"],
+                          h0=t["h0"], cu_seqlens=t.get("cu_seqlens"), conv_w=t["conv_w"], conv_b=t["conv_b"],
+                          conv_state_in=t["conv_state_in"], y=y, h_final=self.hf, conv_state_out=self.cso,
+                          workspace=self.ws, **self.inter)
+
+    def e2e_pipelined(self):
+        """Whether the end-to-end leg overlaps copies with compute (forward scans and decode)."""
+        return self.split is None and self.bwd is None
+
+    def e2e_run(self, n, out_hosts, stream):
+        """n end-to-end steps of a forward scan, pipelined across steps: step i's
+        inputs go host->device on one stream while step i-1 computes on `stream`
+        and step i-2's y goes device->host on a third (both PCIe directions at
+        once); device inputs and y are double-buffered.  Every step copies all of
+        its inputs in and its y out.  Returns (h2d, d2h) bytes per step."""
+        torch = self.torch
+        if self.w.kind == "decode":
+            return self._e2e_decode(n, out_hosts, stream)
+        keys = [k for k in ("x", "z", "dt", "B", "C", "h0") if self.host.get(k) is not None]
+        if not hasattr(self, "_t2"):
+            self._t2 = dict(self.t)
+            for k in keys:
+                self._t2[k] = torch.empty_like(self.t[k])
+            self._y2 = torch.empty_like(self.y)
+        sets = [(self.t, self.y), (self._t2, self._y2)]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = {name: [torch.cuda.Event(), torch.cuda.Event()] for name in ("in", "comp", "out")}
+        start = torch.cuda.Event()
+        start.record(stream)
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+        for i in range(n):
+            b = i % 2
+            tb, yb = sets[b]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev["comp"][b])          # step i-2 has finished reading these inputs
+                for k in keys:
+                    tb[k].copy_(self.host[k], non_blocking=True)
+                ev["in"][b].record(s_in)
+            stream.wait_event(ev["in"][b])
+            if i >= 2:
+                stream.wait_event(ev["out"][b])             # step i-2's y has reached the host
+            self._scan(tb, yb)
+            ev["comp"][b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev["comp"][b])
+                out_hosts[b].copy_(yb, non_blocking=True)
+                ev["out"][b].record(s_out)
+        for b in range(min(n, 2)):
+            stream.wait_event(ev["out"][b])
+        h2d = sum(self.host[k].numel() * self.host[k].element_size() for k in keys)
+        return h2d, out_hosts[0].numel() * out_hosts[0].element_size()
+
+    def _e2e_decode(self, n, out_hosts, stream):
+        """Decode steps with the copies overlapped: the token inputs of step i go
+        into its input set (sets cycle, so a set is rewritten only after the
+        step that last read it) while earlier steps compute; y alternates
+        between two buffers.  The state update itself stays in order on
+        `stream`, one step after the other."""
+        torch, t = self.torch, self.t
+        keys = [k for k in ("x", "z", "dt", "B", "C") if self.host.get(k) is not None]
+        if not hasattr(self, "_y2"):
+            self._y2 = torch.empty_like(self.y)
+        ys = [self.y, self._y2]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(self.nsets)]
+        ev_comp = [torch.cuda.Event() for _ in range(self.nsets)]
+        ev_out = [torch.cuda.Event(), torch.cuda.Event()]
+        start = torch.cuda.Event()
+        start.record(stream)
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+        for j in range(n):
+            i = self.step_i % self.nsets
+            self.step_i += 1
+            b = j % 2
+            with torch.cuda.stream(s_in):
+                if j >= self.nsets:
+                    s_in.wait_event(ev_comp[i])
+                for k in keys:
+                    t[k][i].copy_(self.host[k][i], non_blocking=True)
+                ev_in[i].record(s_in)
+            stream.wait_event(ev_in[i])
+            if j >= 2:
+                stream.wait_event(ev_out[b])
+            self._decode(i, ys[b])
+            ev_comp[i].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[i])
+                out_hosts[b].copy_(ys[b], non_blocking=True)
+                ev_out[b].record(s_out)
+        for b in range(min(n, 2)):
+            stream.wait_event(ev_out[b])
+        h2d = sum(self.host[k][0].numel() * self.host[k][0].element_size() for k in keys)
+        return h2d, out_hosts[0].numel() * out_hosts[0].element_size()
 
     def e2e_step(self, out_host):
         """Host-resident inputs: pinned H2D copies, the step, then y back to the host."""
@@ -498,20 +597,30 @@ def run_cuda(args):
     if not args.no_e2e:
         out_host = torch.empty(job.y.shape, dtype=job.y.dtype).pin_memory()
         ne = max(1, min(args.steps, 10))
-        job.e2e_step(out_host)
+        pipelined = job.e2e_pipelined()
+        if pipelined:
+            out_hosts = [out_host, torch.empty(job.y.shape, dtype=job.y.dtype).pin_memory()]
+            job.e2e_run(2, out_hosts, stream)                  # warm-up (allocates the second buffer set)
+        else:
+            job.e2e_step(out_host)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         h2d = d2h = 0
-        for _ in range(ne):
-            h2d, d2h = job.e2e_step(out_host)
+        if pipelined:
+            h2d, d2h = job.e2e_run(ne, out_hosts, stream)
+        else:
+            for _ in range(ne):
+                h2d, d2h = job.e2e_step(out_host)
         e1.record(stream)
         torch.cuda.synchronize()
         ems = reduce_max_ms(e0.elapsed_time(e1), world, "cuda")
         e2e = {"value": weak_scaling_value(job.units, ne, world, ems), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "steps": ne}
+               "d2h_bytes_per_step": int(d2h), "steps": ne,
+               "copies": ("overlapped across steps: inputs in on one stream, y out on another, compute on a third; "
+                          "device buffers double-buffered" if pipelined else "in order within each step")}
 
     if world > 1:
         dist.barrier()
