@@ -481,11 +481,11 @@ constexpr size_t kFtSmemBytes = FT_OFF_AUX + sizeof(FtAux) + 1024;
 constexpr uint32_t ID_FT = tc::idesc_bf16(128, 64, 0, 1);
 
 SSM_DEVINL bool ft_wait(FtAux &ax, int i, uint32_t parity) {
-    if (tc::mbar_try_wait_sleep(&ax.mb[i], parity, 20000)) return true;
+    if (tc::mbar_try_wait(&ax.mb[i], parity)) return true;
     const uint64_t t0 = tc::globaltimer_ns();
     for (;;) {
         if (*reinterpret_cast<volatile int *>(&ax.abort)) return false;
-        if (tc::mbar_try_wait_sleep(&ax.mb[i], parity, 20000)) return true;
+        if (tc::mbar_try_wait(&ax.mb[i], parity)) return true;
         if (tc::globaltimer_ns() - t0 > 2000000000ull) break;
     }
     *reinterpret_cast<volatile int *>(&ax.abort) = 1;

@@ -123,19 +123,6 @@ SSM_DEVINL bool mbar_try_wait(uint64_t *mbar, uint32_t parity) {
     return ok != 0;
 }
 
-// try_wait with a suspend-time hint: a thread whose phase is not complete yet
-// sleeps until it completes or about `hint_ns` nanoseconds pass, instead of
-// spinning on the barrier (spinning threads take issue slots from the warps
-// that do the work).
-SSM_DEVINL bool mbar_try_wait_sleep(uint64_t *mbar, uint32_t parity, uint32_t hint_ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\nselp.b32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(mbar)), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return ok != 0;
-}
 SSM_DEVINL uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
