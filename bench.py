@@ -74,8 +74,51 @@ def source_sha(*names):
 
 
 # ------------------------------------------------------------------ clocks
+def _nvml_poll(uuid, index, phase, done, ready, out):
+    """Sampling process: NVML's SM clock and clock-event reasons of one GPU,
+    as fast as the queries return (a few ms each), tagged with the phase the
+    launching process has set (0: none, 1: timed region, 2: end-to-end leg);
+    read-only queries."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByUUID(uuid) if uuid else pynvml.nvmlDeviceGetHandleByIndex(index)
+        names = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                 "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                 "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                 "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+        mx = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+    except Exception:
+        ready.set()
+        out.put(None)
+        return
+    ready.set()
+    samples = []
+    errors = 0
+    while not done.is_set():
+        ph = phase.value
+        if ph:
+            try:
+                sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:
+                errors += 1
+                time.sleep(0.001)
+                continue
+            if phase.value == ph:                      # the phase did not end during the queries
+                samples.append((ph, sm, sorted(n for n, bit in names.items() if r & bit)))
+            time.sleep(0.0002)
+        else:
+            time.sleep(0.0005)
+    out.put((mx, samples, errors))
+
+
 class ClockSampler:
-    """nvidia-smi samples every 200 ms while the timed region runs."""
+    """SM clock and clock-event reasons of this process's GPU during the timed
+    region: a spawned process polls NVML back to back (no GIL shared with the
+    launching thread) and keeps only samples between mark_start() and
+    mark_stop(); without NVML, nvidia-smi samples every 200 ms.  The GPU is
+    found by its UUID, so the index CUDA sees needs no translation."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -83,23 +126,80 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.idx = device_index
         self.proc = None
+        self.child = None
         self.lines = []
+        self.source = None
+        try:
+            import torch
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+        except Exception:
+            self.uuid = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+            import multiprocessing as mp
+            ctx = mp.get_context("spawn")
+            self.phase, self.done, ready = ctx.Value("i", 0), ctx.Event(), ctx.Event()
+            self.q = ctx.Queue()
+            self.child = ctx.Process(target=_nvml_poll, args=(self.uuid, self.idx, self.phase, self.done, ready, self.q),
+                                     daemon=True)
+            self.child.start()
+            if ready.wait(timeout=30):
+                self.source = "nvml, back-to-back queries"
+                return
+            self.child.terminate()
+        except Exception:
+            pass
+        self.child = None
+        try:
+            dev = self.uuid if self.uuid else str(self.idx)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", dev, f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            self.source = "nvidia-smi, 200 ms"
         except FileNotFoundError:
             self.proc = None
+
+    def mark_start(self, phase=1):
+        if self.child is not None:
+            self.phase.value = phase
+
+    def mark_stop(self):
+        if self.child is not None:
+            self.phase.value = 0
 
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def _stop_child(self):
+        self.done.set()
+        try:
+            res = self.q.get(timeout=30)
+        except Exception:
+            res = None
+        self.child.join(timeout=5)
+        if not res:
+            return None
+        mx, samples, errors = res
+        out = {}
+        for ph, key in ((1, "timed"), (2, "e2e")):
+            sm = [x[1] for x in samples if x[0] == ph]
+            if sm:
+                out[key] = {"sm_mhz": float(np.median(sm)), "sm_min_mhz": float(min(sm)), "sm_max_mhz": mx,
+                            "reasons": sorted({n for x in samples if x[0] == ph for n in x[2]}), "samples": len(sm)}
+        if "timed" not in out:
+            return None
+        clk = dict(out["timed"], source=self.source, query_errors=errors)
+        if "e2e" in out:
+            clk["during_e2e_leg"] = out["e2e"]
+        return clk
+
     def stop(self):
+        if self.child is not None:
+            return self._stop_child()
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -124,7 +224,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": self.source}
 
 
 # --------------------------------------------------------------- workloads
@@ -573,18 +673,19 @@ def run_cuda(args):
     ssm.kernel_time_ms()                       # drop any earlier tally
     ssm.kernel_timing(True)                    # events around the dominant kernel of each call, on its stream
     job.timing_on = True
+    clocks.mark_start()
     for i in range(args.steps):
         flush_l2(flush)
         evs[i][0].record(stream)
         job.step()
         evs[i][1].record(stream)
     torch.cuda.synchronize()
+    clocks.mark_stop()
     ssm.kernel_timing(False)
     job.timing_on = False
     kern_ms_total, kern_launches = ssm.kernel_time_ms()
     if world > 1:
         dist.barrier()
-    clk = clocks.stop() if rank == 0 else None
     step_ms = [a.elapsed_time(b) for a, b in evs]
     total_ms = reduce_max_ms(float(sum(step_ms)), world, "cuda")
     # the dominant kernel's own average launch duration (max over ranks), for the roofline
@@ -607,6 +708,7 @@ def run_cuda(args):
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        clocks.mark_start(2)
         e0.record(stream)
         h2d = d2h = 0
         if pipelined:
@@ -616,12 +718,14 @@ def run_cuda(args):
                 h2d, d2h = job.e2e_step(out_host)
         e1.record(stream)
         torch.cuda.synchronize()
+        clocks.mark_stop()
         ems = reduce_max_ms(e0.elapsed_time(e1), world, "cuda")
         e2e = {"value": weak_scaling_value(job.units, ne, world, ems), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": ne,
                "copies": ("overlapped across steps: inputs in on one stream, y out on another, compute on a third; "
                           "device buffers double-buffered" if pipelined else "in order within each step")}
 
+    clk = clocks.stop() if rank == 0 else None
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

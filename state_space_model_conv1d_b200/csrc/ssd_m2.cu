@@ -897,18 +897,12 @@ ssd_state_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, cons
     const float A2 = a.A[hh] * kLog2e;
     const float dtb = a.dt_bias ? a.dt_bias[hh] : 0.f;
     const __nv_bfloat16 *dtg = a.dt + row * a.dt_bs + start * a.dt_ts + hh;
-    // delta of token t (lane l of half chunk hc: t = 32 hc + l) and its inclusive
-    // prefix of delta A over the half chunk
-    auto half_scan = [&](int hc, float &d, float &sc) {
-        const float u = __bfloat162float(dtg[((int64_t)hc * 32 + lane) * a.dt_ts]) + dtb;
-        d = a.softplus ? softplus(u) : u;
-        sc = d * A2;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float v = __shfl_up_sync(0xffffffffu, sc, o);
-            if (lane >= o) sc += v;
-        }
-    };
+    // Warp w takes the half chunks hc = w + 8 k (k < kMaxHc; lane l: token
+    // 32 hc + l): every dt load of the warp is issued first, then delta and its
+    // inclusive prefix of delta A over the half chunk stay in registers for both
+    // prologue passes.
+    constexpr int kMaxHc = 2 * kMaxSegChunks / kComputeWarps;
+    float dv[kMaxHc], sv[kMaxHc];
 
     if (tid == 0) {
         ax.abort = (a.err && *a.err != 0) ? 1 : 0;
@@ -921,10 +915,27 @@ ssd_state_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, cons
     if (warp == kComputeWarps) {
         tc::tmem_alloc(&ax.tmem, 64);
     } else {
-        for (int hc = warp; hc < 2 * n; hc += kComputeWarps) {
-            float d, sc;
-            half_scan(hc, d, sc);
-            if (lane == 31) ax.half[hc] = sc;
+#pragma unroll
+        for (int k = 0; k < kMaxHc; ++k) {
+            const int hc = warp + k * kComputeWarps;
+            dv[k] = hc < 2 * n ? __bfloat162float(dtg[((int64_t)hc * 32 + lane) * a.dt_ts]) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < kMaxHc; ++k) {
+            const int hc = warp + k * kComputeWarps;
+            if (hc < 2 * n) {                                 // uniform over the warp
+                const float u = dv[k] + dtb;
+                const float d = a.softplus ? softplus(u) : u;
+                float sc = d * A2;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float v = __shfl_up_sync(0xffffffffu, sc, o);
+                    if (lane >= o) sc += v;
+                }
+                dv[k] = d;
+                sv[k] = sc;
+                if (lane == 31) ax.half[hc] = sc;
+            }
         }
         // conv halo of chunk 0: the row's carried conv state before its first
         // segment, else the raw x rows before the segment
@@ -959,13 +970,15 @@ ssd_state_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, cons
     if (warp < kComputeWarps) {
         // X' weight of every token: the decay left in its chunk after it, then
         // that of the later chunks, times its delta
-        for (int hc = warp; hc < 2 * n; hc += kComputeWarps) {
-            const int c = hc >> 1;
-            float d, sc;
-            half_scan(hc, d, sc);
-            const float pre = (hc & 1) ? ax.half[hc - 1] : 0.f;
-            const float tot = ax.half[2 * c] + ax.half[2 * c + 1];
-            wt[hc * 32 + lane] = ex2((tot - (pre + sc)) + ax.suf[c + 1]) * d;
+#pragma unroll
+        for (int k = 0; k < kMaxHc; ++k) {
+            const int hc = warp + k * kComputeWarps;
+            if (hc < 2 * n) {
+                const int c = hc >> 1;
+                const float pre = (hc & 1) ? ax.half[hc - 1] : 0.f;
+                const float tot = ax.half[2 * c] + ax.half[2 * c + 1];
+                wt[hc * 32 + lane] = ex2((tot - (pre + sv[k])) + ax.suf[c + 1]) * dv[k];
+            }
         }
     }
     __syncthreads();
@@ -1105,11 +1118,13 @@ ssd_state_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, cons
 // ------------------------------------------------------------------ B / C pre-pass
 // Causal conv + SiLU of the B and C channels of x|B|C, once per group (every
 // head of the group reads the result), into bf16 [tokens][G*N] workspace
-// tiles.  One thread per (8 channels of B or C, 8 consecutive tokens): the
+// tiles.  One thread per (4 channels of B or C, 8 consecutive tokens): the
 // K-1 rows before the run are loaded first (from the sequence's carried conv
-// state before its first token), every row is one 16-byte load, and a warp
-// covers 32 consecutive channel vectors of one token row.  Packed sequences
-// restart the history at every sequence start.
+// state before its first token), every row is one 8-byte load issued before
+// any math, and a warp covers 32 consecutive channel vectors of one token
+// row.  Four channels rather than eight keep a thread at 92 registers, so
+// five CTAs (20 warps) fit per SM instead of three: the pass is bound by load
+// latency.  Packed sequences restart the history at every sequence start.
 struct BcArgs {
     const __nv_bfloat16 *B, *C;
     int64_t b_bs, b_ts, c_bs, c_ts;
@@ -1119,12 +1134,23 @@ struct BcArgs {
     const int32_t *cu;
     int nseqs;
     int64_t seqlen, GN, HP, cdim;
-    bool w16, b16;                    // taps / bias of every 8-channel vector start 16-byte aligned
+    bool w16, b16;                    // taps / bias of every 4-channel vector start 16-byte aligned
 };
 
+constexpr int kBcV = 4;               // channels per thread (one 8-byte row load)
+
+SSM_DEVINL void unpack_bf16x4(uint2 r, float (&v)[kBcV]) {
+    v[0] = __uint_as_float(r.x << 16); v[1] = __uint_as_float(r.x & 0xffff0000u);
+    v[2] = __uint_as_float(r.y << 16); v[3] = __uint_as_float(r.y & 0xffff0000u);
+}
+SSM_DEVINL uint2 pack_bf16x4(const float (&v)[kBcV]) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(v[0], v[1]), hi = __floats2bfloat162_rn(v[2], v[3]);
+    return make_uint2(*reinterpret_cast<const uint32_t *>(&lo), *reinterpret_cast<const uint32_t *>(&hi));
+}
+
 template <int K>
-__global__ void __launch_bounds__(128, 3) bc_conv_kernel(const BcArgs a) {
-    const int64_t nvec = a.GN / 4;                        // B and C vectors of one token row
+__global__ void __launch_bounds__(128, 5) bc_conv_kernel(const BcArgs a) {
+    const int64_t nvec = 2 * a.GN / kBcV;                 // B and C vectors of one token row
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t vec = idx % nvec, run = idx / nvec;
     const int64_t t0 = run * 8;
@@ -1141,36 +1167,35 @@ __global__ void __launch_bounds__(128, 3) bc_conv_kernel(const BcArgs a) {
     }
     if (t0 >= a.seqlen) return;
     const int which = vec >= nvec / 2;                    // 0: B, 1: C
-    const int64_t c0 = (vec - which * (nvec / 2)) * 8;    // channel within B (or C)
+    const int64_t c0 = (vec - which * (nvec / 2)) * kBcV; // channel within B (or C)
     const __nv_bfloat16 *src = which ? a.C + row * a.c_bs : a.B + row * a.b_bs;
     const int64_t ts = which ? a.c_ts : a.b_ts;
     __nv_bfloat16 *dst = (which ? a.oC : a.oB) + row * a.seqlen * a.GN + c0;
-    const int64_t cch = a.HP + which * a.GN + c0;         // conv channel of the first of the 8
-    if (!SSM_BOUNDS(c0 + 7, a.GN, BS_BC_CHANNEL) || !SSM_BOUNDS(row * a.seqlen + t0, (int64_t)gridDim.y * a.seqlen, BS_BC_ROW))
+    const int64_t cch = a.HP + which * a.GN + c0;         // conv channel of the first of the 4
+    if (!SSM_BOUNDS(c0 + kBcV - 1, a.GN, BS_BC_CHANNEL) ||
+        !SSM_BOUNDS(row * a.seqlen + t0, (int64_t)gridDim.y * a.seqlen, BS_BC_ROW))
         return;
-    // taps and bias of the 8 channels: 16-byte loads when they are aligned (the
-    // weight rows are contiguous: 8 channels x K taps), scalar loads otherwise
-    float wk[K][8], bb[8];
+    // taps and bias of the 4 channels: 16-byte loads when they are aligned (one
+    // channel's 4 taps; 4 biases), scalar loads otherwise
+    float wk[K][kBcV], bb[kBcV];
     if (K == 4 && a.w16) {
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
+        for (int v = 0; v < kBcV; ++v) {
             const float4 q = *reinterpret_cast<const float4 *>(a.w + (cch + v) * 4);
             wk[0][v] = q.x; wk[1 % K][v] = q.y; wk[2 % K][v] = q.z; wk[3 % K][v] = q.w;
         }
     } else {
 #pragma unroll
-        for (int v = 0; v < 8; ++v)
+        for (int v = 0; v < kBcV; ++v)
 #pragma unroll
             for (int k = 0; k < K; ++k) wk[k][v] = a.w[(cch + v) * K + k];
     }
     if (a.bias && a.b16) {
         const float4 b0 = *reinterpret_cast<const float4 *>(a.bias + cch);
-        const float4 b1 = *reinterpret_cast<const float4 *>(a.bias + cch + 4);
         bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w;
-        bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
     } else {
 #pragma unroll
-        for (int v = 0; v < 8; ++v) bb[v] = a.bias ? a.bias[cch + v] : 0.f;
+        for (int v = 0; v < kBcV; ++v) bb[v] = a.bias ? a.bias[cch + v] : 0.f;
     }
     // sequence of the run's first token and its bounds (clamped: a malformed
     // cu_seqlens gives wrong values but no out-of-bounds access)
@@ -1181,20 +1206,20 @@ __global__ void __launch_bounds__(128, 3) bc_conv_kernel(const BcArgs a) {
     }
     int64_t start = a.cu ? min(max((int64_t)a.cu[s], (int64_t)0), a.seqlen) : 0;
     int64_t end = a.cu ? min(max((int64_t)a.cu[s + 1], start), a.seqlen) : a.seqlen;
-    float hist[K > 1 ? K - 1 : 1][8];
+    float hist[K > 1 ? K - 1 : 1][kBcV];
     auto load_hist = [&](int64_t t) {
 #pragma unroll
         for (int j = 0; j < K - 1; ++j) {                 // hist[j] holds token t-(K-1)+j
             const int64_t tau = t - (K - 1) + j;
             if (tau >= start) {
-                Vec8<__nv_bfloat16>::ld(src + tau * ts + c0, hist[j]);
+                unpack_bf16x4(*reinterpret_cast<const uint2 *>(src + tau * ts + c0), hist[j]);
             } else {
                 const int64_t q = tau - start + (K - 1);
                 const bool in = a.state_in && q >= 0 &&
-                                SSM_BOUNDS(((int64_t)s * a.cdim + cch + 7) * (K - 1) + q,
+                                SSM_BOUNDS(((int64_t)s * a.cdim + cch + kBcV - 1) * (K - 1) + q,
                                            (int64_t)(a.cu ? a.nseqs : gridDim.y) * a.cdim * (K - 1), BS_BC_STATE);
 #pragma unroll
-                for (int v = 0; v < 8; ++v)
+                for (int v = 0; v < kBcV; ++v)
                     hist[j][v] = in ? __bfloat162float(a.state_in[((int64_t)s * a.cdim + cch + v) * (K - 1) + q]) : 0.f;
             }
         }
@@ -1202,10 +1227,10 @@ __global__ void __launch_bounds__(128, 3) bc_conv_kernel(const BcArgs a) {
     load_hist(t0);
     const int64_t t1 = min(t0 + 8, a.seqlen);
     // every row's load is issued before any math
-    uint4 rows[8];
+    uint2 rows[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-        if (t0 + i < t1) rows[i] = *reinterpret_cast<const uint4 *>(src + (t0 + i) * ts + c0);
+        if (t0 + i < t1) rows[i] = *reinterpret_cast<const uint2 *>(src + (t0 + i) * ts + c0);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t t = t0 + i;
@@ -1217,24 +1242,24 @@ __global__ void __launch_bounds__(128, 3) bc_conv_kernel(const BcArgs a) {
             if (t < start || t >= end) return;
             load_hist(t);
         }
-        float cur[8], o[8];
-        tc::unpack_bf16x8(rows[i], cur);
+        float cur[kBcV], o[kBcV];
+        unpack_bf16x4(rows[i], cur);
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
+        for (int v = 0; v < kBcV; ++v) {
             float acc = bb[v];
 #pragma unroll
             for (int k = 0; k < K - 1; ++k) acc = fmaf(wk[k][v], hist[k][v], acc);
             acc = fmaf(wk[K - 1][v], cur[v], acc);
             o[v] = silu_fast<__nv_bfloat16>(acc);
         }
-        *reinterpret_cast<uint4 *>(dst + t * a.GN) = tc::pack_bf16x8(o);
+        *reinterpret_cast<uint2 *>(dst + t * a.GN) = pack_bf16x4(o);
 #pragma unroll
         for (int k = 0; k + 1 < K - 1; ++k)
 #pragma unroll
-            for (int v = 0; v < 8; ++v) hist[k][v] = hist[k + 1][v];
+            for (int v = 0; v < kBcV; ++v) hist[k][v] = hist[k + 1][v];
         if (K > 1)
 #pragma unroll
-            for (int v = 0; v < 8; ++v) hist[K > 1 ? K - 2 : 0][v] = cur[v];
+            for (int v = 0; v < kBcV; ++v) hist[K > 1 ? K - 2 : 0][v] = cur[v];
     }
 }
 
@@ -1418,7 +1443,7 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
         // rows start 16-byte aligned whenever the arrays do
         b.w16 = ((uintptr_t)s.conv_w % 16) == 0;
         b.b16 = s.conv_b != nullptr && ((uintptr_t)s.conv_b % 16) == 0;
-        const int64_t threads = (s.seqlen + 7) / 8 * (GN / 4);
+        const int64_t threads = (s.seqlen + 7) / 8 * (2 * GN / kBcV);
         const dim3 bgrid((unsigned)((threads + 127) / 128), (unsigned)rows);
         if (threads > 0) {
             switch (s.d_conv) {
