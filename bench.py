@@ -88,7 +88,8 @@ def _nvml_poll(uuid, index, phase, done, ready, out):
                  "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
                  "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
         mx = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
-    except Exception:
+    except Exception as exc:
+        print(f"clock sampler: NVML unavailable ({exc!r})", file=sys.stderr, flush=True)
         ready.set()
         out.put(None)
         return
@@ -105,8 +106,7 @@ def _nvml_poll(uuid, index, phase, done, ready, out):
                 errors += 1
                 time.sleep(0.001)
                 continue
-            if phase.value == ph:                      # the phase did not end during the queries
-                samples.append((ph, sm, sorted(n for n, bit in names.items() if r & bit)))
+            samples.append((ph, sm, sorted(n for n, bit in names.items() if r & bit)))   # phase at the query's start
             time.sleep(0.0002)
         else:
             time.sleep(0.0005)
@@ -144,13 +144,16 @@ class ClockSampler:
             self.child = ctx.Process(target=_nvml_poll, args=(self.uuid, self.idx, self.phase, self.done, ready, self.q),
                                      daemon=True)
             self.child.start()
-            if ready.wait(timeout=30):
-                self.source = "nvml, back-to-back queries"
-                return
-            self.child.terminate()
-        except Exception:
-            pass
-        self.child = None
+            if ready.wait(timeout=60):
+                self.source = "nvml, every ~0.2 ms"
+            else:
+                print("clock sampler: NVML process did not start", file=sys.stderr, flush=True)
+                self.child.terminate()
+                self.child = None
+        except Exception as exc:
+            print(f"clock sampler: {exc!r}", file=sys.stderr, flush=True)
+            self.child = None
+        # nvidia-smi alongside: the fallback when NVML gives no sample of the timed region
         try:
             dev = self.uuid if self.uuid else str(self.idx)
             self.proc = subprocess.Popen(["nvidia-smi", "-i", dev, f"--query-gpu={self.FIELDS}",
@@ -158,7 +161,6 @@ class ClockSampler:
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
-            self.source = "nvidia-smi, 200 ms"
         except FileNotFoundError:
             self.proc = None
 
@@ -182,8 +184,12 @@ class ClockSampler:
             res = None
         self.child.join(timeout=5)
         if not res:
+            print("clock sampler: the NVML process returned nothing", file=sys.stderr, flush=True)
             return None
         mx, samples, errors = res
+        if not any(x[0] == 1 for x in samples):
+            print(f"clock sampler: {len(samples)} NVML samples, none in the timed region ({errors} query errors)",
+                  file=sys.stderr, flush=True)
         out = {}
         for ph, key in ((1, "timed"), (2, "e2e")):
             sm = [x[1] for x in samples if x[0] == ph]
@@ -198,8 +204,16 @@ class ClockSampler:
         return clk
 
     def stop(self):
-        if self.child is not None:
-            return self._stop_child()
+        clk = self._stop_child() if self.child is not None else None
+        smi = self._stop_smi()
+        if clk is not None:
+            return clk
+        if smi is not None:
+            print("clock sampler: no NVML sample of the timed region; nvidia-smi's window is reported",
+                  file=sys.stderr, flush=True)
+        return smi
+
+    def _stop_smi(self):
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -224,7 +238,7 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "reasons": sorted(reasons),
-                "samples": len(sm), "source": self.source}
+                "samples": len(sm), "source": "nvidia-smi, 200 ms, from 0.3 s before the timed region to its end"}
 
 
 # --------------------------------------------------------------- workloads

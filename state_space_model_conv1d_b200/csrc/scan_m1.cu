@@ -488,9 +488,10 @@ cudaError_t launch_typed(M1Args a, int nseqs, cudaStream_t st) {
 // state-spaces/mamba issue 285: the pair, composed associatively, seeded with
 // (1, h0) and carried across chunks in fp32).
 //
-// One CTA owns one sequence and TP_DB = 16 channels; 8 warps; chunks of
-// TP_TC = 64 tokens.  In the scan, warp w takes channels 2w and 2w + 1 in
-// turn, and lane l = 4 r + q takes the run of tokens 8r .. 8r+7 and the four
+// One CTA owns one sequence and DB = 16 channels (8 when 16 would leave SMs
+// without a CTA); 8 warps; chunks of TP_TC = 64 tokens.  In the scan, warp w
+// takes channels 2w and 2w + 1 in turn (channel w when DB = 8), and lane
+// l = 4 r + q takes the run of tokens 8r .. 8r+7 and the four
 // states 16 g + 4 q .. 16 g + 4 q + 3 of state group g.  Per (channel, group):
 //   1. each lane walks its run from the identity (1, 0):
 //      a_t = exp(delta_t A), P = prod a_t, Q = a_t Q + delta_t x_t B_t
@@ -506,14 +507,13 @@ cudaError_t launch_typed(M1Args a, int nseqs, cudaStream_t st) {
 // shuffle reduce-scatter over the four state lanes sums them (two tokens per
 // lane), then y = (sum + D xc) silu(z).
 //
-// A cooperative prologue per chunk (thread = channel x 4 tokens) computes the
+// A cooperative prologue per chunk (thread = channel x 4 or 2 tokens) computes the
 // conv + SiLU, delta = softplus(dt + dt_bias), delta xc, D xc and the gate,
 // and widens B / C to fp32, into shared-memory layouts padded so that both
 // the prologue's writes (lanes = channels) and the scan's reads (lanes = runs)
 // are free of bank conflicts.  Software pipeline, one barrier per chunk:
 // iteration c scans chunk c, stores y of chunk c-1, runs the prologue of chunk
 // c+1 and issues the copies of chunk c+2 (raw tiles double-buffered).
-constexpr int TP_DB = 16;            // channels per CTA
 constexpr int TP_TC = 64;            // tokens per chunk
 constexpr int TP_THREADS = 256;
 constexpr int TP_RUNS = 8;           // runs of 8 tokens per chunk (one per 4 lanes)
@@ -525,22 +525,22 @@ SSM_DEVINL int tp_dd(int c, int t) { return c * TP_CH_F2 + (t >> 3) * TP_RUN_F2 
 template <int N>
 SSM_DEVINL int tp_bc(int t, int n) { return t * N + (t >> 3) * 16 + n; }
 
-template <typename T, int N>
+template <typename T, int N, int DB>
 struct SmemTP {
     static constexpr int BCROWS = TP_TC * N + (TP_TC / 8) * 16;
-    T rx[2][TP_TC][TP_DB];
-    T rdt[2][TP_TC][TP_DB];
-    T rz[2][TP_TC][TP_DB];
+    T rx[2][TP_TC][DB];
+    T rdt[2][TP_TC][DB];
+    T rz[2][TP_TC][DB];
     T rB[2][TP_TC][N];
     T rC[2][TP_TC][N];
-    float halo[2][kHalo][TP_DB];
-    float2 dd[2][TP_DB * TP_CH_F2];      // (delta, delta * xc)
-    float2 ep[2][TP_DB * TP_CH_F2];      // (D * xc, gate)
+    float halo[2][kHalo][DB];
+    float2 dd[2][DB * TP_CH_F2];      // (delta, delta * xc)
+    float2 ep[2][DB * TP_CH_F2];      // (D * xc, gate)
     alignas(16) float Bf[2][BCROWS];
     alignas(16) float Cf[2][BCROWS];
-    float y[2][TP_TC][TP_DB + 1];        // +1: conflict-free column writes
-    alignas(16) float carry[TP_DB][N];   // state at the chunk start
-    alignas(16) float A2[TP_DB][N];      // A * log2(e)
+    float y[2][TP_TC][DB + 1];        // +1: conflict-free column writes
+    alignas(16) float carry[DB][N];   // state at the chunk start
+    alignas(16) float A2[DB][N];      // A * log2(e)
 };
 
 // rows [0, nv) x NCOLS columns of a token-major tensor -> dst[TP_TC][NCOLS]
@@ -564,15 +564,17 @@ SSM_DEVINL void tp_stage(T *dst, const T *src, int64_t ts, int nv, int64_t col0,
     }
 }
 
-template <typename T, int N, bool INTER>
+template <typename T, int N, int DB, bool INTER>
 __global__ void __launch_bounds__(TP_THREADS, 2)
 scan_m1_tp_kernel(const M1Args a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    auto &sm = *reinterpret_cast<SmemTP<T, N> *>(smem_raw);
+    auto &sm = *reinterpret_cast<SmemTP<T, N, DB> *>(smem_raw);
+    constexpr int TPR = TP_TC * DB / TP_THREADS;     // prologue tokens per thread
+    constexpr int CPW = DB / (TP_THREADS / 32);       // channels per warp in the scan
     constexpr int NG = N / 16;               // state groups of 16 (4 lanes x 4 states)
     if (a.sv.err && *a.sv.err != 0) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t d0 = (int64_t)blockIdx.x * TP_DB;
+    const int64_t d0 = (int64_t)blockIdx.x * DB;
     const int s = a.sv.order ? a.sv.order[blockIdx.y] : (int)blockIdx.y;
     int64_t start = 0, len = a.seqlen, row = s;
     if (a.sv.cu) {
@@ -600,18 +602,18 @@ scan_m1_tp_kernel(const M1Args a) {
         const int64_t t0 = (int64_t)c * TP_TC;
         const int nv = chunk_len(c);
         if (nv > 0) {
-            tp_stage<T, TP_DB>(&sm.rx[rb][0][0], xg + t0 * a.x_ts, a.x_ts, nv, d0, Dn, a.async_act);
-            tp_stage<T, TP_DB>(&sm.rdt[rb][0][0], dtg + t0 * a.dt_ts, a.dt_ts, nv, d0, Dn, a.async_act);
-            if (zg) tp_stage<T, TP_DB>(&sm.rz[rb][0][0], zg + t0 * a.z_ts, a.z_ts, nv, d0, Dn, a.async_act);
+            tp_stage<T, DB>(&sm.rx[rb][0][0], xg + t0 * a.x_ts, a.x_ts, nv, d0, Dn, a.async_act);
+            tp_stage<T, DB>(&sm.rdt[rb][0][0], dtg + t0 * a.dt_ts, a.dt_ts, nv, d0, Dn, a.async_act);
+            if (zg) tp_stage<T, DB>(&sm.rz[rb][0][0], zg + t0 * a.z_ts, a.z_ts, nv, d0, Dn, a.async_act);
             tp_stage<T, N>(&sm.rB[rb][0][0], Bg + t0 * a.B_ts, a.B_ts, nv, 0, N, a.async_bc);
             tp_stage<T, N>(&sm.rC[rb][0][0], Cg + t0 * a.C_ts, a.C_ts, nv, 0, N, a.async_bc);
         }
         cp_async_commit();
     };
 
-    // ---- prologue role: channel pc = tid % 16, tokens 4 * (tid / 16) .. + 3
-    const int pc = tid % TP_DB;
-    const int pt0 = (tid / TP_DB) * 4;
+    // ---- prologue role: channel pc = tid % DB, tokens TPR * (tid / DB) .. + TPR - 1
+    const int pc = tid % DB;
+    const int pt0 = (tid / DB) * TPR;
     const int64_t pch = d0 + pc;
     const bool pvalid = pch < Dn;
     float wr[4], cb = 0.f, dtb = 0.f;                  // taps right-aligned: wr[3] multiplies the current token
@@ -637,7 +639,7 @@ scan_m1_tp_kernel(const M1Args a) {
             if (K > 1) w2 = raw_at(pt0 - 1);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < TPR; ++i) {
             const int t = pt0 + i;
             float xcv = 0.f, dlt = 0.f, gv = 1.f;
             float cur = 0.f;
@@ -661,7 +663,7 @@ scan_m1_tp_kernel(const M1Args a) {
             sm.ep[wb][tp_dd(pc, t)] = make_float2(Dp * xcv, gv);
         }
         // halo of the next chunk: the last K-1 raw inputs up to this chunk's end
-        if (K > 1 && tid < TP_DB)
+        if (K > 1 && tid < DB)
             for (int j = 0; j < K - 1; ++j) {
                 const int v = nv - (K - 1) + j;
                 sm.halo[wb ^ 1][kHalo - (K - 1) + j][pc] = pvalid ? raw_at(v) : 0.f;
@@ -680,24 +682,24 @@ scan_m1_tp_kernel(const M1Args a) {
         const int yb = c & 1;
         const int nv = chunk_len(c);
         const int64_t t0 = (int64_t)c * TP_TC;
-        if (a.vec_y && d0 + TP_DB <= Dn) {
-            for (int i = tid; i < nv * (TP_DB / 8); i += TP_THREADS) {
-                const int r = i / (TP_DB / 8), v = i % (TP_DB / 8);
+        if (a.vec_y && d0 + DB <= Dn) {
+            for (int i = tid; i < nv * (DB / 8); i += TP_THREADS) {
+                const int r = i / (DB / 8), v = i % (DB / 8);
                 float o[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) o[e] = sm.y[yb][r][v * 8 + e];
                 if (SSM_BOUNDS(start + t0 + r, a.seqlen, BS_M1_Y)) Vec8<T>::st(yg + (t0 + r) * a.y_ts + d0 + v * 8, o);
             }
         } else {
-            for (int i = tid; i < nv * TP_DB; i += TP_THREADS) {
-                const int r = i / TP_DB, v = i % TP_DB;
+            for (int i = tid; i < nv * DB; i += TP_THREADS) {
+                const int r = i / DB, v = i % DB;
                 if (d0 + v < Dn && SSM_BOUNDS(start + t0 + r, a.seqlen, BS_M1_Y))
                     Elem<T>::st(yg + (t0 + r) * a.y_ts + d0 + v, sm.y[yb][r][v]);
             }
         }
     };
 
-    // ---- scan role: lane = 4 r + q (run r, state quarter q), channels 2 warp, 2 warp + 1
+    // ---- scan role: lane = 4 r + q (run r, state quarter q), channels CPW warp .. CPW warp + CPW - 1
     const int r = lane >> 2, q = lane & 3;
     // where the reduce-scatter leaves this lane's two tokens: 8 r + jb, 8 r + jb + 1
     const int jb = (q & 1) * 4 + (q & 2);
@@ -705,8 +707,8 @@ scan_m1_tp_kernel(const M1Args a) {
     auto scan = [&](int c) {
         const int wb = c & 1;
 #pragma unroll 1
-        for (int cc = 0; cc < 2; ++cc) {
-            const int ch = warp * 2 + cc;
+        for (int cc = 0; cc < CPW; ++cc) {
+            const int ch = warp * CPW + cc;
             float acc[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] = 0.f;
@@ -807,22 +809,22 @@ scan_m1_tp_kernel(const M1Args a) {
         const int64_t slot = a.iv.slot_after(s, (int64_t)(c + 1) * TP_TC);
         if (slot < 0 || !SSM_BOUNDS(slot, a.iv.nslots, BS_M1_POOL)) return;
         if (a.iv.states)
-            for (int i = tid; i < TP_DB * N; i += TP_THREADS) {
+            for (int i = tid; i < DB * N; i += TP_THREADS) {
                 const int cidx = i / N, n = i % N;
                 if (d0 + cidx < Dn) a.iv.states[(slot * Dn + d0 + cidx) * N + n] = sm.carry[cidx][n];
             }
         if (a.iv.conv && K > 1) {
             T *cdst = static_cast<T *>(a.iv.conv) + slot * Dn * (K - 1);
             const int hb = (c + 1) & 1;
-            for (int idx = tid; idx < (K - 1) * TP_DB; idx += TP_THREADS) {
-                const int j = idx / TP_DB, dd = idx % TP_DB;
+            for (int idx = tid; idx < (K - 1) * DB; idx += TP_THREADS) {
+                const int j = idx / DB, dd = idx % DB;
                 if (d0 + dd < Dn) Elem<T>::st(cdst + (d0 + dd) * (K - 1) + j, sm.halo[hb][kHalo - (K - 1) + j][dd]);
             }
         }
     };
 
     // ---- initial state, A, conv halo of chunk 0
-    for (int i = tid; i < TP_DB * N; i += TP_THREADS) {
+    for (int i = tid; i < DB * N; i += TP_THREADS) {
         const int cidx = i / N, n = i % N;
         const int64_t ch = d0 + cidx;
         const bool ok = ch < Dn;
@@ -831,8 +833,8 @@ scan_m1_tp_kernel(const M1Args a) {
     }
     if (K > 1) {
         const T *csi = static_cast<const T *>(a.conv_state_in);
-        for (int idx = tid; idx < (K - 1) * TP_DB; idx += TP_THREADS) {
-            const int j = idx / TP_DB, dd = idx % TP_DB;
+        for (int idx = tid; idx < (K - 1) * DB; idx += TP_THREADS) {
+            const int j = idx / DB, dd = idx % DB;
             const int64_t ch = d0 + dd;
             sm.halo[0][kHalo - (K - 1) + j][dd] =
                 (csi && ch < Dn) ? Elem<T>::ld(csi + ((int64_t)s * Dn + ch) * (K - 1) + j) : 0.f;
@@ -861,28 +863,28 @@ scan_m1_tp_kernel(const M1Args a) {
     if (K > 1 && a.conv_state_out) {
         T *cso = static_cast<T *>(a.conv_state_out);
         const int hb = nchunks & 1;
-        for (int idx = tid; idx < (K - 1) * TP_DB; idx += TP_THREADS) {
-            const int j = idx / TP_DB, dd = idx % TP_DB;
+        for (int idx = tid; idx < (K - 1) * DB; idx += TP_THREADS) {
+            const int j = idx / DB, dd = idx % DB;
             const int64_t ch = d0 + dd;
             if (ch < Dn) Elem<T>::st(cso + ((int64_t)s * Dn + ch) * (K - 1) + j, sm.halo[hb][kHalo - (K - 1) + j][dd]);
         }
     }
     cp_async_wait<0>();
     if (a.h_final)
-        for (int i = tid; i < TP_DB * N; i += TP_THREADS) {
+        for (int i = tid; i < DB * N; i += TP_THREADS) {
             const int cidx = i / N, n = i % N;
             const int64_t ch = d0 + cidx;
             if (ch < Dn) a.h_final[((int64_t)s * Dn + ch) * N + n] = sm.carry[cidx][n];
         }
 }
 
-template <typename T, int N>
+template <typename T, int N, int DB>
 cudaError_t launch_tp_n(const M1Args &a, int nseqs, cudaStream_t st) {
-    const size_t smem = sizeof(SmemTP<T, N>);
-    auto kern = a.iv.interval > 0 ? scan_m1_tp_kernel<T, N, true> : scan_m1_tp_kernel<T, N, false>;
+    const size_t smem = sizeof(SmemTP<T, N, DB>);
+    auto kern = a.iv.interval > 0 ? scan_m1_tp_kernel<T, N, DB, true> : scan_m1_tp_kernel<T, N, DB, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((a.Dn + TP_DB - 1) / TP_DB), (unsigned)nseqs);
+    dim3 grid((unsigned)((a.Dn + DB - 1) / DB), (unsigned)nseqs);
     timing_begin(st);
     kern<<<grid, TP_THREADS, smem, st>>>(a);
     timing_end(st);
@@ -897,7 +899,10 @@ cudaError_t launch_tp(M1Args a, int nseqs, cudaStream_t st) {
     constexpr int E = 16 / sizeof(T);
     // B / C rows: 16-byte copies when dstate fills whole vectors (16 and 32 do)
     a.async_bc = a.async_bc && a.N % E == 0;
-    return a.N == 16 ? launch_tp_n<T, 16>(a, nseqs, st) : launch_tp_n<T, 32>(a, nseqs, st);
+    // 8 channels per CTA (one warp per channel) when 16 would leave SMs without a CTA
+    if ((int64_t)nseqs * ((a.Dn + 15) / 16) < sm_count())
+        return a.N == 16 ? launch_tp_n<T, 16, 8>(a, nseqs, st) : launch_tp_n<T, 32, 8>(a, nseqs, st);
+    return a.N == 16 ? launch_tp_n<T, 16, 16>(a, nseqs, st) : launch_tp_n<T, 32, 16>(a, nseqs, st);
 }
 
 

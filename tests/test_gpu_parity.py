@@ -74,6 +74,8 @@ M1_CASES = [
     (2, 70, 24, 13, 4, "f32"),        # dstate not a multiple of 4
     (2, 65, 64, 16, 0, "bf16"),       # no conv in front
     (1, 2113, 48, 16, 4, "f32"),      # fp32 over many chunks (66 of 32 tokens) and a ragged tail
+    (4, 130, 640, 16, 4, "bf16"),     # time-parallel form with 16-channel blocks (160 CTAs)
+    (3, 200, 1000, 32, 3, "f32"),     # the same, dstate 32, a ragged channel block
 ]
 
 
