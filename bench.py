@@ -654,6 +654,22 @@ def rank_seed(base: int, rank: int) -> int:
     return base + 7919 * rank
 
 
+def gpu_local_cpus(device_index: int):
+    """The host CPUs NVML names as closest to this process's GPU (read-only
+    query; found by UUID), or None."""
+    try:
+        import torch
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(torch.cuda.get_device_properties(device_index).uuid))
+        words = pynvml.nvmlDeviceGetCpuAffinity(h, 64)
+        cpus = {64 * i + b for i, w in enumerate(words) for b in range(64) if (int(w) >> b) & 1}
+        cpus &= os.sched_getaffinity(0)
+        return cpus or None
+    except Exception:
+        return None
+
+
 def run_cuda(args):
     import torch
     import torch.distributed as dist
@@ -668,6 +684,13 @@ def run_cuda(args):
                                 device_id=torch.device("cuda", local))
     import state_space_model_conv1d_b200 as ssm
 
+    # Keep this process (and so its pinned host buffers) on the GPU's own CPU
+    # socket while the GPU runs: host<->device copies then cross no socket link.
+    # The full CPU set comes back for the CPU baseline.
+    all_cpus = os.sched_getaffinity(0)
+    near = gpu_local_cpus(local)
+    if near:
+        os.sched_setaffinity(0, near)
     w = W.WORKLOADS[args.workload]
     job = Job(w, rank, torch, ssm)
     flush = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
@@ -737,7 +760,9 @@ def run_cuda(args):
         e2e = {"value": weak_scaling_value(job.units, ne, world, ems), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "steps": ne,
                "copies": ("overlapped across steps: inputs in on one stream, y out on another, compute on a third; "
-                          "device buffers double-buffered" if pipelined else "in order within each step")}
+                          "device buffers double-buffered" if pipelined else "in order within each step"),
+               "host_cpus": (f"{len(near)} CPUs local to the GPU (NVML affinity), pinned buffers allocated there"
+                             if near else "unrestricted")}
 
     clk = clocks.stop() if rank == 0 else None
     if world > 1:
@@ -796,6 +821,7 @@ def run_cuda(args):
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
+        os.sched_setaffinity(0, all_cpus)
         cpu = cpu_baseline(w, args)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,

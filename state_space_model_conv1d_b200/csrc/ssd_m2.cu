@@ -39,8 +39,10 @@
 // chunks ahead, so no compute warp issues, waits to issue, or scans delta.
 // Compute iteration k:
 //   conv(k+1)   raw x -> X (double-buffered), X'             overlaps MMA Y(k)
-//   epilogue(k) y = (Y + exp(cs) Yo) silu(z) -> TMA store
-//   S(k)        S = exp(cs_Q) S + Sc (fp32 registers) -> bf16 copy for Yo(k+1)
+//   epilogue(k) y = (Y + exp(cs) Yo) silu(z) into the staging tile
+//   S(k)        S = exp(cs_Q) S + Sc (fp32 registers) -> bf16 copy for Yo(k+1),
+//               announced before the staging tile's TMA store (which waits for
+//               every warp), so Sc / Yo of k+1 do not wait for that barrier
 //   mask(k+1)   G -> M
 // and the control warp, for chunk k+1: G as soon as B / C have landed; the
 // raw x of chunk k+3 once conv(k+1) has read its staging buffer (raw x is
@@ -655,11 +657,6 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                 // z(k) has been read: the control warp may load z(k + 1)
                 __syncwarp();
                 if (lane == 0) mb_arrive(&ax.mb[MB_ZFREE]);
-                if (y_tma) {
-                    tc::fence_proxy_async();
-                    bar_compute();
-                    if (tid == 0 && !aborted(ax)) tc::tma_store_3d(&tm_y, (int)(hh * kP), (int)(start + t0), crow, stg);
-                }
                 {
                     const float2 dA2 = make_float2(tb.dAc, tb.dAc);
                     float Sc[32];
@@ -671,10 +668,16 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                         st16(smem + OFF_S + tc::off_sw128(sn, half * 32 + q * 8, 8192),
                              tc::pack_bf16x8(reinterpret_cast<const float *>(&S[q * 4])));
                 }
+                // the state is ready before the y store's barrier, so the control warp
+                // can issue Sc / Yo of the next chunk while the warps meet there
                 tc::fence_proxy_async();
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mb_arrive(&ax.mb[MB_SREADY]);
+                if (y_tma) {
+                    bar_compute();
+                    if (tid == 0 && !aborted(ax)) tc::tma_store_3d(&tm_y, (int)(hh * kP), (int)(start + t0), crow, stg);
+                }
                 // intermediate state after this chunk when it closes a state interval
                 if (a.iv.interval > 0 && nv == kQ && !aborted(ax)) {
                     const int64_t slot = a.iv.slot_after(s, seg_off() + t0 + kQ);
