@@ -39,10 +39,10 @@
 // chunks ahead, so no compute warp issues, waits to issue, or scans delta.
 // Compute iteration k:
 //   conv(k+1)   raw x -> X (double-buffered), X'             overlaps MMA Y(k)
-//   epilogue(k) y = (Y + exp(cs) Yo) silu(z) into the staging tile
+//   epilogue(k) y = (Y + exp(cs) Yo) silu(z), written over z(k) in the z tile
 //   S(k)        S = exp(cs_Q) S + Sc (fp32 registers) -> bf16 copy for Yo(k+1),
-//               announced before the staging tile's TMA store (which waits for
-//               every warp), so Sc / Yo of k+1 do not wait for that barrier
+//               announced before the y tile's TMA store (which waits for every
+//               warp), so Sc / Yo of k+1 do not wait for that barrier
 //   mask(k+1)   G -> M
 // and the control warp, for chunk k+1: G as soon as B / C have landed; the
 // raw x of chunk k+3 once conv(k+1) has read its staging buffer (raw x is
@@ -84,10 +84,10 @@ constexpr uint32_t OFF_C = 0;          // C rows i, K = n: two 8 KB K-atoms (n 0
 constexpr uint32_t OFF_B = 16384;      // B rows j, K = n (G); read as MN-major MN = n, K = j (Sc)
 constexpr uint32_t OFF_S = 32768;      // bf16 S rows n, 64 p each: MN-major MN = p, K = n (Yo)
 constexpr uint32_t OFF_M = 49152;      // M rows i, K = j (blocks above the diagonal stay zero)
-constexpr uint32_t OFF_X = 57344;      // X rows j, 64 p: two buffers (chunk parity); y staging
+constexpr uint32_t OFF_X = 57344;      // X rows j, 64 p: two buffers (chunk parity)
 constexpr uint32_t OFF_XP = 73728;     // X' rows j, 64 p
 constexpr uint32_t OFF_XR = 81920;     // raw x rows (row-major, 128 bytes each): two buffers
-constexpr uint32_t OFF_Z = 98304;      // z rows i, 64 p (128-byte swizzle)
+constexpr uint32_t OFF_Z = 98304;      // z rows i, 64 p (128-byte swizzle); y staged over it
 constexpr uint32_t OFF_AUX = 106496;
 
 // per-chunk decay tables (three slots: chunk c lives in slot c % 3 and is read
@@ -192,7 +192,7 @@ SSM_DEVINL float2 conv_silu2(float2 cur, float2 h2, float2 h1, float2 h0, float2
 //   tm_x  raw x, box 64 x 64 rows, no swizzle    -> row-major staging rows of 128 bytes
 //   tm_b, tm_c  conv'd B / C, box 64 x 64, 128-byte swizzle -> one K-atom of the operand tile
 //   tm_z  z, box 64 x 64, 128-byte swizzle       -> the z tile the epilogue reads
-//   tm_y  y, box 64 x 64, 128-byte swizzle       <- the y staging tile (rows past the tensor are skipped)
+//   tm_y  y, box 64 x 64, 128-byte swizzle       <- the z tile holding y (rows past the tensor are skipped)
 __global__ void __launch_bounds__(kThreads, 2)
 ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
            const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_z,
@@ -238,7 +238,7 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
         // one thread reads the error word, so every thread of the CTA takes the same branch below
         ax.abort = (a.sv.err && *a.sv.err != 0) ? 1 : 0;
         for (int i = 0; i < kNumMbar; ++i)
-            tc::mbar_init(&ax.mb[i], (i == MB_CONV || i == MB_ZFREE || i == MB_SREADY || i == MB_MREADY) ? kComputeWarps : 1);
+            tc::mbar_init(&ax.mb[i], (i == MB_CONV || i == MB_SREADY || i == MB_MREADY) ? kComputeWarps : 1);
         tc::mbar_init_fence();
         if (n > 0) {                       // a CTA with no chunk touches no tensor map
             tc::prefetch_map(&tm_x);
@@ -525,11 +525,9 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
         // frag_off + (((4 half + k) ^ (lane / 4)) << 4); row i1 is 1024 bytes further
         const uint32_t frag_off = (uint32_t)q4 * 2048u + (uint32_t)(lane >> 2) * 128u + (uint32_t)(lane & 3) * 4u;
 
+        bar_compute();                    // the chunk-0 halo and the initial state tile are written
         for (int k = -1; k < n; ++k) {
             const int c1 = k + 1;
-            // the y staging of chunk k - 1 sat in the X buffer conv(c1) writes now
-            if (tid == 0) tc::bulk_wait_read();
-            bar_compute();
 
             // ---- conv(c1): raw x rows -> X and X' (bf16, swizzled), halo of chunk c1 + 1
             if (c1 < n) {
@@ -600,7 +598,7 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                 const int64_t t0 = (int64_t)k * kQ;
                 const int nv = (int)min((int64_t)kQ, len - t0);
                 const Tables &tb = ax.tab[k % 3];
-                unsigned char *stg = smem + OFF_X + (k & 1) * 8192;
+                unsigned char *stg = smem + OFF_Z;     // y is staged over z, element by element
                 // Whole chunks (and the tensor's last, clipped chunk) leave through a TMA
                 // store of the staging tile; the partial last chunk of a packed sequence
                 // is stored directly.
@@ -654,9 +652,6 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                     if (y_tma) epi(std::true_type{});
                     else epi(std::false_type{});
                 }
-                // z(k) has been read: the control warp may load z(k + 1)
-                __syncwarp();
-                if (lane == 0) mb_arrive(&ax.mb[MB_ZFREE]);
                 {
                     const float2 dA2 = make_float2(tb.dAc, tb.dAc);
                     float Sc[32];
@@ -674,9 +669,15 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mb_arrive(&ax.mb[MB_SREADY]);
-                if (y_tma) {
-                    bar_compute();
-                    if (tid == 0 && !aborted(ax)) tc::tma_store_3d(&tm_y, (int)(hh * kP), (int)(start + t0), crow, stg);
+                // every warp has staged its y: store the tile, and once the store has read
+                // it the z tile is free for the control warp to load z(k + 1)
+                bar_compute();
+                if (tid == 0) {
+                    if (y_tma && !aborted(ax)) {
+                        tc::tma_store_3d(&tm_y, (int)(hh * kP), (int)(start + t0), crow, stg);
+                        tc::bulk_wait_read();
+                    }
+                    mb_arrive(&ax.mb[MB_ZFREE]);
                 }
                 // intermediate state after this chunk when it closes a state interval
                 if (a.iv.interval > 0 && nv == kQ && !aborted(ax)) {
