@@ -306,6 +306,8 @@ SSM_API ssm_status ssm_kernel_time_ms(float *total_ms, int32_t *launches);
  * address.  A malformed cu_seqlens leaves every output (y, h_final,
  * conv_state_out) unwritten, as in ssm_scan_fwd; a bounded wait that runs
  * out (SSM_DEVERR_TIMEOUT) can leave them partly written. */
+/* With segments = 0, a call that would fit the scratch only with its rows
+ * kept whole runs them whole. */
 #define SSM_NOALLOC_SCRATCH_BYTES (4u << 20)
 SSM_API ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *args, void *stream);
 

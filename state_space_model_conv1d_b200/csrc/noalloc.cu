@@ -53,7 +53,16 @@ extern "C" {
 
 ssm_status ssm_scan_fwd_noalloc(const ssm_scan_args *args, void *stream) {
     if (!args) return SSM_ERR_INVALID_ARG;
-    const size_t need = ssm_scan_workspace_size(args);
+    size_t need = ssm_scan_workspace_size(args);
+    ssm_scan_args whole;
+    if (need > (size_t)SSM_NOALLOC_SCRATCH_BYTES && args->segments == 0) {
+        // the library's choice of token segments keeps their states in the
+        // workspace: without them the call may still fit the fixed scratch
+        whole = *args;
+        whole.segments = 1;
+        need = ssm_scan_workspace_size(&whole);
+        args = &whole;
+    }
     if (need > (size_t)SSM_NOALLOC_SCRATCH_BYTES) return SSM_ERR_WORKSPACE;
     void *ws = nullptr;
     if (need > 0) {

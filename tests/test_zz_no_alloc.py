@@ -77,3 +77,27 @@ def test_noalloc_rejects_oversized_workspace():
                        None, None, t["conv_w"], None, None, None, y, True, 0)
     st = _abi.lib().ssm_scan_fwd_noalloc(C.byref(a), C.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == _abi.SSM_ERR_WORKSPACE
+
+
+def test_noalloc_keeps_rows_whole_when_segment_states_do_not_fit():
+    """A fixed-length batch the library would cut into token segments needs
+    their states in the workspace (over the fixed scratch here); the no-alloc
+    entry point then runs the rows whole, bit for bit like segments=1."""
+    d = W.mamba2_inputs(912, 2, 1024, 8, 64, 1, 128, dtype="bf16", conv_state=True)
+    t = to_dev(d, "bf16")
+    kw = dict(conv_w=t["conv_w"])
+    assert ssm.scan_segments(oracle.MAMBA2, t["x"], t["dt"], t["A"], t["B"], t["C"], z=t["z"], **kw) > 1
+    assert ssm.scan_workspace_size(oracle.MAMBA2, t["x"], t["dt"], t["A"], t["B"], t["C"], **kw) > 4 << 20
+    assert ssm.scan_workspace_size(oracle.MAMBA2, t["x"], t["dt"], t["A"], t["B"], t["C"], segments=1, **kw) <= 4 << 20
+    y_ref, h_ref, c_ref = ssm.scan_fwd(oracle.MAMBA2, t["x"], t["dt"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"],
+                                       dt_bias=t["dt_bias"], h0=t["h0"], conv_w=t["conv_w"], conv_b=t["conv_b"],
+                                       conv_state_in=t["conv_state_in"], segments=1)
+    y = torch.full_like(y_ref, float("nan"))
+    hf = torch.full_like(h_ref, float("nan"))
+    cso = torch.full_like(c_ref, float("nan"))
+    t["cu_seqlens"] = None
+    _noalloc(t, y, hf, cso)
+    torch.cuda.synchronize()
+    for got, ref, what in ((y, y_ref, "y"), (hf, h_ref, "h_final"), (cso, c_ref, "conv_state_out")):
+        ib = torch.int16 if got.dtype == torch.bfloat16 else torch.int32
+        assert torch.equal(got.view(ib), ref.view(ib)), f"{what}: not bit-identical to whole rows"
