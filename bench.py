@@ -773,6 +773,7 @@ def run_cuda(args):
 
     peaks, peak_src = load_peaks()
     hbm_peak = float(peaks["hbm_gbs"])
+    src = lambda key: f"measured (MEASURED_PEAKS.json {key})" if peak_src == "measured" else f"fallback ({key})"
     gbs = job.bytes_per_step / (ms_per_step / 1e3) / 1e9
     kbytes = job.fix_bytes if job.split is not None else job.bytes_per_step   # the timed kernel's own bytes
     kgbs = kbytes / (kern_ms / 1e3) / 1e9 if kern_ms > 0 else gbs
@@ -792,21 +793,21 @@ def run_cuda(args):
                     "frac": achieved / peak_g, "traffic": traffic, "kernel": job.kernel,
                     "peak_source": f"derived: {NUM_SMS} SMs x {MUFU_PER_CLK_PER_SM} MUFU ex2/clk x {clock_mhz:.0f} MHz",
                     "hbm": {"achieved": kgbs, "peak": hbm_peak, "unit": "GB/s", "frac": kgbs / hbm_peak,
-                            "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback"}}
+                            "peak_source": src("hbm_gbs")}}
     else:
         roofline = {"bound": "hbm", "achieved": kgbs, "peak": hbm_peak, "unit": "GB/s", "frac": kgbs / hbm_peak,
                     "traffic": traffic, "kernel": job.kernel,
-                    "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback"}
+                    "peak_source": src("hbm_gbs")}
         if job.flops:
             tf = job.flops / (kern_ms / 1e3) / 1e12
             tpk = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1400.0)))
             roofline["tensor"] = {"achieved": tf, "peak": tpk, "unit": "TFLOP/s", "frac": tf / tpk,
-                                  "flops_per_step": int(job.flops), "peak_source": "MEASURED_PEAKS.json bf16_tflops_sustained"}
+                                  "flops_per_step": int(job.flops), "peak_source": src("bf16_tflops_sustained")}
     if job.split is not None and job.fix_flops and job.kernel == "split_fixup_tc_kernel":
         tpk = float(peaks.get("bf16_tflops", 1590.0))
         ftf = job.fix_flops / (kern_ms / 1e3) / 1e12
         roofline["tensor"] = {"achieved": ftf, "peak": tpk, "unit": "TFLOP/s", "frac": ftf / tpk,
-                              "flops_per_launch": int(job.fix_flops), "peak_source": "MEASURED_PEAKS.json bf16_tflops"}
+                              "flops_per_launch": int(job.fix_flops), "peak_source": src("bf16_tflops")}
     elif job.split is not None and job.fix_flops:
         fma_peak = NUM_SMS * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
         ftf = job.fix_flops / (kern_ms / 1e3) / 1e12

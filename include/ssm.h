@@ -173,10 +173,13 @@ typedef struct ssm_scan_args {
     int64_t inter_nslots;         /* pool rows (>= 0) */
     float *inter_states;          /* [inter_nslots][state size] fp32, rows laid out as h_final's; may be NULL */
     void *inter_conv;             /* [inter_nslots][conv_dim][K-1] in dtype; may be NULL */
-    /* Token segments of the Mamba-2 tensor-core path (rows without
-     * cu_seqlens; ignored elsewhere): 0 lets the library choose, 1 keeps one
-     * CTA per (row, head), n >= 2 cuts every row into about n runs of whole
-     * 64-token chunks that separate CTAs scan at the same time.  Each run's
+    /* Token segments of the Mamba-2 tensor-core path (ignored elsewhere): 0
+     * lets the library choose, 1 keeps one CTA per (sequence, head), n >= 2
+     * cuts every row into about n runs of whole 64-token chunks that separate
+     * CTAs scan at the same time.  Packed sequences (cu_seqlens) are cut into
+     * runs of one length for all of them, chosen from the total: about n runs
+     * for a sequence of the mean length; the library cuts them only when the
+     * sequences x heads leave the GPU short of CTAs.  Each run's
      * entering state comes from a state-only pass over the runs before it (the
      * pair (exp(delta A), h) composes associatively, seed (1, h0): "Adding
      * Initial Value Support to Selective Scan Forward Kernel"), so results
@@ -251,8 +254,11 @@ SSM_API ssm_status ssm_conv1d_fwd(const ssm_conv_args *args, void *stream);
  * the choice of token segments depends on. */
 SSM_API size_t ssm_scan_workspace_size(const ssm_scan_args *args);
 /* Token segments ssm_scan_fwd cuts every row into for these arguments: 1 when
- * rows stay whole (packed sequences, Mamba-1, the SIMT Mamba-2 path, rows of
- * one chunk), 0 for arguments ssm_scan_fwd would reject.  Launches nothing. */
+ * rows stay whole (Mamba-1, the SIMT Mamba-2 path, rows of one chunk), 0 for
+ * arguments ssm_scan_fwd would reject.  For packed sequences, which are cut on
+ * the device, it is 1 or, when they are cut, the bound nseqs + ceil(total /
+ * run length) on the runs of all sequences together (the CTA rows launched).
+ * Launches nothing. */
 SSM_API int64_t ssm_scan_segments(const ssm_scan_args *args);
 
 /* Forward scan.  `workspace` (device, 256-byte aligned, ws_bytes long) may be

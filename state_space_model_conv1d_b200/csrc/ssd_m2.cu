@@ -17,10 +17,11 @@
 // ssd_state_passing, ssd_chunk_scan) are these four steps; here they are one
 // kernel whose carried state never leaves the SM.
 //
-// Work: one CTA per (sequence, head), two CTAs per SM; fixed-length rows that
-// leave the GPU short of CTAs are cut into token segments, one CTA per
-// (segment, head), seeded by a state-only pass (the segment-states section
-// below).  The B / C causal conv + SiLU is shared by the heads of a group, so
+// Work: one CTA per (sequence, head), two CTAs per SM; sequences that leave
+// the GPU short of CTAs are cut into token segments, one CTA per (segment,
+// head), seeded by a state-only pass (the segment-states section below).
+// Fixed-length rows are cut on the host; packed sequences, whose lengths only
+// the device holds, by a segment table a one-CTA pre-pass writes.  The B / C causal conv + SiLU is shared by the heads of a group, so
 // it runs once per group in a pre-pass that writes bf16 B, C into the
 // workspace; the x conv + SiLU runs here.  Per chunk of Q = 64 tokens, four
 // tensor-core products:
@@ -138,16 +139,40 @@ struct SsdArgs {
     InterView iv;
     const __nv_bfloat16 *Braw, *Craw;   // the unconvolved B / C (intermediate conv history)
     int64_t braw_bs, braw_ts, craw_bs, craw_ts;
-    // Segments (fixed-length batches only; nseg = 1 otherwise): row s is cut into
+    // Segments of fixed-length rows (nseg = 1 otherwise): row s is cut into
     // nseg runs of seg_len tokens (whole chunks; the last one takes the rest).
     // sloc / slog hold, for every segment but the last, the state it leaves when
-    // scanned from zero and its total log2-decay ([s][sg][H] rows of P x N, [s][sg][H]).
+    // scanned from zero and its total log2-decay ([s][sg][H] rows of P x N, [s][sg][H];
+    // for packed sequences [table entry][H]).
     int nseg;
     int64_t seg_len;
     float *sloc, *slog;
+    // Packed sequences cut on the device: entry y of seg_tab is (sequence,
+    // segment, segments of the sequence, sloc row of its segment 0); CTAs
+    // from *seg_count on have no segment.  Null otherwise.
+    const int4 *seg_tab;
+    const int32_t *seg_count;
+    int64_t nsloc;                      // rows of sloc / slog
 };
 
 SSM_DEVINL void st16(void *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
+
+// The segment a CTA row scans: its index within the sequence, whether it is
+// the sequence's last, and the sloc / slog row of the sequence's segment 0.
+SSM_DEVINL int seg_index(const SsdArgs &a) {
+    if (a.seg_tab) return a.seg_tab[blockIdx.y].y;
+    return a.sv.order ? 0 : (int)blockIdx.y % a.nseg;
+}
+SSM_DEVINL bool seg_is_last(const SsdArgs &a) {
+    if (a.seg_tab) {
+        const int4 e = a.seg_tab[blockIdx.y];
+        return e.y == e.z - 1;
+    }
+    return a.sv.order || (int)blockIdx.y % a.nseg == a.nseg - 1;
+}
+SSM_DEVINL int64_t seg_row0(const SsdArgs &a, int s) {
+    return a.seg_tab ? (int64_t)a.seg_tab[blockIdx.y].w : (int64_t)s * (a.nseg - 1);
+}
 SSM_DEVINL void bar_compute() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
 SSM_DEVINL void mb_arrive(uint64_t *mbar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(tc::smem_u32(mbar)) : "memory");
@@ -204,10 +229,14 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int hh = blockIdx.x;
-    // sequence s, segment sg of it (packed sequences and plain rows without
-    // segments: sg = 0 and the segment is the whole sequence)
-    const int s = a.sv.order ? a.sv.order[blockIdx.y] : (int)blockIdx.y / a.nseg;
-    const int sg = a.sv.order ? 0 : (int)blockIdx.y % a.nseg;
+    // sequence s, segment sg of it: from the segment table when packed
+    // sequences are cut (rows past its count have none), else packed sequences
+    // in schedule order and plain rows without segments have sg = 0 and the
+    // segment is the whole sequence
+    if (a.seg_tab && (int)blockIdx.y >= *a.seg_count) return;
+    const int s = a.seg_tab ? a.seg_tab[blockIdx.y].x
+                            : a.sv.order ? a.sv.order[blockIdx.y] : (int)blockIdx.y / a.nseg;
+    const int sg = seg_index(a);
     int64_t seq_start = 0, seq_len = a.seqlen, row = s;
     if (a.sv.cu) {
         const int64_t c0 = min(max((int64_t)a.sv.cu[s], (int64_t)0), a.seqlen);
@@ -218,7 +247,7 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
     const int64_t len = max(min(a.seg_len, seq_len - (int64_t)sg * a.seg_len), (int64_t)0);
     // tokens of the sequence before the segment, recomputed where needed (keeps
     // it out of the registers the chunk loop holds)
-    auto seg_off = [&]() -> int64_t { return a.sv.order ? 0 : (int64_t)((int)blockIdx.y % a.nseg) * a.seg_len; };
+    auto seg_off = [&]() -> int64_t { return (int64_t)seg_index(a) * a.seg_len; };
     const int64_t H = a.H, g = hh / (H / a.G);
     const int K = a.K;
     const int n = (int)((len + kQ - 1) / kQ);
@@ -230,7 +259,8 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
         !SSM_BOUNDS((int64_t)g0 + kN - 1, a.G * kN, BS_SSD_GROUP) ||
         !SSM_BOUNDS((int64_t)s * H + hh, (int64_t)a.sv.nseqs * H, BS_SSD_STATE) ||
         !SSM_BOUNDS(((int64_t)s + 1) * a.cdim - 1, (int64_t)a.sv.nseqs * a.cdim, BS_SSD_CONV_STATE) ||
-        !SSM_BOUNDS(sg, a.nseg, BS_SSD_SEGMENT))
+        !SSM_BOUNDS(sg, a.seg_tab ? a.nsloc : a.nseg, BS_SSD_SEGMENT) ||
+        (sg > 0 && !SSM_BOUNDS(seg_row0(a, s) + sg - 1, a.nsloc, BS_SSD_SEGMENT)))
         return;
     const float A2 = a.A[hh] * kLog2e;
 
@@ -486,8 +516,9 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
                            : make_float2(0.f, 0.f);
             // the state entering segment sg: fold (exp(cs_end), S_loc) of every
             // segment before it onto h0, in order
+            const int64_t q0 = sg > 0 ? seg_row0(a, s) : 0;
             for (int t = 0; t < sg; ++t) {
-                const int64_t q = ((int64_t)s * (a.nseg - 1) + t) * H + hh;
+                const int64_t q = (q0 + t) * H + hh;
                 const float e = ex2(a.slog[q]);
                 const float2 e2 = make_float2(e, e);
                 const float *lp = a.sloc + q * kP * kN;
@@ -783,7 +814,7 @@ ssd_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, const __gr
             }
         }
         if (tid == 0) tc::bulk_wait_all();
-        if (!aborted(ax) && (a.sv.order || (int)blockIdx.y % a.nseg == a.nseg - 1)) {   // the last segment
+        if (!aborted(ax) && seg_is_last(a)) {   // the last segment
             if (a.h_final) {
                 float *hf = a.h_final + ((int64_t)s * H + hh) * kP * kN;
 #pragma unroll
@@ -886,17 +917,30 @@ ssd_state_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap tm_x, cons
     float *wt = reinterpret_cast<float *>(smem + ST_OFF_W);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int hh = blockIdx.x;
-    const int nsp = a.nseg - 1;                           // segments that have a successor
-    const int s = (int)blockIdx.y / nsp, sg = (int)blockIdx.y % nsp;
-    const int64_t start = (int64_t)sg * a.seg_len, row = s;
+    // sequence s and segment sg (one with a successor): from the segment table
+    // for packed sequences (the row of a last segment has nothing to do), else
+    // nseg - 1 rows per fixed-length row
+    int s, sg;
+    int64_t start, row, qrow;
+    if (a.seg_tab) {
+        if ((int)blockIdx.y >= *a.seg_count) return;
+        const int4 e = a.seg_tab[blockIdx.y];
+        if (e.y >= e.z - 1) return;
+        s = e.x; sg = e.y; row = 0; qrow = (int64_t)e.w + e.y;
+        start = min(max((int64_t)a.sv.cu[s], (int64_t)0), a.seqlen) + (int64_t)sg * a.seg_len;
+    } else {
+        const int nsp = a.nseg - 1;                       // segments that have a successor
+        s = (int)blockIdx.y / nsp; sg = (int)blockIdx.y % nsp;
+        start = (int64_t)sg * a.seg_len; row = s; qrow = (int64_t)s * nsp + sg;
+    }
     const int n = (int)(a.seg_len / kQ);                  // only whole segments come here
     const int64_t H = a.H, g = hh / (H / a.G);
     const int crow = (int)row, g0 = (int)(g * kN), K = a.K;
-    const int64_t q = ((int64_t)s * nsp + sg) * H + hh;   // row of sloc / slog
+    const int64_t q = qrow * H + hh;                      // row of sloc / slog
     if (!SSM_BOUNDS(start + a.seg_len - 1, a.seqlen, BS_SSD_SEQ) || !SSM_BOUNDS(n - 1, kMaxSegChunks, BS_SSD_SEGMENT) ||
         !SSM_BOUNDS((int64_t)hh * kP + kP - 1, a.H * kP, BS_SSD_HEAD) ||
         !SSM_BOUNDS((int64_t)g0 + kN - 1, a.G * kN, BS_SSD_GROUP) ||
-        !SSM_BOUNDS(q, (int64_t)a.sv.nseqs * nsp * H, BS_SSD_STATE))
+        !SSM_BOUNDS(q, a.nsloc * H, BS_SSD_STATE))
         return;
     const float A2 = a.A[hh] * kLog2e;
     const float dtb = a.dt_bias ? a.dt_bias[hh] : 0.f;
@@ -1267,6 +1311,48 @@ __global__ void __launch_bounds__(128, 5) bc_conv_kernel(const BcArgs a) {
     }
 }
 
+// Segment table of packed sequences: in schedule order (longest first), each
+// sequence of length len gets max(1, ceil(len / seg_len)) consecutive entries
+// (sequence, segment, its segment count, the entry of its segment 0).  One
+// CTA; a block-wide prefix sum over tiles of sequences.  Nothing is listed
+// when the pre-pass found cu_seqlens malformed.
+constexpr int kSegTabThreads = 1024;
+__global__ void __launch_bounds__(kSegTabThreads)
+seg_table_kernel(const int32_t *__restrict__ cu, const int32_t *__restrict__ order, const int32_t *err, int nseqs,
+                 int64_t total, int64_t seg_len, int max_entries, int4 *__restrict__ tab, int32_t *count) {
+    __shared__ int sh[kSegTabThreads];
+    const int tid = threadIdx.x;
+    if (err && *err != 0) {
+        if (tid == 0) *count = 0;
+        return;
+    }
+    int carry = 0;
+    for (int p0 = 0; p0 < nseqs; p0 += kSegTabThreads) {
+        const int p = p0 + tid;
+        int sq = -1, ns = 0;
+        if (p < nseqs) {
+            sq = order ? order[p] : p;
+            const int64_t c0 = min(max((int64_t)cu[sq], (int64_t)0), total);
+            const int64_t c1 = min(max((int64_t)cu[sq + 1], c0), total);
+            ns = (int)max((int64_t)1, (c1 - c0 + seg_len - 1) / seg_len);
+        }
+        sh[tid] = ns;
+        __syncthreads();
+        for (int o = 1; o < kSegTabThreads; o <<= 1) {        // inclusive scan
+            const int v = tid >= o ? sh[tid - o] : 0;
+            __syncthreads();
+            sh[tid] += v;
+            __syncthreads();
+        }
+        const int base = carry + sh[tid] - ns;
+        for (int j = 0; j < ns; ++j)
+            if (base + j < max_entries) tab[base + j] = make_int4(sq, j, ns, base);
+        carry += sh[kSegTabThreads - 1];
+        __syncthreads();
+    }
+    if (tid == 0) *count = min(carry, max_entries);
+}
+
 }  // namespace
 
 bool ssd_shape_ok(const ssm_scan_args &s) {
@@ -1297,12 +1383,44 @@ inline size_t round256(size_t v) { return (v + 255) / 256 * 256; }
 //   state  waves x (0.45 chunks per run + 2.5)               (prologue)
 // A candidate must beat the whole-row plan by 3%.
 struct SegPlan {
-    int nseg;
+    int nseg;                           // fixed-length rows: segments per row
     int64_t seg_len;
+    int64_t nslots = 0;                 // packed sequences: (segment) CTA rows launched, 0 = not cut
 };
+// Packed sequences (lengths known on the device only): every sequence is cut
+// into ceil(len / seg_len) segments of seg_len tokens (at least one), listed
+// by a device pre-pass; nseqs + total / seg_len rows bound their count.  Cut
+// when requested (segments >= 2: about that many runs for a sequence of the
+// mean length) or, when chosen, if the sequences x heads give fewer chains
+// than the GPU has CTA slots and the mean sequence spans two runs of the
+// shortest length (4 chunks; shorter work would not pay for the extra
+// launches): then seg_len aims at about two waves of (segment, head) CTAs,
+// 4 to kMaxSegChunks chunks.
+SegPlan plan_packed(const ssm_scan_args &s) {
+    SegPlan one{1, s.seqlen > 0 ? s.seqlen : 1};
+    if (s.segments == 1 || s.nseqs <= 0 || s.seqlen <= kQ) return one;
+    const int64_t nch = (s.seqlen + kQ - 1) / kQ;
+    const double slots = 2.0 * sm_count();
+    int64_t per;
+    if (s.segments >= 2) {
+        per = (nch + (int64_t)s.nseqs * s.segments - 1) / ((int64_t)s.nseqs * s.segments);
+        if (per < 1) per = 1;
+    } else {
+        if ((double)s.nseqs * (double)s.nheads >= slots || nch < 8 * (int64_t)s.nseqs) return one;
+        per = (int64_t)std::ceil((double)nch * (double)s.nheads / (2.0 * slots));
+        if (per < 4) per = 4;
+    }
+    if (per > kMaxSegChunks) per = kMaxSegChunks;
+    const int64_t seg_len = per * kQ;
+    const int64_t nslots = (int64_t)s.nseqs + (s.seqlen + seg_len - 1) / seg_len;
+    if (nslots > 65535) return one;
+    SegPlan p{1, seg_len, nslots};
+    return p;
+}
 SegPlan plan_segments(const ssm_scan_args &s) {
     SegPlan one{1, s.seqlen};
-    if (s.cu_seqlens || s.batch <= 0 || s.seqlen <= kQ || s.segments == 1) return one;
+    if (s.cu_seqlens) return plan_packed(s);
+    if (s.batch <= 0 || s.seqlen <= kQ || s.segments == 1) return one;
     const int64_t nch = (s.seqlen + kQ - 1) / kQ;
     auto make = [&](int64_t k) {
         int64_t per = (nch + k - 1) / k;
@@ -1333,16 +1451,26 @@ SegPlan plan_segments(const ssm_scan_args &s) {
 }
 }  // namespace
 
-int ssd_segments(const ssm_scan_args &s) { return plan_segments(s).nseg; }
+int ssd_segments(const ssm_scan_args &s) {
+    const SegPlan p = plan_segments(s);
+    return p.nslots > 0 ? (int)p.nslots : p.nseg;
+}
+
+// Rows of segment states a plan keeps: fixed-length rows (nseg - 1) per row
+// and head; packed sequences one per launched segment row and head.
+size_t seg_state_rows(const ssm_scan_args &s, const SegPlan &p) {
+    if (p.nslots > 0) return (size_t)p.nslots * (size_t)s.nheads;
+    if (p.nseg > 1) return (size_t)s.batch * (size_t)(p.nseg - 1) * (size_t)s.nheads;
+    return 0;
+}
 
 size_t ssd_workspace_bytes(const ssm_scan_args &s) {
     size_t total = 0;
     if (s.d_conv > 0) total += 2 * round256((size_t)s.batch * (size_t)s.seqlen * (size_t)(s.ngroups * s.dstate) * 2);
     const SegPlan sp = plan_segments(s);
-    if (sp.nseg > 1) {
-        const size_t rows = (size_t)s.batch * (size_t)(sp.nseg - 1) * (size_t)s.nheads;
-        total += round256(rows * (size_t)(kP * kN) * 4) + round256(rows * 4);
-    }
+    const size_t rows = seg_state_rows(s, sp);
+    if (rows > 0) total += round256(rows * (size_t)(kP * kN) * 4) + round256(rows * 4);
+    if (sp.nslots > 0) total += round256((size_t)sp.nslots * sizeof(int4) + 16);
     return total;
 }
 
@@ -1403,11 +1531,20 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     }
     // then the segment states (fixed-length rows cut into segments)
     const SegPlan sp = plan_segments(s);
+    const bool packed_cut = sp.nslots > 0;
+    const bool cut = sp.nseg > 1 || packed_cut;
     float *sloc = nullptr, *slog = nullptr;
-    if (sp.nseg > 1) {
-        const size_t rows = (size_t)s.batch * (size_t)(sp.nseg - 1) * (size_t)s.nheads;
+    int4 *seg_tab = nullptr;
+    int32_t *seg_count = nullptr;
+    const size_t srows = seg_state_rows(s, sp);
+    if (srows > 0) {
         sloc = reinterpret_cast<float *>(wp);
-        slog = reinterpret_cast<float *>(wp + round256(rows * (size_t)(kP * kN) * 4));
+        slog = reinterpret_cast<float *>(wp + round256(srows * (size_t)(kP * kN) * 4));
+        wp += round256(srows * (size_t)(kP * kN) * 4) + round256(srows * 4);
+    }
+    if (packed_cut) {
+        seg_tab = reinterpret_cast<int4 *>(wp);
+        seg_count = reinterpret_cast<int32_t *>(wp + (size_t)sp.nslots * sizeof(int4));
     }
     // Host work first (tensor maps over the whole packed / batched token range,
     // the kernel attribute), so nothing on the host separates the pre-pass
@@ -1429,8 +1566,15 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     }
     cudaError_t e = cudaFuncSetAttribute(ssd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    if (sp.nseg > 1) {
+    if (cut) {
         e = cudaFuncSetAttribute(ssd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStSmemBytes);
+        if (e != cudaSuccess) return e;
+    }
+    if (packed_cut) {
+        // the segment table of the packed sequences (their lengths live on the device)
+        seg_table_kernel<<<1, kSegTabThreads, 0, st>>>(sv.cu, sv.order, sv.err, s.nseqs, s.seqlen, sp.seg_len,
+                                                        (int)sp.nslots, seg_tab, seg_count);
+        e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     if (s.d_conv > 0) {
@@ -1480,13 +1624,15 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
     a.Braw = static_cast<const __nv_bfloat16 *>(s.B); a.Craw = static_cast<const __nv_bfloat16 *>(s.C);
     a.braw_bs = s.B_batch_stride; a.braw_ts = s.B_token_stride;
     a.craw_bs = s.C_batch_stride; a.craw_ts = s.C_token_stride;
-    a.nseg = sp.nseg; a.seg_len = sp.nseg > 1 ? sp.seg_len : (s.seqlen > 0 ? s.seqlen : 1);
+    a.nseg = sp.nseg; a.seg_len = cut ? sp.seg_len : (s.seqlen > 0 ? s.seqlen : 1);
     a.sloc = sloc; a.slog = slog;
+    a.seg_tab = seg_tab; a.seg_count = seg_count;
+    a.nsloc = (int64_t)(srows / (size_t)s.nheads);
     // the timed region holds the state pass and the scan
     timing_begin(st);
-    if (sp.nseg > 1) {
+    if (cut) {
         // the state each segment but the last leaves, from zero
-        const dim3 sgrid((unsigned)s.nheads, (unsigned)(nseqs * (sp.nseg - 1)));
+        const dim3 sgrid((unsigned)s.nheads, (unsigned)(packed_cut ? sp.nslots : (int64_t)nseqs * (sp.nseg - 1)));
         ssd_state_kernel<<<sgrid, kThreads, kStSmemBytes, st>>>(a, tm_x, tm_b);
         e = cudaGetLastError();
         if (e != cudaSuccess) {
@@ -1494,7 +1640,7 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
             return e;
         }
     }
-    dim3 grid((unsigned)s.nheads, (unsigned)(nseqs * sp.nseg));
+    dim3 grid((unsigned)s.nheads, (unsigned)(packed_cut ? sp.nslots : (int64_t)nseqs * sp.nseg));
     ssd_kernel<<<grid, kThreads, kSmemBytes, st>>>(a, tm_x, tm_b, tm_c, tm_z, tm_y);
     timing_end(st);
     return cudaGetLastError();

@@ -161,8 +161,18 @@ def test_segment_plan_is_host_only():
     assert lib.ssm_scan_segments(C.byref(_scan(segments=3, **big))) == 3          # runs of 22, 22, 20 chunks
     # many chains already fill the GPU: rows stay whole
     assert lib.ssm_scan_segments(C.byref(_scan(**dict(big, batch=64, x_batch_stride=5120 * 4096)))) == 1
-    # packed sequences and Mamba-1 are never cut; bad arguments give 0
-    assert lib.ssm_scan_segments(C.byref(_scan(segments=4, **dict(big, batch=1, cu_seqlens=FAKE, nseqs=3)))) == 1
+    # packed sequences: one run length for all, chosen from the total (64
+    # chunks); the count is the bound nseqs + ceil(total / run) on their runs
+    packed = dict(big, batch=1, cu_seqlens=FAKE, nseqs=3)
+    assert lib.ssm_scan_segments(C.byref(_scan(segments=4, **packed))) == 3 + 11    # runs of 6 chunks
+    assert lib.ssm_scan_segments(C.byref(_scan(segments=1, **packed))) == 1
+    per = -(-64 * 80 // (2 * 2 * 148))                                              # about two waves of CTAs
+    assert lib.ssm_scan_segments(C.byref(_scan(**packed))) == 3 + -(-4096 // (64 * per))
+    # many sequences fill the GPU, or are too short to cut: they stay whole
+    assert lib.ssm_scan_segments(C.byref(_scan(**dict(packed, nseqs=1000)))) == 1
+    assert lib.ssm_scan_segments(C.byref(_scan(**dict(packed, nseqs=9)))) == 1       # 7 chunks each
+    assert lib.ssm_scan_segments(C.byref(_scan(segments=2, **dict(packed, nseqs=9)))) == 9 + 16
+    # Mamba-1 is never cut; bad arguments give 0
     assert lib.ssm_scan_segments(C.byref(_scan(mode=1, d_inner=8, ngroups=1, dt_token_stride=8, dt_batch_stride=128))) == 1
     assert lib.ssm_scan_segments(C.byref(_scan(segments=-1, **big))) == 0
     assert lib.ssm_scan_fwd(C.byref(_scan(segments=-1, **big)), None, 0, None) == _abi.SSM_ERR_INVALID_ARG
@@ -181,10 +191,14 @@ def test_workspace_holds_segment_states():
     four = lib.ssm_scan_workspace_size(C.byref(_scan(segments=4, **kw)))
     rows = 2 * 3 * 4
     assert four - one == rows * 64 * 128 * 4 + 256
-    # packed sequences are never cut
+    # packed sequences, 10 chunks asked in about 4 runs each: runs of 2 chunks,
+    # at most 2 + 5 table entries, each with a state row per head, plus the
+    # table itself and its count
     packed = dict(kw, batch=1, cu_seqlens=FAKE, nseqs=2)
-    assert lib.ssm_scan_workspace_size(C.byref(_scan(segments=4, **packed))) == \
-        lib.ssm_scan_workspace_size(C.byref(_scan(segments=1, **packed)))
+    entries = 2 + 5
+    extra = entries * 4 * 64 * 128 * 4 + 256 + 256
+    assert lib.ssm_scan_workspace_size(C.byref(_scan(segments=4, **packed))) - \
+        lib.ssm_scan_workspace_size(C.byref(_scan(segments=1, **packed))) == extra
 
 
 def _conv(**kw):

@@ -103,12 +103,13 @@ def test_mamba2_tensor_core_batch(interval, segments):
     _run(M2, d, "bf16", interval, stride=5, nslots=7, seed=13, segments=segments)
 
 
-def test_mamba2_tensor_core_varlen():
+@pytest.mark.parametrize("segments", [0, 2])       # whole sequences; runs of one chunk
+def test_mamba2_tensor_core_varlen(segments):
     lengths = [130, 0, 64, 257, 63, 192]
     d = W.mamba2_inputs(804, 1, sum(lengths), 4, 64, 2, 128, dtype="bf16", conv_bias=True, conv_state=True,
                         nseqs=len(lengths))
     d["cu_seqlens"] = W.cu_from_lengths(lengths)
-    _run(M2, d, "bf16", 64, stride=4, nslots=10, seed=14)
+    _run(M2, d, "bf16", 64, stride=4, nslots=10, seed=14, segments=segments)
 
 
 @pytest.mark.parametrize("dtype,P,N", [("f32", 64, 128), ("bf16", 48, 64), ("f32", 16, 32)])

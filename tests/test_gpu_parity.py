@@ -155,6 +155,43 @@ def test_mamba2_segments_match_unsegmented():
         assert np.array_equal(c2, c1), nseg
 
 
+# Packed sequences cut on the device: one run length for all of them, a table
+# of (sequence, run) entries built from cu_seqlens, surplus CTA rows idle.
+# Empty, one-token and exactly-one-run sequences sit between long ones.
+VARLEN_SEG_CASES = [
+    # (lengths, H, G, K, segments)
+    ([3000, 0, 1, 700, 64, 2049], 2, 1, 4, 2),     # runs of 8 chunks
+    ([1000, 1000], 4, 2, 3, 4),                    # runs of 4 chunks, the last 232 tokens
+    ([5000], 2, 1, 4, 0),                          # one sequence x 2 heads: cut by the library
+    ([130, 4100, 0, 65], 2, 2, 0, 3),              # no conv; runs of 6 chunks
+    ([64, 128, 192], 2, 1, 2, 2),                  # runs of one chunk, every sequence ends on a run edge
+]
+
+
+@pytest.mark.parametrize("lengths,H,G,K,segments", VARLEN_SEG_CASES)
+def test_mamba2_varlen_segments(lengths, H, G, K, segments):
+    cu = W.cu_from_lengths(lengths)
+    d = W.mamba2_inputs(470 + len(lengths) + H + K, 1, int(cu[-1]), H, 64, G, 128, d_conv=K, dtype="bf16",
+                        conv_bias=True, conv_state=True, nseqs=len(lengths))
+    d["cu_seqlens"] = cu
+    check_scan(M2, d, "bf16", segments=segments, what=f"M2 varlen segments={segments} {lengths}")
+
+
+def test_mamba2_varlen_segments_match_unsegmented():
+    lengths = [2500, 3, 0, 900, 1300]
+    cu = W.cu_from_lengths(lengths)
+    d = W.mamba2_inputs(480, 1, int(cu[-1]), 4, 64, 2, 128, dtype="bf16", conv_bias=True, conv_state=True,
+                        nseqs=len(lengths))
+    d["cu_seqlens"] = cu
+    t = to_dev(d, "bf16")
+    y1, h1, c1 = gpu_scan(M2, t, segments=1)
+    for nseg in (2, 5, 9):
+        y2, h2, c2 = gpu_scan(M2, t, segments=nseg)
+        assert rel_err(y2, y1) <= TOL["bf16"], nseg
+        assert rel_err(h2, h1) <= TOL["bf16"], nseg
+        assert np.array_equal(c2, c1), nseg
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_mamba2_strided_views(dtype):
     d = W.mamba2_inputs(410, 2, 50, 4, 32, 2, 32, dtype=dtype, conv_state=True)
