@@ -255,6 +255,7 @@ class Job:
         self.bwd = None            # set by the backward workloads
         self.timing_on = False     # kernel timing enabled (the timed region)
         self.segments = 1          # token segments per row (tensor-core Mamba-2 path)
+        self.varlen = False
         if w.kind in ("mamba1", "mamba2", "mamba2_varlen"):
             mode = ssm.MAMBA1 if w.kind == "mamba1" else ssm.MAMBA2
             ww = W.Workload(**{**w.__dict__, "seed": w.seed + seed_shift})
@@ -289,7 +290,7 @@ class Job:
                                            conv_w=t["conv_w"])
             self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev) if need else None
             self.ssd = mode == ssm.MAMBA2 and w.dtype == "bf16" and w.headdim == 64 and w.dstate == 128 and w.d_conv <= 4
-            varlen = t.get("cu_seqlens") is not None
+            varlen = self.varlen = t.get("cu_seqlens") is not None
             if self.ssd:
                 # the B / C conv pre-pass, then the chunked tensor-core scan (+ the varlen plan)
                 self.launches_per_step = 2 + (1 if varlen else 0)
@@ -364,7 +365,8 @@ class Job:
                                                   cu_seqlens=t.get("cu_seqlens"), conv_w=t["conv_w"])
                 if self.segments > 1:
                     self.kernel = "ssd_state_kernel+ssd_kernel"
-                    self.launches_per_step += 1
+                    # packed sequences: also the segment-table pre-pass
+                    self.launches_per_step += 2 if varlen else 1
                 self.mufu = None
                 # tensor-core work of the 64-token chunked form: per (sequence, head, chunk)
                 # C.B^T (2 Q^2 N) + M.X (2 Q^2 P) + C'.S^T (2 Q N P) + B'^T.X (2 Q N P)
@@ -832,7 +834,8 @@ def run_cuda(args):
                    "parallelism": (f"seqsplit{w.split_ranks}: rank {w.split_rank}'s step, exchanges staged in HBM"
                                    if w.split_ranks else (f"replicas{world}" if world > 1 else "single")),
                    "l2": "flushed between timed steps (256 MiB write, outside the events)",
-                   "tokens_per_step": job.units, "token_segments_per_row": job.segments},
+                   "tokens_per_step": job.units,
+                   ("token_segment_rows_launched" if job.varlen else "token_segments_per_row"): job.segments},
         "hbm_gbs": gbs, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         "gpu_launches": job.launches_per_step * args.steps, "impl": "cuda",
         "step_ms": {"min": min(step_ms), "median": float(np.median(step_ms)), "max": max(step_ms)},

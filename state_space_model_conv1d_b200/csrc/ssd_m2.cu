@@ -1387,39 +1387,8 @@ struct SegPlan {
     int64_t seg_len;
     int64_t nslots = 0;                 // packed sequences: (segment) CTA rows launched, 0 = not cut
 };
-// Packed sequences (lengths known on the device only): every sequence is cut
-// into ceil(len / seg_len) segments of seg_len tokens (at least one), listed
-// by a device pre-pass; nseqs + total / seg_len rows bound their count.  Cut
-// when requested (segments >= 2: about that many runs for a sequence of the
-// mean length) or, when chosen, if the sequences x heads give fewer chains
-// than the GPU has CTA slots and the mean sequence spans two runs of the
-// shortest length (4 chunks; shorter work would not pay for the extra
-// launches): then seg_len aims at about two waves of (segment, head) CTAs,
-// 4 to kMaxSegChunks chunks.
-SegPlan plan_packed(const ssm_scan_args &s) {
-    SegPlan one{1, s.seqlen > 0 ? s.seqlen : 1};
-    if (s.segments == 1 || s.nseqs <= 0 || s.seqlen <= kQ) return one;
-    const int64_t nch = (s.seqlen + kQ - 1) / kQ;
-    const double slots = 2.0 * sm_count();
-    int64_t per;
-    if (s.segments >= 2) {
-        per = (nch + (int64_t)s.nseqs * s.segments - 1) / ((int64_t)s.nseqs * s.segments);
-        if (per < 1) per = 1;
-    } else {
-        if ((double)s.nseqs * (double)s.nheads >= slots || nch < 8 * (int64_t)s.nseqs) return one;
-        per = (int64_t)std::ceil((double)nch * (double)s.nheads / (2.0 * slots));
-        if (per < 4) per = 4;
-    }
-    if (per > kMaxSegChunks) per = kMaxSegChunks;
-    const int64_t seg_len = per * kQ;
-    const int64_t nslots = (int64_t)s.nseqs + (s.seqlen + seg_len - 1) / seg_len;
-    if (nslots > 65535) return one;
-    SegPlan p{1, seg_len, nslots};
-    return p;
-}
-SegPlan plan_segments(const ssm_scan_args &s) {
+SegPlan plan_fixed(const ssm_scan_args &s) {
     SegPlan one{1, s.seqlen};
-    if (s.cu_seqlens) return plan_packed(s);
     if (s.batch <= 0 || s.seqlen <= kQ || s.segments == 1) return one;
     const int64_t nch = (s.seqlen + kQ - 1) / kQ;
     auto make = [&](int64_t k) {
@@ -1449,6 +1418,39 @@ SegPlan plan_segments(const ssm_scan_args &s) {
     }
     return best;
 }
+// Packed sequences (lengths known on the device only): every sequence is cut
+// into ceil(len / seg_len) segments of seg_len tokens (at least one), listed
+// by a device pre-pass; nseqs + total / seg_len rows bound their count.  Cut
+// when requested (segments >= 2: about that many runs for a sequence of the
+// mean length) or, when chosen, if the sequences x heads give fewer chains
+// than the GPU has CTA slots: then seg_len is the fixed-length choice for
+// nseqs rows of the mean length.
+SegPlan plan_packed(const ssm_scan_args &s) {
+    SegPlan one{1, s.seqlen > 0 ? s.seqlen : 1};
+    if (s.segments == 1 || s.nseqs <= 0 || s.seqlen <= kQ) return one;
+    int64_t seg_len;
+    if (s.segments >= 2) {
+        const int64_t nch = (s.seqlen + kQ - 1) / kQ;
+        int64_t per = (nch + (int64_t)s.nseqs * s.segments - 1) / ((int64_t)s.nseqs * s.segments);
+        if (per < 1) per = 1;
+        if (per > kMaxSegChunks) per = kMaxSegChunks;
+        seg_len = per * kQ;
+    } else {
+        if ((double)s.nseqs * (double)s.nheads >= 2.0 * sm_count()) return one;
+        ssm_scan_args m = s;
+        m.cu_seqlens = nullptr;
+        m.batch = s.nseqs;
+        m.seqlen = (s.seqlen + s.nseqs - 1) / s.nseqs;
+        const SegPlan f = plan_fixed(m);
+        if (f.nseg < 2) return one;
+        seg_len = f.seg_len;
+    }
+    const int64_t nslots = (int64_t)s.nseqs + (s.seqlen + seg_len - 1) / seg_len;
+    if (nslots > 65535) return one;
+    SegPlan p{1, seg_len, nslots};
+    return p;
+}
+SegPlan plan_segments(const ssm_scan_args &s) { return s.cu_seqlens ? plan_packed(s) : plan_fixed(s); }
 }  // namespace
 
 int ssd_segments(const ssm_scan_args &s) {

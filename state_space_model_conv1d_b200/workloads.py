@@ -231,6 +231,12 @@ WORKLOADS = {
     "mamba2_seq_b1_l16384_h80_p64_g8_n128": Workload("mamba2_seq_b1_l16384_h80_p64_g8_n128", "mamba2", "bf16",
                                                      batch=1, seqlen=16384, nheads=80, headdim=64, ngroups=8,
                                                      dstate=128, chunk=256, seed=BASE_SEED + 6),
+    # two long packed sequences (4096 to 16384 tokens each): 160 (sequence,
+    # head) chains for 296 CTA slots, so the device cuts the sequences into
+    # token segments from their cu_seqlens
+    "mamba2_varlen_2seq_h80_p64_g8_n128": Workload("mamba2_varlen_2seq_h80_p64_g8_n128", "mamba2_varlen", "bf16",
+                                                   nheads=80, headdim=64, ngroups=8, dstate=128, nseqs=2,
+                                                   len_lo=4096, len_hi=16384, chunk=256, seed=BASE_SEED + 7),
     # the Mamba-1 layer's backward (same inputs; upstream gradients drawn alongside)
     "mamba1_layer_b8_l2048_d1536_n16_bwd": Workload("mamba1_layer_b8_l2048_d1536_n16_bwd", "mamba1", "bf16", batch=8,
                                                     seqlen=2048, d_inner=1536, dstate=16, backward=True,

@@ -166,11 +166,15 @@ def test_segment_plan_is_host_only():
     packed = dict(big, batch=1, cu_seqlens=FAKE, nseqs=3)
     assert lib.ssm_scan_segments(C.byref(_scan(segments=4, **packed))) == 3 + 11    # runs of 6 chunks
     assert lib.ssm_scan_segments(C.byref(_scan(segments=1, **packed))) == 1
-    per = -(-64 * 80 // (2 * 2 * 148))                                              # about two waves of CTAs
-    assert lib.ssm_scan_segments(C.byref(_scan(**packed))) == 3 + -(-4096 // (64 * per))
-    # many sequences fill the GPU, or are too short to cut: they stay whole
+    # chosen: the fixed-length choice for nseqs rows of the mean length; one
+    # sequence of 4096 tokens is cut like a row of 4096 (3 runs of 22 chunks)
+    one = dict(packed, nseqs=1)
+    assert lib.ssm_scan_segments(C.byref(_scan(**dict(big, batch=1)))) == 3
+    assert lib.ssm_scan_segments(C.byref(_scan(**one))) == 1 + 3
+    # three means of 22 chunks (240 chains) stay whole, as do many sequences
+    assert lib.ssm_scan_segments(C.byref(_scan(**packed))) == 1
     assert lib.ssm_scan_segments(C.byref(_scan(**dict(packed, nseqs=1000)))) == 1
-    assert lib.ssm_scan_segments(C.byref(_scan(**dict(packed, nseqs=9)))) == 1       # 7 chunks each
+    assert lib.ssm_scan_segments(C.byref(_scan(**dict(packed, nseqs=9)))) == 1
     assert lib.ssm_scan_segments(C.byref(_scan(segments=2, **dict(packed, nseqs=9)))) == 9 + 16
     # Mamba-1 is never cut; bad arguments give 0
     assert lib.ssm_scan_segments(C.byref(_scan(mode=1, d_inner=8, ngroups=1, dt_token_stride=8, dt_batch_stride=128))) == 1

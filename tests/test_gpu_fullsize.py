@@ -48,17 +48,20 @@ def _m2_head_problem(d, h, H, P, G, N):
     return sub
 
 
-# The fixed-length workloads run cut into token segments (the library's choice
-# for these shapes), the packed one whole.
-@pytest.mark.parametrize("name", ["mamba2_ssd_b4_l4096_h80_p64_g8_n128", "mamba2_varlen_16seq_h64_p64_g1_n128",
-                                  "mamba2_seq_b1_l16384_h80_p64_g8_n128"])
-def test_mamba2_fullsize_sampled_heads(name):
+# The library's choice for these shapes: the fixed-length workloads and the
+# two long packed sequences run cut into token segments, the 16 packed
+# sequences (1024 chains) whole.
+@pytest.mark.parametrize("name,cut", [("mamba2_ssd_b4_l4096_h80_p64_g8_n128", True),
+                                      ("mamba2_varlen_16seq_h64_p64_g1_n128", False),
+                                      ("mamba2_seq_b1_l16384_h80_p64_g8_n128", True),
+                                      ("mamba2_varlen_2seq_h80_p64_g8_n128", True)])
+def test_mamba2_fullsize_sampled_heads(name, cut):
     w = W.WORKLOADS[name]
     d = W.workload_inputs(w)
     t = to_dev(d, "bf16")
     nseg = ssm.scan_segments(M2, t["x"], t["dt"], t["A"], t["B"], t["C"], z=t["z"], cu_seqlens=t.get("cu_seqlens"),
                              conv_w=t["conv_w"])
-    assert (nseg == 1) == (d.get("cu_seqlens") is not None), nseg
+    assert (nseg > 1) == cut, nseg
     y, hf, cs = gpu_scan(M2, t)
     H, P, G, N = w.nheads, w.headdim, w.ngroups, w.dstate
     for h in (0, H // 2 - 1, H // 2, H - 1):
