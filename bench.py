@@ -54,6 +54,8 @@ def parse():
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--segments", type=int, default=0,
+                   help="token segments asked of the Mamba-2 tensor-core scan (0: the library's choice, 1: whole rows)")
     return p.parse_args()
 
 
@@ -245,8 +247,9 @@ class ClockSampler:
 class Job:
     """One workload on the device: step(), bytes and units per step, e2e step."""
 
-    def __init__(self, w: W.Workload, rank: int, torch, ssm):
+    def __init__(self, w: W.Workload, rank: int, torch, ssm, segments: int = 0):
         self.w, self.torch, self.ssm = w, torch, ssm
+        self.seg_request = segments    # passed to every scan call (0: the library's choice)
         dev = torch.device("cuda", torch.cuda.current_device())
         seed_shift = rank_seed(0, rank)
         bf = torch.bfloat16 if w.dtype == "bf16" else torch.float32
@@ -287,7 +290,7 @@ class Job:
             self.hf = torch.empty(hshape, dtype=torch.float32, device=dev)
             self.cso = torch.empty((nseq, cdim, t["conv_w"].shape[1] - 1), dtype=bf, device=dev)
             need = ssm.scan_workspace_size(mode, x, t["dt"], t["A"], t["B"], t["C"], cu_seqlens=t.get("cu_seqlens"),
-                                           conv_w=t["conv_w"])
+                                           conv_w=t["conv_w"], segments=segments)
             self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev) if need else None
             self.ssd = mode == ssm.MAMBA2 and w.dtype == "bf16" and w.headdim == 64 and w.dstate == 128 and w.d_conv <= 4
             varlen = self.varlen = t.get("cu_seqlens") is not None
@@ -362,7 +365,8 @@ class Job:
                 # rows the library cuts into token segments add the state-only pass, which
                 # the kernel timing brackets together with the scan
                 self.segments = ssm.scan_segments(mode, x, t["dt"], t["A"], t["B"], t["C"], z=t["z"],
-                                                  cu_seqlens=t.get("cu_seqlens"), conv_w=t["conv_w"])
+                                                  cu_seqlens=t.get("cu_seqlens"), conv_w=t["conv_w"],
+                                                  segments=segments)
                 if self.segments > 1:
                     self.kernel = "ssd_state_kernel+ssd_kernel"
                     # packed sequences: also the segment-table pre-pass
@@ -518,7 +522,7 @@ class Job:
         self.ssm.scan_fwd(self.mode, t["x"], t["dt"], t["A"], t["B"], t["C"], D=t["D"], z=t["z"], dt_bias=t["dt_bias"],
                           h0=t["h0"], cu_seqlens=t.get("cu_seqlens"), conv_w=t["conv_w"], conv_b=t["conv_b"],
                           conv_state_in=t["conv_state_in"], y=y, h_final=self.hf, conv_state_out=self.cso,
-                          workspace=self.ws, **self.inter)
+                          workspace=self.ws, segments=self.seg_request, **self.inter)
 
     def e2e_pipelined(self):
         """Whether the end-to-end leg overlaps copies with compute (forward scans and decode)."""
@@ -694,7 +698,7 @@ def run_cuda(args):
     if near:
         os.sched_setaffinity(0, near)
     w = W.WORKLOADS[args.workload]
-    job = Job(w, rank, torch, ssm)
+    job = Job(w, rank, torch, ssm, segments=args.segments)
     flush = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
     for _ in range(max(args.warmup, 0)):
@@ -835,7 +839,8 @@ def run_cuda(args):
                                    if w.split_ranks else (f"replicas{world}" if world > 1 else "single")),
                    "l2": "flushed between timed steps (256 MiB write, outside the events)",
                    "tokens_per_step": job.units,
-                   ("token_segment_rows_launched" if job.varlen else "token_segments_per_row"): job.segments},
+                   ("token_segment_rows_launched" if job.varlen else "token_segments_per_row"): job.segments,
+                   "token_segments_requested": args.segments or "library choice"},
         "hbm_gbs": gbs, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
         "gpu_launches": job.launches_per_step * args.steps, "impl": "cuda",
         "step_ms": {"min": min(step_ms), "median": float(np.median(step_ms)), "max": max(step_ms)},
