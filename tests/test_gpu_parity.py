@@ -177,6 +177,23 @@ def test_mamba2_varlen_segments(lengths, H, G, K, segments):
     check_scan(M2, d, "bf16", segments=segments, what=f"M2 varlen segments={segments} {lengths}")
 
 
+def test_mamba2_varlen_segments_many_sequences():
+    """More sequences than the table pre-pass has threads (its prefix sum
+    carries across tiles of 1024 sequences), most of them cut into runs of
+    one chunk."""
+    rng = np.random.default_rng(491)
+    lengths = rng.integers(0, 200, size=2500)
+    lengths[rng.integers(0, 2500, size=40)] = 0
+    cu = W.cu_from_lengths(lengths)
+    d = W.mamba2_inputs(492, 1, int(cu[-1]), 1, 64, 1, 128, d_conv=4, dtype="bf16", conv_bias=True,
+                        conv_state=True, nseqs=len(lengths))
+    d["cu_seqlens"] = cu
+    t = to_dev(d, "bf16")
+    assert ssm.scan_segments(M2, t["x"], t["dt"], t["A"], t["B"], t["C"], z=t["z"], cu_seqlens=t["cu_seqlens"],
+                             conv_w=t["conv_w"], segments=2) > len(lengths)
+    check_scan(M2, d, "bf16", segments=2, what="M2 varlen segments, 2500 sequences")
+
+
 def test_mamba2_varlen_segments_match_unsegmented():
     lengths = [2500, 3, 0, 900, 1300]
     cu = W.cu_from_lengths(lengths)
