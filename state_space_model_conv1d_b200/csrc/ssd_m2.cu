@@ -1196,33 +1196,31 @@ SSM_DEVINL uint2 pack_bf16x4(const float (&v)[kBcV]) {
     return make_uint2(*reinterpret_cast<const uint32_t *>(&lo), *reinterpret_cast<const uint32_t *>(&hi));
 }
 
+// One thread per (4 channels of B or C, kBcR consecutive tokens); a warp
+// covers 32 consecutive channel vectors of one token run.  Every load that
+// does not depend on the sequence bounds (taps, bias, the K-1 rows before the
+// run and its kBcR rows) is issued first, so their latency overlaps the
+// search for the run's sequence in cu_seqlens (one thread per CTA, then each
+// thread walks on from it); the conv history restarts at every sequence start.
+constexpr int kBcR = 16;              // tokens per thread
+
 template <int K>
-__global__ void __launch_bounds__(128, 5) bc_conv_kernel(const BcArgs a) {
+__global__ void __launch_bounds__(128, 4) bc_conv_kernel(const BcArgs a) {
+    constexpr int KH = K - 1;                             // rows before the run
     const int64_t nvec = 2 * a.GN / kBcV;                 // B and C vectors of one token row
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t vec = idx % nvec, run = idx / nvec;
-    const int64_t t0 = run * 8;
+    const int64_t t0 = run * kBcR;
     const int64_t row = blockIdx.y;
-    // packed sequences: one thread finds the sequence of the CTA's first token,
-    // every thread walks on from there (its run starts at most a few tokens later)
-    __shared__ int s_first;
-    if (a.cu) {
-        if (threadIdx.x == 0) {
-            const int64_t tf = ((int64_t)blockIdx.x * blockDim.x / nvec) * 8;
-            s_first = seq_of_token(a.cu, a.nseqs, min(tf, a.seqlen > 0 ? a.seqlen - 1 : (int64_t)0));
-        }
-        __syncthreads();
-    }
-    if (t0 >= a.seqlen) return;
+    const bool live = t0 < a.seqlen;
     const int which = vec >= nvec / 2;                    // 0: B, 1: C
     const int64_t c0 = (vec - which * (nvec / 2)) * kBcV; // channel within B (or C)
-    const __nv_bfloat16 *src = which ? a.C + row * a.c_bs : a.B + row * a.b_bs;
     const int64_t ts = which ? a.c_ts : a.b_ts;
+    const __nv_bfloat16 *src = (which ? a.C + row * a.c_bs : a.B + row * a.b_bs) + c0;
     __nv_bfloat16 *dst = (which ? a.oC : a.oB) + row * a.seqlen * a.GN + c0;
     const int64_t cch = a.HP + which * a.GN + c0;         // conv channel of the first of the 4
-    if (!SSM_BOUNDS(c0 + kBcV - 1, a.GN, BS_BC_CHANNEL) ||
-        !SSM_BOUNDS(row * a.seqlen + t0, (int64_t)gridDim.y * a.seqlen, BS_BC_ROW))
-        return;
+    const bool in_range = SSM_BOUNDS(c0 + kBcV - 1, a.GN, BS_BC_CHANNEL) &&
+                          (!live || SSM_BOUNDS(row * a.seqlen + t0, (int64_t)gridDim.y * a.seqlen, BS_BC_ROW));
     // taps and bias of the 4 channels: 16-byte loads when they are aligned (one
     // channel's 4 taps; 4 biases), scalar loads otherwise
     float wk[K][kBcV], bb[kBcV];
@@ -1245,6 +1243,24 @@ __global__ void __launch_bounds__(128, 5) bc_conv_kernel(const BcArgs a) {
 #pragma unroll
         for (int v = 0; v < kBcV; ++v) bb[v] = a.bias ? a.bias[cch + v] : 0.f;
     }
+    // raw[j]: token t0 - (K-1) + j of the row (zero outside the tensor)
+    uint2 raw[KH + kBcR];
+#pragma unroll
+    for (int j = 0; j < KH + kBcR; ++j) {
+        const int64_t tau = t0 - KH + j;
+        raw[j] = (live && in_range && tau >= 0 && tau < a.seqlen) ? *reinterpret_cast<const uint2 *>(src + tau * ts)
+                                                                  : make_uint2(0u, 0u);
+    }
+    // packed sequences: one thread finds the sequence of the CTA's first token
+    __shared__ int s_first;
+    if (a.cu) {
+        if (threadIdx.x == 0) {
+            const int64_t tf = ((int64_t)blockIdx.x * blockDim.x / nvec) * kBcR;
+            s_first = seq_of_token(a.cu, a.nseqs, min(tf, a.seqlen > 0 ? a.seqlen - 1 : (int64_t)0));
+        }
+        __syncthreads();
+    }
+    if (!live || !in_range) return;
     // sequence of the run's first token and its bounds (clamped: a malformed
     // cu_seqlens gives wrong values but no out-of-bounds access)
     int s = (int)row;
@@ -1254,33 +1270,24 @@ __global__ void __launch_bounds__(128, 5) bc_conv_kernel(const BcArgs a) {
     }
     int64_t start = a.cu ? min(max((int64_t)a.cu[s], (int64_t)0), a.seqlen) : 0;
     int64_t end = a.cu ? min(max((int64_t)a.cu[s + 1], start), a.seqlen) : a.seqlen;
-    float hist[K > 1 ? K - 1 : 1][kBcV];
-    auto load_hist = [&](int64_t t) {
+    // carried conv state of sequence s, tap q (0 .. K-2), or zero
+    auto carried = [&](int q, float (&h)[kBcV]) {
+        const bool in = a.state_in && SSM_BOUNDS(((int64_t)s * a.cdim + cch + kBcV - 1) * KH + q,
+                                                 (int64_t)(a.cu ? a.nseqs : gridDim.y) * a.cdim * KH, BS_BC_STATE);
 #pragma unroll
-        for (int j = 0; j < K - 1; ++j) {                 // hist[j] holds token t-(K-1)+j
-            const int64_t tau = t - (K - 1) + j;
-            if (tau >= start) {
-                unpack_bf16x4(*reinterpret_cast<const uint2 *>(src + tau * ts + c0), hist[j]);
-            } else {
-                const int64_t q = tau - start + (K - 1);
-                const bool in = a.state_in && q >= 0 &&
-                                SSM_BOUNDS(((int64_t)s * a.cdim + cch + kBcV - 1) * (K - 1) + q,
-                                           (int64_t)(a.cu ? a.nseqs : gridDim.y) * a.cdim * (K - 1), BS_BC_STATE);
-#pragma unroll
-                for (int v = 0; v < kBcV; ++v)
-                    hist[j][v] = in ? __bfloat162float(a.state_in[((int64_t)s * a.cdim + cch + v) * (K - 1) + q]) : 0.f;
-            }
-        }
+        for (int v = 0; v < kBcV; ++v)
+            h[v] = in ? __bfloat162float(a.state_in[((int64_t)s * a.cdim + cch + v) * KH + q]) : 0.f;
     };
-    load_hist(t0);
-    const int64_t t1 = min(t0 + 8, a.seqlen);
-    // every row's load is issued before any math
-    uint2 rows[8];
+    float hist[KH > 0 ? KH : 1][kBcV];                    // hist[j] holds token t - (K-1) + j
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-        if (t0 + i < t1) rows[i] = *reinterpret_cast<const uint2 *>(src + (t0 + i) * ts + c0);
+    for (int j = 0; j < KH; ++j) {
+        const int64_t tau = t0 - KH + j;
+        if (tau >= start) unpack_bf16x4(raw[j], hist[j]);
+        else carried((int)(tau - start + KH), hist[j]);   // tau >= t0 - (K-1) >= start - (K-1)
+    }
+    const int64_t t1 = min(t0 + kBcR, a.seqlen);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kBcR; ++i) {
         const int64_t t = t0 + i;
         if (t >= t1) break;
         if (a.cu && t >= end) {                           // the next non-empty sequence starts here
@@ -1288,26 +1295,31 @@ __global__ void __launch_bounds__(128, 5) bc_conv_kernel(const BcArgs a) {
             start = min(max((int64_t)a.cu[s], (int64_t)0), a.seqlen);
             end = min(max((int64_t)a.cu[s + 1], start), a.seqlen);
             if (t < start || t >= end) return;
-            load_hist(t);
+#pragma unroll
+            for (int j = 0; j < KH; ++j) {                // taps before the sequence: its carried state
+                const int64_t tau = t - KH + j;
+                if (tau >= start) unpack_bf16x4(raw[i + j], hist[j]);
+                else carried((int)(tau - start + KH), hist[j]);
+            }
         }
         float cur[kBcV], o[kBcV];
-        unpack_bf16x4(rows[i], cur);
+        unpack_bf16x4(raw[KH + i], cur);
 #pragma unroll
         for (int v = 0; v < kBcV; ++v) {
             float acc = bb[v];
 #pragma unroll
-            for (int k = 0; k < K - 1; ++k) acc = fmaf(wk[k][v], hist[k][v], acc);
+            for (int k = 0; k < KH; ++k) acc = fmaf(wk[k][v], hist[k][v], acc);
             acc = fmaf(wk[K - 1][v], cur[v], acc);
             o[v] = silu_fast<__nv_bfloat16>(acc);
         }
         *reinterpret_cast<uint2 *>(dst + t * a.GN) = pack_bf16x4(o);
 #pragma unroll
-        for (int k = 0; k + 1 < K - 1; ++k)
+        for (int k = 0; k + 1 < KH; ++k)
 #pragma unroll
             for (int v = 0; v < kBcV; ++v) hist[k][v] = hist[k + 1][v];
-        if (K > 1)
+        if (KH > 0)
 #pragma unroll
-            for (int v = 0; v < kBcV; ++v) hist[K > 1 ? K - 2 : 0][v] = cur[v];
+            for (int v = 0; v < kBcV; ++v) hist[KH > 0 ? KH - 1 : 0][v] = cur[v];
     }
 }
 
@@ -1593,7 +1605,7 @@ cudaError_t launch_ssd(const ssm_scan_args &s, const SeqView &sv, void *ws, cuda
         // rows start 16-byte aligned whenever the arrays do
         b.w16 = ((uintptr_t)s.conv_w % 16) == 0;
         b.b16 = s.conv_b != nullptr && ((uintptr_t)s.conv_b % 16) == 0;
-        const int64_t threads = (s.seqlen + 7) / 8 * (2 * GN / kBcV);
+        const int64_t threads = (s.seqlen + kBcR - 1) / kBcR * (2 * GN / kBcV);
         const dim3 bgrid((unsigned)((threads + 127) / 128), (unsigned)rows);
         if (threads > 0) {
             switch (s.d_conv) {
