@@ -462,8 +462,8 @@ class Job:
         wrote = self.y.numel() * self.y.element_size() + self.hf.numel() * 4 + tails[0].numel() * tails.element_size() \
             + pairs[0].numel() * pairs.element_size()
         self.bytes_per_step = read + wrote
-        # tail, the scan's launches, cum_delta, combine, fix-up (the pair packing and the
-        # staging copy are torch's)
+        # tail, the scan's launches, cum_delta, combine, fix-up (the scan and cum_delta
+        # write the pair into the exchange buffer; the combine reads it in place)
         self.launches_per_step = 1 + self.launches_per_step + 3
         # The fix-up is the step's largest kernel: the roofline names it, with its own
         # algorithmic bytes (y read and written, z, the raw C rows and their conv taps,
@@ -489,7 +489,9 @@ class Job:
         if timed:
             self.ssm.kernel_timing(False)         # only the fix-up is bracketed
         seg.tail()
-        sp["pairs"][sp["r"]].copy_(seg.scan(sp["tails"]))
+        # this rank's pair goes straight into its block of the exchange buffer, as an
+        # in-place all-gather (all_gather_into_tensor with the rank's own slice as input) has it
+        seg.scan(sp["tails"], out=sp["pairs"][sp["r"]])
         if timed:
             self.ssm.kernel_timing(True)
         self.y, self.hf, _ = seg.join(sp["pairs"])

@@ -74,7 +74,7 @@
 extern "C" {
 #endif
 
-#define SSM_ABI_VERSION 2
+#define SSM_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define SSM_API __attribute__((visibility("default")))
@@ -378,6 +378,11 @@ typedef struct ssm_split_args {
     const float *h_local;     /* [nranks][batch][state] fp32, every rank's h_loc */
     float *h_in;              /* [batch][state] out, or NULL */
     float *h_out;             /* [batch][state] out, or NULL */
+    /* Elements from one rank's sum_delta (h_local) to the next rank's; 0 for
+     * the dense [nranks][batch][...] layout, else at least batch x U (batch x
+     * state) and a multiple of 4, so the gathered (sum_delta, h_loc) pairs of
+     * one buffer per rank can be read in place.  Added with ABI version 3. */
+    int64_t sum_delta_rank_stride, h_local_rank_stride;
 } ssm_split_args;
 
 /* Step 1.  `tail` is [batch][conv_dim][K-1] in the activation dtype, oldest

@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(_HERE, "libssm.so")
 SSM_OK, SSM_ERR_INVALID_ARG, SSM_ERR_UNSUPPORTED, SSM_ERR_ALIGNMENT = 0, -1, -2, -3
 SSM_ERR_WORKSPACE, SSM_ERR_CUDA, SSM_ERR_DEVICE = -4, -5, -6
 SSM_F32, SSM_BF16 = 0, 1
-ABI_VERSION = 2                # SSM_ABI_VERSION of the header this mirror follows
+ABI_VERSION = 3                # SSM_ABI_VERSION of the header this mirror follows
 SSM_MAMBA1, SSM_MAMBA2 = 1, 2
 SSM_DEVERR_NONE, SSM_DEVERR_CU_SEQLENS, SSM_DEVERR_TIMEOUT, SSM_DEVERR_BOUNDS = 0, 1, 2, 3
 
@@ -92,6 +92,7 @@ class SplitArgs(C.Structure):
         ("mode", _i32), ("rank", _i32), ("nranks", _i32), ("reserved0", _i32),
         ("batch", _i64), ("d_inner", _i64), ("nheads", _i64), ("headdim", _i64), ("dstate", _i64),
         ("A", _vp), ("sum_delta", _vp), ("h_local", _vp), ("h_in", _vp), ("h_out", _vp),
+        ("sum_delta_rank_stride", _i64), ("h_local_rank_stride", _i64),
     ]
 
 

@@ -206,27 +206,55 @@ split_cum_offset_kernel(int64_t U, int64_t seqlen, float *__restrict__ cum) {
 }
 
 // ------------------------------------------------------------- combine
-// One thread per (row, state element): the pairs of segments 0..rank folded
-// in order.  `per_unit` state elements share one delta unit (N for Mamba-1,
-// P*N for Mamba-2); Mamba-1 A is indexed like the state, Mamba-2 A per head.
+// One thread per (row, 4 consecutive state elements; the grid's y is the
+// row): the pairs of segments 0..rank folded in order.  `per_unit` state
+// elements share one delta unit (N for Mamba-1, P*N for Mamba-2, both
+// multiples of 4 on the vector path); Mamba-1 A is indexed like the state,
+// Mamba-2 A per head.  Rank k's sum_delta / h_local start sd_rs / hl_rs
+// elements after rank k-1's.  Element indices within a row fit 32 bits (the
+// API refuses larger states).
 __global__ void split_combine_kernel(const float *__restrict__ A, int m2, const float *__restrict__ sd,
                                      const float *__restrict__ hl, float *__restrict__ h_in,
-                                     float *__restrict__ h_out, int rank, int64_t batch, int64_t S, int64_t U,
-                                     int64_t per_unit) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= batch * S) return;
-    const int64_t b = i / S, e = i % S;
-    const int64_t u = e / per_unit;
+                                     float *__restrict__ h_out, int rank, uint32_t S, uint32_t U, uint32_t per_unit,
+                                     int64_t sd_rs, int64_t hl_rs, bool vec4) {
+    const uint32_t b = blockIdx.y;
+    const int64_t row = (int64_t)b * S;
+    const float *sdr = sd + (int64_t)b * U;
+    if (vec4) {
+        const uint32_t e = (blockIdx.x * blockDim.x + threadIdx.x) * 4u;
+        if (e >= S) return;
+        const uint32_t u = e / per_unit;                  // the same unit for all 4
+        float4 a4;
+        if (m2) a4 = make_float4(A[u], A[u], A[u], A[u]);
+        else a4 = *reinterpret_cast<const float4 *>(A + e);
+        float4 H = *reinterpret_cast<const float4 *>(hl + row + e);
+        float4 before = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 1; k <= rank; ++k) {
+            before = H;
+            const float sdk = sdr[(int64_t)k * sd_rs + u] * kLog2e;
+            const float4 l = *reinterpret_cast<const float4 *>(hl + (int64_t)k * hl_rs + row + e);
+            H.x = fmaf(ex2(a4.x * sdk), H.x, l.x);
+            H.y = fmaf(ex2(a4.y * sdk), H.y, l.y);
+            H.z = fmaf(ex2(a4.z * sdk), H.z, l.z);
+            H.w = fmaf(ex2(a4.w * sdk), H.w, l.w);
+        }
+        if (h_in) *reinterpret_cast<float4 *>(h_in + row + e) = before;
+        if (h_out) *reinterpret_cast<float4 *>(h_out + row + e) = H;
+        return;
+    }
+    const uint32_t e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= S) return;
+    const uint32_t u = e / per_unit;
     const float a = m2 ? A[u] : A[e];
-    float H = hl[i];
+    float H = hl[row + e];
     float before = 0.f;
     for (int k = 1; k <= rank; ++k) {
         before = H;
-        const float decay = ex2(a * sd[((int64_t)k * batch + b) * U + u] * kLog2e);
-        H = fmaf(decay, H, hl[(int64_t)k * batch * S + i]);
+        const float decay = ex2(a * sdr[(int64_t)k * sd_rs + u] * kLog2e);
+        H = fmaf(decay, H, hl[(int64_t)k * hl_rs + row + e]);
     }
-    if (h_in) h_in[i] = before;
-    if (h_out) h_out[i] = H;
+    if (h_in) h_in[row + e] = before;
+    if (h_out) h_out[row + e] = H;
 }
 
 // ------------------------------------------------------- fix-up, Mamba-1
@@ -830,11 +858,20 @@ cudaError_t launch_split_cum_delta(const ssm_scan_args &a, float *cum, float *su
 cudaError_t launch_split_combine(const ssm_split_args &a, cudaStream_t st) {
     const bool m2 = a.mode == SSM_MAMBA2;
     const int64_t S = a.d_inner * a.dstate;
-    const int64_t n = a.batch * S;
-    if (n == 0) return cudaSuccess;
-    split_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-        a.A, m2, a.sum_delta, a.h_local, a.h_in, a.h_out, a.rank, a.batch, S, m2 ? a.nheads : a.d_inner,
-        m2 ? a.headdim * a.dstate : a.dstate);
+    const int64_t U = m2 ? a.nheads : a.d_inner;
+    const int64_t per_unit = m2 ? a.headdim * a.dstate : a.dstate;
+    if (a.batch * S == 0) return cudaSuccess;
+    const int64_t sd_rs = a.sum_delta_rank_stride > 0 ? a.sum_delta_rank_stride : a.batch * U;
+    const int64_t hl_rs = a.h_local_rank_stride > 0 ? a.h_local_rank_stride : a.batch * S;
+    // 16-byte accesses when every row and rank block starts on a 16-byte boundary
+    // and 4 consecutive elements share their delta unit
+    const bool vec4 = per_unit % 4 == 0 && S % 4 == 0 && hl_rs % 4 == 0 && ((uintptr_t)a.h_local % 16) == 0 &&
+                      ((uintptr_t)a.h_in % 16) == 0 && ((uintptr_t)a.h_out % 16) == 0 &&
+                      (m2 || ((uintptr_t)a.A % 16) == 0);
+    const int64_t per_row = vec4 ? S / 4 : S;
+    const dim3 grid((unsigned)((per_row + 255) / 256), (unsigned)a.batch);
+    split_combine_kernel<<<grid, 256, 0, st>>>(a.A, m2, a.sum_delta, a.h_local, a.h_in, a.h_out, a.rank,
+                                               (uint32_t)S, (uint32_t)U, (uint32_t)per_unit, sd_rs, hl_rs, vec4);
     return cudaGetLastError();
 }
 

@@ -333,6 +333,13 @@ ssm_status ssm_split_combine(const ssm_split_args *a, void *stream) {
     if (!aligned(a->A, 4) || !aligned(a->sum_delta, 4) || !aligned(a->h_local, 4) || !aligned(a->h_in, 4) ||
         !aligned(a->h_out, 4))
         return SSM_ERR_ALIGNMENT;
+    const int64_t U = a->mode == SSM_MAMBA2 ? a->nheads : a->d_inner;
+    const int64_t S = a->d_inner * a->dstate;
+    if (a->sum_delta_rank_stride < 0 || (a->sum_delta_rank_stride > 0 && a->sum_delta_rank_stride < a->batch * U) ||
+        a->h_local_rank_stride < 0 || (a->h_local_rank_stride > 0 && a->h_local_rank_stride < a->batch * S) ||
+        a->sum_delta_rank_stride % 4 != 0 || a->h_local_rank_stride % 4 != 0)
+        return SSM_ERR_INVALID_ARG;
+    if (S > INT32_MAX || a->batch > 65535) return SSM_ERR_UNSUPPORTED;   // 32-bit indices in the kernel
     return cuda_status(ssm::launch_split_combine(*a, (cudaStream_t)stream));
 }
 

@@ -397,27 +397,50 @@ def split_conv_tail(mode, x, dt, A, B, C_, *, conv_w, D=None, z=None, dt_bias=No
     return tail
 
 
-def split_cum_delta(mode, x, dt, A, B, C_, *, dt_bias=None, delta_softplus=True, cum=True, D=None, z=None,
-                    conv_w=None, conv_b=None, conv_state_in=None, stream=None):
-    """``(cum_delta [b, T, U] or None, sum_delta [b, U])`` of the segment, fp32 (U = channels or heads)."""
+def split_cum_delta(mode, x, dt, A, B, C_, *, dt_bias=None, delta_softplus=True, cum=True, sum_delta=None, D=None,
+                    z=None, conv_w=None, conv_b=None, conv_state_in=None, stream=None):
+    """``(cum_delta [b, T, U] or None, sum_delta [b, U])`` of the segment, fp32 (U = channels or heads);
+    ``sum_delta`` (contiguous fp32 ``[b, U]``) receives the totals when given."""
     U = x.shape[2]
     b, T = x.shape[0], x.shape[1]
     cd = torch.empty((b, T, U), dtype=torch.float32, device=x.device) if cum else None
-    sd = torch.empty((b, U), dtype=torch.float32, device=x.device)
+    if sum_delta is None:
+        sd = torch.empty((b, U), dtype=torch.float32, device=x.device)
+    else:
+        sd = _c32(sum_delta, "sum_delta")
+        if tuple(sd.shape) != (b, U):
+            raise ValueError(f"sum_delta must be [{b}, {U}]")
     a = _split_scan_args(mode, x, dt, A, B, C_, D, z, dt_bias, conv_w, conv_b, conv_state_in, None, delta_softplus)
     _abi.check(_abi.lib().ssm_split_cum_delta(C.byref(a), _p(cd), _p(sd), _stream(stream)), "ssm_split_cum_delta")
     return cd, sd
 
 
+def _rank_blocks(t, name):
+    """``(t, rank stride)`` for a ``[R, ...]`` fp32 tensor whose rank blocks are each
+    contiguous: stride 0 (dense) or the view's own, else a contiguous copy."""
+    _need(t, name, torch.float32)
+    if t.is_contiguous():
+        return t, 0
+    blk = 1
+    for v in t.shape[1:]:
+        blk *= v
+    inner = t[0] if t.shape[0] > 0 else t
+    if t.shape[0] > 0 and inner.is_contiguous() and t.stride(0) >= blk and t.stride(0) % 4 == 0:
+        return t, int(t.stride(0))
+    return t.contiguous(), 0
+
+
 def split_combine(mode, A, sum_delta_all, h_local_all, rank, *, h_in=None, h_out=None, stream=None):
     """Fold the gathered ``(sum_delta, h_loc)`` of ranks 0..rank: ``(h_in, h_out)`` of this rank's segment.
 
-    ``sum_delta_all`` is ``[R, b, U]`` and ``h_local_all`` ``[R, b, *state]``, both fp32 contiguous.
+    ``sum_delta_all`` is ``[R, b, U]`` and ``h_local_all`` ``[R, b, *state]``, fp32.  Each rank's block
+    must be contiguous; the rank dimension may be strided (views of one gathered buffer of packed pairs),
+    which the library reads in place when the stride is a multiple of 4 elements.
     """
     R, b = h_local_all.shape[0], h_local_all.shape[1]
     state = tuple(h_local_all.shape[2:])
-    _c32(sum_delta_all, "sum_delta_all")
-    _c32(h_local_all, "h_local_all")
+    sum_delta_all, sd_rs = _rank_blocks(sum_delta_all, "sum_delta_all")
+    h_local_all, hl_rs = _rank_blocks(h_local_all, "h_local_all")
     if h_in is None:
         h_in = torch.empty((b,) + state, dtype=torch.float32, device=h_local_all.device)
     if h_out is None:
@@ -431,6 +454,7 @@ def split_combine(mode, A, sum_delta_all, h_local_all, rank, *, h_in=None, h_out
         a.nheads, a.headdim, a.dstate = state
         a.d_inner = state[0] * state[1]
     a.A, a.sum_delta, a.h_local = _p(_c32(A, "A")), _p(sum_delta_all), _p(h_local_all)
+    a.sum_delta_rank_stride, a.h_local_rank_stride = sd_rs, hl_rs
     a.h_in, a.h_out = _p(_c32(h_in, "h_in")), _p(_c32(h_out, "h_out"))
     _abi.check(_abi.lib().ssm_split_combine(C.byref(a), _stream(stream)), "ssm_split_combine")
     return h_in, h_out

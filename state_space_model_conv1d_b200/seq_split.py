@@ -44,7 +44,10 @@ class SegmentScan:
     """One rank's part of a split scan, phase by phase.
 
     ``tail()`` -> tensor for exchange 1; ``scan(tails)`` -> packed pair for
-    exchange 2; ``join(pairs)`` -> ``(y, h_out, conv_state_out)``.  ``h_out``
+    exchange 2; ``join(pairs)`` -> ``(y, h_out, conv_state_out)``.  The packed
+    pair is ``[sum_delta (b*U) | pad | h_loc (b*state) | pad]`` fp32 with both
+    parts starting on a 4-element boundary, so ``join`` reads the gathered
+    ``[R, pack]`` buffer in place.  ``h_out``
     is the state after this rank's segment (the last rank's is the
     sequences' final state), ``conv_state_out`` the segment's conv tail.
     """
@@ -67,6 +70,18 @@ class SegmentScan:
         t = self.t
         return (self.mode, t["x"], t["dt"], t["A"], t["B"], t["C_"])
 
+    def _layout(self):
+        """``(b, U, state shape, offset of h_loc, pack length)`` of the packed pair."""
+        x, A, B = self.t["x"], self.t["A"], self.t["B"]
+        b, U = x.shape[0], x.shape[2]
+        state = (b,) + tuple(A.shape) if x.dim() == 3 else (b, x.shape[2], x.shape[3], B.shape[3])
+        off = (b * U + 3) // 4 * 4
+        return b, U, state, off, off + (self._nhl(state) + 3) // 4 * 4
+
+    def pack_size(self):
+        """Elements of this rank's packed pair."""
+        return self._layout()[4]
+
     def tail(self):
         """This segment's last K-1 raw conv inputs (None without a conv of width > 1)."""
         if self.K < 2:
@@ -74,27 +89,46 @@ class SegmentScan:
         return self.be.split_conv_tail(*self._args(), conv_state_in=self.conv_state_in, stream=self.stream,
                                        **self.kw)
 
-    def scan(self, tails=None):
-        """Scan the segment from zero (rank 0: from h0); return the packed ``(sum_delta, h_loc)``."""
+    def scan(self, tails=None, out=None):
+        """Scan the segment from zero (rank 0: from h0); return the packed
+        ``(sum_delta, h_loc)``, written straight into ``out`` (fp32, ``pack_size()``
+        elements: this rank's block of the exchange buffer) when given."""
         if self.rank > 0 and tails is not None:
             self.conv_state_in = tails[self.rank - 1]
-        self.y, self.h_loc, self.conv_out = self.be.scan_fwd(*self._args(), h0=self.h0,
+        b, U, state, off, n = self._layout()
+        x = self.t["x"]
+        dtype = getattr(self.be, "PACK_DTYPE", torch.float32)     # the backend's state precision
+        if out is None:
+            out = torch.empty(n, dtype=dtype, device=x.device)
+        elif out.dtype != dtype or out.numel() != n or not out.is_contiguous():
+            raise ValueError(f"out must be a contiguous {dtype} tensor of {n} elements")
+        h_loc = out[off:off + self._nhl(state)].view(state)
+        self.y, self.h_loc, self.conv_out = self.be.scan_fwd(*self._args(), h0=self.h0, h_final=h_loc,
                                                              conv_state_in=self.conv_state_in,
                                                              stream=self.stream, **self.kw)
         kw = {k: self.kw[k] for k in ("dt_bias", "delta_softplus")}
-        self.cum, sd = self.be.split_cum_delta(*self._args(), cum=self.rank > 0, stream=self.stream, **kw)
-        return torch.cat([sd.reshape(-1), self.h_loc.reshape(-1)])
+        self.cum, _ = self.be.split_cum_delta(*self._args(), cum=self.rank > 0, sum_delta=out[:b * U].view(b, U),
+                                              stream=self.stream, **kw)
+        return out
+
+    @staticmethod
+    def _nhl(state):
+        n = 1
+        for v in state:
+            n *= v
+        return n
 
     def join(self, pairs):
         """Fold the gathered pairs ``[R, b*U + b*state]`` and fix up y: ``(y, h_out, conv_state_out)``."""
         R = pairs.shape[0]
         if R != self.nranks:
             raise ValueError("expected one pair per rank")
-        b = self.h_loc.shape[0]
-        U = self.t["x"].shape[2]
-        nsd = b * U
-        sd_all = pairs[:, :nsd].reshape(R, b, U).contiguous()
-        hl_all = pairs[:, nsd:].reshape((R,) + tuple(self.h_loc.shape)).contiguous()
+        b, U, state, off, n = self._layout()
+        if pairs.dim() != 2 or pairs.shape[1] != n:
+            raise ValueError(f"expected [R, {n}] packed pairs")
+        # views of the gathered buffer: each rank's block is contiguous
+        sd_all = pairs[:, :b * U].unflatten(1, (b, U))
+        hl_all = pairs[:, off:off + self._nhl(state)].unflatten(1, state)
         h_in, h_out = self.be.split_combine(self.mode, self.t["A"], sd_all, hl_all, self.rank, stream=self.stream)
         if self.rank > 0:
             self.be.split_fixup(*self._args(), self.y, self.cum, h_in, conv_state_in=self.conv_state_in,

@@ -22,6 +22,7 @@ import torch
 import oracle
 
 M1 = oracle.MAMBA1
+PACK_DTYPE = torch.float64     # the exchanged pairs keep the oracle's precision
 
 
 def _np(t):
@@ -37,11 +38,15 @@ def _silu(v):
 
 
 def scan_fwd(mode, x, dt, A, B, C_, *, D=None, z=None, dt_bias=None, h0=None, conv_w=None, conv_b=None,
-             conv_state_in=None, delta_softplus=True, stream=None):
+             conv_state_in=None, delta_softplus=True, h_final=None, stream=None):
     y, hf, cs = oracle.scan_fwd(mode, _np(x), _np(dt), _np(A), _np(B), _np(C_), D=_np(D), z=_np(z),
                                 dt_bias=_np(dt_bias), h0=_np(h0), conv_w=_np(conv_w), conv_b=_np(conv_b),
                                 conv_state_in=_np(conv_state_in), delta_softplus=delta_softplus)
-    return _t(y), _t(hf), _t(cs)
+    hf = _t(hf)
+    if h_final is not None:
+        h_final.copy_(hf)
+        hf = h_final
+    return _t(y), hf, _t(cs)
 
 
 def _conv_inputs(mode, x, B, C_):
@@ -61,11 +66,16 @@ def split_conv_tail(mode, x, dt, A, B, C_, *, conv_w, conv_state_in=None, stream
     return _t(full[:, :, full.shape[2] - (K - 1):])
 
 
-def split_cum_delta(mode, x, dt, A, B, C_, *, dt_bias=None, delta_softplus=True, cum=True, stream=None, **_):
+def split_cum_delta(mode, x, dt, A, B, C_, *, dt_bias=None, delta_softplus=True, cum=True, sum_delta=None,
+                    stream=None, **_):
     r = _np(dt) + (0.0 if dt_bias is None else _np(dt_bias))
     d = np.log1p(np.exp(r)) if delta_softplus else r
     cs = np.cumsum(d, axis=1)
-    return (_t(cs) if cum else None), _t(d.sum(axis=1))
+    sd = _t(d.sum(axis=1))
+    if sum_delta is not None:
+        sum_delta.copy_(sd)
+        sd = sum_delta
+    return (_t(cs) if cum else None), sd
 
 
 def split_combine(mode, A, sum_delta_all, h_local_all, rank, *, stream=None):

@@ -29,7 +29,7 @@ def declared_symbols():
 def test_library_exists_and_loads():
     assert os.path.exists(_abi.LIB_PATH), "build libssm.so first"
     lib = _abi.lib()
-    assert lib.ssm_abi_version() == _abi.ABI_VERSION == 2
+    assert lib.ssm_abi_version() == _abi.ABI_VERSION == 3
 
 
 def test_every_declared_symbol_is_exported():
@@ -319,6 +319,14 @@ def _split(**kw):
     (dict(sum_delta=None), _abi.SSM_ERR_INVALID_ARG),
     (dict(A=FAKE + 2), _abi.SSM_ERR_ALIGNMENT),
     (dict(h_out=FAKE + 1), _abi.SSM_ERR_ALIGNMENT),
+    # rank strides: at least one rank's block (batch x U = 8, batch x state = 256), multiples of 4
+    (dict(sum_delta_rank_stride=4), _abi.SSM_ERR_INVALID_ARG),
+    (dict(sum_delta_rank_stride=10), _abi.SSM_ERR_INVALID_ARG),
+    (dict(sum_delta_rank_stride=-8), _abi.SSM_ERR_INVALID_ARG),
+    (dict(h_local_rank_stride=252), _abi.SSM_ERR_INVALID_ARG),
+    (dict(h_local_rank_stride=258), _abi.SSM_ERR_INVALID_ARG),
+    # a state of more than 2^31 elements per row
+    (dict(mode=1, d_inner=1 << 20, dstate=1 << 12), _abi.SSM_ERR_UNSUPPORTED),
 ])
 def test_split_combine_rejects(kw, status):
     a = _split(**kw)
