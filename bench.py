@@ -874,12 +874,25 @@ def oracle_sample(w: W.Workload, target_s: float):
                                       dt_bias=d["dt_bias"], h0=d["h0"], conv_w=d["conv_w"], nthreads=nrows)
         return run, nrows * w.seqlen, nrows, f"{nrows} of {w.batch} batch rows x {w.seqlen} tokens, all {w.d_inner} channels"
     if w.kind in ("mamba2", "mamba2_varlen"):
-        T = 256 if w.kind == "mamba2" else 256
-        nrows = min(4, max(1, cores))
-        ww = W.Workload(**{**w.__dict__, "kind": "mamba2", "batch": nrows, "seqlen": T})
-        d = W.workload_inputs(ww)
-        run = lambda: oracle.scan_fwd(oracle.MAMBA2, d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"], z=d["z"],
-                                      dt_bias=d["dt_bias"], h0=d["h0"], conv_w=d["conv_w"], nthreads=nrows)
+        # nrows sequences of T tokens (all heads): T grows in steps of 256 tokens, up
+        # to the workload's sequence length, until one run takes about target_s
+        # (timed once at 256 tokens)
+        nrows = min(8, max(1, cores), w.batch if w.kind == "mamba2" else w.nseqs)
+        t_max = max(256, (w.seqlen if w.kind == "mamba2" else w.len_hi) // 256 * 256)
+
+        def make(T):
+            ww = W.Workload(**{**w.__dict__, "kind": "mamba2", "batch": nrows, "seqlen": T})
+            d = W.workload_inputs(ww)
+            return lambda: oracle.scan_fwd(oracle.MAMBA2, d["x"], d["dt"], d["A"], d["B"], d["C"], D=d["D"],
+                                           z=d["z"], dt_bias=d["dt_bias"], h0=d["h0"], conv_w=d["conv_w"],
+                                           nthreads=nrows)
+        T, run = 256, make(256)
+        t0 = time.perf_counter()
+        run()
+        per256 = time.perf_counter() - t0
+        steps = int(min(t_max // 256, max(1, target_s // max(per256, 1e-3))))
+        if steps > 1:
+            T, run = 256 * steps, make(256 * steps)
         return run, nrows * T, nrows, f"{nrows} sequences x {T} tokens, all {w.nheads} heads"
     if w.kind == "decode":
         nb = 16
@@ -894,7 +907,7 @@ def oracle_sample(w: W.Workload, target_s: float):
 
 
 def cpu_baseline(w: W.Workload, args):
-    run, units, cores, what = oracle_sample(w, 20.0)
+    run, units, cores, what = oracle_sample(w, 10.0)
     t0 = time.perf_counter()
     run()
     dt = time.perf_counter() - t0
@@ -908,7 +921,8 @@ def run_reference(args):
     if rank != 0:
         return
     w = W.WORKLOADS[args.workload]
-    run, units, cores, what = oracle_sample(w, 20.0)
+    # every step a sample sized so the whole run takes about two minutes
+    run, units, cores, what = oracle_sample(w, 120.0 / max(1, args.steps + max(args.warmup, 0)))
     for _ in range(max(args.warmup, 0)):
         run()
     times = []

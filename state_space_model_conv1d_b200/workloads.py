@@ -34,9 +34,11 @@ BASE_SEED = 20261202
 def round_bf16(a: np.ndarray) -> np.ndarray:
     """Quantise float32 values to the nearest bf16 (ties to even), kept as float32."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
-    return u.astype(np.uint32).view(np.float32)
+    u = a.view(np.uint32)
+    r = u + np.uint32(0x7FFF)                       # half an ulp of bf16, less one
+    r += (u >> np.uint32(16)) & np.uint32(1)        # ties go to the even bf16 value
+    r &= np.uint32(0xFFFF0000)
+    return r.view(np.float32)
 
 
 def _act(rng, shape, dtype, scale=1.0):
