@@ -161,3 +161,44 @@ def test_cum_delta_prefix_sums(mode, T, U):
     np.testing.assert_allclose(sd.cpu().numpy(), ref[:, -1], rtol=5e-5)
     np.testing.assert_allclose(sd_only.cpu().numpy(), sd.cpu().numpy(), rtol=1e-6)
     np.testing.assert_array_equal(sd.cpu().numpy(), got[:, -1].astype(np.float32))
+
+
+# The combine reads every rank's (sum of delta, h_loc) in place from one
+# gathered buffer of packed pairs (rank strides), or from dense stacks; both
+# give the same bits, and both the fold H_k = exp(A sum_delta_k) H_{k-1} + h_k
+# computed here in fp64 (the combine uses the MUFU exp: 2^-21 relative).
+@pytest.mark.parametrize("mode,state", [(M2, (3, 4, 8, 16)), (M1, (3, 24, 16)), (M1, (2, 10, 5))])
+@pytest.mark.parametrize("pad", [0, 3])          # rank strides a multiple of 4, or not (copied)
+def test_split_combine_strided_pairs(mode, state, pad):
+    from state_space_model_conv1d_b200 import ops
+    rng = np.random.default_rng(601 + len(state) + state[-1] + pad)
+    R, rank = 3, 2
+    b = state[0]
+    U = state[1]
+    A = -rng.uniform(0.1, 1.0, size=(U,) if mode == M2 else state[1:]).astype(np.float32)
+    sd = rng.uniform(0.1, 2.0, size=(R, b, U)).astype(np.float32)
+    hl = rng.standard_normal((R,) + state).astype(np.float32)
+    dev = lambda a: torch.from_numpy(a).cuda()
+    h_in, h_out = ops.split_combine(mode, dev(A), dev(sd), dev(hl), rank)
+    nsd, nhl = b * U, int(np.prod(state))
+    off = (nsd + 3) // 4 * 4
+    buf = torch.full((R, off + nhl + pad + 4), float("nan"), dtype=torch.float32, device="cuda")
+    buf[:, :nsd] = dev(sd.reshape(R, -1))
+    buf[:, off:off + nhl] = dev(hl.reshape(R, -1))
+    s_in, s_out = ops.split_combine(mode, dev(A), buf[:, :nsd].unflatten(1, (b, U)),
+                                    buf[:, off:off + nhl].unflatten(1, state), rank)
+    torch.cuda.synchronize()
+    assert torch.equal(s_in, h_in) and torch.equal(s_out, h_out)
+    # fp64 fold
+    a64 = A.astype(np.float64)
+    H = hl[0].astype(np.float64)
+    before = np.zeros_like(H)
+    for k in range(1, rank + 1):
+        before = H
+        if mode == M2:
+            dec = np.exp(a64[None, :, None, None] * sd[k].astype(np.float64)[:, :, None, None])
+        else:
+            dec = np.exp(a64[None] * sd[k].astype(np.float64)[:, :, None])
+        H = dec * H + hl[k]
+    np.testing.assert_allclose(h_in.cpu().numpy(), before, rtol=1e-5, atol=1e-5)
+    np.testing.assert_allclose(h_out.cpu().numpy(), H, rtol=1e-5, atol=1e-5)
