@@ -179,7 +179,8 @@ typedef struct ssm_scan_args {
      * CTAs scan at the same time.  Packed sequences (cu_seqlens) are cut into
      * runs of one length for all of them, chosen from the total: about n runs
      * for a sequence of the mean length; the library cuts them only when the
-     * sequences x heads leave the GPU short of CTAs.  Each run's
+     * sequences x heads leave the GPU short of CTAs, with the run length it
+     * would choose for nseqs rows of the mean length.  Each run's
      * entering state comes from a state-only pass over the runs before it (the
      * pair (exp(delta A), h) composes associatively, seed (1, h0): "Adding
      * Initial Value Support to Selective Scan Forward Kernel"), so results
