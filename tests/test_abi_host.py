@@ -176,6 +176,9 @@ def test_segment_plan_is_host_only():
     assert lib.ssm_scan_segments(C.byref(_scan(**dict(packed, nseqs=1000)))) == 1
     assert lib.ssm_scan_segments(C.byref(_scan(**dict(packed, nseqs=9)))) == 1
     assert lib.ssm_scan_segments(C.byref(_scan(segments=2, **dict(packed, nseqs=9)))) == 9 + 16
+    # more runs than a grid's second dimension holds (65535): the sequences stay whole
+    many = dict(packed, nseqs=60000, seqlen=6000000, x_batch_stride=5120 * 6000000)
+    assert lib.ssm_scan_segments(C.byref(_scan(segments=2, **many))) == 1
     # Mamba-1 is never cut; bad arguments give 0
     assert lib.ssm_scan_segments(C.byref(_scan(mode=1, d_inner=8, ngroups=1, dt_token_stride=8, dt_batch_stride=128))) == 1
     assert lib.ssm_scan_segments(C.byref(_scan(segments=-1, **big))) == 0
