@@ -194,6 +194,23 @@ def test_mamba2_varlen_segments_many_sequences():
     check_scan(M2, d, "bf16", segments=2, what="M2 varlen segments, 2500 sequences")
 
 
+def test_mamba2_varlen_segments_bad_cu_seqlens():
+    """With the sequences cut on the device, a decreasing cu_seqlens still
+    leaves y unwritten and sets the error word (the segment table stays empty)."""
+    d = W.mamba2_inputs(494, 1, 600, 2, 64, 1, 128, dtype="bf16", conv_bias=True, nseqs=2)
+    t = to_dev(d, "bf16")
+    cu = torch.tensor([0, 500, 300], dtype=torch.int32, device="cuda")
+    assert ssm.scan_segments(M2, t["x"], t["dt"], t["A"], t["B"], t["C"], cu_seqlens=cu, conv_w=t["conv_w"],
+                             segments=3) > 1
+    y = torch.full(t["x"].shape, 7.0, dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(ssm.scan_workspace_size(M2, t["x"], t["dt"], t["A"], t["B"], t["C"], cu_seqlens=cu,
+                                             conv_w=t["conv_w"], segments=3), dtype=torch.uint8, device="cuda")
+    ssm.scan_fwd(M2, t["x"], t["dt"], t["A"], t["B"], t["C"], cu_seqlens=cu, conv_w=t["conv_w"], y=y, workspace=ws,
+                 segments=3)
+    assert ssm.workspace_error(ws) == 1
+    assert torch.all(y == 7.0)
+
+
 def test_mamba2_varlen_segments_match_unsegmented():
     lengths = [2500, 3, 0, 900, 1300]
     cu = W.cu_from_lengths(lengths)
